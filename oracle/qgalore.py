@@ -1,0 +1,511 @@
+"""Plain CPU oracle for the Q-GaLore per-layer optimizer step and subspace refresh.
+
+TEST INFRASTRUCTURE ONLY.  This module is imported by ``tests/``, by
+``__graft_entry__.smoke()`` and by the ``cpu_baseline`` / reference arm of
+``bench.py``; nothing in the product path may import it.  It shares no code with
+the CUDA path: every formula here is written out independently.
+
+What the pages fix, and where (titles of the source pages):
+
+* [QG-abs]  "Q-GaLore: Quantized GaLore with INT4 Projection and Layer-Adaptive
+  Low-Rank Gradients", abstract (paper index record): gradients are projected into
+  a low-rank subspace found by SVD; projection matrices kept in INT4, weights in
+  INT8, stochastic rounding accumulates small updates.
+* [QG-sched] AIMech curated page "Q-GaLore (Quantized GaLore with INT4 Projection
+  and Layer-Adaptive Low-Rank Gradients)", mechanism "layer-adaptive subspace
+  cosine schedule" (paper section 3.1, Eq. (5)):
+  CosSim(P_t, P_{t-D}) = (1/r) * sum_i sigma_i(P_t^T P_{t-D}); the layer's
+  interval D doubles whenever CosSim > gamma, gamma = 0.4 by default.
+* [QG-quant] same page, mechanism "INT4 projection and INT8 stochastic rounding"
+  (paper section 3.2): P_t stored in INT4; low-rank first and second moments
+  (M^Q, V^Q) in INT8; W^Q_t = W^Q_{t-1} + xi(alpha * P^Q_t * G~_t) with xi an
+  unbiased stochastic rounding.
+
+Everything the pages leave open is a stated reading (they are listed, numbered,
+in the design notes of this repository); each function below names the reading
+it takes.  Floating point: contractions (the two projections, the refresh
+products) are carried out in float64 from the exact float32/bf16 operands and
+rounded once to float32; element-wise arithmetic that decides an integer (a
+quantised code, a rounding decision) is done in IEEE float32, one rounding per
+operation, in the order written, exactly as the GPU path must do it.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+F32 = np.float32
+U32_MASK = np.uint64(0xFFFFFFFF)
+
+# --------------------------------------------------------------------------
+# bf16 rounding (round to nearest, ties to even) — the operand precision of the
+# projections.  Pinned against torch's float32 -> bfloat16 conversion.
+# --------------------------------------------------------------------------
+
+
+def bf16_bits(x) -> np.ndarray:
+    """float32 -> bfloat16 bit patterns (uint16), round-to-nearest-even."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    b = x.view(np.uint32).astype(np.uint64)
+    lsb = (b >> np.uint64(16)) & np.uint64(1)
+    r = ((b + np.uint64(0x7FFF) + lsb) >> np.uint64(16)).astype(np.uint16)
+    nan = np.isnan(x)
+    if nan.any():
+        r = np.where(nan, np.uint16(0x7FC0), r)
+    return r
+
+
+def bf16_from_bits(bits) -> np.ndarray:
+    """bfloat16 bit patterns -> float32 values (exact)."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32)
+
+
+def bf16_round(x) -> np.ndarray:
+    """float32 -> float32 values representable in bfloat16 (RNE)."""
+    return bf16_from_bits(bf16_bits(x))
+
+
+# --------------------------------------------------------------------------
+# Philox counter-based generator (Salmon, Moraes, Dror, Shaw, "Parallel random
+# numbers: as easy as 1, 2, 3", SC'11).  The pages only say the rounding is
+# stochastic and unbiased; the random stream is a reading (counter-based so
+# that any element's draw is computable on its own).
+# --------------------------------------------------------------------------
+
+PHILOX4x32 = dict(width=32, mult=(0xD2511F53, 0xCD9E8D57), weyl=(0x9E3779B9, 0xBB67AE85))
+PHILOX4x64 = dict(width=64, mult=(0xD2E7470EE14C6C93, 0xCA5A826395121157),
+                  weyl=(0x9E3779B97F4A7C15, 0xBB67AE8584CAA73B))
+
+
+def philox_generic(ctr, key, width, mult, weyl, rounds=10):
+    """Philox-4xW on Python integers (slow, any word width).
+
+    One round: the two products mult0*c0 and mult1*c2 are formed at double
+    width; the new block is (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0).  The key is
+    bumped by the Weyl constants before every round but the first.
+    """
+    mask = (1 << width) - 1
+    c = [int(v) & mask for v in ctr]
+    k = [int(v) & mask for v in key]
+    for rnd in range(rounds):
+        if rnd:
+            k = [(k[0] + weyl[0]) & mask, (k[1] + weyl[1]) & mask]
+        p0 = mult[0] * c[0]
+        p1 = mult[1] * c[2]
+        c = [((p1 >> width) ^ c[1] ^ k[0]) & mask, p1 & mask,
+             ((p0 >> width) ^ c[3] ^ k[1]) & mask, p0 & mask]
+    return c
+
+
+def philox4x32_10(c0, c1, c2, c3, k0, k1):
+    """Vectorised Philox-4x32-10: arrays of counters -> four uint32 arrays."""
+    c = np.broadcast_arrays(*(np.asarray(v, dtype=np.uint64) & U32_MASK for v in (c0, c1, c2, c3)))
+    c = [np.array(v, dtype=np.uint64) for v in c]
+    k0 = np.uint64(int(k0) & 0xFFFFFFFF)
+    k1 = np.uint64(int(k1) & 0xFFFFFFFF)
+    m0, m1 = (np.uint64(v) for v in PHILOX4x32["mult"])
+    w0, w1 = (np.uint64(v) for v in PHILOX4x32["weyl"])
+    s32 = np.uint64(32)
+    for rnd in range(10):
+        if rnd:
+            k0 = (k0 + w0) & U32_MASK
+            k1 = (k1 + w1) & U32_MASK
+        p0 = m0 * c[0]
+        p1 = m1 * c[2]
+        c = [(p1 >> s32) ^ c[1] ^ k0, p1 & U32_MASK, (p0 >> s32) ^ c[3] ^ k1, p0 & U32_MASK]
+    return [v.astype(np.uint32) for v in c]
+
+
+# --------------------------------------------------------------------------
+# Quantizers.  [QG-quant] fixes the widths (INT4 projection, INT8 moments and
+# weights); the grids are readings: symmetric absmax, scale = absmax / qmax
+# (IEEE float32 division), code = clamp(rint(x / scale)) with ties to even, and
+# a zero group gets scale 0 and codes 0.
+# --------------------------------------------------------------------------
+
+INT4_QMAX = 7
+INT8_QMAX = 127
+
+
+def quant_int4_groups(P, group=64):
+    """INT4 absmax quantization of the flattened row-major array, groups of `group`.
+
+    Returns (codes int8 in [-7, 7] of length P.size, scales float32 of length
+    ceil(P.size / group)).  [QG-quant]: P_t is kept in INT4.
+    """
+    x = np.asarray(P, dtype=np.float32).ravel()
+    ng = -(-x.size // group)
+    xp = np.zeros(ng * group, dtype=np.float32)
+    xp[: x.size] = x
+    xg = xp.reshape(ng, group)
+    absmax = np.max(np.abs(xg), axis=1)
+    s = (absmax / F32(INT4_QMAX)).astype(np.float32)
+    safe = np.where(s > 0, s, F32(1))
+    q = np.clip(np.rint(xg / safe[:, None]), -INT4_QMAX, INT4_QMAX)
+    q = np.where((s > 0)[:, None], q, 0).astype(np.int8)
+    return q.ravel()[: x.size], s
+
+
+def pack_int4(codes) -> np.ndarray:
+    """Two's-complement nibbles, two per byte, the even index in the low nibble."""
+    q = np.asarray(codes, dtype=np.int8).ravel()
+    if q.size % 2:
+        q = np.concatenate([q, np.zeros(1, np.int8)])
+    lo = q[0::2].astype(np.uint8) & np.uint8(0xF)
+    hi = q[1::2].astype(np.uint8) & np.uint8(0xF)
+    return (lo | (hi << np.uint8(4))).astype(np.uint8)
+
+
+def unpack_int4(packed, count) -> np.ndarray:
+    b = np.asarray(packed, dtype=np.uint8)
+    nib = np.empty(b.size * 2, dtype=np.int16)
+    nib[0::2] = b & 0xF
+    nib[1::2] = b >> 4
+    nib = np.where(nib >= 8, nib - 16, nib)
+    return nib[:count].astype(np.int8)
+
+
+def dequant_int4_f32(packed, scales, m, r, group=64) -> np.ndarray:
+    """P = code * scale in float32 (one rounding), shape (m, r)."""
+    q = unpack_int4(packed, m * r).astype(np.float32)
+    s = np.asarray(scales, dtype=np.float32)[np.arange(m * r) // group]
+    return (q * s).astype(np.float32).reshape(m, r)
+
+
+def dequant_P_bf16(packed, scales, m, r, group=64) -> np.ndarray:
+    """Step a1: P~ = bf16_rn(code * scale): the projection as the tensor cores see it."""
+    return bf16_round(dequant_int4_f32(packed, scales, m, r, group))
+
+
+def quant_rowblock_int8(x, block=256, unsigned=False):
+    """INT8 absmax quantization in blocks of `block` consecutive columns of each row.
+
+    The last block of a row is short when n % block != 0 (blocks never cross
+    rows).  unsigned=True is used for the second moment (v >= 0): codes in
+    [0, 127].  Returns (codes int8 (rows, n), scales float32 (rows, nblocks)).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    rows, n = x.shape
+    nb = -(-n // block)
+    codes = np.zeros((rows, n), dtype=np.int8)
+    scales = np.zeros((rows, nb), dtype=np.float32)
+    lo = 0 if unsigned else -INT8_QMAX
+    for b in range(nb):
+        xs = x[:, b * block: min((b + 1) * block, n)]
+        s = (np.max(np.abs(xs), axis=1) / F32(INT8_QMAX)).astype(np.float32)
+        safe = np.where(s > 0, s, F32(1))
+        q = np.clip(np.rint(xs / safe[:, None]), lo, INT8_QMAX)
+        codes[:, b * block: min((b + 1) * block, n)] = np.where((s > 0)[:, None], q, 0)
+        scales[:, b] = s
+    return codes, scales
+
+
+def dequant_rowblock(codes, scales, block=256) -> np.ndarray:
+    codes = np.asarray(codes)
+    cols = np.arange(codes.shape[1]) // block
+    return (codes.astype(np.float32) * np.asarray(scales, np.float32)[:, cols]).astype(np.float32)
+
+
+# --------------------------------------------------------------------------
+# Configuration and host-side constants
+# --------------------------------------------------------------------------
+
+
+@dataclass
+class Config:
+    m: int
+    n: int
+    r: int
+    w_group: int = 256
+    p_group: int = 64
+    mom_block: int = 256
+    beta1: float = 0.9
+    beta2: float = 0.999
+    eps: float = 1e-8
+    lr: float = 1e-3
+    alpha: float = 0.25
+    gamma: float = 0.4
+    delta0: int = 200
+    oversample: int = 16
+    power_iters: int = 2
+    seed: int = 0
+    layer_id: int = 0
+
+    def f32(self, name):
+        return F32(getattr(self, name))
+
+
+def adam_constants(cfg: Config, t: int):
+    """float32 constants of step t (t counted from 1 per layer): (1-b1), (1-b2),
+    and the bias corrections 1-b1^t, 1-b2^t, formed in float64 from the float32
+    betas and rounded once to float32."""
+    b1 = float(F32(cfg.beta1))
+    b2 = float(F32(cfg.beta2))
+    return (F32(1.0 - b1), F32(1.0 - b2), F32(1.0 - b1 ** t), F32(1.0 - b2 ** t))
+
+
+# --------------------------------------------------------------------------
+# The step, a1..a5
+# --------------------------------------------------------------------------
+
+
+def project(P_bf16, G) -> np.ndarray:
+    """Step a2: R = P~^T G (r x n), float64 sum of the exact products, rounded to
+    float32.  [QG-abs]: the gradient is projected into the low-rank subspace;
+    reading: the left factor is always projected (P is m x r)."""
+    return (np.asarray(P_bf16, np.float64).T @ np.asarray(G, np.float64)).astype(np.float32)
+
+
+def adam_moments(R, m0, v0, cfg: Config, t: int):
+    """Adam moment update and normalised low-rank step (float32, no fused
+    multiply-add).  Readings: bias correction on, epsilon added after the square
+    root, no weight decay, the descent sign carried by N:
+
+        m = b1*m0 + (1-b1)*R
+        v = b2*v0 + (1-b2)*(R*R)
+        N = (-lr * (m / (1-b1^t))) / (sqrt(v / (1-b2^t)) + eps)
+
+    Returns (N float32 before bf16 rounding, m, v).
+    """
+    om1, om2, bc1, bc2 = adam_constants(cfg, t)
+    R = np.asarray(R, np.float32)
+    m = (cfg.f32("beta1") * m0 + om1 * R).astype(np.float32)
+    v = (cfg.f32("beta2") * v0 + om2 * (R * R)).astype(np.float32)
+    mhat = (m / bc1).astype(np.float32)
+    vhat = (v / bc2).astype(np.float32)
+    num = (F32(-cfg.lr) * mhat).astype(np.float32)
+    den = (np.sqrt(vhat) + cfg.f32("eps")).astype(np.float32)
+    return (num / den).astype(np.float32), m, v
+
+
+def lowrank_adam_int8(R, Mq, sM, Vq, sV, cfg: Config, t: int):
+    """Step a3: Adam on the INT8 moments.  [QG-quant]: (M^Q, V^Q) are kept in
+    INT8.  Readings: per-row blocks of `mom_block` columns, re-quantized with a
+    fresh absmax scale every step; N is formed from the float32 moments before
+    they are re-quantized, then rounded to bf16 (the operand of step a4).
+
+    Returns (N as bf16 values in float32, Mq', sM', Vq', sV')."""
+    m0 = dequant_rowblock(Mq, sM, cfg.mom_block)
+    v0 = dequant_rowblock(Vq, sV, cfg.mom_block)
+    upd, m, v = adam_moments(R, m0, v0, cfg, t)
+    N = bf16_round(upd)
+    Mq2, sM2 = quant_rowblock_int8(m, cfg.mom_block, unsigned=False)
+    Vq2, sV2 = quant_rowblock_int8(v, cfg.mom_block, unsigned=True)
+    return N, Mq2, sM2, Vq2, sV2
+
+
+def backproject(P_bf16, N_bf16) -> np.ndarray:
+    """Step a4: U = P~ N (m x n) in float64 from the exact bf16 operands, rounded
+    to float32.  alpha is applied in step a5.  [QG-quant]: alpha * P_t * G~_t."""
+    return (np.asarray(P_bf16, np.float64) @ np.asarray(N_bf16, np.float64)).astype(np.float32)
+
+
+def sr_uniform24(m, n, seed, t, layer_id):
+    """The 24-bit uniform draw of every weight element (m x n uint32 in [0, 2^24)).
+
+    Element e = i*n + j (logical index) takes word (e mod 4) of
+    Philox-4x32-10(counter = (e/4 low 32 bits, e/4 high 32 bits, t, layer_id),
+    key = (seed low 32 bits, seed high 32 bits)) and keeps its top 24 bits.
+    """
+    e = np.arange(m * n, dtype=np.uint64)
+    quad = e >> np.uint64(2)
+    w = philox4x32_10(quad & U32_MASK, quad >> np.uint64(32), t, layer_id,
+                      seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
+    sel = (e & np.uint64(3)).astype(np.int64)
+    words = np.stack(w, axis=0)[sel, np.arange(m * n)]
+    return (words >> np.uint32(8)).reshape(m, n)
+
+
+def stochastic_round_update(Wq, sW, U, cfg: Config, t: int, u24=None):
+    """Step a5: W^Q <- W^Q + xi(alpha * U), in code units of the fixed weight grid.
+
+    Readings: the weight scale is one float32 per 256 consecutive elements of
+    the row-major m x n array (logical index), fixed after initialisation;
+    c_g = alpha / s_g (IEEE float32; a zero scale freezes its group);
+    x = U * c_g; y = q + x; f = floor(y); phi = y - f (exact);
+    xi rounds up iff u < phi with u = u24 * 2^-24 (compared as u24 < phi * 2^24,
+    exact); the result is clamped to [-127, 127]; a NaN y keeps the old code.
+    E[xi(y)] = y up to 2^-24 (the draw grid) away from the clamp."""
+    m, n = Wq.shape
+    e = np.arange(m * n, dtype=np.int64).reshape(m, n)
+    sW = np.asarray(sW, np.float32)
+    c = np.where(sW > 0, F32(cfg.alpha) / np.where(sW > 0, sW, F32(1)), F32(0)).astype(np.float32)
+    x = (np.asarray(U, np.float32) * c[e // cfg.w_group]).astype(np.float32)
+    y = (Wq.astype(np.float32) + x).astype(np.float32)
+    with np.errstate(invalid="ignore"):
+        f = np.floor(y)
+        phi = (y - f).astype(np.float32)
+        if u24 is None:
+            u24 = sr_uniform24(m, n, cfg.seed, t, cfg.layer_id)
+        up = u24.astype(np.float32) < (phi * F32(2 ** 24))
+        qf = np.clip(f + up.astype(np.float32), -INT8_QMAX, INT8_QMAX)
+    out = np.where(np.isnan(y), Wq, np.nan_to_num(qf).astype(np.int8))
+    return out.astype(np.int8)
+
+
+@dataclass
+class LayerState:
+    """Everything one weight matrix carries between steps."""
+    cfg: Config
+    Wq: np.ndarray            # m x n int8
+    sW: np.ndarray            # ceil(m*n/256) float32, fixed
+    Pq: np.ndarray | None = None      # packed INT4 (ceil(m*r/2) uint8)
+    sP: np.ndarray | None = None      # ceil(m*r/64) float32
+    Pq_prev: np.ndarray | None = None
+    sP_prev: np.ndarray | None = None
+    Mq: np.ndarray = None     # r x n int8
+    sM: np.ndarray = None     # r x ceil(n/256) float32
+    Vq: np.ndarray = None
+    sV: np.ndarray = None
+    t: int = 0
+    delta: int = 0
+    t_next: int = 0
+    n_refresh: int = 0
+    cossim_trace: list = field(default_factory=list)
+
+    @staticmethod
+    def create(cfg: Config, Wq, sW):
+        nb = -(-cfg.n // cfg.mom_block)
+        return LayerState(cfg=cfg, Wq=np.array(Wq, np.int8), sW=np.array(sW, np.float32),
+                          Mq=np.zeros((cfg.r, cfg.n), np.int8), sM=np.zeros((cfg.r, nb), np.float32),
+                          Vq=np.zeros((cfg.r, cfg.n), np.int8), sV=np.zeros((cfg.r, nb), np.float32),
+                          delta=cfg.delta0)
+
+
+def step(st: LayerState, G) -> dict:
+    """One optimizer step a1..a5 on one weight matrix (mutates `st`).
+
+    Returns the intermediates (P~, R, N, U) for inspection."""
+    cfg = st.cfg
+    st.t += 1
+    Pb = dequant_P_bf16(st.Pq, st.sP, cfg.m, cfg.r, cfg.p_group)
+    R = project(Pb, G)
+    N, st.Mq, st.sM, st.Vq, st.sV = lowrank_adam_int8(R, st.Mq, st.sM, st.Vq, st.sV, cfg, st.t)
+    U = backproject(Pb, N)
+    st.Wq = stochastic_round_update(st.Wq, st.sW, U, cfg, st.t)
+    return dict(P=Pb, R=R, N=N, U=U)
+
+
+# --------------------------------------------------------------------------
+# Subspace refresh (a6) and the layer-adaptive schedule (a7)
+# --------------------------------------------------------------------------
+
+OMEGA_KEY_SALT = 0x52454652
+
+
+def refresh_width(cfg: Config) -> int:
+    """k = r + oversampling, capped by min(m, n)."""
+    return min(cfg.r + cfg.oversample, cfg.m, cfg.n)
+
+
+def rademacher_omega(n, k, seed, refresh_idx, layer_id) -> np.ndarray:
+    """Test matrix Omega (n x k) of +-1.  Entry e = j*k + c takes bit (e mod 32)
+    of word ((e / 32) mod 4) of Philox-4x32-10(counter = (e / 128, refresh_idx,
+    layer_id, 0), key = (seed_lo ^ 0x52454652, seed_hi)); a set bit gives -1."""
+    assert n * k < (1 << 39)
+    e = np.arange(n * k, dtype=np.uint64)
+    w = philox4x32_10(e >> np.uint64(7), refresh_idx, layer_id, 0,
+                      (seed & 0xFFFFFFFF) ^ OMEGA_KEY_SALT, (seed >> 32) & 0xFFFFFFFF)
+    words = np.stack(w, 0)[((e >> np.uint64(5)) & np.uint64(3)).astype(np.int64), np.arange(n * k)]
+    bit = (words >> (e & np.uint64(31)).astype(np.uint32)) & np.uint32(1)
+    return np.where(bit == 1, -1.0, 1.0).reshape(n, k)
+
+
+def canonical_signs(P) -> np.ndarray:
+    """Make the entry of largest magnitude of every column positive (the first
+    such row on ties): fixes the sign freedom of singular vectors."""
+    P = np.array(P, dtype=np.float64)
+    idx = np.argmax(np.abs(P), axis=0)
+    sgn = np.where(P[idx, np.arange(P.shape[1])] < 0, -1.0, 1.0)
+    return P * sgn[None, :]
+
+
+def _orth(Y):
+    """Orthonormal basis of the column span (Householder QR, a library step)."""
+    Q, _ = np.linalg.qr(Y, mode="reduced")
+    return Q
+
+
+def randomized_topr(G, r, k, power_iters, Omega) -> tuple[np.ndarray, np.ndarray]:
+    """Randomized subspace iteration for the top-r left singular vectors of G
+    (Halko, Martinsson, Tropp 2011: range finder with power iterations, then
+    Rayleigh-Ritz), in float64:
+
+        Q = orth(G Omega);  repeat q times: Z = orth(G^T Q); Q = orth(G Z)
+        B = Q^T G;  S = B B^T = V diag(lambda) V^T (descending)
+        P = Q V[:, :r], columns sign-canonical.
+
+    The span of each orth() is independent of the basis it returns, and so is
+    P: any orthonormalisation (QR, Cholesky-QR) gives the same P in exact
+    arithmetic.  Returns (P m x r, sigma = sqrt(lambda[:r]))."""
+    G = np.asarray(G, np.float64)
+    Q = _orth(G @ Omega)
+    for _ in range(power_iters):
+        Z = _orth(G.T @ Q)
+        Q = _orth(G @ Z)
+    B = Q.T @ G
+    lam, V = np.linalg.eigh(B @ B.T)
+    order = np.argsort(-lam, kind="stable")
+    lam, V = lam[order], V[:, order]
+    P = canonical_signs(Q @ V[:, :r])
+    return P, np.sqrt(np.maximum(lam[:r], 0.0))
+
+
+def exact_topr(G, r) -> tuple[np.ndarray, np.ndarray]:
+    """Top-r left singular vectors by a full SVD (LAPACK), sign-canonical."""
+    U, s, _ = np.linalg.svd(np.asarray(G, np.float64), full_matrices=False)
+    return canonical_signs(U[:, :r]), s[:r]
+
+
+def cossim(Pa, Pb) -> float:
+    """[QG-sched] Eq. (5): CosSim(Pa, Pb) = (1/r) * sum_i sigma_i(Pa^T Pb)."""
+    Pa = np.asarray(Pa, np.float64)
+    Pb = np.asarray(Pb, np.float64)
+    s = np.linalg.svd(Pa.T @ Pb, compute_uv=False)
+    return float(s.sum() / Pa.shape[1])
+
+
+def schedule_after_refresh(t, delta, cs, gamma):
+    """[QG-sched]: after a refresh at step t with CosSim `cs` against the previous
+    projection (None at the first refresh), the interval doubles iff cs > gamma
+    (strict); the next refresh is due at t + delta.  Returns (delta, t_next)."""
+    if cs is not None and cs > gamma:
+        delta = 2 * delta
+    return delta, t + delta
+
+
+def refresh_due(st: LayerState, force=False) -> bool:
+    return bool(force) or st.t == st.t_next
+
+
+def refresh(st: LayerState, G, force=False) -> dict | None:
+    """Subspace refresh of one layer, if due: randomized top-r SVD of G, INT4
+    quantization of the new P, CosSim against the previous INT4 P (both
+    dequantized to float32), the doubling rule.  Reading: the moments are kept
+    as they are across a refresh.  Returns None when not due."""
+    if not refresh_due(st, force):
+        return None
+    cfg = st.cfg
+    k = refresh_width(cfg)
+    Omega = rademacher_omega(cfg.n, k, cfg.seed, st.n_refresh, cfg.layer_id)
+    P, sigma = randomized_topr(G, cfg.r, k, cfg.power_iters, Omega)
+    codes, sP = quant_int4_groups(P.astype(np.float32), cfg.p_group)
+    Pq = pack_int4(codes)
+    cs = None
+    if st.Pq is not None:
+        cs = cossim(dequant_int4_f32(Pq, sP, cfg.m, cfg.r, cfg.p_group),
+                    dequant_int4_f32(st.Pq, st.sP, cfg.m, cfg.r, cfg.p_group))
+        st.Pq_prev, st.sP_prev = st.Pq, st.sP
+    st.Pq, st.sP = Pq, sP
+    st.delta, st.t_next = schedule_after_refresh(st.t, st.delta, cs, cfg.gamma)
+    st.n_refresh += 1
+    st.cossim_trace.append((st.t, cs))
+    return dict(P=P, sigma=sigma, cossim=cs, Omega=Omega)
+
+
+def set_projection(st: LayerState, P):
+    """Quantize and install a given float projection (m x r) as P^Q."""
+    codes, sP = quant_int4_groups(np.asarray(P, np.float32), st.cfg.p_group)
+    st.Pq, st.sP = pack_int4(codes), sP

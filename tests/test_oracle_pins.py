@@ -1,0 +1,460 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test checks one oracle function against a library routine, a closed form,
+a brute-force computation or a hand-worked golden fixture, chosen so that a
+plausible slip (a dropped term, a wrong sign or index, a transposed operand)
+fails at least one of them.  No GPU needed.
+"""
+import ctypes
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- Philox
+
+def _curand_host_philox(seed, count):
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    path = os.path.join(cuda, "lib64", "libcurand.so")
+    if not os.path.exists(path):
+        pytest.skip("libcurand not found")
+    lib = ctypes.CDLL(path)
+    gen = ctypes.c_void_p()
+    CURAND_RNG_PSEUDO_PHILOX4_32_10 = 161
+    assert lib.curandCreateGeneratorHost(ctypes.byref(gen), CURAND_RNG_PSEUDO_PHILOX4_32_10) == 0
+    try:
+        assert lib.curandSetPseudoRandomGeneratorSeed(gen, ctypes.c_ulonglong(seed)) == 0
+        out = np.zeros(count, dtype=np.uint32)
+        assert lib.curandGenerate(gen, out.ctypes.data_as(ctypes.c_void_p), ctypes.c_size_t(count)) == 0
+    finally:
+        lib.curandDestroyGenerator(gen)
+    return out
+
+
+@pytest.mark.parametrize("seed", [0, 1, 0x123456789ABCDEF0, 2**64 - 1])
+def test_philox4x32_matches_curand_host_generator(seed):
+    # cuRAND's host Philox4x32-10 emits block s as Philox(counter=(0,0,s,0), key=seed).
+    blocks = 96
+    ref = _curand_host_philox(seed, 4 * blocks)
+    s = np.arange(blocks)
+    w = O.philox4x32_10(0, 0, s, 0, seed & 0xFFFFFFFF, seed >> 32)
+    got = np.stack(w, axis=1).ravel()
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_philox_round_structure_matches_numpy_philox4x64():
+    # numpy's Philox is the 4x64-10 member of the same family; its first block
+    # uses counter + 1.  Same round function, other word width and constants.
+    rng = np.random.default_rng(5)
+    for _ in range(20):
+        key = [int(x) for x in rng.integers(0, 2**63, size=2, dtype=np.int64)]
+        ctr = [int(x) for x in rng.integers(0, 2**62, size=4, dtype=np.int64)]
+        bg = np.random.Philox(key=np.array(key, dtype=np.uint64), counter=np.array(ctr, dtype=np.uint64))
+        raw = [int(x) for x in bg.random_raw(4)]
+        ref = O.philox_generic([ctr[0] + 1] + ctr[1:], key, **O.PHILOX4x64)
+        assert raw == ref
+
+
+def test_philox_vectorised_equals_generic():
+    rng = np.random.default_rng(9)
+    c = rng.integers(0, 2**32, size=(4, 500), dtype=np.uint64)
+    for key in [(0, 0), (0xFFFFFFFF, 0xFFFFFFFF), (123456789, 987654321)]:
+        w = O.philox4x32_10(c[0], c[1], c[2], c[3], *key)
+        for i in range(0, 500, 37):
+            ref = O.philox_generic([int(c[j, i]) for j in range(4)], key, **O.PHILOX4x32)
+            assert [int(w[j][i]) for j in range(4)] == ref
+
+
+def test_philox_top_byte_uniform_chi2():
+    e = np.arange(250_000, dtype=np.uint64)
+    w = np.concatenate(O.philox4x32_10(e, 0, 7, 3, 42, 0))
+    hist = np.bincount((w >> np.uint32(24)).astype(np.int64), minlength=256)
+    exp = w.size / 256
+    chi2 = float(((hist - exp) ** 2 / exp).sum())
+    # 255 degrees of freedom: mean 255, sd ~22.6; 6 sd bound
+    assert chi2 < 255 + 6 * math.sqrt(2 * 255)
+
+
+# ---------------------------------------------------------------- bf16
+
+def test_bf16_round_matches_torch():
+    rng = np.random.default_rng(1)
+    x = (rng.standard_normal(200_000) * np.exp2(rng.integers(-60, 60, 200_000))).astype(np.float32)
+    ties = (np.arange(1, 2001, dtype=np.uint32) << np.uint32(16)) | np.uint32(0x8000)
+    edge = np.array([0.0, -0.0, 1.0, -1.0, 3.3895314e38, 1e-40, -1e-45, np.inf, -np.inf], np.float32)
+    x = np.concatenate([x, ties.view(np.float32), edge])
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(O.bf16_bits(x), ref)
+
+
+# ---------------------------------------------------------------- quantizers
+
+def test_int4_golden_groups():
+    g = json.load(open(os.path.join(GOLDEN, "int4_groups.json")))
+    for case in g["cases"]:
+        v = np.zeros(g["group"], np.float32)
+        v[: len(case["values"])] = case["values"]
+        codes, s = O.quant_int4_groups(v, g["group"])
+        assert s.shape == (1,) and float(s[0]) == case["scale"]
+        assert codes[: len(case["codes"])].tolist() == case["codes"]
+    pk = g["packing"]
+    assert O.pack_int4(np.array(pk["codes"], np.int8)).tolist() == pk["bytes"]
+    assert O.unpack_int4(np.array(pk["bytes"], np.uint8), len(pk["codes"])).tolist() == pk["codes"]
+
+
+def test_int4_roundtrip_bound_and_idempotence():
+    rng = np.random.default_rng(2)
+    m, r = 96, 32   # groups of 64 span two rows of 32
+    P = O.qgalore.np.linalg.qr(rng.standard_normal((m, r)))[0].astype(np.float32)
+    codes, s = O.quant_int4_groups(P)
+    assert codes.min() >= -7 and codes.max() <= 7
+    deq = O.dequant_int4_f32(O.pack_int4(codes), s, m, r)
+    err = np.abs(deq - P).ravel()
+    bound = s[np.arange(m * r) // 64] / 2 * (1 + 1e-6)
+    assert np.all(err <= bound)
+    codes2, s2 = O.quant_int4_groups(deq)
+    np.testing.assert_array_equal(codes2, codes)
+    np.testing.assert_array_equal(s2, s)
+    # every group reaches +-7 at its absmax element
+    g = np.abs(codes.reshape(-1, 64)).max(axis=1)
+    assert np.all(g == 7)
+
+
+def test_int8_rowblock_golden():
+    g = json.load(open(os.path.join(GOLDEN, "int8_rowblock.json")))
+    row = np.zeros((1, 256), np.float32)
+    row[0, :5] = g["signed"]["row"]
+    c, s = O.quant_rowblock_int8(row, g["block"])
+    assert float(s[0, 0]) == g["signed"]["scale"] and c[0, :5].tolist() == g["signed"]["codes"]
+    row = np.zeros((1, 256), np.float32)
+    row[0, :4] = g["unsigned"]["row"]
+    c, s = O.quant_rowblock_int8(row, g["block"], unsigned=True)
+    assert float(s[0, 0]) == g["unsigned"]["scale"] and c[0, :4].tolist() == g["unsigned"]["codes"]
+    rg = g["ragged"]
+    row = np.zeros((1, rg["n"]), np.float32)
+    row[0, 0] = rg["head_absmax"]
+    row[0, 256:258] = rg["tail_values"]
+    c, s = O.quant_rowblock_int8(row, g["block"])
+    assert s.shape == (1, 2)
+    assert float(s[0, 0]) == rg["head_scale"] and float(s[0, 1]) == rg["tail_scale"]
+    assert c[0, 256:258].tolist() == rg["tail_codes"]
+
+
+def test_int8_rowblock_roundtrip():
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((7, 600)) * 1e-3).astype(np.float32)
+    c, s = O.quant_rowblock_int8(x, 256)
+    d = O.dequant_rowblock(c, s, 256)
+    cols = np.arange(600) // 256
+    assert np.all(np.abs(d - x) <= s[:, cols] / 2 * (1 + 1e-6))
+    c2, s2 = O.quant_rowblock_int8(d, 256)
+    np.testing.assert_array_equal(c2, c)
+    v = np.abs(x)
+    cu, su = O.quant_rowblock_int8(v, 256, unsigned=True)
+    assert cu.min() >= 0 and cu.max() == 127
+
+
+# ---------------------------------------------------------------- Adam
+
+def test_adam_matches_torch_optim_adam():
+    cfg = O.Config(m=8, n=50, r=4, lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8)
+    rng = np.random.default_rng(4)
+    shape = (4, 50)
+    p = torch.zeros(shape, dtype=torch.float64, requires_grad=True)
+    opt = torch.optim.Adam([p], lr=float(np.float32(cfg.lr)),
+                           betas=(float(np.float32(cfg.beta1)), float(np.float32(cfg.beta2))),
+                           eps=float(np.float32(cfg.eps)))
+    m0 = np.zeros(shape, np.float32)
+    v0 = np.zeros(shape, np.float32)
+    # magnitudes from 1e-9 (epsilon matters) to 1
+    scale = np.exp2(rng.integers(-30, 0, size=shape)).astype(np.float32)
+    for t in range(1, 8):
+        R = (rng.standard_normal(shape).astype(np.float32) * scale).astype(np.float32)
+        before = p.detach().clone()
+        p.grad = torch.from_numpy(R.astype(np.float64))
+        opt.step()
+        ref = (p.detach() - before).numpy()
+        N, m0, v0 = O.adam_moments(R, m0, v0, cfg, t)
+        np.testing.assert_allclose(N, ref, rtol=1e-4, atol=1e-9)
+
+
+def test_adam_first_step_closed_form():
+    cfg = O.Config(m=8, n=300, r=4)
+    rng = np.random.default_rng(6)
+    R = (rng.standard_normal((4, 300)) * 1e-2).astype(np.float32)
+    z8 = np.zeros((4, 300), np.int8)
+    z = np.zeros((4, 2), np.float32)
+    N, Mq, sM, Vq, sV = O.lowrank_adam_int8(R, z8, z, z8, z, cfg, 1)
+    # t = 1, zero moments: m_hat = R, v_hat = R^2, N = -lr R / (|R| + eps)
+    ref = -np.float64(np.float32(cfg.lr)) * R / (np.abs(R.astype(np.float64)) + np.float32(cfg.eps))
+    np.testing.assert_allclose(N, ref, rtol=2 ** -8)
+    assert np.all(np.sign(N) == -np.sign(R))
+    # second moment codes are non-negative, first-moment codes carry R's sign
+    assert Vq.min() >= 0
+    assert np.all((Mq == 0) | (np.sign(Mq) == np.sign(R)))
+
+
+# ---------------------------------------------------------------- projections
+
+def test_project_and_backproject_brute_force():
+    rng = np.random.default_rng(7)
+    m, n, r = 6, 9, 3
+    P = O.bf16_round(rng.standard_normal((m, r)).astype(np.float32))
+    G = O.bf16_round(rng.standard_normal((m, n)).astype(np.float32))
+    N = O.bf16_round(rng.standard_normal((r, n)).astype(np.float32))
+    R = O.project(P, G)
+    U = O.backproject(P, N)
+    assert R.shape == (r, n) and U.shape == (m, n)
+    for a in range(r):
+        for j in range(n):
+            s = math.fsum(float(P[i, a]) * float(G[i, j]) for i in range(m))
+            assert R[a, j] == np.float32(s)
+    for i in range(m):
+        for j in range(n):
+            s = math.fsum(float(P[i, a]) * float(N[a, j]) for a in range(r))
+            assert U[i, j] == np.float32(s)
+
+
+# ---------------------------------------------------------------- stochastic rounding
+
+def _sr(Wq, sW, U, alpha=1.0, seed=0, t=1, layer=0):
+    m, n = Wq.shape
+    cfg = O.Config(m=m, n=n, r=1, alpha=alpha, seed=seed, layer_id=layer)
+    return O.stochastic_round_update(Wq, sW, U, cfg, t)
+
+
+@pytest.mark.parametrize("x", [0.1, 0.5, 0.9, 0.01, 1e-3, -0.3, 2.75])
+def test_sr_unbiased_over_a_million_draws(x):
+    m, n = 1000, 1000
+    W = np.zeros((m, n), np.int8)
+    sW = np.ones(-(-m * n // 256), np.float32)
+    U = np.full((m, n), x, np.float32)
+    out = _sr(W, sW, U, seed=11, t=3)
+    f = math.floor(np.float32(x))
+    phi = float(np.float32(x)) - f
+    mean = out.astype(np.float64).mean()
+    sd = math.sqrt(max(phi * (1 - phi), 1e-12) / (m * n))
+    assert abs(mean - float(np.float32(x))) <= 5 * sd + 2 ** -24
+    assert set(np.unique(out).tolist()) <= {f, f + 1}
+
+
+def test_sr_integers_fixed_clamp_and_zero_scale():
+    rng = np.random.default_rng(8)
+    W = rng.integers(-120, 121, size=(64, 64)).astype(np.int8)
+    sW = np.full(16, 0.5, np.float32)
+    np.testing.assert_array_equal(_sr(W, sW, np.zeros((64, 64), np.float32)), W)
+    # x = U * alpha / s = 3 exactly
+    np.testing.assert_array_equal(_sr(W, sW, np.full((64, 64), 1.5, np.float32)), W + 3)
+    top = np.full((8, 32), 127, np.int8)
+    assert np.all(_sr(top, np.ones(1, np.float32), np.full((8, 32), 5.0, np.float32)) == 127)
+    assert np.all(_sr(-top, np.ones(1, np.float32), np.full((8, 32), -5.0, np.float32)) == -127)
+    sW0 = np.ones(16, np.float32)
+    sW0[3] = 0
+    out = _sr(W, sW0, np.full((64, 64), 7.0, np.float32))
+    flat_w, flat_o = W.ravel(), out.ravel()
+    np.testing.assert_array_equal(flat_o[3 * 256:4 * 256], flat_w[3 * 256:4 * 256])
+
+
+def test_sr_group_index_is_flattened_logical():
+    # n = 100 (not a multiple of 256): groups straddle rows; scale g applies to e // 256
+    m, n = 10, 100
+    sW = np.arange(1, 5, dtype=np.float32)   # ceil(1000/256) = 4 groups
+    U = np.ones((m, n), np.float32)
+    W = np.zeros((m, n), np.int8)
+    out = _sr(W, sW, U * 12.0, alpha=1.0)
+    e = np.arange(m * n).reshape(m, n)
+    expect = 12.0 / sW[e // 256]
+    assert np.all(np.abs(out - expect) < 1.0)
+
+
+def test_sr_uniform_draw_mapping():
+    u = O.sr_uniform24(3, 5, seed=77, t=2, layer_id=9)
+    for e in [0, 1, 4, 7, 14]:
+        i, j = divmod(e, 5)
+        w = O.philox_generic([e // 4, 0, 2, 9], [77, 0], **O.PHILOX4x32)[e % 4]
+        assert int(u[i, j]) == w >> 8
+
+
+# ---------------------------------------------------------------- composed step
+
+def _small_layer(m=64, n=96, r=32, seed=0, alpha=0.25):
+    import synth
+    cfg = O.Config(m=m, n=n, r=r, alpha=alpha, seed=seed)
+    st = O.LayerState.create(cfg, synth.weight_codes(m, n, seed), synth.weight_scales(m, n, seed=seed))
+    O.set_projection(st, synth.orthonormal(m, r, seed))
+    gen = synth.lowrank_gradient(m, n, rank=16, seed=seed)
+    return st, gen
+
+
+def test_step_alpha_zero_keeps_weights():
+    st, gen = _small_layer(alpha=0.0)
+    W0 = st.Wq.copy()
+    for t in range(3):
+        G, _ = gen.draw(t)
+        O.step(st, G)
+    np.testing.assert_array_equal(st.Wq, W0)
+    assert np.abs(st.Mq).max() > 0 and st.Vq.max() > 0
+
+
+def test_step_mean_update_is_alpha_P_N_over_scale():
+    base, gen = _small_layer()
+    G, _ = gen.draw(0)
+    diffs = []
+    for seed in range(200):
+        st = O.LayerState.create(O.Config(**{**base.cfg.__dict__, "seed": seed}), base.Wq, base.sW)
+        st.Pq, st.sP = base.Pq, base.sP
+        inter = O.step(st, G)
+        diffs.append(st.Wq.astype(np.float64) - base.Wq)
+    mean = np.mean(diffs, axis=0)
+    m, n = base.Wq.shape
+    e = np.arange(m * n).reshape(m, n)
+    expect = np.float64(base.cfg.alpha) * inter["U"] / base.sW[e // 256]
+    y = base.Wq.astype(np.float64) + expect
+    phi = y - np.floor(y)
+    sd = np.sqrt(phi * (1 - phi) / len(diffs))
+    use = (np.abs(y) < 126) & (sd > 0.01)
+    z = ((mean - expect) / np.where(use, sd, 1))[use]
+    # standardized errors: no bias, unit variance (a wrong factor or index fails)
+    assert abs(z.mean()) < 5 / math.sqrt(z.size)
+    assert 0.8 < (z ** 2).mean() < 1.2
+
+
+# ---------------------------------------------------------------- CosSim
+
+def test_cossim_closed_forms():
+    rng = np.random.default_rng(10)
+    m, r = 40, 6
+    P = np.linalg.qr(rng.standard_normal((m, r)))[0]
+    Orot = np.linalg.qr(rng.standard_normal((r, r)))[0]
+    assert abs(O.cossim(P, P) - 1) < 1e-12
+    assert abs(O.cossim(P, P @ Orot) - 1) < 1e-12
+    Pfull = np.linalg.qr(rng.standard_normal((m, 2 * r)))[0]
+    assert abs(O.cossim(Pfull[:, :r], Pfull[:, r:])) < 1e-12
+    theta = np.linspace(0.0, 1.4, r)
+    A = np.zeros((m, r))
+    B = np.zeros((m, r))
+    A[np.arange(r), np.arange(r)] = 1
+    B[np.arange(r), np.arange(r)] = np.cos(theta)
+    B[r + np.arange(r), np.arange(r)] = np.sin(theta)
+    assert abs(O.cossim(A, B) - np.cos(theta).mean()) < 1e-12
+
+
+def test_cossim_matches_scipy_subspace_angles():
+    rng = np.random.default_rng(12)
+    for m, r in [(30, 5), (64, 16)]:
+        A = np.linalg.qr(rng.standard_normal((m, r)))[0]
+        B = np.linalg.qr(A + 0.3 * rng.standard_normal((m, r)))[0]
+        ang = scipy.linalg.subspace_angles(A, B)
+        assert abs(O.cossim(A, B) - np.cos(ang).mean()) < 1e-10
+
+
+# ---------------------------------------------------------------- refresh (randomized SVD)
+
+def test_randomized_topr_full_width_equals_exact_svd():
+    rng = np.random.default_rng(13)
+    m, n, r = 40, 24, 5
+    G = rng.standard_normal((m, n)) * np.exp(-np.arange(n) / 3)[None, :]
+    k = min(m, n)
+    Om = O.rademacher_omega(n, k, 1, 0, 0)
+    P, s = O.randomized_topr(G, r, k, 2, Om)
+    Pe, se = O.exact_topr(G, r)
+    np.testing.assert_allclose(s, se, rtol=1e-10)
+    np.testing.assert_allclose(P, Pe, atol=1e-9)
+
+
+def test_randomized_topr_gap_input_matches_exact_subspace():
+    import synth
+    G, _ = synth.gap_gradient(200, 150, 12, seed=3)
+    cfg = O.Config(m=200, n=150, r=12)
+    Om = O.rademacher_omega(150, O.refresh_width(cfg), 5, 0, 0)
+    P, s = O.randomized_topr(G, 12, O.refresh_width(cfg), 2, Om)
+    Pe, se = O.exact_topr(G, 12)
+    cos = np.cos(scipy.linalg.subspace_angles(P, Pe))
+    assert cos.min() > 0.99999
+    np.testing.assert_allclose(s, se, rtol=1e-6)
+    np.testing.assert_allclose(P.T @ P, np.eye(12), atol=1e-12)
+
+
+def test_randomized_range_exact_on_rank_k_input():
+    rng = np.random.default_rng(14)
+    m, n, k = 60, 50, 8
+    G = rng.standard_normal((m, k)) @ rng.standard_normal((k, n))
+    Om = O.rademacher_omega(n, k, 2, 0, 0)
+    P, _ = O.randomized_topr(G, k, k, 0, Om)
+    # P spans range(G) exactly
+    resid = G - P @ (P.T @ G)
+    assert np.abs(resid).max() < 1e-9 * np.abs(G).max()
+
+
+def test_canonical_signs_rule():
+    P = np.array([[0.1, -0.9], [-0.8, 0.2], [0.3, 0.9]])
+    C = O.canonical_signs(P)
+    np.testing.assert_array_equal(C[:, 0], -P[:, 0])   # largest |.| is -0.8 -> flip
+    np.testing.assert_array_equal(C[:, 1], -P[:, 1])   # tie 0.9: first row (-0.9) decides
+
+
+def test_omega_rademacher_mapping():
+    n, k = 37, 11
+    Om = O.rademacher_omega(n, k, seed=0xABCDEF0123, refresh_idx=4, layer_id=6)
+    assert set(np.unique(Om).tolist()) <= {-1.0, 1.0}
+    for e in [0, 31, 32, 127, 128, 300, n * k - 1]:
+        w = O.philox_generic([e // 128, 4, 6, 0],
+                             [(0xABCDEF0123 & 0xFFFFFFFF) ^ O.OMEGA_KEY_SALT, 0xABCDEF0123 >> 32],
+                             **O.PHILOX4x32)[(e // 32) % 4]
+        bit = (w >> (e % 32)) & 1
+        assert Om.ravel()[e] == (-1.0 if bit else 1.0)
+    big = O.rademacher_omega(1000, 400, 1, 0, 0)
+    assert abs(big.mean()) < 5 / math.sqrt(big.size)
+    assert not np.array_equal(big, O.rademacher_omega(1000, 400, 1, 1, 0))
+
+
+# ---------------------------------------------------------------- schedule
+
+def test_schedule_doubling_rule_scripted():
+    seq = [None, 0.5, 0.3, 0.41, 0.4, 0.9]
+    t, delta, log = 0, 200, []
+    for cs in seq:
+        delta, t_next = O.schedule_after_refresh(t, delta, cs, 0.4)
+        log.append((t, delta, t_next))
+        t = t_next
+    assert log == [(0, 200, 200), (200, 400, 600), (600, 400, 1000),
+                   (1000, 800, 1800), (1800, 800, 2600), (2600, 1600, 4200)]
+
+
+def test_schedule_gamma_limits():
+    # gamma > 1: CosSim <= 1 never exceeds it -> GaLore's fixed interval
+    t, delta = 0, 50
+    for cs in [None, 1.0, 0.99, 1.0]:
+        delta, t = O.schedule_after_refresh(t, delta, cs, 1.5)
+    assert delta == 50 and t == 200
+    t, delta = 0, 50
+    for cs in [None, 0.0, 0.1]:
+        delta, t = O.schedule_after_refresh(t, delta, cs, -1.5)
+    assert delta == 200 and t == 50 + 100 + 200
+
+
+def test_refresh_layer_state_flow():
+    import synth
+    m, n, r = 64, 80, 8
+    cfg = O.Config(m=m, n=n, r=r, delta0=3, gamma=0.4, seed=1)
+    st = O.LayerState.create(cfg, synth.weight_codes(m, n), synth.weight_scales(m, n))
+    gen = synth.lowrank_gradient(m, n, rank=8, s0=1.0, decay=0.7, sigma=1e-4, seed=1)
+    counts = []
+    for t in range(10):
+        G, _ = gen.draw(t)
+        info = O.refresh(st, G, force=(t == 0))
+        counts.append(info is not None)
+        O.step(st, G)
+    # refreshes at t = 0, 3 (cs ~ 1 -> delta 6), 9
+    assert counts == [True, False, False, True, False, False, False, False, False, True]
+    assert st.cossim_trace[0][1] is None and st.cossim_trace[1][1] > 0.9
+    assert st.n_refresh == 3
