@@ -1,0 +1,204 @@
+/*
+ * qgalore.h - C ABI of the B200 (sm_100a) Q-GaLore optimizer-step library.
+ *
+ * The method (sources: the paper-index record "Q-GaLore: Quantized GaLore with
+ * INT4 Projection and Layer-Adaptive Low-Rank Gradients", abstract; the AIMech
+ * curated page on Q-GaLore, mechanisms "layer-adaptive subspace cosine
+ * schedule" (paper section 3.1, Eq. (5)) and "INT4 projection and INT8
+ * stochastic rounding" (paper section 3.2)):
+ *
+ *   per weight matrix W (m x n, INT8 codes with fixed float32 group scales)
+ *     a1  P~ = bf16(dequant(P^Q))             P^Q: m x r INT4, one scale / 64
+ *     a2  R  = P~^T G                          G: m x n bf16 gradient
+ *     a3  Adam on (M^Q, V^Q), r x n INT8 with per-row-block scales -> N (bf16)
+ *     a4  U  = P~ N
+ *     a5  W^Q <- W^Q + xi(alpha U / s_W)       xi: unbiased stochastic rounding
+ *   beside it, when due: top-r randomized SVD of G -> new P^Q; CosSim against
+ *   the previous P^Q; the refresh interval doubles when CosSim > gamma.
+ *
+ * Conventions for every entry point:
+ *   - Arrays are row-major.  Pointers named d_* are DEVICE pointers; they are
+ *     owned by the caller, who allocates and frees them (e.g. with PyTorch).
+ *     The library owns only the opaque host handle qg_layer.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously on it; only qg_refresh (when a
+ *     refresh runs) and qg_layer_status wait for the device.
+ *   - A handle must not be used from two streams at once.
+ *   - Argument errors are reported before anything is enqueued: nothing is
+ *     launched and the state is unchanged.  Launch failures return QG_ECUDA.
+ *     Errors found by kernels (a device wait that ran out, a non-finite
+ *     gradient projection) set bits of the layer's device status word, read
+ *     and cleared by qg_layer_status.
+ *   - bf16 arrays are passed as void* (16-bit patterns).
+ *   - Nothing here allocates device memory.
+ */
+#ifndef QGALORE_H
+#define QGALORE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QG_OK = 0,
+  QG_EINVAL = 1,      /* null pointer or hyper-parameter out of range */
+  QG_ESHAPE = 2,      /* unsupported sizes */
+  QG_EALIGN = 3,      /* pointer or leading dimension not aligned as required */
+  QG_ESTATE = 4,      /* buffer too small, or the layer has no projection yet */
+  QG_ECUDA = 5,       /* CUDA runtime or driver error */
+  QG_ETIMEOUT = 6,    /* a bounded device wait gave up (kernel returned early) */
+  QG_ENONFINITE = 7   /* a non-finite value was met on the device */
+} qg_status;
+
+/* Hyper-parameters of one weight matrix.  qg_config_default fills the values
+ * used by the paper's setting where the pages give one (gamma = 0.4) and the
+ * plain readings elsewhere. */
+typedef struct {
+  int32_t m, n, r;          /* W is m x n, P is m x r; 32 <= r <= min(m, n), r % 32 == 0 */
+  int32_t w_group;          /* weight-scale group (consecutive elements), must be 256 */
+  int32_t p_group;          /* INT4 projection group, must be 64 */
+  int32_t mom_block;        /* moment block along a row, must be 256 */
+  float beta1, beta2, eps;  /* Adam: 0.9, 0.999, 1e-8 */
+  float lr;                 /* learning rate, 1e-3 */
+  float alpha;              /* scale of the low-rank update, 0.25 */
+  float gamma;              /* CosSim threshold, 0.4 */
+  int32_t delta0;           /* initial refresh interval (steps), 200 */
+  int32_t oversample;       /* randomized SVD oversampling p, 16 */
+  int32_t power_iters;      /* randomized SVD power iterations q, 2 */
+  uint64_t seed;            /* Philox key of the stochastic rounding and of Omega */
+  uint32_t layer_id;        /* Philox counter word: distinguishes matrices */
+} qg_config;
+
+typedef struct qg_layer qg_layer;
+
+/* Device pointers into a layer's state (for inspection, checkpointing). */
+typedef struct {
+  uint32_t* status;         /* device status word (bits: 1 timeout, 2 non-finite) */
+  uint8_t* Pq;              /* ceil(m*r/2) bytes: INT4 P, two nibbles per byte, even index low */
+  float* sP;                /* ceil(m*r/64) float32 scales */
+  uint8_t* Pq_prev;         /* previous projection (for CosSim) */
+  float* sP_prev;
+  int8_t* Mq;               /* r x ld_mom INT8 first moment (columns >= n unused) */
+  int8_t* Vq;               /* r x ld_mom INT8 second moment, codes 0..127 */
+  float* sM;                /* r x nblk float32 */
+  float* sV;                /* r x nblk float32 */
+  int64_t ld_mom;           /* row stride of Mq, Vq in bytes: n rounded up to 32 */
+  int32_t nblk;             /* ceil(n / 256) */
+} qg_layer_views;
+
+/* Schedule state of the layer-adaptive refresh (host side). */
+typedef struct {
+  int64_t t;                /* steps taken (the next step is t + 1) */
+  int32_t delta;            /* current refresh interval */
+  int64_t t_next;           /* a refresh is due when t == t_next */
+  int32_t n_refresh;        /* refreshes done so far */
+  int32_t has_projection;   /* a projection has been installed or computed */
+} qg_sched;
+
+typedef struct {
+  int32_t refreshed;        /* 1 if a refresh ran in this call */
+  int32_t has_cossim;       /* 1 if a previous projection existed */
+  float cossim;             /* CosSim(P_new, P_prev), Eq. (5) of the paper */
+  int32_t delta;            /* interval after the call */
+  int64_t t_next;           /* next due step after the call */
+  int32_t n_refresh;
+} qg_refresh_info;
+
+const char* qg_status_str(qg_status s);
+void qg_config_default(qg_config* cfg, int32_t m, int32_t n, int32_t r);
+
+/* Sizes of the caller-provided buffers (bytes).  The state holds what a layer
+ * carries between steps; the workspace is scratch for one call and may be
+ * shared by layers that run one after another on the same stream. */
+size_t qg_state_bytes(const qg_config* cfg);
+size_t qg_step_workspace_bytes(const qg_config* cfg);
+size_t qg_refresh_workspace_bytes(const qg_config* cfg);
+
+/* Create a layer handle over caller-owned device memory.
+ *   d_state : >= qg_state_bytes(cfg) bytes, 256-byte aligned; zero-initialised
+ *             here (moments and scales start at zero) on `stream`.
+ *   d_W     : m x ldw INT8 weight codes, 16-byte aligned, ldw >= n, ldw % 16 == 0;
+ *             updated in place by qg_step.
+ *   d_Wscale: ceil(m*n/256) float32 scales, group g covering logical elements
+ *             [256 g, 256 g + 256) of the row-major m x n array; read only.
+ * Returns QG_EINVAL / QG_ESHAPE / QG_EALIGN / QG_ESTATE on bad arguments. */
+qg_status qg_layer_init(qg_layer** out, const qg_config* cfg, void* d_state, size_t state_bytes,
+                        int8_t* d_W, int64_t ldw, const float* d_Wscale, void* stream);
+qg_status qg_layer_destroy(qg_layer* layer);
+qg_status qg_layer_views_get(const qg_layer* layer, qg_layer_views* views);
+qg_status qg_layer_sched_get(const qg_layer* layer, qg_sched* sched);
+qg_status qg_layer_sched_set(qg_layer* layer, const qg_sched* sched);
+
+/* Install an INT4 projection (e.g. from a checkpoint): copies ceil(m*r/2)
+ * packed bytes and ceil(m*r/64) scales device-to-device into the state.  The
+ * previous projection is kept for CosSim only when keep_prev != 0. */
+qg_status qg_layer_set_projection(qg_layer* layer, const uint8_t* d_Pq, const float* d_sP,
+                                  int32_t keep_prev, void* stream);
+
+/* One optimizer step a1..a5 (paper section 3.2) on one matrix.
+ *   d_G : m x ldg bf16 gradient, 16-byte aligned, ldg >= n, ldg % 8 == 0.
+ *   d_ws: >= qg_step_workspace_bytes(cfg) bytes, 256-byte aligned.
+ * Never refreshes; QG_ESTATE if no projection is installed. */
+qg_status qg_step(qg_layer* layer, const void* d_G, int64_t ldg, void* d_ws, size_t ws_bytes,
+                  void* stream);
+
+/* The same step for `count` matrices in few launches (one persistent grid per
+ * stage for up to 8 matrices).  d_ws must hold the sum of the matrices'
+ * qg_step_workspace_bytes, each rounded up to 256. */
+qg_status qg_step_batch(qg_layer* const* layers, const void* const* d_G, const int64_t* ldg,
+                        int32_t count, void* d_ws, size_t ws_bytes, void* stream);
+size_t qg_step_batch_workspace_bytes(const qg_config* const* cfgs, int32_t count);
+
+/* Layer-adaptive subspace refresh (paper section 3.1, Eq. (5)).  Runs when
+ * force != 0 or the layer is due (t == t_next); otherwise returns QG_OK with
+ * info->refreshed = 0 and touches nothing.  When it runs: randomized top-r SVD
+ * of G -> new INT4 P; if a projection existed, CosSim(P_new, P_prev) on the
+ * device; the interval doubles iff CosSim > gamma; t_next = t + delta.  This
+ * call synchronises `stream` to read CosSim.  `info` may be NULL. */
+qg_status qg_refresh(qg_layer* layer, const void* d_G, int64_t ldg, int32_t force, void* d_ws,
+                     size_t ws_bytes, qg_refresh_info* info, void* stream);
+
+/* CosSim(Pa, Pb) = (1/r) sum_i sigma_i(Pa^T Pb) for float32 m x r matrices with
+ * row stride ld (elements), result written to d_out[0] on the device.
+ * d_ws >= qg_cossim_workspace_bytes(m, r). */
+size_t qg_cossim_workspace_bytes(int32_t m, int32_t r);
+qg_status qg_cossim(const float* d_Pa, const float* d_Pb, int32_t m, int32_t r, int64_t ld,
+                    float* d_out, void* d_ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, reads and clears the layer's device status word:
+ * QG_OK, QG_ETIMEOUT or QG_ENONFINITE. */
+qg_status qg_layer_status(qg_layer* layer, void* stream);
+
+/* Host-only rule of the paper's layer-adaptive schedule: after a refresh at
+ * step t, delta doubles iff has_cossim and cossim > gamma; t_next = t + delta. */
+qg_status qg_sched_after_refresh(int64_t t, int32_t delta, int32_t has_cossim, float cossim,
+                                 float gamma, int32_t* delta_out, int64_t* t_next_out);
+
+/* ---- Single-stage entry points (used by the tests to check each stage) ---- */
+
+/* Philox-4x32-10 words for `count` counters given as four device arrays of
+ * uint32 (c0[i], c1[i], c2[i], c3[i]); writes out[4*i + w]. */
+qg_status qg_philox4x32_10(const uint32_t* d_c0, const uint32_t* d_c1, const uint32_t* d_c2,
+                           const uint32_t* d_c3, int64_t count, uint32_t k0, uint32_t k1,
+                           uint32_t* d_out, void* stream);
+
+/* Stage a1: P~ (m x r bf16, row stride r) from packed INT4 codes and scales. */
+qg_status qg_dequant_projection(const uint8_t* d_Pq, const float* d_sP, int32_t m, int32_t r,
+                                void* d_out_bf16, void* stream);
+
+/* D (M x N float32, row stride ldd) = A B on the tcgen05 tensor cores, bf16
+ * operands, float32 accumulation.  A is M x K given as row-major M x K
+ * (a_trans = 0, stride lda) or as row-major K x M (a_trans = 1); B is K x N
+ * given as row-major K x N (b_trans = 0) or as row-major N x K (b_trans = 1).
+ * Strides in elements, multiples of 8; pointers 16-byte aligned. */
+qg_status qg_gemm_bf16(const void* d_A, int64_t lda, int32_t a_trans, const void* d_B, int64_t ldb,
+                       int32_t b_trans, float* d_D, int64_t ldd, int32_t M, int32_t N, int32_t K,
+                       void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QGALORE_H */

@@ -1,0 +1,526 @@
+// The optimizer step a1..a5 on sm_100a.
+//
+//   a1  dequant_projection_kernel : INT4 P^Q -> P~ (bf16, m x r) in scratch
+//   a2+a3  gemm_tc_kernel<AdamEpi, A MN-major, B MN-major>:
+//          R = P~^T G in TMEM; the epilogue runs Adam on the INT8 moments,
+//          re-quantizes them and writes N (bf16, r x n) to scratch.  R never
+//          leaves the SM.
+//   a4+a5  gemm_tc_kernel<StochRoundEpi, A K-major, B MN-major>:
+//          U = P~ N in TMEM; the epilogue adds alpha*U/s_W to the INT8 weights
+//          with Philox-keyed stochastic rounding.  U never leaves the SM.
+//
+// Arithmetic follows the Q-GaLore step as described on the AIMech Q-GaLore
+// page (mechanism "INT4 projection and INT8 stochastic rounding", paper
+// section 3.2) with the readings documented in the repository's design notes;
+// every float32 operation that decides a code uses an explicitly rounded
+// intrinsic so that no multiply-add is contracted.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "qg_gemm.cuh"
+#include "qg_internal.h"
+#include "qg_philox.cuh"
+#include "qg_refresh.h"
+
+namespace qg {
+
+static_assert(kErrTimeout == kStatusTimeout && kErrNonFinite == kStatusNonFinite, "status bits");
+
+// ------------------------------------------------------------------ helpers
+
+QG_DEV int8_t byte_of(const uint4& v, int k) {
+  const uint32_t w = k < 4 ? v.x : k < 8 ? v.y : k < 12 ? v.z : v.w;
+  return static_cast<int8_t>((w >> (8 * (k & 3))) & 0xFFu);
+}
+
+QG_DEV uint16_t bf16_bits_rn(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+// ------------------------------------------------------------------ a2 + a3 epilogue
+
+struct AdamEpi {
+  struct Args {
+    int8_t* Mq;
+    int8_t* Vq;
+    float* sM;
+    float* sV;
+    uint16_t* Nout;
+    int64_t ld_mom;
+    int64_t ldN;
+    int32_t nblk;
+    float beta1, beta2, om1, om2, bc1, bc2, neg_lr, eps;
+  };
+
+  // m = b1*m0 + (1-b1)*R ; v = b2*v0 + (1-b2)*(R*R), one rounding per operation.
+  static QG_DEV void moments(float R, int8_t mc, int8_t vc, float sm, float sv, const Args& a,
+                             float& mm, float& vv) {
+    const float m0 = __fmul_rn(static_cast<float>(mc), sm);
+    const float v0 = __fmul_rn(static_cast<float>(vc), sv);
+    mm = __fadd_rn(__fmul_rn(a.beta1, m0), __fmul_rn(a.om1, R));
+    vv = __fadd_rn(__fmul_rn(a.beta2, v0), __fmul_rn(a.om2, __fmul_rn(R, R)));
+  }
+
+  // One thread owns row `row` of the 128 x 256 tile: rows are moment rows a,
+  // the 256 columns are exactly one moment block (BN == 256 == block).
+  static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
+                           uint32_t* status) {
+    const int arow = mb * BM + row;
+    const bool row_ok = arow < M;
+    const int j0 = nb * BN;
+    const int ncols = min(BN, N - j0);
+    const int nchunks = (ncols + 31) >> 5;
+    float sm = 0.f, sv = 0.f;
+    int8_t* mrow = nullptr;
+    int8_t* vrow = nullptr;
+    uint16_t* nrow = nullptr;
+    if (row_ok) {
+      sm = a.sM[static_cast<int64_t>(arow) * a.nblk + nb];
+      sv = a.sV[static_cast<int64_t>(arow) * a.nblk + nb];
+      mrow = a.Mq + static_cast<int64_t>(arow) * a.ld_mom + j0;
+      vrow = a.Vq + static_cast<int64_t>(arow) * a.ld_mom + j0;
+      nrow = a.Nout + static_cast<int64_t>(arow) * a.ldN + j0;
+    }
+    float amax_m = 0.f, amax_v = 0.f;
+    bool bad = false;
+
+    // pass 1: moments, block absmax, N = -lr * m_hat / (sqrt(v_hat) + eps) -> bf16
+    for (int c = 0; c < nchunks; ++c) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(taddr + c * 32, v);
+      tmem_ld_wait();
+      if (!row_ok) continue;
+      const uint4 mq0 = *reinterpret_cast<const uint4*>(mrow + c * 32);
+      const uint4 mq1 = *reinterpret_cast<const uint4*>(mrow + c * 32 + 16);
+      const uint4 vq0 = *reinterpret_cast<const uint4*>(vrow + c * 32);
+      const uint4 vq1 = *reinterpret_cast<const uint4*>(vrow + c * 32 + 16);
+      const int valid = ncols - c * 32;
+      uint32_t packed[16];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float R = __uint_as_float(v[e]);
+        const int8_t mc = e < 16 ? byte_of(mq0, e) : byte_of(mq1, e - 16);
+        const int8_t vc = e < 16 ? byte_of(vq0, e) : byte_of(vq1, e - 16);
+        float mm, vv;
+        moments(R, mc, vc, sm, sv, a, mm, vv);
+        if (e < valid) {
+          amax_m = fmaxf(amax_m, fabsf(mm));
+          amax_v = fmaxf(amax_v, vv);
+          bad |= !isfinite(R);
+        }
+        const float mhat = __fdiv_rn(mm, a.bc1);
+        const float vhat = __fdiv_rn(vv, a.bc2);
+        const float upd = __fdiv_rn(__fmul_rn(a.neg_lr, mhat), __fadd_rn(__fsqrt_rn(vhat), a.eps));
+        const uint32_t b = bf16_bits_rn(upd);
+        if (e & 1)
+          packed[e >> 1] |= b << 16;
+        else
+          packed[e >> 1] = b;
+      }
+      uint4* dst = reinterpret_cast<uint4*>(nrow + c * 32);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+    }
+
+    // new block scales: absmax / 127 (IEEE division); zero block -> scale 0
+    const float s_m = __fdiv_rn(amax_m, 127.0f);
+    const float s_v = __fdiv_rn(amax_v, 127.0f);
+
+    // pass 2: recompute the same moments bit for bit, re-quantize them
+    for (int c = 0; c < nchunks; ++c) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(taddr + c * 32, v);
+      tmem_ld_wait();
+      if (!row_ok) continue;
+      const uint4 mq0 = *reinterpret_cast<const uint4*>(mrow + c * 32);
+      const uint4 mq1 = *reinterpret_cast<const uint4*>(mrow + c * 32 + 16);
+      const uint4 vq0 = *reinterpret_cast<const uint4*>(vrow + c * 32);
+      const uint4 vq1 = *reinterpret_cast<const uint4*>(vrow + c * 32 + 16);
+      uint32_t om[8], ov[8];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float R = __uint_as_float(v[e]);
+        const int8_t mc = e < 16 ? byte_of(mq0, e) : byte_of(mq1, e - 16);
+        const int8_t vc = e < 16 ? byte_of(vq0, e) : byte_of(vq1, e - 16);
+        float mm, vv;
+        moments(R, mc, vc, sm, sv, a, mm, vv);
+        int qm = 0, qv = 0;
+        if (s_m > 0.f) qm = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(mm, s_m)), -127.f), 127.f));
+        if (s_v > 0.f) qv = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(vv, s_v)), 0.f), 127.f));
+        const uint32_t bm = static_cast<uint32_t>(qm) & 0xFFu;
+        const uint32_t bv = static_cast<uint32_t>(qv) & 0xFFu;
+        if ((e & 3) == 0) {
+          om[e >> 2] = bm;
+          ov[e >> 2] = bv;
+        } else {
+          om[e >> 2] |= bm << (8 * (e & 3));
+          ov[e >> 2] |= bv << (8 * (e & 3));
+        }
+      }
+      *reinterpret_cast<uint4*>(mrow + c * 32) = make_uint4(om[0], om[1], om[2], om[3]);
+      *reinterpret_cast<uint4*>(mrow + c * 32 + 16) = make_uint4(om[4], om[5], om[6], om[7]);
+      *reinterpret_cast<uint4*>(vrow + c * 32) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+      *reinterpret_cast<uint4*>(vrow + c * 32 + 16) = make_uint4(ov[4], ov[5], ov[6], ov[7]);
+    }
+    if (row_ok) {
+      a.sM[static_cast<int64_t>(arow) * a.nblk + nb] = s_m;
+      a.sV[static_cast<int64_t>(arow) * a.nblk + nb] = s_v;
+    }
+    if (bad && status) atomicOr(status, kErrNonFinite);
+  }
+};
+
+// ------------------------------------------------------------------ a4 + a5 epilogue
+
+struct StochRoundEpi {
+  struct Args {
+    int8_t* W;
+    const float* sW;
+    int64_t ldw;
+    float alpha;
+    uint32_t t, layer_id;
+    PhiloxKey key;
+    int32_t aligned4;  // n % 4 == 0: every 32-column chunk starts a Philox quad
+  };
+
+  static QG_DEV float coef(const float* sW, int64_t g, float alpha) {
+    const float s = sW[g];
+    return s > 0.f ? __fdiv_rn(alpha, s) : 0.f;
+  }
+
+  template <bool kAligned4>
+  static QG_DEV void words(const Args& a, int64_t e0, uint32_t (&w)[32]) {
+    const uint64_t qb = static_cast<uint64_t>(e0) >> 2;
+    if (kAligned4) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        uint32_t o[4];
+        const uint64_t q = qb + k;
+        philox4x32_10(static_cast<uint32_t>(q), static_cast<uint32_t>(q >> 32), a.t, a.layer_id, a.key, o);
+        w[4 * k] = o[0];
+        w[4 * k + 1] = o[1];
+        w[4 * k + 2] = o[2];
+        w[4 * k + 3] = o[3];
+      }
+    } else {
+      uint32_t ww[36];
+#pragma unroll
+      for (int k = 0; k < 9; ++k) {
+        uint32_t o[4];
+        const uint64_t q = qb + k;
+        philox4x32_10(static_cast<uint32_t>(q), static_cast<uint32_t>(q >> 32), a.t, a.layer_id, a.key, o);
+        ww[4 * k] = o[0];
+        ww[4 * k + 1] = o[1];
+        ww[4 * k + 2] = o[2];
+        ww[4 * k + 3] = o[3];
+      }
+      const int s = static_cast<int>(e0 & 3);
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        w[k] = s == 0 ? ww[k] : s == 1 ? ww[k + 1] : s == 2 ? ww[k + 2] : ww[k + 3];
+    }
+  }
+
+  template <bool kAligned4>
+  static QG_DEV void apply_impl(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr) {
+    const int irow = mb * BM + row;
+    const bool row_ok = irow < M;
+    const int j0 = nb * BN;
+    const int ncols = min(BN, N - j0);
+    const int nchunks = (ncols + 31) >> 5;
+    for (int c = 0; c < nchunks; ++c) {
+      uint32_t U[32];
+      tmem_ld_32x32b_x32(taddr + c * 32, U);
+      tmem_ld_wait();
+      if (!row_ok) continue;
+      const int jc = j0 + c * 32;
+      const int valid = min(32, N - jc);
+      const int64_t e0 = static_cast<int64_t>(irow) * N + jc;
+      const int64_t g0 = e0 >> 8;
+      const int64_t g1 = (e0 + valid - 1) >> 8;
+      const float c0 = coef(a.sW, g0, a.alpha);
+      const float c1 = g1 != g0 ? coef(a.sW, g1, a.alpha) : c0;
+      const int split = g1 != g0 ? static_cast<int>((g1 << 8) - e0) : 32;
+      int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + jc;
+      uint4 q0 = make_uint4(0, 0, 0, 0), q1 = make_uint4(0, 0, 0, 0);
+      q0 = *reinterpret_cast<const uint4*>(wrow);
+      if (valid > 16) q1 = *reinterpret_cast<const uint4*>(wrow + 16);
+      uint32_t w[32];
+      words<kAligned4>(a, e0, w);
+      uint32_t out[8];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const int8_t q = k < 16 ? byte_of(q0, k) : byte_of(q1, k - 16);
+        const float ck = k < split ? c0 : c1;
+        const float x = __fmul_rn(__uint_as_float(U[k]), ck);
+        const float y = __fadd_rn(static_cast<float>(q), x);
+        const float f = floorf(y);
+        const float phi = __fsub_rn(y, f);
+        const bool up = __uint2float_rn(w[k] >> 8) < __fmul_rn(phi, 16777216.0f);
+        float qf = __fadd_rn(f, up ? 1.0f : 0.0f);
+        qf = fminf(fmaxf(qf, -127.0f), 127.0f);
+        const int res = (y != y) ? static_cast<int>(q) : static_cast<int>(qf);
+        const uint32_t b = static_cast<uint32_t>(res) & 0xFFu;
+        if ((k & 3) == 0)
+          out[k >> 2] = b;
+        else
+          out[k >> 2] |= b << (8 * (k & 3));
+      }
+      if (valid == 32) {
+        *reinterpret_cast<uint4*>(wrow) = make_uint4(out[0], out[1], out[2], out[3]);
+        *reinterpret_cast<uint4*>(wrow + 16) = make_uint4(out[4], out[5], out[6], out[7]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (k < valid) wrow[k] = static_cast<int8_t>((out[k >> 2] >> (8 * (k & 3))) & 0xFFu);
+      }
+    }
+  }
+
+  static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
+                           uint32_t* /*status*/) {
+    if (a.aligned4)
+      apply_impl<true>(a, M, N, mb, nb, row, taddr);
+    else
+      apply_impl<false>(a, M, N, mb, nb, row, taddr);
+  }
+};
+
+// ------------------------------------------------------------------ plain fp32 store
+
+struct StoreF32Epi {
+  struct Args {
+    float* D;
+    int64_t ldd;
+  };
+  static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
+                           uint32_t* /*status*/) {
+    const int grow = mb * BM + row;
+    const bool ok = grow < M;
+    const int j0 = nb * BN;
+    const int ncols = min(BN, N - j0);
+    const int nchunks = (ncols + 31) >> 5;
+    for (int c = 0; c < nchunks; ++c) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(taddr + c * 32, v);
+      tmem_ld_wait();
+      if (!ok) continue;
+      float* d = a.D + static_cast<int64_t>(grow) * a.ldd + j0 + c * 32;
+      const int valid = ncols - c * 32;
+      if (valid >= 32) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          reinterpret_cast<float4*>(d)[q] =
+              make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                          __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (e < valid) d[e] = __uint_as_float(v[e]);
+      }
+    }
+  }
+};
+
+static_assert(sizeof(GemmParams<AdamEpi>) <= 4096, "kernel parameter block");
+static_assert(sizeof(GemmParams<StochRoundEpi>) <= 4096, "kernel parameter block");
+static_assert(sizeof(GemmParams<StoreF32Epi>) <= 4096, "kernel parameter block");
+
+// ------------------------------------------------------------------ a1 and test kernels
+
+// Eight INT4 codes (one 32-bit word, element 2i in the low nibble of byte i)
+// -> eight bf16 of P~ = bf16_rn(code * scale).  Groups of 64 never split a word.
+__global__ void dequant_projection_kernel(const uint8_t* __restrict__ Pq, const float* __restrict__ sP,
+                                          int64_t total, uint16_t* __restrict__ out) {
+  const int64_t i8 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t e0 = i8 * 8;
+  if (e0 >= total) return;
+  const uint32_t word = *reinterpret_cast<const uint32_t*>(Pq + (e0 >> 1));
+  const float s = sP[e0 >> 6];
+  uint32_t pk[4];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int nib = static_cast<int>((word >> (4 * k)) & 0xFu);
+    const int code = (nib ^ 8) - 8;
+    const uint32_t b = bf16_bits_rn(__fmul_rn(static_cast<float>(code), s));
+    if (k & 1)
+      pk[k >> 1] |= b << 16;
+    else
+      pk[k >> 1] = b;
+  }
+  *reinterpret_cast<uint4*>(out + e0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+}
+
+__global__ void philox_kernel(const uint32_t* c0, const uint32_t* c1, const uint32_t* c2, const uint32_t* c3,
+                              int64_t count, PhiloxKey key, uint32_t* out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= count) return;
+  uint32_t o[4];
+  philox4x32_10(c0[i], c1[i], c2[i], c3[i], key, o);
+  reinterpret_cast<uint4*>(out)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// ------------------------------------------------------------------ host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+static std::once_flag g_encode_once;
+
+bool encode_map_bf16(void* map, const void* base, uint64_t inner, uint64_t outer, uint64_t ld_elems,
+                     uint32_t box_inner, uint32_t box_outer) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {ld_elems * 2};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(reinterpret_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+int64_t step_ldN(int32_t n) { return (static_cast<int64_t>(n) + 31) / 32 * 32; }
+
+static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+size_t step_scratch_bytes(int32_t m, int32_t n, int32_t r) {
+  return round256(static_cast<size_t>(m) * r * 2) + round256(static_cast<size_t>(r) * step_ldN(n) * 2);
+}
+
+template <class Epi, bool kAMN, bool kBMN>
+static cudaError_t launch_gemm(const GemmParams<Epi>& p, cudaStream_t stream) {
+  auto kern = gemm_tc_kernel<Epi, kAMN, kBMN>;
+  static bool attr_set = false;  // per instantiation
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kGemmSmemBytes));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  if (p.total_tiles == 0) return cudaSuccess;
+  const int grid = std::min(p.total_tiles, sm_count());
+  kern<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <class Epi>
+static void add_problem(GemmParams<Epi>& p, int M, int N, int K) {
+  GemmProblem<Epi>& pr = p.prob[p.nprob];
+  pr.M = M;
+  pr.N = N;
+  pr.K = K;
+  pr.tiles_m = (M + BM - 1) / BM;
+  pr.tiles_n = (N + BN - 1) / BN;
+  pr.tile_begin = p.total_tiles;
+  p.total_tiles += pr.tiles_m * pr.tiles_n;
+  p.nprob += 1;
+}
+
+cudaError_t launch_dequant_projection(const uint8_t* Pq, const float* sP, int64_t total, uint16_t* out,
+                                      cudaStream_t stream) {
+  const int64_t chunks = total / 8;
+  if (chunks == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (chunks + threads - 1) / threads;
+  dequant_projection_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(Pq, sP, total, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_philox(const uint32_t* c0, const uint32_t* c1, const uint32_t* c2, const uint32_t* c3,
+                          int64_t count, uint32_t k0, uint32_t k1, uint32_t* out, cudaStream_t stream) {
+  if (count == 0) return cudaSuccess;
+  const int threads = 256;
+  philox_kernel<<<static_cast<unsigned>((count + threads - 1) / threads), threads, 0, stream>>>(
+      c0, c1, c2, c3, count, PhiloxKey{k0, k1}, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream) {
+  cudaError_t e;
+  for (int i = 0; i < count; ++i) {
+    e = launch_dequant_projection(probs[i].Pq, probs[i].sP, static_cast<int64_t>(probs[i].m) * probs[i].r,
+                                  probs[i].Pbf, stream);
+    if (e != cudaSuccess) return e;
+  }
+  for (int base = 0; base < count; base += kMaxProblems) {
+    const int cnt = std::min(kMaxProblems, count - base);
+    GemmParams<AdamEpi> p1;
+    memset(&p1, 0, sizeof(p1));
+    for (int i = 0; i < cnt; ++i) {
+      const StepProblem& s = probs[base + i];
+      GemmProblem<AdamEpi>& pr = p1.prob[p1.nprob];
+      // A = P~^T (M = r, K = m), MN-major over P~ (m x r): box {64 (r), 64 (m)}
+      if (!encode_map_bf16(&pr.tmA, s.Pbf, s.r, s.m, s.r, 64, 64)) return cudaErrorInvalidValue;
+      // B = G (K = m, N = n), MN-major: box {64 (n), 64 (m)}
+      if (!encode_map_bf16(&pr.tmB, s.G, s.n, s.m, s.ldg, 64, 64)) return cudaErrorInvalidValue;
+      pr.status = s.status;
+      pr.epi = AdamEpi::Args{s.Mq, s.Vq, s.sM, s.sV, s.Nbuf, s.ld_mom, s.ldN, s.nblk,
+                             s.beta1, s.beta2, s.om1, s.om2, s.bc1, s.bc2, s.neg_lr, s.eps};
+      add_problem(p1, s.r, s.n, s.m);
+    }
+    e = launch_gemm<AdamEpi, true, true>(p1, stream);
+    if (e != cudaSuccess) return e;
+
+    GemmParams<StochRoundEpi> p2;
+    memset(&p2, 0, sizeof(p2));
+    for (int i = 0; i < cnt; ++i) {
+      const StepProblem& s = probs[base + i];
+      GemmProblem<StochRoundEpi>& pr = p2.prob[p2.nprob];
+      // A = P~ (M = m, K = r), K-major: box {64 (r), 128 (m)}
+      if (!encode_map_bf16(&pr.tmA, s.Pbf, s.r, s.m, s.r, 64, 128)) return cudaErrorInvalidValue;
+      // B = N (K = r, N = n), MN-major: box {64 (n), 64 (r)}
+      if (!encode_map_bf16(&pr.tmB, s.Nbuf, s.n, s.r, s.ldN, 64, 64)) return cudaErrorInvalidValue;
+      pr.status = s.status;
+      pr.epi = StochRoundEpi::Args{s.W, s.sW, s.ldw, s.alpha, s.t, s.layer_id,
+                                   PhiloxKey{static_cast<uint32_t>(s.seed), static_cast<uint32_t>(s.seed >> 32)},
+                                   (s.n % 4) == 0 ? 1 : 0};
+      add_problem(p2, s.m, s.n, s.r);
+    }
+    e = launch_gemm<StochRoundEpi, false, true>(p2, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_gemm_f32(const void* A, int64_t lda, bool a_trans, const void* B, int64_t ldb, bool b_trans,
+                            float* D, int64_t ldd, int M, int N, int K, cudaStream_t stream) {
+  GemmParams<StoreF32Epi> p;
+  memset(&p, 0, sizeof(p));
+  GemmProblem<StoreF32Epi>& pr = p.prob[0];
+  // A: a_trans = 0 -> given M x K row-major (K-major operand, box {64, 128});
+  //    a_trans = 1 -> given K x M row-major (MN-major operand, box {64, 64}).
+  const bool okA = a_trans ? encode_map_bf16(&pr.tmA, A, M, K, lda, 64, 64)
+                           : encode_map_bf16(&pr.tmA, A, K, M, lda, 64, 128);
+  // B: b_trans = 0 -> given K x N row-major (MN-major, box {64, 64});
+  //    b_trans = 1 -> given N x K row-major (K-major, box {64, 256}).
+  const bool okB = b_trans ? encode_map_bf16(&pr.tmB, B, K, N, ldb, 64, 256)
+                           : encode_map_bf16(&pr.tmB, B, N, K, ldb, 64, 64);
+  if (!okA || !okB) return cudaErrorInvalidValue;
+  pr.status = nullptr;
+  pr.epi = StoreF32Epi::Args{D, ldd};
+  add_problem(p, M, N, K);
+  if (a_trans && b_trans) return launch_gemm<StoreF32Epi, true, false>(p, stream);
+  if (a_trans) return launch_gemm<StoreF32Epi, true, true>(p, stream);
+  if (b_trans) return launch_gemm<StoreF32Epi, false, false>(p, stream);
+  return launch_gemm<StoreF32Epi, false, true>(p, stream);
+}
+
+}  // namespace qg

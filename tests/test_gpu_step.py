@@ -1,0 +1,199 @@
+"""GPU parity of the optimizer step a1..a5 against the CPU oracle, through the C ABI.
+
+Bars (floating point decides integers here, so both sides take every such
+decision in IEEE float32 with the same operation order):
+  * Philox words, INT4 dequantization: bit-exact.
+  * INT8 weights: every element within one code of the oracle, and at most
+    1e-4 of the elements differ at all.
+  * Moments (dequantized): relative L2 error <= 1e-2.
+  * GEMM core: |D - A B| <= 1e-5 * (|A| |B|) element-wise (float32 accumulation).
+"""
+from ctypes import byref, c_void_p
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import quantized_rank_gradient_b200 as qg
+import synth
+from gpu_layer import GpuLayer, round_up, stream, upload_gradient
+
+pytestmark = pytest.mark.gpu
+
+W_DIFF_FRAC = 1e-4
+MOM_REL_L2 = 1e-2
+
+
+@pytest.fixture(autouse=True)
+def _cuda(cuda_ok):
+    torch.cuda.synchronize()
+    yield
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------- single stages
+
+def test_philox_bit_exact_million_counters():
+    rng = np.random.default_rng(0)
+    cnt = 1 << 20
+    c = rng.integers(0, 2**32, size=(4, cnt), dtype=np.uint64).astype(np.uint32)
+    k0, k1 = 0xDEADBEEF, 0x01234567
+    dc = [torch.from_numpy(c[i].view(np.int32)).cuda() for i in range(4)]
+    out = torch.zeros(4 * cnt, dtype=torch.int32, device="cuda")
+    qg.check(qg.qg_philox4x32_10(*(t.data_ptr() for t in dc), cnt, k0, k1, out.data_ptr(), stream()))
+    got = out.cpu().numpy().view(np.uint32).reshape(cnt, 4)
+    ref = np.stack(O.philox4x32_10(c[0], c[1], c[2], c[3], k0, k1), axis=1)
+    np.testing.assert_array_equal(got, ref)
+
+
+@pytest.mark.parametrize("m,r", [(256, 32), (1376, 128), (300, 64), (4096, 1024)])
+def test_dequant_projection_bit_exact(m, r):
+    P = synth.orthonormal(m, r, seed=m + r).astype(np.float32)
+    codes, sP = O.quant_int4_groups(P)
+    Pq = O.pack_int4(codes)
+    ref = O.bf16_bits(O.dequant_int4_f32(Pq, sP, m, r))
+    dPq = torch.from_numpy(Pq).cuda()
+    dsP = torch.from_numpy(sP).cuda()
+    out = torch.zeros(m * r, dtype=torch.int16, device="cuda")
+    qg.check(qg.qg_dequant_projection(dPq.data_ptr(), dsP.data_ptr(), m, r, out.data_ptr(), stream()))
+    np.testing.assert_array_equal(out.cpu().numpy().view(np.uint16).reshape(m, r), ref)
+
+
+@pytest.mark.parametrize("a_trans", [0, 1])
+@pytest.mark.parametrize("b_trans", [0, 1])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 300, 136), (384, 520, 1000), (64, 40, 16)])
+def test_gemm_core_tcgen05(M, N, K, a_trans, b_trans):
+    g = torch.Generator().manual_seed(M * 7 + N * 3 + K)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    B = torch.randn(K, N, generator=g).to(torch.bfloat16)
+    ref = A.double() @ B.double()
+    bound = A.double().abs() @ B.double().abs()
+    A_src = A.t().contiguous() if a_trans else A
+    B_src = B.t().contiguous() if b_trans else B
+    lda = round_up(A_src.shape[1], 8)
+    ldb = round_up(B_src.shape[1], 8)
+    dA = torch.zeros(A_src.shape[0], lda, dtype=torch.bfloat16, device="cuda")
+    dA[:, : A_src.shape[1]] = A_src.cuda()
+    dB = torch.zeros(B_src.shape[0], ldb, dtype=torch.bfloat16, device="cuda")
+    dB[:, : B_src.shape[1]] = B_src.cuda()
+    ldd = round_up(N, 4)
+    dD = torch.full((M, ldd), float("nan"), dtype=torch.float32, device="cuda")
+    qg.check(qg.qg_gemm_bf16(dA.data_ptr(), lda, a_trans, dB.data_ptr(), ldb, b_trans, dD.data_ptr(), ldd, M, N, K,
+                             stream()))
+    D = dD[:, :N].double().cpu()
+    err = (D - ref).abs()
+    assert torch.all(err <= 1e-5 * bound + 1e-30), float((err / (bound + 1e-30)).max())
+
+
+# ---------------------------------------------------------------- step parity
+
+def make_layer(m, n, r, seed=0, rank=None, s0=1e-2, decay=0.8, sigma=1e-4, layer_id=0):
+    oc = O.Config(m=m, n=n, r=r, seed=seed, layer_id=layer_id)
+    Wq = synth.weight_codes(m, n, seed)
+    sW = synth.weight_scales(m, n, seed=seed)
+    gen = synth.lowrank_gradient(m, n, rank=rank or min(256, m, n), s0=s0, decay=decay, sigma=sigma, seed=seed)
+    ost = O.LayerState.create(oc, Wq, sW)
+    G0, _ = gen.draw(0)
+    P, _ = O.exact_topr(G0, r)
+    O.set_projection(ost, P)
+    gl = GpuLayer(oc, Wq, sW)
+    gl.set_projection(ost.Pq, ost.sP)
+    return ost, gl, gen
+
+
+def compare_state(ost, gl, label=""):
+    Wg = gl.weights()
+    d = np.abs(Wg.astype(np.int32) - ost.Wq.astype(np.int32))
+    assert d.max() <= 1, f"{label}: W differs by {d.max()} codes"
+    frac = float((d > 0).mean())
+    assert frac <= W_DIFF_FRAC, f"{label}: {frac:.2e} of W differ"
+    Mq, sM, Vq, sV = gl.moments()
+    for (q, s, oq, os_) in [(Mq, sM, ost.Mq, ost.sM), (Vq, sV, ost.Vq, ost.sV)]:
+        a = O.dequant_rowblock(q, s)
+        b = O.dequant_rowblock(oq, os_)
+        rel = np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30)
+        assert rel <= MOM_REL_L2, f"{label}: moment rel L2 {rel:.2e}"
+    return frac
+
+
+@pytest.mark.parametrize("m,n,r,steps", [
+    (256, 256, 32, 10),      # single-layer parity case
+    (512, 512, 128, 4),      # LLaMA-60M shapes
+    (512, 1376, 128, 4),
+    (1376, 512, 128, 4),
+    (300, 700, 64, 3),       # ragged M, N and K tails everywhere
+    (640, 1365, 96, 3),      # n % 4 != 0: Philox quads straddle rows
+])
+def test_step_parity_with_oracle(m, n, r, steps):
+    ost, gl, gen = make_layer(m, n, r, seed=m + n + r, layer_id=3)
+    for t in range(steps):
+        G, Gb = gen.draw(t)
+        dG, ldg = upload_gradient(Gb)
+        gl.step(dG, ldg)
+        inter = O.step(ost, G)
+        if t == 0:
+            Nb = gl.scratch_N()
+            refN = O.bf16_bits(inter["N"])
+            assert float((Nb != refN).mean()) <= 1e-3
+        compare_state(ost, gl, f"step {t + 1}")
+    assert gl.status() == qg.QG_OK
+    assert gl.sched().t == steps
+
+
+def test_step_is_deterministic():
+    outs = []
+    for _ in range(2):
+        ost, gl, gen = make_layer(512, 1376, 128, seed=5)
+        for t in range(3):
+            dG, ldg = upload_gradient(gen.draw(t)[1])
+            gl.step(dG, ldg)
+        outs.append((gl.weights(), gl.moments()))
+    np.testing.assert_array_equal(outs[0][0], outs[1][0])
+    for a, b in zip(outs[0][1], outs[1][1]):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_step_batch_equals_single_steps():
+    shapes = [(512, 512, 128), (512, 1376, 128), (1376, 512, 128), (256, 256, 32)]
+    singles, batched, grads = [], [], []
+    for i, (m, n, r) in enumerate(shapes):
+        _, gl1, gen = make_layer(m, n, r, seed=10 + i, layer_id=i)
+        _, gl2, _ = make_layer(m, n, r, seed=10 + i, layer_id=i)
+        singles.append(gl1)
+        batched.append(gl2)
+        grads.append(upload_gradient(gen.draw(0)[1]))
+    for gl, (dG, ldg) in zip(singles, grads):
+        gl.step(dG, ldg)
+    cfgs = [gl.cfg for gl in batched]
+    arr = (qg.POINTER(qg.qg_config) * len(cfgs))(*[qg.ctypes.pointer(c) for c in cfgs])
+    wsb = qg.qg_step_batch_workspace_bytes(arr, len(cfgs))
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    hs = (c_void_p * len(batched))(*[gl.h.value for gl in batched])
+    gs = (c_void_p * len(batched))(*[g.data_ptr() for g, _ in grads])
+    lds = (qg.c_int64 * len(batched))(*[ld for _, ld in grads])
+    qg.check(qg.qg_step_batch(hs, gs, lds, len(batched), ws.data_ptr(), wsb, stream()))
+    for a, b in zip(singles, batched):
+        np.testing.assert_array_equal(a.weights(), b.weights())
+        for x, y in zip(a.moments(), b.moments()):
+            np.testing.assert_array_equal(x, y)
+
+
+def test_step_without_projection_is_rejected():
+    oc = O.Config(m=256, n=256, r=32)
+    gl = GpuLayer(oc, synth.weight_codes(256, 256), synth.weight_scales(256, 256))
+    dG, ldg = upload_gradient(np.zeros((256, 256), np.uint16))
+    st = qg.qg_step(gl.h, dG.data_ptr(), ldg, gl.ws.data_ptr(), gl.ws.numel(), stream())
+    assert st == qg.QG_ESTATE
+    assert gl.sched().t == 0
+
+
+def test_nonfinite_gradient_sets_status():
+    ost, gl, gen = make_layer(256, 256, 32, seed=1)
+    G, Gb = gen.draw(0)
+    Gb = Gb.copy()
+    Gb[3, 5] = 0x7FC0  # bf16 NaN
+    dG, ldg = upload_gradient(Gb)
+    gl.step(dG, ldg)
+    assert gl.status() == qg.QG_ENONFINITE
+    assert gl.status() == qg.QG_OK  # cleared by the read
