@@ -280,19 +280,29 @@ def adam_moments(R, m0, v0, cfg: Config, t: int):
     return (num / den).astype(np.float32), m, v
 
 
+def dequant_second_moment(Vq, sV, block=256) -> np.ndarray:
+    """v = (code * scale)^2 in float32: V^Q holds the INT8 grid of sqrt(v)."""
+    d = dequant_rowblock(Vq, sV, block)
+    return (d * d).astype(np.float32)
+
+
 def lowrank_adam_int8(R, Mq, sM, Vq, sV, cfg: Config, t: int):
     """Step a3: Adam on the INT8 moments.  [QG-quant]: (M^Q, V^Q) are kept in
     INT8.  Readings: per-row blocks of `mom_block` columns, re-quantized with a
-    fresh absmax scale every step; N is formed from the float32 moments before
-    they are re-quantized, then rounded to bf16 (the operand of step a4).
+    fresh absmax scale every step; the first moment m on a linear grid; the
+    second moment through its square root (codes 0..127 of sqrt(v), so that
+    v = (code * scale)^2) -- a linear grid on v itself sends the small second
+    moments of a block to zero and lets m / sqrt(v) explode; N is formed from
+    the float32 moments before they are re-quantized, then rounded to bf16 (the
+    operand of step a4).
 
     Returns (N as bf16 values in float32, Mq', sM', Vq', sV')."""
     m0 = dequant_rowblock(Mq, sM, cfg.mom_block)
-    v0 = dequant_rowblock(Vq, sV, cfg.mom_block)
+    v0 = dequant_second_moment(Vq, sV, cfg.mom_block)
     upd, m, v = adam_moments(R, m0, v0, cfg, t)
     N = bf16_round(upd)
     Mq2, sM2 = quant_rowblock_int8(m, cfg.mom_block, unsigned=False)
-    Vq2, sV2 = quant_rowblock_int8(v, cfg.mom_block, unsigned=True)
+    Vq2, sV2 = quant_rowblock_int8(np.sqrt(v).astype(np.float32), cfg.mom_block, unsigned=True)
     return N, Mq2, sM2, Vq2, sV2
 
 

@@ -203,6 +203,34 @@ def test_adam_first_step_closed_form():
     assert np.all((Mq == 0) | (np.sign(Mq) == np.sign(R)))
 
 
+def test_int8_moments_keep_adam_step_bound():
+    # Adam's normalised step obeys |m_hat / sqrt(v_hat)| <= (1 - b1) / sqrt(1 - b2)
+    # (Kingma and Ba, section 2.1); the INT8 moment grids must not break it.
+    import synth
+    cfg = O.Config(m=512, n=512, r=128, seed=4)
+    st = O.LayerState.create(cfg, synth.weight_codes(512, 512, 4), synth.weight_scales(512, 512, seed=4))
+    gen = synth.lowrank_gradient(512, 512, rank=256, seed=4)
+    O.set_projection(st, O.exact_topr(gen.draw(0)[0], 128)[0])
+    bound = np.float32(cfg.lr) * (1 - np.float32(cfg.beta1)) / math.sqrt(1 - np.float32(cfg.beta2))
+    for t in range(6):
+        inter = O.step(st, gen.draw(t)[0])
+        assert np.abs(inter["N"]).max() <= bound * 1.01
+
+
+def test_second_moment_grid_is_sqrt_of_v():
+    rng = np.random.default_rng(21)
+    R = (rng.standard_normal((3, 300)) * np.exp2(rng.integers(-12, 0, (3, 300)))).astype(np.float32)
+    cfg = O.Config(m=8, n=300, r=3)
+    z8 = np.zeros((3, 300), np.int8)
+    z = np.zeros((3, 2), np.float32)
+    _, _, _, Vq, sV = O.lowrank_adam_int8(R, z8, z, z8, z, cfg, 1)
+    v = (np.float32(1 - np.float32(cfg.beta2)) * (R * R)).astype(np.float32)
+    root = np.sqrt(v)
+    cols = np.arange(300) // 256
+    assert np.all(np.abs(O.dequant_rowblock(Vq, sV) - root) <= sV[:, cols] / 2 * (1 + 1e-6))
+    np.testing.assert_allclose(O.dequant_second_moment(Vq, sV), O.dequant_rowblock(Vq, sV) ** 2, rtol=1e-6)
+
+
 # ---------------------------------------------------------------- projections
 
 def test_project_and_backproject_brute_force():
