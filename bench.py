@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Throughput of the Q-GaLore optimizer step on B200: INT8 weights updated per second.
+
+Workload: a LLaMA-7B-shaped stack, 32 decoder layers x {q, k, v, o: 4096 x 4096;
+gate, up: 4096 x 11008; down: 11008 x 4096}, rank r = 1024: 224 weight matrices,
+6.48 G INT8 weights.  One step = the optimizer step a1..a5 on every matrix
+(dequantize INT4 P, R = P^T G, Adam on the INT8 moments, U = P N, stochastic
+rounding into INT8 W), issued as one batched call per decoder layer.  Inputs are
+seeded synthetic bf16 gradients (rank-256 signal, s_i = 1e-2 * 0.97^i, noise
+sigma = 1e-4) resident in HBM (13 GB, far larger than L2).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank updates its own full stack (weak scaling, no
+collective on the data path); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+from ctypes import byref, c_int64, c_void_p
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Q-GaLore step: INT8 weights updated/s at 7B shapes; % of step roofline"
+UNIT = "weights/s"
+WORKLOAD = "llama7b-stack-r1024"
+R_RANK = 1024
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=32, help="decoder layers (32 = the 7B stack)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def stack_shapes(layers):
+    per = [(4096, 4096)] * 4 + [(4096, 11008)] * 2 + [(11008, 4096)]
+    return [per for _ in range(layers)]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id):
+        self.bus_id = bus_id
+        self.proc = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.bus_id:
+            cmd += ["-i", self.bus_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def bus_id_of(dev):
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+
+def oracle_sample_seconds(cols, seed=1):
+    """One oracle step on a 4096 x `cols` column slice of a 4096 x 4096 (r = 1024)
+    matrix.  Columns are independent in every stage of the step, so the weights
+    per second of a slice equal those of the full matrix."""
+    import numpy as np
+
+    import oracle as O
+    import synth
+    m, r = 4096, R_RANK
+    oc = O.Config(m=m, n=cols, r=r, seed=seed)
+    st = O.LayerState.create(oc, synth.weight_codes(m, cols, seed), synth.weight_scales(m, cols, seed=seed))
+    O.set_projection(st, synth.orthonormal(m, r, seed))
+    G = O.bf16_round((np.random.default_rng(seed).standard_normal((m, cols)) * 1e-4).astype(np.float32))
+    t0 = time.perf_counter()
+    O.step(st, G)
+    return time.perf_counter() - t0
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cols=2048):
+    t = oracle_sample_seconds(cols)
+    return {"value": 4096 * cols / t, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"one oracle step on a 4096x{cols} column slice of a 4096x4096 r=1024 matrix "
+                      f"({t:.1f} s); columns are independent, so weights/s carry over",
+            "host_cpus": os.cpu_count()}
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    cols = 512
+    for _ in range(args.warmup):
+        oracle_sample_seconds(cols)
+    ts = [oracle_sample_seconds(cols, seed=3 + k) for k in range(args.steps)]
+    ms = 1000.0 * sum(ts) / len(ts)
+    value = 4096 * cols / (ms / 1000.0)
+    cores = oracle_threads()
+    sample = f"each step: one oracle step on a 4096x{cols} column slice of a 4096x4096 r=1024 matrix"
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64/f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": sample}, "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+
+class Stack:
+    """The 7B stack on one GPU: per matrix W, W scales, state, gradient."""
+
+    def __init__(self, layers, rank, device):
+        import torch
+
+        import quantized_rank_gradient_b200 as qg
+        import synth
+        self.qg = qg
+        self.device = device
+        self.layers = []
+        self.keep = []
+        stream = c_void_p(torch.cuda.current_stream().cuda_stream)
+        lid = 0
+        for li, shapes in enumerate(stack_shapes(layers)):
+            group = []
+            for (m, n) in shapes:
+                seed = 1_000_003 * (rank + 1) + lid
+                c = qg.config(m, n, R_RANK, seed=seed, layer_id=lid)
+                ldw = -(-n // 16) * 16
+                W = synth.device_weight_codes(m, n, ldw, seed, device)
+                sW = synth.device_weight_scales(m, n, seed, device)
+                G = synth.device_lowrank_gradient(m, n, 256, 1e-2, 0.97, 1e-4, seed, device)
+                state = torch.empty(qg.qg_state_bytes(byref(c)), dtype=torch.uint8, device=device)
+                h = c_void_p()
+                qg.check(qg.qg_layer_init(byref(h), byref(c), state.data_ptr(), state.numel(), W.data_ptr(), ldw,
+                                          sW.data_ptr(), stream), "qg_layer_init")
+                # starting projection: an orthonormal basis quantized to INT4 on the device
+                g = torch.Generator(device=device)
+                g.manual_seed(seed + 17)
+                P = torch.linalg.qr(torch.randn(m, R_RANK, generator=g, device=device))[0].contiguous()
+                Pq = torch.empty((m * R_RANK + 1) // 2, dtype=torch.uint8, device=device)
+                sP = torch.empty(-(-m * R_RANK // 64), dtype=torch.float32, device=device)
+                qg.check(qg.qg_quantize_projection(P.data_ptr(), R_RANK, m, R_RANK, Pq.data_ptr(), sP.data_ptr(),
+                                                   stream))
+                qg.check(qg.qg_layer_set_projection(h, Pq.data_ptr(), sP.data_ptr(), 0, stream))
+                torch.cuda.synchronize()
+                del P, Pq, sP
+                group.append(dict(cfg=c, h=h, W=W, sW=sW, G=G, ldg=G.shape[1], state=state, m=m, n=n))
+                lid += 1
+            self.layers.append(group)
+        # one workspace, reused by every decoder layer (they run in order on one stream)
+        need = 0
+        for group in self.layers:
+            arr = (qg.POINTER(qg.qg_config) * len(group))(*[qg.ctypes.pointer(e["cfg"]) for e in group])
+            need = max(need, qg.qg_step_batch_workspace_bytes(arr, len(group)))
+        self.ws = torch.empty(need, dtype=torch.uint8, device=device)
+        self.calls = []
+        for group in self.layers:
+            k = len(group)
+            self.calls.append(((c_void_p * k)(*[e["h"].value for e in group]),
+                               (c_void_p * k)(*[e["G"].data_ptr() for e in group]),
+                               (c_int64 * k)(*[e["ldg"] for e in group]), k))
+        self.weights = sum(e["m"] * e["n"] for group in self.layers for e in group)
+        self.flops = sum(4.0 * e["m"] * e["n"] * R_RANK for group in self.layers for e in group)
+        self.alg_bytes = sum(alg_bytes(e["m"], e["n"], R_RANK) for group in self.layers for e in group)
+
+    def step(self, stream):
+        qg = self.qg
+        for hs, gs, lds, k in self.calls:
+            st = qg.qg_step_batch(hs, gs, lds, k, self.ws.data_ptr(), self.ws.numel(), stream)
+            if st != qg.QG_OK:
+                raise qg.QGError(st, "qg_step_batch")
+
+    def statuses(self):
+        return [e["state"] for group in self.layers for e in group]
+
+
+def alg_bytes(m, n, r):
+    """Algorithmic HBM bytes of one matrix step: G, W read and written, W scales,
+    INT4 P and scales, moments read and written, their scales."""
+    nb = -(-n // 256)
+    return 2 * m * n + 2 * m * n + 4 * math.ceil(m * n / 256) + m * r / 2 + 4 * m * r / 64 + 4 * r * n + 16 * r * nb
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import quantized_rank_gradient_b200 as qg
+    qg.lib()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stack = Stack(args.layers, rank, device)
+    stream = c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        stack.step(stream)
+    torch.cuda.synchronize()
+
+    # ---- device-timed region: inputs resident in HBM
+    clocks = ClockSampler(bus_id_of(device))
+    clocks.start()
+    time.sleep(0.3)
+    qg.check(qg.qg_profile_enable(1))
+    barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for _ in range(args.steps):
+        stack.step(stream)
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    kt = (qg.qg_kernel_times * qg.QG_KERNEL_KINDS)()
+    qg.check(qg.qg_profile_collect(kt, qg.QG_KERNEL_KINDS))
+    qg.check(qg.qg_profile_enable(0))
+    clk = clocks.stop()
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---- end to end: gradients copied from pinned host memory every step,
+    # the per-matrix status words read back
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(stack, args, stream, world, device, barrier)
+
+    if rank != 0:
+        return 0
+    peaks = load_peaks()
+    value = world * stack.weights / (ms / 1000.0)
+    names = {qg.QG_KERNEL_DEQUANT: "dequant_projection", qg.QG_KERNEL_PROJECT_ADAM: "project_adam_tcgen05",
+             qg.QG_KERNEL_BACKPROJECT_SR: "backproject_sround_tcgen05"}
+    kernels = {}
+    for k, nm in names.items():
+        e = kt[k]
+        if e.launches:
+            kernels[nm] = {"launches_per_step": e.launches / args.steps, "ms_per_step": e.device_ms / args.steps,
+                           "avg_launch_ms": e.device_ms / e.launches,
+                           "tflops": e.flops / (e.device_ms / 1000.0) / 1e12 if e.flops else None,
+                           "gbs": e.bytes / (e.device_ms / 1000.0) / 1e9}
+    dom_k = max([qg.QG_KERNEL_PROJECT_ADAM, qg.QG_KERNEL_BACKPROJECT_SR], key=lambda k: kt[k].device_ms)
+    dom = kt[dom_k]
+    achieved = (dom.flops / dom.launches) / (dom.device_ms / dom.launches / 1000.0) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    launches = sum(kt[k].launches for k in range(qg.QG_KERNEL_KINDS)) / args.steps
+    t_roof_ms = max(stack.flops / (peaks["bf16_tflops"] * 1e12), stack.alg_bytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/f32/int8",
+        "data": "synthetic (seeded low-rank-plus-noise bf16 gradients)",
+        "config": {"workload": WORKLOAD, "matrices": 7 * args.layers, "weights_per_gpu": stack.weights,
+                   "rank": R_RANK, "l2": "inputs larger than L2 (13 GB of gradients per step)",
+                   "parallelism": f"independent stacks x{world}"},
+        "step_roofline": {"t_roof_ms": t_roof_ms, "frac": t_roof_ms / ms,
+                          "bound": "tensor" if stack.flops / (peaks["bf16_tflops"] * 1e12) >
+                          stack.alg_bytes / (peaks["hbm_gbs"] * 1e9) else "hbm",
+                          "peaks": "burst bf16 %.1f TF/s, HBM %.1f GB/s (%s)" % (peaks["bf16_tflops"], peaks["hbm_gbs"],
+                                                                              peaks["source"])},
+        "roofline": {"bound": "tensor", "kernel": names[dom_k], "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_kind": "sustained bf16 (%s)" % peaks["source"]},
+        "kernels": kernels,
+        "gpu_launches": launches * args.steps,
+        "clocks": clk,
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_e2e(stack, args, stream, world, device, barrier):
+    import torch
+    import torch.distributed as dist
+    qg = stack.qg
+    # one pinned host gradient per distinct shape; every matrix's gradient is
+    # copied from host memory each step
+    host = {}
+    for group in stack.layers:
+        for e in group:
+            key = tuple(e["G"].shape)
+            if key not in host:
+                host[key] = e["G"].cpu().pin_memory()
+    status_host = torch.zeros(sum(len(g) for g in stack.layers), dtype=torch.int32).pin_memory()
+    views = []
+    for group in stack.layers:
+        for e in group:
+            v = qg.qg_layer_views()
+            qg.check(qg.qg_layer_views_get(e["h"], byref(v)))
+            off = v.status - e["state"].data_ptr()
+            views.append(e["state"][off: off + 4].view(torch.int32))
+    h2d = sum(e["G"].numel() * 2 for group in stack.layers for e in group)
+    d2h = 4 * len(views)
+
+    def one():
+        i = 0
+        for (hs, gs, lds, k), group in zip(stack.calls, stack.layers):
+            for e in group:
+                e["G"].copy_(host[tuple(e["G"].shape)], non_blocking=True)
+            st = qg.qg_step_batch(hs, gs, lds, k, stack.ws.data_ptr(), stack.ws.numel(), stream)
+            if st != qg.QG_OK:
+                raise qg.QGError(st, "qg_step_batch")
+        for j, v in enumerate(views):
+            status_host[j: j + 1].copy_(v, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        if int(status_host.max()) != 0:
+            raise RuntimeError("device status word set during the e2e run")
+
+    one()
+    steps = max(2, min(args.steps, 5))
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        one()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = t0.elapsed_time(t1) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": world * stack.weights / (ms / 1000.0), "unit": UNIT, "ms_per_step": ms, "steps": steps,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "note": "bf16 gradients copied from pinned host memory each step; status words read back"}
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

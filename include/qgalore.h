@@ -82,7 +82,7 @@ typedef struct {
   uint8_t* Pq_prev;         /* previous projection (for CosSim) */
   float* sP_prev;
   int8_t* Mq;               /* r x ld_mom INT8 first moment (columns >= n unused) */
-  int8_t* Vq;               /* r x ld_mom INT8 second moment, codes 0..127 */
+  int8_t* Vq;               /* r x ld_mom INT8 codes 0..127 of sqrt(v), v the second moment */
   float* sM;                /* r x nblk float32 */
   float* sV;                /* r x nblk float32 */
   int64_t ld_mom;           /* row stride of Mq, Vq in bytes: n rounded up to 32 */
@@ -176,6 +176,37 @@ qg_status qg_layer_status(qg_layer* layer, void* stream);
  * step t, delta doubles iff has_cossim and cossim > gamma; t_next = t + delta. */
 qg_status qg_sched_after_refresh(int64_t t, int32_t delta, int32_t has_cossim, float cossim,
                                  float gamma, int32_t* delta_out, int64_t* t_next_out);
+
+/* INT4 quantization of a float32 projection (refresh stage): m x r matrix with
+ * row stride ld (elements) -> ceil(m*r/2) packed bytes (two's-complement
+ * nibbles, even index in the low nibble) and ceil(m*r/64) scales; groups of 64
+ * consecutive elements of the row-major m x r array, scale = absmax / 7,
+ * code = clamp(rint(x / scale), -7, 7), a zero group gets scale 0. */
+qg_status qg_quantize_projection(const float* d_P, int64_t ld, int32_t m, int32_t r, uint8_t* d_Pq,
+                                 float* d_sP, void* stream);
+
+/* ---- Device-time accounting of this library's own launches ----
+ * While enabled, every kernel the library launches is bracketed by CUDA events
+ * recorded on the launch stream.  qg_profile_collect synchronises those events
+ * and returns, per kernel kind, the launch count, the summed device time, and
+ * the algorithmic FLOPs and bytes of those launches. */
+typedef enum {
+  QG_KERNEL_DEQUANT = 0,      /* a1: INT4 P -> bf16 */
+  QG_KERNEL_PROJECT_ADAM = 1, /* a2 + a3: tcgen05 P^T G with the moment epilogue */
+  QG_KERNEL_BACKPROJECT_SR = 2, /* a4 + a5: tcgen05 P N with stochastic rounding */
+  QG_KERNEL_OTHER = 3,        /* refresh and single-stage kernels */
+  QG_KERNEL_KINDS = 4
+} qg_kernel_kind;
+
+typedef struct {
+  int64_t launches;
+  double device_ms;   /* sum over launches */
+  double flops;       /* algorithmic: 2*m*n*r per GEMM problem */
+  double bytes;       /* algorithmic HBM bytes (see the design notes) */
+} qg_kernel_times;
+
+qg_status qg_profile_enable(int32_t on);  /* on != 0 starts a new window */
+qg_status qg_profile_collect(qg_kernel_times* out, int32_t kinds);
 
 /* ---- Single-stage entry points (used by the tests to check each stage) ---- */
 

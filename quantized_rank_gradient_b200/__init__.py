@@ -10,8 +10,8 @@ from __future__ import annotations
 
 import ctypes
 import os
-from ctypes import (POINTER, Structure, byref, c_char_p, c_float, c_int32, c_int64, c_size_t, c_uint32,
-                    c_uint64, c_void_p)
+from ctypes import (POINTER, Structure, byref, c_char_p, c_double, c_float, c_int32, c_int64, c_size_t,
+                    c_uint32, c_uint64, c_void_p)
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libqgalore.so")
@@ -48,6 +48,12 @@ class qg_refresh_info(Structure):
                 ("t_next", c_int64), ("n_refresh", c_int32)]
 
 
+class qg_kernel_times(Structure):
+    _fields_ = [("launches", c_int64), ("device_ms", c_double), ("flops", c_double), ("bytes", c_double)]
+
+
+QG_KERNEL_DEQUANT, QG_KERNEL_PROJECT_ADAM, QG_KERNEL_BACKPROJECT_SR, QG_KERNEL_OTHER, QG_KERNEL_KINDS = range(5)
+
 _SIGNATURES = {
     "qg_status_str": (c_char_p, [c_int32]),
     "qg_config_default": (None, [POINTER(qg_config), c_int32, c_int32, c_int32]),
@@ -72,6 +78,9 @@ _SIGNATURES = {
     "qg_layer_status": (c_int32, [c_void_p, c_void_p]),
     "qg_sched_after_refresh": (c_int32, [c_int64, c_int32, c_int32, c_float, c_float, POINTER(c_int32),
                                          POINTER(c_int64)]),
+    "qg_quantize_projection": (c_int32, [c_void_p, c_int64, c_int32, c_int32, c_void_p, c_void_p, c_void_p]),
+    "qg_profile_enable": (c_int32, [c_int32]),
+    "qg_profile_collect": (c_int32, [POINTER(qg_kernel_times), c_int32]),
     "qg_philox4x32_10": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_uint32, c_uint32, c_void_p,
                                    c_void_p]),
     "qg_dequant_projection": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p]),

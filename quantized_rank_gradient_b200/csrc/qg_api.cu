@@ -430,6 +430,14 @@ qg_status qg_dequant_projection(const uint8_t* d_Pq, const float* d_sP, int32_t 
                                                    static_cast<uint16_t*>(d_out), static_cast<cudaStream_t>(stream)));
 }
 
+qg_status qg_quantize_projection(const float* d_P, int64_t ld, int32_t m, int32_t r, uint8_t* d_Pq, float* d_sP,
+                                 void* stream) {
+  if (!d_P || !d_Pq || !d_sP) return QG_EINVAL;
+  if (m <= 0 || r <= 0 || ld < r) return QG_ESHAPE;
+  if (!aligned(d_P, 4) || !aligned(d_sP, 4)) return QG_EALIGN;
+  return cuda_status(qg::launch_quantize_projection(d_P, ld, m, r, d_Pq, d_sP, static_cast<cudaStream_t>(stream)));
+}
+
 qg_status qg_gemm_bf16(const void* d_A, int64_t lda, int32_t a_trans, const void* d_B, int64_t ldb,
                        int32_t b_trans, float* d_D, int64_t ldd, int32_t M, int32_t N, int32_t K, void* stream) {
   if (!d_A || !d_B || !d_D) return QG_EINVAL;

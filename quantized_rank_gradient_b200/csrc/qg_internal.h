@@ -56,4 +56,12 @@ bool encode_map_bf16(void* map, const void* base, uint64_t inner, uint64_t outer
 
 int sm_count();
 
+// Launch accounting (qg_profile.cu): returns a token for profile_end, or -1
+// when accounting is off.  `kind` is a qg_kernel_kind.
+int profile_begin(cudaStream_t s, int kind, double flops, double bytes);
+void profile_end(cudaStream_t s, int token);
+
+cudaError_t launch_quantize_projection(const float* P, int64_t ld, int32_t m, int32_t r, uint8_t* Pq, float* sP,
+                                       cudaStream_t stream);
+
 }  // namespace qg

@@ -17,6 +17,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 
@@ -24,6 +25,7 @@
 #include "qg_internal.h"
 #include "qg_philox.cuh"
 #include "qg_refresh.h"
+#include "../../include/qgalore.h"
 
 namespace qg {
 
@@ -56,10 +58,12 @@ struct AdamEpi {
   };
 
   // m = b1*m0 + (1-b1)*R ; v = b2*v0 + (1-b2)*(R*R), one rounding per operation.
+  // M^Q holds m on a linear grid; V^Q holds sqrt(v), so v0 = (code*scale)^2.
   static QG_DEV void moments(float R, int8_t mc, int8_t vc, float sm, float sv, const Args& a,
                              float& mm, float& vv) {
     const float m0 = __fmul_rn(static_cast<float>(mc), sm);
-    const float v0 = __fmul_rn(static_cast<float>(vc), sv);
+    const float d0 = __fmul_rn(static_cast<float>(vc), sv);
+    const float v0 = __fmul_rn(d0, d0);
     mm = __fadd_rn(__fmul_rn(a.beta1, m0), __fmul_rn(a.om1, R));
     vv = __fadd_rn(__fmul_rn(a.beta2, v0), __fmul_rn(a.om2, __fmul_rn(R, R)));
   }
@@ -108,7 +112,7 @@ struct AdamEpi {
         moments(R, mc, vc, sm, sv, a, mm, vv);
         if (e < valid) {
           amax_m = fmaxf(amax_m, fabsf(mm));
-          amax_v = fmaxf(amax_v, vv);
+          amax_v = fmaxf(amax_v, __fsqrt_rn(vv));
           bad |= !isfinite(R);
         }
         const float mhat = __fdiv_rn(mm, a.bc1);
@@ -126,7 +130,8 @@ struct AdamEpi {
         dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
     }
 
-    // new block scales: absmax / 127 (IEEE division); zero block -> scale 0
+    // new block scales: absmax(|m|) / 127 and absmax(sqrt(v)) / 127 (IEEE
+    // division); a zero block gets scale 0
     const float s_m = __fdiv_rn(amax_m, 127.0f);
     const float s_v = __fdiv_rn(amax_v, 127.0f);
 
@@ -150,7 +155,7 @@ struct AdamEpi {
         moments(R, mc, vc, sm, sv, a, mm, vv);
         int qm = 0, qv = 0;
         if (s_m > 0.f) qm = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(mm, s_m)), -127.f), 127.f));
-        if (s_v > 0.f) qv = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(vv, s_v)), 0.f), 127.f));
+        if (s_v > 0.f) qv = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(__fsqrt_rn(vv), s_v)), 0.f), 127.f));
         const uint32_t bm = static_cast<uint32_t>(qm) & 0xFFu;
         const uint32_t bv = static_cast<uint32_t>(qv) & 0xFFu;
         if ((e & 3) == 0) {
@@ -406,7 +411,8 @@ size_t step_scratch_bytes(int32_t m, int32_t n, int32_t r) {
 }
 
 template <class Epi, bool kAMN, bool kBMN>
-static cudaError_t launch_gemm(const GemmParams<Epi>& p, cudaStream_t stream) {
+static cudaError_t launch_gemm(const GemmParams<Epi>& p, cudaStream_t stream, int kind, double flops,
+                               double bytes) {
   auto kern = gemm_tc_kernel<Epi, kAMN, kBMN>;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
@@ -417,7 +423,9 @@ static cudaError_t launch_gemm(const GemmParams<Epi>& p, cudaStream_t stream) {
   }
   if (p.total_tiles == 0) return cudaSuccess;
   const int grid = std::min(p.total_tiles, sm_count());
+  const int tok = profile_begin(stream, kind, flops, bytes);
   kern<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(p);
+  profile_end(stream, tok);
   return cudaGetLastError();
 }
 
@@ -440,7 +448,10 @@ cudaError_t launch_dequant_projection(const uint8_t* Pq, const float* sP, int64_
   if (chunks == 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (chunks + threads - 1) / threads;
+  const double bytes = total / 2.0 + (total + 63) / 64 * 4.0 + total * 2.0;
+  const int tok = profile_begin(stream, QG_KERNEL_DEQUANT, 0.0, bytes);
   dequant_projection_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(Pq, sP, total, out);
+  profile_end(stream, tok);
   return cudaGetLastError();
 }
 
@@ -464,8 +475,16 @@ cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream
     const int cnt = std::min(kMaxProblems, count - base);
     GemmParams<AdamEpi> p1;
     memset(&p1, 0, sizeof(p1));
+    double fl1 = 0, by1 = 0, fl2 = 0, by2 = 0;
     for (int i = 0; i < cnt; ++i) {
       const StepProblem& s = probs[base + i];
+      const double m = s.m, n = s.n, r = s.r;
+      fl1 += 2 * m * n * r;
+      fl2 += 2 * m * n * r;
+      // a2+a3: G, P~, moments read + written, their scales, N written
+      by1 += 2 * m * n + 2 * m * r + 4 * r * n + 16.0 * r * s.nblk + 2 * r * n;
+      // a4+a5: W read + written, W scales, P~, N
+      by2 += 2 * m * n + 4 * std::ceil(m * n / 256.0) + 2 * m * r + 2 * r * n;
       GemmProblem<AdamEpi>& pr = p1.prob[p1.nprob];
       // A = P~^T (M = r, K = m), MN-major over P~ (m x r): box {64 (r), 64 (m)}
       if (!encode_map_bf16(&pr.tmA, s.Pbf, s.r, s.m, s.r, 64, 64)) return cudaErrorInvalidValue;
@@ -476,7 +495,7 @@ cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream
                              s.beta1, s.beta2, s.om1, s.om2, s.bc1, s.bc2, s.neg_lr, s.eps};
       add_problem(p1, s.r, s.n, s.m);
     }
-    e = launch_gemm<AdamEpi, true, true>(p1, stream);
+    e = launch_gemm<AdamEpi, true, true>(p1, stream, QG_KERNEL_PROJECT_ADAM, fl1, by1);
     if (e != cudaSuccess) return e;
 
     GemmParams<StochRoundEpi> p2;
@@ -494,7 +513,7 @@ cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream
                                    (s.n % 4) == 0 ? 1 : 0};
       add_problem(p2, s.m, s.n, s.r);
     }
-    e = launch_gemm<StochRoundEpi, false, true>(p2, stream);
+    e = launch_gemm<StochRoundEpi, false, true>(p2, stream, QG_KERNEL_BACKPROJECT_SR, fl2, by2);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -517,10 +536,11 @@ cudaError_t launch_gemm_f32(const void* A, int64_t lda, bool a_trans, const void
   pr.status = nullptr;
   pr.epi = StoreF32Epi::Args{D, ldd};
   add_problem(p, M, N, K);
-  if (a_trans && b_trans) return launch_gemm<StoreF32Epi, true, false>(p, stream);
-  if (a_trans) return launch_gemm<StoreF32Epi, true, true>(p, stream);
-  if (b_trans) return launch_gemm<StoreF32Epi, false, false>(p, stream);
-  return launch_gemm<StoreF32Epi, false, true>(p, stream);
+  const double fl = 2.0 * M * N * K, by = 2.0 * M * K + 2.0 * K * N + 4.0 * M * N;
+  if (a_trans && b_trans) return launch_gemm<StoreF32Epi, true, false>(p, stream, QG_KERNEL_OTHER, fl, by);
+  if (a_trans) return launch_gemm<StoreF32Epi, true, true>(p, stream, QG_KERNEL_OTHER, fl, by);
+  if (b_trans) return launch_gemm<StoreF32Epi, false, false>(p, stream, QG_KERNEL_OTHER, fl, by);
+  return launch_gemm<StoreF32Epi, false, true>(p, stream, QG_KERNEL_OTHER, fl, by);
 }
 
 }  // namespace qg

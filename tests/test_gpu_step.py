@@ -109,9 +109,9 @@ def compare_state(ost, gl, label=""):
     frac = float((d > 0).mean())
     assert frac <= W_DIFF_FRAC, f"{label}: {frac:.2e} of W differ"
     Mq, sM, Vq, sV = gl.moments()
-    for (q, s, oq, os_) in [(Mq, sM, ost.Mq, ost.sM), (Vq, sV, ost.Vq, ost.sV)]:
-        a = O.dequant_rowblock(q, s)
-        b = O.dequant_rowblock(oq, os_)
+    pairs = [(O.dequant_rowblock(Mq, sM), O.dequant_rowblock(ost.Mq, ost.sM)),
+             (O.dequant_second_moment(Vq, sV), O.dequant_second_moment(ost.Vq, ost.sV))]
+    for a, b in pairs:
         rel = np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30)
         assert rel <= MOM_REL_L2, f"{label}: moment rel L2 {rel:.2e}"
     return frac
