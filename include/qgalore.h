@@ -152,6 +152,24 @@ qg_status qg_step_batch(qg_layer* const* layers, const void* const* d_G, const i
                         int32_t count, void* d_ws, size_t ws_bytes, void* stream);
 size_t qg_step_batch_workspace_bytes(const qg_config* const* cfgs, int32_t count);
 
+/* qg_step without a workspace argument, for callers that cannot allocate
+ * device memory (for instance a host program whose device memory belongs to
+ * another allocator with a fixed budget, or a thread that must not take the
+ * implicit synchronisation of cudaMalloc / cudaFree).  The paper has no
+ * counterpart: this is a property of the library only.
+ *   The scratch (P~ and N) lives in a static device array of
+ *   QG_NOALLOC_SCRATCH_BYTES (32 MiB), held by every GPU that loads the library
+ *   until the process exits; every LLaMA-7B-shaped matrix at r = 1024 fits.
+ *   Larger matrices are refused with QG_ESHAPE before anything is launched.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.  All calls share the array and it keeps the
+ *   previous call's contents (the step overwrites everything it reads), so
+ *   calls whose GPU work overlaps, from other streams or threads, race.
+ * Arguments, state handling and errors are otherwise those of qg_step. */
+#define QG_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+qg_status qg_step_noalloc(qg_layer* layer, const void* d_G, int64_t ldg, void* stream);
+
 /* Layer-adaptive subspace refresh (paper section 3.1, Eq. (5)).  Runs when
  * force != 0 or the layer is due (t == t_next); otherwise returns QG_OK with
  * info->refreshed = 0 and touches nothing.  When it runs: randomized top-r SVD

@@ -68,6 +68,7 @@ _SIGNATURES = {
     "qg_layer_sched_set": (c_int32, [c_void_p, POINTER(qg_sched)]),
     "qg_layer_set_projection": (c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_void_p]),
     "qg_step": (c_int32, [c_void_p, c_void_p, c_int64, c_void_p, c_size_t, c_void_p]),
+    "qg_step_noalloc": (c_int32, [c_void_p, c_void_p, c_int64, c_void_p]),
     "qg_step_batch": (c_int32, [POINTER(c_void_p), POINTER(c_void_p), POINTER(c_int64), c_int32, c_void_p, c_size_t,
                                 c_void_p]),
     "qg_step_batch_workspace_bytes": (c_size_t, [POINTER(POINTER(qg_config)), c_int32]),

@@ -130,6 +130,14 @@ qg_status check_step_args(const qg_layer* L, const void* G, int64_t ldg) {
 
 }  // namespace
 
+namespace qg {
+qg_status layer_config(const qg_layer* layer, qg_config* out) {
+  if (!layer || !out) return QG_EINVAL;
+  *out = layer->cfg;
+  return QG_OK;
+}
+}  // namespace qg
+
 extern "C" {
 
 const char* qg_status_str(qg_status s) {
