@@ -120,13 +120,26 @@ def philox4x32_10(c0, c1, c2, c3, k0, k1):
 
 # --------------------------------------------------------------------------
 # Quantizers.  [QG-quant] fixes the widths (INT4 projection, INT8 moments and
-# weights); the grids are readings: symmetric absmax, scale = absmax / qmax
-# (IEEE float32 division), code = clamp(rint(x / scale)) with ties to even, and
-# a zero group gets scale 0 and codes 0.
+# weights); the grids are readings: symmetric absmax; the stored scale is
+# absmax / qmax and the codes are clamp(rint(x * (qmax / absmax))) with ties to
+# even -- the inverse scale is formed once per group (IEEE float32 division)
+# and applied by one multiplication per element; a group whose absmax is below
+# 2^-120 (zero, subnormal or so small that qmax / absmax would overflow) gets
+# scale 0 and codes 0.
 # --------------------------------------------------------------------------
 
 INT4_QMAX = 7
 INT8_QMAX = 127
+ABSMAX_FLOOR = F32(2.0 ** -120)
+
+
+def _absmax_grid(absmax, qmax):
+    """(scale, inverse scale, live) per group; zero for a group below the floor."""
+    absmax = np.asarray(absmax, np.float32)
+    live = absmax >= ABSMAX_FLOOR
+    s = np.where(live, absmax / F32(qmax), F32(0)).astype(np.float32)
+    inv = np.where(live, F32(qmax) / np.where(live, absmax, F32(1)), F32(0)).astype(np.float32)
+    return s, inv, live
 
 
 def quant_int4_groups(P, group=64):
@@ -140,11 +153,9 @@ def quant_int4_groups(P, group=64):
     xp = np.zeros(ng * group, dtype=np.float32)
     xp[: x.size] = x
     xg = xp.reshape(ng, group)
-    absmax = np.max(np.abs(xg), axis=1)
-    s = (absmax / F32(INT4_QMAX)).astype(np.float32)
-    safe = np.where(s > 0, s, F32(1))
-    q = np.clip(np.rint(xg / safe[:, None]), -INT4_QMAX, INT4_QMAX)
-    q = np.where((s > 0)[:, None], q, 0).astype(np.int8)
+    s, inv, live = _absmax_grid(np.max(np.abs(xg), axis=1), INT4_QMAX)
+    q = np.clip(np.rint((xg * inv[:, None]).astype(np.float32)), -INT4_QMAX, INT4_QMAX)
+    q = np.where(live[:, None], q, 0).astype(np.int8)
     return q.ravel()[: x.size], s
 
 
@@ -194,10 +205,9 @@ def quant_rowblock_int8(x, block=256, unsigned=False):
     lo = 0 if unsigned else -INT8_QMAX
     for b in range(nb):
         xs = x[:, b * block: min((b + 1) * block, n)]
-        s = (np.max(np.abs(xs), axis=1) / F32(INT8_QMAX)).astype(np.float32)
-        safe = np.where(s > 0, s, F32(1))
-        q = np.clip(np.rint(xs / safe[:, None]), lo, INT8_QMAX)
-        codes[:, b * block: min((b + 1) * block, n)] = np.where((s > 0)[:, None], q, 0)
+        s, inv, live = _absmax_grid(np.max(np.abs(xs), axis=1), INT8_QMAX)
+        q = np.clip(np.rint((xs * inv[:, None]).astype(np.float32)), lo, INT8_QMAX)
+        codes[:, b * block: min((b + 1) * block, n)] = np.where(live[:, None], q, 0)
         scales[:, b] = s
     return codes, scales
 
@@ -238,12 +248,13 @@ class Config:
 
 
 def adam_constants(cfg: Config, t: int):
-    """float32 constants of step t (t counted from 1 per layer): (1-b1), (1-b2),
-    and the bias corrections 1-b1^t, 1-b2^t, formed in float64 from the float32
-    betas and rounded once to float32."""
+    """float32 constants of step t (t counted from 1 per layer), each formed in
+    float64 from the float32 hyper-parameters and rounded once to float32:
+    (1 - b1), (1 - b2), c1 = -lr / (1 - b1^t), c2 = 1 / sqrt(1 - b2^t)."""
     b1 = float(F32(cfg.beta1))
     b2 = float(F32(cfg.beta2))
-    return (F32(1.0 - b1), F32(1.0 - b2), F32(1.0 - b1 ** t), F32(1.0 - b2 ** t))
+    lr = float(F32(cfg.lr))
+    return (F32(1.0 - b1), F32(1.0 - b2), F32(-lr / (1.0 - b1 ** t)), F32(1.0 / np.sqrt(1.0 - b2 ** t)))
 
 
 # --------------------------------------------------------------------------
@@ -265,18 +276,20 @@ def adam_moments(R, m0, v0, cfg: Config, t: int):
 
         m = b1*m0 + (1-b1)*R
         v = b2*v0 + (1-b2)*(R*R)
-        N = (-lr * (m / (1-b1^t))) / (sqrt(v / (1-b2^t)) + eps)
+        N = -lr * m_hat / (sqrt(v_hat) + eps),  m_hat = m/(1-b1^t), v_hat = v/(1-b2^t)
+
+    evaluated as N = (m * c1) / (sqrt(v) * c2 + eps) with the per-step scalars
+    c1 = -lr/(1-b1^t) and c2 = 1/sqrt(1-b2^t) (the same quantity; one float32
+    rounding per operation, in this order).
 
     Returns (N float32 before bf16 rounding, m, v).
     """
-    om1, om2, bc1, bc2 = adam_constants(cfg, t)
+    om1, om2, c1, c2 = adam_constants(cfg, t)
     R = np.asarray(R, np.float32)
     m = (cfg.f32("beta1") * m0 + om1 * R).astype(np.float32)
     v = (cfg.f32("beta2") * v0 + om2 * (R * R)).astype(np.float32)
-    mhat = (m / bc1).astype(np.float32)
-    vhat = (v / bc2).astype(np.float32)
-    num = (F32(-cfg.lr) * mhat).astype(np.float32)
-    den = (np.sqrt(vhat) + cfg.f32("eps")).astype(np.float32)
+    num = (m * c1).astype(np.float32)
+    den = ((np.sqrt(v) * c2).astype(np.float32) + cfg.f32("eps")).astype(np.float32)
     return (num / den).astype(np.float32), m, v
 
 

@@ -149,6 +149,19 @@ def test_int8_rowblock_golden():
     assert c[0, 256:258].tolist() == rg["tail_codes"]
 
 
+def test_zero_and_subnormal_groups_quantize_to_zero():
+    x = np.zeros((2, 256), np.float32)
+    x[1, 3] = np.float32(1e-39)   # subnormal absmax
+    c, s = O.quant_rowblock_int8(x, 256)
+    assert np.all(c == 0) and np.all(s == 0)
+    q4, s4 = O.quant_int4_groups(np.full(64, 1e-40, np.float32))
+    assert np.all(q4 == 0) and s4[0] == 0
+    c, s = O.quant_rowblock_int8(np.full((1, 4), 2.0 ** -121, np.float32), 256)
+    assert np.all(c == 0) and s[0, 0] == 0
+    c, s = O.quant_rowblock_int8(np.array([[2.0 ** -120, 0.0, -2.0 ** -121]], np.float32), 256)
+    assert c[0].tolist() == [127, 0, -64] and s[0, 0] > 0
+
+
 def test_int8_rowblock_roundtrip():
     rng = np.random.default_rng(3)
     x = (rng.standard_normal((7, 600)) * 1e-3).astype(np.float32)
