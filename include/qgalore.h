@@ -199,7 +199,8 @@ qg_status qg_sched_after_refresh(int64_t t, int32_t delta, int32_t has_cossim, f
  * row stride ld (elements) -> ceil(m*r/2) packed bytes (two's-complement
  * nibbles, even index in the low nibble) and ceil(m*r/64) scales; groups of 64
  * consecutive elements of the row-major m x r array, scale = absmax / 7,
- * code = clamp(rint(x / scale), -7, 7), a zero group gets scale 0. */
+ * code = clamp(rint(x * (7 / absmax)), -7, 7); a group whose absmax is below
+ * 2^-120 gets scale 0 and codes 0. */
 qg_status qg_quantize_projection(const float* d_P, int64_t ld, int32_t m, int32_t r, uint8_t* d_Pq,
                                  float* d_sP, void* stream);
 

@@ -109,9 +109,8 @@ void fill_step_problem(const qg_layer* L, const void* G, int64_t ldg, uint8_t* w
   s->beta2 = c.beta2;
   s->om1 = static_cast<float>(1.0 - b1);
   s->om2 = static_cast<float>(1.0 - b2);
-  s->bc1 = static_cast<float>(1.0 - pow(b1, static_cast<double>(t)));
-  s->bc2 = static_cast<float>(1.0 - pow(b2, static_cast<double>(t)));
-  s->neg_lr = -c.lr;
+  s->c1 = static_cast<float>(-static_cast<double>(c.lr) / (1.0 - pow(b1, static_cast<double>(t))));
+  s->c2 = static_cast<float>(1.0 / sqrt(1.0 - pow(b2, static_cast<double>(t))));
   s->eps = c.eps;
   s->alpha = c.alpha;
   s->t = static_cast<uint32_t>(t);

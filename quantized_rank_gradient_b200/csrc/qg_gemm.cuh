@@ -5,7 +5,10 @@
 //
 //   warp 0      : TMA producer (one elected lane)
 //   warp 1      : TMEM allocator + MMA issuer (one elected lane)
-//   warps 2..5  : epilogue, one TMEM lane quarter each (row = quarter*32 + lane)
+//   warps 2..9  : two epilogue warpgroups; warpgroup g drains TMEM buffer g, i.e.
+//                 every other tile of the CTA, so two tiles' epilogues overlap
+//                 each other and the MMAs.  Within a warpgroup each warp owns one
+//                 TMEM lane quarter (row = quarter*32 + lane).
 //
 // A grid of at most one CTA per SM walks a flat list of tiles that spans up to
 // kMaxProblems independent problems (a batch of weight matrices).  Within a
@@ -28,7 +31,7 @@ constexpr int BK = 64;
 constexpr int kStages = 4;
 constexpr int kAStageBytes = BM * BK * 2;  // 16 KiB
 constexpr int kBStageBytes = BN * BK * 2;  // 32 KiB
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;
 constexpr int kMaxProblems = 8;
 constexpr int kTmemCols = 2 * BN;  // 512: the whole TMEM of the SM
 constexpr size_t kGemmSmemBytes = size_t(kStages) * (kAStageBytes + kBStageBytes) + 1024;
@@ -203,21 +206,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    const uint32_t eg = static_cast<uint32_t>(warp - 2) >> 2;  // warpgroup = TMEM buffer
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    uint32_t acc = 0, acc_phase = 0;
-    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
+    uint32_t acc_phase = 0, it = 0;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++it) {
+      if ((it & 1u) != eg) continue;
       const TileRef tr = locate_tile(p, tile);
       const GemmProblem<Epi>& pr = p.prob[tr.prob];
-      if (!mbar_wait(&acc_full[acc], acc_phase, &abort_flag, status)) break;
+      if (!mbar_wait(&acc_full[eg], acc_phase, &abort_flag, status)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + eg * BN;
       Epi::apply(pr.epi, pr.M, pr.N, tr.mb, tr.nb, row, taddr, pr.status);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
-      acc ^= 1u;
-      if (acc == 0) acc_phase ^= 1u;
+      if (lane == 0) mbar_arrive(&acc_empty[eg]);
+      acc_phase ^= 1u;
     }
   }
 

@@ -25,7 +25,7 @@ struct StepProblem {
   uint16_t* Nbuf;       // scratch: r x ldN bf16
   int64_t ldN;
   int32_t m, n, r;
-  float beta1, beta2, om1, om2, bc1, bc2, neg_lr, eps, alpha;
+  float beta1, beta2, om1, om2, c1, c2, eps, alpha;  // c1 = -lr/(1-b1^t), c2 = 1/sqrt(1-b2^t)
   uint32_t t, layer_id;
   uint64_t seed;
   uint32_t* status;

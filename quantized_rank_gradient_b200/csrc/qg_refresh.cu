@@ -7,8 +7,8 @@
 namespace qg {
 
 // One warp per group of 64 consecutive elements of the row-major m x r array:
-// scale = absmax / 7 (IEEE division), code = clamp(rint(x / scale), -7, 7),
-// packed two per byte with the even element in the low nibble.
+// scale = absmax / 7, code = clamp(rint(x * (7 / absmax)), -7, 7) (both IEEE
+// divisions once per group), packed two per byte, even element in the low nibble.
 __global__ void quantize_int4_kernel(const float* __restrict__ P, int64_t ld, int32_t m, int32_t r,
                                      uint8_t* __restrict__ Pq, float* __restrict__ sP, int64_t ngroups) {
   const int64_t g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -25,11 +25,14 @@ __global__ void quantize_int4_kernel(const float* __restrict__ P, int64_t ld, in
   float amax = fmaxf(fabsf(x[0]), fabsf(x[1]));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-  const float s = __fdiv_rn(amax, 7.0f);
+  // scale absmax / 7, codes rint(x * (7 / absmax)); absmax below 2^-120: zero group
+  const bool live = amax >= 7.52316384526264e-37f;
+  const float s = live ? __fdiv_rn(amax, 7.0f) : 0.f;
+  const float inv = live ? __fdiv_rn(7.0f, amax) : 0.f;
   int q[2] = {0, 0};
-  if (s > 0.f) {
+  if (live) {
 #pragma unroll
-    for (int k = 0; k < 2; ++k) q[k] = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(x[k], s)), -7.f), 7.f));
+    for (int k = 0; k < 2; ++k) q[k] = static_cast<int>(fminf(fmaxf(rintf(__fmul_rn(x[k], inv)), -7.f), 7.f));
   }
   const int64_t e0 = g * 64 + 2 * lane;
   if (e0 < total) Pq[e0 >> 1] = static_cast<uint8_t>((q[0] & 0xF) | ((q[1] & 0xF) << 4));

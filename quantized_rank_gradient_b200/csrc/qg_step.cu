@@ -31,6 +31,10 @@ namespace qg {
 
 static_assert(kErrTimeout == kStatusTimeout && kErrNonFinite == kStatusNonFinite, "status bits");
 
+// Groups / blocks whose absmax is below this are quantized as zero (127 / absmax
+// would overflow float32).
+constexpr float kAbsmaxFloor = 7.52316384526264e-37f;  // 2^-120
+
 // ------------------------------------------------------------------ helpers
 
 QG_DEV int8_t byte_of(const uint4& v, int k) {
@@ -54,7 +58,7 @@ struct AdamEpi {
     int64_t ld_mom;
     int64_t ldN;
     int32_t nblk;
-    float beta1, beta2, om1, om2, bc1, bc2, neg_lr, eps;
+    float beta1, beta2, om1, om2, c1, c2, eps;
   };
 
   // m = b1*m0 + (1-b1)*R ; v = b2*v0 + (1-b2)*(R*R), one rounding per operation.
@@ -91,7 +95,8 @@ struct AdamEpi {
     float amax_m = 0.f, amax_v = 0.f;
     bool bad = false;
 
-    // pass 1: moments, block absmax, N = -lr * m_hat / (sqrt(v_hat) + eps) -> bf16
+    // pass 1: moments, block absmax of |m| and sqrt(v),
+    // N = -lr * m_hat / (sqrt(v_hat) + eps) = (m * c1) / (sqrt(v) * c2 + eps) -> bf16
     for (int c = 0; c < nchunks; ++c) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(taddr + c * 32, v);
@@ -110,14 +115,13 @@ struct AdamEpi {
         const int8_t vc = e < 16 ? byte_of(vq0, e) : byte_of(vq1, e - 16);
         float mm, vv;
         moments(R, mc, vc, sm, sv, a, mm, vv);
+        const float rv = __fsqrt_rn(vv);
         if (e < valid) {
           amax_m = fmaxf(amax_m, fabsf(mm));
-          amax_v = fmaxf(amax_v, __fsqrt_rn(vv));
+          amax_v = fmaxf(amax_v, rv);
           bad |= !isfinite(R);
         }
-        const float mhat = __fdiv_rn(mm, a.bc1);
-        const float vhat = __fdiv_rn(vv, a.bc2);
-        const float upd = __fdiv_rn(__fmul_rn(a.neg_lr, mhat), __fadd_rn(__fsqrt_rn(vhat), a.eps));
+        const float upd = __fdiv_rn(__fmul_rn(mm, a.c1), __fadd_rn(__fmul_rn(rv, a.c2), a.eps));
         const uint32_t b = bf16_bits_rn(upd);
         if (e & 1)
           packed[e >> 1] |= b << 16;
@@ -130,10 +134,14 @@ struct AdamEpi {
         dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
     }
 
-    // new block scales: absmax(|m|) / 127 and absmax(sqrt(v)) / 127 (IEEE
-    // division); a zero block gets scale 0
-    const float s_m = __fdiv_rn(amax_m, 127.0f);
-    const float s_v = __fdiv_rn(amax_v, 127.0f);
+    // new block scales absmax / 127 and inverse scales 127 / absmax (IEEE
+    // divisions, once per block); a block whose absmax is below 2^-120 is a zero
+    // block (scale 0, codes 0)
+    const bool live_m = amax_m >= kAbsmaxFloor, live_v = amax_v >= kAbsmaxFloor;
+    const float s_m = live_m ? __fdiv_rn(amax_m, 127.0f) : 0.f;
+    const float s_v = live_v ? __fdiv_rn(amax_v, 127.0f) : 0.f;
+    const float inv_m = live_m ? __fdiv_rn(127.0f, amax_m) : 0.f;
+    const float inv_v = live_v ? __fdiv_rn(127.0f, amax_v) : 0.f;
 
     // pass 2: recompute the same moments bit for bit, re-quantize them
     for (int c = 0; c < nchunks; ++c) {
@@ -154,8 +162,8 @@ struct AdamEpi {
         float mm, vv;
         moments(R, mc, vc, sm, sv, a, mm, vv);
         int qm = 0, qv = 0;
-        if (s_m > 0.f) qm = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(mm, s_m)), -127.f), 127.f));
-        if (s_v > 0.f) qv = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(__fsqrt_rn(vv), s_v)), 0.f), 127.f));
+        if (live_m) qm = static_cast<int>(fminf(fmaxf(rintf(__fmul_rn(mm, inv_m)), -127.f), 127.f));
+        if (live_v) qv = static_cast<int>(fminf(fmaxf(rintf(__fmul_rn(__fsqrt_rn(vv), inv_v)), 0.f), 127.f));
         const uint32_t bm = static_cast<uint32_t>(qm) & 0xFFu;
         const uint32_t bv = static_cast<uint32_t>(qv) & 0xFFu;
         if ((e & 3) == 0) {
@@ -339,25 +347,35 @@ static_assert(sizeof(GemmParams<StoreF32Epi>) <= 4096, "kernel parameter block")
 
 // Eight INT4 codes (one 32-bit word, element 2i in the low nibble of byte i)
 // -> eight bf16 of P~ = bf16_rn(code * scale).  Groups of 64 never split a word.
-__global__ void dequant_projection_kernel(const uint8_t* __restrict__ Pq, const float* __restrict__ sP,
-                                          int64_t total, uint16_t* __restrict__ out) {
+// One launch covers up to kMaxProblems projections.
+struct DequantBatch {
+  const uint8_t* Pq[kMaxProblems];
+  const float* sP[kMaxProblems];
+  uint16_t* out[kMaxProblems];
+  int64_t chunk_begin[kMaxProblems + 1];  // prefix sums of (m*r / 8)
+  int32_t n;
+};
+
+__global__ void dequant_projection_kernel(const __grid_constant__ DequantBatch b) {
   const int64_t i8 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t e0 = i8 * 8;
-  if (e0 >= total) return;
-  const uint32_t word = *reinterpret_cast<const uint32_t*>(Pq + (e0 >> 1));
-  const float s = sP[e0 >> 6];
+  if (i8 >= b.chunk_begin[b.n]) return;
+  int p = 0;
+  while (p + 1 < b.n && i8 >= b.chunk_begin[p + 1]) ++p;
+  const int64_t e0 = (i8 - b.chunk_begin[p]) * 8;
+  const uint32_t word = *reinterpret_cast<const uint32_t*>(b.Pq[p] + (e0 >> 1));
+  const float s = b.sP[p][e0 >> 6];
   uint32_t pk[4];
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     const int nib = static_cast<int>((word >> (4 * k)) & 0xFu);
     const int code = (nib ^ 8) - 8;
-    const uint32_t b = bf16_bits_rn(__fmul_rn(static_cast<float>(code), s));
+    const uint32_t bits = bf16_bits_rn(__fmul_rn(static_cast<float>(code), s));
     if (k & 1)
-      pk[k >> 1] |= b << 16;
+      pk[k >> 1] |= bits << 16;
     else
-      pk[k >> 1] = b;
+      pk[k >> 1] = bits;
   }
-  *reinterpret_cast<uint4*>(out + e0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  *reinterpret_cast<uint4*>(b.out[p] + e0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
 }
 
 __global__ void philox_kernel(const uint32_t* c0, const uint32_t* c1, const uint32_t* c2, const uint32_t* c3,
@@ -442,17 +460,29 @@ static void add_problem(GemmParams<Epi>& p, int M, int N, int K) {
   p.nprob += 1;
 }
 
-cudaError_t launch_dequant_projection(const uint8_t* Pq, const float* sP, int64_t total, uint16_t* out,
-                                      cudaStream_t stream) {
-  const int64_t chunks = total / 8;
+static cudaError_t launch_dequant_batch(const DequantBatch& b, cudaStream_t stream) {
+  const int64_t chunks = b.chunk_begin[b.n];
   if (chunks == 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (chunks + threads - 1) / threads;
-  const double bytes = total / 2.0 + (total + 63) / 64 * 4.0 + total * 2.0;
+  const double total = chunks * 8.0;
+  const double bytes = total / 2.0 + total / 64.0 * 4.0 + total * 2.0;
   const int tok = profile_begin(stream, QG_KERNEL_DEQUANT, 0.0, bytes);
-  dequant_projection_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(Pq, sP, total, out);
+  dequant_projection_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(b);
   profile_end(stream, tok);
   return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_projection(const uint8_t* Pq, const float* sP, int64_t total, uint16_t* out,
+                                      cudaStream_t stream) {
+  DequantBatch b;
+  memset(&b, 0, sizeof(b));
+  b.Pq[0] = Pq;
+  b.sP[0] = sP;
+  b.out[0] = out;
+  b.chunk_begin[1] = total / 8;
+  b.n = 1;
+  return launch_dequant_batch(b, stream);
 }
 
 cudaError_t launch_philox(const uint32_t* c0, const uint32_t* c1, const uint32_t* c2, const uint32_t* c3,
@@ -466,13 +496,21 @@ cudaError_t launch_philox(const uint32_t* c0, const uint32_t* c1, const uint32_t
 
 cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream) {
   cudaError_t e;
-  for (int i = 0; i < count; ++i) {
-    e = launch_dequant_projection(probs[i].Pq, probs[i].sP, static_cast<int64_t>(probs[i].m) * probs[i].r,
-                                  probs[i].Pbf, stream);
-    if (e != cudaSuccess) return e;
-  }
   for (int base = 0; base < count; base += kMaxProblems) {
     const int cnt = std::min(kMaxProblems, count - base);
+    DequantBatch db;
+    memset(&db, 0, sizeof(db));
+    for (int i = 0; i < cnt; ++i) {
+      const StepProblem& s = probs[base + i];
+      db.Pq[i] = s.Pq;
+      db.sP[i] = s.sP;
+      db.out[i] = s.Pbf;
+      db.chunk_begin[i + 1] = db.chunk_begin[i] + static_cast<int64_t>(s.m) * s.r / 8;
+    }
+    db.n = cnt;
+    e = launch_dequant_batch(db, stream);
+    if (e != cudaSuccess) return e;
+
     GemmParams<AdamEpi> p1;
     memset(&p1, 0, sizeof(p1));
     double fl1 = 0, by1 = 0, fl2 = 0, by2 = 0;
@@ -492,7 +530,7 @@ cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream
       if (!encode_map_bf16(&pr.tmB, s.G, s.n, s.m, s.ldg, 64, 64)) return cudaErrorInvalidValue;
       pr.status = s.status;
       pr.epi = AdamEpi::Args{s.Mq, s.Vq, s.sM, s.sV, s.Nbuf, s.ld_mom, s.ldN, s.nblk,
-                             s.beta1, s.beta2, s.om1, s.om2, s.bc1, s.bc2, s.neg_lr, s.eps};
+                             s.beta1, s.beta2, s.om1, s.om2, s.c1, s.c2, s.eps};
       add_problem(p1, s.r, s.n, s.m);
     }
     e = launch_gemm<AdamEpi, true, true>(p1, stream, QG_KERNEL_PROJECT_ADAM, fl1, by1);
