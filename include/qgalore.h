@@ -175,7 +175,14 @@ qg_status qg_step_noalloc(qg_layer* layer, const void* d_G, int64_t ldg, void* s
  * info->refreshed = 0 and touches nothing.  When it runs: randomized top-r SVD
  * of G -> new INT4 P; if a projection existed, CosSim(P_new, P_prev) on the
  * device; the interval doubles iff CosSim > gamma; t_next = t + delta.  This
- * call synchronises `stream` to read CosSim.  `info` may be NULL. */
+ * call synchronises `stream` to read CosSim.  `info` may be NULL.
+ *   d_ws: >= qg_refresh_workspace_bytes(cfg) bytes, 256-byte aligned.  After a
+ *   refresh its first m*r*4 bytes hold the float32 projection (row-major m x r,
+ *   orthonormal columns sorted by descending singular value, each column's
+ *   largest-magnitude entry positive) from which the INT4 one was quantized.
+ * Randomized SVD: k = min(r + oversample, m, n) columns, Rademacher test
+ * matrix from Philox keyed by the seed and counted by (refresh index, layer_id),
+ * power_iters power iterations, Rayleigh-Ritz on the k-dimensional range. */
 qg_status qg_refresh(qg_layer* layer, const void* d_G, int64_t ldg, int32_t force, void* d_ws,
                      size_t ws_bytes, qg_refresh_info* info, void* stream);
 

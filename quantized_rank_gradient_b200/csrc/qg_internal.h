@@ -45,9 +45,10 @@ cudaError_t launch_dequant_projection(const uint8_t* Pq, const float* sP, int64_
 cudaError_t launch_philox(const uint32_t* c0, const uint32_t* c1, const uint32_t* c2,
                           const uint32_t* c3, int64_t count, uint32_t k0, uint32_t k1, uint32_t* out,
                           cudaStream_t stream);
+// D = A B (or D += A B when accumulate), bf16 operands on the tcgen05 core.
 cudaError_t launch_gemm_f32(const void* A, int64_t lda, bool a_trans, const void* B, int64_t ldb,
                             bool b_trans, float* D, int64_t ldd, int M, int N, int K,
-                            cudaStream_t stream);
+                            cudaStream_t stream, bool accumulate = false);
 
 // Tensor-map encoder (driver entry point, resolved once).  Returns false when
 // the driver refuses the map.

@@ -1,10 +1,341 @@
-// Subspace refresh on sm_100a: INT4 quantization of a projection (being
-// extended to the full randomized top-r SVD and CosSim).
+// Layer-adaptive subspace refresh on sm_100a (the method's SVD step and its
+// CosSim interval rule: AIMech Q-GaLore page, mechanism "layer-adaptive
+// subspace cosine schedule", paper section 3.1, Eq. (5)).
+//
+// Top-r left singular vectors of G by randomized subspace iteration (Halko,
+// Martinsson, Tropp 2011): Omega (n x k, Rademacher from Philox), Y = G Omega,
+// Q = orth(Y); q times { Z = orth(G^T Q); Q = orth(G Z) }; B = Q^T G;
+// S = B B^T = V diag(lambda) V^T; P = Q V[:, top r].  The products with G run on
+// the tcgen05 core (bf16 operands, fp32 accumulation); orth() is shifted
+// Cholesky-QR in three passes (Fukaya et al. 2020) with fp32 SIMT Gram matrices;
+// the k x k eigenproblem and the r x r singular values of CosSim use a one-sided
+// Jacobi with a bounded grid barrier.  Then: sign canonicalisation, INT4
+// quantization, and CosSim(P_new, P_prev) = (1/r) sum_i sigma_i(P_new^T P_prev)
+// on the dequantized projections.
+#include <algorithm>
+#include <cstring>
+
 #include "qg_device.cuh"
 #include "qg_internal.h"
+#include "qg_linalg.cuh"
+#include "qg_philox.cuh"
 #include "qg_refresh.h"
 
 namespace qg {
+
+namespace {
+
+constexpr float kAbsmaxFloorR = 7.52316384526264e-37f;  // 2^-120
+constexpr uint32_t kOmegaSalt = 0x52454652u;
+constexpr int kJacobiMaxSweeps = 30;
+constexpr float kJacobiTol = 2e-6f;
+
+size_t r256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct RefreshLayout {
+  int k, ldk, ldn4;
+  size_t P, omega, Y, Yb, Ylo, Z, Zb, gram, linv, Bm, At, Vt, lam, perm, Vsel, Pa, Pb, Ct, misc, total;
+};
+
+RefreshLayout refresh_layout(int m, int n, int r, int p) {
+  RefreshLayout L;
+  L.k = std::min(std::min(r + p, m), n);
+  L.ldk = (L.k + 7) / 8 * 8;
+  L.ldn4 = (n + 3) / 4 * 4;
+  const size_t k = L.k, ldk = L.ldk;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += r256(bytes);
+    return o;
+  };
+  L.P = take(size_t(m) * r * 4);
+  L.omega = take(size_t(n) * ldk * 2);
+  L.Y = take(size_t(m) * ldk * 4);
+  L.Yb = take(size_t(m) * ldk * 2);
+  L.Ylo = take(size_t(m) * ldk * 2);
+  L.Z = take(size_t(n) * ldk * 4);
+  L.Zb = take(size_t(n) * ldk * 2);
+  L.gram = take(k * ldk * 4);
+  L.linv = take(((k + 31) / 32) * 1024 * 4);
+  L.Bm = take(k * L.ldn4 * 4);
+  L.At = take(k * ldk * 4);
+  L.Vt = take(k * ldk * 4);
+  L.lam = take(k * 4);
+  L.perm = take(k * 4);
+  L.Vsel = take(k * size_t(r) * 4);
+  L.Pa = take(size_t(m) * r * 4);
+  L.Pb = take(size_t(m) * r * 4);
+  L.Ct = take(size_t(r) * r * 4);
+  L.misc = take(256);
+  L.total = off;
+  return L;
+}
+
+// misc region: [0..3] grid barrier + rotation counter, [4] Cholesky flag,
+// [5] Jacobi sweeps, [6] CosSim value (float)
+struct Misc {
+  unsigned bar[4];
+  int chol_flag;
+  int sweeps;
+  float cossim;
+};
+
+// ------------------------------------------------------------------ kernels
+
+// Omega (n x ldk bf16): entry e = j*k + c (c < k) takes bit (e mod 32) of word
+// ((e / 32) mod 4) of Philox-4x32-10(counter = (e / 128, refresh, layer, 0),
+// key = (seed_lo ^ salt, seed_hi)); a set bit gives -1, else +1.  Padding 0.
+__global__ void omega_kernel(uint16_t* Om, int64_t ld, int n, int k, uint32_t refresh_idx, uint32_t layer_id,
+                             PhiloxKey key) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(n) * ld) return;
+  const int64_t j = idx / ld, c = idx % ld;
+  uint16_t out = 0;
+  if (c < k) {
+    const uint64_t e = static_cast<uint64_t>(j) * k + c;
+    uint32_t w[4];
+    philox4x32_10(static_cast<uint32_t>(e >> 7), refresh_idx, layer_id, 0u, key, w);
+    const uint32_t word = w[(e >> 5) & 3];
+    out = ((word >> (e & 31)) & 1u) ? 0xBF80u : 0x3F80u;  // bf16 -1 / +1
+  }
+  Om[idx] = out;
+}
+
+// Diagonal shift of the first Cholesky-QR pass: s = 11 (rows k + k (k + 1)) u tr(A),
+// u = 2^-24, tr(A) = ||X||_F^2.
+__global__ void __launch_bounds__(1024) add_shift_kernel(float* A, int64_t ld, int k, int rows) {
+  __shared__ float part[32];
+  float s = 0.f;
+  for (int i = threadIdx.x; i < k; i += blockDim.x) s += A[static_cast<int64_t>(i) * ld + i];
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = (threadIdx.x < (blockDim.x >> 5)) ? part[threadIdx.x] : 0.f;
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+    if (threadIdx.x == 0) part[0] = t;
+  }
+  __syncthreads();
+  const float shift = 11.f * (static_cast<float>(rows) * k + static_cast<float>(k) * (k + 1)) * 5.9604645e-8f * part[0];
+  for (int i = threadIdx.x; i < k; i += blockDim.x) A[static_cast<int64_t>(i) * ld + i] += shift;
+}
+
+__global__ void identity_kernel(float* V, int64_t ld, int k) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(k) * ld) return;
+  V[idx] = (idx / ld == idx % ld) ? 1.f : 0.f;
+}
+
+// out[p] = || row p of At ||  (one warp per row)
+__global__ void row_norms_kernel(const float* At, int64_t ld, int k, int cols, float* out) {
+  const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (w >= k) return;
+  float s = 0.f;
+  for (int t = lane; t < cols; t += 32) {
+    const float x = __ldcg(At + static_cast<int64_t>(w) * ld + t);
+    s = __fmaf_rn(x, x, s);
+  }
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+  if (lane == 0) out[w] = sqrtf(s);
+}
+
+// perm[rank] = p with ranks by descending lambda, ties to the lower index.
+__global__ void __launch_bounds__(1024) rank_sort_kernel(const float* lam, int k, int* perm) {
+  for (int p = threadIdx.x; p < k; p += blockDim.x) {
+    const float v = lam[p];
+    int rank = 0;
+    for (int q = 0; q < k; ++q) {
+      const float u = lam[q];
+      rank += (u > v) || (u == v && q < p);
+    }
+    perm[rank] = p;
+  }
+}
+
+// Vsel[t][c] = V[t][perm[c]] = Vt[perm[c]][t]  (k x r)
+__global__ void gather_kernel(const float* Vt, int64_t ld, const int* perm, int k, int r, float* Vsel) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(k) * r) return;
+  const int t = static_cast<int>(idx / r), c = static_cast<int>(idx % r);
+  int pc = perm[c];
+  if (pc < 0 || pc >= k) pc = 0;  // only reachable with non-finite eigenvalues
+  Vsel[idx] = Vt[static_cast<int64_t>(pc) * ld + t];
+}
+
+// Column c of P (m x r): the entry of largest magnitude (first row on ties) is
+// made positive by negating the column when needed.
+__global__ void __launch_bounds__(256) canonical_signs_kernel(float* P, int m, int r) {
+  const int c = blockIdx.x;
+  __shared__ float bv[256];
+  __shared__ int bi[256];
+  float best = -1.f;
+  int besti = 0x7FFFFFFF;
+  for (int i = threadIdx.x; i < m; i += blockDim.x) {
+    const float a = fabsf(P[static_cast<int64_t>(i) * r + c]);
+    if (a > best) {
+      best = a;
+      besti = i;
+    }
+  }
+  bv[threadIdx.x] = best;
+  bi[threadIdx.x] = besti;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) {
+      const float ov = bv[threadIdx.x + s];
+      const int oi = bi[threadIdx.x + s];
+      if (ov > bv[threadIdx.x] || (ov == bv[threadIdx.x] && oi < bi[threadIdx.x])) {
+        bv[threadIdx.x] = ov;
+        bi[threadIdx.x] = oi;
+      }
+    }
+    __syncthreads();
+  }
+  __shared__ int flip_s;
+  if (threadIdx.x == 0) flip_s = bi[0] < m && P[static_cast<int64_t>(bi[0]) * r + c] < 0.f;
+  __syncthreads();
+  if (flip_s)
+    for (int i = threadIdx.x; i < m; i += blockDim.x) P[static_cast<int64_t>(i) * r + c] = -P[static_cast<int64_t>(i) * r + c];
+}
+
+// P = code * scale in float32 (m x r, row stride r) from packed INT4.
+__global__ void dequant_f32_kernel(const uint8_t* Pq, const float* sP, int64_t total, float* out) {
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= total) return;
+  const uint8_t b = Pq[e >> 1];
+  const int nib = (e & 1) ? (b >> 4) : (b & 0xF);
+  const int code = (nib ^ 8) - 8;
+  out[e] = __fmul_rn(static_cast<float>(code), sP[e >> 6]);
+}
+
+// out = (1/r) sum_p || row p of Ct ||   (Ct rows: the columns of C after Jacobi)
+__global__ void __launch_bounds__(1024) mean_row_norm_kernel(const float* Ct, int64_t ld, int r, float* out) {
+  __shared__ float part[32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  float acc = 0.f;
+  for (int p = w; p < r; p += nw) {
+    float s = 0.f;
+    for (int t = lane; t < r; t += 32) {
+      const float x = __ldcg(Ct + static_cast<int64_t>(p) * ld + t);
+      s = __fmaf_rn(x, x, s);
+    }
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    acc += sqrtf(s);
+  }
+  if (lane == 0) part[w] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int i = 0; i < nw; ++i) t += part[i];
+    *out = t / static_cast<float>(r);
+  }
+}
+
+// ------------------------------------------------------------------ host helpers
+
+cudaError_t sgemm(bool ta, bool tb, const float* A, int64_t lda, const float* B, int64_t ldb, float* C, int64_t ldc,
+                  int M, int N, int K, cudaStream_t s) {
+  const dim3 grid((N + kSgBN - 1) / kSgBN, (M + kSgBM - 1) / kSgBM);
+  const int tok = profile_begin(s, QG_KERNEL_OTHER, 2.0 * M * N * K, 4.0 * (double(M) * K + double(K) * N + double(M) * N));
+  if (ta && tb)
+    sgemm_kernel<true, true><<<grid, 256, 0, s>>>(A, lda, B, ldb, C, ldc, M, N, K, 1.f, 0.f);
+  else if (ta)
+    sgemm_kernel<true, false><<<grid, 256, 0, s>>>(A, lda, B, ldb, C, ldc, M, N, K, 1.f, 0.f);
+  else if (tb)
+    sgemm_kernel<false, true><<<grid, 256, 0, s>>>(A, lda, B, ldb, C, ldc, M, N, K, 1.f, 0.f);
+  else
+    sgemm_kernel<false, false><<<grid, 256, 0, s>>>(A, lda, B, ldb, C, ldc, M, N, K, 1.f, 0.f);
+  profile_end(s, tok);
+  return cudaGetLastError();
+}
+
+// Lower Cholesky factor of the k x k matrix A in place (blocked, 32-wide panels);
+// Linv receives the inverses of the diagonal blocks.
+cudaError_t cholesky(float* A, int64_t ld, int k, float* Linv, int* flag, cudaStream_t s) {
+  for (int j0 = 0; j0 < k; j0 += 32) {
+    const int nb = std::min(32, k - j0);
+    potrf_diag_kernel<<<1, dim3(32, 32), 0, s>>>(A, ld, j0, nb, Linv + static_cast<size_t>(j0 / 32) * 1024, flag);
+    const int rest = k - j0 - 32;
+    if (rest > 0) {
+      const int T = (rest + 31) / 32;
+      trsm_panel_kernel<<<T, dim3(32, 32), 0, s>>>(A, ld, j0, k, Linv + static_cast<size_t>(j0 / 32) * 1024);
+      syrk_update_kernel<<<T * (T + 1) / 2, dim3(32, 32), 0, s>>>(A, ld, j0, k);
+    }
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t trsm_rows(float* X, int64_t ldx, uint16_t* Xb, uint16_t* Xlo, int64_t ldb, int rows, int k,
+                      const float* L, int64_t ldl, const float* Linv, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(32) * (k + 1) * sizeof(float);
+  static size_t smem_set = 0;
+  if (smem > smem_set) {
+    cudaError_t e = cudaFuncSetAttribute(trsm_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    smem_set = smem;
+  }
+  trsm_rows_kernel<<<(rows + 31) / 32, 256, smem, s>>>(X, ldx, Xb, Xlo, ldb, rows, k, L, ldl, Linv);
+  return cudaGetLastError();
+}
+
+// Shifted Cholesky-QR, three passes: X (rows x k fp32, stride ld) becomes an
+// orthonormal basis of its column span; Xb receives its bf16 copy and Xlo (if
+// non-null) the bf16 residual.
+cudaError_t orth(float* X, uint16_t* Xb, uint16_t* Xlo, int rows, int k, int64_t ld, float* gram, float* linv,
+                 int* flag, cudaStream_t s) {
+  cudaError_t e;
+  for (int pass = 0; pass < 3; ++pass) {
+    if ((e = sgemm(true, false, X, ld, X, ld, gram, ld, k, k, rows, s)) != cudaSuccess) return e;
+    if (pass == 0) {
+      add_shift_kernel<<<1, 1024, 0, s>>>(gram, ld, k, rows);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if ((e = cholesky(gram, ld, k, linv, flag, s)) != cudaSuccess) return e;
+    if ((e = trsm_rows(X, ld, pass == 2 ? Xb : nullptr, pass == 2 ? Xlo : nullptr, ld, rows, k, gram, ld, linv, s)) !=
+        cudaSuccess)
+      return e;
+  }
+  return cudaSuccess;
+}
+
+// One-sided Jacobi on the k x k matrix stored transposed in At (and Vt, if any).
+cudaError_t jacobi(float* At, float* Vt, int64_t ld, int k, unsigned* bar, int* sweeps, uint32_t* status,
+                   cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(bar, 0, 4 * sizeof(unsigned), s);
+  if (e != cudaSuccess) return e;
+  const int pairs = (k + 1) / 2;
+  int grid = std::min(sm_count(), std::max(1, (pairs + 7) / 8));
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, jacobi_kernel, 256, 0);
+  if (e != cudaSuccess) return e;
+  grid = std::min(grid, std::max(1, per_sm) * sm_count());
+  int max_sweeps = kJacobiMaxSweeps;
+  float tol = kJacobiTol;
+  void* args[] = {&At, &Vt, &ld, &k, &max_sweeps, &tol, &bar, &sweeps, &status};
+  const int tok = profile_begin(s, QG_KERNEL_OTHER, 0.0, 0.0);
+  e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(jacobi_kernel), dim3(grid), dim3(256), args, 0, s);
+  profile_end(s, tok);
+  return e;
+}
+
+// CosSim of Pa, Pb (fp32 m x r, stride ld) into d_out: Ct = Pb^T Pa holds the
+// columns of C = Pa^T Pb as rows; one-sided Jacobi; mean of the column norms.
+cudaError_t cossim_core(const float* Pa, const float* Pb, int m, int r, int64_t ld, float* Ct, unsigned* bar,
+                        int* sweeps, float* d_out, uint32_t* status, cudaStream_t s) {
+  cudaError_t e = sgemm(true, false, Pb, ld, Pa, ld, Ct, r, r, r, m, s);
+  if (e != cudaSuccess) return e;
+  if ((e = jacobi(Ct, nullptr, r, r, bar, sweeps, status, s)) != cudaSuccess) return e;
+  mean_row_norm_kernel<<<1, 1024, 0, s>>>(Ct, r, r, d_out);
+  return cudaGetLastError();
+}
+
+qg_status st_of(cudaError_t e) { return e == cudaSuccess ? QG_OK : QG_ECUDA; }
+
+}  // namespace
+
+// ------------------------------------------------------------------ INT4 quantizer
 
 // One warp per group of 64 consecutive elements of the row-major m x r array:
 // scale = absmax / 7, code = clamp(rint(x * (7 / absmax)), -7, 7) (both IEEE
@@ -26,7 +357,7 @@ __global__ void quantize_int4_kernel(const float* __restrict__ P, int64_t ld, in
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
   // scale absmax / 7, codes rint(x * (7 / absmax)); absmax below 2^-120: zero group
-  const bool live = amax >= 7.52316384526264e-37f;
+  const bool live = amax >= kAbsmaxFloorR;
   const float s = live ? __fdiv_rn(amax, 7.0f) : 0.f;
   const float inv = live ? __fdiv_rn(7.0f, amax) : 0.f;
   int q[2] = {0, 0};
@@ -52,13 +383,106 @@ cudaError_t launch_quantize_projection(const float* P, int64_t ld, int32_t m, in
   return cudaGetLastError();
 }
 
-size_t refresh_scratch_bytes(int32_t, int32_t, int32_t, int32_t) { return 256; }
-size_t cossim_scratch_bytes(int32_t, int32_t) { return 256; }
+// ------------------------------------------------------------------ refresh
 
-qg_status run_refresh(const RefreshArgs&, uint8_t*, size_t, cudaStream_t, float*) { return QG_ESHAPE; }
+size_t refresh_scratch_bytes(int32_t m, int32_t n, int32_t r, int32_t oversample) {
+  return refresh_layout(m, n, r, oversample).total;
+}
 
-qg_status run_cossim(const float*, const float*, int32_t, int32_t, int64_t, float*, uint8_t*, cudaStream_t) {
-  return QG_ESHAPE;
+size_t cossim_scratch_bytes(int32_t, int32_t r) { return r256(size_t(r) * r * 4) + 256; }
+
+qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaStream_t s, float* cossim) {
+  const RefreshLayout L = refresh_layout(a.m, a.n, a.r, a.oversample);
+  if (ws_bytes < L.total) return QG_ESTATE;
+  const int m = a.m, n = a.n, r = a.r, k = L.k;
+  const int64_t ldk = L.ldk;
+  float* P = reinterpret_cast<float*>(ws + L.P);
+  uint16_t* Om = reinterpret_cast<uint16_t*>(ws + L.omega);
+  float* Y = reinterpret_cast<float*>(ws + L.Y);
+  uint16_t* Yb = reinterpret_cast<uint16_t*>(ws + L.Yb);
+  uint16_t* Ylo = reinterpret_cast<uint16_t*>(ws + L.Ylo);
+  float* Z = reinterpret_cast<float*>(ws + L.Z);
+  uint16_t* Zb = reinterpret_cast<uint16_t*>(ws + L.Zb);
+  float* gram = reinterpret_cast<float*>(ws + L.gram);
+  float* linv = reinterpret_cast<float*>(ws + L.linv);
+  float* Bm = reinterpret_cast<float*>(ws + L.Bm);
+  float* At = reinterpret_cast<float*>(ws + L.At);
+  float* Vt = reinterpret_cast<float*>(ws + L.Vt);
+  float* lam = reinterpret_cast<float*>(ws + L.lam);
+  int* perm = reinterpret_cast<int*>(ws + L.perm);
+  float* Vsel = reinterpret_cast<float*>(ws + L.Vsel);
+  Misc* misc = reinterpret_cast<Misc*>(ws + L.misc);
+  if (cudaMemsetAsync(misc, 0, sizeof(Misc), s) != cudaSuccess) return QG_ECUDA;
+
+  // Omega and the range finder
+  {
+    const int64_t cnt = int64_t(n) * ldk;
+    const PhiloxKey key{static_cast<uint32_t>(a.seed) ^ kOmegaSalt, static_cast<uint32_t>(a.seed >> 32)};
+    omega_kernel<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, s>>>(Om, ldk, n, k, a.refresh_idx, a.layer_id,
+                                                                          key);
+    if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
+  }
+  if (launch_gemm_f32(a.G, a.ldg, false, Om, ldk, false, Y, ldk, m, k, n, s) != cudaSuccess) return QG_ECUDA;
+  if (orth(Y, Yb, Ylo, m, k, ldk, gram, linv, &misc->chol_flag, s) != cudaSuccess) return QG_ECUDA;
+  for (int it = 0; it < a.power_iters; ++it) {
+    if (launch_gemm_f32(a.G, a.ldg, true, Yb, ldk, false, Z, ldk, n, k, m, s) != cudaSuccess) return QG_ECUDA;
+    if (orth(Z, Zb, nullptr, n, k, ldk, gram, linv, &misc->chol_flag, s) != cudaSuccess) return QG_ECUDA;
+    if (launch_gemm_f32(a.G, a.ldg, false, Zb, ldk, false, Y, ldk, m, k, n, s) != cudaSuccess) return QG_ECUDA;
+    if (orth(Y, Yb, Ylo, m, k, ldk, gram, linv, &misc->chol_flag, s) != cudaSuccess) return QG_ECUDA;
+  }
+  // Rayleigh-Ritz: B = Q^T G, S = B B^T, eigenpairs of S
+  // B = Q^T G with Q split into bf16 hi + lo parts (about 16 significant bits)
+  if (launch_gemm_f32(Yb, ldk, true, a.G, a.ldg, false, Bm, L.ldn4, k, n, m, s) != cudaSuccess) return QG_ECUDA;
+  if (launch_gemm_f32(Ylo, ldk, true, a.G, a.ldg, false, Bm, L.ldn4, k, n, m, s, true) != cudaSuccess)
+    return QG_ECUDA;
+  if (sgemm(false, true, Bm, L.ldn4, Bm, L.ldn4, At, ldk, k, k, n, s) != cudaSuccess) return QG_ECUDA;
+  {
+    const int64_t cnt = int64_t(k) * ldk;
+    identity_kernel<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, s>>>(Vt, ldk, k);
+    if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
+  }
+  if (jacobi(At, Vt, ldk, k, misc->bar, &misc->sweeps, a.status, s) != cudaSuccess) return QG_ECUDA;
+  row_norms_kernel<<<(k * 32 + 255) / 256, 256, 0, s>>>(At, ldk, k, k, lam);
+  if (cudaMemsetAsync(perm, 0, size_t(k) * sizeof(int), s) != cudaSuccess) return QG_ECUDA;
+  rank_sort_kernel<<<1, 1024, 0, s>>>(lam, k, perm);
+  gather_kernel<<<static_cast<unsigned>((int64_t(k) * r + 255) / 256), 256, 0, s>>>(Vt, ldk, perm, k, r, Vsel);
+  if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
+  // P = Q V[:, top r], sign-canonical, INT4
+  if (sgemm(false, false, Y, ldk, Vsel, r, P, r, m, r, k, s) != cudaSuccess) return QG_ECUDA;
+  canonical_signs_kernel<<<r, 256, 0, s>>>(P, m, r);
+  if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
+  const size_t mr = size_t(m) * r, pq = (mr + 1) / 2, ps = ((mr + 63) / 64) * 4;
+  if (a.has_prev) {
+    if (cudaMemcpyAsync(a.Pq_prev, a.Pq, pq, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return QG_ECUDA;
+    if (cudaMemcpyAsync(a.sP_prev, a.sP, ps, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return QG_ECUDA;
+  }
+  if (launch_quantize_projection(P, r, m, r, a.Pq, a.sP, s) != cudaSuccess) return QG_ECUDA;
+  // CosSim on the dequantized INT4 projections
+  *cossim = 0.f;
+  if (a.has_prev) {
+    float* Pa = reinterpret_cast<float*>(ws + L.Pa);
+    float* Pb = reinterpret_cast<float*>(ws + L.Pb);
+    float* Ct = reinterpret_cast<float*>(ws + L.Ct);
+    const unsigned blocks = static_cast<unsigned>((mr + 255) / 256);
+    dequant_f32_kernel<<<blocks, 256, 0, s>>>(a.Pq, a.sP, static_cast<int64_t>(mr), Pa);
+    dequant_f32_kernel<<<blocks, 256, 0, s>>>(a.Pq_prev, a.sP_prev, static_cast<int64_t>(mr), Pb);
+    if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
+    if (cossim_core(Pa, Pb, m, r, r, Ct, misc->bar, &misc->sweeps, &misc->cossim, a.status, s) != cudaSuccess)
+      return QG_ECUDA;
+    float host = 0.f;
+    if (cudaMemcpyAsync(&host, &misc->cossim, sizeof(float), cudaMemcpyDeviceToHost, s) != cudaSuccess) return QG_ECUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return QG_ECUDA;
+    *cossim = host;
+  }
+  return QG_OK;
+}
+
+qg_status run_cossim(const float* Pa, const float* Pb, int32_t m, int32_t r, int64_t ld, float* d_out, uint8_t* ws,
+                     cudaStream_t stream) {
+  float* Ct = reinterpret_cast<float*>(ws);
+  unsigned* bar = reinterpret_cast<unsigned*>(ws + r256(size_t(r) * r * 4));
+  int* sweeps = reinterpret_cast<int*>(bar + 4);
+  return st_of(cossim_core(Pa, Pb, m, r, ld, Ct, bar, sweeps, d_out, nullptr, stream));
 }
 
 }  // namespace qg

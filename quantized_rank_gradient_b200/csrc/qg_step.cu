@@ -309,6 +309,7 @@ struct StoreF32Epi {
   struct Args {
     float* D;
     int64_t ldd;
+    int32_t accumulate;  // D += A B instead of D = A B
   };
   static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
                            uint32_t* /*status*/) {
@@ -324,7 +325,11 @@ struct StoreF32Epi {
       if (!ok) continue;
       float* d = a.D + static_cast<int64_t>(grow) * a.ldd + j0 + c * 32;
       const int valid = ncols - c * 32;
-      if (valid >= 32) {
+      if (a.accumulate) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (e < valid) d[e] = __fadd_rn(d[e], __uint_as_float(v[e]));
+      } else if (valid >= 32) {
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           reinterpret_cast<float4*>(d)[q] =
@@ -558,7 +563,7 @@ cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream
 }
 
 cudaError_t launch_gemm_f32(const void* A, int64_t lda, bool a_trans, const void* B, int64_t ldb, bool b_trans,
-                            float* D, int64_t ldd, int M, int N, int K, cudaStream_t stream) {
+                            float* D, int64_t ldd, int M, int N, int K, cudaStream_t stream, bool accumulate) {
   GemmParams<StoreF32Epi> p;
   memset(&p, 0, sizeof(p));
   GemmProblem<StoreF32Epi>& pr = p.prob[0];
@@ -572,7 +577,7 @@ cudaError_t launch_gemm_f32(const void* A, int64_t lda, bool a_trans, const void
                            : encode_map_bf16(&pr.tmB, B, N, K, ldb, 64, 64);
   if (!okA || !okB) return cudaErrorInvalidValue;
   pr.status = nullptr;
-  pr.epi = StoreF32Epi::Args{D, ldd};
+  pr.epi = StoreF32Epi::Args{D, ldd, accumulate ? 1 : 0};
   add_problem(p, M, N, K);
   const double fl = 2.0 * M * N * K, by = 2.0 * M * K + 2.0 * K * N + 4.0 * M * N;
   if (a_trans && b_trans) return launch_gemm<StoreF32Epi, true, false>(p, stream, QG_KERNEL_OTHER, fl, by);

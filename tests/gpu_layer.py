@@ -102,6 +102,19 @@ class GpuLayer:
         ldN = round_up(n, 32)
         return self.ws[off: off + r * ldN * 2].view(torch.int16).view(r, ldN)[:, :n].cpu().numpy().view(np.uint16)
 
+    def refresh(self, G_dev: torch.Tensor, ldg: int, force=0):
+        """qg_refresh; returns (info, float32 projection from the workspace)."""
+        if not hasattr(self, "rws"):
+            self.rws = torch.zeros(qg.qg_refresh_workspace_bytes(byref(self.cfg)), dtype=torch.uint8,
+                                   device=self.device)
+        info = qg.qg_refresh_info()
+        qg.check(qg.qg_refresh(self.h, G_dev.data_ptr(), ldg, force, self.rws.data_ptr(), self.rws.numel(),
+                               byref(info), stream()), "qg_refresh")
+        torch.cuda.synchronize()
+        m, r = self.oc.m, self.oc.r
+        P = self.rws[: m * r * 4].view(torch.float32).view(m, r).cpu().numpy().copy()
+        return info, P
+
     def status(self):
         return qg.qg_layer_status(self.h, stream())
 

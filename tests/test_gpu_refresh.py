@@ -1,0 +1,171 @@
+"""GPU parity of the subspace refresh and of CosSim against the CPU oracle.
+
+Bars:
+  * CosSim (qg_cossim, identical float32 inputs): |gpu - oracle| <= 1e-4.
+  * Refreshed subspace: principal-angle cosines >= 0.999 between the GPU's
+    float32 projection and the oracle's, on every direction for inputs with a
+    singular-value gap after r, and on the signal-dominated leading directions
+    for noise-dominated inputs (the rest are reported, not gated: near-equal
+    noise singular values have no stable basis).
+  * The layer-adaptive schedule (refresh times, interval doubling) follows the
+    oracle's decisions.
+"""
+from ctypes import byref, c_void_p
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle as O
+import quantized_rank_gradient_b200 as qg
+import synth
+from gpu_layer import GpuLayer, stream, upload_gradient
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _cuda(cuda_ok):
+    torch.cuda.synchronize()
+    yield
+    torch.cuda.synchronize()
+
+
+def gpu_cossim(Pa, Pb):
+    m, r = Pa.shape
+    a = torch.from_numpy(np.ascontiguousarray(Pa, np.float32)).cuda()
+    b = torch.from_numpy(np.ascontiguousarray(Pb, np.float32)).cuda()
+    out = torch.zeros(1, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(qg.qg_cossim_workspace_bytes(m, r), dtype=torch.uint8, device="cuda")
+    qg.check(qg.qg_cossim(a.data_ptr(), b.data_ptr(), m, r, r, out.data_ptr(), ws.data_ptr(), ws.numel(), stream()))
+    return float(out.item())
+
+
+def test_cossim_closed_forms_and_oracle():
+    rng = np.random.default_rng(0)
+    m, r = 256, 32
+    P = np.linalg.qr(rng.standard_normal((m, r)))[0]
+    Orot = np.linalg.qr(rng.standard_normal((r, r)))[0]
+    assert abs(gpu_cossim(P, P) - 1) < 1e-4
+    assert abs(gpu_cossim(P, P @ Orot) - 1) < 1e-4
+    F = np.linalg.qr(rng.standard_normal((m, 2 * r)))[0]
+    assert abs(gpu_cossim(F[:, :r], F[:, r:])) < 1e-4
+    theta = np.linspace(0, 1.5, r)
+    A = np.zeros((m, r))
+    B = np.zeros((m, r))
+    A[np.arange(r), np.arange(r)] = 1
+    B[np.arange(r), np.arange(r)] = np.cos(theta)
+    B[r + np.arange(r), np.arange(r)] = np.sin(theta)
+    assert abs(gpu_cossim(A, B) - np.cos(theta).mean()) < 1e-4
+    for (mm, rr) in [(300, 64), (1376, 128), (4096, 1024)]:
+        X = np.linalg.qr(rng.standard_normal((mm, rr)))[0]
+        Y = np.linalg.qr(X + 0.7 * rng.standard_normal((mm, rr)) / np.sqrt(mm))[0]
+        assert abs(gpu_cossim(X, Y) - O.cossim(X.astype(np.float32), Y.astype(np.float32))) < 1e-4
+
+
+def principal_cosines(A, B):
+    return np.sort(np.cos(scipy.linalg.subspace_angles(np.asarray(A, np.float64), np.asarray(B, np.float64))))[::-1]
+
+
+def _refresh_pair(m, n, r, G_vals, G_bits, seed=3, layer_id=2):
+    oc = O.Config(m=m, n=n, r=r, seed=seed, layer_id=layer_id)
+    ost = O.LayerState.create(oc, np.zeros((m, n), np.int8), np.ones(-(-m * n // 256), np.float32))
+    oinfo = O.refresh(ost, G_vals, force=True)
+    gl = GpuLayer(oc, np.zeros((m, n), np.int8), np.ones(-(-m * n // 256), np.float32))
+    dG, ldg = upload_gradient(G_bits)
+    info, Pg = gl.refresh(dG, ldg, force=1)
+    return ost, oinfo, gl, info, Pg
+
+
+@pytest.mark.parametrize("m,n,r", [(256, 256, 32), (300, 250, 32), (1376, 512, 128), (512, 1376, 96)])
+def test_refresh_gap_input_matches_oracle_subspace(m, n, r):
+    G, Gb = synth.gap_gradient(m, n, r, seed=m + n)
+    ost, oinfo, gl, info, Pg = _refresh_pair(m, n, r, G, Gb)
+    assert info.refreshed == 1 and info.has_cossim == 0 and info.n_refresh == 1
+    Po = oinfo["P"]
+    cos = principal_cosines(Pg, Po)
+    assert cos.min() >= 0.999, cos.min()
+    # orthonormal, sorted, sign-canonical columns agree one by one; the sign
+    # rule (largest-magnitude entry positive) may only differ where the
+    # oracle's two largest magnitudes in the column are within 1e-3 of each
+    # other (a numerical tie between float32 and float64)
+    np.testing.assert_allclose(Pg.T @ Pg, np.eye(r), atol=2e-3)
+    col = np.sum(Pg.astype(np.float64) * Po, axis=0)
+    top2 = -np.sort(-np.abs(Po), axis=0)[:2]
+    tie = (top2[0] - top2[1]) / top2[0] < 1e-3
+    assert np.all((col > 0.99) | ((col < -0.99) & tie)), col.min()
+    assert np.all(np.abs(col) > 0.99)
+    # the GPU's own columns obey the rule
+    idx = np.argmax(np.abs(Pg), axis=0)
+    assert np.all(Pg[idx, np.arange(r)] > 0)
+    # the INT4 projection installed in the layer is the quantization of that P
+    Pq, sP = gl.projection()
+    ref_codes, ref_s = O.quant_int4_groups(Po.astype(np.float32))
+    got_codes = O.unpack_int4(Pq, m * r)
+    assert (got_codes == ref_codes).mean() > 0.98
+    np.testing.assert_allclose(sP, ref_s, rtol=2e-2)
+    assert gl.status() == qg.QG_OK
+
+
+def leading_block(sigma, edge, min_gap=0.05, margin=1.5):
+    """Largest j whose leading j singular values sit above margin * noise edge
+    and are separated from sigma_j by a relative gap >= min_gap."""
+    best = 0
+    for j in range(1, len(sigma)):
+        if sigma[j - 1] < margin * edge:
+            break
+        if (sigma[j - 1] - sigma[j]) / sigma[j - 1] >= min_gap:
+            best = j
+    return best
+
+
+@pytest.mark.parametrize("m,n,r,s0", [(256, 256, 32, 1e-2), (512, 512, 128, 1e-2), (1376, 512, 128, 3e-2)])
+def test_refresh_noise_dominated_leading_directions(m, n, r, s0):
+    gen = synth.lowrank_gradient(m, n, rank=min(256, m, n), s0=s0, decay=0.8, sigma=1e-4, seed=m)
+    G, Gb = gen.draw(0)
+    ost, oinfo, gl, info, Pg = _refresh_pair(m, n, r, G, Gb)
+    edge = 1e-4 * (np.sqrt(m) + np.sqrt(n))
+    k_sig = leading_block(np.linalg.svd(G.astype(np.float64), compute_uv=False), edge)
+    assert k_sig >= 1
+    Po = oinfo["P"]
+    cos = principal_cosines(Pg[:, :k_sig], Po[:, :k_sig])
+    assert cos.min() >= 0.999, (k_sig, cos.min())
+    np.testing.assert_allclose(Pg.T @ Pg, np.eye(r), atol=2e-3)
+
+
+def test_quantize_projection_bit_exact():
+    for (m, r) in [(256, 32), (300, 64), (4096, 1024)]:
+        P = synth.orthonormal(m, r, seed=r).astype(np.float32)
+        codes, s = O.quant_int4_groups(P)
+        dP = torch.from_numpy(P).cuda()
+        Pq = torch.zeros((m * r + 1) // 2, dtype=torch.uint8, device="cuda")
+        sP = torch.zeros(-(-m * r // 64), dtype=torch.float32, device="cuda")
+        qg.check(qg.qg_quantize_projection(dP.data_ptr(), r, m, r, Pq.data_ptr(), sP.data_ptr(), stream()))
+        np.testing.assert_array_equal(Pq.cpu().numpy(), O.pack_int4(codes))
+        np.testing.assert_array_equal(sP.cpu().numpy(), s)
+
+
+def test_schedule_follows_oracle_over_refreshes():
+    m, n, r = 256, 320, 32
+    oc = O.Config(m=m, n=n, r=r, delta0=2, gamma=0.4, seed=9, layer_id=1)
+    Wq, sW = synth.weight_codes(m, n, 9), synth.weight_scales(m, n, seed=9)
+    ost = O.LayerState.create(oc, Wq, sW)
+    gl = GpuLayer(oc, Wq, sW)
+    gen = synth.lowrank_gradient(m, n, rank=32, s0=1.0, decay=0.9, sigma=1e-3, seed=9)
+    trace = []
+    for t in range(9):
+        G, Gb = gen.draw(t)
+        dG, ldg = upload_gradient(Gb)
+        oi = O.refresh(ost, G, force=(t == 0))
+        info, _ = gl.refresh(dG, ldg, force=1 if t == 0 else 0)
+        assert bool(info.refreshed) == (oi is not None)
+        if oi is not None:
+            assert info.delta == ost.delta and info.t_next == ost.t_next and info.n_refresh == ost.n_refresh
+            if oi["cossim"] is not None:
+                assert abs(info.cossim - oi["cossim"]) < 2e-2
+                trace.append(info.cossim)
+        gl.step(dG, ldg)
+        O.step(ost, G)
+    assert len(trace) >= 2 and min(trace) > 0.4   # stable subspace -> intervals doubled
+    assert gl.sched().delta > 2
