@@ -72,6 +72,13 @@ struct AdamEpi {
     vv = __fadd_rn(__fmul_rn(a.beta2, v0), __fmul_rn(a.om2, __fmul_rn(R, R)));
   }
 
+  static QG_DEV void load_codes(const int8_t* mrow, const int8_t* vrow, int c, uint4 (&q)[4]) {
+    q[0] = *reinterpret_cast<const uint4*>(mrow + c * 32);
+    q[1] = *reinterpret_cast<const uint4*>(mrow + c * 32 + 16);
+    q[2] = *reinterpret_cast<const uint4*>(vrow + c * 32);
+    q[3] = *reinterpret_cast<const uint4*>(vrow + c * 32 + 16);
+  }
+
   // One thread owns row `row` of the 128 x 256 tile: rows are moment rows a,
   // the 256 columns are exactly one moment block (BN == 256 == block).
   static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
@@ -96,23 +103,23 @@ struct AdamEpi {
     bool bad = false;
 
     // pass 1: moments, block absmax of |m| and sqrt(v),
-    // N = -lr * m_hat / (sqrt(v_hat) + eps) = (m * c1) / (sqrt(v) * c2 + eps) -> bf16
+    // N = -lr * m_hat / (sqrt(v_hat) + eps) = (m * c1) / (sqrt(v) * c2 + eps) -> bf16.
+    // The codes of chunk c + 1 are loaded while chunk c is computed.
+    uint4 cur[4] = {}, nxt[4] = {};
+    if (row_ok) load_codes(mrow, vrow, 0, cur);
     for (int c = 0; c < nchunks; ++c) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(taddr + c * 32, v);
       tmem_ld_wait();
       if (!row_ok) continue;
-      const uint4 mq0 = *reinterpret_cast<const uint4*>(mrow + c * 32);
-      const uint4 mq1 = *reinterpret_cast<const uint4*>(mrow + c * 32 + 16);
-      const uint4 vq0 = *reinterpret_cast<const uint4*>(vrow + c * 32);
-      const uint4 vq1 = *reinterpret_cast<const uint4*>(vrow + c * 32 + 16);
+      if (c + 1 < nchunks) load_codes(mrow, vrow, c + 1, nxt);
       const int valid = ncols - c * 32;
       uint32_t packed[16];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const float R = __uint_as_float(v[e]);
-        const int8_t mc = e < 16 ? byte_of(mq0, e) : byte_of(mq1, e - 16);
-        const int8_t vc = e < 16 ? byte_of(vq0, e) : byte_of(vq1, e - 16);
+        const int8_t mc = e < 16 ? byte_of(cur[0], e) : byte_of(cur[1], e - 16);
+        const int8_t vc = e < 16 ? byte_of(cur[2], e) : byte_of(cur[3], e - 16);
         float mm, vv;
         moments(R, mc, vc, sm, sv, a, mm, vv);
         const float rv = __fsqrt_rn(vv);
@@ -132,6 +139,8 @@ struct AdamEpi {
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
     }
 
     // new block scales absmax / 127 and inverse scales 127 / absmax (IEEE
@@ -144,21 +153,19 @@ struct AdamEpi {
     const float inv_v = live_v ? __fdiv_rn(127.0f, amax_v) : 0.f;
 
     // pass 2: recompute the same moments bit for bit, re-quantize them
+    if (row_ok) load_codes(mrow, vrow, 0, cur);
     for (int c = 0; c < nchunks; ++c) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(taddr + c * 32, v);
       tmem_ld_wait();
       if (!row_ok) continue;
-      const uint4 mq0 = *reinterpret_cast<const uint4*>(mrow + c * 32);
-      const uint4 mq1 = *reinterpret_cast<const uint4*>(mrow + c * 32 + 16);
-      const uint4 vq0 = *reinterpret_cast<const uint4*>(vrow + c * 32);
-      const uint4 vq1 = *reinterpret_cast<const uint4*>(vrow + c * 32 + 16);
+      if (c + 1 < nchunks) load_codes(mrow, vrow, c + 1, nxt);
       uint32_t om[8], ov[8];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const float R = __uint_as_float(v[e]);
-        const int8_t mc = e < 16 ? byte_of(mq0, e) : byte_of(mq1, e - 16);
-        const int8_t vc = e < 16 ? byte_of(vq0, e) : byte_of(vq1, e - 16);
+        const int8_t mc = e < 16 ? byte_of(cur[0], e) : byte_of(cur[1], e - 16);
+        const int8_t vc = e < 16 ? byte_of(cur[2], e) : byte_of(cur[3], e - 16);
         float mm, vv;
         moments(R, mc, vc, sm, sv, a, mm, vv);
         int qm = 0, qv = 0;
@@ -178,6 +185,8 @@ struct AdamEpi {
       *reinterpret_cast<uint4*>(mrow + c * 32 + 16) = make_uint4(om[4], om[5], om[6], om[7]);
       *reinterpret_cast<uint4*>(vrow + c * 32) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
       *reinterpret_cast<uint4*>(vrow + c * 32 + 16) = make_uint4(ov[4], ov[5], ov[6], ov[7]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
     }
     if (row_ok) {
       a.sM[static_cast<int64_t>(arow) * a.nblk + nb] = s_m;
@@ -199,11 +208,6 @@ struct StochRoundEpi {
     PhiloxKey key;
     int32_t aligned4;  // n % 4 == 0: every 32-column chunk starts a Philox quad
   };
-
-  static QG_DEV float coef(const float* sW, int64_t g, float alpha) {
-    const float s = sW[g];
-    return s > 0.f ? __fdiv_rn(alpha, s) : 0.f;
-  }
 
   template <bool kAligned4>
   static QG_DEV void words(const Args& a, int64_t e0, uint32_t (&w)[32]) {
@@ -238,6 +242,24 @@ struct StochRoundEpi {
     }
   }
 
+  // Raw inputs of one 32-column chunk of a row: W codes and the scales of the
+  // (at most two) weight groups it touches.
+  struct ChunkIn {
+    uint4 q0, q1;
+    float s0, s1;
+  };
+
+  static QG_DEV void load_chunk(const Args& a, int N, int irow, int jc, ChunkIn& in) {
+    const int valid = min(32, N - jc);
+    const int64_t e0 = static_cast<int64_t>(irow) * N + jc;
+    const int64_t g0 = e0 >> 8, g1 = (e0 + valid - 1) >> 8;
+    const int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + jc;
+    in.q0 = *reinterpret_cast<const uint4*>(wrow);
+    in.q1 = valid > 16 ? *reinterpret_cast<const uint4*>(wrow + 16) : make_uint4(0, 0, 0, 0);
+    in.s0 = a.sW[g0];
+    in.s1 = g1 != g0 ? a.sW[g1] : in.s0;
+  }
+
   template <bool kAligned4>
   static QG_DEV void apply_impl(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr) {
     const int irow = mb * BM + row;
@@ -245,29 +267,29 @@ struct StochRoundEpi {
     const int j0 = nb * BN;
     const int ncols = min(BN, N - j0);
     const int nchunks = (ncols + 31) >> 5;
+    ChunkIn cur = {}, nxt = {};
+    if (row_ok) load_chunk(a, N, irow, j0, cur);
     for (int c = 0; c < nchunks; ++c) {
       uint32_t U[32];
       tmem_ld_32x32b_x32(taddr + c * 32, U);
       tmem_ld_wait();
       if (!row_ok) continue;
       const int jc = j0 + c * 32;
+      if (c + 1 < nchunks) load_chunk(a, N, irow, jc + 32, nxt);
       const int valid = min(32, N - jc);
       const int64_t e0 = static_cast<int64_t>(irow) * N + jc;
       const int64_t g0 = e0 >> 8;
       const int64_t g1 = (e0 + valid - 1) >> 8;
-      const float c0 = coef(a.sW, g0, a.alpha);
-      const float c1 = g1 != g0 ? coef(a.sW, g1, a.alpha) : c0;
+      const float c0 = cur.s0 > 0.f ? __fdiv_rn(a.alpha, cur.s0) : 0.f;
+      const float c1 = g1 != g0 ? (cur.s1 > 0.f ? __fdiv_rn(a.alpha, cur.s1) : 0.f) : c0;
       const int split = g1 != g0 ? static_cast<int>((g1 << 8) - e0) : 32;
       int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + jc;
-      uint4 q0 = make_uint4(0, 0, 0, 0), q1 = make_uint4(0, 0, 0, 0);
-      q0 = *reinterpret_cast<const uint4*>(wrow);
-      if (valid > 16) q1 = *reinterpret_cast<const uint4*>(wrow + 16);
       uint32_t w[32];
       words<kAligned4>(a, e0, w);
       uint32_t out[8];
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
-        const int8_t q = k < 16 ? byte_of(q0, k) : byte_of(q1, k - 16);
+        const int8_t q = k < 16 ? byte_of(cur.q0, k) : byte_of(cur.q1, k - 16);
         const float ck = k < split ? c0 : c1;
         const float x = __fmul_rn(__uint_as_float(U[k]), ck);
         const float y = __fadd_rn(static_cast<float>(q), x);
@@ -291,6 +313,7 @@ struct StochRoundEpi {
         for (int k = 0; k < 32; ++k)
           if (k < valid) wrow[k] = static_cast<int8_t>((out[k >> 2] >> (8 * (k & 3))) & 0xFFu);
       }
+      cur = nxt;
     }
   }
 
