@@ -325,32 +325,34 @@ def backproject(P_bf16, N_bf16) -> np.ndarray:
     return (np.asarray(P_bf16, np.float64) @ np.asarray(N_bf16, np.float64)).astype(np.float32)
 
 
-def sr_uniform24(m, n, seed, t, layer_id):
-    """The 24-bit uniform draw of every weight element (m x n uint32 in [0, 2^24)).
+def sr_uniform16(m, n, seed, t, layer_id):
+    """The 16-bit uniform draw of every weight element (m x n uint32 in [0, 2^16)).
 
-    Element e = i*n + j (logical index) takes word (e mod 4) of
-    Philox-4x32-10(counter = (e/4 low 32 bits, e/4 high 32 bits, t, layer_id),
-    key = (seed low 32 bits, seed high 32 bits)) and keeps its top 24 bits.
+    Element e = i*n + j (logical index) takes the 16-bit half (e mod 2) -- the low
+    half first -- of word ((e / 2) mod 4) of Philox-4x32-10(counter = (e/8 low 32
+    bits, e/8 high 32 bits, t, layer_id), key = (seed low 32 bits, seed high 32
+    bits)): one Philox call serves eight consecutive elements.
     """
     e = np.arange(m * n, dtype=np.uint64)
-    quad = e >> np.uint64(2)
-    w = philox4x32_10(quad & U32_MASK, quad >> np.uint64(32), t, layer_id,
+    call = e >> np.uint64(3)
+    w = philox4x32_10(call & U32_MASK, call >> np.uint64(32), t, layer_id,
                       seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
-    sel = (e & np.uint64(3)).astype(np.int64)
+    sel = ((e >> np.uint64(1)) & np.uint64(3)).astype(np.int64)
     words = np.stack(w, axis=0)[sel, np.arange(m * n)]
-    return (words >> np.uint32(8)).reshape(m, n)
+    shift = ((e & np.uint64(1)) * np.uint64(16)).astype(np.uint32)
+    return ((words >> shift) & np.uint32(0xFFFF)).reshape(m, n)
 
 
-def stochastic_round_update(Wq, sW, U, cfg: Config, t: int, u24=None):
+def stochastic_round_update(Wq, sW, U, cfg: Config, t: int, u16=None):
     """Step a5: W^Q <- W^Q + xi(alpha * U), in code units of the fixed weight grid.
 
     Readings: the weight scale is one float32 per 256 consecutive elements of
     the row-major m x n array (logical index), fixed after initialisation;
     c_g = alpha / s_g (IEEE float32; a zero scale freezes its group);
     x = U * c_g; y = q + x; f = floor(y); phi = y - f (exact);
-    xi rounds up iff u < phi with u = u24 * 2^-24 (compared as u24 < phi * 2^24,
-    exact); the result is clamped to [-127, 127]; a NaN y keeps the old code.
-    E[xi(y)] = y up to 2^-24 (the draw grid) away from the clamp."""
+    xi rounds up iff u < phi with u = u16 * 2^-16 (exact in float32); the result
+    is clamped to [-127, 127]; a NaN y keeps the old code.
+    E[xi(y)] = y up to 2^-16 (the draw grid) away from the clamp."""
     m, n = Wq.shape
     e = np.arange(m * n, dtype=np.int64).reshape(m, n)
     sW = np.asarray(sW, np.float32)
@@ -360,9 +362,9 @@ def stochastic_round_update(Wq, sW, U, cfg: Config, t: int, u24=None):
     with np.errstate(invalid="ignore"):
         f = np.floor(y)
         phi = (y - f).astype(np.float32)
-        if u24 is None:
-            u24 = sr_uniform24(m, n, cfg.seed, t, cfg.layer_id)
-        up = u24.astype(np.float32) < (phi * F32(2 ** 24))
+        if u16 is None:
+            u16 = sr_uniform16(m, n, cfg.seed, t, cfg.layer_id)
+        up = (u16.astype(np.float32) * F32(2.0 ** -16)) < phi
         qf = np.clip(f + up.astype(np.float32), -INT8_QMAX, INT8_QMAX)
     out = np.where(np.isnan(y), Wq, np.nan_to_num(qf).astype(np.int8))
     return out.astype(np.int8)

@@ -284,7 +284,7 @@ def test_sr_unbiased_over_a_million_draws(x):
     phi = float(np.float32(x)) - f
     mean = out.astype(np.float64).mean()
     sd = math.sqrt(max(phi * (1 - phi), 1e-12) / (m * n))
-    assert abs(mean - float(np.float32(x))) <= 5 * sd + 2 ** -24
+    assert abs(mean - float(np.float32(x))) <= 5 * sd + 2 ** -16
     assert set(np.unique(out).tolist()) <= {f, f + 1}
 
 
@@ -318,11 +318,20 @@ def test_sr_group_index_is_flattened_logical():
 
 
 def test_sr_uniform_draw_mapping():
-    u = O.sr_uniform24(3, 5, seed=77, t=2, layer_id=9)
-    for e in [0, 1, 4, 7, 14]:
+    u = O.sr_uniform16(3, 5, seed=77, t=2, layer_id=9)
+    for e in [0, 1, 2, 7, 8, 14]:
         i, j = divmod(e, 5)
-        w = O.philox_generic([e // 4, 0, 2, 9], [77, 0], **O.PHILOX4x32)[e % 4]
-        assert int(u[i, j]) == w >> 8
+        w = O.philox_generic([e // 8, 0, 2, 9], [77, 0], **O.PHILOX4x32)[(e // 2) % 4]
+        assert int(u[i, j]) == (w >> (16 * (e % 2))) & 0xFFFF
+    assert u.max() < 2 ** 16
+
+
+def test_sr_small_updates_keep_their_mean():
+    # an update far below one code (x = 1e-3) is kept on average, not rounded away
+    m, n = 1000, 1000
+    out = _sr(np.zeros((m, n), np.int8), np.ones(-(-m * n // 256), np.float32),
+              np.full((m, n), 1e-3, np.float32), seed=5)
+    assert abs(out.mean() - 1e-3) < 5 * np.sqrt(1e-3 / (m * n)) + 2 ** -16
 
 
 # ---------------------------------------------------------------- composed step
