@@ -5,10 +5,10 @@
 //
 //   warp 0      : TMA producer (one elected lane)
 //   warp 1      : TMEM allocator + MMA issuer (one elected lane)
-//   warps 2..9  : two epilogue warpgroups; warpgroup g drains TMEM buffer g, i.e.
-//                 every other tile of the CTA, so two tiles' epilogues overlap
-//                 each other and the MMAs.  Within a warpgroup each warp owns one
-//                 TMEM lane quarter (row = quarter*32 + lane).
+//   warps 2..9  : two epilogue warpgroups that share every tile, each taking
+//                 128 of its 256 columns; while they drain one TMEM buffer the
+//                 MMAs fill the other.  Within a warpgroup each warp owns one TMEM
+//                 lane quarter (row = quarter*32 + lane).
 //
 // A grid of at most one CTA per SM walks a flat list of tiles that spans up to
 // kMaxProblems independent problems (a batch of weight matrices).  Within a
@@ -57,6 +57,20 @@ struct TileRef {
   int prob, mb, nb;
 };
 
+// Both epilogue warpgroups work on every tile: warpgroup `half` takes the
+// tile's columns [128 half, 128 half + 128).  Row-wise reductions over the whole
+// tile width (the Adam block absmax) combine the two halves through `xchg`,
+// guarded by a per-lane-quarter mbarrier completing once per tile.
+struct EpiPair {
+  int half;
+  float2* xchg_mine;    // this warp's slot for its 32 rows
+  float2* xchg_other;   // the partner warp's slot (same rows, other half)
+  uint64_t* xbar;       // count 2: one arrival per partner warp
+  uint32_t xphase;
+  volatile int* abort;
+  uint32_t* status;
+};
+
 template <class Epi>
 QG_DEV TileRef locate_tile(const GemmParams<Epi>& p, int tile) {
   int pi = 0;
@@ -79,6 +93,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __shared__ __align__(8) uint64_t acc_full[2];
   __shared__ __align__(8) uint64_t acc_empty[2];
   __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ __align__(8) uint64_t xbar[4];
+  __shared__ float2 xchg[2][2][BM];  // [tile parity][half][row]
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -93,8 +109,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], 8);  // all 8 epilogue warps
     }
+    for (int q = 0; q < 4; ++q) mbar_init(&xbar[q], 2);
     mbar_init(&drain_bar, 1);
     abort_flag = 0;
     fence_barrier_init();
@@ -206,22 +223,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const uint32_t eg = static_cast<uint32_t>(warp - 2) >> 2;  // warpgroup = TMEM buffer
+    const int half = (warp - 2) >> 2;  // warpgroup: which 128 columns of every tile
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    uint32_t acc_phase = 0, it = 0;
+    uint32_t it = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++it) {
-      if ((it & 1u) != eg) continue;
+      const uint32_t buf = it & 1u, ph = (it >> 1) & 1u;
       const TileRef tr = locate_tile(p, tile);
       const GemmProblem<Epi>& pr = p.prob[tr.prob];
-      if (!mbar_wait(&acc_full[eg], acc_phase, &abort_flag, status)) break;
+      if (!mbar_wait(&acc_full[buf], ph, &abort_flag, status)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + eg * BN;
-      Epi::apply(pr.epi, pr.M, pr.N, tr.mb, tr.nb, row, taddr, pr.status);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * BN;
+      EpiPair ep{half, &xchg[it & 1u][half][quarter * 32], &xchg[it & 1u][half ^ 1][quarter * 32], &xbar[quarter],
+                 it & 1u, &abort_flag, pr.status};
+      Epi::apply(pr.epi, pr.M, pr.N, tr.mb, tr.nb, row, taddr, ep);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[eg]);
-      acc_phase ^= 1u;
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
   }
 
@@ -234,6 +252,219 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The same GEMM on CTA pairs (clusters of 2, tcgen05 cta_group::2): a 256 x 256
+// tile per pair, each CTA loading its 128 rows of A and 128 columns of B (half
+// the B traffic per SM of the one-CTA kernel), a 6-stage ring of 32 KiB per
+// CTA, one MMA issuer in the even CTA (M = 256, N = 256, K = 16), and each
+// CTA's TMEM holding its 128 rows of the accumulator, drained by its own two
+// epilogue warpgroups.  Loads of both CTAs complete on the even CTA's
+// full-barrier; the issuer's commits arrive on both CTAs' barriers; epilogues
+// of both CTAs release an accumulator buffer on the even CTA's barrier.
+// B must be MN-major here (64-column boxes).
+// ---------------------------------------------------------------------------
+
+constexpr int kStagesPair = 6;
+constexpr int kHalfStageBytes = 128 * BK * 2;  // 16 KiB: 128 rows of A or 128 columns of B
+constexpr size_t kGemmPairSmemBytes = size_t(kStagesPair) * 2 * kHalfStageBytes + 1024;
+
+template <class Epi, bool kAMN, bool kBMN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_pair_kernel(const __grid_constant__ GemmParams<Epi> p) {
+  static_assert(kBMN, "the pair kernel loads B in 64-column boxes");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStagesPair * kHalfStageBytes;
+
+  __shared__ __align__(8) uint64_t full_bar[kStagesPair];
+  __shared__ __align__(8) uint64_t empty_bar[kStagesPair];
+  __shared__ __align__(8) uint64_t acc_full[2];
+  __shared__ __align__(8) uint64_t acc_empty[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ __align__(8) uint64_t xbar[4];
+  __shared__ float2 xchg[2][2][BM];  // [tile parity][half][row]
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int cluster = blockIdx.x >> 1;
+  const int nclusters = gridDim.x >> 1;
+  uint32_t* const status = nullptr;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStagesPair; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 16);  // 8 epilogue warps x 2 CTAs (used in the even CTA)
+    }
+    for (int q = 0; q < 4; ++q) mbar_init(&xbar[q], 2);
+    mbar_init(&drain_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < p.nprob; ++i) {
+      tma_prefetch_map(&p.prob[i].tmA);
+      tma_prefetch_map(&p.prob[i].tmB);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&tmem_base_sh, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_sh;
+
+  // tiles are 256 x 256 here: 128-row block index of this CTA = 2 * pair block + rank
+  auto pair_tiles = [&](const GemmProblem<Epi>& pr) { return ((pr.M + 255) / 256) * pr.tiles_n; };
+  auto locate = [&](int tile, int& pi, int& mb2, int& nb) {
+    pi = 0;
+    int begin = 0;
+    while (pi + 1 < p.nprob && tile >= begin + pair_tiles(p.prob[pi])) {
+      begin += pair_tiles(p.prob[pi]);
+      ++pi;
+    }
+    const int local = tile - begin;
+    const int tm = (p.prob[pi].M + 255) / 256;
+    mb2 = local % tm;
+    nb = local / tm;
+  };
+  int total = 0;
+  for (int i = 0; i < p.nprob; ++i) total += pair_tiles(p.prob[i]);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, armed = 0, armed_parity = 0;
+      bool ok = true;
+      for (int tile = cluster; ok && tile < total; tile += nclusters) {
+        int pi, mb2, nb;
+        locate(tile, pi, mb2, nb);
+        const GemmProblem<Epi>& pr = p.prob[pi];
+        const int nkb = (pr.K + BK - 1) / BK;
+        const int row0 = mb2 * 256 + static_cast<int>(rank) * 128;
+        const int col0 = nb * BN + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 4 * kHalfStageBytes);
+          const uint32_t fb = mapa_shared(&full_bar[stage], 0);
+          uint8_t* a_dst = sA + stage * kHalfStageBytes;
+          uint8_t* b_dst = sB + stage * kHalfStageBytes;
+          if (kAMN) {
+            tma_load_2d_pair(a_dst, &pr.tmA, fb, row0, kb * BK);
+            tma_load_2d_pair(a_dst + 8192, &pr.tmA, fb, row0 + 64, kb * BK);
+          } else {
+            tma_load_2d_pair(a_dst, &pr.tmA, fb, kb * BK, row0);
+          }
+          tma_load_2d_pair(b_dst, &pr.tmB, fb, col0, kb * BK);
+          tma_load_2d_pair(b_dst + 8192, &pr.tmB, fb, col0 + 64, kb * BK);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStagesPair) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (abort_flag && rank == 0) {
+        for (int s = 0; s < kStagesPair; ++s)
+          if (armed & (1u << s)) mbar_wait_drain(&full_bar[s], (armed_parity >> s) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(256, 256, kAMN, kBMN);
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = cluster; ok && tile < total; tile += nclusters) {
+        int pi, mb2, nb;
+        locate(tile, pi, mb2, nb);
+        const GemmProblem<Epi>& pr = p.prob[pi];
+        const int nkb = (pr.K + BK - 1) / BK;
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, &abort_flag, status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * kHalfStageBytes);
+          const uint32_t b_base = smem_u32(sB + stage * kHalfStageBytes);
+          const int kleft = pr.K - kb * BK;
+          const int ksteps = kleft >= BK ? BK / 16 : (kleft + 15) / 16;
+          for (int kk = 0; kk < ksteps; ++kk) {
+            const uint64_t ad = kAMN ? sdesc_sw128(a_base + kk * 2048, 8192, 1024)
+                                     : sdesc_sw128(a_base + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b_base + kk * 2048, 8192, 1024);
+            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair_mc(&empty_bar[stage], 0x3);
+          if (++stage == kStagesPair) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair_mc(&acc_full[acc], 0x3);
+        acc ^= 1u;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (abort_flag) {
+        umma_commit_pair(&drain_bar);
+        mbar_wait_drain(&drain_bar, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int half = (warp - 2) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    uint32_t it = 0;
+    for (int tile = cluster; tile < total; tile += nclusters, ++it) {
+      const uint32_t buf = it & 1u, ph = (it >> 1) & 1u;
+      int pi, mb2, nb;
+      locate(tile, pi, mb2, nb);
+      const GemmProblem<Epi>& pr = p.prob[pi];
+      if (!mbar_wait(&acc_full[buf], ph, &abort_flag, status)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * BN;
+      EpiPair ep{half, &xchg[it & 1u][half][quarter * 32], &xchg[it & 1u][half ^ 1][quarter * 32], &xbar[quarter],
+                 it & 1u, &abort_flag, pr.status};
+      Epi::apply(pr.epi, pr.M, pr.N, mb2 * 2 + static_cast<int>(rank), nb, row, taddr, ep);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(&acc_empty[buf], 0));
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && abort_flag) {
+    for (int i = 0; i < p.nprob; ++i)
+      if (p.prob[i].status) atomicOr(p.prob[i].status, kErrTimeout);
+  }
+  cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 

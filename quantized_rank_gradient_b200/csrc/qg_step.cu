@@ -37,13 +37,50 @@ constexpr float kAbsmaxFloor = 7.52316384526264e-37f;  // 2^-120
 
 // ------------------------------------------------------------------ helpers
 
-QG_DEV int8_t byte_of(const uint4& v, int k) {
-  const uint32_t w = k < 4 ? v.x : k < 8 ? v.y : k < 12 ? v.z : v.w;
-  return static_cast<int8_t>((w >> (8 * (k & 3))) & 0xFFu);
-}
+QG_DEV uint32_t word_of(const uint4& v, int k) { return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w; }
 
 QG_DEV uint16_t bf16_bits_rn(float x) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+QG_DEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Conversions between small integers and float32 done with integer/FP-add
+// arithmetic (exact for |value| < 2^22) instead of the conversion pipe.
+// 12582912 = 1.5 * 2^23: a float in [2^23, 2^24) has an integer ulp of 1.
+constexpr float kMagic = 12582912.0f;
+constexpr uint32_t kMagicBits = 0x4B400000u;
+
+// Byte k (0..3) of w as a signed int8, converted to float exactly (k is a
+// constant after unrolling, so the selector is an immediate).
+QG_DEV float sbyte_f32(uint32_t w, int k) {
+  const uint32_t sel = k | ((k | 8) << 4) | ((k | 8) << 8) | ((k | 8) << 12);  // sign-extend byte k
+  const uint32_t sx = prmt(w, 0u, sel);
+  return __fsub_rn(__uint_as_float(kMagicBits + sx), kMagic);
+}
+
+// Code e (0..31) of a 32-byte chunk held in two uint4, as float.
+QG_DEV float code_f32(const uint4& lo, const uint4& hi, int e) {
+  return sbyte_f32(word_of(e < 16 ? lo : hi, (e >> 2) & 3), e & 3);
+}
+
+// 16-bit draw h (0: low half, 1: high half) of w as u = u16 * 2^-16, exact.
+QG_DEV float draw_u(uint32_t w, int h) {
+  const uint32_t m = h ? ((w >> 9) & 0x007FFF80u) : ((w << 7) & 0x007FFF80u);
+  return __fsub_rn(__uint_as_float(0x3F800000u | m), 1.0f);
+}
+
+// x (integer-valued or not, already clamped to [-127, 127]) rounded to the
+// nearest integer, ties to even, returned in the low byte.
+QG_DEV uint32_t round_to_byte(float x) { return __float_as_uint(__fadd_rn(x, kMagic)); }
+
+// Low bytes of four words packed into one word.
+QG_DEV uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  return prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
 }
 
 // ------------------------------------------------------------------ a2 + a3 epilogue
@@ -63,10 +100,10 @@ struct AdamEpi {
 
   // m = b1*m0 + (1-b1)*R ; v = b2*v0 + (1-b2)*(R*R), one rounding per operation.
   // M^Q holds m on a linear grid; V^Q holds sqrt(v), so v0 = (code*scale)^2.
-  static QG_DEV void moments(float R, int8_t mc, int8_t vc, float sm, float sv, const Args& a,
-                             float& mm, float& vv) {
-    const float m0 = __fmul_rn(static_cast<float>(mc), sm);
-    const float d0 = __fmul_rn(static_cast<float>(vc), sv);
+  static QG_DEV void moments(float R, float mc, float vc, float sm, float sv, const Args& a, float& mm,
+                             float& vv) {
+    const float m0 = __fmul_rn(mc, sm);
+    const float d0 = __fmul_rn(vc, sv);
     const float v0 = __fmul_rn(d0, d0);
     mm = __fadd_rn(__fmul_rn(a.beta1, m0), __fmul_rn(a.om1, R));
     vv = __fadd_rn(__fmul_rn(a.beta2, v0), __fmul_rn(a.om2, __fmul_rn(R, R)));
@@ -79,15 +116,74 @@ struct AdamEpi {
     q[3] = *reinterpret_cast<const uint4*>(vrow + c * 32 + 16);
   }
 
-  // One thread owns row `row` of the 128 x 256 tile: rows are moment rows a,
-  // the 256 columns are exactly one moment block (BN == 256 == block).
+  // Pass 1 on one 32-column chunk: the new moments and the running block maxima of
+  // |m| and of v (max over the block of sqrt(v) is sqrt of the max of v, the
+  // correctly rounded square root being monotone).
+  static QG_DEV void pass1_chunk(const Args& a, const uint32_t (&v)[32], const uint4 (&cq)[4], float sm, float sv,
+                                 int valid, float& amax_m, float& amax_vv, bool& bad) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float R = __uint_as_float(v[e]);
+      float mm, vv;
+      moments(R, code_f32(cq[0], cq[1], e), code_f32(cq[2], cq[3], e), sm, sv, a, mm, vv);
+      if (e < valid) {
+        amax_m = fmaxf(amax_m, fabsf(mm));
+        amax_vv = fmaxf(amax_vv, vv);
+        bad |= !isfinite(R);
+      }
+    }
+  }
+
+  // Pass 2 on one chunk: the same moments; N = -lr m_hat / (sqrt(v_hat) + eps)
+  // = (m c1) / (sqrt(v) c2 + eps) -> bf16; codes of m and sqrt(v) on the block's
+  // new grids.
+  static QG_DEV void pass2_chunk(const Args& a, const uint32_t (&v)[32], const uint4 (&cq)[4], float sm, float sv,
+                                 bool live_m, bool live_v, float inv_m, float inv_v, uint16_t* nptr, int8_t* mptr,
+                                 int8_t* vptr) {
+    uint32_t om[8], ov[8], packed[16], bm[4], bv[4];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float R = __uint_as_float(v[e]);
+      float mm, vv;
+      moments(R, code_f32(cq[0], cq[1], e), code_f32(cq[2], cq[3], e), sm, sv, a, mm, vv);
+      const float rv = __fsqrt_rn(vv);
+      const float upd = __fdiv_rn(__fmul_rn(mm, a.c1), __fadd_rn(__fmul_rn(rv, a.c2), a.eps));
+      const uint32_t b = bf16_bits_rn(upd);
+      if (e & 1)
+        packed[e >> 1] |= b << 16;
+      else
+        packed[e >> 1] = b;
+      // rint then clamp to integer bounds == clamp then rint (ties to even)
+      bm[e & 3] = live_m ? round_to_byte(fminf(fmaxf(__fmul_rn(mm, inv_m), -127.f), 127.f)) : 0u;
+      bv[e & 3] = live_v ? round_to_byte(fminf(fmaxf(__fmul_rn(rv, inv_v), 0.f), 127.f)) : 0u;
+      if ((e & 3) == 3) {
+        om[e >> 2] = pack4(bm[0], bm[1], bm[2], bm[3]);
+        ov[e >> 2] = pack4(bv[0], bv[1], bv[2], bv[3]);
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(nptr);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+    *reinterpret_cast<uint4*>(mptr) = make_uint4(om[0], om[1], om[2], om[3]);
+    *reinterpret_cast<uint4*>(mptr + 16) = make_uint4(om[4], om[5], om[6], om[7]);
+    *reinterpret_cast<uint4*>(vptr) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+    *reinterpret_cast<uint4*>(vptr + 16) = make_uint4(ov[4], ov[5], ov[6], ov[7]);
+  }
+
+  // One thread owns row `row` of its warpgroup's 128-column half of the
+  // 128 x 256 tile; the tile's 256 columns are exactly one moment block, so the
+  // block maxima of the two halves are combined with the partner warp before
+  // the codes are formed.  Codes of chunk c + 1 are loaded while chunk c is
+  // computed.
   static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
-                           uint32_t* status) {
+                           const EpiPair& ep) {
     const int arow = mb * BM + row;
     const bool row_ok = arow < M;
     const int j0 = nb * BN;
     const int ncols = min(BN, N - j0);
-    const int nchunks = (ncols + 31) >> 5;
+    const int c0 = ep.half * 4;
+    const int c1 = min(c0 + 4, (ncols + 31) >> 5);
     float sm = 0.f, sv = 0.f;
     int8_t* mrow = nullptr;
     int8_t* vrow = nullptr;
@@ -99,49 +195,42 @@ struct AdamEpi {
       vrow = a.Vq + static_cast<int64_t>(arow) * a.ld_mom + j0;
       nrow = a.Nout + static_cast<int64_t>(arow) * a.ldN + j0;
     }
-    float amax_m = 0.f, amax_v = 0.f;
+    float amax_m = 0.f, amax_vv = 0.f;
     bool bad = false;
+    uint4 qa[4] = {}, qb[4] = {};
 
-    // pass 1: moments, block absmax of |m| and sqrt(v),
-    // N = -lr * m_hat / (sqrt(v_hat) + eps) = (m * c1) / (sqrt(v) * c2 + eps) -> bf16.
-    // The codes of chunk c + 1 are loaded while chunk c is computed.
-    uint4 cur[4] = {}, nxt[4] = {};
-    if (row_ok) load_codes(mrow, vrow, 0, cur);
-    for (int c = 0; c < nchunks; ++c) {
+    if (row_ok && c0 < c1) load_codes(mrow, vrow, c0, qa);
+#pragma unroll 1
+    for (int c = c0; c < c1; c += 2) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(taddr + c * 32, v);
       tmem_ld_wait();
-      if (!row_ok) continue;
-      if (c + 1 < nchunks) load_codes(mrow, vrow, c + 1, nxt);
-      const int valid = ncols - c * 32;
-      uint32_t packed[16];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float R = __uint_as_float(v[e]);
-        const int8_t mc = e < 16 ? byte_of(cur[0], e) : byte_of(cur[1], e - 16);
-        const int8_t vc = e < 16 ? byte_of(cur[2], e) : byte_of(cur[3], e - 16);
-        float mm, vv;
-        moments(R, mc, vc, sm, sv, a, mm, vv);
-        const float rv = __fsqrt_rn(vv);
-        if (e < valid) {
-          amax_m = fmaxf(amax_m, fabsf(mm));
-          amax_v = fmaxf(amax_v, rv);
-          bad |= !isfinite(R);
-        }
-        const float upd = __fdiv_rn(__fmul_rn(mm, a.c1), __fadd_rn(__fmul_rn(rv, a.c2), a.eps));
-        const uint32_t b = bf16_bits_rn(upd);
-        if (e & 1)
-          packed[e >> 1] |= b << 16;
-        else
-          packed[e >> 1] = b;
+      if (row_ok) {
+        if (c + 1 < c1) load_codes(mrow, vrow, c + 1, qb);
+        pass1_chunk(a, v, qa, sm, sv, ncols - c * 32, amax_m, amax_vv, bad);
       }
-      uint4* dst = reinterpret_cast<uint4*>(nrow + c * 32);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
+      if (c + 1 < c1) {
+        tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v);
+        tmem_ld_wait();
+        if (row_ok) {
+          if (c + 2 < c1) load_codes(mrow, vrow, c + 2, qa);
+          pass1_chunk(a, v, qb, sm, sv, ncols - (c + 1) * 32, amax_m, amax_vv, bad);
+        }
+      }
     }
+
+    // block maxima over both halves (the partner warp owns the same rows)
+    const int lane = row & 31;
+    ep.xchg_mine[lane] = make_float2(amax_m, amax_vv);
+    __threadfence_block();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(ep.xbar);
+    if (mbar_wait(ep.xbar, ep.xphase, ep.abort, ep.status)) {
+      const float2 o = ep.xchg_other[lane];
+      amax_m = fmaxf(amax_m, o.x);
+      amax_vv = fmaxf(amax_vv, o.y);
+    }
+    const float amax_v = __fsqrt_rn(amax_vv);
 
     // new block scales absmax / 127 and inverse scales 127 / absmax (IEEE
     // divisions, once per block); a block whose absmax is below 2^-120 is a zero
@@ -152,47 +241,31 @@ struct AdamEpi {
     const float inv_m = live_m ? __fdiv_rn(127.0f, amax_m) : 0.f;
     const float inv_v = live_v ? __fdiv_rn(127.0f, amax_v) : 0.f;
 
-    // pass 2: recompute the same moments bit for bit, re-quantize them
-    if (row_ok) load_codes(mrow, vrow, 0, cur);
-    for (int c = 0; c < nchunks; ++c) {
+    if (row_ok && c0 < c1) load_codes(mrow, vrow, c0, qa);
+#pragma unroll 1
+    for (int c = c0; c < c1; c += 2) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(taddr + c * 32, v);
       tmem_ld_wait();
-      if (!row_ok) continue;
-      if (c + 1 < nchunks) load_codes(mrow, vrow, c + 1, nxt);
-      uint32_t om[8], ov[8];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float R = __uint_as_float(v[e]);
-        const int8_t mc = e < 16 ? byte_of(cur[0], e) : byte_of(cur[1], e - 16);
-        const int8_t vc = e < 16 ? byte_of(cur[2], e) : byte_of(cur[3], e - 16);
-        float mm, vv;
-        moments(R, mc, vc, sm, sv, a, mm, vv);
-        int qm = 0, qv = 0;
-        if (live_m) qm = static_cast<int>(fminf(fmaxf(rintf(__fmul_rn(mm, inv_m)), -127.f), 127.f));
-        if (live_v) qv = static_cast<int>(fminf(fmaxf(rintf(__fmul_rn(__fsqrt_rn(vv), inv_v)), 0.f), 127.f));
-        const uint32_t bm = static_cast<uint32_t>(qm) & 0xFFu;
-        const uint32_t bv = static_cast<uint32_t>(qv) & 0xFFu;
-        if ((e & 3) == 0) {
-          om[e >> 2] = bm;
-          ov[e >> 2] = bv;
-        } else {
-          om[e >> 2] |= bm << (8 * (e & 3));
-          ov[e >> 2] |= bv << (8 * (e & 3));
+      if (row_ok) {
+        if (c + 1 < c1) load_codes(mrow, vrow, c + 1, qb);
+        pass2_chunk(a, v, qa, sm, sv, live_m, live_v, inv_m, inv_v, nrow + c * 32, mrow + c * 32, vrow + c * 32);
+      }
+      if (c + 1 < c1) {
+        tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v);
+        tmem_ld_wait();
+        if (row_ok) {
+          if (c + 2 < c1) load_codes(mrow, vrow, c + 2, qa);
+          pass2_chunk(a, v, qb, sm, sv, live_m, live_v, inv_m, inv_v, nrow + (c + 1) * 32, mrow + (c + 1) * 32,
+                      vrow + (c + 1) * 32);
         }
       }
-      *reinterpret_cast<uint4*>(mrow + c * 32) = make_uint4(om[0], om[1], om[2], om[3]);
-      *reinterpret_cast<uint4*>(mrow + c * 32 + 16) = make_uint4(om[4], om[5], om[6], om[7]);
-      *reinterpret_cast<uint4*>(vrow + c * 32) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
-      *reinterpret_cast<uint4*>(vrow + c * 32 + 16) = make_uint4(ov[4], ov[5], ov[6], ov[7]);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
     }
-    if (row_ok) {
+    if (row_ok && ep.half == 0) {
       a.sM[static_cast<int64_t>(arow) * a.nblk + nb] = s_m;
       a.sV[static_cast<int64_t>(arow) * a.nblk + nb] = s_v;
     }
-    if (bad && status) atomicOr(status, kErrNonFinite);
+    if (bad && ep.status) atomicOr(ep.status, kErrNonFinite);
   }
 };
 
@@ -206,39 +279,58 @@ struct StochRoundEpi {
     float alpha;
     uint32_t t, layer_id;
     PhiloxKey key;
-    int32_t aligned4;  // n % 4 == 0: every 32-column chunk starts a Philox quad
+    int32_t aligned8;  // n % 8 == 0: every 32-column chunk starts a Philox call
   };
 
-  template <bool kAligned4>
-  static QG_DEV void words(const Args& a, int64_t e0, uint32_t (&w)[32]) {
-    const uint64_t qb = static_cast<uint64_t>(e0) >> 2;
-    if (kAligned4) {
+  // The 16-bit draws of elements e0 .. e0+31: element i's draw is half (i & 1)
+  // of d[i >> 1].  Element e takes half (e mod 2) of word ((e / 2) mod 4) of
+  // Philox-4x32-10(counter = (e / 8, t, layer_id), key = seed).
+  template <bool kAligned8>
+  static QG_DEV void draws(const Args& a, int64_t e0, uint32_t (&d)[16]) {
+    const uint64_t cb = static_cast<uint64_t>(e0) >> 3;
+    if (kAligned8) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < 4; ++k) {
         uint32_t o[4];
-        const uint64_t q = qb + k;
-        philox4x32_10(static_cast<uint32_t>(q), static_cast<uint32_t>(q >> 32), a.t, a.layer_id, a.key, o);
-        w[4 * k] = o[0];
-        w[4 * k + 1] = o[1];
-        w[4 * k + 2] = o[2];
-        w[4 * k + 3] = o[3];
+        const uint64_t c = cb + k;
+        philox4x32_10(static_cast<uint32_t>(c), static_cast<uint32_t>(c >> 32), a.t, a.layer_id, a.key, o);
+        d[4 * k] = o[0];
+        d[4 * k + 1] = o[1];
+        d[4 * k + 2] = o[2];
+        d[4 * k + 3] = o[3];
       }
     } else {
-      uint32_t ww[36];
+      // chunk starts at draw s = e0 mod 8 of call cb: five calls cover it
+      uint32_t dd[20];
 #pragma unroll
-      for (int k = 0; k < 9; ++k) {
+      for (int k = 0; k < 5; ++k) {
         uint32_t o[4];
-        const uint64_t q = qb + k;
-        philox4x32_10(static_cast<uint32_t>(q), static_cast<uint32_t>(q >> 32), a.t, a.layer_id, a.key, o);
-        ww[4 * k] = o[0];
-        ww[4 * k + 1] = o[1];
-        ww[4 * k + 2] = o[2];
-        ww[4 * k + 3] = o[3];
+        const uint64_t c = cb + k;
+        philox4x32_10(static_cast<uint32_t>(c), static_cast<uint32_t>(c >> 32), a.t, a.layer_id, a.key, o);
+        dd[4 * k] = o[0];
+        dd[4 * k + 1] = o[1];
+        dd[4 * k + 2] = o[2];
+        dd[4 * k + 3] = o[3];
       }
-      const int s = static_cast<int>(e0 & 3);
+      const int s = static_cast<int>(e0 & 7);
+      // draw j of the calls is half (j & 1) of dd[j >> 1]; element i needs draw s + i
 #pragma unroll
-      for (int k = 0; k < 32; ++k)
-        w[k] = s == 0 ? ww[k] : s == 1 ? ww[k + 1] : s == 2 ? ww[k + 2] : ww[k + 3];
+      for (int w = 0; w < 16; ++w) {
+        uint32_t lohi[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int i = 2 * w + h;
+          uint32_t val = 0;
+#pragma unroll
+          for (int ss = 0; ss < 8; ++ss) {
+            const int j = ss + i;
+            const uint32_t x = (dd[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+            val = (s == ss) ? x : val;
+          }
+          lohi[h] = val;
+        }
+        d[w] = lohi[0] | (lohi[1] << 16);
+      }
     }
   }
 
@@ -260,69 +352,85 @@ struct StochRoundEpi {
     in.s1 = g1 != g0 ? a.sW[g1] : in.s0;
   }
 
-  template <bool kAligned4>
-  static QG_DEV void apply_impl(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr) {
+  // One 32-column chunk of row irow: W codes from `in`, U from TMEM, updated
+  // codes written back.  y = q + U c_g; round up iff u < y - floor(y); clamp to
+  // [-127, 127]; a NaN y keeps the old code.
+  template <bool kAligned8>
+  static QG_DEV void sr_chunk(const Args& a, int N, int irow, int jc, const uint32_t (&U)[32], const ChunkIn& in) {
+    const int valid = min(32, N - jc);
+    const int64_t e0 = static_cast<int64_t>(irow) * N + jc;
+    const int64_t g0 = e0 >> 8;
+    const int64_t g1 = (e0 + valid - 1) >> 8;
+    const float c0 = in.s0 > 0.f ? __fdiv_rn(a.alpha, in.s0) : 0.f;
+    const float c1 = g1 != g0 ? (in.s1 > 0.f ? __fdiv_rn(a.alpha, in.s1) : 0.f) : c0;
+    const int split = g1 != g0 ? static_cast<int>((g1 << 8) - e0) : 32;
+    int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + jc;
+    uint32_t d[16];
+    draws<kAligned8>(a, e0, d);
+    uint32_t out[8], bytes[4];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const float q = code_f32(in.q0, in.q1, k);
+      const float ck = k < split ? c0 : c1;
+      const float x = __fmul_rn(__uint_as_float(U[k]), ck);
+      const float y = __fadd_rn(q, x);
+      const float f = floorf(y);
+      const float phi = __fsub_rn(y, f);
+      const bool up = draw_u(d[k >> 1], k & 1) < phi;
+      float qf = up ? __fadd_rn(f, 1.0f) : f;
+      qf = fminf(fmaxf(qf, -127.0f), 127.0f);
+      bytes[k & 3] = round_to_byte((y != y) ? q : qf);
+      if ((k & 3) == 3) out[k >> 2] = pack4(bytes[0], bytes[1], bytes[2], bytes[3]);
+    }
+    if (valid == 32) {
+      *reinterpret_cast<uint4*>(wrow) = make_uint4(out[0], out[1], out[2], out[3]);
+      *reinterpret_cast<uint4*>(wrow + 16) = make_uint4(out[4], out[5], out[6], out[7]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        if (k < valid) wrow[k] = static_cast<int8_t>((out[k >> 2] >> (8 * (k & 3))) & 0xFFu);
+    }
+  }
+
+  // This warpgroup's half of the tile's columns, in chunk pairs: the inputs of
+  // chunk c + 1 are loaded while chunk c is computed, the two input buffers
+  // alternating without copies.
+  template <bool kAligned8>
+  static QG_DEV void apply_impl(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr, int half) {
     const int irow = mb * BM + row;
     const bool row_ok = irow < M;
     const int j0 = nb * BN;
     const int ncols = min(BN, N - j0);
-    const int nchunks = (ncols + 31) >> 5;
-    ChunkIn cur = {}, nxt = {};
-    if (row_ok) load_chunk(a, N, irow, j0, cur);
-    for (int c = 0; c < nchunks; ++c) {
+    const int c0 = half * 4;
+    const int c1 = min(c0 + 4, (ncols + 31) >> 5);
+    ChunkIn ia = {}, ib = {};
+    if (row_ok && c0 < c1) load_chunk(a, N, irow, j0 + c0 * 32, ia);
+#pragma unroll 1
+    for (int c = c0; c < c1; c += 2) {
       uint32_t U[32];
       tmem_ld_32x32b_x32(taddr + c * 32, U);
       tmem_ld_wait();
-      if (!row_ok) continue;
-      const int jc = j0 + c * 32;
-      if (c + 1 < nchunks) load_chunk(a, N, irow, jc + 32, nxt);
-      const int valid = min(32, N - jc);
-      const int64_t e0 = static_cast<int64_t>(irow) * N + jc;
-      const int64_t g0 = e0 >> 8;
-      const int64_t g1 = (e0 + valid - 1) >> 8;
-      const float c0 = cur.s0 > 0.f ? __fdiv_rn(a.alpha, cur.s0) : 0.f;
-      const float c1 = g1 != g0 ? (cur.s1 > 0.f ? __fdiv_rn(a.alpha, cur.s1) : 0.f) : c0;
-      const int split = g1 != g0 ? static_cast<int>((g1 << 8) - e0) : 32;
-      int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + jc;
-      uint32_t w[32];
-      words<kAligned4>(a, e0, w);
-      uint32_t out[8];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const int8_t q = k < 16 ? byte_of(cur.q0, k) : byte_of(cur.q1, k - 16);
-        const float ck = k < split ? c0 : c1;
-        const float x = __fmul_rn(__uint_as_float(U[k]), ck);
-        const float y = __fadd_rn(static_cast<float>(q), x);
-        const float f = floorf(y);
-        const float phi = __fsub_rn(y, f);
-        const bool up = __uint2float_rn(w[k] >> 8) < __fmul_rn(phi, 16777216.0f);
-        float qf = __fadd_rn(f, up ? 1.0f : 0.0f);
-        qf = fminf(fmaxf(qf, -127.0f), 127.0f);
-        const int res = (y != y) ? static_cast<int>(q) : static_cast<int>(qf);
-        const uint32_t b = static_cast<uint32_t>(res) & 0xFFu;
-        if ((k & 3) == 0)
-          out[k >> 2] = b;
-        else
-          out[k >> 2] |= b << (8 * (k & 3));
+      if (row_ok) {
+        if (c + 1 < c1) load_chunk(a, N, irow, j0 + (c + 1) * 32, ib);
+        sr_chunk<kAligned8>(a, N, irow, j0 + c * 32, U, ia);
       }
-      if (valid == 32) {
-        *reinterpret_cast<uint4*>(wrow) = make_uint4(out[0], out[1], out[2], out[3]);
-        *reinterpret_cast<uint4*>(wrow + 16) = make_uint4(out[4], out[5], out[6], out[7]);
-      } else {
-#pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (k < valid) wrow[k] = static_cast<int8_t>((out[k >> 2] >> (8 * (k & 3))) & 0xFFu);
+      if (c + 1 < c1) {
+        tmem_ld_32x32b_x32(taddr + (c + 1) * 32, U);
+        tmem_ld_wait();
+        if (row_ok) {
+          if (c + 2 < c1) load_chunk(a, N, irow, j0 + (c + 2) * 32, ia);
+          sr_chunk<kAligned8>(a, N, irow, j0 + (c + 1) * 32, U, ib);
+        }
       }
-      cur = nxt;
     }
   }
 
   static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
-                           uint32_t* /*status*/) {
-    if (a.aligned4)
-      apply_impl<true>(a, M, N, mb, nb, row, taddr);
+                           const EpiPair& ep) {
+    if (a.aligned8)
+      apply_impl<true>(a, M, N, mb, nb, row, taddr, ep.half);
     else
-      apply_impl<false>(a, M, N, mb, nb, row, taddr);
+      apply_impl<false>(a, M, N, mb, nb, row, taddr, ep.half);
   }
 };
 
@@ -335,13 +443,14 @@ struct StoreF32Epi {
     int32_t accumulate;  // D += A B instead of D = A B
   };
   static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
-                           uint32_t* /*status*/) {
+                           const EpiPair& ep) {
     const int grow = mb * BM + row;
     const bool ok = grow < M;
     const int j0 = nb * BN;
     const int ncols = min(BN, N - j0);
-    const int nchunks = (ncols + 31) >> 5;
-    for (int c = 0; c < nchunks; ++c) {
+    const int c0 = ep.half * 4;
+    const int c1 = min(c0 + 4, (ncols + 31) >> 5);
+    for (int c = c0; c < c1; ++c) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(taddr + c * 32, v);
       tmem_ld_wait();
@@ -475,6 +584,28 @@ static cudaError_t launch_gemm(const GemmParams<Epi>& p, cudaStream_t stream, in
   return cudaGetLastError();
 }
 
+// The same GEMMs on CTA pairs (256 x 256 tiles, cta_group::2).
+template <class Epi, bool kAMN>
+static cudaError_t launch_gemm_pair(const GemmParams<Epi>& p, cudaStream_t stream, int kind, double flops,
+                                    double bytes) {
+  auto kern = gemm_tc_pair_kernel<Epi, kAMN, true>;
+  static bool attr_set = false;  // per instantiation
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kGemmPairSmemBytes));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  int pair_tiles = 0;
+  for (int i = 0; i < p.nprob; ++i) pair_tiles += ((p.prob[i].M + 255) / 256) * p.prob[i].tiles_n;
+  if (pair_tiles == 0) return cudaSuccess;
+  const int clusters = std::min(pair_tiles, std::max(1, sm_count() / 2));
+  const int tok = profile_begin(stream, kind, flops, bytes);
+  kern<<<2 * clusters, kGemmThreads, kGemmPairSmemBytes, stream>>>(p);
+  profile_end(stream, tok);
+  return cudaGetLastError();
+}
+
 template <class Epi>
 static void add_problem(GemmParams<Epi>& p, int M, int N, int K) {
   GemmProblem<Epi>& pr = p.prob[p.nprob];
@@ -561,7 +692,7 @@ cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream
                              s.beta1, s.beta2, s.om1, s.om2, s.c1, s.c2, s.eps};
       add_problem(p1, s.r, s.n, s.m);
     }
-    e = launch_gemm<AdamEpi, true, true>(p1, stream, QG_KERNEL_PROJECT_ADAM, fl1, by1);
+    e = launch_gemm_pair<AdamEpi, true>(p1, stream, QG_KERNEL_PROJECT_ADAM, fl1, by1);
     if (e != cudaSuccess) return e;
 
     GemmParams<StochRoundEpi> p2;
@@ -576,10 +707,10 @@ cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream
       pr.status = s.status;
       pr.epi = StochRoundEpi::Args{s.W, s.sW, s.ldw, s.alpha, s.t, s.layer_id,
                                    PhiloxKey{static_cast<uint32_t>(s.seed), static_cast<uint32_t>(s.seed >> 32)},
-                                   (s.n % 4) == 0 ? 1 : 0};
+                                   (s.n % 8) == 0 ? 1 : 0};
       add_problem(p2, s.m, s.n, s.r);
     }
-    e = launch_gemm<StochRoundEpi, false, true>(p2, stream, QG_KERNEL_BACKPROJECT_SR, fl2, by2);
+    e = launch_gemm_pair<StochRoundEpi, false>(p2, stream, QG_KERNEL_BACKPROJECT_SR, fl2, by2);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
