@@ -255,6 +255,21 @@ qg_status qg_gemm_bf16(const void* d_A, int64_t lda, int32_t a_trans, const void
                        int32_t b_trans, float* d_D, int64_t ldd, int32_t M, int32_t N, int32_t K,
                        void* stream);
 
+/* Self-check of the branch-free correctly rounded float32 reciprocal, square
+ * root and division that the Adam epilogue uses in place of the IEEE
+ * intrinsics (the update of the AIMech Q-GaLore page, "INT8 optimizer states":
+ * one square root and one division per element).
+ *   op 0: reciprocal, every float in [2^-100, 2^100];
+ *   op 1: square root, every float in [2^-100, 2^100] and +-0;
+ *   op 2: division, n Philox-drawn pairs (seeded by `seed`) with b > 0 in
+ *         [2^-100, 2^100], |a| in [2^-90, 2^90] or +-0, quotient in range.
+ * d_out: 3 device uint64; [0] mismatches against __frcp_rn / __fsqrt_rn /
+ * __fdiv_rn, [1] operands tested, [2] smallest failing (a bits << 32 | b bits)
+ * (all ones if none).  Asynchronous on `stream`; QG_EINVAL for a bad op or a
+ * null d_out. */
+qg_status qg_selfcheck_exact_math(int32_t op, uint64_t n, uint64_t seed, unsigned long long* d_out,
+                                  void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -87,6 +87,7 @@ _SIGNATURES = {
     "qg_dequant_projection": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p]),
     "qg_gemm_bf16": (c_int32, [c_void_p, c_int64, c_int32, c_void_p, c_int64, c_int32, c_void_p, c_int64, c_int32,
                                c_int32, c_int32, c_void_p]),
+    "qg_selfcheck_exact_math": (c_int32, [c_int32, c_uint64, c_uint64, c_void_p, c_void_p]),
 }
 
 _lib = None

@@ -21,6 +21,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "qg_exact.cuh"
 #include "qg_gemm.cuh"
 #include "qg_internal.h"
 #include "qg_philox.cuh"
@@ -118,9 +119,12 @@ struct AdamEpi {
 
   // Pass 1 on one 32-column chunk: the new moments and the running block maxima of
   // |m| and of v (max over the block of sqrt(v) is sqrt of the max of v, the
-  // correctly rounded square root being monotone).
+  // correctly rounded square root being monotone).  It also keeps the smallest
+  // nonzero |m| and v as (bits << 1) - 1, zero mapping to all ones, which decide
+  // whether pass 2 may use the branch-free square root and division.
   static QG_DEV void pass1_chunk(const Args& a, const uint32_t (&v)[32], const uint4 (&cq)[4], float sm, float sv,
-                                 int valid, float& amax_m, float& amax_vv, bool& bad) {
+                                 int valid, float& amax_m, float& amax_vv, uint32_t& mmin_b, uint32_t& vmin_b,
+                                 bool& bad) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const float R = __uint_as_float(v[e]);
@@ -129,14 +133,39 @@ struct AdamEpi {
       if (e < valid) {
         amax_m = fmaxf(amax_m, fabsf(mm));
         amax_vv = fmaxf(amax_vv, vv);
+        mmin_b = min(mmin_b, (__float_as_uint(mm) << 1) - 1u);
+        vmin_b = min(vmin_b, (__float_as_uint(vv) << 1) - 1u);
         bad |= !isfinite(R);
       }
     }
   }
 
+  // True when every square root and division of this thread's pass 2 has its
+  // operands and quotient inside the ranges where sqrt_exact and div_exact equal
+  // the IEEE operations: v in {0} U [2^-100, 2^100], the denominator
+  // sqrt(v) c2 + eps in [eps, dmax] within [2^-100, 2^100], the numerator m c1
+  // zero or in [2^-90, 2^90], and every nonzero quotient in [2^-100, 2^100].
+  static QG_DEV bool exact_fast_ok(const Args& a, float amax_m, float amax_vv, uint32_t mmin_b, uint32_t vmin_b,
+                                   bool bad) {
+    const float c1a = fabsf(a.c1);
+    bool ok = !bad && a.eps >= kSafeLo && amax_vv <= kSafeHi && a.c2 > 0.f;
+    if (vmin_b != 0xffffffffu) ok = ok && __uint_as_float((vmin_b + 1u) >> 1) >= kSafeLo;
+    const float dmax = __fadd_rn(__fmul_rn(__fsqrt_rn(amax_vv), a.c2), a.eps);
+    const float nmax = __fmul_rn(amax_m, c1a);
+    ok = ok && dmax <= kSafeHi && nmax <= kSafeDivHi && nmax <= __fmul_rn(kSafeHi, a.eps);
+    if (mmin_b != 0xffffffffu) {
+      const float nmin = __fmul_rn(__uint_as_float((mmin_b + 1u) >> 1), c1a);
+      ok = ok && nmin >= kSafeDivLo && nmin >= __fmul_rn(kSafeLo, dmax);
+    }
+    return ok;
+  }
+
   // Pass 2 on one chunk: the same moments; N = -lr m_hat / (sqrt(v_hat) + eps)
   // = (m c1) / (sqrt(v) c2 + eps) -> bf16; codes of m and sqrt(v) on the block's
   // new grids.
+  // kExact selects sqrt_exact / div_exact, equal to the IEEE operations on the
+  // ranges exact_fast_ok checks, over the intrinsics.
+  template <bool kExact>
   static QG_DEV void pass2_chunk(const Args& a, const uint32_t (&v)[32], const uint4 (&cq)[4], float sm, float sv,
                                  bool live_m, bool live_v, float inv_m, float inv_v, uint16_t* nptr, int8_t* mptr,
                                  int8_t* vptr) {
@@ -146,8 +175,9 @@ struct AdamEpi {
       const float R = __uint_as_float(v[e]);
       float mm, vv;
       moments(R, code_f32(cq[0], cq[1], e), code_f32(cq[2], cq[3], e), sm, sv, a, mm, vv);
-      const float rv = __fsqrt_rn(vv);
-      const float upd = __fdiv_rn(__fmul_rn(mm, a.c1), __fadd_rn(__fmul_rn(rv, a.c2), a.eps));
+      const float rv = kExact ? sqrt_exact(vv) : __fsqrt_rn(vv);
+      const float num = __fmul_rn(mm, a.c1), den = __fadd_rn(__fmul_rn(rv, a.c2), a.eps);
+      const float upd = kExact ? div_exact(num, den) : __fdiv_rn(num, den);
       const uint32_t b = bf16_bits_rn(upd);
       if (e & 1)
         packed[e >> 1] |= b << 16;
@@ -196,6 +226,7 @@ struct AdamEpi {
       nrow = a.Nout + static_cast<int64_t>(arow) * a.ldN + j0;
     }
     float amax_m = 0.f, amax_vv = 0.f;
+    uint32_t mmin_b = 0xffffffffu, vmin_b = 0xffffffffu;
     bool bad = false;
     uint4 qa[4] = {}, qb[4] = {};
 
@@ -207,17 +238,19 @@ struct AdamEpi {
       tmem_ld_wait();
       if (row_ok) {
         if (c + 1 < c1) load_codes(mrow, vrow, c + 1, qb);
-        pass1_chunk(a, v, qa, sm, sv, ncols - c * 32, amax_m, amax_vv, bad);
+        pass1_chunk(a, v, qa, sm, sv, ncols - c * 32, amax_m, amax_vv, mmin_b, vmin_b, bad);
       }
       if (c + 1 < c1) {
         tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v);
         tmem_ld_wait();
         if (row_ok) {
           if (c + 2 < c1) load_codes(mrow, vrow, c + 2, qa);
-          pass1_chunk(a, v, qb, sm, sv, ncols - (c + 1) * 32, amax_m, amax_vv, bad);
+          pass1_chunk(a, v, qb, sm, sv, ncols - (c + 1) * 32, amax_m, amax_vv, mmin_b, vmin_b, bad);
         }
       }
     }
+
+    const bool exact = exact_fast_ok(a, amax_m, amax_vv, mmin_b, vmin_b, bad);
 
     // block maxima over both halves (the partner warp owns the same rows)
     const int lane = row & 31;
@@ -249,15 +282,24 @@ struct AdamEpi {
       tmem_ld_wait();
       if (row_ok) {
         if (c + 1 < c1) load_codes(mrow, vrow, c + 1, qb);
-        pass2_chunk(a, v, qa, sm, sv, live_m, live_v, inv_m, inv_v, nrow + c * 32, mrow + c * 32, vrow + c * 32);
+        if (exact)
+          pass2_chunk<true>(a, v, qa, sm, sv, live_m, live_v, inv_m, inv_v, nrow + c * 32, mrow + c * 32,
+                            vrow + c * 32);
+        else
+          pass2_chunk<false>(a, v, qa, sm, sv, live_m, live_v, inv_m, inv_v, nrow + c * 32, mrow + c * 32,
+                             vrow + c * 32);
       }
       if (c + 1 < c1) {
         tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v);
         tmem_ld_wait();
         if (row_ok) {
           if (c + 2 < c1) load_codes(mrow, vrow, c + 2, qa);
-          pass2_chunk(a, v, qb, sm, sv, live_m, live_v, inv_m, inv_v, nrow + (c + 1) * 32, mrow + (c + 1) * 32,
-                      vrow + (c + 1) * 32);
+          if (exact)
+            pass2_chunk<true>(a, v, qb, sm, sv, live_m, live_v, inv_m, inv_v, nrow + (c + 1) * 32,
+                              mrow + (c + 1) * 32, vrow + (c + 1) * 32);
+          else
+            pass2_chunk<false>(a, v, qb, sm, sv, live_m, live_v, inv_m, inv_v, nrow + (c + 1) * 32,
+                               mrow + (c + 1) * 32, vrow + (c + 1) * 32);
         }
       }
     }
