@@ -55,6 +55,38 @@ def stack_shapes(layers):
     return [per for _ in range(layers)]
 
 
+KERNEL_SOURCES = ["qg_step.cu", "qg_gemm.cuh", "qg_device.cuh", "qg_philox.cuh", "qg_exact.cuh"]
+PROFILE = os.path.join(ROOT, "profiles", "step_kernels_llama7b_layer_ncu.md")
+
+
+def kernel_digest():
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "quantized_rank_gradient_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary of one
+    decoder layer (one launch = one layer batch, as here), or None when the
+    kernel sources changed since that capture."""
+    try:
+        text = open(PROFILE).read()
+    except OSError:
+        return None
+    digest = traffic = None
+    for line in text.splitlines():
+        if line.startswith("kernel sources digest:"):
+            digest = line.split(":", 1)[1].strip()
+        if line.startswith("traffic_per_launch_bytes:"):
+            traffic = dict(kv.split("=") for kv in line.split(":", 1)[1].split())
+    if digest != kernel_digest() or not traffic or kernel not in traffic:
+        return None
+    return int(traffic[kernel])
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -332,7 +364,9 @@ def run_ours(args, rank, world, local_rank):
                           "peaks": "burst bf16 %.1f TF/s, HBM %.1f GB/s (%s)" % (peaks["bf16_tflops"], peaks["hbm_gbs"],
                                                                               peaks["source"])},
         "roofline": {"bound": "tensor", "kernel": names[dom_k], "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": profiled_traffic(names[dom_k]) if args.layers == 32 else None,
+                     "traffic_unit": "bytes per launch (ncu, one decoder layer)",
+                     "algorithmic_bytes_per_launch": dom.bytes / dom.launches,
                      "peak_kind": "sustained bf16 (%s)" % peaks["source"]},
         "kernels": kernels,
         "gpu_launches": launches * args.steps,
