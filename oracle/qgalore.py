@@ -346,28 +346,35 @@ def sr_uniform16(m, n, seed, t, layer_id):
 def stochastic_round_update(Wq, sW, U, cfg: Config, t: int, u16=None):
     """Step a5: W^Q <- W^Q + xi(alpha * U), in code units of the fixed weight grid.
 
-    Readings: the weight scale is one float32 per 256 consecutive elements of
-    the row-major m x n array (logical index), fixed after initialisation;
-    c_g = alpha / s_g (IEEE float32; a zero scale freezes its group);
-    x = U * c_g; y = q + x; f = floor(y); phi = y - f (exact);
-    xi rounds up iff u < phi with u = u16 * 2^-16 (exact in float32); the result
-    is clamped to [-127, 127]; a NaN y keeps the old code.
-    E[xi(y)] = y up to 2^-16 (the draw grid) away from the clamp."""
+    [QG-quant] asks only that xi be an unbiased stochastic rounding; the form is
+    a reading.  The weight scale is one float32 per 256 consecutive elements of
+    the row-major m x n array (logical index), fixed after initialisation.  The
+    update is carried in fixed point with 16 fraction bits:
+      c'_g = (alpha / s_g) * 2^16   (IEEE float32 division, exact scaling; a zero
+                                     scale gives c'_g = 0 and freezes its group)
+      X    = U * c'_g               (float32: the update in units of 2^-16 code)
+      K    = ceil(X)                (an integer)
+      r    = floor((K + d) / 2^16)  (d = the element's 16-bit uniform draw)
+      W'   = clamp(W + r, -127, 127);  a NaN X keeps the old code.
+    Adding a uniform 16-bit integer and dropping the 16 fraction bits rounds
+    K / 2^16 up with probability equal to its fractional part, so
+    E[r] = K / 2^16, which lies in [X / 2^16, X / 2^16 + 2^-16): unbiased up to
+    the 2^-16 grid of the draws.  |X| is clipped to 2^30 before the ceiling,
+    which changes no clamped result (|r| >= 2^14 saturates either way)."""
     m, n = Wq.shape
     e = np.arange(m * n, dtype=np.int64).reshape(m, n)
     sW = np.asarray(sW, np.float32)
     c = np.where(sW > 0, F32(cfg.alpha) / np.where(sW > 0, sW, F32(1)), F32(0)).astype(np.float32)
-    x = (np.asarray(U, np.float32) * c[e // cfg.w_group]).astype(np.float32)
-    y = (Wq.astype(np.float32) + x).astype(np.float32)
-    with np.errstate(invalid="ignore"):
-        f = np.floor(y)
-        phi = (y - f).astype(np.float32)
-        if u16 is None:
-            u16 = sr_uniform16(m, n, cfg.seed, t, cfg.layer_id)
-        up = (u16.astype(np.float32) * F32(2.0 ** -16)) < phi
-        qf = np.clip(f + up.astype(np.float32), -INT8_QMAX, INT8_QMAX)
-    out = np.where(np.isnan(y), Wq, np.nan_to_num(qf).astype(np.int8))
-    return out.astype(np.int8)
+    with np.errstate(over="ignore", invalid="ignore"):
+        cp = (c * F32(65536.0)).astype(np.float32)
+        X = (np.asarray(U, np.float32) * cp[e // cfg.w_group]).astype(np.float32)
+        nan = np.isnan(X)
+        K = np.ceil(np.clip(np.where(nan, F32(0), X), F32(-2.0 ** 30), F32(2.0 ** 30))).astype(np.int64)
+    if u16 is None:
+        u16 = sr_uniform16(m, n, cfg.seed, t, cfg.layer_id)
+    r = (K + np.asarray(u16, np.int64)) >> 16          # floor division by 2^16
+    out = np.clip(Wq.astype(np.int64) + r, -INT8_QMAX, INT8_QMAX)
+    return np.where(nan, Wq, out).astype(np.int8)
 
 
 @dataclass

@@ -317,6 +317,39 @@ def test_sr_group_index_is_flattened_logical():
     assert np.all(np.abs(out - expect) < 1.0)
 
 
+@pytest.mark.parametrize("X", [0.0, 1.0, 0.25, 0.5, 32767.5, 65535.25, 65536.0, 98304.75, -0.5, -1.0,
+                               -65536.0, -70000.1, 3.0e6, -3.0e6 + 0.5])
+def test_sr_exhaustive_over_the_draw_space(X):
+    # alpha = 1, s_g = 2^16: c' = 1, so the update in units of 2^-16 code is X itself.
+    # Over all 2^16 draws the rounded result takes only the two neighbouring codes,
+    # and the draws sum to ceil(X) exactly: the mean is ceil(X) / 2^16, the value
+    # on the draw grid nearest above X (a floor, a missing draw or an off-by-one
+    # in the shift changes the sum).
+    W = np.zeros((256, 256), np.int8)
+    sW = np.full(256, 65536.0, np.float32)
+    U = np.full((256, 256), X, np.float32)
+    cfg = O.Config(m=256, n=256, r=1, alpha=1.0)
+    out = O.stochastic_round_update(W, sW, U, cfg, 1, u16=np.arange(65536, dtype=np.uint32).reshape(256, 256))
+    Xf = float(np.float32(X))
+    lo = math.floor(Xf / 65536.0)
+    assert set(np.unique(out).tolist()) <= {lo, lo + 1}
+    assert int(out.astype(np.int64).sum()) == math.ceil(Xf)
+
+
+def test_sr_nan_keeps_code_inf_and_huge_saturate():
+    W = np.array([[5, -5, 100, -100, 0, 7, -7, 3]], np.int8)
+    sW = np.ones(1, np.float32)
+    U = np.array([[np.nan, np.nan, np.inf, -np.inf, 1e30, -1e30, 2.0 ** 31, 0.0]], np.float32)
+    out = O.stochastic_round_update(W, sW, U, O.Config(m=1, n=8, r=1, alpha=1.0), 1,
+                                    u16=np.full((1, 8), 12345, np.uint32))
+    np.testing.assert_array_equal(out, [[5, -5, 127, -127, 127, -127, 127, 3]])
+    # an overflowing alpha / s (c' = inf): a zero update stays a NaN -> kept; nonzero saturates
+    tiny = np.full(1, 1e-38, np.float32)
+    out = O.stochastic_round_update(np.array([[4, 4]], np.int8), tiny, np.array([[0.0, 1e-3]], np.float32),
+                                    O.Config(m=1, n=2, r=1, alpha=1.0), 1, u16=np.zeros((1, 2), np.uint32))
+    np.testing.assert_array_equal(out, [[4, 127]])
+
+
 def test_sr_uniform_draw_mapping():
     u = O.sr_uniform16(3, 5, seed=77, t=2, layer_id=9)
     for e in [0, 1, 2, 7, 8, 14]:
