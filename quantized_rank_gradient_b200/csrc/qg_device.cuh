@@ -105,6 +105,11 @@ QG_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, i
       : "memory");
 }
 
+// Orders this thread's earlier generic-proxy shared-memory accesses (and, after a
+// barrier, those of the threads it synchronised with) before its later
+// async-proxy (TMA) accesses to shared memory.
+QG_DEV void fence_proxy_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // ------------------------------------------------------------------ tcgen05
 
 QG_DEV void tmem_alloc(uint32_t* smem_result, uint32_t ncols) {
@@ -182,8 +187,11 @@ QG_DEV void cluster_sync() {
 }
 
 // Arrive on an mbarrier of another CTA of the cluster (shared::cluster address).
+// Release at CTA scope: the arrival orders this thread's tcgen05 and shared-memory
+// work (the callers fence their TMEM loads first) but does not wait for its
+// global stores to become visible across the cluster, which nothing here needs.
 QG_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // Tile load into this CTA's shared memory whose completion is counted on an

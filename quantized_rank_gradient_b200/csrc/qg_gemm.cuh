@@ -40,6 +40,7 @@ template <class Epi>
 struct GemmProblem {
   CUtensorMap tmA;  // K-major A: box {64 (K), 128 (M)}; MN-major A: box {64 (M), 64 (K)}
   CUtensorMap tmB;  // MN-major B: box {64 (N), 64 (K)}; K-major B: box {64 (K), 256 (N)}
+  CUtensorMap tmS[2];  // side operands of the epilogue (int8 tiles staged in shared memory)
   int32_t M, N, K;
   int32_t tiles_m, tiles_n, tile_begin;
   uint32_t* status;  // the matrix's device status word (may be null)
@@ -83,6 +84,7 @@ QG_DEV TileRef locate_tile(const GemmParams<Epi>& p, int tile) {
 template <class Epi, bool kAMN, bool kBMN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ GemmParams<Epi> p) {
+  static_assert(Epi::kSideBytes == 0, "the one-CTA kernel stages no side operands");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -236,7 +238,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * BN;
       EpiPair ep{half, &xchg[it & 1u][half][quarter * 32], &xchg[it & 1u][half ^ 1][quarter * 32], &xbar[quarter],
                  it & 1u, &abort_flag, pr.status};
-      Epi::apply(pr.epi, pr.M, pr.N, tr.mb, tr.nb, row, taddr, ep);
+      Epi::apply(pr.epi, pr.M, pr.N, tr.mb, tr.nb, row, taddr, ep, nullptr);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
@@ -258,35 +260,65 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // ---------------------------------------------------------------------------
 // The same GEMM on CTA pairs (clusters of 2, tcgen05 cta_group::2): a 256 x 256
 // tile per pair, each CTA loading its 128 rows of A and 128 columns of B (half
-// the B traffic per SM of the one-CTA kernel), a 6-stage ring of 32 KiB per
+// the B traffic per SM of the one-CTA kernel), a ring of 32 KiB stages per
 // CTA, one MMA issuer in the even CTA (M = 256, N = 256, K = 16), and each
 // CTA's TMEM holding its 128 rows of the accumulator, drained by its own two
 // epilogue warpgroups.  Loads of both CTAs complete on the even CTA's
 // full-barrier; the issuer's commits arrive on both CTAs' barriers; epilogues
 // of both CTAs release an accumulator buffer on the even CTA's barrier.
 // B must be MN-major here (64-column boxes).
+//
+// Side operands.  An epilogue may declare Epi::kSideBytes > 0: int8 tiles that
+// belong to the output tile (the weight codes, the moment codes) are then
+// staged in shared memory by TMA, Epi::kSideBufs buffers deep, so that the
+// epilogue reads them at shared-memory latency.  One epilogue thread issues the
+// loads of tile j + kSideBufs - 1 when the epilogue starts tile j, after every
+// epilogue warp has released that buffer (side_empty, one arrival per warp);
+// the loads complete on side_full.
 // ---------------------------------------------------------------------------
 
-constexpr int kStagesPair = 6;
 constexpr int kHalfStageBytes = 128 * BK * 2;  // 16 KiB: 128 rows of A or 128 columns of B
-constexpr size_t kGemmPairSmemBytes = size_t(kStagesPair) * 2 * kHalfStageBytes + 1024;
+
+template <class Epi>
+struct PairLayout {
+  static constexpr int kSideBytes = Epi::kSideBytes;
+  static constexpr int kSideBufs = Epi::kSideBufs;
+  static constexpr int kSideTotal = kSideBytes * kSideBufs;
+  // shared memory a CTA may hold (227 KiB) less the static part: barriers and
+  // flags, plus the row-maxima exchange when the epilogue uses it
+  static constexpr int kBudget = 232448 - 512 - (Epi::kExchange ? int(sizeof(float2)) * 2 * 2 * BM : 0) - 1024;
+  // as many ring stages as fit beside the side buffers, at most 6
+  static constexpr int kStages = (kBudget - kSideTotal) / (2 * kHalfStageBytes) > 6
+                                     ? 6
+                                     : (kBudget - kSideTotal) / (2 * kHalfStageBytes);
+  static constexpr size_t kSmemBytes = size_t(kStages) * 2 * kHalfStageBytes + kSideTotal + 1024;
+  static_assert(kStages >= 3, "side buffers leave too few ring stages");
+  static_assert(kSideBytes % 1024 == 0, "side buffers keep 1024-byte alignment");
+};
 
 template <class Epi, bool kAMN, bool kBMN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_tc_pair_kernel(const __grid_constant__ GemmParams<Epi> p) {
   static_assert(kBMN, "the pair kernel loads B in 64-column boxes");
+  using L = PairLayout<Epi>;
+  constexpr int kStagesP = L::kStages;
+  constexpr int kSide = L::kSideBytes;
+  constexpr int kSB = L::kSideBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + kStagesPair * kHalfStageBytes;
+  uint8_t* sB = smem + kStagesP * kHalfStageBytes;
+  uint8_t* sSide = smem + 2 * kStagesP * kHalfStageBytes;
 
-  __shared__ __align__(8) uint64_t full_bar[kStagesPair];
-  __shared__ __align__(8) uint64_t empty_bar[kStagesPair];
+  __shared__ __align__(8) uint64_t full_bar[kStagesP];
+  __shared__ __align__(8) uint64_t empty_bar[kStagesP];
   __shared__ __align__(8) uint64_t acc_full[2];
   __shared__ __align__(8) uint64_t acc_empty[2];
+  __shared__ __align__(8) uint64_t side_full[2];
+  __shared__ __align__(8) uint64_t side_empty[2];
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ __align__(8) uint64_t xbar[4];
-  __shared__ float2 xchg[2][2][BM];  // [tile parity][half][row]
+  __shared__ float2 xchg[Epi::kExchange ? 2 : 1][2][Epi::kExchange ? BM : 32];  // [tile parity][half][row]
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -298,13 +330,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint32_t* const status = nullptr;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStagesPair; ++s) {
+    for (int s = 0; s < kStagesP; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 16);  // 8 epilogue warps x 2 CTAs (used in the even CTA)
+      mbar_init(&side_full[a], 1);
+      mbar_init(&side_empty[a], 8);  // this CTA's 8 epilogue warps
     }
     for (int q = 0; q < 4; ++q) mbar_init(&xbar[q], 2);
     mbar_init(&drain_bar, 1);
@@ -315,6 +349,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int i = 0; i < p.nprob; ++i) {
       tma_prefetch_map(&p.prob[i].tmA);
       tma_prefetch_map(&p.prob[i].tmB);
+      if (kSide > 0) {
+        tma_prefetch_map(&p.prob[i].tmS[0]);
+        tma_prefetch_map(&p.prob[i].tmS[1]);
+      }
     }
   }
   if (warp == 1) {
@@ -348,6 +386,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, armed = 0, armed_parity = 0;
+      const uint32_t fb0 = mapa_shared(&full_bar[0], 0);  // the even CTA's full barriers, 8 bytes apart
       bool ok = true;
       for (int tile = cluster; ok && tile < total; tile += nclusters) {
         int pi, mb2, nb;
@@ -362,7 +401,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             break;
           }
           if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 4 * kHalfStageBytes);
-          const uint32_t fb = mapa_shared(&full_bar[stage], 0);
+          const uint32_t fb = fb0 + stage * 8u;
           uint8_t* a_dst = sA + stage * kHalfStageBytes;
           uint8_t* b_dst = sB + stage * kHalfStageBytes;
           if (kAMN) {
@@ -375,14 +414,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           tma_load_2d_pair(b_dst + 8192, &pr.tmB, fb, col0 + 64, kb * BK);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == kStagesPair) {
+          if (++stage == kStagesP) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
       if (abort_flag && rank == 0) {
-        for (int s = 0; s < kStagesPair; ++s)
+        for (int s = 0; s < kStagesP; ++s)
           if (armed & (1u << s)) mbar_wait_drain(&full_bar[s], (armed_parity >> s) & 1u);
       }
     }
@@ -390,13 +429,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (lane == 0 && rank == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(256, 256, kAMN, kBMN);
+      // Descriptors of stage 0; a stage or a K step moves only the 14-bit start
+      // address field (16-byte units, shared addresses < 256 KiB), so the
+      // descriptors of any stage and step are one 64-bit add away.  This keeps
+      // the issuing thread's instruction stream short while the epilogue warps
+      // share its scheduler.
+      const uint64_t a_desc0 = kAMN ? sdesc_sw128(smem_u32(sA), 8192, 1024) : sdesc_sw128(smem_u32(sA), 16, 1024);
+      const uint64_t b_desc0 = sdesc_sw128(smem_u32(sB), 8192, 1024);
+      constexpr uint64_t kStageStep = kHalfStageBytes >> 4;
+      constexpr uint64_t kAStep = kAMN ? (2048 >> 4) : (32 >> 4);  // one K step of 16
+      constexpr uint64_t kBStep = 2048 >> 4;
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (int tile = cluster; ok && tile < total; tile += nclusters) {
         int pi, mb2, nb;
         locate(tile, pi, mb2, nb);
-        const GemmProblem<Epi>& pr = p.prob[pi];
-        const int nkb = (pr.K + BK - 1) / BK;
+        const int K = p.prob[pi].K;
+        const int nkb = (K + BK - 1) / BK;
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, &abort_flag, status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
@@ -406,18 +455,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + stage * kHalfStageBytes);
-          const uint32_t b_base = smem_u32(sB + stage * kHalfStageBytes);
-          const int kleft = pr.K - kb * BK;
-          const int ksteps = kleft >= BK ? BK / 16 : (kleft + 15) / 16;
-          for (int kk = 0; kk < ksteps; ++kk) {
-            const uint64_t ad = kAMN ? sdesc_sw128(a_base + kk * 2048, 8192, 1024)
-                                     : sdesc_sw128(a_base + kk * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(b_base + kk * 2048, 8192, 1024);
-            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          const uint64_t ad = a_desc0 + stage * kStageStep;
+          const uint64_t bd = b_desc0 + stage * kStageStep;
+          const int kleft = K - kb * BK;
+          if (kleft >= BK) {
+            umma_bf16_pair(d_tmem, ad, bd, idesc, kb != 0 ? 1u : 0u);
+#pragma unroll
+            for (int kk = 1; kk < BK / 16; ++kk) umma_bf16_pair(d_tmem, ad + kk * kAStep, bd + kk * kBStep, idesc, 1u);
+          } else {
+            const int ksteps = (kleft + 15) / 16;
+            for (int kk = 0; kk < ksteps; ++kk)
+              umma_bf16_pair(d_tmem, ad + kk * kAStep, bd + kk * kBStep, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit_pair_mc(&empty_bar[stage], 0x3);
-          if (++stage == kStagesPair) {
+          if (++stage == kStagesP) {
             stage = 0;
             phase ^= 1u;
           }
@@ -437,21 +488,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int half = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
+    const bool side_issuer = kSide > 0 && warp == 2 && lane == 0;
+    uint32_t side_armed = 0, side_parity = 0;  // per-buffer bit masks (issuer only)
+    bool ok = true;
+    // side loads of local tile j (the CTA's j-th tile) into buffer j % kSB;
+    // returns false when the wait for the buffer's release ran out
+    auto issue_side = [&](int j) -> bool {
+      const int tile = cluster + j * nclusters;
+      if (tile >= total) return true;
+      const int b = j % kSB;
+      if (j >= kSB && !mbar_wait(&side_empty[b], static_cast<uint32_t>(j / kSB - 1) & 1u, &abort_flag, status))
+        return false;
+      int pi, mb2, nb;
+      locate(tile, pi, mb2, nb);
+      fence_proxy_async_shared();
+      mbar_arrive_expect_tx(&side_full[b], kSide);
+      Epi::issue_side(p.prob[pi].tmS, mb2 * 2 + static_cast<int>(rank), nb, sSide + b * kSide, &side_full[b]);
+      side_armed |= 1u << b;
+      side_parity = (side_parity & ~(1u << b)) | ((static_cast<uint32_t>(j / kSB) & 1u) << b);
+      return true;
+    };
+    if (side_issuer)
+      for (int j = 0; j + 1 < kSB; ++j) ok = ok && issue_side(j);
     uint32_t it = 0;
-    for (int tile = cluster; tile < total; tile += nclusters, ++it) {
+    for (int tile = cluster; ok && tile < total; tile += nclusters, ++it) {
+      if (side_issuer && !issue_side(static_cast<int>(it) + kSB - 1)) break;
       const uint32_t buf = it & 1u, ph = (it >> 1) & 1u;
       int pi, mb2, nb;
       locate(tile, pi, mb2, nb);
       const GemmProblem<Epi>& pr = p.prob[pi];
       if (!mbar_wait(&acc_full[buf], ph, &abort_flag, status)) break;
+      const uint8_t* side = nullptr;
+      if (kSide > 0) {
+        const uint32_t sb = it % kSB;
+        if (!mbar_wait(&side_full[sb], (it / kSB) & 1u, &abort_flag, status)) break;
+        side = sSide + sb * kSide;
+      }
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * BN;
-      EpiPair ep{half, &xchg[it & 1u][half][quarter * 32], &xchg[it & 1u][half ^ 1][quarter * 32], &xbar[quarter],
-                 it & 1u, &abort_flag, pr.status};
-      Epi::apply(pr.epi, pr.M, pr.N, mb2 * 2 + static_cast<int>(rank), nb, row, taddr, ep);
+      float2* xm = Epi::kExchange ? &xchg[it & 1u][half][quarter * 32] : nullptr;
+      float2* xo = Epi::kExchange ? &xchg[it & 1u][half ^ 1][quarter * 32] : nullptr;
+      EpiPair ep{half, xm, xo, &xbar[quarter], it & 1u, &abort_flag, pr.status};
+      Epi::apply(pr.epi, pr.M, pr.N, mb2 * 2 + static_cast<int>(rank), nb, row, taddr, ep, side);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(&acc_empty[buf], 0));
+      if (lane == 0) {
+        if (kSide > 0) mbar_arrive(&side_empty[it % kSB]);
+        mbar_arrive_cluster(mapa_shared(&acc_empty[buf], 0));
+      }
+    }
+    if (side_issuer && abort_flag) {
+      for (int b = 0; b < kSB; ++b)
+        if (side_armed & (1u << b)) mbar_wait_drain(&side_full[b], (side_parity >> b) & 1u);
     }
   }
 

@@ -79,6 +79,20 @@ QG_DEV float draw_u(uint32_t w, int h) {
 // nearest integer, ties to even, returned in the low byte.
 QG_DEV uint32_t round_to_byte(float x) { return __float_as_uint(__fadd_rn(x, kMagic)); }
 
+// max(m, |x|) propagating NaN: a NaN x makes the result NaN.
+QG_DEV float max_nan_abs(float m, float x) {
+  float r;
+  asm("{\n\t.reg .f32 t;\n\tabs.f32 t, %2;\n\tmax.NaN.f32 %0, %1, t;\n\t}" : "=f"(r) : "f"(m), "f"(x));
+  return r;
+}
+
+// 16-byte granule g (0..15) of row `row` of a 128 x 256 int8 side tile, staged by
+// TMA as two 128 x 128 boxes with the 128-byte swizzle (granule j of a 128-byte
+// row r is stored at position j ^ (r mod 8)).
+QG_DEV uint4 side_granule(const uint8_t* side, int row, int g) {
+  return *reinterpret_cast<const uint4*>(side + (g >> 3) * 16384 + row * 128 + (((g & 7) ^ (row & 7)) << 4));
+}
+
 // Low bytes of four words packed into one word.
 QG_DEV uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
   return prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
@@ -87,6 +101,19 @@ QG_DEV uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
 // ------------------------------------------------------------------ a2 + a3 epilogue
 
 struct AdamEpi {
+  // side operands: the tile's M^Q codes (bytes [0, 32K)) and V^Q codes ([32K, 64K))
+  static constexpr int kSideBytes = 65536;
+  static constexpr int kSideBufs = 1;
+  static constexpr bool kExchange = true;  // block maxima combined across the two warpgroups
+
+  static QG_DEV void issue_side(const CUtensorMap* tmS, int mb, int nb, uint8_t* dst, uint64_t* bar) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      tma_load_2d(dst + k * 32768, &tmS[k], bar, nb * BN, mb * BM);
+      tma_load_2d(dst + k * 32768 + 16384, &tmS[k], bar, nb * BN + 128, mb * BM);
+    }
+  }
+
   struct Args {
     int8_t* Mq;
     int8_t* Vq;
@@ -110,11 +137,12 @@ struct AdamEpi {
     vv = __fadd_rn(__fmul_rn(a.beta2, v0), __fmul_rn(a.om2, __fmul_rn(R, R)));
   }
 
-  static QG_DEV void load_codes(const int8_t* mrow, const int8_t* vrow, int c, uint4 (&q)[4]) {
-    q[0] = *reinterpret_cast<const uint4*>(mrow + c * 32);
-    q[1] = *reinterpret_cast<const uint4*>(mrow + c * 32 + 16);
-    q[2] = *reinterpret_cast<const uint4*>(vrow + c * 32);
-    q[3] = *reinterpret_cast<const uint4*>(vrow + c * 32 + 16);
+  // codes of 32-column chunk c of this row from the staged side tiles
+  static QG_DEV void load_codes(const uint8_t* side, int row, int c, uint4 (&q)[4]) {
+    q[0] = side_granule(side, row, 2 * c);
+    q[1] = side_granule(side, row, 2 * c + 1);
+    q[2] = side_granule(side + 32768, row, 2 * c);
+    q[3] = side_granule(side + 32768, row, 2 * c + 1);
   }
 
   // Pass 1 on one 32-column chunk: the new moments and the running block maxima of
@@ -204,10 +232,9 @@ struct AdamEpi {
   // One thread owns row `row` of its warpgroup's 128-column half of the
   // 128 x 256 tile; the tile's 256 columns are exactly one moment block, so the
   // block maxima of the two halves are combined with the partner warp before
-  // the codes are formed.  Codes of chunk c + 1 are loaded while chunk c is
-  // computed.
+  // the codes are formed.  The tile's codes are staged in shared memory.
   static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
-                           const EpiPair& ep) {
+                           const EpiPair& ep, const uint8_t* side) {
     const int arow = mb * BM + row;
     const bool row_ok = arow < M;
     const int j0 = nb * BN;
@@ -228,25 +255,16 @@ struct AdamEpi {
     float amax_m = 0.f, amax_vv = 0.f;
     uint32_t mmin_b = 0xffffffffu, vmin_b = 0xffffffffu;
     bool bad = false;
-    uint4 qa[4] = {}, qb[4] = {};
 
-    if (row_ok && c0 < c1) load_codes(mrow, vrow, c0, qa);
 #pragma unroll 1
-    for (int c = c0; c < c1; c += 2) {
+    for (int c = c0; c < c1; ++c) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(taddr + c * 32, v);
       tmem_ld_wait();
       if (row_ok) {
-        if (c + 1 < c1) load_codes(mrow, vrow, c + 1, qb);
-        pass1_chunk(a, v, qa, sm, sv, ncols - c * 32, amax_m, amax_vv, mmin_b, vmin_b, bad);
-      }
-      if (c + 1 < c1) {
-        tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v);
-        tmem_ld_wait();
-        if (row_ok) {
-          if (c + 2 < c1) load_codes(mrow, vrow, c + 2, qa);
-          pass1_chunk(a, v, qb, sm, sv, ncols - (c + 1) * 32, amax_m, amax_vv, mmin_b, vmin_b, bad);
-        }
+        uint4 q[4];
+        load_codes(side, row, c, q);
+        pass1_chunk(a, v, q, sm, sv, ncols - c * 32, amax_m, amax_vv, mmin_b, vmin_b, bad);
       }
     }
 
@@ -274,33 +292,20 @@ struct AdamEpi {
     const float inv_m = live_m ? __fdiv_rn(127.0f, amax_m) : 0.f;
     const float inv_v = live_v ? __fdiv_rn(127.0f, amax_v) : 0.f;
 
-    if (row_ok && c0 < c1) load_codes(mrow, vrow, c0, qa);
 #pragma unroll 1
-    for (int c = c0; c < c1; c += 2) {
+    for (int c = c0; c < c1; ++c) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(taddr + c * 32, v);
       tmem_ld_wait();
       if (row_ok) {
-        if (c + 1 < c1) load_codes(mrow, vrow, c + 1, qb);
+        uint4 q[4];
+        load_codes(side, row, c, q);
         if (exact)
-          pass2_chunk<true>(a, v, qa, sm, sv, live_m, live_v, inv_m, inv_v, nrow + c * 32, mrow + c * 32,
+          pass2_chunk<true>(a, v, q, sm, sv, live_m, live_v, inv_m, inv_v, nrow + c * 32, mrow + c * 32,
                             vrow + c * 32);
         else
-          pass2_chunk<false>(a, v, qa, sm, sv, live_m, live_v, inv_m, inv_v, nrow + c * 32, mrow + c * 32,
+          pass2_chunk<false>(a, v, q, sm, sv, live_m, live_v, inv_m, inv_v, nrow + c * 32, mrow + c * 32,
                              vrow + c * 32);
-      }
-      if (c + 1 < c1) {
-        tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v);
-        tmem_ld_wait();
-        if (row_ok) {
-          if (c + 2 < c1) load_codes(mrow, vrow, c + 2, qa);
-          if (exact)
-            pass2_chunk<true>(a, v, qb, sm, sv, live_m, live_v, inv_m, inv_v, nrow + (c + 1) * 32,
-                              mrow + (c + 1) * 32, vrow + (c + 1) * 32);
-          else
-            pass2_chunk<false>(a, v, qb, sm, sv, live_m, live_v, inv_m, inv_v, nrow + (c + 1) * 32,
-                               mrow + (c + 1) * 32, vrow + (c + 1) * 32);
-        }
       }
     }
     if (row_ok && ep.half == 0) {
@@ -314,6 +319,16 @@ struct AdamEpi {
 // ------------------------------------------------------------------ a4 + a5 epilogue
 
 struct StochRoundEpi {
+  // side operand: the tile's W codes (128 rows x 256 columns), double-buffered
+  static constexpr int kSideBytes = 32768;
+  static constexpr int kSideBufs = 2;
+  static constexpr bool kExchange = false;
+
+  static QG_DEV void issue_side(const CUtensorMap* tmS, int mb, int nb, uint8_t* dst, uint64_t* bar) {
+    tma_load_2d(dst, &tmS[0], bar, nb * BN, mb * BM);
+    tma_load_2d(dst + 16384, &tmS[0], bar, nb * BN + 128, mb * BM);
+  }
+
   struct Args {
     int8_t* W;
     const float* sW;
@@ -321,7 +336,8 @@ struct StochRoundEpi {
     float alpha;
     uint32_t t, layer_id;
     PhiloxKey key;
-    int32_t aligned8;  // n % 8 == 0: every 32-column chunk starts a Philox call
+    int32_t aligned8;    // n % 8 == 0: every 32-column chunk starts a Philox call
+    int32_t aligned256;  // n % 256 == 0: a tile row is exactly one weight group
   };
 
   // The 16-bit draws of elements e0 .. e0+31: element i's draw is half (i & 1)
@@ -376,116 +392,135 @@ struct StochRoundEpi {
     }
   }
 
-  // Raw inputs of one 32-column chunk of a row: W codes and the scales of the
-  // (at most two) weight groups it touches.
-  struct ChunkIn {
-    uint4 q0, q1;
-    float s0, s1;
-  };
-
-  static QG_DEV void load_chunk(const Args& a, int N, int irow, int jc, ChunkIn& in) {
-    const int valid = min(32, N - jc);
-    const int64_t e0 = static_cast<int64_t>(irow) * N + jc;
-    const int64_t g0 = e0 >> 8, g1 = (e0 + valid - 1) >> 8;
-    const int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + jc;
-    in.q0 = *reinterpret_cast<const uint4*>(wrow);
-    in.q1 = valid > 16 ? *reinterpret_cast<const uint4*>(wrow + 16) : make_uint4(0, 0, 0, 0);
-    in.s0 = a.sW[g0];
-    in.s1 = g1 != g0 ? a.sW[g1] : in.s0;
+  // c'_g = (alpha / s_g) * 2^16: the update factor in units of 2^-16 code; a
+  // scale that is not positive freezes its group.
+  static QG_DEV float update_factor(float alpha, float s) {
+    return s > 0.f ? __fmul_rn(__fdiv_rn(alpha, s), 65536.0f) : 0.f;
   }
 
-  // One 32-column chunk of row irow: W codes from `in`, U from TMEM, updated
-  // codes written back.  y = q + U c_g; round up iff u < y - floor(y); clamp to
-  // [-127, 127]; a NaN y keeps the old code.
-  template <bool kAligned8>
-  static QG_DEV void sr_chunk(const Args& a, int N, int irow, int jc, const uint32_t (&U)[32], const ChunkIn& in) {
-    const int valid = min(32, N - jc);
-    const int64_t e0 = static_cast<int64_t>(irow) * N + jc;
-    const int64_t g0 = e0 >> 8;
-    const int64_t g1 = (e0 + valid - 1) >> 8;
-    const float c0 = in.s0 > 0.f ? __fdiv_rn(a.alpha, in.s0) : 0.f;
-    const float c1 = g1 != g0 ? (in.s1 > 0.f ? __fdiv_rn(a.alpha, in.s1) : 0.f) : c0;
-    const int split = g1 != g0 ? static_cast<int>((g1 << 8) - e0) : 32;
-    int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + jc;
-    uint32_t d[16];
-    draws<kAligned8>(a, e0, d);
-    uint32_t out[8], bytes[4];
+  // One 32-column chunk: W codes in (wa, wb), U from TMEM, draws d; the new codes
+  // in out[8].  With X = U c' (the update in units of 2^-16 code) and
+  // K = ceil(X), the new code is clamp(q + floor((K + draw) / 2^16), -127, 127),
+  // and a NaN X keeps q.
+  //
+  // Fast form, valid while |X| < 2^22: fadd.rp(X, 1.5 * 2^23) has the bits
+  // 0x4B400000 + K; adding the draw less 2^22 and q * 2^16 gives
+  // 0x4B000000 + K + draw + q * 2^16, whose bits [16, 32) are 0x4B00 + q + r with
+  // r = floor((K + draw) / 2^16).  The clamp of q + r to [-127, 127] is a clamp
+  // of that sum, and its byte 2 is the new code.  When |X| reaches 2^22, or X is
+  // NaN, the chunk is redone in the general form.
+  template <bool kOneFactor>
+  static QG_DEV void sr_chunk(const uint32_t (&U)[32], const uint4& wa, const uint4& wb, const uint32_t (&d)[16],
+                              float cp0, float cp1, int split, uint32_t (&out)[8]) {
+    constexpr int kLo = (0x4B00 - 127) << 16;
+    constexpr int kHi = ((0x4B00 + 127) << 16) | 0xFFFF;
+    float mx = 0.f;
+    uint32_t S[4];
 #pragma unroll
     for (int k = 0; k < 32; ++k) {
-      const float q = code_f32(in.q0, in.q1, k);
-      const float ck = k < split ? c0 : c1;
-      const float x = __fmul_rn(__uint_as_float(U[k]), ck);
-      const float y = __fadd_rn(q, x);
-      const float f = floorf(y);
-      const float phi = __fsub_rn(y, f);
-      const bool up = draw_u(d[k >> 1], k & 1) < phi;
-      float qf = up ? __fadd_rn(f, 1.0f) : f;
-      qf = fminf(fmaxf(qf, -127.0f), 127.0f);
-      bytes[k & 3] = round_to_byte((y != y) ? q : qf);
-      if ((k & 3) == 3) out[k >> 2] = pack4(bytes[0], bytes[1], bytes[2], bytes[3]);
+      const float cp = (kOneFactor || k < split) ? cp0 : cp1;
+      const float X = __fmul_rn(__uint_as_float(U[k]), cp);
+      mx = max_nan_abs(mx, X);
+      const uint32_t tb = __float_as_uint(__fadd_ru(X, kMagic));
+      const uint32_t dq = prmt(d[k >> 1], 0xFFC00000u, (k & 1) ? 0x7632u : 0x7610u);
+      const uint32_t wsel = 0x44u | (static_cast<uint32_t>(k & 3) << 8) | (static_cast<uint32_t>((k & 3) | 8) << 12);
+      const uint32_t q16 = prmt(word_of(k < 16 ? wa : wb, (k >> 2) & 3), 0u, wsel);
+      const int sum = static_cast<int>(tb + dq + q16);
+      S[k & 3] = static_cast<uint32_t>(min(max(sum, kLo), kHi));
+      if ((k & 3) == 3) out[k >> 2] = prmt(prmt(S[0], S[1], 0x62u), prmt(S[2], S[3], 0x62u), 0x5410u);
     }
-    if (valid == 32) {
-      *reinterpret_cast<uint4*>(wrow) = make_uint4(out[0], out[1], out[2], out[3]);
-      *reinterpret_cast<uint4*>(wrow + 16) = make_uint4(out[4], out[5], out[6], out[7]);
-    } else {
+    if (!(mx < 4194304.0f)) {
 #pragma unroll
-      for (int k = 0; k < 32; ++k)
-        if (k < valid) wrow[k] = static_cast<int8_t>((out[k >> 2] >> (8 * (k & 3))) & 0xFFu);
+      for (int k = 0; k < 32; ++k) {
+        const float cp = (kOneFactor || k < split) ? cp0 : cp1;
+        const float X = __fmul_rn(__uint_as_float(U[k]), cp);
+        const uint4& w = k < 16 ? wa : wb;
+        const int q = static_cast<int8_t>((word_of(w, (k >> 2) & 3) >> (8 * (k & 3))) & 0xFFu);
+        int v = q;
+        if (X == X) {
+          const int K = __float2int_ru(fminf(fmaxf(X, -1073741824.0f), 1073741824.0f));
+          const int draw = static_cast<int>((d[k >> 1] >> (16 * (k & 1))) & 0xFFFFu);
+          v = min(max(q + ((K + draw) >> 16), -127), 127);
+        }
+        const uint32_t sh = 8 * (k & 3);
+        out[k >> 2] = (out[k >> 2] & ~(0xFFu << sh)) | ((static_cast<uint32_t>(v) & 0xFFu) << sh);
+      }
     }
   }
 
-  // This warpgroup's half of the tile's columns, in chunk pairs: the inputs of
-  // chunk c + 1 are loaded while chunk c is computed, the two input buffers
-  // alternating without copies.
-  template <bool kAligned8>
-  static QG_DEV void apply_impl(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr, int half) {
+  // This warpgroup's half of the tile's columns, 32-column chunks; W codes come
+  // from the staged side tile, the new codes go straight to global memory.
+  template <bool kAligned8, bool kOneGroup>
+  static QG_DEV void apply_impl(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr, int half,
+                                const uint8_t* side) {
     const int irow = mb * BM + row;
     const bool row_ok = irow < M;
     const int j0 = nb * BN;
     const int ncols = min(BN, N - j0);
     const int c0 = half * 4;
     const int c1 = min(c0 + 4, (ncols + 31) >> 5);
-    ChunkIn ia = {}, ib = {};
-    if (row_ok && c0 < c1) load_chunk(a, N, irow, j0 + c0 * 32, ia);
+    float cp_row = 0.f;
+    if (kOneGroup && row_ok) cp_row = update_factor(a.alpha, a.sW[(static_cast<int64_t>(irow) * N + j0) >> 8]);
+    int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + j0;
 #pragma unroll 1
-    for (int c = c0; c < c1; c += 2) {
+    for (int c = c0; c < c1; ++c) {
       uint32_t U[32];
       tmem_ld_32x32b_x32(taddr + c * 32, U);
       tmem_ld_wait();
-      if (row_ok) {
-        if (c + 1 < c1) load_chunk(a, N, irow, j0 + (c + 1) * 32, ib);
-        sr_chunk<kAligned8>(a, N, irow, j0 + c * 32, U, ia);
+      if (!row_ok) continue;
+      const int jc = c * 32;
+      const int valid = min(32, ncols - jc);
+      const int64_t e0 = static_cast<int64_t>(irow) * N + j0 + jc;
+      float cp0 = cp_row, cp1 = cp_row;
+      int split = 32;
+      if (!kOneGroup) {
+        const int64_t g0 = e0 >> 8, g1 = (e0 + valid - 1) >> 8;
+        cp0 = update_factor(a.alpha, a.sW[g0]);
+        cp1 = g1 != g0 ? update_factor(a.alpha, a.sW[g1]) : cp0;
+        split = g1 != g0 ? static_cast<int>((g1 << 8) - e0) : 32;
       }
-      if (c + 1 < c1) {
-        tmem_ld_32x32b_x32(taddr + (c + 1) * 32, U);
-        tmem_ld_wait();
-        if (row_ok) {
-          if (c + 2 < c1) load_chunk(a, N, irow, j0 + (c + 2) * 32, ia);
-          sr_chunk<kAligned8>(a, N, irow, j0 + (c + 1) * 32, U, ib);
-        }
+      const uint4 wa = side_granule(side, row, 2 * c), wb = side_granule(side, row, 2 * c + 1);
+      uint32_t d[16];
+      draws<kAligned8>(a, e0, d);
+      uint32_t out[8];
+      sr_chunk<kOneGroup>(U, wa, wb, d, cp0, cp1, split, out);
+      if (valid == 32) {
+        *reinterpret_cast<uint4*>(wrow + jc) = make_uint4(out[0], out[1], out[2], out[3]);
+        *reinterpret_cast<uint4*>(wrow + jc + 16) = make_uint4(out[4], out[5], out[6], out[7]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (k < valid) wrow[jc + k] = static_cast<int8_t>((out[k >> 2] >> (8 * (k & 3))) & 0xFFu);
       }
     }
   }
 
   static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
-                           const EpiPair& ep) {
-    if (a.aligned8)
-      apply_impl<true>(a, M, N, mb, nb, row, taddr, ep.half);
+                           const EpiPair& ep, const uint8_t* side) {
+    if (a.aligned256)
+      apply_impl<true, true>(a, M, N, mb, nb, row, taddr, ep.half, side);
+    else if (a.aligned8)
+      apply_impl<true, false>(a, M, N, mb, nb, row, taddr, ep.half, side);
     else
-      apply_impl<false>(a, M, N, mb, nb, row, taddr, ep.half);
+      apply_impl<false, false>(a, M, N, mb, nb, row, taddr, ep.half, side);
   }
 };
 
 // ------------------------------------------------------------------ plain fp32 store
 
 struct StoreF32Epi {
+  static constexpr int kSideBytes = 0;
+  static constexpr int kSideBufs = 1;
+  static constexpr bool kExchange = false;
+  static QG_DEV void issue_side(const CUtensorMap*, int, int, uint8_t*, uint64_t*) {}
+
   struct Args {
     float* D;
     int64_t ldd;
     int32_t accumulate;  // D += A B instead of D = A B
   };
   static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
-                           const EpiPair& ep) {
+                           const EpiPair& ep, const uint8_t*) {
     const int grow = mb * BM + row;
     const bool ok = grow < M;
     const int j0 = nb * BN;
@@ -518,9 +553,10 @@ struct StoreF32Epi {
   }
 };
 
-static_assert(sizeof(GemmParams<AdamEpi>) <= 4096, "kernel parameter block");
-static_assert(sizeof(GemmParams<StochRoundEpi>) <= 4096, "kernel parameter block");
-static_assert(sizeof(GemmParams<StoreF32Epi>) <= 4096, "kernel parameter block");
+// kernel parameters up to 32764 bytes (CUDA 12.1 and later on sm_70 and newer)
+static_assert(sizeof(GemmParams<AdamEpi>) <= 32764, "kernel parameter block");
+static_assert(sizeof(GemmParams<StochRoundEpi>) <= 32764, "kernel parameter block");
+static_assert(sizeof(GemmParams<StoreF32Epi>) <= 32764, "kernel parameter block");
 
 // ------------------------------------------------------------------ a1 and test kernels
 
@@ -571,8 +607,8 @@ __global__ void philox_kernel(const uint32_t* c0, const uint32_t* c1, const uint
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 static std::once_flag g_encode_once;
 
-bool encode_map_bf16(void* map, const void* base, uint64_t inner, uint64_t outer, uint64_t ld_elems,
-                     uint32_t box_inner, uint32_t box_outer) {
+static bool encode_map(void* map, CUtensorMapDataType dtype, uint32_t esize, const void* base, uint64_t inner,
+                       uint64_t outer, uint64_t ld_elems, uint32_t box_inner, uint32_t box_outer) {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -582,14 +618,24 @@ bool encode_map_bf16(void* map, const void* base, uint64_t inner, uint64_t outer
   });
   if (!g_encode) return false;
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {ld_elems * 2};
+  const cuuint64_t strides[1] = {ld_elems * esize};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = g_encode(reinterpret_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  const CUresult r = g_encode(reinterpret_cast<CUtensorMap*>(map), dtype, 2,
                               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_map_bf16(void* map, const void* base, uint64_t inner, uint64_t outer, uint64_t ld_elems,
+                     uint32_t box_inner, uint32_t box_outer) {
+  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, outer, ld_elems, box_inner, box_outer);
+}
+
+// int8 side tiles: boxes of 128 rows x 128 bytes, 128-byte swizzle
+static bool encode_map_i8_side(void* map, const void* base, uint64_t inner, uint64_t outer, uint64_t ld_bytes) {
+  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, inner, outer, ld_bytes, 128, 128);
 }
 
 int sm_count() {
@@ -631,10 +677,11 @@ template <class Epi, bool kAMN>
 static cudaError_t launch_gemm_pair(const GemmParams<Epi>& p, cudaStream_t stream, int kind, double flops,
                                     double bytes) {
   auto kern = gemm_tc_pair_kernel<Epi, kAMN, true>;
+  constexpr size_t kSmem = PairLayout<Epi>::kSmemBytes;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kGemmPairSmemBytes));
+                                         static_cast<int>(kSmem));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -643,7 +690,7 @@ static cudaError_t launch_gemm_pair(const GemmParams<Epi>& p, cudaStream_t strea
   if (pair_tiles == 0) return cudaSuccess;
   const int clusters = std::min(pair_tiles, std::max(1, sm_count() / 2));
   const int tok = profile_begin(stream, kind, flops, bytes);
-  kern<<<2 * clusters, kGemmThreads, kGemmPairSmemBytes, stream>>>(p);
+  kern<<<2 * clusters, kGemmThreads, kSmem, stream>>>(p);
   profile_end(stream, tok);
   return cudaGetLastError();
 }
@@ -729,6 +776,9 @@ cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream
       if (!encode_map_bf16(&pr.tmA, s.Pbf, s.r, s.m, s.r, 64, 64)) return cudaErrorInvalidValue;
       // B = G (K = m, N = n), MN-major: box {64 (n), 64 (m)}
       if (!encode_map_bf16(&pr.tmB, s.G, s.n, s.m, s.ldg, 64, 64)) return cudaErrorInvalidValue;
+      // side operands: M^Q and V^Q (r x n int8, leading dimension ld_mom)
+      if (!encode_map_i8_side(&pr.tmS[0], s.Mq, s.n, s.r, s.ld_mom)) return cudaErrorInvalidValue;
+      if (!encode_map_i8_side(&pr.tmS[1], s.Vq, s.n, s.r, s.ld_mom)) return cudaErrorInvalidValue;
       pr.status = s.status;
       pr.epi = AdamEpi::Args{s.Mq, s.Vq, s.sM, s.sV, s.Nbuf, s.ld_mom, s.ldN, s.nblk,
                              s.beta1, s.beta2, s.om1, s.om2, s.c1, s.c2, s.eps};
@@ -746,10 +796,12 @@ cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream
       if (!encode_map_bf16(&pr.tmA, s.Pbf, s.r, s.m, s.r, 64, 128)) return cudaErrorInvalidValue;
       // B = N (K = r, N = n), MN-major: box {64 (n), 64 (r)}
       if (!encode_map_bf16(&pr.tmB, s.Nbuf, s.n, s.r, s.ldN, 64, 64)) return cudaErrorInvalidValue;
+      // side operand: W^Q (m x n int8, leading dimension ldw)
+      if (!encode_map_i8_side(&pr.tmS[0], s.W, s.n, s.m, s.ldw)) return cudaErrorInvalidValue;
       pr.status = s.status;
       pr.epi = StochRoundEpi::Args{s.W, s.sW, s.ldw, s.alpha, s.t, s.layer_id,
                                    PhiloxKey{static_cast<uint32_t>(s.seed), static_cast<uint32_t>(s.seed >> 32)},
-                                   (s.n % 8) == 0 ? 1 : 0};
+                                   (s.n % 8) == 0 ? 1 : 0, (s.n % 256) == 0 ? 1 : 0};
       add_problem(p2, s.m, s.n, s.r);
     }
     e = launch_gemm_pair<StochRoundEpi, false>(p2, stream, QG_KERNEL_BACKPROJECT_SR, fl2, by2);

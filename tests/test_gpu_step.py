@@ -141,6 +141,35 @@ def test_step_parity_with_oracle(m, n, r, steps):
     assert gl.sched().t == steps
 
 
+@pytest.mark.parametrize("m,n,r", [(256, 512, 32), (300, 700, 64)])
+def test_step_parity_extreme_weight_scales(m, n, r):
+    # Weight groups whose scale makes the update huge (every code saturates),
+    # large but not saturating (|x| ~ 100 codes: the general form of the
+    # stochastic rounding instead of the fixed-point fast form), zero (frozen)
+    # and ordinary, in one matrix.
+    oc = O.Config(m=m, n=n, r=r, seed=9, layer_id=2)
+    Wq = synth.weight_codes(m, n, 9)
+    sW = synth.weight_scales(m, n, seed=9).copy()
+    sW[0:3] = 1e-12
+    sW[3:5] = 3e-7
+    sW[5] = 0.0
+    gen = synth.lowrank_gradient(m, n, rank=min(256, m, n), seed=9)
+    ost = O.LayerState.create(oc, Wq, sW)
+    O.set_projection(ost, O.exact_topr(gen.draw(0)[0], r)[0])
+    gl = GpuLayer(oc, Wq, sW)
+    gl.set_projection(ost.Pq, ost.sP)
+    for t in range(2):
+        G, Gb = gen.draw(t)
+        dG, ldg = upload_gradient(Gb)
+        gl.step(dG, ldg)
+        O.step(ost, G)
+        compare_state(ost, gl, f"step {t + 1}")
+    W = gl.weights().ravel()
+    assert np.all(np.abs(W[0:3 * 256].astype(np.int32)) == 127)
+    np.testing.assert_array_equal(W[5 * 256:6 * 256], Wq.ravel()[5 * 256:6 * 256])
+    assert gl.status() == qg.QG_OK
+
+
 def test_step_is_deterministic():
     outs = []
     for _ in range(2):
