@@ -61,15 +61,34 @@ QG_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete is
+// suspended in hardware (up to kSuspendHintNs, or until the phase completes)
+// instead of spinning, so waiting warps leave the issue slots to the warps that
+// share their scheduler.
+constexpr uint32_t kSuspendHintNs = 1000000u;  // 1 ms
+
+QG_DEV bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return done != 0;
+}
+
 // Waits for the phase of parity `parity` to complete.  Gives up (returns false)
 // when another thread of the CTA has raised *abort, or after kWaitLimitNs, in
-// which case it raises *abort and the timeout bit of *status itself.
+// which case it raises *abort and the timeout bit of *status itself.  The abort
+// flag and the clock are checked every 8 suspensions (at most about 8 ms apart).
 QG_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* status) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_suspend(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
+    if (mbar_try_wait_suspend(bar, parity)) return true;
+    if ((it & 7u) == 0u) {
       if (*abort) return false;
       if (globaltimer() - t0 > kWaitLimitNs) {
         *abort = 1;

@@ -86,6 +86,13 @@ QG_DEV float max_nan_abs(float m, float x) {
   return r;
 }
 
+// max(m, v) propagating NaN.
+QG_DEV float max_nan(float m, float v) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(m), "f"(v));
+  return r;
+}
+
 // 16-byte granule g (0..15) of row `row` of a 128 x 256 int8 side tile, staged by
 // TMA as two 128 x 128 boxes with the 128-byte swizzle (granule j of a 128-byte
 // row r is stored at position j ^ (r mod 8)).
@@ -147,56 +154,55 @@ struct AdamEpi {
 
   // Pass 1 on one 32-column chunk: the new moments and the running block maxima of
   // |m| and of v (max over the block of sqrt(v) is sqrt of the max of v, the
-  // correctly rounded square root being monotone).  It also keeps the smallest
-  // nonzero |m| and v as (bits << 1) - 1, zero mapping to all ones, which decide
-  // whether pass 2 may use the branch-free square root and division.
+  // correctly rounded square root being monotone).  The maxima propagate NaN, so
+  // a non-finite moment shows in them.  It also keeps the smallest |m| and v
+  // (zeros included), which decide whether pass 2 may use the branch-free square
+  // root and division.  kFull: all 32 columns are inside the matrix.
+  template <bool kFull>
   static QG_DEV void pass1_chunk(const Args& a, const uint32_t (&v)[32], const uint4 (&cq)[4], float sm, float sv,
-                                 int valid, float& amax_m, float& amax_vv, uint32_t& mmin_b, uint32_t& vmin_b,
-                                 bool& bad) {
+                                 int valid, float& amax_m, float& amax_vv, float& mmin, float& vmin) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const float R = __uint_as_float(v[e]);
       float mm, vv;
       moments(R, code_f32(cq[0], cq[1], e), code_f32(cq[2], cq[3], e), sm, sv, a, mm, vv);
-      if (e < valid) {
-        amax_m = fmaxf(amax_m, fabsf(mm));
-        amax_vv = fmaxf(amax_vv, vv);
-        mmin_b = min(mmin_b, (__float_as_uint(mm) << 1) - 1u);
-        vmin_b = min(vmin_b, (__float_as_uint(vv) << 1) - 1u);
-        bad |= !isfinite(R);
+      if (kFull || e < valid) {
+        amax_m = max_nan_abs(amax_m, mm);
+        amax_vv = max_nan(amax_vv, vv);
+        mmin = fminf(mmin, fabsf(mm));
+        vmin = fminf(vmin, vv);
       }
     }
   }
 
   // True when every square root and division of this thread's pass 2 has its
   // operands and quotient inside the ranges where sqrt_exact and div_exact equal
-  // the IEEE operations: v in {0} U [2^-100, 2^100], the denominator
-  // sqrt(v) c2 + eps in [eps, dmax] within [2^-100, 2^100], the numerator m c1
-  // zero or in [2^-90, 2^90], and every nonzero quotient in [2^-100, 2^100].
-  static QG_DEV bool exact_fast_ok(const Args& a, float amax_m, float amax_vv, uint32_t mmin_b, uint32_t vmin_b,
-                                   bool bad) {
+  // the IEEE operations: v in [2^-100, 2^100], the denominator sqrt(v) c2 + eps
+  // in [eps, dmax] within [2^-100, 2^100], the numerator m c1 in [2^-90, 2^90],
+  // and every quotient in [2^-100, 2^100].  A zero m or v sends the row to the
+  // intrinsics, as does anything non-finite.
+  static QG_DEV bool exact_fast_ok(const Args& a, float amax_m, float amax_vv, float mmin, float vmin) {
     const float c1a = fabsf(a.c1);
-    bool ok = !bad && a.eps >= kSafeLo && amax_vv <= kSafeHi && a.c2 > 0.f;
-    if (vmin_b != 0xffffffffu) ok = ok && __uint_as_float((vmin_b + 1u) >> 1) >= kSafeLo;
+    bool ok = amax_m <= 3.4028234663852886e38f && amax_vv <= kSafeHi && vmin >= kSafeLo && a.eps >= kSafeLo &&
+              a.c2 > 0.f;
     const float dmax = __fadd_rn(__fmul_rn(__fsqrt_rn(amax_vv), a.c2), a.eps);
     const float nmax = __fmul_rn(amax_m, c1a);
+    const float nmin = __fmul_rn(mmin, c1a);
     ok = ok && dmax <= kSafeHi && nmax <= kSafeDivHi && nmax <= __fmul_rn(kSafeHi, a.eps);
-    if (mmin_b != 0xffffffffu) {
-      const float nmin = __fmul_rn(__uint_as_float((mmin_b + 1u) >> 1), c1a);
-      ok = ok && nmin >= kSafeDivLo && nmin >= __fmul_rn(kSafeLo, dmax);
-    }
+    ok = ok && nmin >= kSafeDivLo && nmin >= __fmul_rn(kSafeLo, dmax);
     return ok;
   }
 
   // Pass 2 on one chunk: the same moments; N = -lr m_hat / (sqrt(v_hat) + eps)
   // = (m c1) / (sqrt(v) c2 + eps) -> bf16; codes of m and sqrt(v) on the block's
-  // new grids.
+  // new grids.  |m| * (127 / absmax) and sqrt(v) * (127 / absmax_v) stay within
+  // 127 (1 + 2^-24), so their nearest integers need no clamp; a zero block has
+  // inverse scale 0 and gets codes 0.
   // kExact selects sqrt_exact / div_exact, equal to the IEEE operations on the
   // ranges exact_fast_ok checks, over the intrinsics.
   template <bool kExact>
   static QG_DEV void pass2_chunk(const Args& a, const uint32_t (&v)[32], const uint4 (&cq)[4], float sm, float sv,
-                                 bool live_m, bool live_v, float inv_m, float inv_v, uint16_t* nptr, int8_t* mptr,
-                                 int8_t* vptr) {
+                                 float inv_m, float inv_v, uint16_t* nptr, int8_t* mptr, int8_t* vptr) {
     uint32_t om[8], ov[8], packed[16], bm[4], bv[4];
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
@@ -211,9 +217,8 @@ struct AdamEpi {
         packed[e >> 1] |= b << 16;
       else
         packed[e >> 1] = b;
-      // rint then clamp to integer bounds == clamp then rint (ties to even)
-      bm[e & 3] = live_m ? round_to_byte(fminf(fmaxf(__fmul_rn(mm, inv_m), -127.f), 127.f)) : 0u;
-      bv[e & 3] = live_v ? round_to_byte(fminf(fmaxf(__fmul_rn(rv, inv_v), 0.f), 127.f)) : 0u;
+      bm[e & 3] = round_to_byte(__fmul_rn(mm, inv_m));
+      bv[e & 3] = round_to_byte(__fmul_rn(rv, inv_v));
       if ((e & 3) == 3) {
         om[e >> 2] = pack4(bm[0], bm[1], bm[2], bm[3]);
         ov[e >> 2] = pack4(bv[0], bv[1], bv[2], bv[3]);
@@ -252,9 +257,7 @@ struct AdamEpi {
       vrow = a.Vq + static_cast<int64_t>(arow) * a.ld_mom + j0;
       nrow = a.Nout + static_cast<int64_t>(arow) * a.ldN + j0;
     }
-    float amax_m = 0.f, amax_vv = 0.f;
-    uint32_t mmin_b = 0xffffffffu, vmin_b = 0xffffffffu;
-    bool bad = false;
+    float amax_m = 0.f, amax_vv = 0.f, mmin = __int_as_float(0x7f800000), vmin = __int_as_float(0x7f800000);
 
 #pragma unroll 1
     for (int c = c0; c < c1; ++c) {
@@ -264,11 +267,17 @@ struct AdamEpi {
       if (row_ok) {
         uint4 q[4];
         load_codes(side, row, c, q);
-        pass1_chunk(a, v, q, sm, sv, ncols - c * 32, amax_m, amax_vv, mmin_b, vmin_b, bad);
+        const int valid = ncols - c * 32;
+        if (valid >= 32)
+          pass1_chunk<true>(a, v, q, sm, sv, valid, amax_m, amax_vv, mmin, vmin);
+        else
+          pass1_chunk<false>(a, v, q, sm, sv, valid, amax_m, amax_vv, mmin, vmin);
       }
     }
 
-    const bool exact = exact_fast_ok(a, amax_m, amax_vv, mmin_b, vmin_b, bad);
+    // a non-finite gradient reaches the maxima (they propagate NaN and Inf)
+    const bool bad = !(amax_m <= 3.4028234663852886e38f) || !(amax_vv <= 3.4028234663852886e38f);
+    const bool exact = exact_fast_ok(a, amax_m, amax_vv, mmin, vmin);
 
     // block maxima over both halves (the partner warp owns the same rows)
     const int lane = row & 31;
@@ -301,11 +310,9 @@ struct AdamEpi {
         uint4 q[4];
         load_codes(side, row, c, q);
         if (exact)
-          pass2_chunk<true>(a, v, q, sm, sv, live_m, live_v, inv_m, inv_v, nrow + c * 32, mrow + c * 32,
-                            vrow + c * 32);
+          pass2_chunk<true>(a, v, q, sm, sv, inv_m, inv_v, nrow + c * 32, mrow + c * 32, vrow + c * 32);
         else
-          pass2_chunk<false>(a, v, q, sm, sv, live_m, live_v, inv_m, inv_v, nrow + c * 32, mrow + c * 32,
-                             vrow + c * 32);
+          pass2_chunk<false>(a, v, q, sm, sv, inv_m, inv_v, nrow + c * 32, mrow + c * 32, vrow + c * 32);
       }
     }
     if (row_ok && ep.half == 0) {
@@ -344,14 +351,14 @@ struct StochRoundEpi {
   // of d[i >> 1].  Element e takes half (e mod 2) of word ((e / 2) mod 4) of
   // Philox-4x32-10(counter = (e / 8, t, layer_id), key = seed).
   template <bool kAligned8>
-  static QG_DEV void draws(const Args& a, int64_t e0, uint32_t (&d)[16]) {
+  static QG_DEV void draws(const Args& a, const PhiloxRoundKeys& rk, int64_t e0, uint32_t (&d)[16]) {
     const uint64_t cb = static_cast<uint64_t>(e0) >> 3;
     if (kAligned8) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         uint32_t o[4];
         const uint64_t c = cb + k;
-        philox4x32_10(static_cast<uint32_t>(c), static_cast<uint32_t>(c >> 32), a.t, a.layer_id, a.key, o);
+        philox4x32_10(static_cast<uint32_t>(c), static_cast<uint32_t>(c >> 32), a.t, a.layer_id, rk, o);
         d[4 * k] = o[0];
         d[4 * k + 1] = o[1];
         d[4 * k + 2] = o[2];
@@ -364,7 +371,7 @@ struct StochRoundEpi {
       for (int k = 0; k < 5; ++k) {
         uint32_t o[4];
         const uint64_t c = cb + k;
-        philox4x32_10(static_cast<uint32_t>(c), static_cast<uint32_t>(c >> 32), a.t, a.layer_id, a.key, o);
+        philox4x32_10(static_cast<uint32_t>(c), static_cast<uint32_t>(c >> 32), a.t, a.layer_id, rk, o);
         dd[4 * k] = o[0];
         dd[4 * k + 1] = o[1];
         dd[4 * k + 2] = o[2];
@@ -462,6 +469,7 @@ struct StochRoundEpi {
     float cp_row = 0.f;
     if (kOneGroup && row_ok) cp_row = update_factor(a.alpha, a.sW[(static_cast<int64_t>(irow) * N + j0) >> 8]);
     int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + j0;
+    const PhiloxRoundKeys rk = philox_round_keys(a.key);
 #pragma unroll 1
     for (int c = c0; c < c1; ++c) {
       uint32_t U[32];
@@ -481,7 +489,7 @@ struct StochRoundEpi {
       }
       const uint4 wa = side_granule(side, row, 2 * c), wb = side_granule(side, row, 2 * c + 1);
       uint32_t d[16];
-      draws<kAligned8>(a, e0, d);
+      draws<kAligned8>(a, rk, e0, d);
       uint32_t out[8];
       sr_chunk<kOneGroup>(U, wa, wb, d, cp0, cp1, split, out);
       if (valid == 32) {
@@ -560,37 +568,55 @@ static_assert(sizeof(GemmParams<StoreF32Epi>) <= 32764, "kernel parameter block"
 
 // ------------------------------------------------------------------ a1 and test kernels
 
-// Eight INT4 codes (one 32-bit word, element 2i in the low nibble of byte i)
-// -> eight bf16 of P~ = bf16_rn(code * scale).  Groups of 64 never split a word.
-// One launch covers up to kMaxProblems projections.
+// Thirty-two INT4 codes (16 bytes, element 2i in the low nibble of byte i) ->
+// thirty-two bf16 of P~ = bf16_rn(code * scale).  Every projection has
+// m*r % 32 == 0 (r % 32 == 0), so a 32-element chunk stays inside one matrix and
+// one 64-element scale group.  One launch covers up to kMaxProblems projections.
+// HBM-bound: 16 bytes read and 64 bytes written per thread, coalesced across
+// the warp; nibbles become floats by exact integer/FP-add arithmetic (no
+// conversion-pipe instructions), and pairs are rounded to bf16 together.
 struct DequantBatch {
   const uint8_t* Pq[kMaxProblems];
   const float* sP[kMaxProblems];
   uint16_t* out[kMaxProblems];
-  int64_t chunk_begin[kMaxProblems + 1];  // prefix sums of (m*r / 8)
+  int64_t chunk_begin[kMaxProblems + 1];  // prefix sums of (m*r / 32)
   int32_t n;
 };
 
-__global__ void dequant_projection_kernel(const __grid_constant__ DequantBatch b) {
-  const int64_t i8 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i8 >= b.chunk_begin[b.n]) return;
+template <bool kVec16>
+__global__ void __launch_bounds__(256) dequant_projection_kernel(const __grid_constant__ DequantBatch b) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= b.chunk_begin[b.n]) return;
   int p = 0;
-  while (p + 1 < b.n && i8 >= b.chunk_begin[p + 1]) ++p;
-  const int64_t e0 = (i8 - b.chunk_begin[p]) * 8;
-  const uint32_t word = *reinterpret_cast<const uint32_t*>(b.Pq[p] + (e0 >> 1));
-  const float s = b.sP[p][e0 >> 6];
-  uint32_t pk[4];
+  while (p + 1 < b.n && i >= b.chunk_begin[p + 1]) ++p;
+  const int64_t e0 = (i - b.chunk_begin[p]) * 32;
+  const uint8_t* src = b.Pq[p] + (e0 >> 1);
+  uint32_t w[4];
+  if (kVec16) {
+    const uint4 v = *reinterpret_cast<const uint4*>(src);
+    w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
+  } else {
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int nib = static_cast<int>((word >> (4 * k)) & 0xFu);
-    const int code = (nib ^ 8) - 8;
-    const uint32_t bits = bf16_bits_rn(__fmul_rn(static_cast<float>(code), s));
-    if (k & 1)
-      pk[k >> 1] |= bits << 16;
-    else
-      pk[k >> 1] = bits;
+    for (int k = 0; k < 4; ++k) w[k] = reinterpret_cast<const uint32_t*>(src)[k];
   }
-  *reinterpret_cast<uint4*>(b.out[p] + e0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  const float s = b.sP[p][e0 >> 6];
+  uint32_t out[16];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    // nibble x ^ 8 is code + 8 in [1, 15]; 0x4B400000 | (code + 8) is the float
+    // 1.5 * 2^23 + code + 8, exact
+    const uint32_t f = w[k] ^ 0x88888888u;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float lo = __fsub_rn(__uint_as_float(0x4B400000u | ((f >> (8 * h)) & 0xFu)), 12582920.0f);
+      const float hi = __fsub_rn(__uint_as_float(0x4B400000u | ((f >> (8 * h + 4)) & 0xFu)), 12582920.0f);
+      const __nv_bfloat162 pr = __floats2bfloat162_rn(__fmul_rn(lo, s), __fmul_rn(hi, s));
+      out[4 * k + h] = *reinterpret_cast<const uint32_t*>(&pr);
+    }
+  }
+  uint4* dst = reinterpret_cast<uint4*>(b.out[p] + e0);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) dst[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
 }
 
 __global__ void philox_kernel(const uint32_t* c0, const uint32_t* c1, const uint32_t* c2, const uint32_t* c3,
@@ -713,10 +739,15 @@ static cudaError_t launch_dequant_batch(const DequantBatch& b, cudaStream_t stre
   if (chunks == 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (chunks + threads - 1) / threads;
-  const double total = chunks * 8.0;
+  const double total = chunks * 32.0;
   const double bytes = total / 2.0 + total / 64.0 * 4.0 + total * 2.0;
+  bool vec16 = true;
+  for (int i = 0; i < b.n; ++i) vec16 = vec16 && (reinterpret_cast<uintptr_t>(b.Pq[i]) % 16 == 0);
   const int tok = profile_begin(stream, QG_KERNEL_DEQUANT, 0.0, bytes);
-  dequant_projection_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(b);
+  if (vec16)
+    dequant_projection_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(b);
+  else
+    dequant_projection_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(b);
   profile_end(stream, tok);
   return cudaGetLastError();
 }
@@ -728,7 +759,7 @@ cudaError_t launch_dequant_projection(const uint8_t* Pq, const float* sP, int64_
   b.Pq[0] = Pq;
   b.sP[0] = sP;
   b.out[0] = out;
-  b.chunk_begin[1] = total / 8;
+  b.chunk_begin[1] = total / 32;
   b.n = 1;
   return launch_dequant_batch(b, stream);
 }
@@ -753,7 +784,7 @@ cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream
       db.Pq[i] = s.Pq;
       db.sP[i] = s.sP;
       db.out[i] = s.Pbf;
-      db.chunk_begin[i + 1] = db.chunk_begin[i] + static_cast<int64_t>(s.m) * s.r / 8;
+      db.chunk_begin[i + 1] = db.chunk_begin[i] + static_cast<int64_t>(s.m) * s.r / 32;
     }
     db.n = cnt;
     e = launch_dequant_batch(db, stream);
