@@ -5,7 +5,8 @@ Workload: a LLaMA-7B-shaped stack, 32 decoder layers x {q, k, v, o: 4096 x 4096;
 gate, up: 4096 x 11008; down: 11008 x 4096}, rank r = 1024: 224 weight matrices,
 6.48 G INT8 weights.  One step = the optimizer step a1..a5 on every matrix
 (dequantize INT4 P, R = P^T G, Adam on the INT8 moments, U = P N, stochastic
-rounding into INT8 W), issued as one batched call per decoder layer.  Inputs are
+rounding into INT8 W), issued as one batched call per decoder layer (three
+launches: the INT4 dequantization and two tcgen05 GEMMs).  Inputs are
 seeded synthetic bf16 gradients (rank-256 signal, s_i = 1e-2 * 0.97^i, noise
 sigma = 1e-4) resident in HBM (13 GB, far larger than L2).
 
@@ -68,23 +69,26 @@ def kernel_digest():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary of one
-    decoder layer (one launch = one layer batch, as here), or None when the
-    kernel sources changed since that capture."""
+def profiled_traffic(kernel, alg_bytes_per_launch):
+    """DRAM bytes per launch of `kernel`: the ratio of measured DRAM traffic to
+    algorithmic bytes in the committed ncu capture, times this run's
+    algorithmic bytes per launch.  The ratio is taken from one launch of
+    the same kernel, an 8-matrix batch of two decoder layers. Traffic grows in
+    proportion to the matrices in a launch. None when the kernel sources
+    changed since that capture."""
     try:
         text = open(PROFILE).read()
     except OSError:
         return None
-    digest = traffic = None
+    digest = ratio = None
     for line in text.splitlines():
         if line.startswith("kernel sources digest:"):
             digest = line.split(":", 1)[1].strip()
-        if line.startswith("traffic_per_launch_bytes:"):
-            traffic = dict(kv.split("=") for kv in line.split(":", 1)[1].split())
-    if digest != kernel_digest() or not traffic or kernel not in traffic:
+        if line.startswith("traffic_over_algorithmic:"):
+            ratio = dict(kv.split("=") for kv in line.split(":", 1)[1].split())
+    if digest != kernel_digest() or not ratio or kernel not in ratio:
         return None
-    return int(traffic[kernel])
+    return float(ratio[kernel]) * alg_bytes_per_launch
 
 
 def load_peaks():
@@ -247,14 +251,18 @@ class Stack:
                 group.append(dict(cfg=c, h=h, W=W, sW=sW, G=G, ldg=G.shape[1], state=state, m=m, n=n))
                 lid += 1
             self.layers.append(group)
-        # one workspace, reused by every decoder layer (they run in order on one stream)
+        # one batched call per decoder layer (its 7 matrices in one batch), or with
+        # QG_BENCH_WHOLE_STACK=1 one call for all matrices (batches of 8 inside the
+        # library); one workspace reused by every call
+        groups = [[e for group in self.layers for e in group]] if os.environ.get("QG_BENCH_WHOLE_STACK") == "1" \
+            else self.layers
         need = 0
-        for group in self.layers:
+        for group in groups:
             arr = (qg.POINTER(qg.qg_config) * len(group))(*[qg.ctypes.pointer(e["cfg"]) for e in group])
             need = max(need, qg.qg_step_batch_workspace_bytes(arr, len(group)))
         self.ws = torch.empty(need, dtype=torch.uint8, device=device)
         self.calls = []
-        for group in self.layers:
+        for group in groups:
             k = len(group)
             self.calls.append(((c_void_p * k)(*[e["h"].value for e in group]),
                                (c_void_p * k)(*[e["G"].data_ptr() for e in group]),
@@ -364,8 +372,8 @@ def run_ours(args, rank, world, local_rank):
                           "peaks": "burst bf16 %.1f TF/s, HBM %.1f GB/s (%s)" % (peaks["bf16_tflops"], peaks["hbm_gbs"],
                                                                               peaks["source"])},
         "roofline": {"bound": "tensor", "kernel": names[dom_k], "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic(names[dom_k]) if args.layers == 32 else None,
-                     "traffic_unit": "bytes per launch (ncu, one decoder layer)",
+                     "frac": achieved / peak, "traffic": profiled_traffic(names[dom_k], dom.bytes / dom.launches),
+                     "traffic_unit": "DRAM bytes per launch (ncu traffic/algorithmic ratio x this launch)",
                      "algorithmic_bytes_per_launch": dom.bytes / dom.launches,
                      "peak_kind": "sustained bf16 (%s)" % peaks["source"]},
         "kernels": kernels,
@@ -404,10 +412,10 @@ def run_e2e(stack, args, stream, world, device, barrier):
     d2h = 4 * len(views)
 
     def one():
-        i = 0
-        for (hs, gs, lds, k), group in zip(stack.calls, stack.layers):
+        for group in stack.layers:
             for e in group:
                 e["G"].copy_(host[tuple(e["G"].shape)], non_blocking=True)
+        for hs, gs, lds, k in stack.calls:
             st = qg.qg_step_batch(hs, gs, lds, k, stack.ws.data_ptr(), stack.ws.numel(), stream)
             if st != qg.QG_OK:
                 raise qg.QGError(st, "qg_step_batch")

@@ -145,9 +145,12 @@ qg_status qg_layer_set_projection(qg_layer* layer, const uint8_t* d_Pq, const fl
 qg_status qg_step(qg_layer* layer, const void* d_G, int64_t ldg, void* d_ws, size_t ws_bytes,
                   void* stream);
 
-/* The same step for `count` matrices in few launches (one persistent grid per
- * stage for up to 8 matrices).  d_ws must hold the sum of the matrices'
- * qg_step_workspace_bytes, each rounded up to 256. */
+/* The same step for `count` matrices in few launches: batches of up to 8
+ * matrices, three launches per batch (dequantize the batch's projections, then
+ * one persistent tcgen05 grid per GEMM stage), batches in order on `stream`.
+ * d_ws (256-byte aligned) must hold qg_step_batch_workspace_bytes of the same
+ * configurations in the same order: the largest batch's sum of
+ * qg_step_workspace_bytes, reused by every batch. */
 qg_status qg_step_batch(qg_layer* const* layers, const void* const* d_G, const int64_t* ldg,
                         int32_t count, void* d_ws, size_t ws_bytes, void* stream);
 size_t qg_step_batch_workspace_bytes(const qg_config* const* cfgs, int32_t count);

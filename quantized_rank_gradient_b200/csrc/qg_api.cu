@@ -5,6 +5,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <vector>
 
 #include "../../include/qgalore.h"
@@ -288,14 +289,29 @@ qg_status qg_step(qg_layer* L, const void* d_G, int64_t ldg, void* d_ws, size_t 
   return st;
 }
 
+// Batch workspace: the matrices go in batches of up to kBatch (one grid per
+// stage each), run in order on one stream, so every batch reuses one slot as
+// large as the largest batch's scratch.
+static constexpr int kBatch = 8;
+
+static size_t batch_slot_bytes(const int32_t* m, const int32_t* n, const int32_t* r, int count) {
+  size_t slot = 0;
+  for (int b = 0; b * kBatch < count; ++b) {
+    size_t sum = 0;
+    for (int i = b * kBatch; i < count && i < (b + 1) * kBatch; ++i) sum += qg::step_scratch_bytes(m[i], n[i], r[i]);
+    slot = std::max(slot, sum);
+  }
+  return slot;
+}
+
 size_t qg_step_batch_workspace_bytes(const qg_config* const* cfgs, int32_t count) {
   if (!cfgs || count < 0) return 0;
-  size_t total = 0;
+  std::vector<int32_t> m(count), n(count), r(count);
   for (int i = 0; i < count; ++i) {
     if (check_config(cfgs[i]) != QG_OK) return 0;
-    total += qg::step_scratch_bytes(cfgs[i]->m, cfgs[i]->n, cfgs[i]->r);
+    m[i] = cfgs[i]->m, n[i] = cfgs[i]->n, r[i] = cfgs[i]->r;
   }
-  return total;
+  return batch_slot_bytes(m.data(), n.data(), r.data(), count);
 }
 
 qg_status qg_step_batch(qg_layer* const* layers, const void* const* d_G, const int64_t* ldg, int32_t count,
@@ -303,20 +319,23 @@ qg_status qg_step_batch(qg_layer* const* layers, const void* const* d_G, const i
   if (count < 0 || (count > 0 && (!layers || !d_G || !ldg || !d_ws))) return QG_EINVAL;
   if (count == 0) return QG_OK;
   if (!aligned(d_ws, 256)) return QG_EALIGN;
-  size_t need = 0;
+  std::vector<int32_t> m(count), n(count), r(count);
   for (int i = 0; i < count; ++i) {
     qg_status st = check_step_args(layers[i], d_G[i], ldg[i]);
     if (st != QG_OK) return st;
     for (int j = 0; j < i; ++j)
       if (layers[j] == layers[i]) return QG_EINVAL;
-    need += qg::step_scratch_bytes(layers[i]->cfg.m, layers[i]->cfg.n, layers[i]->cfg.r);
+    m[i] = layers[i]->cfg.m, n[i] = layers[i]->cfg.n, r[i] = layers[i]->cfg.r;
   }
-  if (ws_bytes < need) return QG_ESTATE;
+  const size_t slot = batch_slot_bytes(m.data(), n.data(), r.data(), count);
+  if (ws_bytes < slot) return QG_ESTATE;
   std::vector<StepProblem> probs(count);
-  uint8_t* ws = static_cast<uint8_t*>(d_ws);
-  for (int i = 0; i < count; ++i) {
-    fill_step_problem(layers[i], d_G[i], ldg[i], ws, layers[i]->sched.t + 1, &probs[i]);
-    ws += qg::step_scratch_bytes(layers[i]->cfg.m, layers[i]->cfg.n, layers[i]->cfg.r);
+  for (int b = 0; b * kBatch < count; ++b) {
+    uint8_t* ws = static_cast<uint8_t*>(d_ws);
+    for (int i = b * kBatch; i < count && i < (b + 1) * kBatch; ++i) {
+      fill_step_problem(layers[i], d_G[i], ldg[i], ws, layers[i]->sched.t + 1, &probs[i]);
+      ws += qg::step_scratch_bytes(m[i], n[i], r[i]);
+    }
   }
   qg_status st = cuda_status(qg::launch_step(probs.data(), count, static_cast<cudaStream_t>(stream)));
   if (st == QG_OK)

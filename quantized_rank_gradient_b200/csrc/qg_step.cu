@@ -26,6 +26,13 @@
 #include "qg_internal.h"
 #include "qg_philox.cuh"
 #include "qg_refresh.h"
+
+#ifndef QG_SR_REVERSE
+#define QG_SR_REVERSE 1
+#endif
+#ifndef QG_DEQUANT_CHUNKS
+#define QG_DEQUANT_CHUNKS 2
+#endif
 #include "../../include/qgalore.h"
 
 namespace qg {
@@ -83,6 +90,14 @@ QG_DEV uint32_t round_to_byte(float x) { return __float_as_uint(__fadd_rn(x, kMa
 QG_DEV float max_nan_abs(float m, float x) {
   float r;
   asm("{\n\t.reg .f32 t;\n\tabs.f32 t, %2;\n\tmax.NaN.f32 %0, %1, t;\n\t}" : "=f"(r) : "f"(m), "f"(x));
+  return r;
+}
+
+// Both signed 16-bit lanes of x clamped to [-127, 127].
+QG_DEV uint32_t clamp127_s16x2(uint32_t x) {
+  uint32_t r;
+  asm("max.s16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0xFF81FF81u));
+  asm("min.s16x2 %0, %1, %2;" : "=r"(r) : "r"(r), "r"(0x007F007Fu));
   return r;
 }
 
@@ -411,30 +426,29 @@ struct StochRoundEpi {
   // and a NaN X keeps q.
   //
   // Fast form, valid while |X| < 2^22: fadd.rp(X, 1.5 * 2^23) has the bits
-  // 0x4B400000 + K; adding the draw less 2^22 and q * 2^16 gives
-  // 0x4B000000 + K + draw + q * 2^16, whose bits [16, 32) are 0x4B00 + q + r with
-  // r = floor((K + draw) / 2^16).  The clamp of q + r to [-127, 127] is a clamp
-  // of that sum, and its byte 2 is the new code.  When |X| reaches 2^22, or X is
-  // NaN, the chunk is redone in the general form.
+  // 0x4B400000 + K; adding the draw less 0x4B400000 and q * 2^16 leaves
+  // K + draw + q * 2^16, whose bits [16, 32) are q + r with
+  // r = floor((K + draw) / 2^16) (|q + r| <= 191).  Two such sums give one pair
+  // of 16-bit lanes, clamped to [-127, 127] by one max and one min on both
+  // lanes; the low bytes of four lanes are the four new codes.  When |X|
+  // reaches 2^22, or X is NaN, the chunk is redone in the general form.
   template <bool kOneFactor>
   static QG_DEV void sr_chunk(const uint32_t (&U)[32], const uint4& wa, const uint4& wb, const uint32_t (&d)[16],
                               float cp0, float cp1, int split, uint32_t (&out)[8]) {
-    constexpr int kLo = (0x4B00 - 127) << 16;
-    constexpr int kHi = ((0x4B00 + 127) << 16) | 0xFFFF;
     float mx = 0.f;
-    uint32_t S[4];
+    uint32_t sum[2], lanes[2];
 #pragma unroll
     for (int k = 0; k < 32; ++k) {
       const float cp = (kOneFactor || k < split) ? cp0 : cp1;
       const float X = __fmul_rn(__uint_as_float(U[k]), cp);
       mx = max_nan_abs(mx, X);
       const uint32_t tb = __float_as_uint(__fadd_ru(X, kMagic));
-      const uint32_t dq = prmt(d[k >> 1], 0xFFC00000u, (k & 1) ? 0x7632u : 0x7610u);
+      const uint32_t dq = prmt(d[k >> 1], 0xB4C00000u, (k & 1) ? 0x7632u : 0x7610u);
       const uint32_t wsel = 0x44u | (static_cast<uint32_t>(k & 3) << 8) | (static_cast<uint32_t>((k & 3) | 8) << 12);
       const uint32_t q16 = prmt(word_of(k < 16 ? wa : wb, (k >> 2) & 3), 0u, wsel);
-      const int sum = static_cast<int>(tb + dq + q16);
-      S[k & 3] = static_cast<uint32_t>(min(max(sum, kLo), kHi));
-      if ((k & 3) == 3) out[k >> 2] = prmt(prmt(S[0], S[1], 0x62u), prmt(S[2], S[3], 0x62u), 0x5410u);
+      sum[k & 1] = tb + dq + q16;
+      if (k & 1) lanes[(k >> 1) & 1] = clamp127_s16x2(prmt(sum[0], sum[1], 0x7632u));
+      if ((k & 3) == 3) out[k >> 2] = prmt(lanes[0], lanes[1], 0x6420u);
     }
     if (!(mx < 4194304.0f)) {
 #pragma unroll
@@ -583,40 +597,56 @@ struct DequantBatch {
   int32_t n;
 };
 
+constexpr int kDequantChunks = QG_DEQUANT_CHUNKS;  // 32-element chunks per thread, their loads issued together
+
 template <bool kVec16>
 __global__ void __launch_bounds__(256) dequant_projection_kernel(const __grid_constant__ DequantBatch b) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= b.chunk_begin[b.n]) return;
-  int p = 0;
-  while (p + 1 < b.n && i >= b.chunk_begin[p + 1]) ++p;
-  const int64_t e0 = (i - b.chunk_begin[p]) * 32;
-  const uint8_t* src = b.Pq[p] + (e0 >> 1);
-  uint32_t w[4];
-  if (kVec16) {
-    const uint4 v = *reinterpret_cast<const uint4*>(src);
-    w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
-  } else {
+  const int64_t total = b.chunk_begin[b.n];
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  uint32_t w[kDequantChunks][4];
+  float s[kDequantChunks];
+  uint16_t* dst[kDequantChunks];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) w[k] = reinterpret_cast<const uint32_t*>(src)[k];
-  }
-  const float s = b.sP[p][e0 >> 6];
-  uint32_t out[16];
+  for (int c = 0; c < kDequantChunks; ++c) {
+    const int64_t i = first + c * stride;
+    dst[c] = nullptr;
+    if (i >= total) continue;
+    int p = 0;
+    while (p + 1 < b.n && i >= b.chunk_begin[p + 1]) ++p;
+    const int64_t e0 = (i - b.chunk_begin[p]) * 32;
+    const uint8_t* src = b.Pq[p] + (e0 >> 1);
+    if (kVec16) {
+      const uint4 v = *reinterpret_cast<const uint4*>(src);
+      w[c][0] = v.x, w[c][1] = v.y, w[c][2] = v.z, w[c][3] = v.w;
+    } else {
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    // nibble x ^ 8 is code + 8 in [1, 15]; 0x4B400000 | (code + 8) is the float
-    // 1.5 * 2^23 + code + 8, exact
-    const uint32_t f = w[k] ^ 0x88888888u;
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const float lo = __fsub_rn(__uint_as_float(0x4B400000u | ((f >> (8 * h)) & 0xFu)), 12582920.0f);
-      const float hi = __fsub_rn(__uint_as_float(0x4B400000u | ((f >> (8 * h + 4)) & 0xFu)), 12582920.0f);
-      const __nv_bfloat162 pr = __floats2bfloat162_rn(__fmul_rn(lo, s), __fmul_rn(hi, s));
-      out[4 * k + h] = *reinterpret_cast<const uint32_t*>(&pr);
+      for (int k = 0; k < 4; ++k) w[c][k] = reinterpret_cast<const uint32_t*>(src)[k];
     }
+    s[c] = b.sP[p][e0 >> 6];
+    dst[c] = b.out[p] + e0;
   }
-  uint4* dst = reinterpret_cast<uint4*>(b.out[p] + e0);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) dst[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+  for (int c = 0; c < kDequantChunks; ++c) {
+    if (!dst[c]) continue;
+    uint32_t out[16];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      // nibble x ^ 8 is code + 8 in [1, 15]; 0x4B400000 | (code + 8) is the float
+      // 1.5 * 2^23 + code + 8, exact
+      const uint32_t f = w[c][k] ^ 0x88888888u;
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float lo = __fsub_rn(__uint_as_float(0x4B400000u | ((f >> (8 * h)) & 0xFu)), 12582920.0f);
+        const float hi = __fsub_rn(__uint_as_float(0x4B400000u | ((f >> (8 * h + 4)) & 0xFu)), 12582920.0f);
+        const __nv_bfloat162 pr = __floats2bfloat162_rn(__fmul_rn(lo, s[c]), __fmul_rn(hi, s[c]));
+        out[4 * k + h] = *reinterpret_cast<const uint32_t*>(&pr);
+      }
+    }
+    uint4* d = reinterpret_cast<uint4*>(dst[c]);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) d[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+  }
 }
 
 __global__ void philox_kernel(const uint32_t* c0, const uint32_t* c1, const uint32_t* c2, const uint32_t* c3,
@@ -738,7 +768,7 @@ static cudaError_t launch_dequant_batch(const DequantBatch& b, cudaStream_t stre
   const int64_t chunks = b.chunk_begin[b.n];
   if (chunks == 0) return cudaSuccess;
   const int threads = 256;
-  const int64_t blocks = (chunks + threads - 1) / threads;
+  const int64_t blocks = (chunks + int64_t(threads) * kDequantChunks - 1) / (int64_t(threads) * kDequantChunks);
   const double total = chunks * 32.0;
   const double bytes = total / 2.0 + total / 64.0 * 4.0 + total * 2.0;
   bool vec16 = true;
@@ -773,28 +803,28 @@ cudaError_t launch_philox(const uint32_t* c0, const uint32_t* c1, const uint32_t
   return cudaGetLastError();
 }
 
-cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream) {
-  cudaError_t e;
-  for (int base = 0; base < count; base += kMaxProblems) {
-    const int cnt = std::min(kMaxProblems, count - base);
-    DequantBatch db;
-    memset(&db, 0, sizeof(db));
-    for (int i = 0; i < cnt; ++i) {
-      const StepProblem& s = probs[base + i];
-      db.Pq[i] = s.Pq;
-      db.sP[i] = s.sP;
-      db.out[i] = s.Pbf;
-      db.chunk_begin[i + 1] = db.chunk_begin[i] + static_cast<int64_t>(s.m) * s.r / 32;
-    }
-    db.n = cnt;
-    e = launch_dequant_batch(db, stream);
-    if (e != cudaSuccess) return e;
+static cudaError_t launch_dequant_for(const StepProblem* probs, int cnt, cudaStream_t stream) {
+  DequantBatch db;
+  memset(&db, 0, sizeof(db));
+  for (int i = 0; i < cnt; ++i) {
+    const StepProblem& s = probs[i];
+    db.Pq[i] = s.Pq;
+    db.sP[i] = s.sP;
+    db.out[i] = s.Pbf;
+    db.chunk_begin[i + 1] = db.chunk_begin[i] + static_cast<int64_t>(s.m) * s.r / 32;
+  }
+  db.n = cnt;
+  return launch_dequant_batch(db, stream);
+}
 
+static cudaError_t launch_gemms_for(const StepProblem* probs, int cnt, cudaStream_t stream) {
+  cudaError_t e;
+  {
     GemmParams<AdamEpi> p1;
     memset(&p1, 0, sizeof(p1));
     double fl1 = 0, by1 = 0, fl2 = 0, by2 = 0;
     for (int i = 0; i < cnt; ++i) {
-      const StepProblem& s = probs[base + i];
+      const StepProblem& s = probs[i];
       const double m = s.m, n = s.n, r = s.r;
       fl1 += 2 * m * n * r;
       fl2 += 2 * m * n * r;
@@ -820,8 +850,15 @@ cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream
 
     GemmParams<StochRoundEpi> p2;
     memset(&p2, 0, sizeof(p2));
-    for (int i = 0; i < cnt; ++i) {
-      const StepProblem& s = probs[base + i];
+    // The batch's matrices in reverse order: the last N written by a2+a3 (and
+    // its P~, read last there) is the likeliest still in L2.
+    for (int ii = 0; ii < cnt; ++ii) {
+#if QG_SR_REVERSE
+      const int i = cnt - 1 - ii;
+#else
+      const int i = ii;
+#endif
+      const StepProblem& s = probs[i];
       GemmProblem<StochRoundEpi>& pr = p2.prob[p2.nprob];
       // A = P~ (M = m, K = r), K-major: box {64 (r), 128 (m)}
       if (!encode_map_bf16(&pr.tmA, s.Pbf, s.r, s.m, s.r, 64, 128)) return cudaErrorInvalidValue;
@@ -836,6 +873,16 @@ cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream
       add_problem(p2, s.m, s.n, s.r);
     }
     e = launch_gemm_pair<StochRoundEpi, false>(p2, stream, QG_KERNEL_BACKPROJECT_SR, fl2, by2);
+  }
+  return e;
+}
+
+cudaError_t launch_step(const StepProblem* probs, int count, cudaStream_t stream) {
+  for (int base = 0; base < count; base += kMaxProblems) {
+    const int cnt = std::min(kMaxProblems, count - base);
+    cudaError_t e = launch_dequant_for(probs + base, cnt, stream);
+    if (e != cudaSuccess) return e;
+    e = launch_gemms_for(probs + base, cnt, stream);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -183,8 +183,15 @@ def test_step_is_deterministic():
         np.testing.assert_array_equal(a, b)
 
 
-def test_step_batch_equals_single_steps():
-    shapes = [(512, 512, 128), (512, 1376, 128), (1376, 512, 128), (256, 256, 32)]
+BATCH_SHAPES = [(512, 512, 128), (512, 1376, 128), (1376, 512, 128), (256, 256, 32)]
+
+
+@pytest.mark.parametrize("shapes", [
+    BATCH_SHAPES,                                   # one batch
+    (BATCH_SHAPES * 3)[:11],                        # two batches sharing one workspace slot
+    (BATCH_SHAPES * 5)[:19] + [(300, 700, 64)],     # three batches
+])
+def test_step_batch_equals_single_steps(shapes):
     singles, batched, grads = [], [], []
     for i, (m, n, r) in enumerate(shapes):
         _, gl1, gen = make_layer(m, n, r, seed=10 + i, layer_id=i)
