@@ -48,6 +48,9 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=32, help="decoder layers (32 = the 7B stack)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["llama7b-stack", "refresh-stress"], default="llama7b-stack",
+                    help="refresh-stress: one 4096 x 11008 layer, r = 1024, a drifting gradient subspace, "
+                         "subspace refreshes on the layer-adaptive schedule (--steps defaults to 2000)")
     return ap.parse_args()
 
 
@@ -388,6 +391,78 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def run_refresh_stress(args, rank, world, local_rank):
+    """One 4096 x 11008 layer at r = 1024 over `steps` steps (2000 by default):
+    the gradient's rank-256 signal subspace (s_i = 1e-2 * 0.97^i, noise 1e-4)
+    turns by 0.02 rad per step until step 800, then stays.  Every step runs
+    qg_refresh (a randomized top-r SVD and CosSim when the layer is due; the
+    interval starts at 200 and doubles when CosSim > 0.4) and then qg_step, both
+    timed with CUDA events; the gradient is drawn outside the timed region."""
+    import torch
+    import quantized_rank_gradient_b200 as qg
+    import synth
+    qg.lib()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    steps = args.steps if args.steps != 20 else 2000
+    m, n, r = 4096, 11008, R_RANK
+    seed = 4_000_037 * (rank + 1)
+    c = qg.config(m, n, r, seed=seed, layer_id=0)
+    c.delta0, c.gamma = 200, 0.4
+    ldw = -(-n // 16) * 16
+    W = synth.device_weight_codes(m, n, ldw, seed, device)
+    sW = synth.device_weight_scales(m, n, seed, device)
+    gen = synth.DeviceDriftingGradient(m, n, 256, 1e-2, 0.97, 1e-4, 0.02, 800, seed, device)
+    cs = torch.cuda.current_stream()
+    stream = c_void_p(cs.cuda_stream)
+    state = torch.empty(qg.qg_state_bytes(byref(c)), dtype=torch.uint8, device=device)
+    h = c_void_p()
+    qg.check(qg.qg_layer_init(byref(h), byref(c), state.data_ptr(), state.numel(), W.data_ptr(), ldw,
+                              sW.data_ptr(), stream), "qg_layer_init")
+    ws = torch.empty(qg.qg_step_workspace_bytes(byref(c)), dtype=torch.uint8, device=device)
+    rws = torch.empty(qg.qg_refresh_workspace_bytes(byref(c)), dtype=torch.uint8, device=device)
+    info = qg.qg_refresh_info()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    refresh_ms, trace = [], []
+    clocks = ClockSampler(bus_id_of(device))
+    clocks.start()
+    for t in range(steps):
+        G = gen.draw(t)
+        e0, e1 = ev[t]
+        e0.record(cs)
+        qg.check(qg.qg_refresh(h, G.data_ptr(), G.shape[1], 1 if t == 0 else 0, rws.data_ptr(), rws.numel(),
+                               byref(info), stream), "qg_refresh")
+        qg.check(qg.qg_step(h, G.data_ptr(), G.shape[1], ws.data_ptr(), ws.numel(), stream), "qg_step")
+        e1.record(cs)
+        if info.refreshed:
+            trace.append({"t": t, "cossim": round(float(info.cossim), 4) if info.has_cossim else None,
+                          "delta": int(info.delta), "t_next": int(info.t_next)})
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    st = qg.qg_layer_status(h, stream)
+    ms = [a.elapsed_time(b) for a, b in ev]
+    for item in trace:
+        refresh_ms.append(ms[item["t"]])
+    total_ms = sum(ms)
+    plain = sorted(ms[t] for t in range(steps) if t not in {i["t"] for i in trace})
+    if rank != 0:
+        return 0
+    value = world * steps * m * n / (total_ms / 1000.0)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": 0,
+            "ms_per_step": total_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16/f32/int8", "data": "synthetic (drifting low-rank-plus-noise bf16 gradients)",
+            "config": {"workload": "refresh-stress-4096x11008-r1024", "steps": steps, "delta0": 200, "gamma": 0.4,
+                       "drift": "0.02 rad/step, frozen after step 800",
+                       "l2": "gradient redrawn every step outside the timed region"},
+            "refreshes": len(trace), "svd_fraction_vs_fixed_interval": len(trace) / max(1, -(-steps // 200)),
+            "refresh_ms": {"mean": sum(refresh_ms) / max(1, len(refresh_ms)), "max": max(refresh_ms or [0.0])},
+            "step_ms_median_without_refresh": plain[len(plain) // 2] if plain else None,
+            "cossim_trace": trace, "status": int(st), "clocks": clk}
+    print(json.dumps(line), flush=True)
+    qg.qg_layer_destroy(h)
+    return 0
+
+
 def run_e2e(stack, args, stream, world, device, barrier):
     import torch
     import torch.distributed as dist
@@ -461,6 +536,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.workload == "refresh-stress":
+            return run_refresh_stress(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:

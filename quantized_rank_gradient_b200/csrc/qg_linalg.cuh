@@ -3,10 +3,15 @@
 //   potrf_diag_kernel   Cholesky of one 32 x 32 diagonal block + its inverse
 //   trsm_panel_kernel   L[i, jb] = A[i, jb] * inv(L[jb, jb])^T below the block
 //   syrk_update_kernel  trailing update A -= L[:, jb] L[:, jb]^T (lower tiles)
+//   sgemm_batched_kernel  the same tiles over a batch of equal-size blocks
+//   trinv_init_kernel   block-diagonal start of L^-1 by recursive doubling
+//   split_bf16_kernel   float32 -> bf16 hi + lo parts (tensor-core operands)
 //   trsm_rows_kernel    X <- X L^-T for a tall X, 32 rows per CTA
-//   jacobi_kernel       one-sided (Hestenes) Jacobi on the columns of a square
-//                       matrix, round-robin pairs, one warp per pair, a bounded
-//                       grid barrier between rounds (cooperative launch)
+//   jacobi_kernel       block one-sided (Hestenes) Jacobi on the columns of a
+//                       square matrix: round-robin pairs of 16-column blocks, one
+//                       CTA per pair, the pair's 32 x 32 Gram diagonalised in
+//                       shared memory, a bounded grid barrier between rounds
+//                       (cooperative launch)
 #pragma once
 
 #include "qg_device.cuh"
@@ -88,48 +93,169 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const float* __restrict__ A,
   }
 }
 
+// Batched form: blockIdx.z selects the problem; operand and result pointers
+// advance by the given element strides, and each problem's M, N, K are clipped
+// to the rows that remain below `limit` (M, N, K = min(b, limit - z * step)).
+template <bool kTA, bool kTB>
+__global__ void __launch_bounds__(256) sgemm_batched_kernel(const float* A, int64_t lda, int64_t sa,
+                                                            const float* B, int64_t ldb, int64_t sb, float* C,
+                                                            int64_t ldc, int64_t sc, int b, int step, int limit,
+                                                            int mlead, int nlead, int klead, float alpha) {
+  // problem z: M rows start at z*step + mlead, N at z*step + nlead, K at z*step + klead
+  const int z = blockIdx.z;
+  const int base = z * step;
+  const int M = min(b, limit - (base + mlead)), N = min(b, limit - (base + nlead)), K = min(b, limit - (base + klead));
+  if (M <= 0 || N <= 0 || K <= 0) return;
+  __shared__ float As[kSgBK][kSgBM + 4];
+  __shared__ float Bs[kSgBK][kSgBN + 4];
+  A += z * sa;
+  B += z * sb;
+  C += z * sc;
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+  const int m0 = blockIdx.y * kSgBM, n0 = blockIdx.x * kSgBN;
+  if (m0 >= M || n0 >= N) return;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += kSgBK) {
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+      const int e = tid + l * 256;
+      int mi, kk;
+      if (kTA) {
+        kk = e >> 6;
+        mi = e & 63;
+      } else {
+        mi = e >> 4;
+        kk = e & 15;
+      }
+      const int gm = m0 + mi, gk = k0 + kk;
+      float v = 0.f;
+      if (gm < M && gk < K) v = kTA ? A[static_cast<int64_t>(gk) * lda + gm] : A[static_cast<int64_t>(gm) * lda + gk];
+      As[kk][mi] = v;
+      int ni;
+      if (kTB) {
+        ni = e >> 4;
+        kk = e & 15;
+      } else {
+        kk = e >> 6;
+        ni = e & 63;
+      }
+      const int gn = n0 + ni, gk2 = k0 + kk;
+      float w = 0.f;
+      if (gn < N && gk2 < K) w = kTB ? B[static_cast<int64_t>(gn) * ldb + gk2] : B[static_cast<int64_t>(gk2) * ldb + gn];
+      Bs[kk][ni] = w;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kSgBK; ++kk) {
+      float a[4], bb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bb[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = __fmaf_rn(a[i], bb[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int gm = m0 + ty * 4 + i;
+    if (gm >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int gn = n0 + tx * 4 + j;
+      if (gn < N) C[static_cast<int64_t>(gm) * ldc + gn] = alpha * acc[i][j];
+    }
+  }
+}
+
+// Li (k x k, stride ld) <- the block-diagonal of L^-1 from the 32 x 32 diagonal
+// block inverses (Linv, 1024 floats each), zero elsewhere.
+__global__ void trinv_init_kernel(float* Li, int64_t ld, int k, const float* Linv) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(k) * ld) return;
+  const int i = static_cast<int>(idx / ld), j = static_cast<int>(idx % ld);
+  float v = 0.f;
+  if (j < k && (i >> 5) == (j >> 5)) v = Linv[static_cast<int64_t>(i >> 5) * 1024 + (i & 31) * 32 + (j & 31)];
+  Li[idx] = v;
+}
+
+// float32 (rows x cols, stride ld) -> bf16 hi (= rn(x)) and lo (= rn(x - hi)),
+// stride ldb; Xlo may be null.
+__global__ void split_bf16_kernel(const float* X, int64_t ld, int rows, int cols, uint16_t* Xhi, uint16_t* Xlo,
+                                  int64_t ldb) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(rows) * ldb) return;
+  const int64_t i = idx / ldb, j = idx % ldb;
+  const float x = j < cols ? X[i * ld + j] : 0.f;
+  const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+  Xhi[idx] = __bfloat16_as_ushort(hi);
+  if (Xlo) Xlo[idx] = __bfloat16_as_ushort(__float2bfloat16_rn(__fsub_rn(x, __bfloat162float(hi))));
+}
+
 // ------------------------------------------------------------------ Cholesky
 
 // Cholesky of the nb x nb diagonal block at (j0, j0) of the lower triangle of A
 // (read from the lower triangle only), written back as L; its inverse (32 x 32,
-// lower, identity-padded) goes to Linv.  A pivot that is not positive (the
-// matrix is not numerically positive definite) raises *flag and is replaced by
-// a tiny positive value so that the factorisation stays finite.
-__global__ void __launch_bounds__(1024) potrf_diag_kernel(float* A, int64_t ld, int j0, int nb, float* Linv,
-                                                          int* flag) {
-  __shared__ float T[32][33];
-  __shared__ float X[32][33];
-  const int i = threadIdx.y, j = threadIdx.x;
-  float v = (i == j) ? 1.f : 0.f;
-  if (i < nb && j < nb && j <= i) v = A[static_cast<int64_t>(j0 + i) * ld + j0 + j];
-  T[i][j] = (j <= i) ? v : 0.f;
-  __syncthreads();
+// lower, identity-padded) goes to Linv.  One warp: lane j holds column j, and
+// the column being eliminated is broadcast by shuffles.  A pivot that is not
+// positive (the matrix is not numerically positive definite) raises *flag and is
+// replaced by a tiny positive value so that the factorisation stays finite.
+__global__ void __launch_bounds__(32) potrf_diag_kernel(float* A, int64_t ld, int j0, int nb, float* Linv,
+                                                        int* flag) {
+  __shared__ float Ls[32][33];
+  const int j = threadIdx.x;
+  float col[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    float v = (i == j) ? 1.f : 0.f;
+    if (i < nb && j < nb && j <= i) v = A[static_cast<int64_t>(j0 + i) * ld + j0 + j];
+    col[i] = (j <= i) ? v : 0.f;
+  }
+#pragma unroll
   for (int c = 0; c < 32; ++c) {
-    if (i == c && j == c) {
-      float d = T[c][c];
-      if (!(d > 0.f)) {
-        if (c < nb) atomicOr(flag, 1);
-        d = 1e-30f;
-      }
-      T[c][c] = sqrtf(d);
+    float d = __shfl_sync(0xFFFFFFFFu, col[c], c);
+    if (!(d > 0.f)) {
+      if (j == 0 && c < nb) atomicOr(flag, 1);
+      d = 1e-30f;
     }
-    __syncthreads();
-    if (j == c && i > c) T[i][c] = T[i][c] / T[c][c];
-    __syncthreads();
-    if (i > c && j > c && j <= i) T[i][j] = T[i][j] - T[i][c] * T[j][c];
-    __syncthreads();
-  }
-  if (i < nb && j < nb) A[static_cast<int64_t>(j0 + i) * ld + j0 + j] = (j <= i) ? T[i][j] : 0.f;
-  // inverse: column j of inv(T) by forward substitution (thread row 0 of each column)
-  if (i == 0) {
-    for (int r = 0; r < 32; ++r) {
-      float s = (r == j) ? 1.f : 0.f;
-      for (int t = j; t < r; ++t) s -= T[r][t] * X[t][j];
-      X[r][j] = (r >= j) ? s / T[r][r] : 0.f;
+    const float l = sqrtf(d);
+    if (j == c) {
+      col[c] = l;
+#pragma unroll
+      for (int i = c + 1; i < 32; ++i) col[i] = col[i] / l;
+    }
+    // broadcast column c (rows > c) and update the columns to its right:
+    // col_j[i] -= L[i][c] L[j][c] for i >= j > c; L[j][c] arrives at i == j,
+    // before any row i >= j needs it
+    float ljc = 0.f;
+#pragma unroll
+    for (int i = c + 1; i < 32; ++i) {
+      const float lic = __shfl_sync(0xFFFFFFFFu, col[i], c);
+      if (i == j) ljc = lic;
+      if (j > c && i >= j) col[i] = col[i] - lic * ljc;
     }
   }
-  __syncthreads();
-  Linv[i * 32 + j] = X[i][j];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    Ls[i][j] = col[i];
+    if (i < nb && j < nb) A[static_cast<int64_t>(j0 + i) * ld + j0 + j] = (j <= i) ? col[i] : 0.f;
+  }
+  __syncwarp();
+  // inverse: column j of inv(L) by forward substitution
+  float x[32];
+#pragma unroll
+  for (int r = 0; r < 32; ++r) {
+    float s = (r == j) ? 1.f : 0.f;
+#pragma unroll
+    for (int t = 0; t < r; ++t) s -= Ls[r][t] * x[t];
+    x[r] = (r >= j) ? s / Ls[r][r] : 0.f;
+  }
+#pragma unroll
+  for (int r = 0; r < 32; ++r) Linv[r * 32 + j] = x[r];
 }
 
 // L[i, j0 + c] = sum_c' A[i, j0 + c'] Linv[c][c'] for rows i >= j0 + 32.
@@ -270,66 +396,320 @@ QG_DEV bool grid_barrier(unsigned* bar, unsigned nblocks, uint32_t* status) {
   return ok_s != 0;
 }
 
-// One-sided Jacobi: rotates pairs of columns of A (k x k, stored transposed:
-// row p of At is column p of A, stride ld) until every pair is orthogonal to
-// |a_p . a_q| <= tol * |a_p| |a_q|; applies the same rotations to V (rows of
-// Vt) when Vt is non-null.  Round-robin pairing (player 0 fixed, the others
-// rotate): every pair meets once per sweep of kk - 1 rounds (kk = k rounded up
-// to even; the dummy player pairs with nobody).  bar[3] counts the rotations of
-// the current sweep.  Stops after a sweep with no rotation or max_sweeps.
+// Block one-sided (Hestenes) Jacobi on the columns of a square matrix A
+// (k x k, stored transposed: row p of At is column p of A, stride ld), applying
+// the same rotations to V (rows of Vt) when Vt is non-null.
+//
+// The columns are grouped in blocks of kBJW; a round-robin tournament pairs the
+// blocks (player 0 fixed, the others rotate; an odd count gets a dummy player),
+// so that every pair of blocks meets once per sweep of nb - 1 rounds.  For a
+// pair, one CTA forms the Gram matrix M of its 2 kBJW columns (streaming the
+// columns through shared memory), and unless every off-diagonal entry already
+// satisfies |M_pq| <= tol sqrt(M_pp M_qq), diagonalises M = J L J^T by cyclic
+// two-sided Jacobi in shared memory and replaces the columns by A J (and V J).
+// The pair's columns are then mutually orthogonal.  Rounds are separated by a
+// bounded grid barrier (cooperative launch); bar[3] counts the pairs rotated in
+// the current sweep, and the solve stops after a sweep without rotation or
+// after max_sweeps.  At convergence the columns of A are orthogonal: for A = S
+// symmetric positive semi-definite, V holds eigenvectors and the column norms
+// are the eigenvalues; for any A they are its singular values.
+constexpr int kBJW = 16;           // columns per block
+constexpr int kBJP = 2 * kBJW;     // columns per block pair
+constexpr int kBJChunk = 128;      // column entries streamed per pass
+constexpr int kBJInnerSweeps = 1;  // one inner sweep per pair: the outer sweeps converge as fast
+constexpr float kBJInnerTol = 1e-7f;
+
+struct BJShared {
+  float X[kBJP][kBJChunk + 1];
+  float M[kBJP][kBJP + 1];
+  float T[kBJP][kBJP + 1];
+  float J[kBJP][kBJP + 1];
+  float JT[kBJP][kBJP + 1];
+  float c[kBJP / 2], s[kBJP / 2];
+  int pp[kBJP / 2], qq[kBJP / 2];  // the pairs of the current inner step
+  int part[kBJP];                  // pair index of each column, + kBJP for the second member
+  int rotate;
+};
+
+// J <- J (3 I - J^T J) / 2: one Newton-Schulz step back towards orthogonality
+// (the float32 product of the inner rotations drifts by a few ulps per rotation,
+// and every application of J would carry that drift into the column norms).
+QG_DEV void bj_reorthogonalize(BJShared& sh) {
+  __syncthreads();
+  for (int e = threadIdx.x; e < kBJP * kBJP; e += blockDim.x) {
+    const int i = e / kBJP, j = e % kBJP;
+    float g = 0.f;
+#pragma unroll 8
+    for (int l = 0; l < kBJP; ++l) g = __fmaf_rn(sh.J[l][i], sh.J[l][j], g);
+    sh.T[i][j] = g;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < kBJP * kBJP; e += blockDim.x) {
+    const int i = e / kBJP, j = e % kBJP;
+    float h = 0.f;
+#pragma unroll 8
+    for (int l = 0; l < kBJP; ++l) h = __fmaf_rn(sh.J[i][l], sh.T[l][j], h);
+    sh.JT[i][j] = __fmaf_rn(-0.5f, h, 1.5f * sh.J[i][j]);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < kBJP * kBJP; e += blockDim.x) sh.J[e / kBJP][e % kBJP] = sh.JT[e / kBJP][e % kBJP];
+  __syncthreads();
+}
+
+// Rows of At (or Vt) belonging to the pair: local l -> global row, or -1.
+QG_DEV int bj_row(int l, int I, int Jb, int k) {
+  const int g = l < kBJW ? I * kBJW + l : Jb * kBJW + (l - kBJW);
+  return g < k ? g : -1;
+}
+
+// Loads columns [c0, c0 + kBJChunk) of the pair's rows into X (0 outside).
+QG_DEV void bj_load(BJShared& sh, const float* Mat, int64_t ld, int I, int Jb, int k, int c0) {
+  for (int e = threadIdx.x; e < kBJP * kBJChunk; e += blockDim.x) {
+    const int l = e / kBJChunk, cc = e % kBJChunk;
+    const int g = bj_row(l, I, Jb, k);
+    sh.X[l][cc] = (g >= 0 && c0 + cc < k) ? __ldcg(Mat + static_cast<int64_t>(g) * ld + c0 + cc) : 0.f;
+  }
+}
+
+// rows <- J^T rows for the pair's rows of Mat (new row i = sum_l J[l][i] row_l).
+QG_DEV void bj_apply(BJShared& sh, float* Mat, int64_t ld, int I, int Jb, int k) {
+  const int cc = threadIdx.x % kBJChunk, ig = threadIdx.x / kBJChunk;  // 2 groups of 16 rows (256 threads)
+  for (int c0 = 0; c0 < k; c0 += kBJChunk) {
+    __syncthreads();
+    bj_load(sh, Mat, ld, I, Jb, k, c0);
+    __syncthreads();
+    float out[kBJP / 2];
+#pragma unroll
+    for (int u = 0; u < kBJP / 2; ++u) out[u] = 0.f;
+#pragma unroll 4
+    for (int l = 0; l < kBJP; ++l) {
+      const float x = sh.X[l][cc];
+#pragma unroll
+      for (int u = 0; u < kBJP / 2; ++u) out[u] = __fmaf_rn(sh.J[l][ig * (kBJP / 2) + u], x, out[u]);
+    }
+    if (c0 + cc < k) {
+#pragma unroll
+      for (int u = 0; u < kBJP / 2; ++u) {
+        const int g = bj_row(ig * (kBJP / 2) + u, I, Jb, k);
+        if (g >= 0) __stcg(Mat + static_cast<int64_t>(g) * ld + c0 + cc, out[u]);
+      }
+    }
+  }
+}
+
+// ---- resident variant: the pair's 2 kBJW rows live in shared memory (one
+// asynchronous load per pass), for k up to kBJResidentMaxK.
+constexpr int kBJResidentMaxK = 1536;
+
+// Row stride (floats) of the resident tile: a multiple of 4 that is 4 mod 32, so
+// that 16-byte reads of the same column by rows 0..31 spread over all banks.
+__host__ __device__ inline int bj_resident_stride(int k) {
+  int kp = (k + 3) / 4 * 4;
+  return kp + ((4 - kp % 32) + 32) % 32;
+}
+
+QG_DEV void cp_async16(void* smem, const void* gmem, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem), "r"(src_bytes)
+               : "memory");
+}
+QG_DEV void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// X (2 kBJW rows x kp) <- the pair's rows of Mat, zero outside the matrix.
+QG_DEV void bj_load_resident(float* X, int kp, const float* Mat, int64_t ld, int I, int Jb, int k) {
+  const int quads = kp / 4;
+  for (int e = threadIdx.x; e < kBJP * quads; e += blockDim.x) {
+    const int l = e / quads, c = (e % quads) * 4;
+    const int g = bj_row(l, I, Jb, k);
+    const int valid = (g >= 0 && c < k) ? min(4, k - c) : 0;
+    const float* src = Mat + (g >= 0 ? static_cast<int64_t>(g) * ld : 0) + (valid ? c : 0);
+    cp_async16(X + l * kp + c, src, valid * 4);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+}
+
+// rows of Mat <- J^T X (new row i = sum_l J[l][i] X[l]), 4 columns x 8 rows per
+// thread and pass.
+QG_DEV void bj_apply_resident(const BJShared& sh, const float* X, int kp, float* Mat, int64_t ld, int I, int Jb,
+                              int k) {
+  constexpr int kRows = kBJP / 4;
+  const int quads = kp / 4;
+  const int ig = threadIdx.x / 64, cq0 = threadIdx.x % 64;
+  for (int cq = cq0; cq < quads; cq += 64) {
+    const int c = cq * 4;
+    if (c >= k) break;
+    float4 out[kRows];
+#pragma unroll
+    for (int u = 0; u < kRows; ++u) out[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int l = 0; l < kBJP; ++l) {
+      const float4 x = *reinterpret_cast<const float4*>(X + l * kp + c);
+#pragma unroll
+      for (int u = 0; u < kRows; ++u) {
+        const float j = sh.J[l][ig * kRows + u];
+        out[u].x = __fmaf_rn(j, x.x, out[u].x);
+        out[u].y = __fmaf_rn(j, x.y, out[u].y);
+        out[u].z = __fmaf_rn(j, x.z, out[u].z);
+        out[u].w = __fmaf_rn(j, x.w, out[u].w);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kRows; ++u) {
+      const int g = bj_row(ig * kRows + u, I, Jb, k);
+      if (g < 0) continue;
+      float* dst = Mat + static_cast<int64_t>(g) * ld + c;
+      if (c + 4 <= k) {
+        __stcg(reinterpret_cast<float4*>(dst), out[u]);
+      } else {
+        __stcg(dst, out[u].x);
+        if (c + 1 < k) __stcg(dst + 1, out[u].y);
+        if (c + 2 < k) __stcg(dst + 2, out[u].z);
+      }
+    }
+  }
+}
+
+template <bool kResident>
 __global__ void __launch_bounds__(256) jacobi_kernel(float* At, float* Vt, int64_t ld, int k, int max_sweeps,
                                                      float tol, unsigned* bar, int* sweeps_out, uint32_t* status) {
-  const int lane = threadIdx.x & 31;
-  const int warps_per_block = blockDim.x >> 5;
-  const int gwarp = blockIdx.x * warps_per_block + (threadIdx.x >> 5);
-  const int nwarps = gridDim.x * warps_per_block;
-  const int kk = (k + 1) & ~1;
+  __shared__ BJShared sh;
+  extern __shared__ float4 dyn_smem[];
+  float* Xr = reinterpret_cast<float*>(dyn_smem);
+  const int kp = bj_resident_stride(k);
+  const int tid = threadIdx.x;
+  const int nblk = (k + kBJW - 1) / kBJW;
+  const int nb = nblk + (nblk & 1);
+  const int npairs = nb / 2;
   unsigned* rot = bar + 3;
   int sweep = 0;
   for (; sweep < max_sweeps; ++sweep) {
-    for (int round = 0; round < kk - 1; ++round) {
-      for (int idx = gwarp; idx < kk / 2; idx += nwarps) {
-        const int a = idx, b = kk - 1 - idx;
-        const int p = (a == 0) ? 0 : ((a - 1 + round) % (kk - 1)) + 1;
-        const int q = ((b - 1 + round) % (kk - 1)) + 1;
-        if (p >= k || q >= k) continue;
-        float* ap = At + static_cast<int64_t>(p) * ld;
-        float* aq = At + static_cast<int64_t>(q) * ld;
-        float al = 0.f, be = 0.f, ga = 0.f;
-        // columns are rewritten by other SMs between rounds: bypass L1
-        for (int t = lane; t < k; t += 32) {
-          const float x = __ldcg(ap + t), y = __ldcg(aq + t);
-          al = __fmaf_rn(x, x, al);
-          be = __fmaf_rn(y, y, be);
-          ga = __fmaf_rn(x, y, ga);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          al += __shfl_xor_sync(0xFFFFFFFFu, al, o);
-          be += __shfl_xor_sync(0xFFFFFFFFu, be, o);
-          ga += __shfl_xor_sync(0xFFFFFFFFu, ga, o);
-        }
-        if (!(fabsf(ga) > tol * sqrtf(al) * sqrtf(be))) continue;
-        const float zeta = (be - al) / (2.f * ga);
-        const float tt = fabsf(zeta) < 1e18f ? copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta))
-                                             : 0.5f / zeta;
-        const float c = 1.f / sqrtf(1.f + tt * tt);
-        const float s = c * tt;
-        for (int t = lane; t < k; t += 32) {
-          const float x = __ldcg(ap + t), y = __ldcg(aq + t);
-          __stcg(ap + t, c * x - s * y);
-          __stcg(aq + t, s * x + c * y);
-        }
-        if (Vt) {
-          float* vp = Vt + static_cast<int64_t>(p) * ld;
-          float* vq = Vt + static_cast<int64_t>(q) * ld;
-          for (int t = lane; t < k; t += 32) {
-            const float x = __ldcg(vp + t), y = __ldcg(vq + t);
-            __stcg(vp + t, c * x - s * y);
-            __stcg(vq + t, s * x + c * y);
+    for (int round = 0; round < nb - 1; ++round) {
+      for (int pidx = blockIdx.x; pidx < npairs; pidx += gridDim.x) {
+        const int a = pidx, b = nb - 1 - pidx;
+        const int I = (a == 0) ? 0 : ((a - 1 + round) % (nb - 1)) + 1;
+        const int Jb = ((b - 1 + round) % (nb - 1)) + 1;
+        if (I >= nblk || Jb >= nblk) continue;  // paired with the dummy player
+        // ---- Gram matrix of the pair's columns (2 x 2 outputs per thread)
+        const int ty = tid >> 4, tx = tid & 15;
+        float g00 = 0.f, g01 = 0.f, g10 = 0.f, g11 = 0.f;
+        if (kResident) {
+          __syncthreads();
+          bj_load_resident(Xr, kp, At, ld, I, Jb, k);
+          const float* ra0 = Xr + (2 * ty) * kp;
+          const float* ra1 = ra0 + kp;
+          const float* rb0 = Xr + (2 * tx) * kp;
+          const float* rb1 = rb0 + kp;
+#pragma unroll 4
+          for (int c = 0; c < kp; c += 4) {
+            const float4 a0 = *reinterpret_cast<const float4*>(ra0 + c), a1 = *reinterpret_cast<const float4*>(ra1 + c);
+            const float4 b0 = *reinterpret_cast<const float4*>(rb0 + c), b1 = *reinterpret_cast<const float4*>(rb1 + c);
+            g00 = __fmaf_rn(a0.x, b0.x, __fmaf_rn(a0.y, b0.y, __fmaf_rn(a0.z, b0.z, __fmaf_rn(a0.w, b0.w, g00))));
+            g01 = __fmaf_rn(a0.x, b1.x, __fmaf_rn(a0.y, b1.y, __fmaf_rn(a0.z, b1.z, __fmaf_rn(a0.w, b1.w, g01))));
+            g10 = __fmaf_rn(a1.x, b0.x, __fmaf_rn(a1.y, b0.y, __fmaf_rn(a1.z, b0.z, __fmaf_rn(a1.w, b0.w, g10))));
+            g11 = __fmaf_rn(a1.x, b1.x, __fmaf_rn(a1.y, b1.y, __fmaf_rn(a1.z, b1.z, __fmaf_rn(a1.w, b1.w, g11))));
           }
         }
-        if (lane == 0) atomicAdd(rot, 1u);
+        for (int c0 = 0; !kResident && c0 < k; c0 += kBJChunk) {
+          __syncthreads();
+          bj_load(sh, At, ld, I, Jb, k, c0);
+          __syncthreads();
+#pragma unroll 8
+          for (int cc = 0; cc < kBJChunk; ++cc) {
+            const float a0 = sh.X[2 * ty][cc], a1 = sh.X[2 * ty + 1][cc];
+            const float b0 = sh.X[2 * tx][cc], b1 = sh.X[2 * tx + 1][cc];
+            g00 = __fmaf_rn(a0, b0, g00);
+            g01 = __fmaf_rn(a0, b1, g01);
+            g10 = __fmaf_rn(a1, b0, g10);
+            g11 = __fmaf_rn(a1, b1, g11);
+          }
+        }
+        sh.M[2 * ty][2 * tx] = g00;
+        sh.M[2 * ty][2 * tx + 1] = g01;
+        sh.M[2 * ty + 1][2 * tx] = g10;
+        sh.M[2 * ty + 1][2 * tx + 1] = g11;
+        if (tid == 0) sh.rotate = 0;
+        __syncthreads();
+        // ---- already orthogonal to tol?
+        for (int e = tid; e < kBJP * kBJP; e += blockDim.x) {
+          const int p = e / kBJP, q = e % kBJP;
+          if (p < q && fabsf(sh.M[p][q]) > tol * sqrtf(sh.M[p][p]) * sqrtf(sh.M[q][q])) sh.rotate = 1;
+        }
+        __syncthreads();
+        if (!sh.rotate) continue;
+        // ---- M = J L J^T by cyclic Jacobi (parallel ordering of the 2 kBJW columns)
+        for (int e = tid; e < kBJP * kBJP; e += blockDim.x) sh.J[e / kBJP][e % kBJP] = (e / kBJP == e % kBJP) ? 1.f : 0.f;
+        for (int is = 0; is < kBJInnerSweeps; ++is) {
+          __syncthreads();
+          if (tid == 0) sh.rotate = 0;
+          __syncthreads();
+          for (int step = 0; step < kBJP - 1; ++step) {
+            if (tid < kBJP / 2) {
+              const int aa = tid, bb = kBJP - 1 - tid;
+              const int p = (aa == 0) ? 0 : ((aa - 1 + step) % (kBJP - 1)) + 1;
+              const int q = ((bb - 1 + step) % (kBJP - 1)) + 1;
+              const float al = sh.M[p][p], be = sh.M[q][q], ga = sh.M[p][q];
+              float c = 1.f, sn = 0.f;
+              if (fabsf(ga) > kBJInnerTol * sqrtf(al) * sqrtf(be)) {
+                const float zeta = (be - al) / (2.f * ga);
+                const float t = fabsf(zeta) < 1e18f ? copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta))
+                                                    : 0.5f / zeta;
+                c = 1.f / sqrtf(1.f + t * t);
+                sn = c * t;
+                sh.rotate = 1;
+              }
+              sh.c[tid] = c;
+              sh.s[tid] = sn;
+              sh.pp[tid] = p;
+              sh.qq[tid] = q;
+              sh.part[p] = tid;
+              sh.part[q] = tid + kBJP;
+            }
+            __syncthreads();
+            // columns: (M, J) <- (M, J) R
+            for (int e = tid; e < kBJP * kBJP; e += blockDim.x) {
+              const int i = e / kBJP, j = e % kBJP;
+              const int pa = sh.part[j], pr = pa & (kBJP - 1);
+              const int p = sh.pp[pr], q = sh.qq[pr];
+              const float c = sh.c[pr], sn = sh.s[pr];
+              if (pa >= kBJP) {
+                sh.T[i][j] = __fmaf_rn(sn, sh.M[i][p], c * sh.M[i][q]);
+                sh.JT[i][j] = __fmaf_rn(sn, sh.J[i][p], c * sh.J[i][q]);
+              } else {
+                sh.T[i][j] = __fmaf_rn(c, sh.M[i][p], -sn * sh.M[i][q]);
+                sh.JT[i][j] = __fmaf_rn(c, sh.J[i][p], -sn * sh.J[i][q]);
+              }
+            }
+            __syncthreads();
+            // rows: M <- R^T M
+            for (int e = tid; e < kBJP * kBJP; e += blockDim.x) {
+              const int i = e / kBJP, j = e % kBJP;
+              const int pa = sh.part[i], pr = pa & (kBJP - 1);
+              const int p = sh.pp[pr], q = sh.qq[pr];
+              const float c = sh.c[pr], sn = sh.s[pr];
+              sh.M[i][j] = pa >= kBJP ? __fmaf_rn(sn, sh.T[p][j], c * sh.T[q][j])
+                                      : __fmaf_rn(c, sh.T[p][j], -sn * sh.T[q][j]);
+              sh.J[i][j] = sh.JT[i][j];
+            }
+            __syncthreads();
+          }
+          if (!sh.rotate) break;
+        }
+        bj_reorthogonalize(sh);
+        // ---- the pair's columns (and V's) become A J
+        if (kResident) {
+          bj_apply_resident(sh, Xr, kp, At, ld, I, Jb, k);
+          if (Vt) {
+            __syncthreads();
+            bj_load_resident(Xr, kp, Vt, ld, I, Jb, k);
+            bj_apply_resident(sh, Xr, kp, Vt, ld, I, Jb, k);
+          }
+        } else {
+          bj_apply(sh, At, ld, I, Jb, k);
+          if (Vt) bj_apply(sh, Vt, ld, I, Jb, k);
+        }
+        if (tid == 0) atomicAdd(rot, 1u);
       }
       if (!grid_barrier(bar, gridDim.x, status)) return;
     }

@@ -7,7 +7,8 @@
 // Q = orth(Y); q times { Z = orth(G^T Q); Q = orth(G Z) }; B = Q^T G;
 // S = B B^T = V diag(lambda) V^T; P = Q V[:, top r].  The products with G run on
 // the tcgen05 core (bf16 operands, fp32 accumulation); orth() is shifted
-// Cholesky-QR in three passes (Fukaya et al. 2020) with fp32 SIMT Gram matrices;
+// Cholesky-QR in three passes (Fukaya et al. 2020) with fp32 SIMT Gram matrices
+// and X L^-T formed on the tensor cores from the explicit inverse;
 // the k x k eigenproblem and the r x r singular values of CosSim use a one-sided
 // Jacobi with a bounded grid barrier.  Then: sign canonicalisation, INT4
 // quantization, and CosSim(P_new, P_prev) = (1/r) sum_i sigma_i(P_new^T P_prev)
@@ -28,13 +29,17 @@ namespace {
 constexpr float kAbsmaxFloorR = 7.52316384526264e-37f;  // 2^-120
 constexpr uint32_t kOmegaSalt = 0x52454652u;
 constexpr int kJacobiMaxSweeps = 30;
-constexpr float kJacobiTol = 2e-6f;
+// Columns count as orthogonal once |a_p . a_q| <= tol |a_p| |a_q|; float32 dot
+// products of length ~1000 carry relative noise of a few 1e-6, so the bound
+// sits above that.
+constexpr float kJacobiTol = 1e-5f;
 
 size_t r256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct RefreshLayout {
   int k, ldk, ldn4;
-  size_t P, omega, Y, Yb, Ylo, Z, Zb, gram, linv, Bm, At, Vt, lam, perm, Vsel, Pa, Pb, Ct, misc, total;
+  size_t P, omega, Y, Yb, Ylo, Z, Zb, Zlo, gram, linv, Li, Tt, Lih, Lil, Bm, At, Vt, lam, perm, Vsel, Pa, Pb, Ct, misc,
+      total;
 };
 
 RefreshLayout refresh_layout(int m, int n, int r, int p) {
@@ -56,8 +61,13 @@ RefreshLayout refresh_layout(int m, int n, int r, int p) {
   L.Ylo = take(size_t(m) * ldk * 2);
   L.Z = take(size_t(n) * ldk * 4);
   L.Zb = take(size_t(n) * ldk * 2);
+  L.Zlo = take(size_t(n) * ldk * 2);
   L.gram = take(k * ldk * 4);
   L.linv = take(((k + 31) / 32) * 1024 * 4);
+  L.Li = take(k * ldk * 4);
+  L.Tt = take(k * ldk * 4);
+  L.Lih = take(k * ldk * 2);
+  L.Lil = take(k * ldk * 2);
   L.Bm = take(k * L.ldn4 * 4);
   L.At = take(k * ldk * 4);
   L.Vt = take(k * ldk * 4);
@@ -255,7 +265,7 @@ cudaError_t sgemm(bool ta, bool tb, const float* A, int64_t lda, const float* B,
 cudaError_t cholesky(float* A, int64_t ld, int k, float* Linv, int* flag, cudaStream_t s) {
   for (int j0 = 0; j0 < k; j0 += 32) {
     const int nb = std::min(32, k - j0);
-    potrf_diag_kernel<<<1, dim3(32, 32), 0, s>>>(A, ld, j0, nb, Linv + static_cast<size_t>(j0 / 32) * 1024, flag);
+    potrf_diag_kernel<<<1, 32, 0, s>>>(A, ld, j0, nb, Linv + static_cast<size_t>(j0 / 32) * 1024, flag);
     const int rest = k - j0 - 32;
     if (rest > 0) {
       const int T = (rest + 31) / 32;
@@ -266,38 +276,70 @@ cudaError_t cholesky(float* A, int64_t ld, int k, float* Linv, int* flag, cudaSt
   return cudaGetLastError();
 }
 
-cudaError_t trsm_rows(float* X, int64_t ldx, uint16_t* Xb, uint16_t* Xlo, int64_t ldb, int rows, int k,
-                      const float* L, int64_t ldl, const float* Linv, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(32) * (k + 1) * sizeof(float);
-  static size_t smem_set = 0;
-  if (smem > smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(trsm_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    smem_set = smem;
+// Li <- L^-1 for the lower Cholesky factor L (k x k, stride ld, lower triangle
+// of `Lf`), by recursive doubling from the 32 x 32 diagonal-block inverses:
+// for blocks [A 0; C B] already inverted on the diagonal,
+// the off-diagonal block of the inverse is -B^-1 (C A^-1).  Tt is k x ld scratch.
+cudaError_t tri_inverse(const float* Lf, float* Li, float* Tt, int64_t ld, int k, const float* linv, cudaStream_t s) {
+  const int64_t cnt = int64_t(k) * ld;
+  trinv_init_kernel<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, s>>>(Li, ld, k, linv);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  for (int b = 32; b < k; b *= 2) {
+    const int step = 2 * b;
+    const int pairs = (k + step - 1) / step;
+    const dim3 grid((b + kSgBN - 1) / kSgBN, (b + kSgBM - 1) / kSgBM, pairs);
+    const int64_t st = int64_t(step) * ld + step;
+    // T = C A^-1   (C = L[base + b.., base..], A^-1 = Li[base.., base..])
+    sgemm_batched_kernel<false, false><<<grid, 256, 0, s>>>(Lf + int64_t(b) * ld, ld, st, Li, ld, st,
+                                                            Tt + int64_t(b) * ld, ld, st, b, step, k, b, 0, 0, 1.f);
+    // Li[base + b.., base..] = -B^-1 T   (B^-1 = Li[base + b.., base + b..])
+    sgemm_batched_kernel<false, false><<<grid, 256, 0, s>>>(Li + int64_t(b) * ld + b, ld, st, Tt + int64_t(b) * ld, ld,
+                                                            st, Li + int64_t(b) * ld, ld, st, b, step, k, b, 0, b,
+                                                            -1.f);
   }
-  trsm_rows_kernel<<<(rows + 31) / 32, 256, smem, s>>>(X, ldx, Xb, Xlo, ldb, rows, k, L, ldl, Linv);
   return cudaGetLastError();
 }
 
-// Shifted Cholesky-QR, three passes: X (rows x k fp32, stride ld) becomes an
-// orthonormal basis of its column span; Xb receives its bf16 copy and Xlo (if
-// non-null) the bf16 residual.
-cudaError_t orth(float* X, uint16_t* Xb, uint16_t* Xlo, int rows, int k, int64_t ld, float* gram, float* linv,
-                 int* flag, cudaStream_t s) {
+struct OrthBufs {
+  float* gram;
+  float* linv;
+  float* Li;
+  float* Tt;
+  uint16_t* Lih;
+  uint16_t* Lil;
+  int* flag;
+};
+
+// Shifted Cholesky-QR, three passes (Fukaya et al. 2020): X (rows x k fp32,
+// stride ld) becomes an orthonormal basis of its column span.  Each pass: Gram
+// matrix in float32 (SIMT), Cholesky L L^T, the explicit inverse L^-1, then
+// X <- X L^-T on the tensor cores with bf16 hi + lo parts of both operands
+// (three products, fp32 accumulation, about 16 significant bits per pass; the
+// next pass corrects the residual).  On return Xb and Xlo hold the bf16 hi and
+// lo parts of the result (both are also used as scratch).
+cudaError_t orth(float* X, uint16_t* Xb, uint16_t* Xlo, int rows, int k, int64_t ld, const OrthBufs& ob,
+                 cudaStream_t s) {
   cudaError_t e;
+  const int64_t xcnt = int64_t(rows) * ld, lcnt = int64_t(k) * ld;
   for (int pass = 0; pass < 3; ++pass) {
-    if ((e = sgemm(true, false, X, ld, X, ld, gram, ld, k, k, rows, s)) != cudaSuccess) return e;
+    if ((e = sgemm(true, false, X, ld, X, ld, ob.gram, ld, k, k, rows, s)) != cudaSuccess) return e;
     if (pass == 0) {
-      add_shift_kernel<<<1, 1024, 0, s>>>(gram, ld, k, rows);
+      add_shift_kernel<<<1, 1024, 0, s>>>(ob.gram, ld, k, rows);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    if ((e = cholesky(gram, ld, k, linv, flag, s)) != cudaSuccess) return e;
-    if ((e = trsm_rows(X, ld, pass == 2 ? Xb : nullptr, pass == 2 ? Xlo : nullptr, ld, rows, k, gram, ld, linv, s)) !=
-        cudaSuccess)
-      return e;
+    if ((e = cholesky(ob.gram, ld, k, ob.linv, ob.flag, s)) != cudaSuccess) return e;
+    if ((e = tri_inverse(ob.gram, ob.Li, ob.Tt, ld, k, ob.linv, s)) != cudaSuccess) return e;
+    split_bf16_kernel<<<static_cast<unsigned>((lcnt + 255) / 256), 256, 0, s>>>(ob.Li, ld, k, k, ob.Lih, ob.Lil, ld);
+    split_bf16_kernel<<<static_cast<unsigned>((xcnt + 255) / 256), 256, 0, s>>>(X, ld, rows, k, Xb, Xlo, ld);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // X = Xhi Lhi^T + Xhi Llo^T + Xlo Lhi^T
+    if ((e = launch_gemm_f32(Xb, ld, false, ob.Lih, ld, true, X, ld, rows, k, k, s)) != cudaSuccess) return e;
+    if ((e = launch_gemm_f32(Xb, ld, false, ob.Lil, ld, true, X, ld, rows, k, k, s, true)) != cudaSuccess) return e;
+    if ((e = launch_gemm_f32(Xlo, ld, false, ob.Lih, ld, true, X, ld, rows, k, k, s, true)) != cudaSuccess) return e;
   }
-  return cudaSuccess;
+  split_bf16_kernel<<<static_cast<unsigned>((xcnt + 255) / 256), 256, 0, s>>>(X, ld, rows, k, Xb, Xlo, ld);
+  return cudaGetLastError();
 }
 
 // One-sided Jacobi on the k x k matrix stored transposed in At (and Vt, if any).
@@ -305,17 +347,25 @@ cudaError_t jacobi(float* At, float* Vt, int64_t ld, int k, unsigned* bar, int* 
                    cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(bar, 0, 4 * sizeof(unsigned), s);
   if (e != cudaSuccess) return e;
-  const int pairs = (k + 1) / 2;
-  int grid = std::min(sm_count(), std::max(1, (pairs + 7) / 8));
+  const int nblk = (k + kBJW - 1) / kBJW;
+  const int pairs = (nblk + (nblk & 1)) / 2;
+  int grid = std::max(1, pairs);
+  const bool resident = k <= kBJResidentMaxK;
+  const size_t dyn = resident ? size_t(kBJP) * bj_resident_stride(k) * sizeof(float) : 0;
+  void* fn = resident ? reinterpret_cast<void*>(jacobi_kernel<true>) : reinterpret_cast<void*>(jacobi_kernel<false>);
+  if (resident) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn));
+    if (e != cudaSuccess) return e;
+  }
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, jacobi_kernel, 256, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, 256, dyn);
   if (e != cudaSuccess) return e;
   grid = std::min(grid, std::max(1, per_sm) * sm_count());
   int max_sweeps = kJacobiMaxSweeps;
   float tol = kJacobiTol;
   void* args[] = {&At, &Vt, &ld, &k, &max_sweeps, &tol, &bar, &sweeps, &status};
   const int tok = profile_begin(s, QG_KERNEL_OTHER, 0.0, 0.0);
-  e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(jacobi_kernel), dim3(grid), dim3(256), args, 0, s);
+  e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(256), args, dyn, s);
   profile_end(s, tok);
   return e;
 }
@@ -403,6 +453,7 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
   uint16_t* Ylo = reinterpret_cast<uint16_t*>(ws + L.Ylo);
   float* Z = reinterpret_cast<float*>(ws + L.Z);
   uint16_t* Zb = reinterpret_cast<uint16_t*>(ws + L.Zb);
+  uint16_t* Zlo = reinterpret_cast<uint16_t*>(ws + L.Zlo);
   float* gram = reinterpret_cast<float*>(ws + L.gram);
   float* linv = reinterpret_cast<float*>(ws + L.linv);
   float* Bm = reinterpret_cast<float*>(ws + L.Bm);
@@ -413,6 +464,9 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
   float* Vsel = reinterpret_cast<float*>(ws + L.Vsel);
   Misc* misc = reinterpret_cast<Misc*>(ws + L.misc);
   if (cudaMemsetAsync(misc, 0, sizeof(Misc), s) != cudaSuccess) return QG_ECUDA;
+  const OrthBufs ob{gram, linv, reinterpret_cast<float*>(ws + L.Li), reinterpret_cast<float*>(ws + L.Tt),
+                    reinterpret_cast<uint16_t*>(ws + L.Lih), reinterpret_cast<uint16_t*>(ws + L.Lil),
+                    &misc->chol_flag};
 
   // Omega and the range finder
   {
@@ -423,12 +477,12 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
     if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
   }
   if (launch_gemm_f32(a.G, a.ldg, false, Om, ldk, false, Y, ldk, m, k, n, s) != cudaSuccess) return QG_ECUDA;
-  if (orth(Y, Yb, Ylo, m, k, ldk, gram, linv, &misc->chol_flag, s) != cudaSuccess) return QG_ECUDA;
+  if (orth(Y, Yb, Ylo, m, k, ldk, ob, s) != cudaSuccess) return QG_ECUDA;
   for (int it = 0; it < a.power_iters; ++it) {
     if (launch_gemm_f32(a.G, a.ldg, true, Yb, ldk, false, Z, ldk, n, k, m, s) != cudaSuccess) return QG_ECUDA;
-    if (orth(Z, Zb, nullptr, n, k, ldk, gram, linv, &misc->chol_flag, s) != cudaSuccess) return QG_ECUDA;
+    if (orth(Z, Zb, Zlo, n, k, ldk, ob, s) != cudaSuccess) return QG_ECUDA;
     if (launch_gemm_f32(a.G, a.ldg, false, Zb, ldk, false, Y, ldk, m, k, n, s) != cudaSuccess) return QG_ECUDA;
-    if (orth(Y, Yb, Ylo, m, k, ldk, gram, linv, &misc->chol_flag, s) != cudaSuccess) return QG_ECUDA;
+    if (orth(Y, Yb, Ylo, m, k, ldk, ob, s) != cudaSuccess) return QG_ECUDA;
   }
   // Rayleigh-Ritz: B = Q^T G, S = B B^T, eigenpairs of S
   // B = Q^T G with Q split into bf16 hi + lo parts (about 16 significant bits)

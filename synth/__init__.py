@@ -152,3 +152,41 @@ def device_weight_scales(m, n, seed, device, group=256, base=4.7e-4):
     g.manual_seed(int(seed) * 7919 + 2)
     ng = -(-(m * n) // group)
     return base * (0.5 + torch.rand(ng, generator=g, device=device, dtype=torch.float32))
+
+
+class DeviceDriftingGradient:
+    """bf16 m x n gradients on the device whose signal subspace drifts.
+
+    G_t = U_t diag(s) V^T + sigma E_t with s_i = s0 * decay^i (i < rank), Haar U_0,
+    V and W (W orthonormal and orthogonal to U_0, drawn with them), and
+    U_t = U_0 cos(theta_t) + W sin(theta_t): each left singular vector turns in
+    its own plane (u_i, w_i) by theta_t = rate * min(t, freeze).  E_t is standard
+    normal noise redrawn at every step from (seed, t)."""
+
+    def __init__(self, m, n, rank, s0, decay, sigma, rate, freeze, seed, device, pad_to=8):
+        g = torch.Generator(device=device)
+        g.manual_seed(int(seed))
+        self.m, self.n, self.rank = m, n, min(rank, m // 2, n)
+        a = torch.randn(m, 2 * self.rank, generator=g, device=device, dtype=torch.float32)
+        q, rr = torch.linalg.qr(a)
+        q = q * torch.sign(torch.diagonal(rr))[None, :]
+        self.U0, self.W = q[:, : self.rank].contiguous(), q[:, self.rank:].contiguous()
+        b = torch.randn(n, self.rank, generator=g, device=device, dtype=torch.float32)
+        qb, rb = torch.linalg.qr(b)
+        s = s0 * decay ** torch.arange(self.rank, device=device, dtype=torch.float32)
+        self.SVt = (s[:, None] * (qb * torch.sign(torch.diagonal(rb))[None, :]).T).contiguous()
+        self.sigma, self.rate, self.freeze, self.seed = sigma, rate, freeze, int(seed)
+        self.ld = -(-n // pad_to) * pad_to
+        self.device = device
+        self.out = torch.zeros(m, self.ld, device=device, dtype=torch.bfloat16)
+
+    def draw(self, t):
+        import math
+        th = self.rate * min(t, self.freeze)
+        U = self.U0 * math.cos(th) + self.W * math.sin(th)
+        g = torch.Generator(device=self.device)
+        g.manual_seed(self.seed * 1000003 + t + 1)
+        full = U @ self.SVt
+        full += self.sigma * torch.randn(self.m, self.n, generator=g, device=self.device, dtype=torch.float32)
+        self.out[:, : self.n] = full.to(torch.bfloat16)
+        return self.out
