@@ -172,6 +172,74 @@ __global__ void __launch_bounds__(256) sgemm_batched_kernel(const float* A, int6
   }
 }
 
+// Gram matrix G = X^T X (X: rows x k, stride ld) for the 64 x 64 tiles on or below
+// the diagonal only (all a Cholesky factorisation reads), with the rows split
+// into gridDim.y slices: CTA (t, s) writes the partial sum of slice s of tile t
+// to Part[s][t] (64 x 64), and gram_reduce_kernel adds the slices in order, so
+// the result does not depend on scheduling.
+QG_DEV void lower_tile(int t, int& tm, int& tn) {
+  int r = static_cast<int>((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
+  while (r * (r + 1) / 2 > t) --r;
+  while ((r + 1) * (r + 2) / 2 <= t) ++r;
+  tm = r;
+  tn = t - r * (r + 1) / 2;
+}
+
+__global__ void __launch_bounds__(256) gram_partial_kernel(const float* __restrict__ X, int64_t ld, int rows, int k,
+                                                           int slice, float* __restrict__ Part, int ntiles) {
+  __shared__ float As[kSgBK][kSgBM + 4];
+  __shared__ float Bs[kSgBK][kSgBN + 4];
+  int tm, tn;
+  lower_tile(blockIdx.x, tm, tn);
+  const int r0 = blockIdx.y * slice, r1 = min(rows, r0 + slice);
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int m0 = tm * kSgBM, n0 = tn * kSgBN;
+  float acc[4][4] = {};
+  for (int k0 = r0; k0 < r1; k0 += kSgBK) {
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+      const int e = tid + l * 256;
+      const int kk = e >> 6, mi = e & 63;
+      const int gk = k0 + kk;
+      As[kk][mi] = (gk < r1 && m0 + mi < k) ? X[static_cast<int64_t>(gk) * ld + m0 + mi] : 0.f;
+      Bs[kk][mi] = (gk < r1 && n0 + mi < k) ? X[static_cast<int64_t>(gk) * ld + n0 + mi] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kSgBK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = __fmaf_rn(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  float* out = Part + (static_cast<int64_t>(blockIdx.y) * ntiles + blockIdx.x) * (kSgBM * kSgBN);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) out[(ty * 4 + i) * kSgBN + tx * 4 + j] = acc[i][j];
+}
+
+__global__ void gram_reduce_kernel(const float* __restrict__ Part, int ntiles, int slices, float* __restrict__ G,
+                                   int64_t ld, int k) {
+  const int t = blockIdx.x;
+  int tm, tn;
+  lower_tile(t, tm, tn);
+  for (int e = threadIdx.x; e < kSgBM * kSgBN; e += blockDim.x) {
+    const int i = tm * kSgBM + e / kSgBN, j = tn * kSgBN + e % kSgBN;
+    if (i >= k || j >= k) continue;
+    float sum = 0.f;
+    for (int s = 0; s < slices; ++s) sum += Part[(static_cast<int64_t>(s) * ntiles + t) * (kSgBM * kSgBN) + e];
+    G[static_cast<int64_t>(i) * ld + j] = sum;
+  }
+}
+
 // Li (k x k, stride ld) <- the block-diagonal of L^-1 from the 32 x 32 diagonal
 // block inverses (Linv, 1024 floats each), zero elsewhere.
 __global__ void trinv_init_kernel(float* Li, int64_t ld, int k, const float* Linv) {
@@ -360,6 +428,130 @@ __global__ void __launch_bounds__(256) trsm_rows_kernel(float* X, int64_t ldx, u
   }
 }
 
+// ------------------------------------------------------------------ Cholesky, one launch
+
+QG_DEV bool grid_barrier(unsigned* bar, unsigned nblocks, uint32_t* status);
+
+// Cholesky of the nb x nb diagonal block at (j0, j0) (lower triangle of A, read
+// through L2) by one CTA: written back as L, its 32 x 32 inverse (lower,
+// identity-padded) to Linv.  Non-positive pivots raise *flag (see below).
+QG_DEV void chol_factor_diag(float* A, int64_t ld, int j0, int nb, float* Linv, int* flag, float (&T)[32][33],
+                             float (&X)[32][33]) {
+  __syncthreads();
+  for (int e = threadIdx.x; e < 1024; e += blockDim.x) {
+    const int i = e >> 5, j = e & 31;
+    float v = (i == j) ? 1.f : 0.f;
+    if (i < nb && j < nb && j <= i) v = __ldcg(A + static_cast<int64_t>(j0 + i) * ld + j0 + j);
+    T[i][j] = (j <= i) ? v : 0.f;
+  }
+  __syncthreads();
+  for (int c = 0; c < 32; ++c) {
+    if (threadIdx.x == 0) {
+      float d = T[c][c];
+      if (!(d > 0.f)) {
+        if (c < nb) atomicOr(flag, 1);
+        d = 1e-30f;
+      }
+      T[c][c] = sqrtf(d);
+    }
+    __syncthreads();
+    if (threadIdx.x > c && threadIdx.x < 32) T[threadIdx.x][c] = T[threadIdx.x][c] / T[c][c];
+    __syncthreads();
+    for (int e = threadIdx.x; e < 1024; e += blockDim.x) {
+      const int i = e >> 5, j = e & 31;
+      if (i > c && j > c && j <= i) T[i][j] = __fmaf_rn(-T[i][c], T[j][c], T[i][j]);
+    }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < 1024; e += blockDim.x) {
+    const int i = e >> 5, j = e & 31;
+    if (i < nb && j < nb) __stcg(A + static_cast<int64_t>(j0 + i) * ld + j0 + j, (j <= i) ? T[i][j] : 0.f);
+  }
+  // inverse, row by row: X[r][j] = (delta_rj - sum_{t<r} T[r][t] X[t][j]) / T[r][r]
+  for (int r = 0; r < 32; ++r) {
+    if (threadIdx.x < 32) {
+      const int j = threadIdx.x;
+      float acc = (r == j) ? 1.f : 0.f;
+      for (int t = j; t < r; ++t) acc = __fmaf_rn(-T[r][t], X[t][j], acc);
+      X[r][j] = (r >= j) ? acc / T[r][r] : 0.f;
+    }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < 1024; e += blockDim.x) __stcg(Linv + e, X[e >> 5][e & 31]);
+}
+
+// The whole blocked (32-wide) Cholesky of the k x k matrix A in one cooperative
+// launch: per panel, the tiles below the diagonal block are solved against its
+// inverse (TRSM), then the trailing lower tiles are updated (SYRK) and the CTA
+// that updates the next diagonal tile factorises it right away; a bounded grid
+// barrier follows each phase.  Linv receives the diagonal blocks' inverses.
+__global__ void __launch_bounds__(256) cholesky_kernel(float* A, int64_t ld, int k, float* Linv, int* flag,
+                                                       unsigned* bar, uint32_t* status) {
+  __shared__ float T[32][33];
+  __shared__ float X[32][33];
+  __shared__ float Li[32][33];
+  const int nblk = (k + 31) / 32;
+  if (blockIdx.x == 0) chol_factor_diag(A, ld, 0, min(32, k), Linv, flag, T, X);
+  if (!grid_barrier(bar, gridDim.x, status)) return;
+  for (int jb = 0; jb < nblk; ++jb) {
+    const int j0 = jb * 32;
+    const int tiles = nblk - jb - 1;
+    if (tiles == 0) break;
+    // TRSM: L[i, j0 + c] = sum_c' A[i, j0 + c'] Linv[c][c'] for the rows below
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+      __syncthreads();
+      for (int e = threadIdx.x; e < 1024; e += blockDim.x) {
+        const int r = e >> 5, c = e & 31;
+        const int row = j0 + 32 + t * 32 + r;
+        Li[r][c] = __ldcg(Linv + static_cast<int64_t>(jb) * 1024 + e);
+        T[r][c] = (row < k && j0 + c < k) ? __ldcg(A + static_cast<int64_t>(row) * ld + j0 + c) : 0.f;
+      }
+      __syncthreads();
+      for (int e = threadIdx.x; e < 1024; e += blockDim.x) {
+        const int r = e >> 5, c = e & 31;
+        const int row = j0 + 32 + t * 32 + r;
+        float acc = 0.f;
+        for (int q = 0; q <= c; ++q) acc = __fmaf_rn(T[r][q], Li[c][q], acc);
+        if (row < k && j0 + c < k) __stcg(A + static_cast<int64_t>(row) * ld + j0 + c, acc);
+      }
+    }
+    if (!grid_barrier(bar, gridDim.x, status)) return;
+    // SYRK on the lower tiles of the trailing matrix; tile 0 is the next
+    // diagonal block, factorised by its CTA as soon as it is updated
+    const int ntiles = tiles * (tiles + 1) / 2;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      int ti = static_cast<int>((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
+      while (ti * (ti + 1) / 2 > t) --ti;
+      while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
+      const int tl = t - ti * (ti + 1) / 2;
+      const int base = j0 + 32;
+      __syncthreads();
+      for (int e = threadIdx.x; e < 1024; e += blockDim.x) {
+        const int r = e >> 5, c = e & 31;
+        const int ri = base + ti * 32 + r, rl = base + tl * 32 + r;
+        T[r][c] = (ri < k) ? __ldcg(A + static_cast<int64_t>(ri) * ld + j0 + c) : 0.f;
+        X[r][c] = (rl < k) ? __ldcg(A + static_cast<int64_t>(rl) * ld + j0 + c) : 0.f;
+      }
+      __syncthreads();
+      for (int e = threadIdx.x; e < 1024; e += blockDim.x) {
+        const int r = e >> 5, c = e & 31;
+        const int gi = base + ti * 32 + r, gl = base + tl * 32 + c;
+        if (gi < k && gl < k && gl <= gi) {
+          float acc = 0.f;
+          for (int q = 0; q < 32; ++q) acc = __fmaf_rn(T[r][q], X[c][q], acc);
+          float* a = A + static_cast<int64_t>(gi) * ld + gl;
+          __stcg(a, __ldcg(a) - acc);
+        }
+      }
+      if (t == 0) {
+        __threadfence_block();
+        chol_factor_diag(A, ld, base, min(32, k - base), Linv + static_cast<int64_t>(jb + 1) * 1024, flag, T, X);
+      }
+    }
+    if (!grid_barrier(bar, gridDim.x, status)) return;
+  }
+}
+
 // ------------------------------------------------------------------ Jacobi
 
 // Bounded grid barrier for a cooperative launch.  bar[0] counts arrivals,
@@ -418,6 +610,7 @@ constexpr int kBJP = 2 * kBJW;     // columns per block pair
 constexpr int kBJChunk = 128;      // column entries streamed per pass
 constexpr int kBJInnerSweeps = 1;  // one inner sweep per pair: the outer sweeps converge as fast
 constexpr float kBJInnerTol = 1e-7f;
+constexpr float kBJStopTol = 1e-4f;
 
 struct BJShared {
   float X[kBJP][kBJChunk + 1];
@@ -429,6 +622,7 @@ struct BJShared {
   int pp[kBJP / 2], qq[kBJP / 2];  // the pairs of the current inner step
   int part[kBJP];                  // pair index of each column, + kBJP for the second member
   int rotate;
+  __align__(16) float Jv[kBJP][kBJP];  // J again, rows 16-byte aligned for vector reads
 };
 
 // J <- J (3 I - J^T J) / 2: one Newton-Schulz step back towards orthogonality
@@ -452,7 +646,10 @@ QG_DEV void bj_reorthogonalize(BJShared& sh) {
     sh.JT[i][j] = __fmaf_rn(-0.5f, h, 1.5f * sh.J[i][j]);
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < kBJP * kBJP; e += blockDim.x) sh.J[e / kBJP][e % kBJP] = sh.JT[e / kBJP][e % kBJP];
+  for (int e = threadIdx.x; e < kBJP * kBJP; e += blockDim.x) {
+    sh.J[e / kBJP][e % kBJP] = sh.JT[e / kBJP][e % kBJP];
+    sh.Jv[e / kBJP][e % kBJP] = sh.JT[e / kBJP][e % kBJP];
+  }
   __syncthreads();
 }
 
@@ -505,7 +702,7 @@ constexpr int kBJResidentMaxK = 1536;
 // that 16-byte reads of the same column by rows 0..31 spread over all banks.
 __host__ __device__ inline int bj_resident_stride(int k) {
   int kp = (k + 3) / 4 * 4;
-  return kp + ((4 - kp % 32) + 32) % 32;
+  return kp + ((4 - kp % 32) + 32) % 32;  // kp = 4 mod 32, so kp / 4 is odd
 }
 
 QG_DEV void cp_async16(void* smem, const void* gmem, int src_bytes) {
@@ -535,6 +732,7 @@ QG_DEV void bj_load_resident(float* X, int kp, const float* Mat, int64_t ld, int
 QG_DEV void bj_apply_resident(const BJShared& sh, const float* X, int kp, float* Mat, int64_t ld, int I, int Jb,
                               int k) {
   constexpr int kRows = kBJP / 4;
+  static_assert(kRows == 8, "two 16-byte reads of J per row");
   const int quads = kp / 4;
   const int ig = threadIdx.x / 64, cq0 = threadIdx.x % 64;
   for (int cq = cq0; cq < quads; cq += 64) {
@@ -546,9 +744,12 @@ QG_DEV void bj_apply_resident(const BJShared& sh, const float* X, int kp, float*
 #pragma unroll 4
     for (int l = 0; l < kBJP; ++l) {
       const float4 x = *reinterpret_cast<const float4*>(X + l * kp + c);
+      const float4 ja = *reinterpret_cast<const float4*>(&sh.Jv[l][ig * kRows]);
+      const float4 jb = *reinterpret_cast<const float4*>(&sh.Jv[l][ig * kRows + 4]);
+      const float jr[kRows] = {ja.x, ja.y, ja.z, ja.w, jb.x, jb.y, jb.z, jb.w};
 #pragma unroll
       for (int u = 0; u < kRows; ++u) {
-        const float j = sh.J[l][ig * kRows + u];
+        const float j = jr[u];
         out[u].x = __fmaf_rn(j, x.x, out[u].x);
         out[u].y = __fmaf_rn(j, x.y, out[u].y);
         out[u].z = __fmaf_rn(j, x.z, out[u].z);
@@ -597,19 +798,32 @@ __global__ void __launch_bounds__(256) jacobi_kernel(float* At, float* Vt, int64
         if (kResident) {
           __syncthreads();
           bj_load_resident(Xr, kp, At, ld, I, Jb, k);
-          const float* ra0 = Xr + (2 * ty) * kp;
-          const float* ra1 = ra0 + kp;
-          const float* rb0 = Xr + (2 * tx) * kp;
-          const float* rb1 = rb0 + kp;
+          // rows ty, ty + 16 against tx, tx + 16: with kp / 4 odd, sixteen
+          // consecutive rows fall on eight different 16-byte bank groups
+          const float* ra0 = Xr + ty * kp;
+          const float* ra1 = ra0 + 16 * kp;
+          const float* rb0 = Xr + tx * kp;
+          const float* rb1 = rb0 + 16 * kp;
+          // four partial sums per entry (one per float4 lane): shorter rounding
+          // chains keep the Gram's noise below the convergence test
+          float4 s00 = make_float4(0.f, 0.f, 0.f, 0.f), s01 = s00, s10 = s00, s11 = s00;
 #pragma unroll 4
           for (int c = 0; c < kp; c += 4) {
             const float4 a0 = *reinterpret_cast<const float4*>(ra0 + c), a1 = *reinterpret_cast<const float4*>(ra1 + c);
             const float4 b0 = *reinterpret_cast<const float4*>(rb0 + c), b1 = *reinterpret_cast<const float4*>(rb1 + c);
-            g00 = __fmaf_rn(a0.x, b0.x, __fmaf_rn(a0.y, b0.y, __fmaf_rn(a0.z, b0.z, __fmaf_rn(a0.w, b0.w, g00))));
-            g01 = __fmaf_rn(a0.x, b1.x, __fmaf_rn(a0.y, b1.y, __fmaf_rn(a0.z, b1.z, __fmaf_rn(a0.w, b1.w, g01))));
-            g10 = __fmaf_rn(a1.x, b0.x, __fmaf_rn(a1.y, b0.y, __fmaf_rn(a1.z, b0.z, __fmaf_rn(a1.w, b0.w, g10))));
-            g11 = __fmaf_rn(a1.x, b1.x, __fmaf_rn(a1.y, b1.y, __fmaf_rn(a1.z, b1.z, __fmaf_rn(a1.w, b1.w, g11))));
+            s00.x = __fmaf_rn(a0.x, b0.x, s00.x); s00.y = __fmaf_rn(a0.y, b0.y, s00.y);
+            s00.z = __fmaf_rn(a0.z, b0.z, s00.z); s00.w = __fmaf_rn(a0.w, b0.w, s00.w);
+            s01.x = __fmaf_rn(a0.x, b1.x, s01.x); s01.y = __fmaf_rn(a0.y, b1.y, s01.y);
+            s01.z = __fmaf_rn(a0.z, b1.z, s01.z); s01.w = __fmaf_rn(a0.w, b1.w, s01.w);
+            s10.x = __fmaf_rn(a1.x, b0.x, s10.x); s10.y = __fmaf_rn(a1.y, b0.y, s10.y);
+            s10.z = __fmaf_rn(a1.z, b0.z, s10.z); s10.w = __fmaf_rn(a1.w, b0.w, s10.w);
+            s11.x = __fmaf_rn(a1.x, b1.x, s11.x); s11.y = __fmaf_rn(a1.y, b1.y, s11.y);
+            s11.z = __fmaf_rn(a1.z, b1.z, s11.z); s11.w = __fmaf_rn(a1.w, b1.w, s11.w);
           }
+          g00 = (s00.x + s00.y) + (s00.z + s00.w);
+          g01 = (s01.x + s01.y) + (s01.z + s01.w);
+          g10 = (s10.x + s10.y) + (s10.z + s10.w);
+          g11 = (s11.x + s11.y) + (s11.z + s11.w);
         }
         for (int c0 = 0; !kResident && c0 < k; c0 += kBJChunk) {
           __syncthreads();
@@ -625,16 +839,34 @@ __global__ void __launch_bounds__(256) jacobi_kernel(float* At, float* Vt, int64
             g11 = __fmaf_rn(a1, b1, g11);
           }
         }
-        sh.M[2 * ty][2 * tx] = g00;
-        sh.M[2 * ty][2 * tx + 1] = g01;
-        sh.M[2 * ty + 1][2 * tx] = g10;
-        sh.M[2 * ty + 1][2 * tx + 1] = g11;
+        if (kResident) {
+          sh.M[ty][tx] = g00;
+          sh.M[ty][tx + 16] = g01;
+          sh.M[ty + 16][tx] = g10;
+          sh.M[ty + 16][tx + 16] = g11;
+        } else {
+          sh.M[2 * ty][2 * tx] = g00;
+          sh.M[2 * ty][2 * tx + 1] = g01;
+          sh.M[2 * ty + 1][2 * tx] = g10;
+          sh.M[2 * ty + 1][2 * tx + 1] = g11;
+        }
         if (tid == 0) sh.rotate = 0;
         __syncthreads();
-        // ---- already orthogonal to tol?
-        for (int e = tid; e < kBJP * kBJP; e += blockDim.x) {
-          const int p = e / kBJP, q = e % kBJP;
-          if (p < q && fabsf(sh.M[p][q]) > tol * sqrtf(sh.M[p][p]) * sqrtf(sh.M[q][q])) sh.rotate = 1;
+        // ---- already orthogonal to tol?  (also the sweep's largest relative
+        // off-diagonal entry, for the stopping rule)
+        {
+          float worst = 0.f;
+          for (int e = tid; e < kBJP * kBJP; e += blockDim.x) {
+            const int p = e / kBJP, q = e % kBJP;
+            if (p < q) {
+              const float den = sqrtf(sh.M[p][p]) * sqrtf(sh.M[q][q]);
+              const float rel = den > 0.f ? fabsf(sh.M[p][q]) / den : 0.f;
+              if (rel > tol) sh.rotate = 1;
+              worst = fmaxf(worst, rel);
+            }
+          }
+          for (int o = 16; o > 0; o >>= 1) worst = fmaxf(worst, __shfl_xor_sync(0xFFFFFFFFu, worst, o));
+          if ((tid & 31) == 0 && worst > 0.f) atomicMax(bar + 4, __float_as_uint(worst));
         }
         __syncthreads();
         if (!sh.rotate) continue;
@@ -667,30 +899,35 @@ __global__ void __launch_bounds__(256) jacobi_kernel(float* At, float* Vt, int64
               sh.part[q] = tid + kBJP;
             }
             __syncthreads();
-            // columns: (M, J) <- (M, J) R
-            for (int e = tid; e < kBJP * kBJP; e += blockDim.x) {
-              const int i = e / kBJP, j = e % kBJP;
+            // columns: (M, J) <- (M, J) R.  Thread t owns column t % 32 and rows
+            // t / 32 + 8 u: one pair lookup per thread.
+            {
+              const int j = tid & (kBJP - 1), i0 = tid >> 5;
               const int pa = sh.part[j], pr = pa & (kBJP - 1);
               const int p = sh.pp[pr], q = sh.qq[pr];
               const float c = sh.c[pr], sn = sh.s[pr];
-              if (pa >= kBJP) {
-                sh.T[i][j] = __fmaf_rn(sn, sh.M[i][p], c * sh.M[i][q]);
-                sh.JT[i][j] = __fmaf_rn(sn, sh.J[i][p], c * sh.J[i][q]);
-              } else {
-                sh.T[i][j] = __fmaf_rn(c, sh.M[i][p], -sn * sh.M[i][q]);
-                sh.JT[i][j] = __fmaf_rn(c, sh.J[i][p], -sn * sh.J[i][q]);
+              const float cp = pa >= kBJP ? sn : c, cq = pa >= kBJP ? c : -sn;  // new = cp * col_p + cq * col_q
+#pragma unroll
+              for (int u = 0; u < kBJP / 8; ++u) {
+                const int i = i0 + 8 * u;
+                sh.T[i][j] = __fmaf_rn(cp, sh.M[i][p], cq * sh.M[i][q]);
+                sh.JT[i][j] = __fmaf_rn(cp, sh.J[i][p], cq * sh.J[i][q]);
               }
             }
             __syncthreads();
-            // rows: M <- R^T M
-            for (int e = tid; e < kBJP * kBJP; e += blockDim.x) {
-              const int i = e / kBJP, j = e % kBJP;
+            // rows: M <- R^T M.  Thread t owns row t % 32 and columns t / 32 + 8 u.
+            {
+              const int i = tid & (kBJP - 1), j0 = tid >> 5;
               const int pa = sh.part[i], pr = pa & (kBJP - 1);
               const int p = sh.pp[pr], q = sh.qq[pr];
               const float c = sh.c[pr], sn = sh.s[pr];
-              sh.M[i][j] = pa >= kBJP ? __fmaf_rn(sn, sh.T[p][j], c * sh.T[q][j])
-                                      : __fmaf_rn(c, sh.T[p][j], -sn * sh.T[q][j]);
-              sh.J[i][j] = sh.JT[i][j];
+              const float cp = pa >= kBJP ? sn : c, cq = pa >= kBJP ? c : -sn;
+#pragma unroll
+              for (int u = 0; u < kBJP / 8; ++u) {
+                const int j = j0 + 8 * u;
+                sh.M[i][j] = __fmaf_rn(cp, sh.T[p][j], cq * sh.T[q][j]);
+                sh.J[j][i] = sh.JT[j][i];
+              }
             }
             __syncthreads();
           }
@@ -714,10 +951,18 @@ __global__ void __launch_bounds__(256) jacobi_kernel(float* At, float* Vt, int64
       if (!grid_barrier(bar, gridDim.x, status)) return;
     }
     const unsigned rotations = *reinterpret_cast<volatile unsigned*>(rot);
+    const float worst = __uint_as_float(*reinterpret_cast<volatile unsigned*>(bar + 4));
     if (!grid_barrier(bar, gridDim.x, status)) return;
-    if (blockIdx.x == 0 && threadIdx.x == 0) atomicExch(rot, 0u);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      atomicExch(rot, 0u);
+      atomicExch(bar + 4, 0u);
+    }
     if (!grid_barrier(bar, gridDim.x, status)) return;
-    if (rotations == 0) {
+    // done after a sweep without rotation, or once every pair met in this sweep
+    // was within kBJStopTol (the rotations of this sweep leave the columns
+    // orthogonal to about tol; float32 rounding keeps a few pairs from ever
+    // passing tol exactly)
+    if (rotations == 0 || worst <= kBJStopTol) {
       ++sweep;
       break;
     }

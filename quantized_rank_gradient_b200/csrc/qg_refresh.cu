@@ -38,9 +38,15 @@ size_t r256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct RefreshLayout {
   int k, ldk, ldn4;
-  size_t P, omega, Y, Yb, Ylo, Z, Zb, Zlo, gram, linv, Li, Tt, Lih, Lil, Bm, At, Vt, lam, perm, Vsel, Pa, Pb, Ct, misc,
+  size_t P, omega, Y, Yb, Ylo, Z, Zb, Zlo, gram, gpart, linv, Li, Tt, Lih, Lil, Bm, At, Vt, lam, perm, Vsel, Pa, Pb, Ct, misc,
       total;
 };
+
+constexpr int kGramSlicesMax = 32;
+int gram_tiles(int k) {
+  const int t = (k + 63) / 64;
+  return t * (t + 1) / 2;
+}
 
 RefreshLayout refresh_layout(int m, int n, int r, int p) {
   RefreshLayout L;
@@ -63,6 +69,7 @@ RefreshLayout refresh_layout(int m, int n, int r, int p) {
   L.Zb = take(size_t(n) * ldk * 2);
   L.Zlo = take(size_t(n) * ldk * 2);
   L.gram = take(k * ldk * 4);
+  L.gpart = take(size_t(kGramSlicesMax) * gram_tiles(L.k) * 64 * 64 * 4);
   L.linv = take(((k + 31) / 32) * 1024 * 4);
   L.Li = take(k * ldk * 4);
   L.Tt = take(k * ldk * 4);
@@ -82,10 +89,10 @@ RefreshLayout refresh_layout(int m, int n, int r, int p) {
   return L;
 }
 
-// misc region: [0..3] grid barrier + rotation counter, [4] Cholesky flag,
-// [5] Jacobi sweeps, [6] CosSim value (float)
+// misc region: [0..7] grid barrier, rotation counter, sweep's largest
+// off-diagonal; then the Cholesky flag, the Jacobi sweeps, the CosSim value
 struct Misc {
-  unsigned bar[4];
+  unsigned bar[8];
   int chol_flag;
   int sweeps;
   float cossim;
@@ -260,20 +267,21 @@ cudaError_t sgemm(bool ta, bool tb, const float* A, int64_t lda, const float* B,
   return cudaGetLastError();
 }
 
-// Lower Cholesky factor of the k x k matrix A in place (blocked, 32-wide panels);
-// Linv receives the inverses of the diagonal blocks.
-cudaError_t cholesky(float* A, int64_t ld, int k, float* Linv, int* flag, cudaStream_t s) {
-  for (int j0 = 0; j0 < k; j0 += 32) {
-    const int nb = std::min(32, k - j0);
-    potrf_diag_kernel<<<1, 32, 0, s>>>(A, ld, j0, nb, Linv + static_cast<size_t>(j0 / 32) * 1024, flag);
-    const int rest = k - j0 - 32;
-    if (rest > 0) {
-      const int T = (rest + 31) / 32;
-      trsm_panel_kernel<<<T, dim3(32, 32), 0, s>>>(A, ld, j0, k, Linv + static_cast<size_t>(j0 / 32) * 1024);
-      syrk_update_kernel<<<T * (T + 1) / 2, dim3(32, 32), 0, s>>>(A, ld, j0, k);
-    }
-  }
-  return cudaGetLastError();
+// Lower Cholesky factor of the k x k matrix A in place (blocked, 32-wide panels,
+// one cooperative launch); Linv receives the inverses of the diagonal blocks.
+cudaError_t cholesky(float* A, int64_t ld, int k, float* Linv, int* flag, unsigned* bar, uint32_t* status,
+                     cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(bar, 0, 8 * sizeof(unsigned), s);
+  if (e != cudaSuccess) return e;
+  const int nblk = (k + 31) / 32;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, cholesky_kernel, 256, 0);
+  if (e != cudaSuccess) return e;
+  // one CTA per SM at most: the grid barriers cost grows with the CTA count
+  const int want = std::max(1, (nblk - 1) * nblk / 2);
+  const int grid = std::min(want, std::min(std::max(1, per_sm), 1) * sm_count());
+  void* args[] = {&A, &ld, &k, &Linv, &flag, &bar, &status};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(cholesky_kernel), dim3(grid), dim3(256), args, 0, s);
 }
 
 // Li <- L^-1 for the lower Cholesky factor L (k x k, stride ld, lower triangle
@@ -302,7 +310,10 @@ cudaError_t tri_inverse(const float* Lf, float* Li, float* Tt, int64_t ld, int k
 }
 
 struct OrthBufs {
+  unsigned* bar;
+  uint32_t* status;
   float* gram;
+  float* gpart;
   float* linv;
   float* Li;
   float* Tt;
@@ -323,12 +334,21 @@ cudaError_t orth(float* X, uint16_t* Xb, uint16_t* Xlo, int rows, int k, int64_t
   cudaError_t e;
   const int64_t xcnt = int64_t(rows) * ld, lcnt = int64_t(k) * ld;
   for (int pass = 0; pass < 3; ++pass) {
-    if ((e = sgemm(true, false, X, ld, X, ld, ob.gram, ld, k, k, rows, s)) != cudaSuccess) return e;
+    {
+      const int ntiles = gram_tiles(k);
+      const int slices = std::max(1, std::min(kGramSlicesMax, rows / 512));
+      const int slice = (rows + slices - 1) / slices;
+      const int tok = profile_begin(s, QG_KERNEL_OTHER, double(k) * k * rows, 4.0 * rows * k);
+      gram_partial_kernel<<<dim3(ntiles, slices), 256, 0, s>>>(X, ld, rows, k, slice, ob.gpart, ntiles);
+      gram_reduce_kernel<<<ntiles, 256, 0, s>>>(ob.gpart, ntiles, slices, ob.gram, ld, k);
+      profile_end(s, tok);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     if (pass == 0) {
       add_shift_kernel<<<1, 1024, 0, s>>>(ob.gram, ld, k, rows);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    if ((e = cholesky(ob.gram, ld, k, ob.linv, ob.flag, s)) != cudaSuccess) return e;
+    if ((e = cholesky(ob.gram, ld, k, ob.linv, ob.flag, ob.bar, ob.status, s)) != cudaSuccess) return e;
     if ((e = tri_inverse(ob.gram, ob.Li, ob.Tt, ld, k, ob.linv, s)) != cudaSuccess) return e;
     split_bf16_kernel<<<static_cast<unsigned>((lcnt + 255) / 256), 256, 0, s>>>(ob.Li, ld, k, k, ob.Lih, ob.Lil, ld);
     split_bf16_kernel<<<static_cast<unsigned>((xcnt + 255) / 256), 256, 0, s>>>(X, ld, rows, k, Xb, Xlo, ld);
@@ -345,7 +365,7 @@ cudaError_t orth(float* X, uint16_t* Xb, uint16_t* Xlo, int rows, int k, int64_t
 // One-sided Jacobi on the k x k matrix stored transposed in At (and Vt, if any).
 cudaError_t jacobi(float* At, float* Vt, int64_t ld, int k, unsigned* bar, int* sweeps, uint32_t* status,
                    cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(bar, 0, 4 * sizeof(unsigned), s);
+  cudaError_t e = cudaMemsetAsync(bar, 0, 8 * sizeof(unsigned), s);
   if (e != cudaSuccess) return e;
   const int nblk = (k + kBJW - 1) / kBJW;
   const int pairs = (nblk + (nblk & 1)) / 2;
@@ -464,7 +484,8 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
   float* Vsel = reinterpret_cast<float*>(ws + L.Vsel);
   Misc* misc = reinterpret_cast<Misc*>(ws + L.misc);
   if (cudaMemsetAsync(misc, 0, sizeof(Misc), s) != cudaSuccess) return QG_ECUDA;
-  const OrthBufs ob{gram, linv, reinterpret_cast<float*>(ws + L.Li), reinterpret_cast<float*>(ws + L.Tt),
+  const OrthBufs ob{misc->bar, a.status, gram, reinterpret_cast<float*>(ws + L.gpart), linv, reinterpret_cast<float*>(ws + L.Li),
+                    reinterpret_cast<float*>(ws + L.Tt),
                     reinterpret_cast<uint16_t*>(ws + L.Lih), reinterpret_cast<uint16_t*>(ws + L.Lil),
                     &misc->chol_flag};
 
@@ -535,7 +556,7 @@ qg_status run_cossim(const float* Pa, const float* Pb, int32_t m, int32_t r, int
                      cudaStream_t stream) {
   float* Ct = reinterpret_cast<float*>(ws);
   unsigned* bar = reinterpret_cast<unsigned*>(ws + r256(size_t(r) * r * 4));
-  int* sweeps = reinterpret_cast<int*>(bar + 4);
+  int* sweeps = reinterpret_cast<int*>(bar + 8);
   return st_of(cossim_core(Pa, Pb, m, r, ld, Ct, bar, sweeps, d_out, nullptr, stream));
 }
 
