@@ -518,8 +518,13 @@ __global__ void __launch_bounds__(256) cholesky_kernel(float* A, int64_t ld, int
     if (!grid_barrier(bar, gridDim.x, status)) return;
     // SYRK on the lower tiles of the trailing matrix; tile 0 is the next
     // diagonal block, factorised by its CTA as soon as it is updated
+    // tile 0 (the next diagonal block, factorised right after its update) goes
+    // to CTA 0 alone; the other tiles are spread over the other CTAs
     const int ntiles = tiles * (tiles + 1) / 2;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    const int others = gridDim.x > 1 ? static_cast<int>(gridDim.x) - 1 : 1;
+    const int first = gridDim.x > 1 ? (blockIdx.x == 0 ? 0 : static_cast<int>(blockIdx.x)) : 0;
+    const int stride = gridDim.x > 1 ? (blockIdx.x == 0 ? ntiles : others) : 1;
+    for (int t = first; t < ntiles; t += stride) {
       int ti = static_cast<int>((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
       while (ti * (ti + 1) / 2 > t) --ti;
       while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
