@@ -230,7 +230,7 @@ class Stack:
         for li, shapes in enumerate(stack_shapes(layers)):
             group = []
             for (m, n) in shapes:
-                seed = 1_000_003 * (rank + 1) + lid
+                seed = matrix_seed(rank, lid)
                 c = qg.config(m, n, R_RANK, seed=seed, layer_id=lid)
                 ldw = -(-n // 16) * 16
                 W = synth.device_weight_codes(m, n, ldw, seed, device)
@@ -285,6 +285,30 @@ class Stack:
         return [e["state"] for group in self.layers for e in group]
 
 
+def matrix_seed(rank, lid):
+    """Seed of matrix `lid` of rank `rank`'s stack: every rank updates its own
+    independent stack (weak scaling)."""
+    return 1_000_003 * (rank + 1) + lid
+
+
+def reduce_max(value, world):
+    """The largest `value` over all ranks (the slowest rank sets the job's time):
+    an all-reduce on the process group's device (CUDA for NCCL, host for gloo)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units processed by all ranks per second, over the max-over-ranks time."""
+    return world * units_per_rank / (ms / 1000.0)
+
+
 def alg_bytes(m, n, r):
     """Algorithmic HBM bytes of one matrix step: G, W read and written, W scales,
     INT4 P and scales, moments read and written, their scales."""
@@ -331,10 +355,7 @@ def run_ours(args, rank, world, local_rank):
     qg.check(qg.qg_profile_collect(kt, qg.QG_KERNEL_KINDS))
     qg.check(qg.qg_profile_enable(0))
     clk = clocks.stop()
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(ms, world)
 
     # ---- end to end: gradients copied from pinned host memory every step,
     # the per-matrix status words read back
@@ -345,7 +366,7 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return 0
     peaks = load_peaks()
-    value = world * stack.weights / (ms / 1000.0)
+    value = whole_job_rate(stack.weights, world, ms)
     names = {qg.QG_KERNEL_DEQUANT: "dequant_projection", qg.QG_KERNEL_PROJECT_ADAM: "project_adam_tcgen05",
              qg.QG_KERNEL_BACKPROJECT_SR: "backproject_sround_tcgen05"}
     kernels = {}
@@ -443,11 +464,11 @@ def run_refresh_stress(args, rank, world, local_rank):
     ms = [a.elapsed_time(b) for a, b in ev]
     for item in trace:
         refresh_ms.append(ms[item["t"]])
-    total_ms = sum(ms)
+    total_ms = reduce_max(sum(ms), world)
     plain = sorted(ms[t] for t in range(steps) if t not in {i["t"] for i in trace})
     if rank != 0:
         return 0
-    value = world * steps * m * n / (total_ms / 1000.0)
+    value = whole_job_rate(steps * m * n, world, total_ms)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": 0,
             "ms_per_step": total_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16/f32/int8", "data": "synthetic (drifting low-rank-plus-noise bf16 gradients)",
@@ -512,12 +533,8 @@ def run_e2e(stack, args, stream, world, device, barrier):
     t1.record()
     torch.cuda.synchronize()
     barrier()
-    ms = t0.elapsed_time(t1) / steps
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": world * stack.weights / (ms / 1000.0), "unit": UNIT, "ms_per_step": ms, "steps": steps,
+    ms = reduce_max(t0.elapsed_time(t1) / steps, world)
+    return {"value": whole_job_rate(stack.weights, world, ms), "unit": UNIT, "ms_per_step": ms, "steps": steps,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "note": "bf16 gradients copied from pinned host memory each step; status words read back"}
 

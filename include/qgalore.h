@@ -273,6 +273,17 @@ qg_status qg_gemm_bf16(const void* d_A, int64_t lda, int32_t a_trans, const void
 qg_status qg_selfcheck_exact_math(int32_t op, uint64_t n, uint64_t seed, unsigned long long* d_out,
                                   void* stream);
 
+/* Self-check of the bounded device waits that every kernel of this library
+ * uses (the failure-detection path; the pages have no counterpart): one
+ * thread waits on an mbarrier that nothing arrives at, with a limit of
+ * limit_ns (1 ns .. 10 s).  The wait must give up after the limit, set the
+ * timeout bit (1, as in a layer's status word) in *d_status (device uint32,
+ * OR-ed) and let the kernel return, leaving the context usable.
+ * d_out: 2 device uint64, [0] = 1 when
+ * the wait reported failure, [1] = nanoseconds spent.  Asynchronous on
+ * `stream`; QG_EINVAL for null pointers or a limit out of range. */
+qg_status qg_selfcheck_wait_timeout(uint64_t limit_ns, uint32_t* d_status, unsigned long long* d_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

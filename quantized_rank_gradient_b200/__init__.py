@@ -88,6 +88,7 @@ _SIGNATURES = {
     "qg_gemm_bf16": (c_int32, [c_void_p, c_int64, c_int32, c_void_p, c_int64, c_int32, c_void_p, c_int64, c_int32,
                                c_int32, c_int32, c_void_p]),
     "qg_selfcheck_exact_math": (c_int32, [c_int32, c_uint64, c_uint64, c_void_p, c_void_p]),
+    "qg_selfcheck_wait_timeout": (c_int32, [c_uint64, c_void_p, c_void_p, c_void_p]),
 }
 
 _lib = None

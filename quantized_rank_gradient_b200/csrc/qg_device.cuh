@@ -83,20 +83,25 @@ QG_DEV bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity) {
 // when another thread of the CTA has raised *abort, or after kWaitLimitNs, in
 // which case it raises *abort and the timeout bit of *status itself.  The abort
 // flag and the clock are checked every 8 suspensions (at most about 8 ms apart).
-QG_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* status) {
+QG_DEV bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* status,
+                          uint64_t limit_ns) {
   if (mbar_try_wait_suspend(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_suspend(bar, parity)) return true;
     if ((it & 7u) == 0u) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort = 1;
         if (status) atomicOr(status, kErrTimeout);
         return false;
       }
     }
   }
+}
+
+QG_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* status) {
+  return mbar_wait_for(bar, parity, abort, status, kWaitLimitNs);
 }
 
 // Wait used only on the way out of an aborted kernel: bounded, ignores *abort.
