@@ -37,6 +37,7 @@ METRIC = "Q-GaLore step: INT8 weights updated/s at 7B shapes; % of step roofline
 UNIT = "weights/s"
 WORKLOAD = "llama7b-stack-r1024"
 R_RANK = 1024
+L2_BYTES = 126 << 20
 
 
 def parse_args():
@@ -45,17 +46,27 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--layers", type=int, default=32, help="decoder layers (32 = the 7B stack)")
+    ap.add_argument("--layers", type=int, default=None, help="decoder layers (default: the stack's own count)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["llama7b-stack", "refresh-stress"], default="llama7b-stack",
-                    help="refresh-stress: one 4096 x 11008 layer, r = 1024, a drifting gradient subspace, "
-                         "subspace refreshes on the layer-adaptive schedule (--steps defaults to 2000)")
+    ap.add_argument("--workload", choices=sorted(STACKS) + ["refresh-stress"], default="llama7b-stack",
+                    help="a decoder stack (llama7b-stack is the default and the headline), or refresh-stress: "
+                         "one 4096 x 11008 layer, r = 1024, a drifting gradient subspace, subspace refreshes on "
+                         "the layer-adaptive schedule (--steps defaults to 2000)")
     return ap.parse_args()
 
 
-def stack_shapes(layers):
-    per = [(4096, 4096)] * 4 + [(4096, 11008)] * 2 + [(11008, 4096)]
+# Decoder stacks: hidden size, MLP size, layers, projection rank r, and the
+# synthetic gradient's signal (rank, s0, decay of s_i = s0 decay^i, noise sigma).
+STACKS = {
+    "llama7b-stack": dict(hidden=4096, inter=11008, layers=32, rank=1024, sig=(256, 1e-2, 0.97, 1e-4)),
+    "llama1b-stack": dict(hidden=2048, inter=5461, layers=24, rank=512, sig=(256, 1e-2, 0.97, 1e-4)),
+    "llama60m-stack": dict(hidden=512, inter=1376, layers=8, rank=128, sig=(64, 1e-2, 0.8, 1e-4)),
+}
+
+
+def stack_shapes(layers, hidden=4096, inter=11008):
+    per = [(hidden, hidden)] * 4 + [(hidden, inter)] * 2 + [(inter, hidden)]
     return [per for _ in range(layers)]
 
 
@@ -216,7 +227,7 @@ def run_reference(args, rank, world):
 class Stack:
     """The 7B stack on one GPU: per matrix W, W scales, state, gradient."""
 
-    def __init__(self, layers, rank, device):
+    def __init__(self, layers, rank, device, spec=None):
         import torch
 
         import quantized_rank_gradient_b200 as qg
@@ -226,16 +237,19 @@ class Stack:
         self.layers = []
         self.keep = []
         stream = c_void_p(torch.cuda.current_stream().cuda_stream)
+        spec = spec or STACKS["llama7b-stack"]
+        R = spec["rank"]
+        self.rank_r = R
         lid = 0
-        for li, shapes in enumerate(stack_shapes(layers)):
+        for li, shapes in enumerate(stack_shapes(layers, spec["hidden"], spec["inter"])):
             group = []
             for (m, n) in shapes:
                 seed = matrix_seed(rank, lid)
-                c = qg.config(m, n, R_RANK, seed=seed, layer_id=lid)
+                c = qg.config(m, n, R, seed=seed, layer_id=lid)
                 ldw = -(-n // 16) * 16
                 W = synth.device_weight_codes(m, n, ldw, seed, device)
                 sW = synth.device_weight_scales(m, n, seed, device)
-                G = synth.device_lowrank_gradient(m, n, 256, 1e-2, 0.97, 1e-4, seed, device)
+                G = synth.device_lowrank_gradient(m, n, *spec["sig"], seed, device)
                 state = torch.empty(qg.qg_state_bytes(byref(c)), dtype=torch.uint8, device=device)
                 h = c_void_p()
                 qg.check(qg.qg_layer_init(byref(h), byref(c), state.data_ptr(), state.numel(), W.data_ptr(), ldw,
@@ -243,10 +257,10 @@ class Stack:
                 # starting projection: an orthonormal basis quantized to INT4 on the device
                 g = torch.Generator(device=device)
                 g.manual_seed(seed + 17)
-                P = torch.linalg.qr(torch.randn(m, R_RANK, generator=g, device=device))[0].contiguous()
-                Pq = torch.empty((m * R_RANK + 1) // 2, dtype=torch.uint8, device=device)
-                sP = torch.empty(-(-m * R_RANK // 64), dtype=torch.float32, device=device)
-                qg.check(qg.qg_quantize_projection(P.data_ptr(), R_RANK, m, R_RANK, Pq.data_ptr(), sP.data_ptr(),
+                P = torch.linalg.qr(torch.randn(m, R, generator=g, device=device))[0].contiguous()
+                Pq = torch.empty((m * R + 1) // 2, dtype=torch.uint8, device=device)
+                sP = torch.empty(-(-m * R // 64), dtype=torch.float32, device=device)
+                qg.check(qg.qg_quantize_projection(P.data_ptr(), R, m, R, Pq.data_ptr(), sP.data_ptr(),
                                                    stream))
                 qg.check(qg.qg_layer_set_projection(h, Pq.data_ptr(), sP.data_ptr(), 0, stream))
                 torch.cuda.synchronize()
@@ -271,8 +285,9 @@ class Stack:
                                (c_void_p * k)(*[e["G"].data_ptr() for e in group]),
                                (c_int64 * k)(*[e["ldg"] for e in group]), k))
         self.weights = sum(e["m"] * e["n"] for group in self.layers for e in group)
-        self.flops = sum(4.0 * e["m"] * e["n"] * R_RANK for group in self.layers for e in group)
-        self.alg_bytes = sum(alg_bytes(e["m"], e["n"], R_RANK) for group in self.layers for e in group)
+        self.flops = sum(4.0 * e["m"] * e["n"] * R for group in self.layers for e in group)
+        self.alg_bytes = sum(alg_bytes(e["m"], e["n"], R) for group in self.layers for e in group)
+        self.grad_bytes = sum(e["G"].numel() * 2 for group in self.layers for e in group)
 
     def step(self, stream):
         qg = self.qg
@@ -324,7 +339,9 @@ def run_ours(args, rank, world, local_rank):
     qg.lib()
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    stack = Stack(args.layers, rank, device)
+    spec = STACKS[args.workload]
+    layers = args.layers or spec["layers"]
+    stack = Stack(layers, rank, device, spec)
     stream = c_void_p(torch.cuda.current_stream().cuda_stream)
 
     def barrier():
@@ -342,15 +359,30 @@ def run_ours(args, rank, world, local_rank):
     qg.check(qg.qg_profile_enable(1))
     barrier()
     torch.cuda.synchronize()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record()
-    for _ in range(args.steps):
-        stack.step(stream)
-    t_end.record()
-    torch.cuda.synchronize()
+    flush = None
+    if stack.grad_bytes < 2 * L2_BYTES:
+        # inputs that fit in L2: each step timed alone, L2 flushed between steps
+        # (a 256 MB write outside the timed events)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    if flush is None:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record()
+        for _ in range(args.steps):
+            stack.step(stream)
+        t_end.record()
+        torch.cuda.synchronize()
+        ms = t_start.elapsed_time(t_end) / args.steps
+    else:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for e0, e1 in evs:
+            flush.fill_(1)
+            e0.record()
+            stack.step(stream)
+            e1.record()
+        torch.cuda.synchronize()
+        ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
     barrier()
-    ms = t_start.elapsed_time(t_end) / args.steps
     kt = (qg.qg_kernel_times * qg.QG_KERNEL_KINDS)()
     qg.check(qg.qg_profile_collect(kt, qg.QG_KERNEL_KINDS))
     qg.check(qg.qg_profile_enable(0))
@@ -387,8 +419,10 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/f32/int8",
         "data": "synthetic (seeded low-rank-plus-noise bf16 gradients)",
-        "config": {"workload": WORKLOAD, "matrices": 7 * args.layers, "weights_per_gpu": stack.weights,
-                   "rank": R_RANK, "l2": "inputs larger than L2 (13 GB of gradients per step)",
+        "config": {"workload": f"{args.workload}-r{spec['rank']}" + ("" if layers == spec["layers"] else f"-{layers}l"),
+                   "matrices": 7 * layers, "weights_per_gpu": stack.weights,
+                   "rank": spec["rank"], "l2": "inputs larger than L2 (%.1f GB of gradients per step)"
+                   % (stack.grad_bytes / 1e9) if flush is None else "L2 flushed between steps (each step timed alone)",
                    "parallelism": f"independent stacks x{world}"},
         "step_roofline": {"t_roof_ms": t_roof_ms, "frac": t_roof_ms / ms,
                           "bound": "tensor" if stack.flops / (peaks["bf16_tflops"] * 1e12) >
@@ -396,7 +430,9 @@ def run_ours(args, rank, world, local_rank):
                           "peaks": "burst bf16 %.1f TF/s, HBM %.1f GB/s (%s)" % (peaks["bf16_tflops"], peaks["hbm_gbs"],
                                                                               peaks["source"])},
         "roofline": {"bound": "tensor", "kernel": names[dom_k], "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic(names[dom_k], dom.bytes / dom.launches),
+                     "frac": achieved / peak,
+                     "traffic": profiled_traffic(names[dom_k], dom.bytes / dom.launches)
+                     if args.workload == "llama7b-stack" else None,
                      "traffic_unit": "DRAM bytes per launch (ncu traffic/algorithmic ratio x this launch)",
                      "algorithmic_bytes_per_launch": dom.bytes / dom.launches,
                      "peak_kind": "sustained bf16 (%s)" % peaks["source"]},
