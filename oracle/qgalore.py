@@ -328,18 +328,19 @@ def backproject(P_bf16, N_bf16) -> np.ndarray:
 def sr_uniform16(m, n, seed, t, layer_id):
     """The 16-bit uniform draw of every weight element (m x n uint32 in [0, 2^16)).
 
-    Element e = i*n + j (logical index) takes the 16-bit half (e mod 2) -- the low
-    half first -- of word ((e / 2) mod 4) of Philox-4x32-10(counter = (e/8 low 32
-    bits, e/8 high 32 bits, t, layer_id), key = (seed low 32 bits, seed high 32
-    bits)): one Philox call serves eight consecutive elements.
+    Element (i, j) takes the 16-bit half (j mod 2) -- the low half first -- of word
+    ((j / 2) mod 4) of Philox-4x32-10(counter = (j / 8, i, t, layer_id), key =
+    (seed low 32 bits, seed high 32 bits)): one Philox call serves eight
+    consecutive elements of a row, and every row starts a call.
     """
-    e = np.arange(m * n, dtype=np.uint64)
-    call = e >> np.uint64(3)
-    w = philox4x32_10(call & U32_MASK, call >> np.uint64(32), t, layer_id,
-                      seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
-    sel = ((e >> np.uint64(1)) & np.uint64(3)).astype(np.int64)
+    i = np.arange(m, dtype=np.uint64)[:, None]
+    j = np.arange(n, dtype=np.uint64)[None, :]
+    call = np.broadcast_to(j >> np.uint64(3), (m, n))
+    row = np.broadcast_to(i, (m, n))
+    w = philox4x32_10(call.ravel(), row.ravel(), t, layer_id, seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
+    sel = np.broadcast_to(((j >> np.uint64(1)) & np.uint64(3)).astype(np.int64), (m, n)).ravel()
     words = np.stack(w, axis=0)[sel, np.arange(m * n)]
-    shift = ((e & np.uint64(1)) * np.uint64(16)).astype(np.uint32)
+    shift = np.broadcast_to(((j & np.uint64(1)) * np.uint64(16)).astype(np.uint32), (m, n)).ravel()
     return ((words >> shift) & np.uint32(0xFFFF)).reshape(m, n)
 
 

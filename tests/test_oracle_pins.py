@@ -351,12 +351,14 @@ def test_sr_nan_keeps_code_inf_and_huge_saturate():
 
 
 def test_sr_uniform_draw_mapping():
-    u = O.sr_uniform16(3, 5, seed=77, t=2, layer_id=9)
-    for e in [0, 1, 2, 7, 8, 14]:
-        i, j = divmod(e, 5)
-        w = O.philox_generic([e // 8, 0, 2, 9], [77, 0], **O.PHILOX4x32)[(e // 2) % 4]
-        assert int(u[i, j]) == (w >> (16 * (e % 2))) & 0xFFFF
+    # element (i, j): half (j mod 2) of word ((j / 2) mod 4) of Philox(j / 8, i, t, layer)
+    u = O.sr_uniform16(3, 21, seed=(5 << 32) | 77, t=2, layer_id=9)
+    for (i, j) in [(0, 0), (0, 1), (0, 7), (1, 8), (2, 13), (2, 20)]:
+        w = O.philox_generic([j // 8, i, 2, 9], [77, 5], **O.PHILOX4x32)[(j // 2) % 4]
+        assert int(u[i, j]) == (w >> (16 * (j % 2))) & 0xFFFF
     assert u.max() < 2 ** 16
+    # rows draw independent streams: the same column of two rows differs
+    assert (u[0] != u[1]).mean() > 0.9
 
 
 def test_sr_small_updates_keep_their_mean():
