@@ -358,59 +358,23 @@ struct StochRoundEpi {
     float alpha;
     uint32_t t, layer_id;
     PhiloxKey key;
-    int32_t aligned8;    // n % 8 == 0: every 32-column chunk starts a Philox call
     int32_t aligned256;  // n % 256 == 0: a tile row is exactly one weight group
   };
 
-  // The 16-bit draws of elements e0 .. e0+31: element i's draw is half (i & 1)
-  // of d[i >> 1].  Element e takes half (e mod 2) of word ((e / 2) mod 4) of
-  // Philox-4x32-10(counter = (e / 8, t, layer_id), key = seed).
-  template <bool kAligned8>
-  static QG_DEV void draws(const Args& a, const PhiloxRoundKeys& rk, int64_t e0, uint32_t (&d)[16]) {
-    const uint64_t cb = static_cast<uint64_t>(e0) >> 3;
-    if (kAligned8) {
+  // The 16-bit draws of columns jc .. jc+31 of row irow (jc a multiple of 32):
+  // column j's draw is half (j mod 2) of word ((j / 2) mod 4) of
+  // Philox-4x32-10(counter = (j / 8, irow, t, layer_id), key = seed), so column
+  // jc + i takes half (i & 1) of d[i >> 1].  Every row starts a Philox call.
+  static QG_DEV void draws(const Args& a, const PhiloxRoundKeys& rk, int irow, int jc, uint32_t (&d)[16]) {
+    const uint32_t cb = static_cast<uint32_t>(jc) >> 3;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint32_t o[4];
-        const uint64_t c = cb + k;
-        philox4x32_10(static_cast<uint32_t>(c), static_cast<uint32_t>(c >> 32), a.t, a.layer_id, rk, o);
-        d[4 * k] = o[0];
-        d[4 * k + 1] = o[1];
-        d[4 * k + 2] = o[2];
-        d[4 * k + 3] = o[3];
-      }
-    } else {
-      // chunk starts at draw s = e0 mod 8 of call cb: five calls cover it
-      uint32_t dd[20];
-#pragma unroll
-      for (int k = 0; k < 5; ++k) {
-        uint32_t o[4];
-        const uint64_t c = cb + k;
-        philox4x32_10(static_cast<uint32_t>(c), static_cast<uint32_t>(c >> 32), a.t, a.layer_id, rk, o);
-        dd[4 * k] = o[0];
-        dd[4 * k + 1] = o[1];
-        dd[4 * k + 2] = o[2];
-        dd[4 * k + 3] = o[3];
-      }
-      const int s = static_cast<int>(e0 & 7);
-      // draw j of the calls is half (j & 1) of dd[j >> 1]; element i needs draw s + i
-#pragma unroll
-      for (int w = 0; w < 16; ++w) {
-        uint32_t lohi[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int i = 2 * w + h;
-          uint32_t val = 0;
-#pragma unroll
-          for (int ss = 0; ss < 8; ++ss) {
-            const int j = ss + i;
-            const uint32_t x = (dd[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-            val = (s == ss) ? x : val;
-          }
-          lohi[h] = val;
-        }
-        d[w] = lohi[0] | (lohi[1] << 16);
-      }
+    for (int k = 0; k < 4; ++k) {
+      uint32_t o[4];
+      philox4x32_10(cb + k, static_cast<uint32_t>(irow), a.t, a.layer_id, rk, o);
+      d[4 * k] = o[0];
+      d[4 * k + 1] = o[1];
+      d[4 * k + 2] = o[2];
+      d[4 * k + 3] = o[3];
     }
   }
 
@@ -471,7 +435,7 @@ struct StochRoundEpi {
 
   // This warpgroup's half of the tile's columns, 32-column chunks; W codes come
   // from the staged side tile, the new codes go straight to global memory.
-  template <bool kAligned8, bool kOneGroup>
+  template <bool kOneGroup>
   static QG_DEV void apply_impl(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr, int half,
                                 const uint8_t* side) {
     const int irow = mb * BM + row;
@@ -503,7 +467,7 @@ struct StochRoundEpi {
       }
       const uint4 wa = side_granule(side, row, 2 * c), wb = side_granule(side, row, 2 * c + 1);
       uint32_t d[16];
-      draws<kAligned8>(a, rk, e0, d);
+      draws(a, rk, irow, j0 + jc, d);
       uint32_t out[8];
       sr_chunk<kOneGroup>(U, wa, wb, d, cp0, cp1, split, out);
       if (valid == 32) {
@@ -520,11 +484,9 @@ struct StochRoundEpi {
   static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
                            const EpiPair& ep, const uint8_t* side) {
     if (a.aligned256)
-      apply_impl<true, true>(a, M, N, mb, nb, row, taddr, ep.half, side);
-    else if (a.aligned8)
-      apply_impl<true, false>(a, M, N, mb, nb, row, taddr, ep.half, side);
+      apply_impl<true>(a, M, N, mb, nb, row, taddr, ep.half, side);
     else
-      apply_impl<false, false>(a, M, N, mb, nb, row, taddr, ep.half, side);
+      apply_impl<false>(a, M, N, mb, nb, row, taddr, ep.half, side);
   }
 };
 
@@ -869,7 +831,7 @@ static cudaError_t launch_gemms_for(const StepProblem* probs, int cnt, cudaStrea
       pr.status = s.status;
       pr.epi = StochRoundEpi::Args{s.W, s.sW, s.ldw, s.alpha, s.t, s.layer_id,
                                    PhiloxKey{static_cast<uint32_t>(s.seed), static_cast<uint32_t>(s.seed >> 32)},
-                                   (s.n % 8) == 0 ? 1 : 0, (s.n % 256) == 0 ? 1 : 0};
+                                   (s.n % 256) == 0 ? 1 : 0};
       add_problem(p2, s.m, s.n, s.r);
     }
     e = launch_gemm_pair<StochRoundEpi, false>(p2, stream, QG_KERNEL_BACKPROJECT_SR, fl2, by2);
