@@ -5,8 +5,9 @@ Workload: a LLaMA-7B-shaped stack, 32 decoder layers x {q, k, v, o: 4096 x 4096;
 gate, up: 4096 x 11008; down: 11008 x 4096}, rank r = 1024: 224 weight matrices,
 6.48 G INT8 weights.  One step = the optimizer step a1..a5 on every matrix
 (dequantize INT4 P, R = P^T G, Adam on the INT8 moments, U = P N, stochastic
-rounding into INT8 W), issued as one batched call per decoder layer (three
-launches: the INT4 dequantization and two tcgen05 GEMMs).  Inputs are
+rounding into INT8 W), issued as one batched call for the whole stack (inside
+it, batches of 8 matrices, three launches each: the INT4 dequantization and two
+tcgen05 GEMMs, alternating between two streams).  Inputs are
 seeded synthetic bf16 gradients (rank-256 signal, s_i = 1e-2 * 0.97^i, noise
 sigma = 1e-4) resident in HBM (13 GB, far larger than L2).
 
@@ -87,7 +88,7 @@ def profiled_traffic(kernel, alg_bytes_per_launch):
     """DRAM bytes per launch of `kernel`: the ratio of measured DRAM traffic to
     algorithmic bytes in the committed ncu capture, times this run's
     algorithmic bytes per launch.  The ratio is taken from one launch of
-    the same kernel, an 8-matrix batch of two decoder layers. Traffic grows in
+    the same kernel, the 7-matrix batch of one decoder layer. Traffic grows in
     proportion to the matrices in a launch. None when the kernel sources
     changed since that capture."""
     try:
@@ -268,30 +269,36 @@ class Stack:
                 group.append(dict(cfg=c, h=h, W=W, sW=sW, G=G, ldg=G.shape[1], state=state, m=m, n=n))
                 lid += 1
             self.layers.append(group)
-        # one batched call per decoder layer (its 7 matrices in one batch), or with
-        # QG_BENCH_WHOLE_STACK=1 one call for all matrices (batches of 8 inside the
-        # library); one workspace reused by every call
-        groups = [[e for group in self.layers for e in group]] if os.environ.get("QG_BENCH_WHOLE_STACK") == "1" \
-            else self.layers
+        # the step: one batched call for all matrices (batches of 8 on two lanes
+        # inside the library), or with QG_BENCH_PER_LAYER=1 one call per decoder
+        # layer.  The per-layer calls (the 7 matrices of a layer in one batch, one
+        # stream, kernels one after another) also serve the kernel-timing pass.
+        whole = [[e for group in self.layers for e in group]]
+        self.per_layer_only = os.environ.get("QG_BENCH_PER_LAYER") == "1"
         need = 0
-        for group in groups:
+        for group in whole + self.layers:
             arr = (qg.POINTER(qg.qg_config) * len(group))(*[qg.ctypes.pointer(e["cfg"]) for e in group])
             need = max(need, qg.qg_step_batch_workspace_bytes(arr, len(group)))
         self.ws = torch.empty(need, dtype=torch.uint8, device=device)
-        self.calls = []
-        for group in groups:
-            k = len(group)
-            self.calls.append(((c_void_p * k)(*[e["h"].value for e in group]),
-                               (c_void_p * k)(*[e["G"].data_ptr() for e in group]),
-                               (c_int64 * k)(*[e["ldg"] for e in group]), k))
+
+        def calls_of(groups):
+            out = []
+            for group in groups:
+                k = len(group)
+                out.append(((c_void_p * k)(*[e["h"].value for e in group]),
+                            (c_void_p * k)(*[e["G"].data_ptr() for e in group]),
+                            (c_int64 * k)(*[e["ldg"] for e in group]), k))
+            return out
+        self.calls_layer = calls_of(self.layers)
+        self.calls = self.calls_layer if self.per_layer_only else calls_of(whole)
         self.weights = sum(e["m"] * e["n"] for group in self.layers for e in group)
         self.flops = sum(4.0 * e["m"] * e["n"] * R for group in self.layers for e in group)
         self.alg_bytes = sum(alg_bytes(e["m"], e["n"], R) for group in self.layers for e in group)
         self.grad_bytes = sum(e["G"].numel() * 2 for group in self.layers for e in group)
 
-    def step(self, stream):
+    def step(self, stream, per_layer=False):
         qg = self.qg
-        for hs, gs, lds, k in self.calls:
+        for hs, gs, lds, k in (self.calls_layer if per_layer else self.calls):
             st = qg.qg_step_batch(hs, gs, lds, k, self.ws.data_ptr(), self.ws.numel(), stream)
             if st != qg.QG_OK:
                 raise qg.QGError(st, "qg_step_batch")
@@ -383,11 +390,23 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
     barrier()
-    kt = (qg.qg_kernel_times * qg.QG_KERNEL_KINDS)()
-    qg.check(qg.qg_profile_collect(kt, qg.QG_KERNEL_KINDS))
+    kt_run = (qg.qg_kernel_times * qg.QG_KERNEL_KINDS)()
+    qg.check(qg.qg_profile_collect(kt_run, qg.QG_KERNEL_KINDS))
     qg.check(qg.qg_profile_enable(0))
     clk = clocks.stop()
     ms = reduce_max(ms, world)
+
+    # ---- kernel durations: in the timed region the two lanes' kernels overlap,
+    # so a launch's events would also span the other lane's work.  The same
+    # kernels on the same data are timed again one after another: one call per
+    # decoder layer on one stream (a step counts once more for every matrix's t).
+    qg.check(qg.qg_profile_enable(1))
+    for _ in range(args.steps):
+        stack.step(stream, per_layer=True)
+    torch.cuda.synchronize()
+    kt = (qg.qg_kernel_times * qg.QG_KERNEL_KINDS)()
+    qg.check(qg.qg_profile_collect(kt, qg.QG_KERNEL_KINDS))
+    qg.check(qg.qg_profile_enable(0))
 
     # ---- end to end: gradients copied from pinned host memory every step,
     # the per-matrix status words read back
@@ -413,7 +432,7 @@ def run_ours(args, rank, world, local_rank):
     dom = kt[dom_k]
     achieved = (dom.flops / dom.launches) / (dom.device_ms / dom.launches / 1000.0) / 1e12
     peak = peaks["bf16_tflops_sustained"]
-    launches = sum(kt[k].launches for k in range(qg.QG_KERNEL_KINDS)) / args.steps
+    launches = sum(kt_run[k].launches for k in range(qg.QG_KERNEL_KINDS)) / args.steps
     t_roof_ms = max(stack.flops / (peaks["bf16_tflops"] * 1e12), stack.alg_bytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -437,6 +456,8 @@ def run_ours(args, rank, world, local_rank):
                      "algorithmic_bytes_per_launch": dom.bytes / dom.launches,
                      "peak_kind": "sustained bf16 (%s)" % peaks["source"]},
         "kernels": kernels,
+        "kernels_timing": "a pass after the timed region, one call per decoder layer on one stream, so that "
+                          "each launch's events span that kernel alone",
         "gpu_launches": launches * args.steps,
         "clocks": clk,
     }

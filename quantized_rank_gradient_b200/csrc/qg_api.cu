@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 #include <vector>
 
 #include "../../include/qgalore.h"
@@ -289,10 +290,40 @@ qg_status qg_step(qg_layer* L, const void* d_G, int64_t ldg, void* d_ws, size_t 
   return st;
 }
 
-// Batch workspace: the matrices go in batches of up to kBatch (one grid per
-// stage each), run in order on one stream, so every batch reuses one slot as
-// large as the largest batch's scratch.
+// Batches and lanes.  The matrices go in batches of up to kBatch (three
+// launches per batch: one dequantization grid, one persistent grid per GEMM
+// stage).  Batches alternate between two lanes, the caller's stream and one
+// stream the library keeps per device, and each lane reuses one workspace slot
+// as large as the largest batch's scratch.  The lanes' kernels overlap, so the
+// SMs that one batch's last wave of tiles leaves idle take tiles of the other
+// lane's batch.  The lanes fork from and join back to the caller's stream
+// through events: the call is ordered on `stream` like a plain launch sequence
+// and can be captured into a CUDA graph.
 static constexpr int kBatch = 8;
+static constexpr int kLanes = 2;
+static constexpr int kMaxDevices = 64;
+
+struct Lane {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+static std::mutex g_lane_mu;  // guards g_lane and each fork / launch / join sequence
+static Lane g_lane[kMaxDevices];
+
+// The current device's second lane, created on first use.
+static qg_status second_lane(Lane** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QG_ECUDA;
+  Lane& L = g_lane[dev];
+  if (!L.s) {
+    if (cudaStreamCreateWithFlags(&L.s, cudaStreamNonBlocking) != cudaSuccess) return QG_ECUDA;
+    if (cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&L.join, cudaEventDisableTiming) != cudaSuccess)
+      return QG_ECUDA;
+  }
+  *out = &L;
+  return QG_OK;
+}
 
 static size_t batch_slot_bytes(const int32_t* m, const int32_t* n, const int32_t* r, int count) {
   size_t slot = 0;
@@ -304,6 +335,8 @@ static size_t batch_slot_bytes(const int32_t* m, const int32_t* n, const int32_t
   return slot;
 }
 
+static int batch_lanes(int count) { return std::min(kLanes, (count + kBatch - 1) / kBatch); }
+
 size_t qg_step_batch_workspace_bytes(const qg_config* const* cfgs, int32_t count) {
   if (!cfgs || count < 0) return 0;
   std::vector<int32_t> m(count), n(count), r(count);
@@ -311,7 +344,7 @@ size_t qg_step_batch_workspace_bytes(const qg_config* const* cfgs, int32_t count
     if (check_config(cfgs[i]) != QG_OK) return 0;
     m[i] = cfgs[i]->m, n[i] = cfgs[i]->n, r[i] = cfgs[i]->r;
   }
-  return batch_slot_bytes(m.data(), n.data(), r.data(), count);
+  return batch_slot_bytes(m.data(), n.data(), r.data(), count) * batch_lanes(count);
 }
 
 qg_status qg_step_batch(qg_layer* const* layers, const void* const* d_G, const int64_t* ldg, int32_t count,
@@ -328,16 +361,36 @@ qg_status qg_step_batch(qg_layer* const* layers, const void* const* d_G, const i
     m[i] = layers[i]->cfg.m, n[i] = layers[i]->cfg.n, r[i] = layers[i]->cfg.r;
   }
   const size_t slot = batch_slot_bytes(m.data(), n.data(), r.data(), count);
-  if (ws_bytes < slot) return QG_ESTATE;
+  const int lanes = batch_lanes(count);
+  if (ws_bytes < slot * lanes) return QG_ESTATE;
   std::vector<StepProblem> probs(count);
   for (int b = 0; b * kBatch < count; ++b) {
-    uint8_t* ws = static_cast<uint8_t*>(d_ws);
+    uint8_t* ws = static_cast<uint8_t*>(d_ws) + (b % lanes) * slot;
     for (int i = b * kBatch; i < count && i < (b + 1) * kBatch; ++i) {
       fill_step_problem(layers[i], d_G[i], ldg[i], ws, layers[i]->sched.t + 1, &probs[i]);
       ws += qg::step_scratch_bytes(m[i], n[i], r[i]);
     }
   }
-  qg_status st = cuda_status(qg::launch_step(probs.data(), count, static_cast<cudaStream_t>(stream)));
+  const cudaStream_t user = static_cast<cudaStream_t>(stream);
+  qg_status st = QG_OK;
+  if (lanes == 1) {
+    st = cuda_status(qg::launch_step(probs.data(), count, user));
+  } else {
+    std::lock_guard<std::mutex> lock(g_lane_mu);
+    Lane* L = nullptr;
+    st = second_lane(&L);
+    if (st != QG_OK) return st;
+    if (cudaEventRecord(L->fork, user) != cudaSuccess || cudaStreamWaitEvent(L->s, L->fork, 0) != cudaSuccess)
+      return QG_ECUDA;
+    for (int b = 0; st == QG_OK && b * kBatch < count; ++b) {
+      const int cnt = std::min(kBatch, count - b * kBatch);
+      st = cuda_status(qg::launch_step(probs.data() + b * kBatch, cnt, (b % 2) ? L->s : user));
+    }
+    // join even after a failed launch, so later work on `stream` stays ordered
+    // after whatever the second lane holds
+    if (cudaEventRecord(L->join, L->s) != cudaSuccess || cudaStreamWaitEvent(user, L->join, 0) != cudaSuccess)
+      st = QG_ECUDA;
+  }
   if (st == QG_OK)
     for (int i = 0; i < count; ++i) layers[i]->sched.t += 1;
   return st;

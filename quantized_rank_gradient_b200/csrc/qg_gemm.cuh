@@ -58,15 +58,16 @@ struct TileRef {
   int prob, mb, nb;
 };
 
-// Both epilogue warpgroups work on every tile: warpgroup `half` takes the
-// tile's columns [128 half, 128 half + 128).  Row-wise reductions over the whole
-// tile width (the Adam block absmax) combine the two halves through `xchg`,
-// guarded by a per-lane-quarter mbarrier completing once per tile.
+// Every epilogue warpgroup works on every tile: of `groups` warpgroups, group g
+// takes the tile's columns [g BN / groups, (g + 1) BN / groups).  Row-wise
+// reductions over the whole tile width (the Adam block absmax) combine the
+// groups' partial values through `xchg` ([group][BM] slots, one per row), guarded
+// by a per-lane-quarter mbarrier that completes once per tile.
 struct EpiPair {
-  int half;
-  float2* xchg_mine;    // this warp's slot for its 32 rows
-  float2* xchg_other;   // the partner warp's slot (same rows, other half)
-  uint64_t* xbar;       // count 2: one arrival per partner warp
+  int group;
+  int groups;
+  float2* xchg;         // slot of group 0 for this warp's 32 rows; group g's is xchg + g * BM
+  uint64_t* xbar;       // count `groups`: one arrival per warp holding these rows
   uint32_t xphase;
   volatile int* abort;
   uint32_t* status;
@@ -236,8 +237,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!mbar_wait(&acc_full[buf], ph, &abort_flag, status)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * BN;
-      EpiPair ep{half, &xchg[it & 1u][half][quarter * 32], &xchg[it & 1u][half ^ 1][quarter * 32], &xbar[quarter],
-                 it & 1u, &abort_flag, pr.status};
+      EpiPair ep{half, 2, &xchg[it & 1u][0][quarter * 32], &xbar[quarter], it & 1u, &abort_flag, pr.status};
       Epi::apply(pr.epi, pr.M, pr.N, tr.mb, tr.nb, row, taddr, ep, nullptr);
       tc_fence_before();
       __syncwarp();
@@ -262,8 +262,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // tile per pair, each CTA loading its 128 rows of A and 128 columns of B (half
 // the B traffic per SM of the one-CTA kernel), a ring of 32 KiB stages per
 // CTA, one MMA issuer in the even CTA (M = 256, N = 256, K = 16), and each
-// CTA's TMEM holding its 128 rows of the accumulator, drained by its own two
-// epilogue warpgroups.  Loads of both CTAs complete on the even CTA's
+// CTA's TMEM holding its 128 rows of the accumulator, drained by its own
+// Epi::kPairGroups epilogue warpgroups (warps 2 .. 4 kPairGroups + 1; warp 0
+// loads, warp 1 issues the MMAs).  Four warpgroups give each SM sub-partition
+// four epilogue warps to hide the epilogue's latencies behind one another.  Loads of both CTAs complete on the even CTA's
 // full-barrier; the issuer's commits arrive on both CTAs' barriers; epilogues
 // of both CTAs release an accumulator buffer on the even CTA's barrier.
 // B must be MN-major here (64-column boxes).
@@ -281,12 +283,15 @@ constexpr int kHalfStageBytes = 128 * BK * 2;  // 16 KiB: 128 rows of A or 128 c
 
 template <class Epi>
 struct PairLayout {
+  static constexpr int kGroups = Epi::kPairGroups;  // epilogue warpgroups per CTA
+  static constexpr int kThreads = 64 + 128 * kGroups;
+  static_assert(kGroups == 2 || kGroups == 4, "the tile's 256 columns split into 2 or 4 slices");
   static constexpr int kSideBytes = Epi::kSideBytes;
   static constexpr int kSideBufs = Epi::kSideBufs;
   static constexpr int kSideTotal = kSideBytes * kSideBufs;
   // shared memory a CTA may hold (227 KiB) less the static part: barriers and
   // flags, plus the row-maxima exchange when the epilogue uses it
-  static constexpr int kBudget = 232448 - 512 - (Epi::kExchange ? int(sizeof(float2)) * 2 * 2 * BM : 0) - 1024;
+  static constexpr int kBudget = 232448 - 512 - (Epi::kExchange ? int(sizeof(float2)) * 2 * kGroups * BM : 0) - 1024;
   // as many ring stages as fit beside the side buffers, at most 6
   static constexpr int kStages = (kBudget - kSideTotal) / (2 * kHalfStageBytes) > 6
                                      ? 6
@@ -297,10 +302,12 @@ struct PairLayout {
 };
 
 template <class Epi, bool kAMN, bool kBMN>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<Epi>::kThreads, 1)
     gemm_tc_pair_kernel(const __grid_constant__ GemmParams<Epi> p) {
   static_assert(kBMN, "the pair kernel loads B in 64-column boxes");
   using L = PairLayout<Epi>;
+  constexpr int kGroups = L::kGroups;
+  constexpr int kEpiWarps = 4 * kGroups;
   constexpr int kStagesP = L::kStages;
   constexpr int kSide = L::kSideBytes;
   constexpr int kSB = L::kSideBufs;
@@ -318,7 +325,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   __shared__ __align__(8) uint64_t side_empty[2];
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ __align__(8) uint64_t xbar[4];
-  __shared__ float2 xchg[Epi::kExchange ? 2 : 1][2][Epi::kExchange ? BM : 32];  // [tile parity][half][row]
+  __shared__ float2 xchg[Epi::kExchange ? 2 : 1][Epi::kExchange ? kGroups : 1][Epi::kExchange ? BM : 32];  // [tile parity][group][row]
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -336,11 +343,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 16);  // 8 epilogue warps x 2 CTAs (used in the even CTA)
+      mbar_init(&acc_empty[a], 2 * kEpiWarps);  // every epilogue warp of both CTAs (used in the even CTA)
       mbar_init(&side_full[a], 1);
-      mbar_init(&side_empty[a], 8);  // this CTA's 8 epilogue warps
+      mbar_init(&side_empty[a], kEpiWarps);  // this CTA's epilogue warps
     }
-    for (int q = 0; q < 4; ++q) mbar_init(&xbar[q], 2);
+    for (int q = 0; q < 4; ++q) mbar_init(&xbar[q], kGroups);
     mbar_init(&drain_bar, 1);
     abort_flag = 0;
     fence_barrier_init();
@@ -485,7 +492,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    const int half = (warp - 2) >> 2;
+    const int group = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const bool side_issuer = kSide > 0 && warp == 2 && lane == 0;
@@ -526,9 +533,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * BN;
-      float2* xm = Epi::kExchange ? &xchg[it & 1u][half][quarter * 32] : nullptr;
-      float2* xo = Epi::kExchange ? &xchg[it & 1u][half ^ 1][quarter * 32] : nullptr;
-      EpiPair ep{half, xm, xo, &xbar[quarter], it & 1u, &abort_flag, pr.status};
+      float2* xs = Epi::kExchange ? &xchg[it & 1u][0][quarter * 32] : nullptr;
+      EpiPair ep{group, kGroups, xs, &xbar[quarter], it & 1u, &abort_flag, pr.status};
       Epi::apply(pr.epi, pr.M, pr.N, mb2 * 2 + static_cast<int>(rank), nb, row, taddr, ep, side);
       tc_fence_before();
       __syncwarp();

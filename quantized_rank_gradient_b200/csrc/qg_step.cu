@@ -71,11 +71,6 @@ QG_DEV float sbyte_f32(uint32_t w, int k) {
   return __fsub_rn(__uint_as_float(kMagicBits + sx), kMagic);
 }
 
-// Code e (0..31) of a 32-byte chunk held in two uint4, as float.
-QG_DEV float code_f32(const uint4& lo, const uint4& hi, int e) {
-  return sbyte_f32(word_of(e < 16 ? lo : hi, (e >> 2) & 3), e & 3);
-}
-
 // 16-bit draw h (0: low half, 1: high half) of w as u = u16 * 2^-16, exact.
 QG_DEV float draw_u(uint32_t w, int h) {
   const uint32_t m = h ? ((w >> 9) & 0x007FFF80u) : ((w << 7) & 0x007FFF80u);
@@ -159,28 +154,24 @@ struct AdamEpi {
     vv = __fadd_rn(__fmul_rn(a.beta2, v0), __fmul_rn(a.om2, __fmul_rn(R, R)));
   }
 
-  // codes of 32-column chunk c of this row from the staged side tiles
-  static QG_DEV void load_codes(const uint8_t* side, int row, int c, uint4 (&q)[4]) {
-    q[0] = side_granule(side, row, 2 * c);
-    q[1] = side_granule(side, row, 2 * c + 1);
-    q[2] = side_granule(side + 32768, row, 2 * c);
-    q[3] = side_granule(side + 32768, row, 2 * c + 1);
-  }
+  // the pair kernel drains every tile with four epilogue warpgroups, 64 columns each
+  static constexpr int kPairGroups = 4;
 
-  // Pass 1 on one 32-column chunk: the new moments and the running block maxima of
-  // |m| and of v (max over the block of sqrt(v) is sqrt of the max of v, the
-  // correctly rounded square root being monotone).  The maxima propagate NaN, so
-  // a non-finite moment shows in them.  It also keeps the smallest |m| and v
-  // (zeros included), which decide whether pass 2 may use the branch-free square
-  // root and division.  kFull: all 32 columns are inside the matrix.
+  // Pass 1 on one 16-column sub-chunk (moment codes in qm, qv): the new moments
+  // and the running block maxima of |m| and of v (max over the block of sqrt(v)
+  // is sqrt of the max of v, the correctly rounded square root being monotone).
+  // The maxima propagate NaN, so a non-finite moment shows in them.  It also
+  // keeps the smallest |m| and v (zeros included), which decide whether pass 2
+  // may use the branch-free square root and division.  kFull: all 16 columns are
+  // inside the matrix.
   template <bool kFull>
-  static QG_DEV void pass1_chunk(const Args& a, const uint32_t (&v)[32], const uint4 (&cq)[4], float sm, float sv,
-                                 int valid, float& amax_m, float& amax_vv, float& mmin, float& vmin) {
+  static QG_DEV void pass1_sub(const Args& a, const uint32_t (&v)[16], const uint4& qm, const uint4& qv, float sm,
+                               float sv, int valid, float& amax_m, float& amax_vv, float& mmin, float& vmin) {
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
+    for (int e = 0; e < 16; ++e) {
       const float R = __uint_as_float(v[e]);
       float mm, vv;
-      moments(R, code_f32(cq[0], cq[1], e), code_f32(cq[2], cq[3], e), sm, sv, a, mm, vv);
+      moments(R, sbyte_f32(word_of(qm, e >> 2), e & 3), sbyte_f32(word_of(qv, e >> 2), e & 3), sm, sv, a, mm, vv);
       if (kFull || e < valid) {
         amax_m = max_nan_abs(amax_m, mm);
         amax_vv = max_nan(amax_vv, vv);
@@ -208,22 +199,22 @@ struct AdamEpi {
     return ok;
   }
 
-  // Pass 2 on one chunk: the same moments; N = -lr m_hat / (sqrt(v_hat) + eps)
-  // = (m c1) / (sqrt(v) c2 + eps) -> bf16; codes of m and sqrt(v) on the block's
-  // new grids.  |m| * (127 / absmax) and sqrt(v) * (127 / absmax_v) stay within
-  // 127 (1 + 2^-24), so their nearest integers need no clamp; a zero block has
-  // inverse scale 0 and gets codes 0.
+  // Pass 2 on one 16-column sub-chunk: the same moments; N = -lr m_hat /
+  // (sqrt(v_hat) + eps) = (m c1) / (sqrt(v) c2 + eps) -> bf16; codes of m and
+  // sqrt(v) on the block's new grids.  |m| * (127 / absmax) and sqrt(v) *
+  // (127 / absmax_v) stay within 127 (1 + 2^-24), so their nearest integers need
+  // no clamp; a zero block has inverse scale 0 and gets codes 0.
   // kExact selects sqrt_exact / div_exact, equal to the IEEE operations on the
   // ranges exact_fast_ok checks, over the intrinsics.
   template <bool kExact>
-  static QG_DEV void pass2_chunk(const Args& a, const uint32_t (&v)[32], const uint4 (&cq)[4], float sm, float sv,
-                                 float inv_m, float inv_v, uint16_t* nptr, int8_t* mptr, int8_t* vptr) {
-    uint32_t om[8], ov[8], packed[16], bm[4], bv[4];
+  static QG_DEV void pass2_sub(const Args& a, const uint32_t (&v)[16], const uint4& qm, const uint4& qv, float sm,
+                               float sv, float inv_m, float inv_v, uint16_t* nptr, int8_t* mptr, int8_t* vptr) {
+    uint32_t om[4], ov[4], packed[8], bm[4], bv[4];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
+    for (int e = 0; e < 16; ++e) {
       const float R = __uint_as_float(v[e]);
       float mm, vv;
-      moments(R, code_f32(cq[0], cq[1], e), code_f32(cq[2], cq[3], e), sm, sv, a, mm, vv);
+      moments(R, sbyte_f32(word_of(qm, e >> 2), e & 3), sbyte_f32(word_of(qv, e >> 2), e & 3), sm, sv, a, mm, vv);
       const float rv = kExact ? sqrt_exact(vv) : __fsqrt_rn(vv);
       const float num = __fmul_rn(mm, a.c1), den = __fadd_rn(__fmul_rn(rv, a.c2), a.eps);
       const float upd = kExact ? div_exact(num, den) : __fdiv_rn(num, den);
@@ -240,27 +231,26 @@ struct AdamEpi {
       }
     }
     uint4* dst = reinterpret_cast<uint4*>(nptr);
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
     *reinterpret_cast<uint4*>(mptr) = make_uint4(om[0], om[1], om[2], om[3]);
-    *reinterpret_cast<uint4*>(mptr + 16) = make_uint4(om[4], om[5], om[6], om[7]);
     *reinterpret_cast<uint4*>(vptr) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
-    *reinterpret_cast<uint4*>(vptr + 16) = make_uint4(ov[4], ov[5], ov[6], ov[7]);
   }
 
-  // One thread owns row `row` of its warpgroup's 128-column half of the
-  // 128 x 256 tile; the tile's 256 columns are exactly one moment block, so the
-  // block maxima of the two halves are combined with the partner warp before
-  // the codes are formed.  The tile's codes are staged in shared memory.
+  // One thread owns row `row` of its warpgroup's slice (BN / groups columns) of
+  // the 128 x 256 tile; the tile's 256 columns are exactly one moment block, so
+  // the block maxima of all slices are combined through the exchange before the
+  // codes are formed.  The tile's codes are staged in shared memory; 16-column
+  // sub-chunks keep the thread's registers within the four-warpgroup budget.
   static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
                            const EpiPair& ep, const uint8_t* side) {
     const int arow = mb * BM + row;
     const bool row_ok = arow < M;
     const int j0 = nb * BN;
     const int ncols = min(BN, N - j0);
-    const int c0 = ep.half * 4;
-    const int c1 = min(c0 + 4, (ncols + 31) >> 5);
+    const int nsub = BN / 16 / ep.groups;
+    const int s0 = ep.group * nsub;
+    const int s1 = min(s0 + nsub, (ncols + 15) >> 4);
     float sm = 0.f, sv = 0.f;
     int8_t* mrow = nullptr;
     int8_t* vrow = nullptr;
@@ -275,18 +265,17 @@ struct AdamEpi {
     float amax_m = 0.f, amax_vv = 0.f, mmin = __int_as_float(0x7f800000), vmin = __int_as_float(0x7f800000);
 
 #pragma unroll 1
-    for (int c = c0; c < c1; ++c) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(taddr + c * 32, v);
+    for (int s = s0; s < s1; ++s) {
+      uint32_t v[16];
+      tmem_ld_32x32b_x16(taddr + s * 16, v);
       tmem_ld_wait();
       if (row_ok) {
-        uint4 q[4];
-        load_codes(side, row, c, q);
-        const int valid = ncols - c * 32;
-        if (valid >= 32)
-          pass1_chunk<true>(a, v, q, sm, sv, valid, amax_m, amax_vv, mmin, vmin);
+        const uint4 qm = side_granule(side, row, s), qv = side_granule(side + 32768, row, s);
+        const int valid = ncols - s * 16;
+        if (valid >= 16)
+          pass1_sub<true>(a, v, qm, qv, sm, sv, valid, amax_m, amax_vv, mmin, vmin);
         else
-          pass1_chunk<false>(a, v, q, sm, sv, valid, amax_m, amax_vv, mmin, vmin);
+          pass1_sub<false>(a, v, qm, qv, sm, sv, valid, amax_m, amax_vv, mmin, vmin);
       }
     }
 
@@ -294,16 +283,20 @@ struct AdamEpi {
     const bool bad = !(amax_m <= 3.4028234663852886e38f) || !(amax_vv <= 3.4028234663852886e38f);
     const bool exact = exact_fast_ok(a, amax_m, amax_vv, mmin, vmin);
 
-    // block maxima over both halves (the partner warp owns the same rows)
+    // block maxima over all slices (the other groups' warps own the same rows);
+    // the combination propagates NaN like the maxima themselves
     const int lane = row & 31;
-    ep.xchg_mine[lane] = make_float2(amax_m, amax_vv);
+    ep.xchg[ep.group * BM + lane] = make_float2(amax_m, amax_vv);
     __threadfence_block();
     __syncwarp();
     if (lane == 0) mbar_arrive(ep.xbar);
     if (mbar_wait(ep.xbar, ep.xphase, ep.abort, ep.status)) {
-      const float2 o = ep.xchg_other[lane];
-      amax_m = fmaxf(amax_m, o.x);
-      amax_vv = fmaxf(amax_vv, o.y);
+      for (int g = 0; g < ep.groups; ++g) {
+        if (g == ep.group) continue;
+        const float2 o = ep.xchg[g * BM + lane];
+        amax_m = max_nan(amax_m, o.x);
+        amax_vv = max_nan(amax_vv, o.y);
+      }
     }
     const float amax_v = __fsqrt_rn(amax_vv);
 
@@ -317,20 +310,19 @@ struct AdamEpi {
     const float inv_v = live_v ? __fdiv_rn(127.0f, amax_v) : 0.f;
 
 #pragma unroll 1
-    for (int c = c0; c < c1; ++c) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(taddr + c * 32, v);
+    for (int s = s0; s < s1; ++s) {
+      uint32_t v[16];
+      tmem_ld_32x32b_x16(taddr + s * 16, v);
       tmem_ld_wait();
       if (row_ok) {
-        uint4 q[4];
-        load_codes(side, row, c, q);
+        const uint4 qm = side_granule(side, row, s), qv = side_granule(side + 32768, row, s);
         if (exact)
-          pass2_chunk<true>(a, v, q, sm, sv, inv_m, inv_v, nrow + c * 32, mrow + c * 32, vrow + c * 32);
+          pass2_sub<true>(a, v, qm, qv, sm, sv, inv_m, inv_v, nrow + s * 16, mrow + s * 16, vrow + s * 16);
         else
-          pass2_chunk<false>(a, v, q, sm, sv, inv_m, inv_v, nrow + c * 32, mrow + c * 32, vrow + c * 32);
+          pass2_sub<false>(a, v, qm, qv, sm, sv, inv_m, inv_v, nrow + s * 16, mrow + s * 16, vrow + s * 16);
       }
     }
-    if (row_ok && ep.half == 0) {
+    if (row_ok && ep.group == 0) {
       a.sM[static_cast<int64_t>(arow) * a.nblk + nb] = s_m;
       a.sV[static_cast<int64_t>(arow) * a.nblk + nb] = s_v;
     }
@@ -360,6 +352,11 @@ struct StochRoundEpi {
     PhiloxKey key;
     int32_t aligned256;  // n % 256 == 0: a tile row is exactly one weight group
   };
+
+  // the pair kernel drains every tile with two epilogue warpgroups, 128 columns
+  // each (the rounding's registers fit the two-warpgroup budget; measured, four
+  // warpgroups with 16-column sub-chunks ran no faster under the power cap)
+  static constexpr int kPairGroups = 2;
 
   // The 16-bit draws of columns jc .. jc+31 of row irow (jc a multiple of 32):
   // column j's draw is half (j mod 2) of word ((j / 2) mod 4) of
@@ -433,17 +430,18 @@ struct StochRoundEpi {
     }
   }
 
-  // This warpgroup's half of the tile's columns, 32-column chunks; W codes come
-  // from the staged side tile, the new codes go straight to global memory.
+  // This warpgroup's slice of the tile's columns, 32-column chunks; W codes
+  // come from the staged side tile, the new codes go straight to global memory.
   template <bool kOneGroup>
-  static QG_DEV void apply_impl(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr, int half,
-                                const uint8_t* side) {
+  static QG_DEV void apply_impl(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
+                                const EpiPair& ep, const uint8_t* side) {
     const int irow = mb * BM + row;
     const bool row_ok = irow < M;
     const int j0 = nb * BN;
     const int ncols = min(BN, N - j0);
-    const int c0 = half * 4;
-    const int c1 = min(c0 + 4, (ncols + 31) >> 5);
+    const int nchunk = BN / 32 / ep.groups;
+    const int c0 = ep.group * nchunk;
+    const int c1 = min(c0 + nchunk, (ncols + 31) >> 5);
     float cp_row = 0.f;
     if (kOneGroup && row_ok) cp_row = update_factor(a.alpha, a.sW[(static_cast<int64_t>(irow) * N + j0) >> 8]);
     int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + j0;
@@ -484,9 +482,9 @@ struct StochRoundEpi {
   static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
                            const EpiPair& ep, const uint8_t* side) {
     if (a.aligned256)
-      apply_impl<true>(a, M, N, mb, nb, row, taddr, ep.half, side);
+      apply_impl<true>(a, M, N, mb, nb, row, taddr, ep, side);
     else
-      apply_impl<false>(a, M, N, mb, nb, row, taddr, ep.half, side);
+      apply_impl<false>(a, M, N, mb, nb, row, taddr, ep, side);
   }
 };
 
@@ -509,8 +507,9 @@ struct StoreF32Epi {
     const bool ok = grow < M;
     const int j0 = nb * BN;
     const int ncols = min(BN, N - j0);
-    const int c0 = ep.half * 4;
-    const int c1 = min(c0 + 4, (ncols + 31) >> 5);
+    const int nchunk = BN / 32 / ep.groups;
+    const int c0 = ep.group * nchunk;
+    const int c1 = min(c0 + nchunk, (ncols + 31) >> 5);
     for (int c = c0; c < c1; ++c) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(taddr + c * 32, v);
@@ -708,7 +707,7 @@ static cudaError_t launch_gemm_pair(const GemmParams<Epi>& p, cudaStream_t strea
   if (pair_tiles == 0) return cudaSuccess;
   const int clusters = std::min(pair_tiles, std::max(1, sm_count() / 2));
   const int tok = profile_begin(stream, kind, flops, bytes);
-  kern<<<2 * clusters, kGemmThreads, kSmem, stream>>>(p);
+  kern<<<2 * clusters, PairLayout<Epi>::kThreads, kSmem, stream>>>(p);
   profile_end(stream, tok);
   return cudaGetLastError();
 }
