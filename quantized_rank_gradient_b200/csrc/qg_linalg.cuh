@@ -613,7 +613,6 @@ QG_DEV bool grid_barrier(unsigned* bar, unsigned nblocks, uint32_t* status) {
 constexpr int kBJW = 16;           // columns per block
 constexpr int kBJP = 2 * kBJW;     // columns per block pair
 constexpr int kBJChunk = 128;      // column entries streamed per pass
-constexpr int kBJInnerSweeps = 1;  // one inner sweep per pair: the outer sweeps converge as fast
 constexpr float kBJInnerTol = 1e-7f;
 constexpr float kBJStopTol = 1e-4f;
 
@@ -864,8 +863,8 @@ __global__ void __launch_bounds__(256) jacobi_kernel(float* At, float* Vt, int64
           for (int e = tid; e < kBJP * kBJP; e += blockDim.x) {
             const int p = e / kBJP, q = e % kBJP;
             if (p < q) {
-              const float den = sqrtf(sh.M[p][p]) * sqrtf(sh.M[q][q]);
-              const float rel = den > 0.f ? fabsf(sh.M[p][q]) / den : 0.f;
+              const float dd = sh.M[p][p] * sh.M[q][q];
+              const float rel = dd > 0.f ? fabsf(sh.M[p][q]) * rsqrtf(sh.M[p][p]) * rsqrtf(sh.M[q][q]) : 0.f;
               if (rel > tol) sh.rotate = 1;
               worst = fmaxf(worst, rel);
             }
@@ -875,26 +874,36 @@ __global__ void __launch_bounds__(256) jacobi_kernel(float* At, float* Vt, int64
         }
         __syncthreads();
         if (!sh.rotate) continue;
-        // ---- M = J L J^T by cyclic Jacobi (parallel ordering of the 2 kBJW columns)
-        for (int e = tid; e < kBJP * kBJP; e += blockDim.x) sh.J[e / kBJP][e % kBJP] = (e / kBJP == e % kBJP) ? 1.f : 0.f;
-        for (int is = 0; is < kBJInnerSweeps; ++is) {
-          __syncthreads();
-          if (tid == 0) sh.rotate = 0;
-          __syncthreads();
+        // ---- M = J L J^T by one cyclic Jacobi sweep (parallel ordering of the
+        // 2 kBJW columns).  The rotations come from rsqrt and approximate
+        // reciprocals: their angles only steer the outer iteration, whose stopping
+        // rule reads the Gram matrix itself, and the Newton-Schulz step below puts
+        // J back on the orthogonal group.
+        {
+          float(*Mc)[kBJP + 1] = sh.M;
+          float(*Mn)[kBJP + 1] = sh.T;
+          float(*Jc)[kBJP + 1] = sh.J;
+          float(*Jn)[kBJP + 1] = sh.JT;
+          for (int e = tid; e < kBJP * kBJP; e += blockDim.x) Jc[e / kBJP][e % kBJP] = (e / kBJP == e % kBJP) ? 1.f : 0.f;
           for (int step = 0; step < kBJP - 1; ++step) {
             if (tid < kBJP / 2) {
               const int aa = tid, bb = kBJP - 1 - tid;
               const int p = (aa == 0) ? 0 : ((aa - 1 + step) % (kBJP - 1)) + 1;
               const int q = ((bb - 1 + step) % (kBJP - 1)) + 1;
-              const float al = sh.M[p][p], be = sh.M[q][q], ga = sh.M[p][q];
+              const float al = Mc[p][p], be = Mc[q][q], ga = Mc[p][q];
               float c = 1.f, sn = 0.f;
-              if (fabsf(ga) > kBJInnerTol * sqrtf(al) * sqrtf(be)) {
-                const float zeta = (be - al) / (2.f * ga);
-                const float t = fabsf(zeta) < 1e18f ? copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta))
-                                                    : 0.5f / zeta;
-                c = 1.f / sqrtf(1.f + t * t);
+              if (fabsf(ga) * rsqrtf(al) * rsqrtf(be) > kBJInnerTol) {
+                const float zeta = __fdividef(be - al, 2.f * ga);
+                const float az = fabsf(zeta);
+                float t;
+                if (az < 1e18f) {
+                  const float x = __fmaf_rn(zeta, zeta, 1.f);
+                  t = copysignf(__fdividef(1.f, az + x * rsqrtf(x)), zeta);
+                } else {
+                  t = __fdividef(0.5f, zeta);
+                }
+                c = rsqrtf(__fmaf_rn(t, t, 1.f));
                 sn = c * t;
-                sh.rotate = 1;
               }
               sh.c[tid] = c;
               sh.s[tid] = sn;
@@ -904,39 +913,38 @@ __global__ void __launch_bounds__(256) jacobi_kernel(float* At, float* Vt, int64
               sh.part[q] = tid + kBJP;
             }
             __syncthreads();
-            // columns: (M, J) <- (M, J) R.  Thread t owns column t % 32 and rows
-            // t / 32 + 8 u: one pair lookup per thread.
+            // M' = R^T M R and J' = J R in one pass: thread t owns column t % 32
+            // and rows t / 32 + 8 u
             {
               const int j = tid & (kBJP - 1), i0 = tid >> 5;
-              const int pa = sh.part[j], pr = pa & (kBJP - 1);
-              const int p = sh.pp[pr], q = sh.qq[pr];
-              const float c = sh.c[pr], sn = sh.s[pr];
-              const float cp = pa >= kBJP ? sn : c, cq = pa >= kBJP ? c : -sn;  // new = cp * col_p + cq * col_q
+              const int paj = sh.part[j], prj = paj & (kBJP - 1);
+              const int pj = sh.pp[prj], qj = sh.qq[prj];
+              const float cj = sh.c[prj], sj = sh.s[prj];
+              const float cpj = paj >= kBJP ? sj : cj, cqj = paj >= kBJP ? cj : -sj;
 #pragma unroll
               for (int u = 0; u < kBJP / 8; ++u) {
                 const int i = i0 + 8 * u;
-                sh.T[i][j] = __fmaf_rn(cp, sh.M[i][p], cq * sh.M[i][q]);
-                sh.JT[i][j] = __fmaf_rn(cp, sh.J[i][p], cq * sh.J[i][q]);
+                const int pai = sh.part[i], pri = pai & (kBJP - 1);
+                const int pi = sh.pp[pri], qi = sh.qq[pri];
+                const float ci = sh.c[pri], si = sh.s[pri];
+                const float cpi = pai >= kBJP ? si : ci, cqi = pai >= kBJP ? ci : -si;
+                const float tp = __fmaf_rn(cpj, Mc[pi][pj], cqj * Mc[pi][qj]);
+                const float tq = __fmaf_rn(cpj, Mc[qi][pj], cqj * Mc[qi][qj]);
+                Mn[i][j] = __fmaf_rn(cpi, tp, cqi * tq);
+                Jn[i][j] = __fmaf_rn(cpj, Jc[i][pj], cqj * Jc[i][qj]);
               }
             }
             __syncthreads();
-            // rows: M <- R^T M.  Thread t owns row t % 32 and columns t / 32 + 8 u.
-            {
-              const int i = tid & (kBJP - 1), j0 = tid >> 5;
-              const int pa = sh.part[i], pr = pa & (kBJP - 1);
-              const int p = sh.pp[pr], q = sh.qq[pr];
-              const float c = sh.c[pr], sn = sh.s[pr];
-              const float cp = pa >= kBJP ? sn : c, cq = pa >= kBJP ? c : -sn;
-#pragma unroll
-              for (int u = 0; u < kBJP / 8; ++u) {
-                const int j = j0 + 8 * u;
-                sh.M[i][j] = __fmaf_rn(cp, sh.T[p][j], cq * sh.T[q][j]);
-                sh.J[j][i] = sh.JT[j][i];
-              }
-            }
-            __syncthreads();
+            float(*tm)[kBJP + 1] = Mc;
+            Mc = Mn;
+            Mn = tm;
+            tm = Jc;
+            Jc = Jn;
+            Jn = tm;
           }
-          if (!sh.rotate) break;
+          if (Jc != sh.J) {
+            for (int e = tid; e < kBJP * kBJP; e += blockDim.x) sh.J[e / kBJP][e % kBJP] = Jc[e / kBJP][e % kBJP];
+          }
         }
         bj_reorthogonalize(sh);
         // ---- the pair's columns (and V's) become A J

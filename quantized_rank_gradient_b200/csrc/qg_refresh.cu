@@ -7,8 +7,9 @@
 // Q = orth(Y); q times { Z = orth(G^T Q); Q = orth(G Z) }; B = Q^T G;
 // S = B B^T = V diag(lambda) V^T; P = Q V[:, top r].  The products with G run on
 // the tcgen05 core (bf16 operands, fp32 accumulation); orth() is shifted
-// Cholesky-QR in three passes (Fukaya et al. 2020) with fp32 SIMT Gram matrices
-// and X L^-T formed on the tensor cores from the explicit inverse;
+// Cholesky-QR (Fukaya et al. 2020) with fp32 SIMT Gram matrices and X L^-T
+// formed on the tensor cores from the explicit inverse: two passes for the
+// intermediate bases of the power iterations, three for the final Q;
 // the k x k eigenproblem and the r x r singular values of CosSim use a one-sided
 // Jacobi with a bounded grid barrier.  Then: sign canonicalisation, INT4
 // quantization, and CosSim(P_new, P_prev) = (1/r) sum_i sigma_i(P_new^T P_prev)
@@ -322,18 +323,31 @@ struct OrthBufs {
   int* flag;
 };
 
-// Shifted Cholesky-QR, three passes (Fukaya et al. 2020): X (rows x k fp32,
-// stride ld) becomes an orthonormal basis of its column span.  Each pass: Gram
+// Shifted Cholesky-QR (Fukaya et al. 2020): X (rows x k fp32, stride ld)
+// becomes a basis of its column span.  The first pass adds the shift to the
+// Gram matrix (it keeps the Cholesky factorisation from breaking down, whatever
+// the condition number of X); the others are plain Cholesky-QR.  Each pass: Gram
 // matrix in float32 (SIMT), Cholesky L L^T, the explicit inverse L^-1, then
 // X <- X L^-T on the tensor cores with bf16 hi + lo parts of both operands
 // (three products, fp32 accumulation, about 16 significant bits per pass; the
 // next pass corrects the residual).  On return Xb and Xlo hold the bf16 hi and
 // lo parts of the result (both are also used as scratch).
+//   Subspace iteration depends only on the subspaces its bases span, so an
+// intermediate basis needs to be well conditioned, not orthonormal to working
+// precision: after the shifted and one plain pass its columns are orthonormal
+// to about kappa^2 u (kappa the condition number of the product with G it came
+// from), so the next product's condition number stays that of G's top
+// directions, and that product reads only the basis' bf16 hi part.  The final
+// basis, which Rayleigh-Ritz needs orthonormal, takes the third pass.  (The
+// shifted pass alone does not lower the condition number much at these sizes:
+// the shift exceeds sigma_max^2 of X once rows k is large, so one shifted pass
+// per intermediate basis lets the condition numbers compound from one product
+// with G to the next.)
 cudaError_t orth(float* X, uint16_t* Xb, uint16_t* Xlo, int rows, int k, int64_t ld, const OrthBufs& ob,
-                 cudaStream_t s) {
+                 int passes, cudaStream_t s) {
   cudaError_t e;
   const int64_t xcnt = int64_t(rows) * ld, lcnt = int64_t(k) * ld;
-  for (int pass = 0; pass < 3; ++pass) {
+  for (int pass = 0; pass < passes; ++pass) {
     {
       const int ntiles = gram_tiles(k);
       const int slices = std::max(1, std::min(kGramSlicesMax, rows / 512));
@@ -498,12 +512,16 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
     if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
   }
   if (launch_gemm_f32(a.G, a.ldg, false, Om, ldk, false, Y, ldk, m, k, n, s) != cudaSuccess) return QG_ECUDA;
-  if (orth(Y, Yb, Ylo, m, k, ldk, ob, s) != cudaSuccess) return QG_ECUDA;
+  // two passes for the intermediate bases, three for the final Q
+  constexpr int kInterPasses = 2, kFinalPasses = 3;
+  if (orth(Y, Yb, Ylo, m, k, ldk, ob, a.power_iters > 0 ? kInterPasses : kFinalPasses, s) != cudaSuccess)
+    return QG_ECUDA;
   for (int it = 0; it < a.power_iters; ++it) {
     if (launch_gemm_f32(a.G, a.ldg, true, Yb, ldk, false, Z, ldk, n, k, m, s) != cudaSuccess) return QG_ECUDA;
-    if (orth(Z, Zb, Zlo, n, k, ldk, ob, s) != cudaSuccess) return QG_ECUDA;
+    if (orth(Z, Zb, Zlo, n, k, ldk, ob, kInterPasses, s) != cudaSuccess) return QG_ECUDA;
     if (launch_gemm_f32(a.G, a.ldg, false, Zb, ldk, false, Y, ldk, m, k, n, s) != cudaSuccess) return QG_ECUDA;
-    if (orth(Y, Yb, Ylo, m, k, ldk, ob, s) != cudaSuccess) return QG_ECUDA;
+    const int passes = it + 1 == a.power_iters ? kFinalPasses : kInterPasses;
+    if (orth(Y, Yb, Ylo, m, k, ldk, ob, passes, s) != cudaSuccess) return QG_ECUDA;
   }
   // Rayleigh-Ritz: B = Q^T G, S = B B^T, eigenpairs of S
   // B = Q^T G with Q split into bf16 hi + lo parts (about 16 significant bits)
