@@ -657,6 +657,82 @@ QG_DEV void bj_reorthogonalize(BJShared& sh) {
   __syncthreads();
 }
 
+// M = J L J^T by one cyclic Jacobi sweep (parallel ordering of the 2 kBJW
+// columns) on the pair's Gram matrix in sh.M; J ends in sh.J.  The rotations
+// come from rsqrt and approximate reciprocals: their angles only steer the
+// outer iteration, whose stopping rule reads the Gram matrix itself, and the
+// Newton-Schulz step that follows puts J back on the orthogonal group.
+QG_DEV void bj_inner_sweep(BJShared& sh) {
+  const int tid = threadIdx.x;
+  {
+    float(*Mc)[kBJP + 1] = sh.M;
+    float(*Mn)[kBJP + 1] = sh.T;
+    float(*Jc)[kBJP + 1] = sh.J;
+    float(*Jn)[kBJP + 1] = sh.JT;
+    for (int e = tid; e < kBJP * kBJP; e += blockDim.x) Jc[e / kBJP][e % kBJP] = (e / kBJP == e % kBJP) ? 1.f : 0.f;
+    for (int step = 0; step < kBJP - 1; ++step) {
+      if (tid < kBJP / 2) {
+        const int aa = tid, bb = kBJP - 1 - tid;
+        const int p = (aa == 0) ? 0 : ((aa - 1 + step) % (kBJP - 1)) + 1;
+        const int q = ((bb - 1 + step) % (kBJP - 1)) + 1;
+        const float al = Mc[p][p], be = Mc[q][q], ga = Mc[p][q];
+        float c = 1.f, sn = 0.f;
+        if (fabsf(ga) * rsqrtf(al) * rsqrtf(be) > kBJInnerTol) {
+          const float zeta = __fdividef(be - al, 2.f * ga);
+          const float az = fabsf(zeta);
+          float t;
+          if (az < 1e18f) {
+            const float x = __fmaf_rn(zeta, zeta, 1.f);
+            t = copysignf(__fdividef(1.f, az + x * rsqrtf(x)), zeta);
+          } else {
+            t = __fdividef(0.5f, zeta);
+          }
+          c = rsqrtf(__fmaf_rn(t, t, 1.f));
+          sn = c * t;
+        }
+        sh.c[tid] = c;
+        sh.s[tid] = sn;
+        sh.pp[tid] = p;
+        sh.qq[tid] = q;
+        sh.part[p] = tid;
+        sh.part[q] = tid + kBJP;
+      }
+      __syncthreads();
+      // M' = R^T M R and J' = J R in one pass: thread t owns column t % 32
+      // and rows t / 32 + 8 u
+      {
+        const int j = tid & (kBJP - 1), i0 = tid >> 5;
+        const int paj = sh.part[j], prj = paj & (kBJP - 1);
+        const int pj = sh.pp[prj], qj = sh.qq[prj];
+        const float cj = sh.c[prj], sj = sh.s[prj];
+        const float cpj = paj >= kBJP ? sj : cj, cqj = paj >= kBJP ? cj : -sj;
+#pragma unroll
+        for (int u = 0; u < kBJP / 8; ++u) {
+          const int i = i0 + 8 * u;
+          const int pai = sh.part[i], pri = pai & (kBJP - 1);
+          const int pi = sh.pp[pri], qi = sh.qq[pri];
+          const float ci = sh.c[pri], si = sh.s[pri];
+          const float cpi = pai >= kBJP ? si : ci, cqi = pai >= kBJP ? ci : -si;
+          const float tp = __fmaf_rn(cpj, Mc[pi][pj], cqj * Mc[pi][qj]);
+          const float tq = __fmaf_rn(cpj, Mc[qi][pj], cqj * Mc[qi][qj]);
+          Mn[i][j] = __fmaf_rn(cpi, tp, cqi * tq);
+          Jn[i][j] = __fmaf_rn(cpj, Jc[i][pj], cqj * Jc[i][qj]);
+        }
+      }
+      __syncthreads();
+      float(*tm)[kBJP + 1] = Mc;
+      Mc = Mn;
+      Mn = tm;
+      tm = Jc;
+      Jc = Jn;
+      Jn = tm;
+    }
+    if (Jc != sh.J) {
+      for (int e = tid; e < kBJP * kBJP; e += blockDim.x) sh.J[e / kBJP][e % kBJP] = Jc[e / kBJP][e % kBJP];
+    }
+  }
+}
+
 // Rows of At (or Vt) belonging to the pair: local l -> global row, or -1.
 QG_DEV int bj_row(int l, int I, int Jb, int k) {
   const int g = l < kBJW ? I * kBJW + l : Jb * kBJW + (l - kBJW);
@@ -874,78 +950,7 @@ __global__ void __launch_bounds__(256) jacobi_kernel(float* At, float* Vt, int64
         }
         __syncthreads();
         if (!sh.rotate) continue;
-        // ---- M = J L J^T by one cyclic Jacobi sweep (parallel ordering of the
-        // 2 kBJW columns).  The rotations come from rsqrt and approximate
-        // reciprocals: their angles only steer the outer iteration, whose stopping
-        // rule reads the Gram matrix itself, and the Newton-Schulz step below puts
-        // J back on the orthogonal group.
-        {
-          float(*Mc)[kBJP + 1] = sh.M;
-          float(*Mn)[kBJP + 1] = sh.T;
-          float(*Jc)[kBJP + 1] = sh.J;
-          float(*Jn)[kBJP + 1] = sh.JT;
-          for (int e = tid; e < kBJP * kBJP; e += blockDim.x) Jc[e / kBJP][e % kBJP] = (e / kBJP == e % kBJP) ? 1.f : 0.f;
-          for (int step = 0; step < kBJP - 1; ++step) {
-            if (tid < kBJP / 2) {
-              const int aa = tid, bb = kBJP - 1 - tid;
-              const int p = (aa == 0) ? 0 : ((aa - 1 + step) % (kBJP - 1)) + 1;
-              const int q = ((bb - 1 + step) % (kBJP - 1)) + 1;
-              const float al = Mc[p][p], be = Mc[q][q], ga = Mc[p][q];
-              float c = 1.f, sn = 0.f;
-              if (fabsf(ga) * rsqrtf(al) * rsqrtf(be) > kBJInnerTol) {
-                const float zeta = __fdividef(be - al, 2.f * ga);
-                const float az = fabsf(zeta);
-                float t;
-                if (az < 1e18f) {
-                  const float x = __fmaf_rn(zeta, zeta, 1.f);
-                  t = copysignf(__fdividef(1.f, az + x * rsqrtf(x)), zeta);
-                } else {
-                  t = __fdividef(0.5f, zeta);
-                }
-                c = rsqrtf(__fmaf_rn(t, t, 1.f));
-                sn = c * t;
-              }
-              sh.c[tid] = c;
-              sh.s[tid] = sn;
-              sh.pp[tid] = p;
-              sh.qq[tid] = q;
-              sh.part[p] = tid;
-              sh.part[q] = tid + kBJP;
-            }
-            __syncthreads();
-            // M' = R^T M R and J' = J R in one pass: thread t owns column t % 32
-            // and rows t / 32 + 8 u
-            {
-              const int j = tid & (kBJP - 1), i0 = tid >> 5;
-              const int paj = sh.part[j], prj = paj & (kBJP - 1);
-              const int pj = sh.pp[prj], qj = sh.qq[prj];
-              const float cj = sh.c[prj], sj = sh.s[prj];
-              const float cpj = paj >= kBJP ? sj : cj, cqj = paj >= kBJP ? cj : -sj;
-#pragma unroll
-              for (int u = 0; u < kBJP / 8; ++u) {
-                const int i = i0 + 8 * u;
-                const int pai = sh.part[i], pri = pai & (kBJP - 1);
-                const int pi = sh.pp[pri], qi = sh.qq[pri];
-                const float ci = sh.c[pri], si = sh.s[pri];
-                const float cpi = pai >= kBJP ? si : ci, cqi = pai >= kBJP ? ci : -si;
-                const float tp = __fmaf_rn(cpj, Mc[pi][pj], cqj * Mc[pi][qj]);
-                const float tq = __fmaf_rn(cpj, Mc[qi][pj], cqj * Mc[qi][qj]);
-                Mn[i][j] = __fmaf_rn(cpi, tp, cqi * tq);
-                Jn[i][j] = __fmaf_rn(cpj, Jc[i][pj], cqj * Jc[i][qj]);
-              }
-            }
-            __syncthreads();
-            float(*tm)[kBJP + 1] = Mc;
-            Mc = Mn;
-            Mn = tm;
-            tm = Jc;
-            Jc = Jn;
-            Jn = tm;
-          }
-          if (Jc != sh.J) {
-            for (int e = tid; e < kBJP * kBJP; e += blockDim.x) sh.J[e / kBJP][e % kBJP] = Jc[e / kBJP][e % kBJP];
-          }
-        }
+        bj_inner_sweep(sh);
         bj_reorthogonalize(sh);
         // ---- the pair's columns (and V's) become A J
         if (kResident) {
@@ -975,6 +980,216 @@ __global__ void __launch_bounds__(256) jacobi_kernel(float* At, float* Vt, int64
     // was within kBJStopTol (the rotations of this sweep leave the columns
     // orthogonal to about tol; float32 rounding keeps a few pairs from ever
     // passing tol exactly)
+    if (rotations == 0 || worst <= kBJStopTol) {
+      ++sweep;
+      break;
+    }
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0 && sweeps_out) *sweeps_out = sweep;
+}
+
+// ---- split variant: each block pair is shared by kBJSplit CTAs, each holding
+// the pair's 2 kBJW rows over one slice of the k columns (the slices are
+// multiples of 4 columns).  The CTAs exchange their partial Gram matrices
+// through global memory (double-buffered by the slot's exchange parity, so that
+// the next exchange never overwrites partials another CTA of the pair still
+// reads), sum them in one fixed order (every CTA gets the same M bit for bit),
+// and then run the same inner sweep and Newton-Schulz step, so that all hold the
+// same J; each applies it to its own slice.  Four times the SMs of the one-CTA
+// form work on each round's Gram matrices and updates.
+constexpr int kBJSplit = 4;
+
+__host__ __device__ inline int bj_split_width(int k) { return ((k + kBJSplit - 1) / kBJSplit + 3) / 4 * 4; }
+
+// X (2 kBJW rows x kps) <- columns [c_lo, c_lo + cw) of the pair's rows of Mat,
+// zero outside the matrix and beyond cw.
+QG_DEV void bj_load_slice(float* X, int kps, const float* Mat, int64_t ld, int I, int Jb, int k, int c_lo, int cw) {
+  const int quads = kps / 4;
+  for (int e = threadIdx.x; e < kBJP * quads; e += blockDim.x) {
+    const int l = e / quads, c = (e % quads) * 4;
+    const int g = bj_row(l, I, Jb, k);
+    const int gc = c_lo + c;
+    const int valid = (g >= 0 && c < cw && gc < k) ? min(4, k - gc) : 0;
+    const float* src = Mat + (valid ? static_cast<int64_t>(g) * ld + gc : 0);
+    cp_async16(X + l * kps + c, src, valid * 4);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+}
+
+// The slice's columns of the pair's rows of Mat <- J^T X.
+QG_DEV void bj_apply_slice(const BJShared& sh, const float* X, int kps, float* Mat, int64_t ld, int I, int Jb, int k,
+                           int c_lo, int cw) {
+  constexpr int kRows = kBJP / 4;
+  const int ig = threadIdx.x / 64, cq0 = threadIdx.x % 64;
+  for (int cq = cq0; cq < cw / 4; cq += 64) {
+    const int c = cq * 4, gc = c_lo + c;
+    if (gc >= k) break;
+    float4 out[kRows];
+#pragma unroll
+    for (int u = 0; u < kRows; ++u) out[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int l = 0; l < kBJP; ++l) {
+      const float4 x = *reinterpret_cast<const float4*>(X + l * kps + c);
+      const float4 ja = *reinterpret_cast<const float4*>(&sh.Jv[l][ig * kRows]);
+      const float4 jb = *reinterpret_cast<const float4*>(&sh.Jv[l][ig * kRows + 4]);
+      const float jr[kRows] = {ja.x, ja.y, ja.z, ja.w, jb.x, jb.y, jb.z, jb.w};
+#pragma unroll
+      for (int u = 0; u < kRows; ++u) {
+        const float j = jr[u];
+        out[u].x = __fmaf_rn(j, x.x, out[u].x);
+        out[u].y = __fmaf_rn(j, x.y, out[u].y);
+        out[u].z = __fmaf_rn(j, x.z, out[u].z);
+        out[u].w = __fmaf_rn(j, x.w, out[u].w);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kRows; ++u) {
+      const int g = bj_row(ig * kRows + u, I, Jb, k);
+      if (g < 0) continue;
+      float* dst = Mat + static_cast<int64_t>(g) * ld + gc;
+      if (gc + 4 <= k) {
+        __stcg(reinterpret_cast<float4*>(dst), out[u]);
+      } else {
+        __stcg(dst, out[u].x);
+        if (gc + 1 < k) __stcg(dst + 1, out[u].y);
+        if (gc + 2 < k) __stcg(dst + 2, out[u].z);
+      }
+    }
+  }
+}
+
+// The same Jacobi as jacobi_kernel, gridDim.x = kBJSplit x slots.  pair_ctr
+// (one counter per slot, zero at launch) and gx (slots x 2 x kBJSplit x kBJP^2
+// floats) carry the Gram exchange.
+__global__ void __launch_bounds__(256) jacobi_split_kernel(float* At, float* Vt, int64_t ld, int k, int max_sweeps,
+                                                           float tol, unsigned* bar, unsigned* pair_ctr, float* gx,
+                                                           int* sweeps_out, uint32_t* status) {
+  __shared__ BJShared sh;
+  __shared__ int ok_s;
+  extern __shared__ float4 dyn_smem[];
+  float* Xr = reinterpret_cast<float*>(dyn_smem);
+  const int cw = bj_split_width(k);
+  const int kps = bj_resident_stride(cw);
+  const int tid = threadIdx.x;
+  const int sub = blockIdx.x % kBJSplit, slot = blockIdx.x / kBJSplit, nslots = gridDim.x / kBJSplit;
+  const int c_lo = sub * cw;
+  const int nblk = (k + kBJW - 1) / kBJW;
+  const int nb = nblk + (nblk & 1);
+  const int npairs = nb / 2;
+  unsigned* rot = bar + 3;
+  unsigned nex = 0;  // exchanges of this slot so far (the same in its kBJSplit CTAs)
+  int sweep = 0;
+  for (; sweep < max_sweeps; ++sweep) {
+    for (int round = 0; round < nb - 1; ++round) {
+      for (int pidx = slot; pidx < npairs; pidx += nslots) {
+        const int a = pidx, b = nb - 1 - pidx;
+        const int I = (a == 0) ? 0 : ((a - 1 + round) % (nb - 1)) + 1;
+        const int Jb = ((b - 1 + round) % (nb - 1)) + 1;
+        if (I >= nblk || Jb >= nblk) continue;  // paired with the dummy player
+        // ---- partial Gram matrix over this CTA's slice (2 x 2 outputs per thread)
+        const int ty = tid >> 4, tx = tid & 15;
+        __syncthreads();
+        bj_load_slice(Xr, kps, At, ld, I, Jb, k, c_lo, cw);
+        {
+          const float* ra0 = Xr + ty * kps;
+          const float* ra1 = ra0 + 16 * kps;
+          const float* rb0 = Xr + tx * kps;
+          const float* rb1 = rb0 + 16 * kps;
+          float4 s00 = make_float4(0.f, 0.f, 0.f, 0.f), s01 = s00, s10 = s00, s11 = s00;
+#pragma unroll 4
+          for (int c = 0; c < kps; c += 4) {
+            const float4 a0 = *reinterpret_cast<const float4*>(ra0 + c), a1 = *reinterpret_cast<const float4*>(ra1 + c);
+            const float4 b0 = *reinterpret_cast<const float4*>(rb0 + c), b1 = *reinterpret_cast<const float4*>(rb1 + c);
+            s00.x = __fmaf_rn(a0.x, b0.x, s00.x); s00.y = __fmaf_rn(a0.y, b0.y, s00.y);
+            s00.z = __fmaf_rn(a0.z, b0.z, s00.z); s00.w = __fmaf_rn(a0.w, b0.w, s00.w);
+            s01.x = __fmaf_rn(a0.x, b1.x, s01.x); s01.y = __fmaf_rn(a0.y, b1.y, s01.y);
+            s01.z = __fmaf_rn(a0.z, b1.z, s01.z); s01.w = __fmaf_rn(a0.w, b1.w, s01.w);
+            s10.x = __fmaf_rn(a1.x, b0.x, s10.x); s10.y = __fmaf_rn(a1.y, b0.y, s10.y);
+            s10.z = __fmaf_rn(a1.z, b0.z, s10.z); s10.w = __fmaf_rn(a1.w, b0.w, s10.w);
+            s11.x = __fmaf_rn(a1.x, b1.x, s11.x); s11.y = __fmaf_rn(a1.y, b1.y, s11.y);
+            s11.z = __fmaf_rn(a1.z, b1.z, s11.z); s11.w = __fmaf_rn(a1.w, b1.w, s11.w);
+          }
+          float* mine = gx + ((static_cast<size_t>(slot) * 2 + (nex & 1u)) * kBJSplit + sub) * (kBJP * kBJP);
+          __stcg(mine + ty * kBJP + tx, (s00.x + s00.y) + (s00.z + s00.w));
+          __stcg(mine + ty * kBJP + tx + 16, (s01.x + s01.y) + (s01.z + s01.w));
+          __stcg(mine + (ty + 16) * kBJP + tx, (s10.x + s10.y) + (s10.z + s10.w));
+          __stcg(mine + (ty + 16) * kBJP + tx + 16, (s11.x + s11.y) + (s11.z + s11.w));
+        }
+        // ---- the pair's kBJSplit partials meet (bounded wait)
+        __syncthreads();
+        ++nex;
+        if (tid == 0) {
+          __threadfence();
+          atomicAdd(pair_ctr + slot, 1u);
+          const unsigned target = kBJSplit * nex;
+          volatile unsigned* ctr = pair_ctr + slot;
+          volatile unsigned* bad = bar + 2;
+          int ok = 1;
+          const uint64_t t0 = globaltimer();
+          while (*ctr < target) {
+            if (*bad || globaltimer() - t0 > kWaitLimitNs) {
+              ok = 0;
+              atomicExch(bar + 2, 1u);
+              if (status) atomicOr(status, kErrTimeout);
+              break;
+            }
+          }
+          __threadfence();
+          ok_s = ok;
+        }
+        __syncthreads();
+        if (!ok_s) return;
+        {
+          const float* base = gx + (static_cast<size_t>(slot) * 2 + ((nex - 1u) & 1u)) * kBJSplit * (kBJP * kBJP);
+          for (int e = tid; e < kBJP * kBJP; e += blockDim.x) {
+            float v = __ldcg(base + e);
+#pragma unroll
+            for (int q = 1; q < kBJSplit; ++q) v += __ldcg(base + q * (kBJP * kBJP) + e);
+            sh.M[e / kBJP][e % kBJP] = v;
+          }
+        }
+        if (tid == 0) sh.rotate = 0;
+        __syncthreads();
+        // ---- already orthogonal to tol?  (and the sweep's largest relative
+        // off-diagonal entry, for the stopping rule)
+        {
+          float worst = 0.f;
+          for (int e = tid; e < kBJP * kBJP; e += blockDim.x) {
+            const int p = e / kBJP, q = e % kBJP;
+            if (p < q) {
+              const float dd = sh.M[p][p] * sh.M[q][q];
+              const float rel = dd > 0.f ? fabsf(sh.M[p][q]) * rsqrtf(sh.M[p][p]) * rsqrtf(sh.M[q][q]) : 0.f;
+              if (rel > tol) sh.rotate = 1;
+              worst = fmaxf(worst, rel);
+            }
+          }
+          for (int o = 16; o > 0; o >>= 1) worst = fmaxf(worst, __shfl_xor_sync(0xFFFFFFFFu, worst, o));
+          if (sub == 0 && (tid & 31) == 0 && worst > 0.f) atomicMax(bar + 4, __float_as_uint(worst));
+        }
+        __syncthreads();
+        if (!sh.rotate) continue;
+        bj_inner_sweep(sh);
+        bj_reorthogonalize(sh);
+        // ---- this slice of the pair's columns (and V's) becomes A J
+        bj_apply_slice(sh, Xr, kps, At, ld, I, Jb, k, c_lo, cw);
+        if (Vt) {
+          __syncthreads();
+          bj_load_slice(Xr, kps, Vt, ld, I, Jb, k, c_lo, cw);
+          bj_apply_slice(sh, Xr, kps, Vt, ld, I, Jb, k, c_lo, cw);
+        }
+        if (sub == 0 && tid == 0) atomicAdd(rot, 1u);
+      }
+      if (!grid_barrier(bar, gridDim.x, status)) return;
+    }
+    const unsigned rotations = *reinterpret_cast<volatile unsigned*>(rot);
+    const float worst = __uint_as_float(*reinterpret_cast<volatile unsigned*>(bar + 4));
+    if (!grid_barrier(bar, gridDim.x, status)) return;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      atomicExch(rot, 0u);
+      atomicExch(bar + 4, 0u);
+    }
+    if (!grid_barrier(bar, gridDim.x, status)) return;
     if (rotations == 0 || worst <= kBJStopTol) {
       ++sweep;
       break;

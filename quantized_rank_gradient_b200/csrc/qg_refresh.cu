@@ -39,9 +39,16 @@ size_t r256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct RefreshLayout {
   int k, ldk, ldn4;
-  size_t P, omega, Y, Yb, Ylo, Z, Zb, Zlo, gram, gpart, linv, Li, Tt, Lih, Lil, Bm, At, Vt, lam, perm, Vsel, Pa, Pb, Ct, misc,
-      total;
+  size_t P, omega, Y, Yb, Ylo, Z, Zb, Zlo, gram, gpart, linv, Li, Tt, Lih, Lil, Bm, At, Vt, lam, perm, Vsel, Pa, Pb, Ct, jx,
+      misc, total;
 };
+
+// Scratch of the split Jacobi on a k x k matrix: one exchange counter per block
+// pair, then two buffers of kBJSplit partial Gram matrices per pair.
+size_t jacobi_scratch_bytes(int k) {
+  const int nblk = (k + kBJW - 1) / kBJW, pairs = (nblk + (nblk & 1)) / 2;
+  return r256(size_t(pairs) * 4) + size_t(pairs) * 2 * kBJSplit * kBJP * kBJP * 4;
+}
 
 constexpr int kGramSlicesMax = 32;
 int gram_tiles(int k) {
@@ -85,6 +92,7 @@ RefreshLayout refresh_layout(int m, int n, int r, int p) {
   L.Pa = take(size_t(m) * r * 4);
   L.Pb = take(size_t(m) * r * 4);
   L.Ct = take(size_t(r) * r * 4);
+  L.jx = take(jacobi_scratch_bytes(L.k));
   L.misc = take(256);
   L.total = off;
   return L;
@@ -376,30 +384,43 @@ cudaError_t orth(float* X, uint16_t* Xb, uint16_t* Xlo, int rows, int k, int64_t
   return cudaGetLastError();
 }
 
-// One-sided Jacobi on the k x k matrix stored transposed in At (and Vt, if any).
+// One-sided Jacobi on the k x k matrix stored transposed in At (and Vt, if any);
+// jx: jacobi_scratch_bytes(k) bytes.  Up to kBJResidentMaxK each block pair is
+// shared by kBJSplit CTAs (jacobi_split_kernel); above, one CTA per pair streams
+// its rows through shared memory.
 cudaError_t jacobi(float* At, float* Vt, int64_t ld, int k, unsigned* bar, int* sweeps, uint32_t* status,
-                   cudaStream_t s) {
+                   uint8_t* jx, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(bar, 0, 8 * sizeof(unsigned), s);
   if (e != cudaSuccess) return e;
   const int nblk = (k + kBJW - 1) / kBJW;
   const int pairs = (nblk + (nblk & 1)) / 2;
-  int grid = std::max(1, pairs);
-  const bool resident = k <= kBJResidentMaxK;
-  const size_t dyn = resident ? size_t(kBJP) * bj_resident_stride(k) * sizeof(float) : 0;
-  void* fn = resident ? reinterpret_cast<void*>(jacobi_kernel<true>) : reinterpret_cast<void*>(jacobi_kernel<false>);
-  if (resident) {
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn));
-    if (e != cudaSuccess) return e;
-  }
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, 256, dyn);
-  if (e != cudaSuccess) return e;
-  grid = std::min(grid, std::max(1, per_sm) * sm_count());
   int max_sweeps = kJacobiMaxSweeps;
   float tol = kJacobiTol;
+  int per_sm = 0;
+  if (k <= kBJResidentMaxK) {
+    unsigned* pair_ctr = reinterpret_cast<unsigned*>(jx);
+    float* gx = reinterpret_cast<float*>(jx + r256(size_t(pairs) * 4));
+    if ((e = cudaMemsetAsync(pair_ctr, 0, size_t(pairs) * 4, s)) != cudaSuccess) return e;
+    const size_t dyn = size_t(kBJP) * bj_resident_stride(bj_split_width(k)) * sizeof(float);
+    void* fn = reinterpret_cast<void*>(jacobi_split_kernel);
+    if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn))) !=
+        cudaSuccess)
+      return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, 256, dyn)) != cudaSuccess) return e;
+    // every CTA of a cooperative launch is resident: as many pair slots as fit
+    const int slots = std::max(1, std::min(pairs, std::max(1, per_sm) * sm_count() / kBJSplit));
+    void* args[] = {&At, &Vt, &ld, &k, &max_sweeps, &tol, &bar, &pair_ctr, &gx, &sweeps, &status};
+    const int tok = profile_begin(s, QG_KERNEL_OTHER, 0.0, 0.0);
+    e = cudaLaunchCooperativeKernel(fn, dim3(slots * kBJSplit), dim3(256), args, dyn, s);
+    profile_end(s, tok);
+    return e;
+  }
+  void* fn = reinterpret_cast<void*>(jacobi_kernel<false>);
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, 256, 0)) != cudaSuccess) return e;
+  const int grid = std::min(std::max(1, pairs), std::max(1, per_sm) * sm_count());
   void* args[] = {&At, &Vt, &ld, &k, &max_sweeps, &tol, &bar, &sweeps, &status};
   const int tok = profile_begin(s, QG_KERNEL_OTHER, 0.0, 0.0);
-  e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(256), args, dyn, s);
+  e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(256), args, 0, s);
   profile_end(s, tok);
   return e;
 }
@@ -407,10 +428,10 @@ cudaError_t jacobi(float* At, float* Vt, int64_t ld, int k, unsigned* bar, int* 
 // CosSim of Pa, Pb (fp32 m x r, stride ld) into d_out: Ct = Pb^T Pa holds the
 // columns of C = Pa^T Pb as rows; one-sided Jacobi; mean of the column norms.
 cudaError_t cossim_core(const float* Pa, const float* Pb, int m, int r, int64_t ld, float* Ct, unsigned* bar,
-                        int* sweeps, float* d_out, uint32_t* status, cudaStream_t s) {
+                        int* sweeps, float* d_out, uint32_t* status, uint8_t* jx, cudaStream_t s) {
   cudaError_t e = sgemm(true, false, Pb, ld, Pa, ld, Ct, r, r, r, m, s);
   if (e != cudaSuccess) return e;
-  if ((e = jacobi(Ct, nullptr, r, r, bar, sweeps, status, s)) != cudaSuccess) return e;
+  if ((e = jacobi(Ct, nullptr, r, r, bar, sweeps, status, jx, s)) != cudaSuccess) return e;
   mean_row_norm_kernel<<<1, 1024, 0, s>>>(Ct, r, r, d_out);
   return cudaGetLastError();
 }
@@ -473,7 +494,7 @@ size_t refresh_scratch_bytes(int32_t m, int32_t n, int32_t r, int32_t oversample
   return refresh_layout(m, n, r, oversample).total;
 }
 
-size_t cossim_scratch_bytes(int32_t, int32_t r) { return r256(size_t(r) * r * 4) + 256; }
+size_t cossim_scratch_bytes(int32_t, int32_t r) { return r256(size_t(r) * r * 4) + 256 + jacobi_scratch_bytes(r); }
 
 qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaStream_t s, float* cossim) {
   const RefreshLayout L = refresh_layout(a.m, a.n, a.r, a.oversample);
@@ -534,7 +555,7 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
     identity_kernel<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, s>>>(Vt, ldk, k);
     if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
   }
-  if (jacobi(At, Vt, ldk, k, misc->bar, &misc->sweeps, a.status, s) != cudaSuccess) return QG_ECUDA;
+  if (jacobi(At, Vt, ldk, k, misc->bar, &misc->sweeps, a.status, ws + L.jx, s) != cudaSuccess) return QG_ECUDA;
   row_norms_kernel<<<(k * 32 + 255) / 256, 256, 0, s>>>(At, ldk, k, k, lam);
   if (cudaMemsetAsync(perm, 0, size_t(k) * sizeof(int), s) != cudaSuccess) return QG_ECUDA;
   rank_sort_kernel<<<1, 1024, 0, s>>>(lam, k, perm);
@@ -560,7 +581,8 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
     dequant_f32_kernel<<<blocks, 256, 0, s>>>(a.Pq, a.sP, static_cast<int64_t>(mr), Pa);
     dequant_f32_kernel<<<blocks, 256, 0, s>>>(a.Pq_prev, a.sP_prev, static_cast<int64_t>(mr), Pb);
     if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
-    if (cossim_core(Pa, Pb, m, r, r, Ct, misc->bar, &misc->sweeps, &misc->cossim, a.status, s) != cudaSuccess)
+    if (cossim_core(Pa, Pb, m, r, r, Ct, misc->bar, &misc->sweeps, &misc->cossim, a.status, ws + L.jx, s) !=
+        cudaSuccess)
       return QG_ECUDA;
     float host = 0.f;
     if (cudaMemcpyAsync(&host, &misc->cossim, sizeof(float), cudaMemcpyDeviceToHost, s) != cudaSuccess) return QG_ECUDA;
@@ -575,7 +597,8 @@ qg_status run_cossim(const float* Pa, const float* Pb, int32_t m, int32_t r, int
   float* Ct = reinterpret_cast<float*>(ws);
   unsigned* bar = reinterpret_cast<unsigned*>(ws + r256(size_t(r) * r * 4));
   int* sweeps = reinterpret_cast<int*>(bar + 8);
-  return st_of(cossim_core(Pa, Pb, m, r, ld, Ct, bar, sweeps, d_out, nullptr, stream));
+  uint8_t* jx = ws + r256(size_t(r) * r * 4) + 256;
+  return st_of(cossim_core(Pa, Pb, m, r, ld, Ct, bar, sweeps, d_out, nullptr, jx, stream));
 }
 
 }  // namespace qg
