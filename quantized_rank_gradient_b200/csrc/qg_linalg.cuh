@@ -672,9 +672,11 @@ QG_DEV void bj_inner_sweep(BJShared& sh) {
     for (int e = tid; e < kBJP * kBJP; e += blockDim.x) Jc[e / kBJP][e % kBJP] = (e / kBJP == e % kBJP) ? 1.f : 0.f;
     for (int step = 0; step < kBJP - 1; ++step) {
       if (tid < kBJP / 2) {
-        const int aa = tid, bb = kBJP - 1 - tid;
-        const int p = (aa == 0) ? 0 : ((aa - 1 + step) % (kBJP - 1)) + 1;
-        const int q = ((bb - 1 + step) % (kBJP - 1)) + 1;
+        // round-robin: player 0 fixed, players 1..31 move one place per step;
+        // pair tid joins positions tid and kBJP - 1 - tid
+        const int vp = tid - 1 + step, vq = kBJP - 2 - tid + step;
+        const int p = tid == 0 ? 0 : (vp >= kBJP - 1 ? vp - (kBJP - 1) : vp) + 1;
+        const int q = (vq >= kBJP - 1 ? vq - (kBJP - 1) : vq) + 1;
         const float al = Mc[p][p], be = Mc[q][q], ga = Mc[p][q];
         float c = 1.f, sn = 0.f;
         if (fabsf(ga) * rsqrtf(al) * rsqrtf(be) > kBJInnerTol) {
@@ -699,24 +701,39 @@ QG_DEV void bj_inner_sweep(BJShared& sh) {
       }
       __syncthreads();
       // M' = R^T M R and J' = J R in one pass: thread t owns column t % 32
-      // and rows t / 32 + 8 u
+      // and rows t / 32 + 8 u.  Every load comes before the first store (the
+      // buffers are distinct, but the compiler cannot know it, and would
+      // otherwise keep each row's loads behind the previous row's stores).
       {
+        constexpr int kU = kBJP / 8;
         const int j = tid & (kBJP - 1), i0 = tid >> 5;
         const int paj = sh.part[j], prj = paj & (kBJP - 1);
         const int pj = sh.pp[prj], qj = sh.qq[prj];
         const float cj = sh.c[prj], sj = sh.s[prj];
         const float cpj = paj >= kBJP ? sj : cj, cqj = paj >= kBJP ? cj : -sj;
+        float cpi[kU], cqi[kU], mpp[kU], mpq[kU], mqp[kU], mqq[kU], jp[kU], jq[kU];
 #pragma unroll
-        for (int u = 0; u < kBJP / 8; ++u) {
+        for (int u = 0; u < kU; ++u) {
           const int i = i0 + 8 * u;
           const int pai = sh.part[i], pri = pai & (kBJP - 1);
           const int pi = sh.pp[pri], qi = sh.qq[pri];
           const float ci = sh.c[pri], si = sh.s[pri];
-          const float cpi = pai >= kBJP ? si : ci, cqi = pai >= kBJP ? ci : -si;
-          const float tp = __fmaf_rn(cpj, Mc[pi][pj], cqj * Mc[pi][qj]);
-          const float tq = __fmaf_rn(cpj, Mc[qi][pj], cqj * Mc[qi][qj]);
-          Mn[i][j] = __fmaf_rn(cpi, tp, cqi * tq);
-          Jn[i][j] = __fmaf_rn(cpj, Jc[i][pj], cqj * Jc[i][qj]);
+          cpi[u] = pai >= kBJP ? si : ci;
+          cqi[u] = pai >= kBJP ? ci : -si;
+          mpp[u] = Mc[pi][pj];
+          mpq[u] = Mc[pi][qj];
+          mqp[u] = Mc[qi][pj];
+          mqq[u] = Mc[qi][qj];
+          jp[u] = Jc[i][pj];
+          jq[u] = Jc[i][qj];
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int i = i0 + 8 * u;
+          const float tp = __fmaf_rn(cpj, mpp[u], cqj * mpq[u]);
+          const float tq = __fmaf_rn(cpj, mqp[u], cqj * mqq[u]);
+          Mn[i][j] = __fmaf_rn(cpi[u], tp, cqi[u] * tq);
+          Jn[i][j] = __fmaf_rn(cpj, jp[u], cqj * jq[u]);
         }
       }
       __syncthreads();
