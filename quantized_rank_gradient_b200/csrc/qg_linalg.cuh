@@ -1,17 +1,18 @@
 // Small dense linear algebra for the subspace refresh (float32, SIMT):
 //   sgemm_kernel        C = op(A) op(B) (64 x 64 tiles, 4 x 4 outputs per thread)
-//   potrf_diag_kernel   Cholesky of one 32 x 32 diagonal block + its inverse
-//   trsm_panel_kernel   L[i, jb] = A[i, jb] * inv(L[jb, jb])^T below the block
-//   syrk_update_kernel  trailing update A -= L[:, jb] L[:, jb]^T (lower tiles)
+//   cholesky_kernel     blocked (32-wide) Cholesky in one cooperative launch
 //   sgemm_batched_kernel  the same tiles over a batch of equal-size blocks
+//   gram_partial_kernel, gram_reduce_kernel
+//                       lower triangle of X^T X, split over row slices with a
+//                       fixed-order reduction
 //   trinv_init_kernel   block-diagonal start of L^-1 by recursive doubling
 //   split_bf16_kernel   float32 -> bf16 hi + lo parts (tensor-core operands)
-//   trsm_rows_kernel    X <- X L^-T for a tall X, 32 rows per CTA
 //   jacobi_kernel       block one-sided (Hestenes) Jacobi on the columns of a
 //                       square matrix: round-robin pairs of 16-column blocks, one
 //                       CTA per pair, the pair's 32 x 32 Gram diagonalised in
 //                       shared memory, a bounded grid barrier between rounds
 //                       (cooperative launch)
+//   jacobi_split_kernel the same with each pair shared by four CTAs
 #pragma once
 
 #include "qg_device.cuh"
@@ -265,168 +266,6 @@ __global__ void split_bf16_kernel(const float* X, int64_t ld, int rows, int cols
 }
 
 // ------------------------------------------------------------------ Cholesky
-
-// Cholesky of the nb x nb diagonal block at (j0, j0) of the lower triangle of A
-// (read from the lower triangle only), written back as L; its inverse (32 x 32,
-// lower, identity-padded) goes to Linv.  One warp: lane j holds column j, and
-// the column being eliminated is broadcast by shuffles.  A pivot that is not
-// positive (the matrix is not numerically positive definite) raises *flag and is
-// replaced by a tiny positive value so that the factorisation stays finite.
-__global__ void __launch_bounds__(32) potrf_diag_kernel(float* A, int64_t ld, int j0, int nb, float* Linv,
-                                                        int* flag) {
-  __shared__ float Ls[32][33];
-  const int j = threadIdx.x;
-  float col[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    float v = (i == j) ? 1.f : 0.f;
-    if (i < nb && j < nb && j <= i) v = A[static_cast<int64_t>(j0 + i) * ld + j0 + j];
-    col[i] = (j <= i) ? v : 0.f;
-  }
-#pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    float d = __shfl_sync(0xFFFFFFFFu, col[c], c);
-    if (!(d > 0.f)) {
-      if (j == 0 && c < nb) atomicOr(flag, 1);
-      d = 1e-30f;
-    }
-    const float l = sqrtf(d);
-    if (j == c) {
-      col[c] = l;
-#pragma unroll
-      for (int i = c + 1; i < 32; ++i) col[i] = col[i] / l;
-    }
-    // broadcast column c (rows > c) and update the columns to its right:
-    // col_j[i] -= L[i][c] L[j][c] for i >= j > c; L[j][c] arrives at i == j,
-    // before any row i >= j needs it
-    float ljc = 0.f;
-#pragma unroll
-    for (int i = c + 1; i < 32; ++i) {
-      const float lic = __shfl_sync(0xFFFFFFFFu, col[i], c);
-      if (i == j) ljc = lic;
-      if (j > c && i >= j) col[i] = col[i] - lic * ljc;
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    Ls[i][j] = col[i];
-    if (i < nb && j < nb) A[static_cast<int64_t>(j0 + i) * ld + j0 + j] = (j <= i) ? col[i] : 0.f;
-  }
-  __syncwarp();
-  // inverse: column j of inv(L) by forward substitution
-  float x[32];
-#pragma unroll
-  for (int r = 0; r < 32; ++r) {
-    float s = (r == j) ? 1.f : 0.f;
-#pragma unroll
-    for (int t = 0; t < r; ++t) s -= Ls[r][t] * x[t];
-    x[r] = (r >= j) ? s / Ls[r][r] : 0.f;
-  }
-#pragma unroll
-  for (int r = 0; r < 32; ++r) Linv[r * 32 + j] = x[r];
-}
-
-// L[i, j0 + c] = sum_c' A[i, j0 + c'] Linv[c][c'] for rows i >= j0 + 32.
-__global__ void __launch_bounds__(1024) trsm_panel_kernel(float* A, int64_t ld, int j0, int n, const float* Linv) {
-  __shared__ float R[32][33];
-  __shared__ float Li[32][33];
-  const int r = threadIdx.y, c = threadIdx.x;
-  const int row = j0 + 32 + blockIdx.x * 32 + r;
-  Li[r][c] = Linv[r * 32 + c];
-  R[r][c] = (row < n && j0 + c < n) ? A[static_cast<int64_t>(row) * ld + j0 + c] : 0.f;
-  __syncthreads();
-  float s = 0.f;
-  for (int t = 0; t <= c; ++t) s = __fmaf_rn(R[r][t], Li[c][t], s);
-  if (row < n && j0 + c < n) A[static_cast<int64_t>(row) * ld + j0 + c] = s;
-}
-
-// A[i, l] -= sum_t L[i, j0 + t] L[l, j0 + t] over the lower tiles of the
-// trailing matrix (rows and columns >= j0 + 32).
-__global__ void __launch_bounds__(1024) syrk_update_kernel(float* A, int64_t ld, int j0, int n) {
-  // blockIdx.x enumerates the lower tiles (ti >= tl) of the trailing part
-  int t = blockIdx.x, ti = 0;
-  while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
-  const int tl = t - ti * (ti + 1) / 2;
-  __shared__ float Li[32][33];
-  __shared__ float Ll[32][33];
-  const int r = threadIdx.y, c = threadIdx.x;
-  const int base = j0 + 32;
-  const int ri = base + ti * 32 + r, rl = base + tl * 32 + r;
-  Li[r][c] = (ri < n) ? A[static_cast<int64_t>(ri) * ld + j0 + c] : 0.f;
-  Ll[r][c] = (rl < n) ? A[static_cast<int64_t>(rl) * ld + j0 + c] : 0.f;
-  __syncthreads();
-  const int gi = base + ti * 32 + r, gl = base + tl * 32 + c;
-  if (gi < n && gl < n && gl <= gi) {
-    float s = 0.f;
-    for (int q = 0; q < 32; ++q) s = __fmaf_rn(Li[r][q], Ll[c][q], s);
-    float* a = A + static_cast<int64_t>(gi) * ld + gl;
-    *a = *a - s;
-  }
-}
-
-// X (rows x k, row stride ldx) <- X L^-T, i.e. solves Y L^T = X row by row, with
-// L the lower Cholesky factor (k x k, stride ldl) and Linv the inverses of its
-// 32 x 32 diagonal blocks.  Each CTA owns 32 rows kept in shared memory; also
-// writes a bf16 copy (stride ldb) when Xb is non-null and, when Xlo is
-// non-null, the bf16 rounding of the residual X - Xb (so that Xb + Xlo carries
-// about 16 significant bits).
-__global__ void __launch_bounds__(256) trsm_rows_kernel(float* X, int64_t ldx, uint16_t* Xb, uint16_t* Xlo,
-                                                        int64_t ldb, int rows, int k, const float* L, int64_t ldl,
-                                                        const float* Linv) {
-  extern __shared__ float Ys[];  // 32 x (k + 1)
-  const int kp = k + 1;
-  const int r0 = blockIdx.x * 32;
-  const int tid = threadIdx.x;
-  for (int e = tid; e < 32 * k; e += 256) {
-    const int i = e / k, c = e % k;
-    Ys[i * kp + c] = (r0 + i < rows) ? X[static_cast<int64_t>(r0 + i) * ldx + c] : 0.f;
-  }
-  __syncthreads();
-  __shared__ float acc_s[32][33];
-  const int i = tid & 31;        // row in the CTA
-  const int cg = tid >> 5;       // 4 columns: cg*4 .. cg*4+3 of the block
-  const int nblk = (k + 31) / 32;
-  for (int jb = 0; jb < nblk; ++jb) {
-    const int c0 = jb * 32;
-    float acc[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = c0 + cg * 4 + u;
-      float s = (c < k) ? Ys[i * kp + c] : 0.f;
-      if (c < k) {
-        const float* lrow = L + static_cast<int64_t>(c) * ldl;
-        for (int t = 0; t < c0; ++t) s = __fmaf_rn(-Ys[i * kp + t], lrow[t], s);
-      }
-      acc[u] = s;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) acc_s[i][cg * 4 + u] = acc[u];
-    __syncthreads();
-    const float* li = Linv + static_cast<int64_t>(jb) * 1024;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int cl = cg * 4 + u, c = c0 + cl;
-      float s = 0.f;
-      for (int t = 0; t <= cl; ++t) s = __fmaf_rn(acc_s[i][t], li[cl * 32 + t], s);
-      if (c < k) Ys[i * kp + c] = s;
-    }
-    __syncthreads();
-  }
-  for (int e = tid; e < 32 * k; e += 256) {
-    const int ii = e / k, c = e % k;
-    if (r0 + ii < rows) {
-      const float y = Ys[ii * kp + c];
-      X[static_cast<int64_t>(r0 + ii) * ldx + c] = y;
-      if (Xb) {
-        const __nv_bfloat16 hi = __float2bfloat16_rn(y);
-        Xb[static_cast<int64_t>(r0 + ii) * ldb + c] = __bfloat16_as_ushort(hi);
-        if (Xlo)
-          Xlo[static_cast<int64_t>(r0 + ii) * ldb + c] =
-              __bfloat16_as_ushort(__float2bfloat16_rn(__fsub_rn(y, __bfloat162float(hi))));
-      }
-    }
-  }
-}
 
 // ------------------------------------------------------------------ Cholesky, one launch
 
