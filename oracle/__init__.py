@@ -18,6 +18,11 @@ Pins (each checked by a CPU test against something other than the oracle):
   schedule_after_refresh - scripted CosSim sequences; gamma > 1 gives a fixed interval
   step (composed)       - alpha = 0 leaves W unchanged; mean update over seeds equals
                           alpha * P N / s (unbiasedness at the step level)
+  dequant_weight_bf16   - torch's float32 -> bfloat16 conversion of each float32
+                          product, groups straddling rows; exact unit / power-of-two /
+                          zero scales
+  linear_forward / linear_backward_data / linear_backward_weight
+                        - brute-force sums on small inputs; integer matrix products
 """
 from .qgalore import *  # noqa: F401,F403
 from . import qgalore  # noqa: F401

@@ -542,3 +542,47 @@ def set_projection(st: LayerState, P):
     """Quantize and install a given float projection (m x r) as P^Q."""
     codes, sP = quant_int4_groups(np.asarray(P, np.float32), st.cfg.p_group)
     st.Pq, st.sP = pack_int4(codes), sP
+
+
+# --------------------------------------------------------------------------
+# Linear layers around the optimizer: simulated weight-only INT8 quantization.
+# [QG-lim] AIMech Q-GaLore page, limitation "simulated weight-quantization
+# throughput" (paper section 3.2 and section 4.4, Fig. 4): activations stay in
+# 16-bit floating point and the INT8 weights are dequantized for the forward and
+# backward matrix products.  [QG-thm] same page, Theorem 3.1 (paper section
+# 3.1, Eqs. (3)-(4)): for a linear layer y = W x the weight gradient is
+# G = (1/B) D_y X^T.
+# Readings: W~ = bf16_rn(fp32(q) * s_g), one float32 product rounded to bf16,
+# with g = floor((i n + j) / 256) the group of the optimizer's own W grid; the
+# three products are the exact sums (float64 here), which the GPU rounds once to
+# bf16 after a float32 accumulation; the 1/B of G is folded into D_y, so G is
+# the bf16 gradient the optimizer step takes.
+# --------------------------------------------------------------------------
+
+
+def dequant_weight_bf16(Wq, sW, group=256) -> np.ndarray:
+    """W~ (m x n float32 holding bf16 values) from INT8 codes and the flattened
+    group scales: each element is float32(q) times its group's scale, rounded
+    once to float32 and then to bf16 (round to nearest even)."""
+    Wq = np.asarray(Wq)
+    m, n = Wq.shape
+    g = (np.arange(m, dtype=np.int64)[:, None] * n + np.arange(n, dtype=np.int64)[None, :]) // group
+    prod = Wq.astype(np.float32) * np.asarray(sW, np.float32)[g]
+    return bf16_round(prod.astype(np.float32))
+
+
+def linear_forward(X, Wt) -> np.ndarray:
+    """Y = X W~^T (T x m) for activations X (T x n) and the dequantized weight
+    W~ (m x n), exact in float64."""
+    return np.asarray(X, np.float64) @ np.asarray(Wt, np.float64).T
+
+
+def linear_backward_data(dY, Wt) -> np.ndarray:
+    """dX = D_y W~ (T x n) for the output gradient D_y (T x m), exact in float64."""
+    return np.asarray(dY, np.float64) @ np.asarray(Wt, np.float64)
+
+
+def linear_backward_weight(dY, X) -> np.ndarray:
+    """G = D_y^T X (m x n), the weight gradient of y = W x over the T rows of the
+    batch, exact in float64."""
+    return np.asarray(dY, np.float64).T @ np.asarray(X, np.float64)

@@ -543,3 +543,57 @@ def test_refresh_layer_state_flow():
     assert counts == [True, False, False, True, False, False, False, False, False, True]
     assert st.cossim_trace[0][1] is None and st.cossim_trace[1][1] > 0.9
     assert st.n_refresh == 3
+
+
+# ---------------------------------------------------------------- linear layers (INT8 weights)
+
+def test_dequant_weight_matches_torch_bf16_of_the_fp32_product():
+    # each element is one float32 product rounded by torch's float32 -> bf16 RNE;
+    # the group of (i, j) is floor((i n + j) / 256), with n = 300 so that groups
+    # straddle rows
+    rng = np.random.default_rng(11)
+    m, n = 5, 300
+    Wq = rng.integers(-127, 128, size=(m, n)).astype(np.int8)
+    ng = -(-(m * n) // 256)
+    sW = (rng.uniform(0.5, 1.5, size=ng) * 3.7e-3).astype(np.float32)
+    got = O.dequant_weight_bf16(Wq, sW)
+    for i in range(m):
+        for j in range(n):
+            p = np.float32(np.float32(Wq[i, j]) * sW[(i * n + j) // 256])
+            ref = torch.tensor([float(p)], dtype=torch.float32).to(torch.bfloat16).to(torch.float32).item()
+            assert got[i, j] == np.float32(ref), (i, j)
+
+
+def test_dequant_weight_exact_cases():
+    # unit scales give the codes; power-of-two scales give q * s with no rounding
+    Wq = np.arange(-127, 128, dtype=np.int64).reshape(5, 51).astype(np.int8)
+    assert np.array_equal(O.dequant_weight_bf16(Wq, np.ones(1, np.float32)), Wq.astype(np.float32))
+    s = np.float32(2.0 ** -9)
+    assert np.array_equal(O.dequant_weight_bf16(Wq, np.array([s], np.float32)), Wq.astype(np.float32) * s)
+    # a zero scale gives zeros
+    assert not O.dequant_weight_bf16(Wq, np.zeros(1, np.float32)).any()
+
+
+def test_linear_products_brute_force_and_integer_exact():
+    rng = np.random.default_rng(12)
+    T, m, n = 4, 3, 5
+    X = rng.standard_normal((T, n)).astype(np.float32)
+    dY = rng.standard_normal((T, m)).astype(np.float32)
+    Wt = rng.standard_normal((m, n)).astype(np.float32)
+    Y, dX, G = O.linear_forward(X, Wt), O.linear_backward_data(dY, Wt), O.linear_backward_weight(dY, X)
+    assert Y.shape == (T, m) and dX.shape == (T, n) and G.shape == (m, n)
+    for t in range(T):
+        for i in range(m):
+            assert Y[t, i] == math.fsum(float(X[t, j]) * float(Wt[i, j]) for j in range(n))
+        for j in range(n):
+            assert dX[t, j] == math.fsum(float(dY[t, i]) * float(Wt[i, j]) for i in range(m))
+    for i in range(m):
+        for j in range(n):
+            assert G[i, j] == math.fsum(float(dY[t, i]) * float(X[t, j]) for t in range(T))
+    # integer inputs: the products equal integer matrix products exactly
+    Xi = rng.integers(-50, 50, size=(7, 11))
+    Wi = rng.integers(-127, 128, size=(6, 11))
+    Di = rng.integers(-50, 50, size=(7, 6))
+    assert np.array_equal(O.linear_forward(Xi, Wi), (Xi @ Wi.T).astype(np.float64))
+    assert np.array_equal(O.linear_backward_data(Di, Wi), (Di @ Wi).astype(np.float64))
+    assert np.array_equal(O.linear_backward_weight(Di, Xi), (Di.T @ Xi).astype(np.float64))
