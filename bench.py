@@ -50,10 +50,11 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=None, help="decoder layers (default: the stack's own count)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=sorted(STACKS) + ["refresh-stress"], default="llama7b-stack",
-                    help="a decoder stack (llama7b-stack is the default and the headline), or refresh-stress: "
+    ap.add_argument("--workload", choices=sorted(STACKS) + ["refresh-stress", "linear-7b"], default="llama7b-stack",
+                    help="a decoder stack (llama7b-stack is the default and the headline); refresh-stress: "
                          "one 4096 x 11008 layer, r = 1024, a drifting gradient subspace, subspace refreshes on "
-                         "the layer-adaptive schedule (--steps defaults to 2000)")
+                         "the layer-adaptive schedule (--steps defaults to 2000); linear-7b: the INT8-weight "
+                         "forward and backward products of the LLaMA-7B stack's 224 linear layers at 8192 tokens")
     return ap.parse_args()
 
 
@@ -541,6 +542,119 @@ def run_refresh_stress(args, rank, world, local_rank):
     return 0
 
 
+LINEAR_TOKENS = 8192
+
+
+def run_linear(args, rank, world, local_rank):
+    """The INT8-weight linear layers around the optimizer (simulated weight-only
+    quantization), LLaMA-7B stack at 8192 tokens.  One step runs, for each of the
+    224 weight matrices, W~ = bf16(q s), Y = X W~^T, dX = D_y W~ and G = D_y^T X
+    through the C ABI on one stream.  Each matrix has its own INT8 weight and
+    scales.  Activations and output gradients are seeded synthetic bf16 matrices,
+    one set per layer shape, all larger than L2 together with a matrix's weight.
+    Every rank runs its own stack (weak scaling)."""
+    import torch
+    import torch.distributed as dist
+
+    import quantized_rank_gradient_b200 as qg
+    import synth
+    qg.lib()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    spec = STACKS["llama7b-stack"]
+    layers = args.layers or spec["layers"]
+    T = LINEAR_TOKENS
+    stream = c_void_p(torch.cuda.current_stream().cuda_stream)
+    shapes = [s for group in stack_shapes(layers, spec["hidden"], spec["inter"]) for s in group]
+    mats = []
+    for lid, (m, n) in enumerate(shapes):
+        seed = matrix_seed(rank, lid)
+        ldw = -(-n // 16) * 16
+        mats.append((m, n, synth.device_weight_codes(m, n, ldw, seed, device), ldw,
+                     synth.device_weight_scales(m, n, seed, device)))
+    gen = torch.Generator(device=device)
+    gen.manual_seed(4_000_117 * (rank + 1))
+    bufs = {}
+    for (m, n) in sorted(set(shapes)):
+        bf = torch.bfloat16
+        bufs[(m, n)] = dict(X=torch.randn(T, n, generator=gen, device=device).to(bf),
+                            D=(torch.randn(T, m, generator=gen, device=device) * 1e-2).to(bf),
+                            Y=torch.empty(T, m, dtype=bf, device=device), dX=torch.empty(T, n, dtype=bf, device=device),
+                            G=torch.empty(m, n, dtype=bf, device=device),
+                            Wt=torch.empty(m, -(-n // 8) * 8, dtype=bf, device=device))
+
+    def step():
+        for (m, n, W, ldw, sW) in mats:
+            b = bufs[(m, n)]
+            ldt = b["Wt"].shape[1]
+            qg.check(qg.qg_linear_dequant_weight(W.data_ptr(), ldw, sW.data_ptr(), m, n, b["Wt"].data_ptr(), ldt,
+                                                 stream), "qg_linear_dequant_weight")
+            qg.check(qg.qg_linear_forward(b["X"].data_ptr(), n, b["Wt"].data_ptr(), ldt, T, m, n, b["Y"].data_ptr(),
+                                          m, stream), "qg_linear_forward")
+            qg.check(qg.qg_linear_backward_data(b["D"].data_ptr(), m, b["Wt"].data_ptr(), ldt, T, m, n,
+                                                b["dX"].data_ptr(), n, stream), "qg_linear_backward_data")
+            qg.check(qg.qg_linear_backward_weight(b["D"].data_ptr(), m, b["X"].data_ptr(), n, T, m, n,
+                                                  b["G"].data_ptr(), n, stream), "qg_linear_backward_weight")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(bus_id_of(device))
+    clocks.start()
+    time.sleep(0.3)
+    qg.check(qg.qg_profile_enable(1))
+    barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / args.steps
+    barrier()
+    kt = (qg.qg_kernel_times * qg.QG_KERNEL_KINDS)()
+    qg.check(qg.qg_profile_collect(kt, qg.QG_KERNEL_KINDS))
+    qg.check(qg.qg_profile_enable(0))
+    clk = clocks.stop()
+    ms = reduce_max(ms, world)
+    if rank != 0:
+        return 0
+    peaks = load_peaks()
+    flops = sum(6.0 * T * m * n for (m, n, *_rest) in mats)
+    gemm, deq = kt[qg.QG_KERNEL_LINEAR_GEMM], kt[qg.QG_KERNEL_LINEAR_DEQUANT]
+    achieved = (gemm.flops / gemm.launches) / (gemm.device_ms / gemm.launches / 1000.0) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    line = {
+        "metric": "INT8-weight linear layers, forward + backward (Y = X W~^T, dX = D_y W~, G = D_y^T X): TFLOP/s",
+        "value": flops / (ms / 1000.0) / 1e12 * world, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 operands (W~ from INT8), f32 accumulate", "data": "synthetic (seeded bf16 activations and "
+        "output gradients; seeded INT8 weights and scales)",
+        "config": {"workload": f"linear-llama7b-stack-{T}tok" + ("" if layers == spec["layers"] else f"-{layers}l"),
+                   "matrices": len(mats), "tokens": T, "weights_per_gpu": sum(m * n for (m, n, *_r) in mats),
+                   "l2": "inputs larger than L2 (a matrix's weight and activations exceed 126 MB)",
+                   "parallelism": f"independent stacks x{world}"},
+        "tokens_per_s": T / (ms / 1000.0) * world,
+        "roofline": {"bound": "tensor", "kernel": "linear_gemm_tcgen05", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "peak_kind": "sustained bf16 (%s)" % peaks["source"]},
+        "kernels": {"linear_dequant_weight": {"launches_per_step": deq.launches / args.steps,
+                                              "ms_per_step": deq.device_ms / args.steps,
+                                              "gbs": deq.bytes / (deq.device_ms / 1000.0) / 1e9},
+                    "linear_gemm_tcgen05": {"launches_per_step": gemm.launches / args.steps,
+                                            "ms_per_step": gemm.device_ms / args.steps, "tflops": achieved}},
+        "gpu_launches": (gemm.launches + deq.launches),
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_e2e(stack, args, stream, world, device, barrier):
     import torch
     import torch.distributed as dist
@@ -612,6 +726,8 @@ def main():
     try:
         if args.workload == "refresh-stress":
             return run_refresh_stress(args, rank, world, local_rank)
+        if args.workload == "linear-7b":
+            return run_linear(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:

@@ -232,7 +232,9 @@ typedef enum {
   QG_KERNEL_PROJECT_ADAM = 1, /* a2 + a3: tcgen05 P^T G with the moment epilogue */
   QG_KERNEL_BACKPROJECT_SR = 2, /* a4 + a5: tcgen05 P N with stochastic rounding */
   QG_KERNEL_OTHER = 3,        /* refresh and single-stage kernels */
-  QG_KERNEL_KINDS = 4
+  QG_KERNEL_LINEAR_DEQUANT = 4, /* INT8 W -> bf16 W~ for the linear-layer products */
+  QG_KERNEL_LINEAR_GEMM = 5,  /* tcgen05 forward / backward products of a linear layer */
+  QG_KERNEL_KINDS = 6
 } qg_kernel_kind;
 
 typedef struct {
@@ -291,6 +293,39 @@ qg_status qg_selfcheck_exact_math(int32_t op, uint64_t n, uint64_t seed, unsigne
  * the wait reported failure, [1] = nanoseconds spent.  Asynchronous on
  * `stream`; QG_EINVAL for null pointers or a limit out of range. */
 qg_status qg_selfcheck_wait_timeout(uint64_t limit_ns, uint32_t* d_status, unsigned long long* d_out, void* stream);
+
+/* ---- Linear layers with INT8 weights (simulated weight-only quantization) ----
+ * The matrix products around the optimizer step (AIMech Q-GaLore page,
+ * limitation "simulated weight-quantization throughput", paper section 3.2 and
+ * section 4.4, Fig. 4: activations stay in 16-bit floating point and the INT8
+ * weights are dequantized for the forward and backward products; Theorem 3.1,
+ * paper section 3.1: the weight gradient of y = W x is G = (1/B) D_y X^T, the
+ * 1/B folded into D_y here).  For a layer whose INT8 weight W is m x n (the
+ * optimizer's W^Q with its flattened groups of 256 scales), a training step
+ * dequantizes W once and runs the three products on the tcgen05 core (bf16
+ * operands, float32 accumulation, bf16 results rounded to nearest even):
+ *   qg_linear_dequant_weight   W~ = bf16(fp32(q_ij) * s_W[(i n + j) / 256])  (m x n)
+ *   qg_linear_forward          Y  = X W~^T    X: T x n   ->  Y: T x m
+ *   qg_linear_backward_data    dX = D_y W~    D_y: T x m ->  dX: T x n
+ *   qg_linear_backward_weight  G  = D_y^T X   ->  G: m x n, the bf16 gradient
+ *                              qg_step / qg_step_batch take
+ * Every matrix is row-major and device-resident, owned by the caller; the
+ * functions allocate nothing and are asynchronous on `stream`.  bf16 strides
+ * (ld*) are in elements, at least the column count and a multiple of 8, and
+ * bf16 bases are 16-byte aligned (tensor-memory-access tiles); the INT8 W has
+ * ldw >= n, ldw % 16 == 0, a 16-byte aligned base (as qg_layer_init requires).
+ * Errors launch nothing: QG_EINVAL for a null pointer where data is needed,
+ * QG_ESHAPE for negative sizes or a bad stride, QG_EALIGN for a misaligned
+ * base, QG_ECUDA when a launch fails.  T = 0 is a no-op, except that G = 0.
+ * No output may overlap an input. */
+qg_status qg_linear_dequant_weight(const int8_t* d_W, int64_t ldw, const float* d_sW, int32_t m, int32_t n,
+                                   void* d_Wt, int64_t ldwt, void* stream);
+qg_status qg_linear_forward(const void* d_X, int64_t ldx, const void* d_Wt, int64_t ldwt, int32_t T, int32_t m,
+                            int32_t n, void* d_Y, int64_t ldy, void* stream);
+qg_status qg_linear_backward_data(const void* d_dY, int64_t lddy, const void* d_Wt, int64_t ldwt, int32_t T,
+                                  int32_t m, int32_t n, void* d_dX, int64_t lddx, void* stream);
+qg_status qg_linear_backward_weight(const void* d_dY, int64_t lddy, const void* d_X, int64_t ldx, int32_t T,
+                                    int32_t m, int32_t n, void* d_G, int64_t ldg, void* stream);
 
 #ifdef __cplusplus
 }

@@ -52,7 +52,8 @@ class qg_kernel_times(Structure):
     _fields_ = [("launches", c_int64), ("device_ms", c_double), ("flops", c_double), ("bytes", c_double)]
 
 
-QG_KERNEL_DEQUANT, QG_KERNEL_PROJECT_ADAM, QG_KERNEL_BACKPROJECT_SR, QG_KERNEL_OTHER, QG_KERNEL_KINDS = range(5)
+(QG_KERNEL_DEQUANT, QG_KERNEL_PROJECT_ADAM, QG_KERNEL_BACKPROJECT_SR, QG_KERNEL_OTHER, QG_KERNEL_LINEAR_DEQUANT,
+ QG_KERNEL_LINEAR_GEMM, QG_KERNEL_KINDS) = range(7)
 
 _SIGNATURES = {
     "qg_status_str": (c_char_p, [c_int32]),
@@ -89,6 +90,14 @@ _SIGNATURES = {
                                c_int32, c_int32, c_void_p]),
     "qg_selfcheck_exact_math": (c_int32, [c_int32, c_uint64, c_uint64, c_void_p, c_void_p]),
     "qg_selfcheck_wait_timeout": (c_int32, [c_uint64, c_void_p, c_void_p, c_void_p]),
+    "qg_linear_dequant_weight": (c_int32, [c_void_p, c_int64, c_void_p, c_int32, c_int32, c_void_p, c_int64,
+                                           c_void_p]),
+    "qg_linear_forward": (c_int32, [c_void_p, c_int64, c_void_p, c_int64, c_int32, c_int32, c_int32, c_void_p,
+                                    c_int64, c_void_p]),
+    "qg_linear_backward_data": (c_int32, [c_void_p, c_int64, c_void_p, c_int64, c_int32, c_int32, c_int32,
+                                          c_void_p, c_int64, c_void_p]),
+    "qg_linear_backward_weight": (c_int32, [c_void_p, c_int64, c_void_p, c_int64, c_int32, c_int32, c_int32,
+                                            c_void_p, c_int64, c_void_p]),
 }
 
 _lib = None

@@ -19,7 +19,8 @@ ROOT = os.path.dirname(HERE)
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libqgalore.so")
 
-SOURCES = ["qg_api.cu", "qg_step.cu", "qg_refresh.cu", "qg_profile.cu", "qg_noalloc.cu", "qg_selfcheck.cu"]
+SOURCES = ["qg_api.cu", "qg_step.cu", "qg_refresh.cu", "qg_profile.cu", "qg_noalloc.cu", "qg_selfcheck.cu",
+           "qg_linear.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-ffp-contract=off",
           "-fmad=false", "-I", os.path.join(ROOT, "include")]

@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // four epilogue warps to hide the epilogue's latencies behind one another.  Loads of both CTAs complete on the even CTA's
 // full-barrier; the issuer's commits arrive on both CTAs' barriers; epilogues
 // of both CTAs release an accumulator buffer on the even CTA's barrier.
-// B must be MN-major here (64-column boxes).
+// B is MN-major (two 64-column boxes per CTA) or K-major (one box of 64 K x 128 N).
 //
 // Side operands.  An epilogue may declare Epi::kSideBytes > 0: int8 tiles that
 // belong to the output tile (the weight codes, the moment codes) are then
@@ -304,7 +304,6 @@ struct PairLayout {
 template <class Epi, bool kAMN, bool kBMN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<Epi>::kThreads, 1)
     gemm_tc_pair_kernel(const __grid_constant__ GemmParams<Epi> p) {
-  static_assert(kBMN, "the pair kernel loads B in 64-column boxes");
   using L = PairLayout<Epi>;
   constexpr int kGroups = L::kGroups;
   constexpr int kEpiWarps = 4 * kGroups;
@@ -417,8 +416,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<Epi>::kTh
           } else {
             tma_load_2d_pair(a_dst, &pr.tmA, fb, kb * BK, row0);
           }
-          tma_load_2d_pair(b_dst, &pr.tmB, fb, col0, kb * BK);
-          tma_load_2d_pair(b_dst + 8192, &pr.tmB, fb, col0 + 64, kb * BK);
+          if (kBMN) {
+            tma_load_2d_pair(b_dst, &pr.tmB, fb, col0, kb * BK);
+            tma_load_2d_pair(b_dst + 8192, &pr.tmB, fb, col0 + 64, kb * BK);
+          } else {
+            tma_load_2d_pair(b_dst, &pr.tmB, fb, kb * BK, col0);
+          }
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStagesP) {
@@ -442,10 +445,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<Epi>::kTh
       // the issuing thread's instruction stream short while the epilogue warps
       // share its scheduler.
       const uint64_t a_desc0 = kAMN ? sdesc_sw128(smem_u32(sA), 8192, 1024) : sdesc_sw128(smem_u32(sA), 16, 1024);
-      const uint64_t b_desc0 = sdesc_sw128(smem_u32(sB), 8192, 1024);
+      const uint64_t b_desc0 = kBMN ? sdesc_sw128(smem_u32(sB), 8192, 1024) : sdesc_sw128(smem_u32(sB), 16, 1024);
       constexpr uint64_t kStageStep = kHalfStageBytes >> 4;
       constexpr uint64_t kAStep = kAMN ? (2048 >> 4) : (32 >> 4);  // one K step of 16
-      constexpr uint64_t kBStep = 2048 >> 4;
+      constexpr uint64_t kBStep = kBMN ? (2048 >> 4) : (32 >> 4);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (int tile = cluster; ok && tile < total; tile += nclusters) {
