@@ -30,42 +30,68 @@ namespace {
 
 // ---------------------------------------------------------------- W~ = bf16(q * s)
 
-// One thread per 16 consecutive elements of a row of W (row stride ldw bytes,
-// ldw % 16 == 0): the group of element (i, j) is (i n + j) / 256, so sixteen
+// Byte k (0..3) of w as a signed integer, converted to float exactly without the
+// conversion unit: the sign-extended byte added to the bits of 1.5 * 2^23 gives
+// the float 1.5 * 2^23 + byte (exact for |byte| < 2^22), less 1.5 * 2^23.
+QG_DEV float sbyte_f32(uint32_t w, int k) {
+  const uint32_t sel = k | ((k | 8) << 4) | ((k | 8) << 8) | ((k | 8) << 12);
+  uint32_t sx;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(sx) : "r"(w), "r"(0u), "r"(sel));
+  return __fsub_rn(__uint_as_float(0x4B400000u + sx), 12582912.0f);
+}
+
+// Sixteen consecutive elements of a row of W (row stride ldw bytes, ldw % 16 ==
+// 0) per chunk: the group of element (i, j) is (i n + j) / 256, so sixteen
 // elements span at most two groups.  One float32 product, rounded to bf16.
+QG_DEV void dequant_chunk(const uint4& q, int64_t i, int j0, int32_t n, const float* __restrict__ sW,
+                          uint16_t* __restrict__ Wt, int64_t ldt) {
+  const int64_t e0 = i * n + j0;
+  const int valid = min(16, n - j0);
+  const int64_t g0 = e0 >> 8, g1 = (e0 + valid - 1) >> 8;
+  const float s0 = __ldg(sW + g0), s1 = __ldg(sW + g1);
+  const int split = g1 != g0 ? static_cast<int>((g1 << 8) - e0) : 16;
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  uint32_t out[8];
+#pragma unroll
+  for (int k = 0; k < 16; k += 2) {
+    const float a = __fmul_rn(sbyte_f32(w[k >> 2], k & 3), k < split ? s0 : s1);
+    const float b = __fmul_rn(sbyte_f32(w[k >> 2], (k + 1) & 3), k + 1 < split ? s0 : s1);
+    const __nv_bfloat162 p2 = __floats2bfloat162_rn(a, b);  // a in the low half
+    out[k >> 1] = *reinterpret_cast<const uint32_t*>(&p2);
+  }
+  uint16_t* dst = Wt + i * ldt + j0;
+  if (valid == 16) {
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(out[0], out[1], out[2], out[3]);
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      if (k < valid) dst[k] = static_cast<uint16_t>(out[k >> 1] >> (16 * (k & 1)));
+  }
+}
+
+// A grid-stride loop over groups of kDqChunks chunks per thread, all of whose
+// loads are issued before the first conversion (more bytes in flight per SM).
+constexpr int kDqChunks = 4;
+
 __global__ void __launch_bounds__(256) dequant_weight_kernel(const int8_t* __restrict__ W, int64_t ldw,
                                                              const float* __restrict__ sW, int32_t m, int32_t n,
                                                              uint16_t* __restrict__ Wt, int64_t ldt) {
   const int64_t chunks = (n + 15) / 16;
   const int64_t total = static_cast<int64_t>(m) * chunks;
-  for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < total;
-       c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t i = c / chunks;
-    const int j0 = static_cast<int>(c % chunks) * 16;
-    const uint4 q = __ldg(reinterpret_cast<const uint4*>(W + i * ldw + j0));
-    const int64_t e0 = i * n + j0;
-    const int valid = min(16, n - j0);
-    const int64_t g0 = e0 >> 8, g1 = (e0 + valid - 1) >> 8;
-    const float s0 = __ldg(sW + g0), s1 = __ldg(sW + g1);
-    const int split = g1 != g0 ? static_cast<int>((g1 << 8) - e0) : 16;
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    uint32_t out[8];
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t c0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c0 < total;
+       c0 += stride * kDqChunks) {
+    uint4 q[kDqChunks];
 #pragma unroll
-    for (int k = 0; k < 16; k += 2) {
-      const float a = static_cast<float>(static_cast<int8_t>((w[k >> 2] >> (8 * (k & 3))) & 0xFFu));
-      const float b = static_cast<float>(static_cast<int8_t>((w[k >> 2] >> (8 * ((k + 1) & 3))) & 0xFFu));
-      const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(a, k < split ? s0 : s1)));
-      const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(b, k + 1 < split ? s0 : s1)));
-      out[k >> 1] = lo | (hi << 16);
+    for (int u = 0; u < kDqChunks; ++u) {
+      const int64_t c = c0 + u * stride;
+      if (c < total) q[u] = __ldg(reinterpret_cast<const uint4*>(W + (c / chunks) * ldw + (c % chunks) * 16));
     }
-    uint16_t* dst = Wt + i * ldt + j0;
-    if (valid == 16) {
-      reinterpret_cast<uint4*>(dst)[0] = make_uint4(out[0], out[1], out[2], out[3]);
-      reinterpret_cast<uint4*>(dst)[1] = make_uint4(out[4], out[5], out[6], out[7]);
-    } else {
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
-        if (k < valid) dst[k] = static_cast<uint16_t>(out[k >> 1] >> (16 * (k & 1)));
+    for (int u = 0; u < kDqChunks; ++u) {
+      const int64_t c = c0 + u * stride;
+      if (c < total) dequant_chunk(q[u], c / chunks, static_cast<int>(c % chunks) * 16, n, sW, Wt, ldt);
     }
   }
 }
@@ -194,7 +220,8 @@ qg_status qg_linear_dequant_weight(const int8_t* d_W, int64_t ldw, const float* 
   if (!aligned16(d_W) || !aligned16(d_Wt)) return QG_EALIGN;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t work = static_cast<int64_t>(m) * ((n + 15) / 16);
-  const int blocks = static_cast<int>(std::min<int64_t>((work + 255) / 256, int64_t(sm_count()) * 16));
+  const int blocks = static_cast<int>(
+      std::max<int64_t>(1, std::min<int64_t>((work + 256 * kDqChunks - 1) / (256 * kDqChunks), int64_t(sm_count()) * 8)));
   const double bytes = 3.0 * m * n + 4.0 * ((static_cast<double>(m) * n + 255) / 256);
   const int tok = profile_begin(s, QG_KERNEL_LINEAR_DEQUANT, 0.0, bytes);
   dequant_weight_kernel<<<blocks, 256, 0, s>>>(d_W, ldw, d_sW, m, n, static_cast<uint16_t*>(d_Wt), ldwt);
