@@ -50,10 +50,13 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=None, help="decoder layers (default: the stack's own count)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=sorted(STACKS) + ["refresh-stress", "linear-7b"], default="llama7b-stack",
+    ap.add_argument("--workload", choices=sorted(STACKS) + ["refresh-stress", "linear-grad-stress", "linear-7b"],
+                    default="llama7b-stack",
                     help="a decoder stack (llama7b-stack is the default and the headline); refresh-stress: "
                          "one 4096 x 11008 layer, r = 1024, a drifting gradient subspace, subspace refreshes on "
-                         "the layer-adaptive schedule (--steps defaults to 2000); linear-7b: the INT8-weight "
+                         "the layer-adaptive schedule (--steps defaults to 2000); linear-grad-stress: the same "
+                         "layer and schedule with G = D^T X of a linear layer over 8192 tokens whose output-"
+                         "gradient subspace turns for 600 steps and then settles; linear-7b: the INT8-weight "
                          "forward and backward products of the LLaMA-7B stack's 224 linear layers at 8192 tokens")
     return ap.parse_args()
 
@@ -476,7 +479,14 @@ def run_refresh_stress(args, rank, world, local_rank):
     turns by 0.02 rad per step until step 800, then stays.  Every step runs
     qg_refresh (a randomized top-r SVD and CosSim when the layer is due; the
     interval starts at 200 and doubles when CosSim > 0.4) and then qg_step, both
-    timed with CUDA events; the gradient is drawn outside the timed region."""
+    timed with CUDA events; the gradient is drawn outside the timed region.
+
+    With --workload linear-grad-stress the gradient is that of a linear layer,
+    G = D^T X over B = 8192 tokens (the weight-gradient model of Theorem 3.1):
+    X and D draw from principal subspaces of width r; the output-gradient one
+    turns by 0.0075 rad per step (1.5 rad between refreshes 200 steps apart)
+    until step 600 and then stays.  G is formed by qg_linear_backward_weight,
+    outside the timed region."""
     import torch
     import quantized_rank_gradient_b200 as qg
     import synth
@@ -491,7 +501,24 @@ def run_refresh_stress(args, rank, world, local_rank):
     ldw = -(-n // 16) * 16
     W = synth.device_weight_codes(m, n, ldw, seed, device)
     sW = synth.device_weight_scales(m, n, seed, device)
-    gen = synth.DeviceDriftingGradient(m, n, 256, 1e-2, 0.97, 1e-4, 0.02, 800, seed, device)
+    linear = args.workload == "linear-grad-stress"
+    if linear:
+        lin = synth.DeviceLinearLayerBatch(m, n, LINEAR_TOKENS, r, 0.999, 1e-3, 0.0075, 600, seed, device)
+        ldg_lin = -(-n // 8) * 8
+        G_lin = torch.zeros(m, ldg_lin, dtype=torch.bfloat16, device=device)
+
+        class _LinearSource:
+            @staticmethod
+            def draw(t):
+                X, D = lin.draw(t)
+                qg.check(qg.qg_linear_backward_weight(D.data_ptr(), lin.ldd, X.data_ptr(), lin.ldx, LINEAR_TOKENS, m,
+                                                      n, G_lin.data_ptr(), ldg_lin,
+                                                      c_void_p(torch.cuda.current_stream().cuda_stream)),
+                         "qg_linear_backward_weight")
+                return G_lin
+        gen = _LinearSource()
+    else:
+        gen = synth.DeviceDriftingGradient(m, n, 256, 1e-2, 0.97, 1e-4, 0.02, 800, seed, device)
     cs = torch.cuda.current_stream()
     stream = c_void_p(cs.cuda_stream)
     state = torch.empty(qg.qg_state_bytes(byref(c)), dtype=torch.uint8, device=device)
@@ -529,9 +556,14 @@ def run_refresh_stress(args, rank, world, local_rank):
     value = whole_job_rate(steps * m * n, world, total_ms)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": 0,
             "ms_per_step": total_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16/f32/int8", "data": "synthetic (drifting low-rank-plus-noise bf16 gradients)",
-            "config": {"workload": "refresh-stress-4096x11008-r1024", "steps": steps, "delta0": 200, "gamma": 0.4,
-                       "drift": "0.02 rad/step, frozen after step 800",
+            "dtype": "bf16/f32/int8",
+            "data": "synthetic (linear-layer gradients G = D^T X over 8192 tokens)" if linear
+            else "synthetic (drifting low-rank-plus-noise bf16 gradients)",
+            "config": {"workload": ("linear-grad-stress-4096x11008-r1024-B8192" if linear
+                                    else "refresh-stress-4096x11008-r1024"),
+                       "steps": steps, "delta0": 200, "gamma": 0.4,
+                       "drift": ("output-gradient subspace turns 0.0075 rad/step, frozen after step 600" if linear
+                                 else "0.02 rad/step, frozen after step 800"),
                        "l2": "gradient redrawn every step outside the timed region"},
             "refreshes": len(trace), "svd_fraction_vs_fixed_interval": len(trace) / max(1, -(-steps // 200)),
             "refresh_ms": {"mean": sum(refresh_ms) / max(1, len(refresh_ms)), "max": max(refresh_ms or [0.0])},
@@ -724,7 +756,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        if args.workload == "refresh-stress":
+        if args.workload in ("refresh-stress", "linear-grad-stress"):
             return run_refresh_stress(args, rank, world, local_rank)
         if args.workload == "linear-7b":
             return run_linear(args, rank, world, local_rank)

@@ -190,3 +190,57 @@ class DeviceDriftingGradient:
         full += self.sigma * torch.randn(self.m, self.n, generator=g, device=self.device, dtype=torch.float32)
         self.out[:, : self.n] = full.to(torch.bfloat16)
         return self.out
+
+
+class DeviceLinearLayerBatch:
+    """Activations and output gradients of one linear layer y = W x over a batch
+    of B tokens, on the device, for gradients G = (1/B) D^T X (the weight-gradient
+    model of the paper's Theorem 3.1: G lies in the principal subspaces of the
+    inputs and of the output gradients).
+
+    X_t = Z_t diag(s) A + sigma E_t                (B x n, bf16)
+    D_t = (Z_t M diag(s) C_t + sigma F_t) / B      (B x m, bf16)
+
+    A (k x n) has orthonormal rows, M is a Haar-random orthogonal k x k matrix
+    (so the k directions of the output gradients stay well conditioned),
+    s_i = decay^i; Z_t, E_t, F_t are standard normal and redrawn at every step
+    from (seed, t).  The output-gradient subspace moves until the layer settles:
+    C_t = cos(theta_t) C_0 + sin(theta_t) C_1, with C_0, C_1 (k x m) orthonormal
+    rows, orthogonal to each other, so each row turns in its own plane by
+    theta_t = rate * min(t, freeze) and then stays."""
+
+    def __init__(self, m, n, B, k, decay, sigma, rate, freeze, seed, device, pad_to=8):
+        g = torch.Generator(device=device)
+        g.manual_seed(int(seed))
+        self.m, self.n, self.B, self.k = m, n, B, min(k, m // 2)
+        k = self.k
+        qa, ra = torch.linalg.qr(torch.randn(n, k, generator=g, device=device))
+        qc, rc = torch.linalg.qr(torch.randn(m, 2 * k, generator=g, device=device))
+        qc = qc * torch.sign(torch.diagonal(rc))[None, :]
+        s = decay ** torch.arange(k, device=device, dtype=torch.float32)
+        self.SA = (s[:, None] * (qa * torch.sign(torch.diagonal(ra))[None, :]).T).contiguous()
+        self.C0, self.C1 = qc[:, :k].T.contiguous(), qc[:, k:].T.contiguous()
+        qm, rm = torch.linalg.qr(torch.randn(k, k, generator=g, device=device))
+        self.SM = (qm * torch.sign(torch.diagonal(rm))[None, :]) * s[None, :]
+        self.sigma, self.rate, self.freeze, self.seed = sigma, rate, freeze, int(seed)
+        self.ldx = -(-n // pad_to) * pad_to
+        self.ldd = -(-m // pad_to) * pad_to
+        self.device = device
+        self.X = torch.zeros(B, self.ldx, device=device, dtype=torch.bfloat16)
+        self.D = torch.zeros(B, self.ldd, device=device, dtype=torch.bfloat16)
+
+    def draw(self, t):
+        """Fills and returns (X, D) for step t (bf16, row strides ldx and ldd)."""
+        import math
+        th = self.rate * min(t, self.freeze)
+        C = self.C0 * math.cos(th) + self.C1 * math.sin(th)
+        g = torch.Generator(device=self.device)
+        g.manual_seed(self.seed * 1000003 + t + 1)
+        Z = torch.randn(self.B, self.k, generator=g, device=self.device)
+        x = Z @ self.SA
+        x += self.sigma * torch.randn(self.B, self.n, generator=g, device=self.device)
+        self.X[:, : self.n] = x.to(torch.bfloat16)
+        d = (Z @ self.SM) @ C
+        d += self.sigma * torch.randn(self.B, self.m, generator=g, device=self.device)
+        self.D[:, : self.m] = (d / self.B).to(torch.bfloat16)
+        return self.X, self.D
