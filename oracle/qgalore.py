@@ -242,6 +242,7 @@ class Config:
     power_iters: int = 2
     seed: int = 0
     layer_id: int = 0
+    mom_refresh: int = 0  # moments at a refresh: 0 keep, 1 reset, 2 rotate (see refresh_moments)
 
     def f32(self, name):
         return F32(getattr(self, name))
@@ -528,14 +529,49 @@ def refresh(st: LayerState, G, force=False) -> dict | None:
     Pq = pack_int4(codes)
     cs = None
     if st.Pq is not None:
-        cs = cossim(dequant_int4_f32(Pq, sP, cfg.m, cfg.r, cfg.p_group),
-                    dequant_int4_f32(st.Pq, st.sP, cfg.m, cfg.r, cfg.p_group))
+        Pa = dequant_int4_f32(Pq, sP, cfg.m, cfg.r, cfg.p_group)
+        Pb = dequant_int4_f32(st.Pq, st.sP, cfg.m, cfg.r, cfg.p_group)
+        cs = cossim(Pa, Pb)
+        refresh_moments(st, Pa, Pb)
         st.Pq_prev, st.sP_prev = st.Pq, st.sP
     st.Pq, st.sP = Pq, sP
     st.delta, st.t_next = schedule_after_refresh(st.t, st.delta, cs, cfg.gamma)
     st.n_refresh += 1
     st.cossim_trace.append((st.t, cs))
     return dict(P=P, sigma=sigma, cossim=cs, Omega=Omega)
+
+
+def refresh_moments(st: LayerState, Pa, Pb):
+    """The low-rank moments at a refresh that replaces the projection Pb (the
+    dequantized previous P, m x r) by Pa (the dequantized new one).  The moments
+    live in P's coordinates (R = P^T G, r x n), and the pages do not say what
+    happens to them when P changes.  cfg.mom_refresh selects a reading:
+      0  keep them as they are (the default);
+      1  reset them to zero;
+      2  rotate them into the new basis: with C = Pa^T Pb (r x r), m' = C m, the
+         first moment mapped as a vector is; v' = (C o C) v, the second moment
+         mapped as the variance of independent coordinates is (C o C the
+         element-wise square).  C, and both products, in float64 from the
+         float32 operands; the results rounded to float32 and re-quantized on the
+         step's grids (linear for m, square root for v)."""
+    cfg = st.cfg
+    if cfg.mom_refresh == 0:
+        return
+    if cfg.mom_refresh == 1:
+        st.Mq = np.zeros_like(st.Mq)
+        st.Vq = np.zeros_like(st.Vq)
+        st.sM = np.zeros_like(st.sM)
+        st.sV = np.zeros_like(st.sV)
+        return
+    if cfg.mom_refresh != 2:
+        raise ValueError("mom_refresh must be 0, 1 or 2")
+    C = np.asarray(Pa, np.float64).T @ np.asarray(Pb, np.float64)
+    m0 = dequant_rowblock(st.Mq, st.sM, cfg.mom_block).astype(np.float64)
+    v0 = dequant_second_moment(st.Vq, st.sV, cfg.mom_block).astype(np.float64)
+    m1 = (C @ m0).astype(np.float32)
+    v1 = ((C * C) @ v0).astype(np.float32)
+    st.Mq, st.sM = quant_rowblock_int8(m1, cfg.mom_block, unsigned=False)
+    st.Vq, st.sV = quant_rowblock_int8(np.sqrt(v1).astype(np.float32), cfg.mom_block, unsigned=True)
 
 
 def set_projection(st: LayerState, P):

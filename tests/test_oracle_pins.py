@@ -16,6 +16,7 @@ import scipy.linalg
 import torch
 
 import oracle as O
+import synth
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -597,3 +598,54 @@ def test_linear_products_brute_force_and_integer_exact():
     assert np.array_equal(O.linear_forward(Xi, Wi), (Xi @ Wi.T).astype(np.float64))
     assert np.array_equal(O.linear_backward_data(Di, Wi), (Di @ Wi).astype(np.float64))
     assert np.array_equal(O.linear_backward_weight(Di, Xi), (Di.T @ Xi).astype(np.float64))
+
+
+# ---------------------------------------------------------------- moments at a refresh
+
+def _state_with_moments(m=64, n=300, r=32, policy=2, seed=5):
+    cfg = O.Config(m=m, n=n, r=r, seed=seed, mom_refresh=policy)
+    rng = np.random.default_rng(seed)
+    st = O.LayerState.create(cfg, np.zeros((m, n), np.int8), np.ones(-(-m * n // 256), np.float32))
+    mom = rng.standard_normal((r, n)).astype(np.float32) * 1e-3
+    st.Mq, st.sM = O.quant_rowblock_int8(mom, 256)
+    st.Vq, st.sV = O.quant_rowblock_int8(np.abs(mom) * 2, 256, unsigned=True)
+    return st
+
+
+def test_refresh_moments_reset_and_keep():
+    st = _state_with_moments(policy=1)
+    P = synth.orthonormal(64, 32, seed=1)
+    O.refresh_moments(st, P, P)
+    assert not st.Mq.any() and not st.Vq.any() and not st.sM.any() and not st.sV.any()
+    st = _state_with_moments(policy=0)
+    before = (st.Mq.copy(), st.sM.copy(), st.Vq.copy(), st.sV.copy())
+    O.refresh_moments(st, P, synth.orthonormal(64, 32, seed=2))
+    for a, b in zip(before, (st.Mq, st.sM, st.Vq, st.sV)):
+        assert np.array_equal(a, b)
+
+
+def test_refresh_moments_rotation_identity_and_permutation():
+    # the same basis (C = I) reproduces the codes: quantizing a dequantized array
+    # gives its codes back
+    st = _state_with_moments()
+    Mq, sM, Vq, sV = st.Mq.copy(), st.sM.copy(), st.Vq.copy(), st.sV.copy()
+    P = synth.orthonormal(64, 32, seed=1)
+    O.refresh_moments(st, P, P)
+    assert np.array_equal(st.Mq, Mq) and np.array_equal(st.Vq, Vq)
+    # a new basis that permutes the old columns permutes the moment rows: the new
+    # column a is old column perm[a], so new row a of m is old row perm[a]; the
+    # second moment's codes follow exactly (C o C is the same permutation)
+    st = _state_with_moments()
+    m_old = O.dequant_rowblock(st.Mq, st.sM)
+    Vq_old = st.Vq.copy()
+    perm = np.random.default_rng(3).permutation(32)
+    O.refresh_moments(st, P[:, perm], P)
+    np.testing.assert_allclose(O.dequant_rowblock(st.Mq, st.sM), m_old[perm], rtol=0, atol=1e-9)
+    assert np.array_equal(st.Vq, Vq_old[perm])
+    # sign flips of new columns: m rows flip sign, v is unchanged (C o C = I)
+    st = _state_with_moments()
+    m_old, Vq_old = O.dequant_rowblock(st.Mq, st.sM), st.Vq.copy()
+    flip = np.where(np.arange(32) % 3 == 0, -1.0, 1.0)
+    O.refresh_moments(st, P * flip[None, :], P)
+    np.testing.assert_allclose(O.dequant_rowblock(st.Mq, st.sM), m_old * flip[:, None], rtol=0, atol=1e-9)
+    assert np.array_equal(st.Vq, Vq_old)
