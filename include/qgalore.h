@@ -70,6 +70,10 @@ typedef struct {
   int32_t power_iters;      /* randomized SVD power iterations q, 2 */
   uint64_t seed;            /* Philox key of the stochastic rounding and of Omega */
   uint32_t layer_id;        /* Philox counter word: distinguishes matrices */
+  int32_t mom_refresh;      /* the low-rank moments at a refresh that replaces P: 0 keep them (default),
+                               1 reset them to zero, 2 rotate them into the new basis with
+                               C = P_new^T P_prev: m' = C m, v' = (C o C) v (element-wise square),
+                               re-quantized on the step's grids */
 } qg_config;
 
 typedef struct qg_layer qg_layer;

@@ -29,7 +29,7 @@ class qg_config(Structure):
     _fields_ = [("m", c_int32), ("n", c_int32), ("r", c_int32), ("w_group", c_int32), ("p_group", c_int32),
                 ("mom_block", c_int32), ("beta1", c_float), ("beta2", c_float), ("eps", c_float), ("lr", c_float),
                 ("alpha", c_float), ("gamma", c_float), ("delta0", c_int32), ("oversample", c_int32),
-                ("power_iters", c_int32), ("seed", c_uint64), ("layer_id", c_uint32)]
+                ("power_iters", c_int32), ("seed", c_uint64), ("layer_id", c_uint32), ("mom_refresh", c_int32)]
 
 
 class qg_layer_views(Structure):

@@ -78,6 +78,7 @@ qg_status check_config(const qg_config* c) {
   if (!(c->beta1 >= 0.f && c->beta1 < 1.f) || !(c->beta2 >= 0.f && c->beta2 < 1.f)) return QG_EINVAL;
   if (!(c->eps > 0.f) || !isfinite(c->eps) || !isfinite(c->lr) || !isfinite(c->alpha)) return QG_EINVAL;
   if (!isfinite(c->gamma) || c->delta0 < 1 || c->oversample < 0 || c->power_iters < 0) return QG_EINVAL;
+  if (c->mom_refresh < 0 || c->mom_refresh > 2) return QG_EINVAL;
   return QG_OK;
 }
 
@@ -445,6 +446,13 @@ qg_status qg_refresh(qg_layer* L, const void* d_G, int64_t ldg, int32_t force, v
   ra.sP_prev = L->v.sP_prev;
   ra.has_prev = has_prev ? 1 : 0;
   ra.status = L->v.status;
+  ra.mom_refresh = c.mom_refresh;
+  ra.Mq = L->v.Mq;
+  ra.Vq = L->v.Vq;
+  ra.sM = L->v.sM;
+  ra.sV = L->v.sV;
+  ra.ld_mom = L->v.ld_mom;
+  ra.nblk = L->v.nblk;
   float cs = 0.f;
   qg_status st = qg::run_refresh(ra, static_cast<uint8_t*>(d_ws), ws_bytes, s, &cs);
   if (st != QG_OK) return st;

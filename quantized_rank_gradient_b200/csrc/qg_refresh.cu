@@ -40,7 +40,7 @@ size_t r256(size_t x) { return (x + 255) / 256 * 256; }
 struct RefreshLayout {
   int k, ldk, ldn4;
   size_t P, omega, Y, Yb, Ylo, Z, Zb, Zlo, gram, gpart, linv, Li, Tt, Lih, Lil, Bm, At, Vt, lam, perm, Vsel, Pa, Pb, Ct, jx,
-      misc, total;
+      mom, misc, total;
 };
 
 // Scratch of the split Jacobi on a k x k matrix: one exchange counter per block
@@ -93,6 +93,7 @@ RefreshLayout refresh_layout(int m, int n, int r, int p) {
   L.Pb = take(size_t(m) * r * 4);
   L.Ct = take(size_t(r) * r * 4);
   L.jx = take(jacobi_scratch_bytes(L.k));
+  L.mom = take(size_t(r) * L.ldn4 * 4);  // the rotated moments (r x n fp32)
   L.misc = take(256);
   L.total = off;
   return L;
@@ -145,6 +146,61 @@ __global__ void __launch_bounds__(1024) add_shift_kernel(float* A, int64_t ld, i
   __syncthreads();
   const float shift = 11.f * (static_cast<float>(rows) * k + static_cast<float>(k) * (k + 1)) * 5.9604645e-8f * part[0];
   for (int i = threadIdx.x; i < k; i += blockDim.x) A[static_cast<int64_t>(i) * ld + i] += shift;
+}
+
+// ---- the low-rank moments at a refresh (cfg.mom_refresh = 2, rotation)
+
+// out = code * scale (fp32), squared when kSquare: the first moment from its
+// linear grid, or v = (code * scale)^2 from the square-root grid of the second
+// (row blocks of 256 columns).
+template <bool kSquare>
+__global__ void moment_dequant_kernel(const int8_t* __restrict__ codes, int64_t ld_mom,
+                                      const float* __restrict__ scales, int nblk, int r, int n, float* __restrict__ out,
+                                      int64_t ldo) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(r) * n) return;
+  const int64_t i = idx / n;
+  const int j = static_cast<int>(idx % n);
+  const float x = __fmul_rn(static_cast<float>(codes[i * ld_mom + j]), scales[i * nblk + (j >> 8)]);
+  out[i * ldo + j] = kSquare ? __fmul_rn(x, x) : x;
+}
+
+// Re-quantization on the step's row-block grid, one warp per (row, block of 256
+// columns): y = x (kSqrt: y = sqrt(x), correctly rounded), scale = absmax / 127,
+// codes rint(y * (127 / absmax)) with both divisions IEEE; a block whose absmax
+// is below 2^-120 gets scale 0 and codes 0.
+template <bool kSqrt>
+__global__ void moment_quant_kernel(const float* __restrict__ x, int64_t ldx, int r, int n, int nblk,
+                                    int8_t* __restrict__ codes, int64_t ld_mom, float* __restrict__ scales) {
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<int64_t>(r) * nblk) return;
+  const int64_t i = w / nblk;
+  const int j0 = static_cast<int>(w % nblk) * 256;
+  float y[8];
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int j = j0 + lane + 32 * k;
+    const float v = j < n ? x[i * ldx + j] : 0.f;
+    y[k] = kSqrt ? __fsqrt_rn(v) : v;
+    amax = fmaxf(amax, fabsf(y[k]));
+  }
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  const bool live = amax >= kAbsmaxFloorR;
+  const float inv = live ? __fdiv_rn(127.0f, amax) : 0.f;
+  const float lo = kSqrt ? 0.f : -127.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int j = j0 + lane + 32 * k;
+    if (j < n) codes[i * ld_mom + j] = static_cast<int8_t>(fminf(fmaxf(rintf(__fmul_rn(y[k], inv)), lo), 127.f));
+  }
+  if (lane == 0) scales[i * nblk + (j0 >> 8)] = live ? __fdiv_rn(amax, 127.0f) : 0.f;
+}
+
+__global__ void square_kernel(const float* __restrict__ a, float* __restrict__ b, int64_t count) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx < count) b[idx] = __fmul_rn(a[idx], a[idx]);
 }
 
 __global__ void identity_kernel(float* V, int64_t ld, int k) {
@@ -438,6 +494,39 @@ cudaError_t cossim_core(const float* Pa, const float* Pb, int m, int r, int64_t 
 
 qg_status st_of(cudaError_t e) { return e == cudaSuccess ? QG_OK : QG_ECUDA; }
 
+// The moments at a refresh that replaces the projection Pb (dequantized, m x r)
+// by Pa: kept, reset to zero, or rotated with C = Pa^T Pb (m' = C m,
+// v' = (C o C) v) and re-quantized.  C and C2 are r x r scratch, X and Y r x ldx.
+cudaError_t refresh_moments(const RefreshArgs& a, const float* Pa, const float* Pb, float* C, float* C2, float* X,
+                            float* Y, int64_t ldx, cudaStream_t s) {
+  const int m = a.m, n = a.n, r = a.r;
+  cudaError_t e;
+  if (a.mom_refresh == 0) return cudaSuccess;
+  if (a.mom_refresh == 1) {
+    const size_t codes = size_t(r) * a.ld_mom, sc = size_t(r) * a.nblk * 4;
+    if ((e = cudaMemsetAsync(a.Mq, 0, codes, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(a.Vq, 0, codes, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(a.sM, 0, sc, s)) != cudaSuccess) return e;
+    return cudaMemsetAsync(a.sV, 0, sc, s);
+  }
+  if ((e = sgemm(true, false, Pa, r, Pb, r, C, r, r, r, m, s)) != cudaSuccess) return e;
+  const int64_t rr = int64_t(r) * r, rn = int64_t(r) * n;
+  square_kernel<<<static_cast<unsigned>((rr + 255) / 256), 256, 0, s>>>(C, C2, rr);
+  const unsigned eb = static_cast<unsigned>((rn + 255) / 256);
+  const unsigned qb = static_cast<unsigned>((int64_t(r) * a.nblk * 32 + 255) / 256);
+  // m' = C m
+  moment_dequant_kernel<false><<<eb, 256, 0, s>>>(a.Mq, a.ld_mom, a.sM, a.nblk, r, n, X, ldx);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = sgemm(false, false, C, r, X, ldx, Y, ldx, r, n, r, s)) != cudaSuccess) return e;
+  moment_quant_kernel<false><<<qb, 256, 0, s>>>(Y, ldx, r, n, a.nblk, a.Mq, a.ld_mom, a.sM);
+  // v' = (C o C) v
+  moment_dequant_kernel<true><<<eb, 256, 0, s>>>(a.Vq, a.ld_mom, a.sV, a.nblk, r, n, X, ldx);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = sgemm(false, false, C2, r, X, ldx, Y, ldx, r, n, r, s)) != cudaSuccess) return e;
+  moment_quant_kernel<true><<<qb, 256, 0, s>>>(Y, ldx, r, n, a.nblk, a.Vq, a.ld_mom, a.sV);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ INT4 quantizer
@@ -582,6 +671,10 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
     dequant_f32_kernel<<<blocks, 256, 0, s>>>(a.Pq_prev, a.sP_prev, static_cast<int64_t>(mr), Pb);
     if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
     if (cossim_core(Pa, Pb, m, r, r, Ct, misc->bar, &misc->sweeps, &misc->cossim, a.status, ws + L.jx, s) !=
+        cudaSuccess)
+      return QG_ECUDA;
+    if (refresh_moments(a, Pa, Pb, reinterpret_cast<float*>(ws + L.At), reinterpret_cast<float*>(ws + L.Vt),
+                        reinterpret_cast<float*>(ws + L.Bm), reinterpret_cast<float*>(ws + L.mom), L.ldn4, s) !=
         cudaSuccess)
       return QG_ECUDA;
     float host = 0.f;

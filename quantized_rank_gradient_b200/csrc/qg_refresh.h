@@ -24,6 +24,14 @@ struct RefreshArgs {
   float* sP_prev;
   int32_t has_prev;
   uint32_t* status;
+  // the layer's INT8 moments, for cfg.mom_refresh (0 keep, 1 reset, 2 rotate)
+  int32_t mom_refresh;
+  int8_t* Mq;
+  int8_t* Vq;
+  float* sM;
+  float* sV;
+  int64_t ld_mom;
+  int32_t nblk;
 };
 
 size_t refresh_scratch_bytes(int32_t m, int32_t n, int32_t r, int32_t oversample);

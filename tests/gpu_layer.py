@@ -20,7 +20,7 @@ def stream():
 def lib_config(oc: O.Config):
     return qg.config(oc.m, oc.n, oc.r, beta1=oc.beta1, beta2=oc.beta2, eps=oc.eps, lr=oc.lr, alpha=oc.alpha,
                      gamma=oc.gamma, delta0=oc.delta0, oversample=oc.oversample, power_iters=oc.power_iters,
-                     seed=oc.seed, layer_id=oc.layer_id)
+                     seed=oc.seed, layer_id=oc.layer_id, mom_refresh=oc.mom_refresh)
 
 
 def upload_gradient(G_bits: np.ndarray, device="cuda"):

@@ -60,6 +60,7 @@ def test_config_defaults_and_sizes():
 @pytest.mark.parametrize("field,value,expect", [
     ("r", 48, qg.QG_ESHAPE), ("r", 512, qg.QG_ESHAPE), ("w_group", 128, qg.QG_ESHAPE),
     ("beta1", 1.0, qg.QG_EINVAL), ("eps", 0.0, qg.QG_EINVAL), ("delta0", 0, qg.QG_EINVAL),
+    ("mom_refresh", 3, qg.QG_EINVAL), ("mom_refresh", -1, qg.QG_EINVAL),
 ])
 def test_layer_init_rejects_bad_config_before_any_launch(field, value, expect):
     c = qg.config(256, 300, 64)

@@ -169,3 +169,48 @@ def test_schedule_follows_oracle_over_refreshes():
         O.step(ost, G)
     assert len(trace) >= 2 and min(trace) > 0.4   # stable subspace -> intervals doubled
     assert gl.sched().delta > 2
+
+
+# ---------------------------------------------------------------- moments at a refresh
+
+@pytest.mark.parametrize("policy", [1, 2])
+def test_refresh_moment_policy_matches_oracle(policy):
+    # a starting projection and three steps give non-zero moments; a forced
+    # refresh then replaces P.  The oracle applies the same moment map to the
+    # GPU's own moments and projections (teacher-forced), so only the map is
+    # compared: reset bit-exact, rotation within the step's moment bar
+    m, n, r = 300, 700, 64
+    oc = O.Config(m=m, n=n, r=r, seed=7, layer_id=3, mom_refresh=policy)
+    Wq, sW = synth.weight_codes(m, n, 7), synth.weight_scales(m, n, seed=7)
+    gen = synth.lowrank_gradient(m, n, rank=32, seed=7)
+    gl = GpuLayer(oc, Wq, sW)
+    G0, _ = gen.draw(0)
+    codes, sP = O.quant_int4_groups(O.exact_topr(G0, r)[0].astype(np.float32))
+    Pq = O.pack_int4(codes)
+    gl.set_projection(Pq, sP)
+    for t in range(3):
+        _, Gb = gen.draw(t)
+        dG, ldg = upload_gradient(Gb)
+        gl.step(dG, ldg)
+    torch.cuda.synchronize()
+    Mq, sM, Vq, sV = gl.moments()
+    assert np.abs(Mq).sum() > 0 and np.abs(Vq).sum() > 0
+    _, Gb = gen.draw(5)
+    dG, ldg = upload_gradient(Gb)
+    info, _P = gl.refresh(dG, ldg, force=1)
+    assert info.refreshed == 1 and info.has_cossim == 1
+    Pq_new, sP_new = gl.projection()
+    st = O.LayerState.create(oc, Wq, sW)
+    st.Mq, st.sM, st.Vq, st.sV = Mq.copy(), sM.copy(), Vq.copy(), sV.copy()
+    O.refresh_moments(st, O.dequant_int4_f32(Pq_new, sP_new, m, r), O.dequant_int4_f32(Pq, sP, m, r))
+    gMq, gsM, gVq, gsV = gl.moments()
+    if policy == 1:
+        assert not gMq.any() and not gVq.any() and not gsM.any() and not gsV.any()
+        return
+    for (gq, gs, oq, os_, second) in ((gMq, gsM, st.Mq, st.sM, False), (gVq, gsV, st.Vq, st.sV, True)):
+        g = O.dequant_second_moment(gq, gs) if second else O.dequant_rowblock(gq, gs)
+        o = O.dequant_second_moment(oq, os_) if second else O.dequant_rowblock(oq, os_)
+        assert np.linalg.norm(g - o) <= 1e-2 * np.linalg.norm(o), (second, np.linalg.norm(g - o) / np.linalg.norm(o))
+        np.testing.assert_allclose(gs, os_, rtol=1e-4, atol=0)
+        assert np.abs(gq.astype(np.int32) - oq.astype(np.int32)).max() <= 1
+    assert gl.status() == qg.QG_OK
