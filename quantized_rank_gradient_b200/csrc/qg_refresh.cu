@@ -10,10 +10,10 @@
 // Cholesky-QR (Fukaya et al. 2020) with fp32 SIMT Gram matrices and X L^-T
 // formed on the tensor cores from the explicit inverse: two passes for the
 // intermediate bases of the power iterations, three for the final Q;
-// the k x k eigenproblem and the r x r singular values of CosSim use a one-sided
-// Jacobi with a bounded grid barrier.  Then: sign canonicalisation, INT4
-// quantization, and CosSim(P_new, P_prev) = (1/r) sum_i sigma_i(P_new^T P_prev)
-// on the dequantized projections.
+// the k x k eigenproblem uses a block one-sided Jacobi with bounded grid
+// barriers.  Then: sign canonicalisation, INT4 quantization, and
+// CosSim(P_new, P_prev) = (1/r) sum_i sigma_i(P_new^T P_prev) on the dequantized
+// projections, the nuclear norm by a Newton-Schulz polar iteration.
 #include <algorithm>
 #include <cstring>
 
@@ -91,7 +91,7 @@ RefreshLayout refresh_layout(int m, int n, int r, int p) {
   L.Vsel = take(k * size_t(r) * 4);
   L.Pa = take(size_t(m) * r * 4);
   L.Pb = take(size_t(m) * r * 4);
-  L.Ct = take(size_t(r) * r * 4);
+  L.Ct = take(size_t(r) * r * 4 * 4);  // CosSim: C and three Newton-Schulz buffers
   L.jx = take(jacobi_scratch_bytes(L.k));
   L.mom = take(size_t(r) * L.ldn4 * 4);  // the rotated moments (r x n fp32)
   L.misc = take(256);
@@ -100,12 +100,14 @@ RefreshLayout refresh_layout(int m, int n, int r, int p) {
 }
 
 // misc region: [0..7] grid barrier, rotation counter, sweep's largest
-// off-diagonal; then the Cholesky flag, the Jacobi sweeps, the CosSim value
+// off-diagonal; then the Cholesky flag, the Jacobi sweeps, the CosSim value and
+// the scale of its Newton-Schulz start
 struct Misc {
   unsigned bar[8];
   int chol_flag;
   int sweeps;
   float cossim;
+  float ns_scale;  // 1 / ||C||_F of CosSim's Newton-Schulz start
 };
 
 // ------------------------------------------------------------------ kernels
@@ -291,26 +293,61 @@ __global__ void dequant_f32_kernel(const uint8_t* Pq, const float* sP, int64_t t
   out[e] = __fmul_rn(static_cast<float>(code), sP[e >> 6]);
 }
 
-// out = (1/r) sum_p || row p of Ct ||   (Ct rows: the columns of C after Jacobi)
-__global__ void __launch_bounds__(1024) mean_row_norm_kernel(const float* Ct, int64_t ld, int r, float* out) {
+// ---- CosSim = (1/r) sum_i sigma_i(C): the nuclear norm of C, which is
+// trace(U^T C) for the polar factor U of C.  U by the Newton-Schulz iteration
+// X <- X (3 I - X^T X) / 2 (Bjorck and Bowie 1971; Higham, "Functions of
+// Matrices", 2008, section 8.3), from X_0 = C / ||C||_F: every singular value
+// of X_0 lies in [0, 1] and moves to 1, small ones growing by 3/2 per step and
+// then converging quadratically.  A direction still short of 1 after the last
+// step adds less than its own sigma_i to the error.  After kNsIters = 40 steps
+// every sigma_i / ||C||_F >= (2/3)^35 (about 7e-7) has converged; ||C||_F <=
+// sqrt(r) for projections with orthonormal columns, so every sigma_i >= 2.3e-5
+// has at r = 1024, and CosSim is within about 2.3e-5.
+constexpr int kNsIters = 40;
+
+// out[0] = 1 / ||A||_F for the n-element array A (0 for a zero array); one block.
+__global__ void __launch_bounds__(1024) inv_frobenius_kernel(const float* __restrict__ A, int64_t n, float* out) {
   __shared__ float part[32];
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  float acc = 0.f;
-  for (int p = w; p < r; p += nw) {
-    float s = 0.f;
-    for (int t = lane; t < r; t += 32) {
-      const float x = __ldcg(Ct + static_cast<int64_t>(p) * ld + t);
-      s = __fmaf_rn(x, x, s);
-    }
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-    acc += sqrtf(s);
-  }
-  if (lane == 0) part[w] = acc;
+  float s = 0.f;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) s = __fmaf_rn(A[i], A[i], s);
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
   __syncthreads();
   if (threadIdx.x == 0) {
     float t = 0.f;
-    for (int i = 0; i < nw; ++i) t += part[i];
-    *out = t / static_cast<float>(r);
+    for (int i = 0; i < (blockDim.x >> 5); ++i) t += part[i];
+    out[0] = t > 0.f ? rsqrtf(t) : 0.f;
+  }
+}
+
+__global__ void scale_kernel(const float* __restrict__ A, const float* __restrict__ factor, float* __restrict__ B,
+                             int64_t n) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) B[i] = __fmul_rn(A[i], factor[0]);
+}
+
+// T <- 1.5 I - 0.5 T for the r x r matrix T.
+__global__ void ns_shift_kernel(float* __restrict__ T, int r) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<int64_t>(r) * r) return;
+  const float d = (i / r == i % r) ? 1.5f : 0.f;
+  T[i] = __fmaf_rn(-0.5f, T[i], d);
+}
+
+// out[0] = (1/r) sum_ij X_ij C_ij = (1/r) trace(X^T C); one block.
+__global__ void __launch_bounds__(1024) trace_product_kernel(const float* __restrict__ X, const float* __restrict__ C,
+                                                             int r, float* out) {
+  __shared__ float part[32];
+  const int64_t n = static_cast<int64_t>(r) * r;
+  float s = 0.f;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) s = __fmaf_rn(X[i], C[i], s);
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int i = 0; i < (blockDim.x >> 5); ++i) t += part[i];
+    out[0] = t / static_cast<float>(r);
   }
 }
 
@@ -481,14 +518,29 @@ cudaError_t jacobi(float* At, float* Vt, int64_t ld, int k, unsigned* bar, int* 
   return e;
 }
 
-// CosSim of Pa, Pb (fp32 m x r, stride ld) into d_out: Ct = Pb^T Pa holds the
-// columns of C = Pa^T Pb as rows; one-sided Jacobi; mean of the column norms.
-cudaError_t cossim_core(const float* Pa, const float* Pb, int m, int r, int64_t ld, float* Ct, unsigned* bar,
-                        int* sweeps, float* d_out, uint32_t* status, uint8_t* jx, cudaStream_t s) {
-  cudaError_t e = sgemm(true, false, Pb, ld, Pa, ld, Ct, r, r, r, m, s);
+// CosSim of Pa, Pb (fp32 m x r, stride ld) into d_out: C = Pb^T Pa (the
+// transpose of Pa^T Pb: the same singular values), then the nuclear norm by the
+// Newton-Schulz polar iteration above.  buf: 4 r x r floats; scal: one float.
+cudaError_t cossim_core(const float* Pa, const float* Pb, int m, int r, int64_t ld, float* buf, float* scal,
+                        float* d_out, cudaStream_t s) {
+  const int64_t rr = int64_t(r) * r;
+  float* C = buf;
+  float* X = buf + rr;
+  float* Xn = buf + 2 * rr;
+  float* T = buf + 3 * rr;
+  cudaError_t e = sgemm(true, false, Pb, ld, Pa, ld, C, r, r, r, m, s);
   if (e != cudaSuccess) return e;
-  if ((e = jacobi(Ct, nullptr, r, r, bar, sweeps, status, jx, s)) != cudaSuccess) return e;
-  mean_row_norm_kernel<<<1, 1024, 0, s>>>(Ct, r, r, d_out);
+  const unsigned blocks = static_cast<unsigned>((rr + 255) / 256);
+  inv_frobenius_kernel<<<1, 1024, 0, s>>>(C, rr, scal);
+  scale_kernel<<<blocks, 256, 0, s>>>(C, scal, X, rr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  for (int it = 0; it < kNsIters; ++it) {
+    if ((e = sgemm(true, false, X, r, X, r, T, r, r, r, r, s)) != cudaSuccess) return e;
+    ns_shift_kernel<<<blocks, 256, 0, s>>>(T, r);
+    if ((e = sgemm(false, false, X, r, T, r, Xn, r, r, r, r, s)) != cudaSuccess) return e;
+    std::swap(X, Xn);
+  }
+  trace_product_kernel<<<1, 1024, 0, s>>>(X, C, r, d_out);
   return cudaGetLastError();
 }
 
@@ -583,7 +635,7 @@ size_t refresh_scratch_bytes(int32_t m, int32_t n, int32_t r, int32_t oversample
   return refresh_layout(m, n, r, oversample).total;
 }
 
-size_t cossim_scratch_bytes(int32_t, int32_t r) { return r256(size_t(r) * r * 4) + 256 + jacobi_scratch_bytes(r); }
+size_t cossim_scratch_bytes(int32_t, int32_t r) { return r256(size_t(r) * r * 4 * 4) + 256; }
 
 qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaStream_t s, float* cossim) {
   const RefreshLayout L = refresh_layout(a.m, a.n, a.r, a.oversample);
@@ -670,9 +722,7 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
     dequant_f32_kernel<<<blocks, 256, 0, s>>>(a.Pq, a.sP, static_cast<int64_t>(mr), Pa);
     dequant_f32_kernel<<<blocks, 256, 0, s>>>(a.Pq_prev, a.sP_prev, static_cast<int64_t>(mr), Pb);
     if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
-    if (cossim_core(Pa, Pb, m, r, r, Ct, misc->bar, &misc->sweeps, &misc->cossim, a.status, ws + L.jx, s) !=
-        cudaSuccess)
-      return QG_ECUDA;
+    if (cossim_core(Pa, Pb, m, r, r, Ct, &misc->ns_scale, &misc->cossim, s) != cudaSuccess) return QG_ECUDA;
     if (refresh_moments(a, Pa, Pb, reinterpret_cast<float*>(ws + L.At), reinterpret_cast<float*>(ws + L.Vt),
                         reinterpret_cast<float*>(ws + L.Bm), reinterpret_cast<float*>(ws + L.mom), L.ldn4, s) !=
         cudaSuccess)
@@ -687,11 +737,9 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
 
 qg_status run_cossim(const float* Pa, const float* Pb, int32_t m, int32_t r, int64_t ld, float* d_out, uint8_t* ws,
                      cudaStream_t stream) {
-  float* Ct = reinterpret_cast<float*>(ws);
-  unsigned* bar = reinterpret_cast<unsigned*>(ws + r256(size_t(r) * r * 4));
-  int* sweeps = reinterpret_cast<int*>(bar + 8);
-  uint8_t* jx = ws + r256(size_t(r) * r * 4) + 256;
-  return st_of(cossim_core(Pa, Pb, m, r, ld, Ct, bar, sweeps, d_out, nullptr, jx, stream));
+  float* buf = reinterpret_cast<float*>(ws);
+  float* scal = reinterpret_cast<float*>(ws + r256(size_t(r) * r * 4 * 4));
+  return st_of(cossim_core(Pa, Pb, m, r, ld, buf, scal, d_out, stream));
 }
 
 }  // namespace qg
