@@ -243,9 +243,20 @@ class Config:
     seed: int = 0
     layer_id: int = 0
     mom_refresh: int = 0  # moments at a refresh: 0 keep, 1 reset, 2 rotate (see refresh_moments)
+    proj_side: int = 0    # 0: P m x r, R = P^T G (the default reading); 1: P n x r, R = G P
 
     def f32(self, name):
         return F32(getattr(self, name))
+
+
+def proj_dims(cfg: Config):
+    """(rows of P, rows of R, columns of R): (m, r, n) for the left projection,
+    (n, m, r) for the right one.  The moments have R's shape."""
+    if cfg.proj_side == 0:
+        return cfg.m, cfg.r, cfg.n
+    if cfg.proj_side == 1:
+        return cfg.n, cfg.m, cfg.r
+    raise ValueError("proj_side must be 0 or 1")
 
 
 def adam_constants(cfg: Config, t: int):
@@ -266,8 +277,21 @@ def adam_constants(cfg: Config, t: int):
 def project(P_bf16, G) -> np.ndarray:
     """Step a2: R = P~^T G (r x n), float64 sum of the exact products, rounded to
     float32.  [QG-abs]: the gradient is projected into the low-rank subspace;
-    reading: the left factor is always projected (P is m x r)."""
+    reading: the left factor is projected (P is m x r) unless the right-side
+    variant is asked for (project_right)."""
     return (np.asarray(P_bf16, np.float64).T @ np.asarray(G, np.float64)).astype(np.float32)
+
+
+def project_right(G, P_bf16) -> np.ndarray:
+    """Step a2 of the right-side variant: R = G P~ (m x r) for P n x r, float64
+    sum of the exact products, rounded to float32."""
+    return (np.asarray(G, np.float64) @ np.asarray(P_bf16, np.float64)).astype(np.float32)
+
+
+def backproject_right(N_bf16, P_bf16) -> np.ndarray:
+    """Step a4 of the right-side variant: U = N P~^T (m x n) for N m x r and
+    P n x r, in float64 from the exact bf16 operands, rounded to float32."""
+    return (np.asarray(N_bf16, np.float64) @ np.asarray(P_bf16, np.float64).T).astype(np.float32)
 
 
 def adam_moments(R, m0, v0, cfg: Config, t: int):
@@ -401,10 +425,11 @@ class LayerState:
 
     @staticmethod
     def create(cfg: Config, Wq, sW):
-        nb = -(-cfg.n // cfg.mom_block)
+        _, rows, cols = proj_dims(cfg)
+        nb = -(-cols // cfg.mom_block)
         return LayerState(cfg=cfg, Wq=np.array(Wq, np.int8), sW=np.array(sW, np.float32),
-                          Mq=np.zeros((cfg.r, cfg.n), np.int8), sM=np.zeros((cfg.r, nb), np.float32),
-                          Vq=np.zeros((cfg.r, cfg.n), np.int8), sV=np.zeros((cfg.r, nb), np.float32),
+                          Mq=np.zeros((rows, cols), np.int8), sM=np.zeros((rows, nb), np.float32),
+                          Vq=np.zeros((rows, cols), np.int8), sV=np.zeros((rows, nb), np.float32),
                           delta=cfg.delta0)
 
 
@@ -414,10 +439,11 @@ def step(st: LayerState, G) -> dict:
     Returns the intermediates (P~, R, N, U) for inspection."""
     cfg = st.cfg
     st.t += 1
-    Pb = dequant_P_bf16(st.Pq, st.sP, cfg.m, cfg.r, cfg.p_group)
-    R = project(Pb, G)
+    p_rows, _, _ = proj_dims(cfg)
+    Pb = dequant_P_bf16(st.Pq, st.sP, p_rows, cfg.r, cfg.p_group)
+    R = project(Pb, G) if cfg.proj_side == 0 else project_right(G, Pb)
     N, st.Mq, st.sM, st.Vq, st.sV = lowrank_adam_int8(R, st.Mq, st.sM, st.Vq, st.sV, cfg, st.t)
-    U = backproject(Pb, N)
+    U = backproject(Pb, N) if cfg.proj_side == 0 else backproject_right(N, Pb)
     st.Wq = stochastic_round_update(st.Wq, st.sW, U, cfg, st.t)
     return dict(P=Pb, R=R, N=N, U=U)
 
@@ -523,14 +549,17 @@ def refresh(st: LayerState, G, force=False) -> dict | None:
         return None
     cfg = st.cfg
     k = refresh_width(cfg)
-    Omega = rademacher_omega(cfg.n, k, cfg.seed, st.n_refresh, cfg.layer_id)
-    P, sigma = randomized_topr(G, cfg.r, k, cfg.power_iters, Omega)
+    # the right-side variant takes the top-r left singular vectors of G^T
+    Geff = np.asarray(G) if cfg.proj_side == 0 else np.asarray(G).T
+    p_rows = Geff.shape[0]
+    Omega = rademacher_omega(Geff.shape[1], k, cfg.seed, st.n_refresh, cfg.layer_id)
+    P, sigma = randomized_topr(Geff, cfg.r, k, cfg.power_iters, Omega)
     codes, sP = quant_int4_groups(P.astype(np.float32), cfg.p_group)
     Pq = pack_int4(codes)
     cs = None
     if st.Pq is not None:
-        Pa = dequant_int4_f32(Pq, sP, cfg.m, cfg.r, cfg.p_group)
-        Pb = dequant_int4_f32(st.Pq, st.sP, cfg.m, cfg.r, cfg.p_group)
+        Pa = dequant_int4_f32(Pq, sP, p_rows, cfg.r, cfg.p_group)
+        Pb = dequant_int4_f32(st.Pq, st.sP, p_rows, cfg.r, cfg.p_group)
         cs = cossim(Pa, Pb)
         refresh_moments(st, Pa, Pb)
         st.Pq_prev, st.sP_prev = st.Pq, st.sP
@@ -553,7 +582,9 @@ def refresh_moments(st: LayerState, Pa, Pb):
          mapped as the variance of independent coordinates is (C o C the
          element-wise square).  C, and both products, in float64 from the
          float32 operands; the results rounded to float32 and re-quantized on the
-         step's grids (linear for m, square root for v)."""
+         step's grids (linear for m, square root for v).  For the right-side
+         projection the r coordinates run along the columns of the moments
+         (m x r): m' = m C^T and v' = v (C o C)^T."""
     cfg = st.cfg
     if cfg.mom_refresh == 0:
         return
@@ -568,8 +599,12 @@ def refresh_moments(st: LayerState, Pa, Pb):
     C = np.asarray(Pa, np.float64).T @ np.asarray(Pb, np.float64)
     m0 = dequant_rowblock(st.Mq, st.sM, cfg.mom_block).astype(np.float64)
     v0 = dequant_second_moment(st.Vq, st.sV, cfg.mom_block).astype(np.float64)
-    m1 = (C @ m0).astype(np.float32)
-    v1 = ((C * C) @ v0).astype(np.float32)
+    if cfg.proj_side == 0:
+        m1 = (C @ m0).astype(np.float32)
+        v1 = ((C * C) @ v0).astype(np.float32)
+    else:
+        m1 = (m0 @ C.T).astype(np.float32)
+        v1 = (v0 @ (C * C).T).astype(np.float32)
     st.Mq, st.sM = quant_rowblock_int8(m1, cfg.mom_block, unsigned=False)
     st.Vq, st.sV = quant_rowblock_int8(np.sqrt(v1).astype(np.float32), cfg.mom_block, unsigned=True)
 

@@ -649,3 +649,52 @@ def test_refresh_moments_rotation_identity_and_permutation():
     O.refresh_moments(st, P * flip[None, :], P)
     np.testing.assert_allclose(O.dequant_rowblock(st.Mq, st.sM), m_old * flip[:, None], rtol=0, atol=1e-9)
     assert np.array_equal(st.Vq, Vq_old)
+
+
+# ---------------------------------------------------------------- right-side projection (P n x r)
+
+def test_right_side_products_brute_force():
+    rng = np.random.default_rng(17)
+    m, n, r = 7, 5, 3
+    P = O.bf16_round(rng.standard_normal((n, r)).astype(np.float32))
+    G = O.bf16_round(rng.standard_normal((m, n)).astype(np.float32))
+    N = O.bf16_round(rng.standard_normal((m, r)).astype(np.float32))
+    R, U = O.project_right(G, P), O.backproject_right(N, P)
+    assert R.shape == (m, r) and U.shape == (m, n)
+    for i in range(m):
+        for a in range(r):
+            assert R[i, a] == np.float32(math.fsum(float(G[i, j]) * float(P[j, a]) for j in range(n)))
+        for j in range(n):
+            assert U[i, j] == np.float32(math.fsum(float(N[i, a]) * float(P[j, a]) for a in range(r)))
+
+
+def test_right_side_refresh_finds_the_right_singular_vectors():
+    # a gap input with m > n: the right-side refresh returns P (n x r) spanning
+    # the top-r right singular vectors that LAPACK's SVD gives
+    m, n, r = 160, 96, 32
+    G, _ = synth.gap_gradient(m, n, r, seed=31)
+    cfg = O.Config(m=m, n=n, r=r, seed=3, proj_side=1)
+    st = O.LayerState.create(cfg, np.zeros((m, n), np.int8), np.ones(-(-m * n // 256), np.float32))
+    assert st.Mq.shape == (m, r) and st.sM.shape == (m, 1)
+    out = O.refresh(st, G, force=True)
+    P = out["P"]
+    assert P.shape == (n, r)
+    Vt = np.linalg.svd(np.asarray(G, np.float64), full_matrices=False)[2]
+    cos = np.cos(scipy.linalg.subspace_angles(P, Vt[:r].T))
+    assert cos.min() > 0.999
+
+
+def test_right_side_moment_rotation_permutes_columns():
+    m, n, r = 300, 64, 32
+    cfg = O.Config(m=m, n=n, r=r, seed=5, mom_refresh=2, proj_side=1)
+    rng = np.random.default_rng(5)
+    st = O.LayerState.create(cfg, np.zeros((m, n), np.int8), np.ones(-(-m * n // 256), np.float32))
+    mom = rng.standard_normal((m, r)).astype(np.float32) * 1e-3
+    st.Mq, st.sM = O.quant_rowblock_int8(mom, 256)
+    st.Vq, st.sV = O.quant_rowblock_int8(np.abs(mom) * 2, 256, unsigned=True)
+    m_old, Vq_old = O.dequant_rowblock(st.Mq, st.sM), st.Vq.copy()
+    P = synth.orthonormal(n, r, seed=1)
+    perm = np.random.default_rng(4).permutation(r)
+    O.refresh_moments(st, P[:, perm], P)
+    np.testing.assert_allclose(O.dequant_rowblock(st.Mq, st.sM), m_old[:, perm], rtol=0, atol=1e-9)
+    assert np.array_equal(st.Vq, Vq_old[:, perm])
