@@ -74,6 +74,9 @@ typedef struct {
                                1 reset them to zero, 2 rotate them into the new basis with
                                C = P_new^T P_prev: m' = C m, v' = (C o C) v (element-wise square),
                                re-quantized on the step's grids */
+  int32_t proj_side;        /* which side is projected: 0 (default) P is m x r and R = P^T G (r x n);
+                               1 P is n x r, R = G P (m x r) and U = N P^T, the projection taken
+                               from the top-r right singular vectors of G */
 } qg_config;
 
 typedef struct qg_layer qg_layer;
@@ -89,8 +92,10 @@ typedef struct {
   int8_t* Vq;               /* r x ld_mom INT8 codes 0..127 of sqrt(v), v the second moment */
   float* sM;                /* r x nblk float32 */
   float* sV;                /* r x nblk float32 */
-  int64_t ld_mom;           /* row stride of Mq, Vq in bytes: n rounded up to 32 */
-  int32_t nblk;             /* ceil(n / 256) */
+  int64_t ld_mom;           /* row stride of Mq, Vq in bytes: mom_cols rounded up to 32 */
+  int32_t nblk;             /* ceil(mom_cols / 256) */
+  int32_t p_rows;           /* rows of P: m (left projection) or n (right) */
+  int32_t mom_rows, mom_cols; /* shape of the moments (that of R): r x n (left) or m x r (right) */
 } qg_layer_views;
 
 /* Schedule state of the layer-adaptive refresh (host side). */
@@ -136,9 +141,10 @@ qg_status qg_layer_views_get(const qg_layer* layer, qg_layer_views* views);
 qg_status qg_layer_sched_get(const qg_layer* layer, qg_sched* sched);
 qg_status qg_layer_sched_set(qg_layer* layer, const qg_sched* sched);
 
-/* Install an INT4 projection (e.g. from a checkpoint): copies ceil(m*r/2)
- * packed bytes and ceil(m*r/64) scales device-to-device into the state.  The
- * previous projection is kept for CosSim only when keep_prev != 0. */
+/* Install an INT4 projection (e.g. from a checkpoint): copies ceil(p*r/2)
+ * packed bytes and ceil(p*r/64) scales device-to-device into the state, p the
+ * rows of P (m, or n for the right-side projection).  The previous projection
+ * is kept for CosSim only when keep_prev != 0. */
 qg_status qg_layer_set_projection(qg_layer* layer, const uint8_t* d_Pq, const float* d_sP,
                                   int32_t keep_prev, void* stream);
 

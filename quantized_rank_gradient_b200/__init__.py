@@ -29,13 +29,15 @@ class qg_config(Structure):
     _fields_ = [("m", c_int32), ("n", c_int32), ("r", c_int32), ("w_group", c_int32), ("p_group", c_int32),
                 ("mom_block", c_int32), ("beta1", c_float), ("beta2", c_float), ("eps", c_float), ("lr", c_float),
                 ("alpha", c_float), ("gamma", c_float), ("delta0", c_int32), ("oversample", c_int32),
-                ("power_iters", c_int32), ("seed", c_uint64), ("layer_id", c_uint32), ("mom_refresh", c_int32)]
+                ("power_iters", c_int32), ("seed", c_uint64), ("layer_id", c_uint32), ("mom_refresh", c_int32),
+                ("proj_side", c_int32)]
 
 
 class qg_layer_views(Structure):
     _fields_ = [("status", c_void_p), ("Pq", c_void_p), ("sP", c_void_p), ("Pq_prev", c_void_p),
                 ("sP_prev", c_void_p), ("Mq", c_void_p), ("Vq", c_void_p), ("sM", c_void_p), ("sV", c_void_p),
-                ("ld_mom", c_int64), ("nblk", c_int32)]
+                ("ld_mom", c_int64), ("nblk", c_int32), ("p_rows", c_int32), ("mom_rows", c_int32),
+                ("mom_cols", c_int32)]
 
 
 class qg_sched(Structure):

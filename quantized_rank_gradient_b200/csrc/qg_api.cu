@@ -36,15 +36,25 @@ struct StateLayout {
   size_t status, Pq, sP, Pq_prev, sP_prev, Mq, Vq, sM, sV, total;
   int64_t ld_mom;
   int32_t nblk;
+  int32_t p_rows, mom_rows, mom_cols;
 };
+
+// Rows of P, and the moments' shape (that of R): P m x r and R r x n for the
+// left projection; P n x r and R m x r for the right one.
+void proj_dims(const qg_config& c, int32_t* p_rows, int32_t* rows, int32_t* cols) {
+  *p_rows = c.proj_side ? c.n : c.m;
+  *rows = c.proj_side ? c.m : c.r;
+  *cols = c.proj_side ? c.r : c.n;
+}
 
 StateLayout state_layout(const qg_config& c) {
   StateLayout L;
-  const size_t mr = static_cast<size_t>(c.m) * c.r;
+  proj_dims(c, &L.p_rows, &L.mom_rows, &L.mom_cols);
+  const size_t mr = static_cast<size_t>(L.p_rows) * c.r;
   const size_t pq = (mr + 1) / 2;
   const size_t ps = ((mr + 63) / 64) * sizeof(float);
-  L.ld_mom = (static_cast<int64_t>(c.n) + 31) / 32 * 32;
-  L.nblk = (c.n + 255) / 256;
+  L.ld_mom = (static_cast<int64_t>(L.mom_cols) + 31) / 32 * 32;
+  L.nblk = (L.mom_cols + 255) / 256;
   size_t off = 0;
   L.status = off;
   off += 256;
@@ -57,13 +67,13 @@ StateLayout state_layout(const qg_config& c) {
   L.sP_prev = off;
   off += round256(ps);
   L.Mq = off;
-  off += round256(static_cast<size_t>(c.r) * L.ld_mom);
+  off += round256(static_cast<size_t>(L.mom_rows) * L.ld_mom);
   L.Vq = off;
-  off += round256(static_cast<size_t>(c.r) * L.ld_mom);
+  off += round256(static_cast<size_t>(L.mom_rows) * L.ld_mom);
   L.sM = off;
-  off += round256(static_cast<size_t>(c.r) * L.nblk * sizeof(float));
+  off += round256(static_cast<size_t>(L.mom_rows) * L.nblk * sizeof(float));
   L.sV = off;
-  off += round256(static_cast<size_t>(c.r) * L.nblk * sizeof(float));
+  off += round256(static_cast<size_t>(L.mom_rows) * L.nblk * sizeof(float));
   L.total = off;
   return L;
 }
@@ -79,6 +89,7 @@ qg_status check_config(const qg_config* c) {
   if (!(c->eps > 0.f) || !isfinite(c->eps) || !isfinite(c->lr) || !isfinite(c->alpha)) return QG_EINVAL;
   if (!isfinite(c->gamma) || c->delta0 < 1 || c->oversample < 0 || c->power_iters < 0) return QG_EINVAL;
   if (c->mom_refresh < 0 || c->mom_refresh > 2) return QG_EINVAL;
+  if (c->proj_side < 0 || c->proj_side > 1) return QG_EINVAL;
   return QG_OK;
 }
 
@@ -101,11 +112,12 @@ void fill_step_problem(const qg_layer* L, const void* G, int64_t ldg, uint8_t* w
   s->ldw = L->ldw;
   s->sW = L->sW;
   s->Pbf = reinterpret_cast<uint16_t*>(ws);
-  s->Nbuf = reinterpret_cast<uint16_t*>(ws + round256(static_cast<size_t>(c.m) * c.r * 2));
-  s->ldN = qg::step_ldN(c.n);
+  s->Nbuf = reinterpret_cast<uint16_t*>(ws + round256(static_cast<size_t>(L->v.p_rows) * c.r * 2));
+  s->ldN = qg::step_ldN(L->v.mom_cols);
   s->m = c.m;
   s->n = c.n;
   s->r = c.r;
+  s->side = c.proj_side;
   const double b1 = static_cast<double>(c.beta1);
   const double b2 = static_cast<double>(c.beta2);
   s->beta1 = c.beta1;
@@ -185,12 +197,13 @@ size_t qg_state_bytes(const qg_config* cfg) {
 
 size_t qg_step_workspace_bytes(const qg_config* cfg) {
   if (check_config(cfg) != QG_OK) return 0;
-  return qg::step_scratch_bytes(cfg->m, cfg->n, cfg->r);
+  return qg::step_scratch_bytes(cfg->m, cfg->n, cfg->r, cfg->proj_side);
 }
 
 size_t qg_refresh_workspace_bytes(const qg_config* cfg) {
   if (check_config(cfg) != QG_OK) return 0;
-  return qg::refresh_scratch_bytes(cfg->m, cfg->n, cfg->r, cfg->oversample);
+  const int32_t pm = cfg->proj_side ? cfg->n : cfg->m, pn = cfg->proj_side ? cfg->m : cfg->n;
+  return qg::refresh_scratch_bytes(pm, pn, cfg->r, cfg->oversample);
 }
 
 qg_status qg_layer_init(qg_layer** out, const qg_config* cfg, void* d_state, size_t state_bytes, int8_t* d_W,
@@ -224,6 +237,9 @@ qg_status qg_layer_init(qg_layer** out, const qg_config* cfg, void* d_state, siz
   L->v.sV = reinterpret_cast<float*>(b + SL.sV);
   L->v.ld_mom = SL.ld_mom;
   L->v.nblk = SL.nblk;
+  L->v.p_rows = SL.p_rows;
+  L->v.mom_rows = SL.mom_rows;
+  L->v.mom_cols = SL.mom_cols;
   L->sched.t = 0;
   L->sched.delta = cfg->delta0;
   L->sched.t_next = 0;
@@ -265,7 +281,7 @@ qg_status qg_layer_set_projection(qg_layer* L, const uint8_t* d_Pq, const float*
                                   void* stream) {
   if (!L || !d_Pq || !d_sP) return QG_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t mr = static_cast<size_t>(L->cfg.m) * L->cfg.r;
+  const size_t mr = static_cast<size_t>(L->v.p_rows) * L->cfg.r;
   const size_t pq = (mr + 1) / 2, ps = ((mr + 63) / 64) * sizeof(float);
   if (keep_prev && L->sched.has_projection) {
     if (cudaMemcpyAsync(L->v.Pq_prev, L->v.Pq, pq, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return QG_ECUDA;
@@ -282,7 +298,7 @@ qg_status qg_step(qg_layer* L, const void* d_G, int64_t ldg, void* d_ws, size_t 
   if (st != QG_OK) return st;
   if (!d_ws) return QG_EINVAL;
   if (!aligned(d_ws, 256)) return QG_EALIGN;
-  if (ws_bytes < qg::step_scratch_bytes(L->cfg.m, L->cfg.n, L->cfg.r)) return QG_ESTATE;
+  if (ws_bytes < qg::step_scratch_bytes(L->cfg.m, L->cfg.n, L->cfg.r, L->cfg.proj_side)) return QG_ESTATE;
   const int64_t t = L->sched.t + 1;
   StepProblem sp;
   fill_step_problem(L, d_G, ldg, static_cast<uint8_t*>(d_ws), t, &sp);
@@ -326,11 +342,13 @@ static qg_status second_lane(Lane** out) {
   return QG_OK;
 }
 
-static size_t batch_slot_bytes(const int32_t* m, const int32_t* n, const int32_t* r, int count) {
+static size_t batch_slot_bytes(const int32_t* m, const int32_t* n, const int32_t* r, const int32_t* side,
+                               int count) {
   size_t slot = 0;
   for (int b = 0; b * kBatch < count; ++b) {
     size_t sum = 0;
-    for (int i = b * kBatch; i < count && i < (b + 1) * kBatch; ++i) sum += qg::step_scratch_bytes(m[i], n[i], r[i]);
+    for (int i = b * kBatch; i < count && i < (b + 1) * kBatch; ++i)
+      sum += qg::step_scratch_bytes(m[i], n[i], r[i], side[i]);
     slot = std::max(slot, sum);
   }
   return slot;
@@ -340,12 +358,12 @@ static int batch_lanes(int count) { return std::min(kLanes, (count + kBatch - 1)
 
 size_t qg_step_batch_workspace_bytes(const qg_config* const* cfgs, int32_t count) {
   if (!cfgs || count < 0) return 0;
-  std::vector<int32_t> m(count), n(count), r(count);
+  std::vector<int32_t> m(count), n(count), r(count), side(count);
   for (int i = 0; i < count; ++i) {
     if (check_config(cfgs[i]) != QG_OK) return 0;
-    m[i] = cfgs[i]->m, n[i] = cfgs[i]->n, r[i] = cfgs[i]->r;
+    m[i] = cfgs[i]->m, n[i] = cfgs[i]->n, r[i] = cfgs[i]->r, side[i] = cfgs[i]->proj_side;
   }
-  return batch_slot_bytes(m.data(), n.data(), r.data(), count) * batch_lanes(count);
+  return batch_slot_bytes(m.data(), n.data(), r.data(), side.data(), count) * batch_lanes(count);
 }
 
 qg_status qg_step_batch(qg_layer* const* layers, const void* const* d_G, const int64_t* ldg, int32_t count,
@@ -353,15 +371,15 @@ qg_status qg_step_batch(qg_layer* const* layers, const void* const* d_G, const i
   if (count < 0 || (count > 0 && (!layers || !d_G || !ldg || !d_ws))) return QG_EINVAL;
   if (count == 0) return QG_OK;
   if (!aligned(d_ws, 256)) return QG_EALIGN;
-  std::vector<int32_t> m(count), n(count), r(count);
+  std::vector<int32_t> m(count), n(count), r(count), side(count);
   for (int i = 0; i < count; ++i) {
     qg_status st = check_step_args(layers[i], d_G[i], ldg[i]);
     if (st != QG_OK) return st;
     for (int j = 0; j < i; ++j)
       if (layers[j] == layers[i]) return QG_EINVAL;
-    m[i] = layers[i]->cfg.m, n[i] = layers[i]->cfg.n, r[i] = layers[i]->cfg.r;
+    m[i] = layers[i]->cfg.m, n[i] = layers[i]->cfg.n, r[i] = layers[i]->cfg.r, side[i] = layers[i]->cfg.proj_side;
   }
-  const size_t slot = batch_slot_bytes(m.data(), n.data(), r.data(), count);
+  const size_t slot = batch_slot_bytes(m.data(), n.data(), r.data(), side.data(), count);
   const int lanes = batch_lanes(count);
   if (ws_bytes < slot * lanes) return QG_ESTATE;
   std::vector<StepProblem> probs(count);
@@ -369,7 +387,7 @@ qg_status qg_step_batch(qg_layer* const* layers, const void* const* d_G, const i
     uint8_t* ws = static_cast<uint8_t*>(d_ws) + (b % lanes) * slot;
     for (int i = b * kBatch; i < count && i < (b + 1) * kBatch; ++i) {
       fill_step_problem(layers[i], d_G[i], ldg[i], ws, layers[i]->sched.t + 1, &probs[i]);
-      ws += qg::step_scratch_bytes(m[i], n[i], r[i]);
+      ws += qg::step_scratch_bytes(m[i], n[i], r[i], side[i]);
     }
   }
   const cudaStream_t user = static_cast<cudaStream_t>(stream);
@@ -425,15 +443,18 @@ qg_status qg_refresh(qg_layer* L, const void* d_G, int64_t ldg, int32_t force, v
   if (ldg < c.n || ldg % 8 != 0 || !aligned(d_G, 16)) return QG_EALIGN;
   if (!d_ws) return QG_EINVAL;
   if (!aligned(d_ws, 256)) return QG_EALIGN;
-  if (ws_bytes < qg::refresh_scratch_bytes(c.m, c.n, c.r, c.oversample)) return QG_ESTATE;
+  // the right-side projection refreshes on G^T: P has n rows
+  const int32_t pm = c.proj_side ? c.n : c.m, pn = c.proj_side ? c.m : c.n;
+  if (ws_bytes < qg::refresh_scratch_bytes(pm, pn, c.r, c.oversample)) return QG_ESTATE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool has_prev = L->sched.has_projection != 0;
   qg::RefreshArgs ra;
   memset(&ra, 0, sizeof(ra));
   ra.G = d_G;
   ra.ldg = ldg;
-  ra.m = c.m;
-  ra.n = c.n;
+  ra.m = pm;
+  ra.n = pn;
+  ra.transpose_g = c.proj_side;
   ra.r = c.r;
   ra.oversample = c.oversample;
   ra.power_iters = c.power_iters;
@@ -453,6 +474,8 @@ qg_status qg_refresh(qg_layer* L, const void* d_G, int64_t ldg, int32_t force, v
   ra.sV = L->v.sV;
   ra.ld_mom = L->v.ld_mom;
   ra.nblk = L->v.nblk;
+  ra.mom_rows = L->v.mom_rows;
+  ra.mom_cols = L->v.mom_cols;
   float cs = 0.f;
   qg_status st = qg::run_refresh(ra, static_cast<uint8_t*>(d_ws), ws_bytes, s, &cs);
   if (st != QG_OK) return st;

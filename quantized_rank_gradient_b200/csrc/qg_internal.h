@@ -12,7 +12,7 @@ struct StepProblem {
   const float* sP;      // m*r/64 scales
   const void* G;        // m x ldg bf16
   int64_t ldg;
-  int8_t* Mq;           // r x ld_mom
+  int8_t* Mq;           // R's shape (r x n, or m x r for the right side), row stride ld_mom
   int8_t* Vq;
   float* sM;            // r x nblk
   float* sV;
@@ -21,10 +21,11 @@ struct StepProblem {
   int8_t* W;            // m x ldw
   int64_t ldw;
   const float* sW;      // ceil(m*n/256)
-  uint16_t* Pbf;        // scratch: m x r bf16
-  uint16_t* Nbuf;       // scratch: r x ldN bf16
+  uint16_t* Pbf;        // scratch: P~ (m x r bf16, or n x r for the right side)
+  uint16_t* Nbuf;       // scratch: N (R's shape, bf16, row stride ldN)
   int64_t ldN;
   int32_t m, n, r;
+  int32_t side;         // 0: P m x r, R = P^T G (r x n); 1: P n x r, R = G P (m x r)
   float beta1, beta2, om1, om2, c1, c2, eps, alpha;  // c1 = -lr/(1-b1^t), c2 = 1/sqrt(1-b2^t)
   uint32_t t, layer_id;
   uint64_t seed;
@@ -34,7 +35,7 @@ struct StepProblem {
 // Scratch layout of one step: P~ (m x r bf16) then N (r x ldN bf16), each
 // starting on a 256-byte boundary.
 int64_t step_ldN(int32_t n);
-size_t step_scratch_bytes(int32_t m, int32_t n, int32_t r);
+size_t step_scratch_bytes(int32_t m, int32_t n, int32_t r, int32_t side);
 
 // Enqueues a1..a5 for `count` problems on `stream`.  Returns cudaSuccess or the
 // first launch / set-up error.

@@ -57,7 +57,7 @@ extern "C" qg_status qg_step_noalloc(qg_layer* layer, const void* d_G, int64_t l
   qg_config cfg;
   if (qg::layer_config(layer, &cfg) != QG_OK) return QG_EINVAL;
   // Matrices whose scratch (P~ and N) does not fit the static array are refused.
-  if (qg::step_scratch_bytes(cfg.m, cfg.n, cfg.r) > QG_NOALLOC_SCRATCH_BYTES) return QG_ESHAPE;
+  if (qg::step_scratch_bytes(cfg.m, cfg.n, cfg.r, cfg.proj_side) > QG_NOALLOC_SCRATCH_BYTES) return QG_ESHAPE;
   void* scratch = nullptr;
   if (scratch_for_current_device(&scratch) != cudaSuccess) return QG_ECUDA;
   // The regular step, with the static array as its workspace.

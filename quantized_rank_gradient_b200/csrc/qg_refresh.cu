@@ -93,7 +93,9 @@ RefreshLayout refresh_layout(int m, int n, int r, int p) {
   L.Pb = take(size_t(m) * r * 4);
   L.Ct = take(size_t(r) * r * 4 * 4);  // CosSim: C and three Newton-Schulz buffers
   L.jx = take(jacobi_scratch_bytes(L.k));
-  L.mom = take(size_t(r) * L.ldn4 * 4);  // the rotated moments (r x n fp32)
+  // the rotated moments: r x n fp32 for the left projection; for the right one
+  // (refresh called with m and n swapped) n x r, which is r x n here as well
+  L.mom = take(size_t(r) * L.ldn4 * 4);
   L.misc = take(256);
   L.total = off;
   return L;
@@ -550,32 +552,39 @@ qg_status st_of(cudaError_t e) { return e == cudaSuccess ? QG_OK : QG_ECUDA; }
 // by Pa: kept, reset to zero, or rotated with C = Pa^T Pb (m' = C m,
 // v' = (C o C) v) and re-quantized.  C and C2 are r x r scratch, X and Y r x ldx.
 cudaError_t refresh_moments(const RefreshArgs& a, const float* Pa, const float* Pb, float* C, float* C2, float* X,
-                            float* Y, int64_t ldx, cudaStream_t s) {
-  const int m = a.m, n = a.n, r = a.r;
+                            float* Y, cudaStream_t s) {
+  // the moments are rows x cols (r x n, or m x r for the right-side projection,
+  // whose r coordinates run along the columns); X and Y rows x cols, stride cols
+  const int pm = a.m, r = a.r, rows = a.mom_rows, cols = a.mom_cols;
+  const int64_t ldx = cols;
   cudaError_t e;
   if (a.mom_refresh == 0) return cudaSuccess;
   if (a.mom_refresh == 1) {
-    const size_t codes = size_t(r) * a.ld_mom, sc = size_t(r) * a.nblk * 4;
+    const size_t codes = size_t(rows) * a.ld_mom, sc = size_t(rows) * a.nblk * 4;
     if ((e = cudaMemsetAsync(a.Mq, 0, codes, s)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(a.Vq, 0, codes, s)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(a.sM, 0, sc, s)) != cudaSuccess) return e;
     return cudaMemsetAsync(a.sV, 0, sc, s);
   }
-  if ((e = sgemm(true, false, Pa, r, Pb, r, C, r, r, r, m, s)) != cudaSuccess) return e;
-  const int64_t rr = int64_t(r) * r, rn = int64_t(r) * n;
+  if ((e = sgemm(true, false, Pa, r, Pb, r, C, r, r, r, pm, s)) != cudaSuccess) return e;
+  const int64_t rr = int64_t(r) * r, rc = int64_t(rows) * cols;
   square_kernel<<<static_cast<unsigned>((rr + 255) / 256), 256, 0, s>>>(C, C2, rr);
-  const unsigned eb = static_cast<unsigned>((rn + 255) / 256);
-  const unsigned qb = static_cast<unsigned>((int64_t(r) * a.nblk * 32 + 255) / 256);
-  // m' = C m
-  moment_dequant_kernel<false><<<eb, 256, 0, s>>>(a.Mq, a.ld_mom, a.sM, a.nblk, r, n, X, ldx);
+  const unsigned eb = static_cast<unsigned>((rc + 255) / 256);
+  const unsigned qb = static_cast<unsigned>((int64_t(rows) * a.nblk * 32 + 255) / 256);
+  // m' = C m (left) or m C^T (right)
+  moment_dequant_kernel<false><<<eb, 256, 0, s>>>(a.Mq, a.ld_mom, a.sM, a.nblk, rows, cols, X, ldx);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = sgemm(false, false, C, r, X, ldx, Y, ldx, r, n, r, s)) != cudaSuccess) return e;
-  moment_quant_kernel<false><<<qb, 256, 0, s>>>(Y, ldx, r, n, a.nblk, a.Mq, a.ld_mom, a.sM);
-  // v' = (C o C) v
-  moment_dequant_kernel<true><<<eb, 256, 0, s>>>(a.Vq, a.ld_mom, a.sV, a.nblk, r, n, X, ldx);
+  e = a.transpose_g ? sgemm(false, true, X, ldx, C, r, Y, ldx, rows, cols, r, s)
+                    : sgemm(false, false, C, r, X, ldx, Y, ldx, rows, cols, r, s);
+  if (e != cudaSuccess) return e;
+  moment_quant_kernel<false><<<qb, 256, 0, s>>>(Y, ldx, rows, cols, a.nblk, a.Mq, a.ld_mom, a.sM);
+  // v' = (C o C) v (left) or v (C o C)^T (right)
+  moment_dequant_kernel<true><<<eb, 256, 0, s>>>(a.Vq, a.ld_mom, a.sV, a.nblk, rows, cols, X, ldx);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = sgemm(false, false, C2, r, X, ldx, Y, ldx, r, n, r, s)) != cudaSuccess) return e;
-  moment_quant_kernel<true><<<qb, 256, 0, s>>>(Y, ldx, r, n, a.nblk, a.Vq, a.ld_mom, a.sV);
+  e = a.transpose_g ? sgemm(false, true, X, ldx, C2, r, Y, ldx, rows, cols, r, s)
+                    : sgemm(false, false, C2, r, X, ldx, Y, ldx, rows, cols, r, s);
+  if (e != cudaSuccess) return e;
+  moment_quant_kernel<true><<<qb, 256, 0, s>>>(Y, ldx, rows, cols, a.nblk, a.Vq, a.ld_mom, a.sV);
   return cudaGetLastError();
 }
 
@@ -673,22 +682,25 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
                                                                           key);
     if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
   }
-  if (launch_gemm_f32(a.G, a.ldg, false, Om, ldk, false, Y, ldk, m, k, n, s) != cudaSuccess) return QG_ECUDA;
+  // G_eff (m x n) is G, or G^T for the right-side projection: the products
+  // below take G as stored with the transposition flags flipped
+  const bool tr = a.transpose_g != 0;
+  if (launch_gemm_f32(a.G, a.ldg, tr, Om, ldk, false, Y, ldk, m, k, n, s) != cudaSuccess) return QG_ECUDA;
   // two passes for the intermediate bases, three for the final Q
   constexpr int kInterPasses = 2, kFinalPasses = 3;
   if (orth(Y, Yb, Ylo, m, k, ldk, ob, a.power_iters > 0 ? kInterPasses : kFinalPasses, s) != cudaSuccess)
     return QG_ECUDA;
   for (int it = 0; it < a.power_iters; ++it) {
-    if (launch_gemm_f32(a.G, a.ldg, true, Yb, ldk, false, Z, ldk, n, k, m, s) != cudaSuccess) return QG_ECUDA;
+    if (launch_gemm_f32(a.G, a.ldg, !tr, Yb, ldk, false, Z, ldk, n, k, m, s) != cudaSuccess) return QG_ECUDA;
     if (orth(Z, Zb, Zlo, n, k, ldk, ob, kInterPasses, s) != cudaSuccess) return QG_ECUDA;
-    if (launch_gemm_f32(a.G, a.ldg, false, Zb, ldk, false, Y, ldk, m, k, n, s) != cudaSuccess) return QG_ECUDA;
+    if (launch_gemm_f32(a.G, a.ldg, tr, Zb, ldk, false, Y, ldk, m, k, n, s) != cudaSuccess) return QG_ECUDA;
     const int passes = it + 1 == a.power_iters ? kFinalPasses : kInterPasses;
     if (orth(Y, Yb, Ylo, m, k, ldk, ob, passes, s) != cudaSuccess) return QG_ECUDA;
   }
   // Rayleigh-Ritz: B = Q^T G, S = B B^T, eigenpairs of S
   // B = Q^T G with Q split into bf16 hi + lo parts (about 16 significant bits)
-  if (launch_gemm_f32(Yb, ldk, true, a.G, a.ldg, false, Bm, L.ldn4, k, n, m, s) != cudaSuccess) return QG_ECUDA;
-  if (launch_gemm_f32(Ylo, ldk, true, a.G, a.ldg, false, Bm, L.ldn4, k, n, m, s, true) != cudaSuccess)
+  if (launch_gemm_f32(Yb, ldk, true, a.G, a.ldg, tr, Bm, L.ldn4, k, n, m, s) != cudaSuccess) return QG_ECUDA;
+  if (launch_gemm_f32(Ylo, ldk, true, a.G, a.ldg, tr, Bm, L.ldn4, k, n, m, s, true) != cudaSuccess)
     return QG_ECUDA;
   if (sgemm(false, true, Bm, L.ldn4, Bm, L.ldn4, At, ldk, k, k, n, s) != cudaSuccess) return QG_ECUDA;
   {
@@ -724,8 +736,7 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
     if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
     if (cossim_core(Pa, Pb, m, r, r, Ct, &misc->ns_scale, &misc->cossim, s) != cudaSuccess) return QG_ECUDA;
     if (refresh_moments(a, Pa, Pb, reinterpret_cast<float*>(ws + L.At), reinterpret_cast<float*>(ws + L.Vt),
-                        reinterpret_cast<float*>(ws + L.Bm), reinterpret_cast<float*>(ws + L.mom), L.ldn4, s) !=
-        cudaSuccess)
+                        reinterpret_cast<float*>(ws + L.Bm), reinterpret_cast<float*>(ws + L.mom), s) != cudaSuccess)
       return QG_ECUDA;
     float host = 0.f;
     if (cudaMemcpyAsync(&host, &misc->cossim, sizeof(float), cudaMemcpyDeviceToHost, s) != cudaSuccess) return QG_ECUDA;

@@ -32,6 +32,10 @@ struct RefreshArgs {
   float* sV;
   int64_t ld_mom;
   int32_t nblk;
+  int32_t mom_rows, mom_cols;  // the moments' shape (that of R)
+  // 1 for the right-side projection: m and n above are then the rows of P
+  // (the layer's n) and the layer's m, and the refresh works on G^T
+  int32_t transpose_g;
 };
 
 size_t refresh_scratch_bytes(int32_t m, int32_t n, int32_t r, int32_t oversample);

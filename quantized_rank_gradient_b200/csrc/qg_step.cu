@@ -666,8 +666,10 @@ int64_t step_ldN(int32_t n) { return (static_cast<int64_t>(n) + 31) / 32 * 32; }
 
 static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
-size_t step_scratch_bytes(int32_t m, int32_t n, int32_t r) {
-  return round256(static_cast<size_t>(m) * r * 2) + round256(static_cast<size_t>(r) * step_ldN(n) * 2);
+size_t step_scratch_bytes(int32_t m, int32_t n, int32_t r, int32_t side) {
+  // P~ (rows of P x r), then N (R's shape: r x n, or m x r for the right side)
+  const int32_t p_rows = side ? n : m, rows = side ? m : r, cols = side ? r : n;
+  return round256(static_cast<size_t>(p_rows) * r * 2) + round256(static_cast<size_t>(rows) * step_ldN(cols) * 2);
 }
 
 template <class Epi, bool kAMN, bool kBMN>
@@ -690,10 +692,10 @@ static cudaError_t launch_gemm(const GemmParams<Epi>& p, cudaStream_t stream, in
 }
 
 // The same GEMMs on CTA pairs (256 x 256 tiles, cta_group::2).
-template <class Epi, bool kAMN>
+template <class Epi, bool kAMN, bool kBMN = true>
 static cudaError_t launch_gemm_pair(const GemmParams<Epi>& p, cudaStream_t stream, int kind, double flops,
                                     double bytes) {
-  auto kern = gemm_tc_pair_kernel<Epi, kAMN, true>;
+  auto kern = gemm_tc_pair_kernel<Epi, kAMN, kBMN>;
   constexpr size_t kSmem = PairLayout<Epi>::kSmemBytes;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
@@ -772,28 +774,40 @@ static cudaError_t launch_dequant_for(const StepProblem* probs, int cnt, cudaStr
     db.Pq[i] = s.Pq;
     db.sP[i] = s.sP;
     db.out[i] = s.Pbf;
-    db.chunk_begin[i + 1] = db.chunk_begin[i] + static_cast<int64_t>(s.m) * s.r / 32;
+    db.chunk_begin[i + 1] = db.chunk_begin[i] + static_cast<int64_t>(s.side ? s.n : s.m) * s.r / 32;
   }
   db.n = cnt;
   return launch_dequant_batch(db, stream);
 }
 
-static cudaError_t launch_gemms_for(const StepProblem* probs, int cnt, cudaStream_t stream) {
+// a2+a3 and a4+a5 for the problems of one projection side (kRight: P n x r,
+// R = G P, U = N P^T; otherwise P m x r, R = P^T G, U = P N): one grid each.
+template <bool kRight>
+static cudaError_t launch_gemms_side(const StepProblem* probs, const int* idx, int cnt, cudaStream_t stream) {
   cudaError_t e;
-  {
-    GemmParams<AdamEpi> p1;
-    memset(&p1, 0, sizeof(p1));
-    double fl1 = 0, by1 = 0, fl2 = 0, by2 = 0;
-    for (int i = 0; i < cnt; ++i) {
-      const StepProblem& s = probs[i];
-      const double m = s.m, n = s.n, r = s.r;
-      fl1 += 2 * m * n * r;
-      fl2 += 2 * m * n * r;
-      // a2+a3: G, P~, moments read + written, their scales, N written
-      by1 += 2 * m * n + 2 * m * r + 4 * r * n + 16.0 * r * s.nblk + 2 * r * n;
-      // a4+a5: W read + written, W scales, P~, N
-      by2 += 2 * m * n + 4 * std::ceil(m * n / 256.0) + 2 * m * r + 2 * r * n;
-      GemmProblem<AdamEpi>& pr = p1.prob[p1.nprob];
+  GemmParams<AdamEpi> p1;
+  memset(&p1, 0, sizeof(p1));
+  double fl1 = 0, by1 = 0, fl2 = 0, by2 = 0;
+  for (int ii = 0; ii < cnt; ++ii) {
+    const StepProblem& s = probs[idx[ii]];
+    const double m = s.m, n = s.n, r = s.r;
+    const double p_rows = kRight ? n : m, rows = kRight ? m : r, cols = kRight ? r : n;
+    fl1 += 2 * m * n * r;
+    fl2 += 2 * m * n * r;
+    // a2+a3: G, P~, moments read + written, their scales, N written
+    by1 += 2 * m * n + 2 * p_rows * r + 4 * rows * cols + 16.0 * rows * s.nblk + 2 * rows * cols;
+    // a4+a5: W read + written, W scales, P~, N
+    by2 += 2 * m * n + 4 * std::ceil(m * n / 256.0) + 2 * p_rows * r + 2 * rows * cols;
+    GemmProblem<AdamEpi>& pr = p1.prob[p1.nprob];
+    if (kRight) {
+      // A = G (M = m, K = n), K-major: box {64 (n), 128 (m)}
+      if (!encode_map_bf16(&pr.tmA, s.G, s.n, s.m, s.ldg, 64, 128)) return cudaErrorInvalidValue;
+      // B = P~ (K = n, N = r), MN-major: box {64 (r), 64 (n)}
+      if (!encode_map_bf16(&pr.tmB, s.Pbf, s.r, s.n, s.r, 64, 64)) return cudaErrorInvalidValue;
+      // side operands: M^Q and V^Q (m x r int8)
+      if (!encode_map_i8_side(&pr.tmS[0], s.Mq, s.r, s.m, s.ld_mom)) return cudaErrorInvalidValue;
+      if (!encode_map_i8_side(&pr.tmS[1], s.Vq, s.r, s.m, s.ld_mom)) return cudaErrorInvalidValue;
+    } else {
       // A = P~^T (M = r, K = m), MN-major over P~ (m x r): box {64 (r), 64 (m)}
       if (!encode_map_bf16(&pr.tmA, s.Pbf, s.r, s.m, s.r, 64, 64)) return cudaErrorInvalidValue;
       // B = G (K = m, N = n), MN-major: box {64 (n), 64 (m)}
@@ -801,40 +815,64 @@ static cudaError_t launch_gemms_for(const StepProblem* probs, int cnt, cudaStrea
       // side operands: M^Q and V^Q (r x n int8, leading dimension ld_mom)
       if (!encode_map_i8_side(&pr.tmS[0], s.Mq, s.n, s.r, s.ld_mom)) return cudaErrorInvalidValue;
       if (!encode_map_i8_side(&pr.tmS[1], s.Vq, s.n, s.r, s.ld_mom)) return cudaErrorInvalidValue;
-      pr.status = s.status;
-      pr.epi = AdamEpi::Args{s.Mq, s.Vq, s.sM, s.sV, s.Nbuf, s.ld_mom, s.ldN, s.nblk,
-                             s.beta1, s.beta2, s.om1, s.om2, s.c1, s.c2, s.eps};
-      add_problem(p1, s.r, s.n, s.m);
     }
-    e = launch_gemm_pair<AdamEpi, true>(p1, stream, QG_KERNEL_PROJECT_ADAM, fl1, by1);
-    if (e != cudaSuccess) return e;
+    pr.status = s.status;
+    pr.epi = AdamEpi::Args{s.Mq, s.Vq, s.sM, s.sV, s.Nbuf, s.ld_mom, s.ldN, s.nblk,
+                           s.beta1, s.beta2, s.om1, s.om2, s.c1, s.c2, s.eps};
+    if (kRight)
+      add_problem(p1, s.m, s.r, s.n);
+    else
+      add_problem(p1, s.r, s.n, s.m);
+  }
+  e = launch_gemm_pair<AdamEpi, !kRight>(p1, stream, QG_KERNEL_PROJECT_ADAM, fl1, by1);
+  if (e != cudaSuccess) return e;
 
-    GemmParams<StochRoundEpi> p2;
-    memset(&p2, 0, sizeof(p2));
-    // The batch's matrices in reverse order: the last N written by a2+a3 (and
-    // its P~, read last there) is the likeliest still in L2.
-    for (int ii = 0; ii < cnt; ++ii) {
+  GemmParams<StochRoundEpi> p2;
+  memset(&p2, 0, sizeof(p2));
+  // The batch's matrices in reverse order: the last N written by a2+a3 (and
+  // its P~, read last there) is the likeliest still in L2.
+  for (int jj = 0; jj < cnt; ++jj) {
 #if QG_SR_REVERSE
-      const int i = cnt - 1 - ii;
+    const int ii = cnt - 1 - jj;
 #else
-      const int i = ii;
+    const int ii = jj;
 #endif
-      const StepProblem& s = probs[i];
-      GemmProblem<StochRoundEpi>& pr = p2.prob[p2.nprob];
+    const StepProblem& s = probs[idx[ii]];
+    GemmProblem<StochRoundEpi>& pr = p2.prob[p2.nprob];
+    if (kRight) {
+      // A = N (M = m, K = r), K-major: box {64 (r), 128 (m)}
+      if (!encode_map_bf16(&pr.tmA, s.Nbuf, s.r, s.m, s.ldN, 64, 128)) return cudaErrorInvalidValue;
+      // B = P~^T (K = r, N = n), K-major over P~ (n x r): box {64 (r), 128 (n)}
+      if (!encode_map_bf16(&pr.tmB, s.Pbf, s.r, s.n, s.r, 64, 128)) return cudaErrorInvalidValue;
+    } else {
       // A = P~ (M = m, K = r), K-major: box {64 (r), 128 (m)}
       if (!encode_map_bf16(&pr.tmA, s.Pbf, s.r, s.m, s.r, 64, 128)) return cudaErrorInvalidValue;
       // B = N (K = r, N = n), MN-major: box {64 (n), 64 (r)}
       if (!encode_map_bf16(&pr.tmB, s.Nbuf, s.n, s.r, s.ldN, 64, 64)) return cudaErrorInvalidValue;
-      // side operand: W^Q (m x n int8, leading dimension ldw)
-      if (!encode_map_i8_side(&pr.tmS[0], s.W, s.n, s.m, s.ldw)) return cudaErrorInvalidValue;
-      pr.status = s.status;
-      pr.epi = StochRoundEpi::Args{s.W, s.sW, s.ldw, s.alpha, s.t, s.layer_id,
-                                   PhiloxKey{static_cast<uint32_t>(s.seed), static_cast<uint32_t>(s.seed >> 32)},
-                                   (s.n % 256) == 0 ? 1 : 0};
-      add_problem(p2, s.m, s.n, s.r);
     }
-    e = launch_gemm_pair<StochRoundEpi, false>(p2, stream, QG_KERNEL_BACKPROJECT_SR, fl2, by2);
+    // side operand: W^Q (m x n int8, leading dimension ldw)
+    if (!encode_map_i8_side(&pr.tmS[0], s.W, s.n, s.m, s.ldw)) return cudaErrorInvalidValue;
+    pr.status = s.status;
+    pr.epi = StochRoundEpi::Args{s.W, s.sW, s.ldw, s.alpha, s.t, s.layer_id,
+                                 PhiloxKey{static_cast<uint32_t>(s.seed), static_cast<uint32_t>(s.seed >> 32)},
+                                 (s.n % 256) == 0 ? 1 : 0};
+    add_problem(p2, s.m, s.n, s.r);
   }
+  return launch_gemm_pair<StochRoundEpi, false, !kRight>(p2, stream, QG_KERNEL_BACKPROJECT_SR, fl2, by2);
+}
+
+// The batch's left-side problems, then its right-side ones.
+static cudaError_t launch_gemms_for(const StepProblem* probs, int cnt, cudaStream_t stream) {
+  int left[kMaxProblems], right[kMaxProblems], nl = 0, nr = 0;
+  for (int i = 0; i < cnt; ++i) {
+    if (probs[i].side)
+      right[nr++] = i;
+    else
+      left[nl++] = i;
+  }
+  cudaError_t e = cudaSuccess;
+  if (nl > 0 && (e = launch_gemms_side<false>(probs, left, nl, stream)) != cudaSuccess) return e;
+  if (nr > 0) e = launch_gemms_side<true>(probs, right, nr, stream);
   return e;
 }
 

@@ -20,7 +20,7 @@ def stream():
 def lib_config(oc: O.Config):
     return qg.config(oc.m, oc.n, oc.r, beta1=oc.beta1, beta2=oc.beta2, eps=oc.eps, lr=oc.lr, alpha=oc.alpha,
                      gamma=oc.gamma, delta0=oc.delta0, oversample=oc.oversample, power_iters=oc.power_iters,
-                     seed=oc.seed, layer_id=oc.layer_id, mom_refresh=oc.mom_refresh)
+                     seed=oc.seed, layer_id=oc.layer_id, mom_refresh=oc.mom_refresh, proj_side=oc.proj_side)
 
 
 def upload_gradient(G_bits: np.ndarray, device="cuda"):
@@ -81,26 +81,28 @@ class GpuLayer:
         return self.W[:, : self.oc.n].cpu().numpy()
 
     def moments(self):
-        r, n = self.oc.r, self.oc.n
+        rows, cols = self.v.mom_rows, self.v.mom_cols
         ld, nb = self.v.ld_mom, self.v.nblk
-        Mq = self.region(self.v.Mq, r * ld).view(torch.int8).view(r, ld)[:, :n].cpu().numpy()
-        Vq = self.region(self.v.Vq, r * ld).view(torch.int8).view(r, ld)[:, :n].cpu().numpy()
-        sM = self.region(self.v.sM, r * nb * 4).view(torch.float32).view(r, nb).cpu().numpy()
-        sV = self.region(self.v.sV, r * nb * 4).view(torch.float32).view(r, nb).cpu().numpy()
+        Mq = self.region(self.v.Mq, rows * ld).view(torch.int8).view(rows, ld)[:, :cols].cpu().numpy()
+        Vq = self.region(self.v.Vq, rows * ld).view(torch.int8).view(rows, ld)[:, :cols].cpu().numpy()
+        sM = self.region(self.v.sM, rows * nb * 4).view(torch.float32).view(rows, nb).cpu().numpy()
+        sV = self.region(self.v.sV, rows * nb * 4).view(torch.float32).view(rows, nb).cpu().numpy()
         return Mq, sM, Vq, sV
 
     def projection(self):
-        mr = self.oc.m * self.oc.r
+        mr = self.v.p_rows * self.oc.r
         Pq = self.region(self.v.Pq, (mr + 1) // 2).cpu().numpy()
         sP = self.region(self.v.sP, -(-mr // 64) * 4).view(torch.float32).cpu().numpy()
         return Pq, sP
 
     def scratch_N(self):
-        """N (r x n bf16 bits) from the step workspace (layout: P~ then N, 256-aligned)."""
-        m, n, r = self.oc.m, self.oc.n, self.oc.r
-        off = round_up(m * r * 2, 256)
-        ldN = round_up(n, 32)
-        return self.ws[off: off + r * ldN * 2].view(torch.int16).view(r, ldN)[:, :n].cpu().numpy().view(np.uint16)
+        """N (R's shape, bf16 bits) from the step workspace (layout: P~ then N, 256-aligned)."""
+        p, r = self.v.p_rows, self.oc.r
+        rows, cols = self.v.mom_rows, self.v.mom_cols
+        off = round_up(p * r * 2, 256)
+        ldN = round_up(cols, 32)
+        return (self.ws[off: off + rows * ldN * 2].view(torch.int16).view(rows, ldN)[:, :cols].cpu().numpy()
+                .view(np.uint16))
 
     def refresh(self, G_dev: torch.Tensor, ldg: int, force=0):
         """qg_refresh; returns (info, float32 projection from the workspace)."""
@@ -111,8 +113,8 @@ class GpuLayer:
         qg.check(qg.qg_refresh(self.h, G_dev.data_ptr(), ldg, force, self.rws.data_ptr(), self.rws.numel(),
                                byref(info), stream()), "qg_refresh")
         torch.cuda.synchronize()
-        m, r = self.oc.m, self.oc.r
-        P = self.rws[: m * r * 4].view(torch.float32).view(m, r).cpu().numpy().copy()
+        p, r = self.v.p_rows, self.oc.r
+        P = self.rws[: p * r * 4].view(torch.float32).view(p, r).cpu().numpy().copy()
         return info, P
 
     def status(self):

@@ -68,8 +68,8 @@ def principal_cosines(A, B):
     return np.sort(np.cos(scipy.linalg.subspace_angles(np.asarray(A, np.float64), np.asarray(B, np.float64))))[::-1]
 
 
-def _refresh_pair(m, n, r, G_vals, G_bits, seed=3, layer_id=2):
-    oc = O.Config(m=m, n=n, r=r, seed=seed, layer_id=layer_id)
+def _refresh_pair(m, n, r, G_vals, G_bits, seed=3, layer_id=2, side=0):
+    oc = O.Config(m=m, n=n, r=r, seed=seed, layer_id=layer_id, proj_side=side)
     ost = O.LayerState.create(oc, np.zeros((m, n), np.int8), np.ones(-(-m * n // 256), np.float32))
     oinfo = O.refresh(ost, G_vals, force=True)
     gl = GpuLayer(oc, np.zeros((m, n), np.int8), np.ones(-(-m * n // 256), np.float32))
@@ -78,10 +78,11 @@ def _refresh_pair(m, n, r, G_vals, G_bits, seed=3, layer_id=2):
     return ost, oinfo, gl, info, Pg
 
 
-@pytest.mark.parametrize("m,n,r", [(256, 256, 32), (300, 250, 32), (1376, 512, 128), (512, 1376, 96)])
-def test_refresh_gap_input_matches_oracle_subspace(m, n, r):
+@pytest.mark.parametrize("m,n,r,side", [(256, 256, 32, 0), (300, 250, 32, 0), (1376, 512, 128, 0),
+                                        (512, 1376, 96, 0), (300, 250, 32, 1), (1376, 512, 128, 1)])
+def test_refresh_gap_input_matches_oracle_subspace(m, n, r, side):
     G, Gb = synth.gap_gradient(m, n, r, seed=m + n)
-    ost, oinfo, gl, info, Pg = _refresh_pair(m, n, r, G, Gb)
+    ost, oinfo, gl, info, Pg = _refresh_pair(m, n, r, G, Gb, side=side)
     assert info.refreshed == 1 and info.has_cossim == 0 and info.n_refresh == 1
     Po = oinfo["P"]
     cos = principal_cosines(Pg, Po)
@@ -102,7 +103,7 @@ def test_refresh_gap_input_matches_oracle_subspace(m, n, r):
     # the INT4 projection installed in the layer is the quantization of that P
     Pq, sP = gl.projection()
     ref_codes, ref_s = O.quant_int4_groups(Po.astype(np.float32))
-    got_codes = O.unpack_int4(Pq, m * r)
+    got_codes = O.unpack_int4(Pq, Po.shape[0] * r)
     assert (got_codes == ref_codes).mean() > 0.98
     np.testing.assert_allclose(sP, ref_s, rtol=2e-2)
     assert gl.status() == qg.QG_OK
@@ -173,19 +174,19 @@ def test_schedule_follows_oracle_over_refreshes():
 
 # ---------------------------------------------------------------- moments at a refresh
 
-@pytest.mark.parametrize("policy", [1, 2])
-def test_refresh_moment_policy_matches_oracle(policy):
+@pytest.mark.parametrize("policy,side", [(1, 0), (2, 0), (2, 1)])
+def test_refresh_moment_policy_matches_oracle(policy, side):
     # a starting projection and three steps give non-zero moments; a forced
     # refresh then replaces P.  The oracle applies the same moment map to the
     # GPU's own moments and projections (teacher-forced), so only the map is
     # compared: reset bit-exact, rotation within the step's moment bar
-    m, n, r = 300, 700, 64
-    oc = O.Config(m=m, n=n, r=r, seed=7, layer_id=3, mom_refresh=policy)
+    m, n, r = (300, 700, 64) if side == 0 else (700, 300, 64)
+    oc = O.Config(m=m, n=n, r=r, seed=7, layer_id=3, mom_refresh=policy, proj_side=side)
     Wq, sW = synth.weight_codes(m, n, 7), synth.weight_scales(m, n, seed=7)
     gen = synth.lowrank_gradient(m, n, rank=32, seed=7)
     gl = GpuLayer(oc, Wq, sW)
     G0, _ = gen.draw(0)
-    codes, sP = O.quant_int4_groups(O.exact_topr(G0, r)[0].astype(np.float32))
+    codes, sP = O.quant_int4_groups(O.exact_topr(G0 if side == 0 else G0.T, r)[0].astype(np.float32))
     Pq = O.pack_int4(codes)
     gl.set_projection(Pq, sP)
     for t in range(3):
@@ -202,7 +203,8 @@ def test_refresh_moment_policy_matches_oracle(policy):
     Pq_new, sP_new = gl.projection()
     st = O.LayerState.create(oc, Wq, sW)
     st.Mq, st.sM, st.Vq, st.sV = Mq.copy(), sM.copy(), Vq.copy(), sV.copy()
-    O.refresh_moments(st, O.dequant_int4_f32(Pq_new, sP_new, m, r), O.dequant_int4_f32(Pq, sP, m, r))
+    p = m if side == 0 else n
+    O.refresh_moments(st, O.dequant_int4_f32(Pq_new, sP_new, p, r), O.dequant_int4_f32(Pq, sP, p, r))
     gMq, gsM, gVq, gsV = gl.moments()
     if policy == 1:
         assert not gMq.any() and not gVq.any() and not gsM.any() and not gsV.any()

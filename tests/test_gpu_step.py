@@ -88,14 +88,14 @@ def test_gemm_core_tcgen05(M, N, K, a_trans, b_trans):
 
 # ---------------------------------------------------------------- step parity
 
-def make_layer(m, n, r, seed=0, rank=None, s0=1e-2, decay=0.8, sigma=1e-4, layer_id=0):
-    oc = O.Config(m=m, n=n, r=r, seed=seed, layer_id=layer_id)
+def make_layer(m, n, r, seed=0, rank=None, s0=1e-2, decay=0.8, sigma=1e-4, layer_id=0, side=0):
+    oc = O.Config(m=m, n=n, r=r, seed=seed, layer_id=layer_id, proj_side=side)
     Wq = synth.weight_codes(m, n, seed)
     sW = synth.weight_scales(m, n, seed=seed)
     gen = synth.lowrank_gradient(m, n, rank=rank or min(256, m, n), s0=s0, decay=decay, sigma=sigma, seed=seed)
     ost = O.LayerState.create(oc, Wq, sW)
     G0, _ = gen.draw(0)
-    P, _ = O.exact_topr(G0, r)
+    P, _ = O.exact_topr(G0 if side == 0 else G0.T, r)
     O.set_projection(ost, P)
     gl = GpuLayer(oc, Wq, sW)
     gl.set_projection(ost.Pq, ost.sP)
@@ -233,3 +233,50 @@ def test_nonfinite_gradient_sets_status():
     gl.step(dG, ldg)
     assert gl.status() == qg.QG_ENONFINITE
     assert gl.status() == qg.QG_OK  # cleared by the read
+
+
+# ---------------------------------------------------------------- right-side projection (P n x r)
+
+@pytest.mark.parametrize("m,n,r,steps", [
+    (700, 300, 64, 3),       # m > n, ragged tails
+    (1376, 512, 128, 3),     # the LLaMA-60M down projection's shape
+    (300, 700, 64, 2),       # the right side on a wide matrix as well
+])
+def test_step_parity_right_side(m, n, r, steps):
+    ost, gl, gen = make_layer(m, n, r, seed=m + n + r, layer_id=4, side=1)
+    assert gl.v.p_rows == n and gl.v.mom_rows == m and gl.v.mom_cols == r
+    for t in range(steps):
+        G, Gb = gen.draw(t)
+        dG, ldg = upload_gradient(Gb)
+        gl.step(dG, ldg)
+        inter = O.step(ost, G)
+        if t == 0:
+            assert float((gl.scratch_N() != O.bf16_bits(inter["N"])).mean()) <= 1e-3
+        compare_state(ost, gl, f"right side, step {t + 1}")
+    assert gl.status() == qg.QG_OK
+
+
+def test_step_batch_mixed_sides_equals_single_steps():
+    shapes = [(700, 300, 64, 1), (256, 256, 32, 0), (1376, 512, 128, 1), (512, 1376, 128, 0), (300, 700, 64, 1),
+              (512, 512, 64, 0), (640, 1365, 96, 0), (1376, 512, 64, 1), (256, 384, 32, 1)]
+    singles, batched, grads = [], [], []
+    for i, (m, n, r, side) in enumerate(shapes):
+        _, gl1, gen = make_layer(m, n, r, seed=40 + i, layer_id=i, side=side)
+        _, gl2, _ = make_layer(m, n, r, seed=40 + i, layer_id=i, side=side)
+        singles.append(gl1)
+        batched.append(gl2)
+        grads.append(upload_gradient(gen.draw(0)[1]))
+    for gl, (dG, ldg) in zip(singles, grads):
+        gl.step(dG, ldg)
+    cfgs = [gl.cfg for gl in batched]
+    arr = (qg.POINTER(qg.qg_config) * len(cfgs))(*[qg.ctypes.pointer(c) for c in cfgs])
+    wsb = qg.qg_step_batch_workspace_bytes(arr, len(cfgs))
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    hs = (c_void_p * len(batched))(*[gl.h.value for gl in batched])
+    gs = (c_void_p * len(batched))(*[g.data_ptr() for g, _ in grads])
+    lds = (qg.c_int64 * len(batched))(*[ld for _, ld in grads])
+    qg.check(qg.qg_step_batch(hs, gs, lds, len(batched), ws.data_ptr(), wsb, stream()))
+    for a, b in zip(singles, batched):
+        np.testing.assert_array_equal(a.weights(), b.weights())
+        for x, y in zip(a.moments(), b.moments()):
+            np.testing.assert_array_equal(x, y)
