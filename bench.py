@@ -246,11 +246,15 @@ class Stack:
         R = spec["rank"]
         self.rank_r = R
         lid = 0
+        # QG_BENCH_SIDE=right-tall projects matrices with m > n on the right
+        # (P n x r), as GaLore does; the default projects every matrix on the left
+        right_tall = os.environ.get("QG_BENCH_SIDE") == "right-tall"
         for li, shapes in enumerate(stack_shapes(layers, spec["hidden"], spec["inter"])):
             group = []
             for (m, n) in shapes:
                 seed = matrix_seed(rank, lid)
-                c = qg.config(m, n, R, seed=seed, layer_id=lid)
+                side = 1 if (right_tall and m > n) else 0
+                c = qg.config(m, n, R, seed=seed, layer_id=lid, proj_side=side)
                 ldw = -(-n // 16) * 16
                 W = synth.device_weight_codes(m, n, ldw, seed, device)
                 sW = synth.device_weight_scales(m, n, seed, device)
@@ -262,15 +266,16 @@ class Stack:
                 # starting projection: an orthonormal basis quantized to INT4 on the device
                 g = torch.Generator(device=device)
                 g.manual_seed(seed + 17)
-                P = torch.linalg.qr(torch.randn(m, R, generator=g, device=device))[0].contiguous()
-                Pq = torch.empty((m * R + 1) // 2, dtype=torch.uint8, device=device)
-                sP = torch.empty(-(-m * R // 64), dtype=torch.float32, device=device)
-                qg.check(qg.qg_quantize_projection(P.data_ptr(), R, m, R, Pq.data_ptr(), sP.data_ptr(),
+                pr = n if side else m
+                P = torch.linalg.qr(torch.randn(pr, R, generator=g, device=device))[0].contiguous()
+                Pq = torch.empty((pr * R + 1) // 2, dtype=torch.uint8, device=device)
+                sP = torch.empty(-(-pr * R // 64), dtype=torch.float32, device=device)
+                qg.check(qg.qg_quantize_projection(P.data_ptr(), R, pr, R, Pq.data_ptr(), sP.data_ptr(),
                                                    stream))
                 qg.check(qg.qg_layer_set_projection(h, Pq.data_ptr(), sP.data_ptr(), 0, stream))
                 torch.cuda.synchronize()
                 del P, Pq, sP
-                group.append(dict(cfg=c, h=h, W=W, sW=sW, G=G, ldg=G.shape[1], state=state, m=m, n=n))
+                group.append(dict(cfg=c, h=h, W=W, sW=sW, G=G, ldg=G.shape[1], state=state, m=m, n=n, side=side))
                 lid += 1
             self.layers.append(group)
         # the step: one batched call for all matrices (batches of 8 on two lanes
@@ -297,7 +302,7 @@ class Stack:
         self.calls = self.calls_layer if self.per_layer_only else calls_of(whole)
         self.weights = sum(e["m"] * e["n"] for group in self.layers for e in group)
         self.flops = sum(4.0 * e["m"] * e["n"] * R for group in self.layers for e in group)
-        self.alg_bytes = sum(alg_bytes(e["m"], e["n"], R) for group in self.layers for e in group)
+        self.alg_bytes = sum(alg_bytes(e["m"], e["n"], R, e["side"]) for group in self.layers for e in group)
         self.grad_bytes = sum(e["G"].numel() * 2 for group in self.layers for e in group)
 
     def step(self, stream, per_layer=False):
@@ -335,11 +340,14 @@ def whole_job_rate(units_per_rank, world, ms):
     return world * units_per_rank / (ms / 1000.0)
 
 
-def alg_bytes(m, n, r):
+def alg_bytes(m, n, r, side=0):
     """Algorithmic HBM bytes of one matrix step: G, W read and written, W scales,
-    INT4 P and scales, moments read and written, their scales."""
-    nb = -(-n // 256)
-    return 2 * m * n + 2 * m * n + 4 * math.ceil(m * n / 256) + m * r / 2 + 4 * m * r / 64 + 4 * r * n + 16 * r * nb
+    INT4 P and scales, moments read and written, their scales.  P is m x r and
+    the moments r x n (left projection), or n x r and m x r (right)."""
+    p_rows, rows, cols = (n, m, r) if side else (m, r, n)
+    nb = -(-cols // 256)
+    return (2 * m * n + 2 * m * n + 4 * math.ceil(m * n / 256) + p_rows * r / 2 + 4 * p_rows * r / 64
+            + 4 * rows * cols + 16 * rows * nb)
 
 
 def run_ours(args, rank, world, local_rank):
