@@ -244,6 +244,7 @@ class Config:
     layer_id: int = 0
     mom_refresh: int = 0  # moments at a refresh: 0 keep, 1 reset, 2 rotate (see refresh_moments)
     proj_side: int = 0    # 0: P m x r, R = P^T G (the default reading); 1: P n x r, R = G P
+    w_rescale: int = 0    # 0: updates saturate at +-127 (default); 1: a group that would leave the grid is re-scaled
 
     def f32(self, name):
         return F32(getattr(self, name))
@@ -374,7 +375,8 @@ def stochastic_round_update(Wq, sW, U, cfg: Config, t: int, u16=None):
 
     [QG-quant] asks only that xi be an unbiased stochastic rounding; the form is
     a reading.  The weight scale is one float32 per 256 consecutive elements of
-    the row-major m x n array (logical index), fixed after initialisation.  The
+    the row-major m x n array (logical index), fixed after initialisation (the
+    re-scaling variant, stochastic_round_rescale, lets it grow instead).  The
     update is carried in fixed point with 16 fraction bits:
       c'_g = (alpha / s_g) * 2^16   (IEEE float32 division, exact scaling; a zero
                                      scale gives c'_g = 0 and freezes its group)
@@ -401,6 +403,52 @@ def stochastic_round_update(Wq, sW, U, cfg: Config, t: int, u16=None):
     r = (K + np.asarray(u16, np.int64)) >> 16          # floor division by 2^16
     out = np.clip(Wq.astype(np.int64) + r, -INT8_QMAX, INT8_QMAX)
     return np.where(nan, Wq, out).astype(np.int8)
+
+
+W_RESCALE_LIMIT = INT8_QMAX * 65536  # 127 in units of 2^-16 code
+
+
+def stochastic_round_rescale(Wq, sW, U, cfg: Config, t: int, u16=None):
+    """Step a5 of the re-scaling variant: a weight group whose updated values
+    would leave the INT8 grid gets a larger scale instead of saturating.
+
+    With X and K = ceil(X) as in stochastic_round_update, each element's value
+    in units of 2^-16 code is the integer T = q * 2^16 + K (T = q * 2^16 where X
+    is NaN).  Per group g of 256 consecutive elements, A = max |T|:
+      A <= 127 * 2^16: the codes are those of stochastic_round_update (no
+                       element can reach the clamp) and the scale is kept;
+      otherwise:       rho = (127 * 2^16) / A and s'_g = s_g / rho (IEEE float32
+                       divisions); Z = fl(T) * rho (float32, fl the nearest
+                       float), K' = ceil(Z), and the code is
+                       clamp(floor((K' + d) / 2^16), -127, 127) with the same
+                       draw d.  E[code' s'] = T 2^-16 s: still unbiased.
+    Returns (codes, scales)."""
+    m, n = Wq.shape
+    e = np.arange(m * n, dtype=np.int64).reshape(m, n)
+    sW = np.asarray(sW, np.float32)
+    c = np.where(sW > 0, F32(cfg.alpha) / np.where(sW > 0, sW, F32(1)), F32(0)).astype(np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        cp = (c * F32(65536.0)).astype(np.float32)
+        X = (np.asarray(U, np.float32) * cp[e // cfg.w_group]).astype(np.float32)
+        nan = np.isnan(X)
+        K = np.ceil(np.clip(np.where(nan, F32(0), X), F32(-2.0 ** 30), F32(2.0 ** 30))).astype(np.int64)
+    if u16 is None:
+        u16 = sr_uniform16(m, n, cfg.seed, t, cfg.layer_id)
+    d = np.asarray(u16, np.int64)
+    T = Wq.astype(np.int64) * 65536 + np.where(nan, 0, K)
+    g = e.ravel() // cfg.w_group
+    flatT, flatd = T.ravel(), d.ravel()
+    A = np.zeros(len(sW), np.int64)
+    np.maximum.at(A, g, np.abs(flatT))                  # per group max |T|
+    grow = (A > W_RESCALE_LIMIT) & (sW > 0)
+    rho = np.ones(len(sW), np.float32)
+    rho[grow] = F32(W_RESCALE_LIMIT) / A[grow].astype(np.float32)
+    s_new = sW.copy()
+    s_new[grow] = (sW[grow] / rho[grow]).astype(np.float32)
+    Z = (flatT.astype(np.float32) * rho[g]).astype(np.float32)
+    Kp = np.where(grow[g], np.ceil(Z).astype(np.int64), flatT)
+    out = np.clip((Kp + flatd) >> 16, -INT8_QMAX, INT8_QMAX)
+    return out.reshape(m, n).astype(np.int8), s_new
 
 
 @dataclass
@@ -444,7 +492,10 @@ def step(st: LayerState, G) -> dict:
     R = project(Pb, G) if cfg.proj_side == 0 else project_right(G, Pb)
     N, st.Mq, st.sM, st.Vq, st.sV = lowrank_adam_int8(R, st.Mq, st.sM, st.Vq, st.sV, cfg, st.t)
     U = backproject(Pb, N) if cfg.proj_side == 0 else backproject_right(N, Pb)
-    st.Wq = stochastic_round_update(st.Wq, st.sW, U, cfg, st.t)
+    if cfg.w_rescale:
+        st.Wq, st.sW = stochastic_round_rescale(st.Wq, st.sW, U, cfg, st.t)
+    else:
+        st.Wq = stochastic_round_update(st.Wq, st.sW, U, cfg, st.t)
     return dict(P=Pb, R=R, N=N, U=U)
 
 

@@ -370,6 +370,116 @@ def test_sr_small_updates_keep_their_mean():
     assert abs(out.mean() - 1e-3) < 5 * np.sqrt(1e-3 / (m * n)) + 2 ** -16
 
 
+# ---------------------------------------------------------------- re-scaling instead of saturating
+
+def test_rescale_equals_saturating_inside_the_grid():
+    # nothing reaches +-127: codes are those of the saturating form, scales unchanged
+    rng = np.random.default_rng(21)
+    W = rng.integers(-100, 101, size=(16, 512)).astype(np.int8)
+    sW = rng.uniform(0.005, 0.02, 32).astype(np.float32)
+    U = (rng.standard_normal((16, 512)) * 0.05).astype(np.float32)
+    U[3, 7] = np.nan
+    cfg = O.Config(m=16, n=512, r=1, alpha=0.5, seed=3)
+    q, s2 = O.stochastic_round_rescale(W, sW, U, cfg, 4)
+    np.testing.assert_array_equal(q, O.stochastic_round_update(W, sW, U, cfg, 4))
+    np.testing.assert_array_equal(s2, sW)
+    assert q[3, 7] == W[3, 7]
+
+
+@pytest.mark.parametrize("q0,X", [(127, 1.0), (120, 8 * 65536 + 0.5), (100, 2.0 ** 29), (-127, -1.0),
+                                  (-90, -100 * 65536 - 12345.25), (0, 2.0 ** 31)])
+def test_rescale_exhaustive_over_the_draw_space(q0, X):
+    # alpha = 1, s_g = 2^16: c' = 1, so every element of the 256 x 256 array has the
+    # same value T = q0 2^16 + ceil(X) (X clipped to 2^30) in units of 2^-16 code,
+    # outside the grid, and meets each 16-bit draw once.  Every group is re-scaled
+    # to the same s', so the codes' sum over the draws is their exact mean: the
+    # value q0 s + X 2^-16 s must come back as sum / 2^16 * s' up to float32
+    # rounding (4 roundings) and the 2^-16 draw grid.  Every code lands on the top
+    # of the new grid (126 or 127 in magnitude) and s' = s |T| / (127 2^16).
+    W = np.full((256, 256), q0, np.int8)
+    sW = np.full(256, 65536.0, np.float32)
+    U = np.full((256, 256), X, np.float32)
+    cfg = O.Config(m=256, n=256, r=1, alpha=1.0)
+    q, s2 = O.stochastic_round_rescale(W, sW, U, cfg, 1, u16=np.arange(65536, dtype=np.uint32).reshape(256, 256))
+    T = q0 * 65536 + math.ceil(max(-2.0 ** 30, min(2.0 ** 30, float(np.float32(X)))))
+    assert abs(T) > 127 * 65536
+    assert np.all(s2 == s2[0]) and s2[0] > sW[0]
+    assert abs(float(s2[0]) - 65536.0 * abs(T) / (127 * 65536)) <= 3e-7 * float(s2[0])
+    assert set(np.abs(np.unique(q)).tolist()) <= {126, 127}
+    mean_value = int(q.astype(np.int64).sum()) / 65536.0 * float(s2[0])
+    target = T / 65536.0 * 65536.0
+    assert abs(mean_value - target) <= 5e-7 * abs(target) + 2.0 ** -16 * float(s2[0])
+
+
+def test_rescale_keeps_each_element_unbiased():
+    # one outlier per group pushes its group off the grid; every other element of
+    # the group must keep its value q s + alpha U on average over the draws
+    m, n, draws = 4, 256, 1500
+    rng = np.random.default_rng(5)
+    W = rng.integers(-60, 61, size=(m, n)).astype(np.int8)
+    sW = np.full(m, 0.01, np.float32)
+    U = (rng.standard_normal((m, n)) * 0.2).astype(np.float32)
+    U[:, 17] = 3.0                     # q + 300 codes: far off the grid
+    cfg = O.Config(m=m, n=n, r=1, alpha=1.0, seed=9)
+    acc = np.zeros((m, n))
+    acc2 = np.zeros((m, n))
+    for t in range(draws):
+        q, s2 = O.stochastic_round_rescale(W, sW, U, cfg, t)
+        v = q.astype(np.float64) * s2[:, None]
+        acc += v
+        acc2 += v * v
+    assert np.all(s2 > sW)
+    mean = acc / draws
+    sd = np.sqrt(np.maximum(acc2 / draws - mean ** 2, 0) / draws)
+    expect = W.astype(np.float64) * np.float64(sW[:, None]) + np.float64(U)
+    use = sd > 1e-4
+    z = ((mean - expect) / np.where(use, sd, 1))[use]
+    assert z.size > 0.9 * m * n
+    assert abs(z.mean()) < 5 / math.sqrt(z.size)
+    assert (z ** 2).mean() < 1.3
+    # a saturating update loses the outlier's value; the re-scaled one keeps it
+    assert np.all(np.abs(mean[:, 17] - expect[:, 17]) < 0.02 * np.abs(expect[:, 17]))
+
+
+def test_rescale_zero_scale_nan_and_mixed_groups():
+    # group 0: zero scale (frozen); group 1: leaves the grid; group 2: stays inside
+    W = np.zeros((3, 256), np.int8)
+    W[1, 0], W[2, 0] = 126, 5
+    sW = np.array([0.0, 1.0, 1.0], np.float32)
+    U = np.zeros((3, 256), np.float32)
+    U[0] = 50.0
+    U[1, 0], U[1, 1] = 3.0, np.nan
+    U[2, 1] = 0.5
+    cfg = O.Config(m=3, n=256, r=1, alpha=1.0)
+    q, s2 = O.stochastic_round_rescale(W, sW, U, cfg, 2, u16=np.full((3, 256), 40000, np.uint32))
+    np.testing.assert_array_equal(q[0], W[0])
+    assert s2[0] == 0 and s2[2] == 1
+    # group 1: T_max = 129 2^16, rho = 127/129, s' = 129/127; the outlier lands on 127
+    assert s2[1] == np.float32(np.float32(1.0) / np.float32(np.float32(127 * 65536) / np.float32(129 * 65536)))
+    assert q[1, 0] == 127 and np.all(q[1, 1:] == 0)   # zeros (and the NaN's zero) stay zero
+    np.testing.assert_array_equal(q[2], O.stochastic_round_update(W[2:], sW[2:], U[2:], O.Config(m=1, n=256, r=1, alpha=1.0), 2,
+                                                                  u16=np.full((1, 256), 40000, np.uint32))[0])
+
+
+def test_rescale_step_with_small_alpha_equals_saturating_step():
+    import synth
+    m, n, r = 64, 256, 16
+    base = dict(m=m, n=n, r=r, alpha=0.25, seed=4)
+    out = []
+    for wr in (0, 1):
+        st = O.LayerState.create(O.Config(**base, w_rescale=wr), np.clip(synth.weight_codes(m, n, 4), -100, 100),
+                                 synth.weight_scales(m, n, seed=4))
+        O.set_projection(st, synth.orthonormal(m, r, 4))
+        gen = synth.lowrank_gradient(m, n, rank=8, seed=4)
+        for t in range(3):
+            O.step(st, gen.draw(t)[0])
+        out.append((st.Wq.copy(), st.sW.copy()))
+    sat = np.abs(out[0][0]) == 127
+    assert not sat.any()
+    np.testing.assert_array_equal(out[0][0], out[1][0])
+    np.testing.assert_array_equal(out[0][1], out[1][1])
+
+
 # ---------------------------------------------------------------- composed step
 
 def _small_layer(m=64, n=96, r=32, seed=0, alpha=0.25):
