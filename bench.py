@@ -249,12 +249,16 @@ class Stack:
         # QG_BENCH_SIDE=right-tall projects matrices with m > n on the right
         # (P n x r), as GaLore does; the default projects every matrix on the left
         right_tall = os.environ.get("QG_BENCH_SIDE") == "right-tall"
+        # QG_BENCH_W_RESCALE=1 lets a weight group that the update would carry off
+        # the INT8 grid grow its scale instead of saturating
+        w_rescale = 1 if os.environ.get("QG_BENCH_W_RESCALE") == "1" else 0
+        self.variant = ("-right-tall" if right_tall else "") + ("-wrescale" if w_rescale else "")
         for li, shapes in enumerate(stack_shapes(layers, spec["hidden"], spec["inter"])):
             group = []
             for (m, n) in shapes:
                 seed = matrix_seed(rank, lid)
                 side = 1 if (right_tall and m > n) else 0
-                c = qg.config(m, n, R, seed=seed, layer_id=lid, proj_side=side)
+                c = qg.config(m, n, R, seed=seed, layer_id=lid, proj_side=side, w_rescale=w_rescale)
                 ldw = -(-n // 16) * 16
                 W = synth.device_weight_codes(m, n, ldw, seed, device)
                 sW = synth.device_weight_scales(m, n, seed, device)
@@ -450,7 +454,8 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/f32/int8",
         "data": "synthetic (seeded low-rank-plus-noise bf16 gradients)",
-        "config": {"workload": f"{args.workload}-r{spec['rank']}" + ("" if layers == spec["layers"] else f"-{layers}l"),
+        "config": {"workload": f"{args.workload}-r{spec['rank']}" + ("" if layers == spec["layers"] else f"-{layers}l")
+                   + stack.variant,
                    "matrices": 7 * layers, "weights_per_gpu": stack.weights,
                    "rank": spec["rank"], "l2": "inputs larger than L2 (%.1f GB of gradients per step)"
                    % (stack.grad_bytes / 1e9) if flush is None else "L2 flushed between steps (each step timed alone)",

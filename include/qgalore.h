@@ -7,7 +7,8 @@
  * schedule" (paper section 3.1, Eq. (5)) and "INT4 projection and INT8
  * stochastic rounding" (paper section 3.2)):
  *
- *   per weight matrix W (m x n, INT8 codes with fixed float32 group scales)
+ *   per weight matrix W (m x n, INT8 codes with float32 group scales, fixed
+ *   unless w_rescale lets a group grow)
  *     a1  P~ = bf16(dequant(P^Q))             P^Q: m x r INT4, one scale / 64
  *     a2  R  = P~^T G                          G: m x n bf16 gradient
  *     a3  Adam on (M^Q, V^Q), r x n INT8 with per-row-block scales -> N (bf16)
@@ -77,6 +78,13 @@ typedef struct {
   int32_t proj_side;        /* which side is projected: 0 (default) P is m x r and R = P^T G (r x n);
                                1 P is n x r, R = G P (m x r) and U = N P^T, the projection taken
                                from the top-r right singular vectors of G */
+  int32_t w_rescale;        /* a weight group whose updated values would leave the INT8 grid: 0 (default)
+                               the codes saturate at +-127; 1 the group's scale grows to
+                               s' = s / rho, rho = (127 * 2^16) / max|T| with T = q * 2^16 + ceil(X)
+                               the values in units of 2^-16 code (X = U * alpha / s * 2^16), and the
+                               group is rounded stochastically again on the new grid
+                               (code = floor((ceil(fl(T) rho) + draw) / 2^16)) with the same draws;
+                               needs n % 256 == 0 (QG_ESHAPE otherwise) */
 } qg_config;
 
 typedef struct qg_layer qg_layer;
@@ -132,10 +140,12 @@ size_t qg_refresh_workspace_bytes(const qg_config* cfg);
  *   d_W     : m x ldw INT8 weight codes, 16-byte aligned, ldw >= n, ldw % 16 == 0;
  *             updated in place by qg_step.
  *   d_Wscale: ceil(m*n/256) float32 scales, group g covering logical elements
- *             [256 g, 256 g + 256) of the row-major m x n array; read only.
+ *             [256 g, 256 g + 256) of the row-major m x n array; read only,
+ *             except with cfg->w_rescale = 1, where qg_step enlarges in place
+ *             the scale of a group that the update would carry off the grid.
  * Returns QG_EINVAL / QG_ESHAPE / QG_EALIGN / QG_ESTATE on bad arguments. */
 qg_status qg_layer_init(qg_layer** out, const qg_config* cfg, void* d_state, size_t state_bytes,
-                        int8_t* d_W, int64_t ldw, const float* d_Wscale, void* stream);
+                        int8_t* d_W, int64_t ldw, float* d_Wscale, void* stream);
 qg_status qg_layer_destroy(qg_layer* layer);
 qg_status qg_layer_views_get(const qg_layer* layer, qg_layer_views* views);
 qg_status qg_layer_sched_get(const qg_layer* layer, qg_sched* sched);

@@ -30,7 +30,7 @@ class qg_config(Structure):
                 ("mom_block", c_int32), ("beta1", c_float), ("beta2", c_float), ("eps", c_float), ("lr", c_float),
                 ("alpha", c_float), ("gamma", c_float), ("delta0", c_int32), ("oversample", c_int32),
                 ("power_iters", c_int32), ("seed", c_uint64), ("layer_id", c_uint32), ("mom_refresh", c_int32),
-                ("proj_side", c_int32)]
+                ("proj_side", c_int32), ("w_rescale", c_int32)]
 
 
 class qg_layer_views(Structure):

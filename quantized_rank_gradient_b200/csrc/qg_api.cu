@@ -21,7 +21,7 @@ struct qg_layer {
   size_t state_bytes;
   int8_t* W;
   int64_t ldw;
-  const float* sW;
+  float* sW;
   qg_layer_views v;
   qg_sched sched;
 };
@@ -90,6 +90,8 @@ qg_status check_config(const qg_config* c) {
   if (!isfinite(c->gamma) || c->delta0 < 1 || c->oversample < 0 || c->power_iters < 0) return QG_EINVAL;
   if (c->mom_refresh < 0 || c->mom_refresh > 2) return QG_EINVAL;
   if (c->proj_side < 0 || c->proj_side > 1) return QG_EINVAL;
+  if (c->w_rescale < 0 || c->w_rescale > 1) return QG_EINVAL;
+  if (c->w_rescale && c->n % 256 != 0) return QG_ESHAPE;
   return QG_OK;
 }
 
@@ -118,6 +120,7 @@ void fill_step_problem(const qg_layer* L, const void* G, int64_t ldg, uint8_t* w
   s->n = c.n;
   s->r = c.r;
   s->side = c.proj_side;
+  s->w_rescale = c.w_rescale;
   const double b1 = static_cast<double>(c.beta1);
   const double b2 = static_cast<double>(c.beta2);
   s->beta1 = c.beta1;
@@ -207,7 +210,7 @@ size_t qg_refresh_workspace_bytes(const qg_config* cfg) {
 }
 
 qg_status qg_layer_init(qg_layer** out, const qg_config* cfg, void* d_state, size_t state_bytes, int8_t* d_W,
-                        int64_t ldw, const float* d_Wscale, void* stream) {
+                        int64_t ldw, float* d_Wscale, void* stream) {
   if (!out) return QG_EINVAL;
   *out = nullptr;
   qg_status st = check_config(cfg);

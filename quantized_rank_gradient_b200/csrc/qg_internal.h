@@ -20,12 +20,13 @@ struct StepProblem {
   int32_t nblk;
   int8_t* W;            // m x ldw
   int64_t ldw;
-  const float* sW;      // ceil(m*n/256)
+  float* sW;            // ceil(m*n/256); grows in place where w_rescale = 1
   uint16_t* Pbf;        // scratch: P~ (m x r bf16, or n x r for the right side)
   uint16_t* Nbuf;       // scratch: N (R's shape, bf16, row stride ldN)
   int64_t ldN;
   int32_t m, n, r;
   int32_t side;         // 0: P m x r, R = P^T G (r x n); 1: P n x r, R = G P (m x r)
+  int32_t w_rescale;    // 1: a weight group leaving the INT8 grid is re-scaled (n % 256 == 0)
   float beta1, beta2, om1, om2, c1, c2, eps, alpha;  // c1 = -lr/(1-b1^t), c2 = 1/sqrt(1-b2^t)
   uint32_t t, layer_id;
   uint64_t seed;

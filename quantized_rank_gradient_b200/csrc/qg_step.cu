@@ -17,6 +17,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -345,7 +346,7 @@ struct StochRoundEpi {
 
   struct Args {
     int8_t* W;
-    const float* sW;
+    float* sW;           // written only by the re-scaling variant
     int64_t ldw;
     float alpha;
     uint32_t t, layer_id;
@@ -393,10 +394,16 @@ struct StochRoundEpi {
   // of 16-bit lanes, clamped to [-127, 127] by one max and one min on both
   // lanes; the low bytes of four lanes are the four new codes.  When |X|
   // reaches 2^22, or X is NaN, the chunk is redone in the general form.
-  template <bool kOneFactor>
+  //
+  // kTrack: also the largest and smallest T = q 2^16 + K over the chunk (K = 0
+  // where X is NaN), each element's value in units of 2^-16 code; in the fast
+  // form T is the magic sum's low bits plus q 2^16.
+  template <bool kOneFactor, bool kTrack = false>
   static QG_DEV void sr_chunk(const uint32_t (&U)[32], const uint4& wa, const uint4& wb, const uint32_t (&d)[16],
-                              float cp0, float cp1, int split, uint32_t (&out)[8]) {
+                              float cp0, float cp1, int split, uint32_t (&out)[8], int* tmax = nullptr,
+                              int* tmin = nullptr) {
     float mx = 0.f;
+    int cmax = INT_MIN, cmin = INT_MAX;
     uint32_t sum[2], lanes[2];
 #pragma unroll
     for (int k = 0; k < 32; ++k) {
@@ -408,25 +415,40 @@ struct StochRoundEpi {
       const uint32_t wsel = 0x44u | (static_cast<uint32_t>(k & 3) << 8) | (static_cast<uint32_t>((k & 3) | 8) << 12);
       const uint32_t q16 = prmt(word_of(k < 16 ? wa : wb, (k >> 2) & 3), 0u, wsel);
       sum[k & 1] = tb + dq + q16;
+      if (kTrack) {
+        const int T = static_cast<int>(tb + q16 - kMagicBits);
+        cmax = max(cmax, T);
+        cmin = min(cmin, T);
+      }
       if (k & 1) lanes[(k >> 1) & 1] = clamp127_s16x2(prmt(sum[0], sum[1], 0x7632u));
       if ((k & 3) == 3) out[k >> 2] = prmt(lanes[0], lanes[1], 0x6420u);
     }
     if (!(mx < 4194304.0f)) {
+      cmax = INT_MIN;
+      cmin = INT_MAX;
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
         const float cp = (kOneFactor || k < split) ? cp0 : cp1;
         const float X = __fmul_rn(__uint_as_float(U[k]), cp);
         const uint4& w = k < 16 ? wa : wb;
         const int q = static_cast<int8_t>((word_of(w, (k >> 2) & 3) >> (8 * (k & 3))) & 0xFFu);
-        int v = q;
+        int v = q, K = 0;
         if (X == X) {
-          const int K = __float2int_ru(fminf(fmaxf(X, -1073741824.0f), 1073741824.0f));
+          K = __float2int_ru(fminf(fmaxf(X, -1073741824.0f), 1073741824.0f));
           const int draw = static_cast<int>((d[k >> 1] >> (16 * (k & 1))) & 0xFFFFu);
           v = min(max(q + ((K + draw) >> 16), -127), 127);
+        }
+        if (kTrack) {
+          cmax = max(cmax, q * 65536 + K);
+          cmin = min(cmin, q * 65536 + K);
         }
         const uint32_t sh = 8 * (k & 3);
         out[k >> 2] = (out[k >> 2] & ~(0xFFu << sh)) | ((static_cast<uint32_t>(v) & 0xFFu) << sh);
       }
+    }
+    if (kTrack) {
+      *tmax = max(*tmax, cmax);
+      *tmin = min(*tmin, cmin);
     }
   }
 
@@ -488,6 +510,111 @@ struct StochRoundEpi {
   }
 };
 
+// ------------------------------------------------------------------ a4 + a5, re-scaling variant
+
+// A weight group that the update would carry off the INT8 grid gets a larger
+// scale instead of saturating.  With X = U c' and K = ceil(X) as above, every
+// element's value in units of 2^-16 code is the integer T = q 2^16 + K
+// (T = q 2^16 where X is NaN); per group, A = max |T|.
+//   A <= 127 2^16: the codes are those of the saturating form (no element can
+//                  reach the clamp) and the scale stays;
+//   otherwise:     rho = (127 2^16) / A and s' = s / rho (IEEE float32
+//                  divisions), and every code of the group becomes
+//                  clamp(floor((ceil(fl(T) rho) + draw) / 2^16), -127, 127)
+//                  with the same draw, fl(T) the nearest float32.
+// The expected value of code' s' stays q s + alpha U (up to the 2^-16 draw
+// grid and float32 rounding).  Needs n % 256 == 0, so that a group is one row
+// of a 256-column tile.  The rounding pass runs as in the saturating form and
+// also takes the row slice's exact max |T|; the two warpgroups combine their
+// maxima through the exchange slots, and only a row whose group grows is
+// rounded again on the new grid (its accumulator and W codes are still staged)
+// and overwritten.
+struct StochRoundRescaleEpi : StochRoundEpi {
+  static constexpr bool kExchange = true;
+  static constexpr int kLimit = 127 * 65536;
+
+  static QG_DEV void rescaled_chunk(const uint32_t (&U)[32], const uint4& wa, const uint4& wb,
+                                    const uint32_t (&d)[16], float cp, float rho, uint32_t (&out)[8]) {
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const float X = __fmul_rn(__uint_as_float(U[k]), cp);
+      const uint4& w = k < 16 ? wa : wb;
+      const int q = static_cast<int8_t>((word_of(w, (k >> 2) & 3) >> (8 * (k & 3))) & 0xFFu);
+      const int K = X == X ? __float2int_ru(fminf(fmaxf(X, -1073741824.0f), 1073741824.0f)) : 0;
+      const float Z = __fmul_rn(__int2float_rn(q * 65536 + K), rho);
+      const int draw = static_cast<int>((d[k >> 1] >> (16 * (k & 1))) & 0xFFFFu);
+      const int v = min(max((__float2int_ru(Z) + draw) >> 16, -127), 127);
+      const uint32_t sh = 8 * (k & 3);
+      if ((k & 3) == 0) out[k >> 2] = 0u;
+      out[k >> 2] |= (static_cast<uint32_t>(v) & 0xFFu) << sh;
+    }
+  }
+
+  static QG_DEV void store_chunk(int8_t* dst, const uint32_t (&out)[8]) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+    *reinterpret_cast<uint4*>(dst + 16) = make_uint4(out[4], out[5], out[6], out[7]);
+  }
+
+  static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
+                           const EpiPair& ep, const uint8_t* side) {
+    const int irow = mb * BM + row;
+    const bool row_ok = irow < M;
+    const int j0 = nb * BN;  // N % 256 == 0: every tile is 256 columns wide
+    const int nchunk = BN / 32 / ep.groups;
+    const int c0 = ep.group * nchunk;
+    const int64_t g = row_ok ? (static_cast<int64_t>(irow) * N + j0) >> 8 : 0;
+    const float s = row_ok ? a.sW[g] : 0.f;
+    const float cp = update_factor(a.alpha, s);
+    int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + j0;
+    const PhiloxRoundKeys rk = philox_round_keys(a.key);
+    int tmax = INT_MIN, tmin = INT_MAX;
+#pragma unroll 1
+    for (int c = c0; c < c0 + nchunk; ++c) {
+      uint32_t U[32];
+      tmem_ld_32x32b_x32(taddr + c * 32, U);
+      tmem_ld_wait();
+      if (!row_ok) continue;
+      const uint4 wa = side_granule(side, row, 2 * c), wb = side_granule(side, row, 2 * c + 1);
+      uint32_t d[16];
+      draws(a, rk, irow, j0 + c * 32, d);
+      uint32_t out[8];
+      sr_chunk<true, true>(U, wa, wb, d, cp, cp, 32, out, &tmax, &tmin);
+      store_chunk(wrow + c * 32, out);
+    }
+    // |T| < 2^31: |q 2^16| <= 127 2^16 and |K| <= 2^30
+    uint32_t amax = row_ok ? static_cast<uint32_t>(max(tmax, -tmin)) : 0u;
+
+    // the group's maximum over both column slices (the other group's warps own
+    // the same rows); the slots carry the integer's bits
+    const int lane = row & 31;
+    ep.xchg[ep.group * BM + lane] = make_float2(__uint_as_float(amax), 0.f);
+    __threadfence_block();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(ep.xbar);
+    if (mbar_wait(ep.xbar, ep.xphase, ep.abort, ep.status)) {
+      for (int o = 0; o < ep.groups; ++o)
+        if (o != ep.group) amax = max(amax, __float_as_uint(ep.xchg[o * BM + lane].x));
+    }
+    const bool grow = row_ok && s > 0.f && amax > static_cast<uint32_t>(kLimit);
+    if (!__any_sync(0xFFFFFFFFu, grow)) return;
+    const float rho = grow ? __fdiv_rn(static_cast<float>(kLimit), __uint2float_rn(amax)) : 1.f;
+#pragma unroll 1
+    for (int c = c0; c < c0 + nchunk; ++c) {
+      uint32_t U[32];
+      tmem_ld_32x32b_x32(taddr + c * 32, U);
+      tmem_ld_wait();
+      if (!grow) continue;
+      const uint4 wa = side_granule(side, row, 2 * c), wb = side_granule(side, row, 2 * c + 1);
+      uint32_t d[16];
+      draws(a, rk, irow, j0 + c * 32, d);
+      uint32_t out[8];
+      rescaled_chunk(U, wa, wb, d, cp, rho, out);
+      store_chunk(wrow + c * 32, out);
+    }
+    if (grow && ep.group == 0) a.sW[g] = __fdiv_rn(s, rho);
+  }
+};
+
 // ------------------------------------------------------------------ plain fp32 store
 
 struct StoreF32Epi {
@@ -539,6 +666,7 @@ struct StoreF32Epi {
 // kernel parameters up to 32764 bytes (CUDA 12.1 and later on sm_70 and newer)
 static_assert(sizeof(GemmParams<AdamEpi>) <= 32764, "kernel parameter block");
 static_assert(sizeof(GemmParams<StochRoundEpi>) <= 32764, "kernel parameter block");
+static_assert(sizeof(GemmParams<StochRoundRescaleEpi>) <= 32764, "kernel parameter block");
 static_assert(sizeof(GemmParams<StoreF32Epi>) <= 32764, "kernel parameter block");
 
 // ------------------------------------------------------------------ a1 and test kernels
@@ -780,6 +908,49 @@ static cudaError_t launch_dequant_for(const StepProblem* probs, int cnt, cudaStr
   return launch_dequant_batch(db, stream);
 }
 
+// a4+a5 for `cnt` problems of one projection side, all with the epilogue Epi
+// (the saturating or the re-scaling stochastic rounding): one grid.
+template <class Epi, bool kRight>
+static cudaError_t launch_backproject(const StepProblem* probs, const int* idx, int cnt, cudaStream_t stream) {
+  GemmParams<Epi> p2;
+  memset(&p2, 0, sizeof(p2));
+  double fl2 = 0, by2 = 0;
+  // The batch's matrices in reverse order: the last N written by a2+a3 (and
+  // its P~, read last there) is the likeliest still in L2.
+  for (int jj = 0; jj < cnt; ++jj) {
+#if QG_SR_REVERSE
+    const int ii = cnt - 1 - jj;
+#else
+    const int ii = jj;
+#endif
+    const StepProblem& s = probs[idx[ii]];
+    const double m = s.m, n = s.n, r = s.r;
+    fl2 += 2 * m * n * r;
+    // W read + written, W scales, P~, N
+    by2 += 2 * m * n + 4 * std::ceil(m * n / 256.0) + 2 * (kRight ? n : m) * r + 2 * (kRight ? m : r) * (kRight ? r : n);
+    GemmProblem<Epi>& pr = p2.prob[p2.nprob];
+    if (kRight) {
+      // A = N (M = m, K = r), K-major: box {64 (r), 128 (m)}
+      if (!encode_map_bf16(&pr.tmA, s.Nbuf, s.r, s.m, s.ldN, 64, 128)) return cudaErrorInvalidValue;
+      // B = P~^T (K = r, N = n), K-major over P~ (n x r): box {64 (r), 128 (n)}
+      if (!encode_map_bf16(&pr.tmB, s.Pbf, s.r, s.n, s.r, 64, 128)) return cudaErrorInvalidValue;
+    } else {
+      // A = P~ (M = m, K = r), K-major: box {64 (r), 128 (m)}
+      if (!encode_map_bf16(&pr.tmA, s.Pbf, s.r, s.m, s.r, 64, 128)) return cudaErrorInvalidValue;
+      // B = N (K = r, N = n), MN-major: box {64 (n), 64 (r)}
+      if (!encode_map_bf16(&pr.tmB, s.Nbuf, s.n, s.r, s.ldN, 64, 64)) return cudaErrorInvalidValue;
+    }
+    // side operand: W^Q (m x n int8, leading dimension ldw)
+    if (!encode_map_i8_side(&pr.tmS[0], s.W, s.n, s.m, s.ldw)) return cudaErrorInvalidValue;
+    pr.status = s.status;
+    pr.epi = typename Epi::Args{s.W, s.sW, s.ldw, s.alpha, s.t, s.layer_id,
+                                PhiloxKey{static_cast<uint32_t>(s.seed), static_cast<uint32_t>(s.seed >> 32)},
+                                (s.n % 256) == 0 ? 1 : 0};
+    add_problem(p2, s.m, s.n, s.r);
+  }
+  return launch_gemm_pair<Epi, false, !kRight>(p2, stream, QG_KERNEL_BACKPROJECT_SR, fl2, by2);
+}
+
 // a2+a3 and a4+a5 for the problems of one projection side (kRight: P n x r,
 // R = G P, U = N P^T; otherwise P m x r, R = P^T G, U = P N): one grid each.
 template <bool kRight>
@@ -787,17 +958,14 @@ static cudaError_t launch_gemms_side(const StepProblem* probs, const int* idx, i
   cudaError_t e;
   GemmParams<AdamEpi> p1;
   memset(&p1, 0, sizeof(p1));
-  double fl1 = 0, by1 = 0, fl2 = 0, by2 = 0;
+  double fl1 = 0, by1 = 0;
   for (int ii = 0; ii < cnt; ++ii) {
     const StepProblem& s = probs[idx[ii]];
     const double m = s.m, n = s.n, r = s.r;
     const double p_rows = kRight ? n : m, rows = kRight ? m : r, cols = kRight ? r : n;
     fl1 += 2 * m * n * r;
-    fl2 += 2 * m * n * r;
     // a2+a3: G, P~, moments read + written, their scales, N written
     by1 += 2 * m * n + 2 * p_rows * r + 4 * rows * cols + 16.0 * rows * s.nblk + 2 * rows * cols;
-    // a4+a5: W read + written, W scales, P~, N
-    by2 += 2 * m * n + 4 * std::ceil(m * n / 256.0) + 2 * p_rows * r + 2 * rows * cols;
     GemmProblem<AdamEpi>& pr = p1.prob[p1.nprob];
     if (kRight) {
       // A = G (M = m, K = n), K-major: box {64 (n), 128 (m)}
@@ -826,39 +994,17 @@ static cudaError_t launch_gemms_side(const StepProblem* probs, const int* idx, i
   }
   e = launch_gemm_pair<AdamEpi, !kRight>(p1, stream, QG_KERNEL_PROJECT_ADAM, fl1, by1);
   if (e != cudaSuccess) return e;
-
-  GemmParams<StochRoundEpi> p2;
-  memset(&p2, 0, sizeof(p2));
-  // The batch's matrices in reverse order: the last N written by a2+a3 (and
-  // its P~, read last there) is the likeliest still in L2.
-  for (int jj = 0; jj < cnt; ++jj) {
-#if QG_SR_REVERSE
-    const int ii = cnt - 1 - jj;
-#else
-    const int ii = jj;
-#endif
-    const StepProblem& s = probs[idx[ii]];
-    GemmProblem<StochRoundEpi>& pr = p2.prob[p2.nprob];
-    if (kRight) {
-      // A = N (M = m, K = r), K-major: box {64 (r), 128 (m)}
-      if (!encode_map_bf16(&pr.tmA, s.Nbuf, s.r, s.m, s.ldN, 64, 128)) return cudaErrorInvalidValue;
-      // B = P~^T (K = r, N = n), K-major over P~ (n x r): box {64 (r), 128 (n)}
-      if (!encode_map_bf16(&pr.tmB, s.Pbf, s.r, s.n, s.r, 64, 128)) return cudaErrorInvalidValue;
-    } else {
-      // A = P~ (M = m, K = r), K-major: box {64 (r), 128 (m)}
-      if (!encode_map_bf16(&pr.tmA, s.Pbf, s.r, s.m, s.r, 64, 128)) return cudaErrorInvalidValue;
-      // B = N (K = r, N = n), MN-major: box {64 (n), 64 (r)}
-      if (!encode_map_bf16(&pr.tmB, s.Nbuf, s.n, s.r, s.ldN, 64, 64)) return cudaErrorInvalidValue;
-    }
-    // side operand: W^Q (m x n int8, leading dimension ldw)
-    if (!encode_map_i8_side(&pr.tmS[0], s.W, s.n, s.m, s.ldw)) return cudaErrorInvalidValue;
-    pr.status = s.status;
-    pr.epi = StochRoundEpi::Args{s.W, s.sW, s.ldw, s.alpha, s.t, s.layer_id,
-                                 PhiloxKey{static_cast<uint32_t>(s.seed), static_cast<uint32_t>(s.seed >> 32)},
-                                 (s.n % 256) == 0 ? 1 : 0};
-    add_problem(p2, s.m, s.n, s.r);
+  // a4+a5: the saturating problems in one grid, the re-scaling ones in another
+  int sat[kMaxProblems], grow[kMaxProblems], ns = 0, ng = 0;
+  for (int ii = 0; ii < cnt; ++ii) {
+    if (probs[idx[ii]].w_rescale)
+      grow[ng++] = idx[ii];
+    else
+      sat[ns++] = idx[ii];
   }
-  return launch_gemm_pair<StochRoundEpi, false, !kRight>(p2, stream, QG_KERNEL_BACKPROJECT_SR, fl2, by2);
+  if (ns > 0 && (e = launch_backproject<StochRoundEpi, kRight>(probs, sat, ns, stream)) != cudaSuccess) return e;
+  if (ng > 0) e = launch_backproject<StochRoundRescaleEpi, kRight>(probs, grow, ng, stream);
+  return e;
 }
 
 // The batch's left-side problems, then its right-side ones.

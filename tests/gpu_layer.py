@@ -20,7 +20,8 @@ def stream():
 def lib_config(oc: O.Config):
     return qg.config(oc.m, oc.n, oc.r, beta1=oc.beta1, beta2=oc.beta2, eps=oc.eps, lr=oc.lr, alpha=oc.alpha,
                      gamma=oc.gamma, delta0=oc.delta0, oversample=oc.oversample, power_iters=oc.power_iters,
-                     seed=oc.seed, layer_id=oc.layer_id, mom_refresh=oc.mom_refresh, proj_side=oc.proj_side)
+                     seed=oc.seed, layer_id=oc.layer_id, mom_refresh=oc.mom_refresh, proj_side=oc.proj_side,
+                     w_rescale=oc.w_rescale)
 
 
 def upload_gradient(G_bits: np.ndarray, device="cuda"):

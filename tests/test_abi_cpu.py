@@ -61,6 +61,8 @@ def test_config_defaults_and_sizes():
     ("r", 48, qg.QG_ESHAPE), ("r", 512, qg.QG_ESHAPE), ("w_group", 128, qg.QG_ESHAPE),
     ("beta1", 1.0, qg.QG_EINVAL), ("eps", 0.0, qg.QG_EINVAL), ("delta0", 0, qg.QG_EINVAL),
     ("mom_refresh", 3, qg.QG_EINVAL), ("mom_refresh", -1, qg.QG_EINVAL),
+    ("proj_side", 2, qg.QG_EINVAL), ("w_rescale", 2, qg.QG_EINVAL),
+    ("w_rescale", 1, qg.QG_ESHAPE),  # n = 300: a weight group is not one tile row
 ])
 def test_layer_init_rejects_bad_config_before_any_launch(field, value, expect):
     c = qg.config(256, 300, 64)

@@ -280,3 +280,123 @@ def test_step_batch_mixed_sides_equals_single_steps():
         np.testing.assert_array_equal(a.weights(), b.weights())
         for x, y in zip(a.moments(), b.moments()):
             np.testing.assert_array_equal(x, y)
+
+
+# ---------------------------------------------------------------- weight groups re-scaled instead of saturating
+
+def _rescale_layer(m, n, r, seed, side=0, layer_id=6):
+    # P = the first r columns of the identity: P~ is exactly 0 / 1, so R = P~^T G
+    # and U = P~ N have one nonzero product per element and are exact on both
+    # sides, whatever the accumulation order: the step is then bit-exact.  The
+    # scales of the projected rows (columns on the right side) range from tiny
+    # (every group grows) through moderate (groups with codes near +-127 grow)
+    # to ordinary.
+    oc = O.Config(m=m, n=n, r=r, seed=seed, layer_id=layer_id, proj_side=side, w_rescale=1, alpha=0.25)
+    Wq = synth.weight_codes(m, n, seed)
+    sW = synth.weight_scales(m, n, seed=seed).copy()
+    gpr = n // 256
+    rows = np.arange(len(sW)) // gpr
+    sW[rows < r // 3] *= np.float32(1e-4)
+    sW[(rows >= r // 3) & (rows < 2 * r // 3)] *= np.float32(0.05)
+    ost = O.LayerState.create(oc, Wq, sW)
+    P = np.eye(n if side else m, r)
+    O.set_projection(ost, P)
+    gl = GpuLayer(oc, Wq, sW)
+    gl.set_projection(ost.Pq, ost.sP)
+    gen = synth.lowrank_gradient(m, n, rank=min(64, m, n), seed=seed)
+    return ost, gl, gen
+
+
+@pytest.mark.parametrize("m,n,r,side", [(512, 768, 96, 0), (300, 512, 64, 0), (768, 512, 64, 1)])
+def test_step_rescale_bit_exact_on_exact_products(m, n, r, side):
+    ost, gl, gen = _rescale_layer(m, n, r, seed=m + n, side=side)
+    sW0 = ost.sW.copy()
+    for t in range(3):
+        G, Gb = gen.draw(t)
+        dG, ldg = upload_gradient(Gb)
+        gl.step(dG, ldg)
+        O.step(ost, G)
+        np.testing.assert_array_equal(gl.weights(), ost.Wq, err_msg=f"codes after step {t + 1}")
+        np.testing.assert_array_equal(gl.sW.cpu().numpy(), ost.sW, err_msg=f"scales after step {t + 1}")
+    grown = ost.sW > sW0
+    assert grown.sum() > len(sW0) // 10          # the case exercises the re-scaling
+    assert not np.all(grown)
+    assert gl.status() == qg.QG_OK
+
+
+@pytest.mark.parametrize("m,n,r", [(512, 1024, 128), (1376, 512, 64)])
+def test_step_rescale_parity_with_oracle(m, n, r):
+    # A random projection: the GPU's U = P~ N is an fp32 tensor-core sum of r
+    # products (and its N may differ from the oracle's in the last bf16 bit of a
+    # few elements), so a group's max |T| -- and the grown scale
+    # s' = s max|T| / (127 2^16) -- can differ from the oracle's.  Each step
+    # starts both sides from the GPU's state, so that only that step's
+    # arithmetic differs; the codes must meet the step's usual bar, and every
+    # scale must lie within the bound that the differences in U allow:
+    #   |dU| <= r 2^-23 (|P~| |N|) + |P~| |N_gpu - N|,  |dT| <= c' |dU| + 2,
+    #   |ds'| <= s max_group |dT| / (127 2^16) + 4 ulp(s').
+    oc = O.Config(m=m, n=n, r=r, seed=31, layer_id=1, w_rescale=1)
+    Wq = synth.weight_codes(m, n, 31)
+    sW = synth.weight_scales(m, n, seed=31).copy()
+    sW[::3] *= np.float32(0.01)
+    gen = synth.lowrank_gradient(m, n, rank=min(256, m, n), seed=31)
+    ost = O.LayerState.create(oc, Wq, sW)
+    O.set_projection(ost, O.exact_topr(gen.draw(0)[0], r)[0])
+    gl = GpuLayer(oc, Wq, sW)
+    gl.set_projection(ost.Pq, ost.sP)
+    grown = 0
+    for t in range(3):
+        ost.Wq = gl.weights().copy()
+        ost.sW = gl.sW.cpu().numpy().copy()
+        ost.Mq, ost.sM, ost.Vq, ost.sV = [x.copy() for x in gl.moments()]
+        s0 = ost.sW.copy()
+        G, Gb = gen.draw(t)
+        dG, ldg = upload_gradient(Gb)
+        gl.step(dG, ldg)
+        inter = O.step(ost, G)
+        compare_state(ost, gl, f"re-scaling, step {t + 1}")
+        Pb, N = np.abs(inter["P"]).astype(np.float64), inter["N"].astype(np.float64)
+        dN = np.abs(O.bf16_from_bits(gl.scratch_N()).astype(np.float64) - N)
+        dU = r * 2.0 ** -23 * (Pb @ np.abs(N)) + Pb @ dN
+        cp = np.float64(oc.alpha) / s0.astype(np.float64) * 65536.0
+        dT = (dU.reshape(-1, 256) * cp[:, None]).max(axis=1) + 2.0
+        sg = gl.sW.cpu().numpy().astype(np.float64)
+        tol = s0 * dT / (127 * 65536.0) + 4 * np.spacing(ost.sW).astype(np.float64)
+        bad = np.abs(sg - ost.sW) > tol
+        assert not bad.any(), f"step {t + 1}: {bad.sum()} scales outside the bound, worst " \
+            f"{(np.abs(sg - ost.sW) / tol).max():.2f} x"
+        grown += int((ost.sW > s0).sum())
+    assert grown > len(sW) // 10
+    assert gl.status() == qg.QG_OK
+
+
+def test_step_batch_mixed_rescale_equals_single_steps():
+    specs = [(512, 768, 96, 0, 1), (512, 768, 96, 0, 0), (768, 512, 64, 1, 1), (300, 512, 64, 0, 1),
+             (256, 256, 32, 0, 0), (768, 512, 64, 1, 0)]
+    singles, batched, grads = [], [], []
+    for i, (m, n, r, side, wr) in enumerate(specs):
+        pair = []
+        for _ in range(2):
+            ost, gl, gen = _rescale_layer(m, n, r, seed=60 + i, side=side, layer_id=i)
+            if not wr:
+                gl.close()
+                oc = O.Config(**{**ost.cfg.__dict__, "w_rescale": 0})
+                gl = GpuLayer(oc, ost.Wq, ost.sW)
+                gl.set_projection(ost.Pq, ost.sP)
+            pair.append(gl)
+        singles.append(pair[0])
+        batched.append(pair[1])
+        grads.append(upload_gradient(gen.draw(0)[1]))
+    for gl, (dG, ldg) in zip(singles, grads):
+        gl.step(dG, ldg)
+    cfgs = [gl.cfg for gl in batched]
+    arr = (qg.POINTER(qg.qg_config) * len(cfgs))(*[qg.ctypes.pointer(c) for c in cfgs])
+    wsb = qg.qg_step_batch_workspace_bytes(arr, len(cfgs))
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    hs = (c_void_p * len(batched))(*[gl.h.value for gl in batched])
+    gs = (c_void_p * len(batched))(*[g.data_ptr() for g, _ in grads])
+    lds = (qg.c_int64 * len(batched))(*[ld for _, ld in grads])
+    qg.check(qg.qg_step_batch(hs, gs, lds, len(batched), ws.data_ptr(), wsb, stream()))
+    for a, b in zip(singles, batched):
+        np.testing.assert_array_equal(a.weights(), b.weights())
+        np.testing.assert_array_equal(a.sW.cpu().numpy(), b.sW.cpu().numpy())
