@@ -15,6 +15,13 @@ sigma = 1e-4) resident in HBM (13 GB, far larger than L2).
 
 Under torchrun (N > 1) every rank updates its own full stack (weak scaling, no
 collective on the data path); rank 0 prints one JSON line.
+
+Variants of the stack workload, by environment (the workload name says which ran):
+    QG_BENCH_SIDE=right-tall   project matrices with m > n on the right (P n x r)
+    QG_BENCH_W_RESCALE=1       weight groups leaving the INT8 grid grow their scale
+    QG_BENCH_PER_LAYER=1       one qg_step_batch call per decoder layer, one stream
+Other workloads: --workload llama1b-stack | llama60m-stack | refresh-stress |
+linear-grad-stress | linear-7b.
 """
 from __future__ import annotations
 
@@ -288,6 +295,8 @@ class Stack:
         # stream, kernels one after another) also serve the kernel-timing pass.
         whole = [[e for group in self.layers for e in group]]
         self.per_layer_only = os.environ.get("QG_BENCH_PER_LAYER") == "1"
+        if self.per_layer_only:
+            self.variant += "-per-layer"
         need = 0
         for group in whole + self.layers:
             arr = (qg.POINTER(qg.qg_config) * len(group))(*[qg.ctypes.pointer(e["cfg"]) for e in group])
