@@ -9,7 +9,9 @@ matrix can be owned by one rank:
    receives the mean over the ranks;
 3. each rank runs the optimizer step (qg_step_batch) on the matrices it owns;
 4. the updated INT8 weights are all-gathered, so that every rank holds the
-   whole model for the next forward pass.
+   whole model for the next forward pass.  Each matrix's group scales sit
+   right after its codes in the same buffer: with qg_config.w_rescale = 1 the
+   owner's step changes them, and the one all-gather carries them too.
 
 Matrices go to ranks longest first, each to the rank with the least work so far
 (work = 4 m n r, the step's FLOPs), ties to the lowest rank.  Gradients and
@@ -27,7 +29,7 @@ import torch
 import torch.distributed as dist
 
 GRAD_ALIGN = 8      # bf16 elements: every gradient starts on a 16-byte boundary
-WEIGHT_ALIGN = 256  # bytes: every weight matrix starts on a 256-byte boundary
+WEIGHT_ALIGN = 256  # bytes: every weight matrix and every scale array starts on a 256-byte boundary
 
 
 def _round(x, a):
@@ -41,6 +43,7 @@ class ShardPlan:
     owner: list            # rank owning matrix i
     grad_offset: list      # element offset of matrix i's gradient (m x ldg) in the flat gradient buffer
     weight_offset: list    # byte offset of matrix i's codes (m x ldw) in the flat weight buffer
+    scale_offset: list     # byte offset of matrix i's ceil(m n / 256) float32 group scales, after its codes
     ldg: list              # gradient row stride (elements)
     ldw: list              # weight row stride (bytes)
     grad_shard: int        # elements per rank shard of the gradient buffer
@@ -65,18 +68,21 @@ def plan_shards(shapes, ranks_r, world) -> ShardPlan:
         work[w] += cost[i]
     ldg = [_round(n, GRAD_ALIGN) for (_, n) in shapes]
     ldw = [_round(n, 16) for (_, n) in shapes]
-    goff, woff = [0] * len(shapes), [0] * len(shapes)
+    goff, woff, soff = [0] * len(shapes), [0] * len(shapes), [0] * len(shapes)
     gsize, wsize = [0] * world, [0] * world
-    for i, (m, _n) in enumerate(shapes):  # within a shard, matrices keep their order
+    for i, (m, n) in enumerate(shapes):  # within a shard, matrices keep their order
         k = owner[i]
         goff[i], woff[i] = gsize[k], wsize[k]
         gsize[k] += _round(m * ldg[i], GRAD_ALIGN)
         wsize[k] += _round(m * ldw[i], WEIGHT_ALIGN)
+        soff[i] = wsize[k]
+        wsize[k] += _round(4 * -(-(m * n) // 256), WEIGHT_ALIGN)
     gshard, wshard = _round(max(gsize), GRAD_ALIGN), _round(max(wsize), WEIGHT_ALIGN)
     for i in range(len(shapes)):
         goff[i] += owner[i] * gshard
         woff[i] += owner[i] * wshard
-    return ShardPlan(world, owner, goff, woff, ldg, ldw, gshard, wshard, work)
+        soff[i] += owner[i] * wshard
+    return ShardPlan(world, owner, goff, woff, soff, ldg, ldw, gshard, wshard, work)
 
 
 def grad_view(flat, plan, i, shape):
@@ -89,6 +95,14 @@ def weight_view(flat, plan, i, shape):
     """Matrix i's INT8 codes (m x ldw) inside the flat weight buffer."""
     m, _n = shape
     return flat[plan.weight_offset[i]: plan.weight_offset[i] + m * plan.ldw[i]].view(m, plan.ldw[i])
+
+
+def scale_view(flat, plan, i, shape):
+    """Matrix i's ceil(m n / 256) float32 group scales inside the flat weight
+    buffer (a uint8 tensor): the d_Wscale array of its qg_layer."""
+    m, n = shape
+    ng = -(-(m * n) // 256)
+    return flat[plan.scale_offset[i]: plan.scale_offset[i] + 4 * ng].view(torch.float32)
 
 
 def reduce_scatter_gradients(flat, plan, rank, group=None):
@@ -108,7 +122,8 @@ def reduce_scatter_gradients(flat, plan, rank, group=None):
 
 
 def all_gather_weights(flat, plan, rank, group=None):
-    """Every rank's shard of the flat weight buffer to every rank."""
+    """Every rank's shard of the flat weight buffer (codes and group scales) to
+    every rank."""
     n = plan.weight_shard
     if plan.world == 1:
         return flat

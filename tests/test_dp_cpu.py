@@ -4,8 +4,11 @@ qg_step_batch on the owned matrices.
 
 Every rank holds the gradients of its own slice of the batch for all matrices;
 after the reduce-scatter each owner steps its matrices on the mean gradient, and
-after the all-gather every rank must hold, bit for bit, the weights of one
-process that averaged the gradients and stepped every matrix itself.
+after the all-gather every rank must hold, bit for bit, the weights (codes and
+group scales) of one process that averaged the gradients and stepped every
+matrix itself.  The second case mixes projection sides and weight policies: a
+matrix whose groups are re-scaled (w_rescale = 1) changes its scales on the
+owner, and the all-gather must carry them.
 """
 import os
 import socket
@@ -15,6 +18,8 @@ import pytest
 import torch.multiprocessing as mp
 
 SHAPES = [(48, 64), (64, 40), (96, 32), (64, 64), (40, 48), (32, 96)]
+# (m, n, proj_side, w_rescale)
+MIXED = [(64, 256, 0, 1), (96, 256, 1, 1), (48, 64, 0, 0), (256, 64, 1, 0), (32, 512, 0, 1), (40, 48, 1, 0)]
 R = 32
 
 
@@ -24,13 +29,18 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _initial_state(i, m, n):
+def _spec(s):
+    return s if len(s) == 4 else (s[0], s[1], 0, 0)
+
+
+def _initial_state(i, spec):
     import oracle as O
     import synth
-    cfg = O.Config(m=m, n=n, r=R, seed=17 + i, layer_id=i)
+    m, n, side, wr = _spec(spec)
+    cfg = O.Config(m=m, n=n, r=R, seed=17 + i, layer_id=i, proj_side=side, w_rescale=wr)
     st = O.LayerState.create(cfg, synth.weight_codes(m, n, seed=i), synth.weight_scales(m, n, seed=i))
     G0, _ = synth.lowrank_gradient(m, n, rank=16, seed=500 + i).draw(0)
-    O.set_projection(st, O.exact_topr(G0, R)[0])
+    O.set_projection(st, O.exact_topr(G0 if side == 0 else G0.T, R)[0])
     return st
 
 
@@ -40,7 +50,7 @@ def _local_gradient(rank, i, m, n):
     return np.asarray(G, np.float32)
 
 
-def _worker(rank, world, port, out):
+def _worker(rank, world, port, out, specs):
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     sys.path.insert(0, root)
@@ -52,22 +62,26 @@ def _worker(rank, world, port, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        plan = dp.plan_shards(SHAPES, [R] * len(SHAPES), world)
+        shapes = [_spec(s)[:2] for s in specs]
+        plan = dp.plan_shards(shapes, [R] * len(shapes), world)
         flat_g = torch.zeros(world * plan.grad_shard, dtype=torch.float32)
         flat_w = torch.zeros(world * plan.weight_shard, dtype=torch.uint8)
-        states = [_initial_state(i, m, n) for i, (m, n) in enumerate(SHAPES)]
-        for i, (m, n) in enumerate(SHAPES):
+        states = [_initial_state(i, s) for i, s in enumerate(specs)]
+        for i, (m, n) in enumerate(shapes):
             dp.grad_view(flat_g, plan, i, (m, n))[:, :n] = torch.from_numpy(_local_gradient(rank, i, m, n))
             dp.weight_view(flat_w, plan, i, (m, n))[:, :n] = torch.from_numpy(states[i].Wq.view(np.uint8))
+            dp.scale_view(flat_w, plan, i, (m, n))[:] = torch.from_numpy(states[i].sW)
         dp.reduce_scatter_gradients(flat_g, plan, rank)
         for i in plan.owned(rank):
-            m, n = SHAPES[i]
+            m, n = shapes[i]
             G = dp.grad_view(flat_g, plan, i, (m, n))[:, :n].numpy().astype(np.float32)
             O.step(states[i], G)
             dp.weight_view(flat_w, plan, i, (m, n))[:, :n] = torch.from_numpy(states[i].Wq.view(np.uint8))
+            dp.scale_view(flat_w, plan, i, (m, n))[:] = torch.from_numpy(states[i].sW)
         dp.all_gather_weights(flat_w, plan, rank)
-        W = [dp.weight_view(flat_w, plan, i, s)[:, : s[1]].numpy().view(np.int8).copy() for i, s in enumerate(SHAPES)]
-        out.put((rank, plan.owner, plan.work, W))
+        W = [dp.weight_view(flat_w, plan, i, s)[:, : s[1]].numpy().view(np.int8).copy() for i, s in enumerate(shapes)]
+        S = [dp.scale_view(flat_w, plan, i, s).numpy().copy() for i, s in enumerate(shapes)]
+        out.put((rank, plan.owner, plan.work, W, S))
     finally:
         dist.destroy_process_group()
 
@@ -85,40 +99,52 @@ def test_plan_balances_work_and_aligns_every_matrix():
         spans_g, spans_w = [], []
         for i, (m, n) in enumerate(shapes):
             assert plan.grad_offset[i] % dp.GRAD_ALIGN == 0 and plan.weight_offset[i] % dp.WEIGHT_ALIGN == 0
+            assert plan.scale_offset[i] % dp.WEIGHT_ALIGN == 0
             k = plan.owner[i]
+            ns = -(-(m * n) // 256)
             assert k * plan.grad_shard <= plan.grad_offset[i] < (k + 1) * plan.grad_shard
             assert plan.grad_offset[i] + m * plan.ldg[i] <= (k + 1) * plan.grad_shard
-            assert plan.weight_offset[i] + m * plan.ldw[i] <= (k + 1) * plan.weight_shard
+            assert k * plan.weight_shard <= plan.weight_offset[i]
+            assert plan.scale_offset[i] + 4 * ns <= (k + 1) * plan.weight_shard
             spans_g.append((plan.grad_offset[i], plan.grad_offset[i] + m * plan.ldg[i]))
             spans_w.append((plan.weight_offset[i], plan.weight_offset[i] + m * plan.ldw[i]))
+            spans_w.append((plan.scale_offset[i], plan.scale_offset[i] + 4 * ns))
         for spans in (spans_g, spans_w):
             spans.sort()
             assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))  # no overlap
 
 
-def test_two_gloo_ranks_match_one_process_bit_for_bit():
+@pytest.mark.parametrize("specs", [SHAPES, MIXED], ids=["default", "mixed-sides-and-rescale"])
+def test_two_gloo_ranks_match_one_process_bit_for_bit(specs):
     import sys
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
     import oracle as O
     ctx = mp.get_context("spawn")
     out = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, out, specs)) for r in range(2)]
     for p in procs:
         p.start()
     res = {}
     for _ in range(2):
-        rank, owner, work, W = out.get(timeout=180)
-        res[rank] = (owner, work, W)
+        rank, owner, work, W, S = out.get(timeout=180)
+        res[rank] = (owner, work, W, S)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
     assert res[0][0] == res[1][0] and set(res[0][0]) == {0, 1}
     # one process: the mean gradient (two float32 terms, then a halving: exact
     # and order-free) and every matrix stepped here
-    for i, (m, n) in enumerate(SHAPES):
-        st = _initial_state(i, m, n)
+    grown = 0
+    for i, spec in enumerate(specs):
+        m, n = _spec(spec)[:2]
+        st = _initial_state(i, spec)
+        s0 = st.sW.copy()
         G = ((_local_gradient(0, i, m, n) + _local_gradient(1, i, m, n)) / np.float32(2)).astype(np.float32)
         O.step(st, G)
+        grown += int((st.sW != s0).sum())
         for rank in (0, 1):
             np.testing.assert_array_equal(res[rank][2][i], st.Wq, err_msg=f"matrix {i} on rank {rank}")
+            np.testing.assert_array_equal(res[rank][3][i], st.sW, err_msg=f"scales {i} on rank {rank}")
+    if specs is MIXED:
+        assert grown > 0  # some owner changed its scales, and every rank received them
