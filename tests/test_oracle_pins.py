@@ -99,6 +99,50 @@ def test_bf16_round_matches_torch():
 
 # ---------------------------------------------------------------- quantizers
 
+def test_bf16_from_bits_matches_torch():
+    # every bf16 bit pattern, decoded by torch as the reference
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()
+    got = O.bf16_from_bits(bits)
+    same = (got.view(np.uint32) == ref.view(np.uint32)) | (np.isnan(got) & np.isnan(ref))
+    assert same.all()
+
+
+def test_dequant_P_bf16_is_torch_bf16_of_the_int4_product():
+    rng = np.random.default_rng(12)
+    m, r = 96, 64
+    P = rng.standard_normal((m, r))
+    packed, scales = O.quant_int4_groups(P)
+    codes = O.unpack_int4(packed, m * r).reshape(m, r).astype(np.float32)
+    prod = codes * np.repeat(scales.astype(np.float32), 64).reshape(m, r)   # one float32 product each
+    ref = torch.from_numpy(prod).to(torch.bfloat16).float().numpy()
+    np.testing.assert_array_equal(O.dequant_P_bf16(packed, scales, m, r), ref)
+
+
+def test_proj_dims_and_adam_constants_closed_forms():
+    assert O.proj_dims(O.Config(m=300, n=700, r=64)) == (300, 64, 700)
+    assert O.proj_dims(O.Config(m=300, n=700, r=64, proj_side=1)) == (700, 300, 64)
+    with pytest.raises(ValueError):
+        O.proj_dims(O.Config(m=300, n=700, r=64, proj_side=2))
+    cfg = O.Config(m=64, n=64, r=32, lr=1e-3, beta1=0.9, beta2=0.999)
+    om1, om2, c1, c2 = O.adam_constants(cfg, 1)
+    # t = 1: c1 = -lr / (1 - b1) and c2 = 1 / sqrt(1 - b2), with b1, b2 and lr the float32 values
+    b1, b2, lr = float(np.float32(0.9)), float(np.float32(0.999)), float(np.float32(1e-3))
+    assert om1 == np.float32(1 - b1) and om2 == np.float32(1 - b2)
+    assert c1 == np.float32(-lr / (1 - b1)) and c2 == np.float32(1 / math.sqrt(1 - b2))
+    # bias corrections vanish as t grows
+    _, _, c1_inf, c2_inf = O.adam_constants(cfg, 100000)
+    assert c1_inf == np.float32(-lr) and c2_inf == np.float32(1.0)
+
+
+def test_refresh_due_rule():
+    st, _ = _small_layer()
+    st.t, st.t_next = 5, 7
+    assert not O.refresh_due(st) and O.refresh_due(st, force=True)
+    st.t = 7
+    assert O.refresh_due(st)
+
+
 def test_int4_golden_groups():
     g = json.load(open(os.path.join(GOLDEN, "int4_groups.json")))
     for case in g["cases"]:
