@@ -19,3 +19,20 @@ def cuda_ok():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return True
+
+
+# A GPU test whose kernel never finishes blocks the host inside a CUDA call,
+# where no signal handler runs; a watchdog thread then ends the process, so a
+# hang costs minutes, not the whole run.  The first test of a fresh process
+# also pays for CUDA start-up and the library load.
+GPU_TEST_TIMEOUT_S = 600
+
+
+def pytest_collection_modifyitems(config, items):
+    try:
+        import pytest_timeout  # noqa: F401
+    except ImportError:
+        return
+    for item in items:
+        if item.get_closest_marker("gpu") and not item.get_closest_marker("timeout"):
+            item.add_marker(pytest.mark.timeout(GPU_TEST_TIMEOUT_S, method="thread"))
