@@ -20,6 +20,7 @@ Variants of the stack workload, by environment (the workload name says which ran
     QG_BENCH_SIDE=right-tall   project matrices with m > n on the right (P n x r)
     QG_BENCH_W_RESCALE=1       weight groups leaving the INT8 grid grow their scale
     QG_BENCH_PER_LAYER=1       one qg_step_batch call per decoder layer, one stream
+A run still going after QG_BENCH_WATCHDOG_S seconds (default 1800) ends itself.
 Other workloads: --workload llama1b-stack | llama60m-stack | refresh-stress |
 linear-grad-stress | linear-7b.
 """
@@ -764,8 +765,29 @@ def run_e2e(stack, args, stream, world, device, barrier):
             "note": "bf16 gradients copied from pinned host memory each step; status words read back"}
 
 
+def start_watchdog():
+    """A run that has not ended after QG_BENCH_WATCHDOG_S seconds (default 1800;
+    the default run takes one to two minutes) is stuck, most likely in a CUDA
+    call that waits for a kernel: a daemon thread then ends the process, which
+    also releases its GPU context."""
+    import threading
+    limit = float(os.environ.get("QG_BENCH_WATCHDOG_S", "1800"))
+    if limit <= 0:
+        return
+
+    def fire():
+        sys.stderr.write(f"bench.py: no result after {limit:.0f} s; exiting\n")
+        sys.stderr.flush()
+        os._exit(3)
+
+    t = threading.Timer(limit, fire)
+    t.daemon = True
+    t.start()
+
+
 def main():
     args = parse_args()
+    start_watchdog()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
