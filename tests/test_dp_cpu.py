@@ -45,9 +45,11 @@ def _initial_state(i, spec):
 
 
 def _local_gradient(rank, i, m, n):
+    # on the 2^-24 grid (|G| << 1/3): a sum over up to three ranks is exact in
+    # float32 in any order, so the mean is one correctly rounded division
     import synth
     G, _ = synth.lowrank_gradient(m, n, rank=16, seed=1000 * (rank + 1) + i).draw(1)
-    return np.asarray(G, np.float32)
+    return (np.round(np.asarray(G, np.float64) * 2.0 ** 24) / 2.0 ** 24).astype(np.float32)
 
 
 def _worker(rank, world, port, out, specs):
@@ -114,36 +116,40 @@ def test_plan_balances_work_and_aligns_every_matrix():
             assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))  # no overlap
 
 
-@pytest.mark.parametrize("specs", [SHAPES, MIXED], ids=["default", "mixed-sides-and-rescale"])
-def test_two_gloo_ranks_match_one_process_bit_for_bit(specs):
+@pytest.mark.parametrize("world,specs", [(2, SHAPES), (2, MIXED), (3, MIXED)],
+                         ids=["2-default", "2-mixed-sides-and-rescale", "3-mixed"])
+def test_gloo_ranks_match_one_process_bit_for_bit(world, specs):
     import sys
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
     import oracle as O
     ctx = mp.get_context("spawn")
     out = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, out, specs)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, out, specs)) for r in range(world)]
     for p in procs:
         p.start()
     res = {}
-    for _ in range(2):
+    for _ in range(world):
         rank, owner, work, W, S = out.get(timeout=180)
         res[rank] = (owner, work, W, S)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    assert res[0][0] == res[1][0] and set(res[0][0]) == {0, 1}
-    # one process: the mean gradient (two float32 terms, then a halving: exact
-    # and order-free) and every matrix stepped here
+    assert all(res[k][0] == res[0][0] for k in range(world)) and set(res[0][0]) == set(range(world))
+    # one process: the mean gradient (an exact float32 sum, then one division)
+    # and every matrix stepped here
     grown = 0
     for i, spec in enumerate(specs):
         m, n = _spec(spec)[:2]
         st = _initial_state(i, spec)
         s0 = st.sW.copy()
-        G = ((_local_gradient(0, i, m, n) + _local_gradient(1, i, m, n)) / np.float32(2)).astype(np.float32)
+        total = _local_gradient(0, i, m, n)
+        for k in range(1, world):
+            total = (total + _local_gradient(k, i, m, n)).astype(np.float32)
+        G = (total / np.float32(world)).astype(np.float32)
         O.step(st, G)
         grown += int((st.sW != s0).sum())
-        for rank in (0, 1):
+        for rank in range(world):
             np.testing.assert_array_equal(res[rank][2][i], st.Wq, err_msg=f"matrix {i} on rank {rank}")
             np.testing.assert_array_equal(res[rank][3][i], st.sW, err_msg=f"scales {i} on rank {rank}")
     if specs is MIXED:
