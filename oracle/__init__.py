@@ -23,6 +23,17 @@ Pins (each checked by a CPU test against something other than the oracle):
                           zero scales
   linear_forward / linear_backward_data / linear_backward_weight
                         - brute-force sums on small inputs; integer matrix products
+  stochastic_round_rescale - equals stochastic_round_update inside the grid; the sum over
+                          all 2^16 draws against the exact value; per-element unbiasedness
+                          in groups carried off the grid; zero-scale, NaN and mixed groups
+  refresh_moments       - reset and keep; rotation by the identity and by a permutation
+  project_right / backproject_right / right-side refresh
+                        - brute-force loops; the refresh finds the right singular vectors
+  bf16_from_bits / dequant_P_bf16
+                        - torch's bfloat16 decoding of every bit pattern; torch's
+                          conversion of each INT4 product
+  proj_dims / adam_constants / refresh_due
+                        - closed forms and the scripted rule
 """
 from .qgalore import *  # noqa: F401,F403
 from . import qgalore  # noqa: F401
