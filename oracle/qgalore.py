@@ -412,6 +412,11 @@ def stochastic_round_rescale(Wq, sW, U, cfg: Config, t: int, u16=None):
     """Step a5 of the re-scaling variant: a weight group whose updated values
     would leave the INT8 grid gets a larger scale instead of saturating.
 
+    [QG-quant] keeps W in INT8 and updates it by unbiased stochastic rounding;
+    it does not say what happens at the ends of the grid.  Saturating (the
+    default, stochastic_round_update) is biased there; this variant is the
+    plainest reading that keeps the rounding unbiased: make the grid fit.
+
     With X and K = ceil(X) as in stochastic_round_update, each element's value
     in units of 2^-16 code is the integer T = q * 2^16 + K (T = q * 2^16 where X
     is NaN).  Per group g of 256 consecutive elements, A = max |T|:
