@@ -12,7 +12,9 @@ Pins (each checked by a CPU test against something other than the oracle):
   quant_rowblock_int8   - same, plus ragged last block
   adam_moments          - torch.optim.Adam on the same gradients; closed form at t = 1
   project / backproject - brute-force loops on small non-square inputs
-  stochastic_round_update - E[xi(y)] = y over 10^6 draws; integers fixed; clamp
+  stochastic_round_update - E[xi(y)] = y over 10^6 draws; the sum over all 2^16 draws is
+                          rint of the update (ties included); odd in the update and no
+                          drift over a dense grid; integers fixed; clamp
   cossim                - closed forms; scipy.linalg.subspace_angles
   randomized_topr       - exact SVD (LAPACK) when k = min(m, n) and on inputs with a gap
   schedule_after_refresh - scripted CosSim sequences; gamma > 1 gives a fixed interval

@@ -381,14 +381,18 @@ def stochastic_round_update(Wq, sW, U, cfg: Config, t: int, u16=None):
       c'_g = (alpha / s_g) * 2^16   (IEEE float32 division, exact scaling; a zero
                                      scale gives c'_g = 0 and freezes its group)
       X    = U * c'_g               (float32: the update in units of 2^-16 code)
-      K    = ceil(X)                (an integer)
+      K    = rint(X)                (nearest integer, ties to even)
       r    = floor((K + d) / 2^16)  (d = the element's 16-bit uniform draw)
       W'   = clamp(W + r, -127, 127);  a NaN X keeps the old code.
     Adding a uniform 16-bit integer and dropping the 16 fraction bits rounds
     K / 2^16 up with probability equal to its fractional part, so
-    E[r] = K / 2^16, which lies in [X / 2^16, X / 2^16 + 2^-16): unbiased up to
-    the 2^-16 grid of the draws.  |X| is clipped to 2^30 before the ceiling,
-    which changes no clamped result (|r| >= 2^14 saturates either way)."""
+    E[r] = K / 2^16 exactly (Hermite's identity: the sum of floor((K + d) / 2^16)
+    over all 2^16 draws is K).  K / 2^16 is X / 2^16 rounded to the nearest
+    point of the 2^-16 draw grid, so it is within 2^-17 code of the update, and
+    rint(-X) = -rint(X) makes that residue odd in X: an update and its negation
+    move the weight by exactly opposite amounts on average, so no sign of update
+    drifts.  |X| is clipped to 2^30 before the rounding, which changes no clamped
+    result (|r| >= 2^14 saturates either way)."""
     m, n = Wq.shape
     e = np.arange(m * n, dtype=np.int64).reshape(m, n)
     sW = np.asarray(sW, np.float32)
@@ -397,7 +401,7 @@ def stochastic_round_update(Wq, sW, U, cfg: Config, t: int, u16=None):
         cp = (c * F32(65536.0)).astype(np.float32)
         X = (np.asarray(U, np.float32) * cp[e // cfg.w_group]).astype(np.float32)
         nan = np.isnan(X)
-        K = np.ceil(np.clip(np.where(nan, F32(0), X), F32(-2.0 ** 30), F32(2.0 ** 30))).astype(np.int64)
+        K = np.rint(np.clip(np.where(nan, F32(0), X), F32(-2.0 ** 30), F32(2.0 ** 30))).astype(np.int64)
     if u16 is None:
         u16 = sr_uniform16(m, n, cfg.seed, t, cfg.layer_id)
     r = (K + np.asarray(u16, np.int64)) >> 16          # floor division by 2^16
@@ -417,16 +421,17 @@ def stochastic_round_rescale(Wq, sW, U, cfg: Config, t: int, u16=None):
     default, stochastic_round_update) is biased there; this variant is the
     plainest reading that keeps the rounding unbiased: make the grid fit.
 
-    With X and K = ceil(X) as in stochastic_round_update, each element's value
+    With X and K = rint(X) as in stochastic_round_update, each element's value
     in units of 2^-16 code is the integer T = q * 2^16 + K (T = q * 2^16 where X
     is NaN).  Per group g of 256 consecutive elements, A = max |T|:
       A <= 127 * 2^16: the codes are those of stochastic_round_update (no
                        element can reach the clamp) and the scale is kept;
       otherwise:       rho = (127 * 2^16) / A and s'_g = s_g / rho (IEEE float32
                        divisions); Z = fl(T) * rho (float32, fl the nearest
-                       float), K' = ceil(Z), and the code is
+                       float), K' = rint(Z) (ties to even), and the code is
                        clamp(floor((K' + d) / 2^16), -127, 127) with the same
-                       draw d.  E[code' s'] = T 2^-16 s: still unbiased.
+                       draw d.  E[code' s'] = T 2^-16 s up to the nearest-point
+                       rounding of Z: still unbiased, and odd in T.
     Returns (codes, scales)."""
     m, n = Wq.shape
     e = np.arange(m * n, dtype=np.int64).reshape(m, n)
@@ -436,7 +441,7 @@ def stochastic_round_rescale(Wq, sW, U, cfg: Config, t: int, u16=None):
         cp = (c * F32(65536.0)).astype(np.float32)
         X = (np.asarray(U, np.float32) * cp[e // cfg.w_group]).astype(np.float32)
         nan = np.isnan(X)
-        K = np.ceil(np.clip(np.where(nan, F32(0), X), F32(-2.0 ** 30), F32(2.0 ** 30))).astype(np.int64)
+        K = np.rint(np.clip(np.where(nan, F32(0), X), F32(-2.0 ** 30), F32(2.0 ** 30))).astype(np.int64)
     if u16 is None:
         u16 = sr_uniform16(m, n, cfg.seed, t, cfg.layer_id)
     d = np.asarray(u16, np.int64)
@@ -451,7 +456,7 @@ def stochastic_round_rescale(Wq, sW, U, cfg: Config, t: int, u16=None):
     s_new = sW.copy()
     s_new[grow] = (sW[grow] / rho[grow]).astype(np.float32)
     Z = (flatT.astype(np.float32) * rho[g]).astype(np.float32)
-    Kp = np.where(grow[g], np.ceil(Z).astype(np.int64), flatT)
+    Kp = np.where(grow[g], np.rint(Z).astype(np.int64), flatT)
     out = np.clip((Kp + flatd) >> 16, -INT8_QMAX, INT8_QMAX)
     return out.reshape(m, n).astype(np.int8), s_new
 

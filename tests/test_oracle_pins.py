@@ -329,7 +329,9 @@ def test_sr_unbiased_over_a_million_draws(x):
     phi = float(np.float32(x)) - f
     mean = out.astype(np.float64).mean()
     sd = math.sqrt(max(phi * (1 - phi), 1e-12) / (m * n))
-    assert abs(mean - float(np.float32(x))) <= 5 * sd + 2 ** -16
+    # the draws' mean is within 5 sd of x, plus the 2^-17 code of the nearest-point
+    # rounding of the update onto the 2^-16 draw grid
+    assert abs(mean - float(np.float32(x))) <= 5 * sd + 2 ** -17
     assert set(np.unique(out).tolist()) <= {f, f + 1}
 
 
@@ -362,14 +364,16 @@ def test_sr_group_index_is_flattened_logical():
     assert np.all(np.abs(out - expect) < 1.0)
 
 
-@pytest.mark.parametrize("X", [0.0, 1.0, 0.25, 0.5, 32767.5, 65535.25, 65536.0, 98304.75, -0.5, -1.0,
-                               -65536.0, -70000.1, 3.0e6, -3.0e6 + 0.5])
+@pytest.mark.parametrize("X", [0.0, 1.0, 0.25, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 32767.5, 65535.25, 65536.0,
+                               98304.75, -1.0, -65536.0, -70000.1, 3.0e6, -3.0e6 + 0.5])
 def test_sr_exhaustive_over_the_draw_space(X):
     # alpha = 1, s_g = 2^16: c' = 1, so the update in units of 2^-16 code is X itself.
     # Over all 2^16 draws the rounded result takes only the two neighbouring codes,
-    # and the draws sum to ceil(X) exactly: the mean is ceil(X) / 2^16, the value
-    # on the draw grid nearest above X (a floor, a missing draw or an off-by-one
-    # in the shift changes the sum).
+    # and the draws sum to rint(X) exactly (nearest integer, ties to even): the mean
+    # is X / 2^16 rounded to the nearest point of the draw grid.  A ceiling or a
+    # floor in place of the nearest point, a missing draw or an off-by-one in the
+    # shift changes the sum (the ties 0.5, 1.5, 2.5, -0.5, -1.5, -2.5 and 32767.5
+    # each separate rint from ceil, floor and round-half-away).
     W = np.zeros((256, 256), np.int8)
     sW = np.full(256, 65536.0, np.float32)
     U = np.full((256, 256), X, np.float32)
@@ -378,7 +382,53 @@ def test_sr_exhaustive_over_the_draw_space(X):
     Xf = float(np.float32(X))
     lo = math.floor(Xf / 65536.0)
     assert set(np.unique(out).tolist()) <= {lo, lo + 1}
-    assert int(out.astype(np.int64).sum()) == math.ceil(Xf)
+    assert int(out.astype(np.int64).sum()) == round(Xf)      # Python's round: ties to even
+
+
+def _draw_space_sums(X):
+    """For each value of X (the update in units of 2^-16 code), the sum of the
+    oracle's code changes over all 2^16 draws: one row of 2^16 elements per value."""
+    X = np.asarray(X, np.float32)
+    out = np.empty(X.size, np.int64)
+    rows = 32
+    d = np.tile(np.arange(65536, dtype=np.uint32), (rows, 1))
+    for b in range(0, X.size, rows):
+        x = X[b:b + rows]
+        m = x.size
+        W = np.zeros((m, 65536), np.int8)
+        sW = np.full(m * 256, 65536.0, np.float32)
+        U = np.repeat(x[:, None], 65536, axis=1)
+        cfg = O.Config(m=m, n=65536, r=1, alpha=1.0)
+        q = O.stochastic_round_update(W, sW, U, cfg, 1, u16=d[:m])
+        out[b:b + m] = q.astype(np.int64).sum(axis=1)
+    return out
+
+
+def _dense_update_grid():
+    # fractions i / 256 on both sides of integers of both parities and signs
+    f = np.arange(256, dtype=np.float64) / 256.0
+    return np.concatenate([k + f for k in (-3.0, -2.0, 2.0, 3.0, 1000.0, 1001.0)]).astype(np.float32)
+
+
+def test_sr_expected_update_is_odd_in_the_update():
+    # E[xi(-x)] = -E[xi(x)] exactly over the whole draw space, for non-integer
+    # updates too: an update and its negation move the weight by opposite amounts
+    # on average.  A ceiling (or floor) on the draw grid fails at every
+    # non-integer X: ceil(X) + ceil(-X) = 1 there.
+    X = _dense_update_grid()
+    X = X[X != np.rint(X)]
+    np.testing.assert_array_equal(_draw_space_sums(X) + _draw_space_sums(-X), 0)
+
+
+def test_sr_no_drift_over_a_dense_grid_of_updates():
+    # The exact expected change (sum over all draws) minus the update, averaged
+    # over a dense grid of fractional parts, is zero: the residue of the
+    # nearest-point rounding has no sign.  Each value is also within half a draw
+    # step of its update.  A ceiling leaves a mean residue of +1/2 step.
+    X = _dense_update_grid()
+    res = _draw_space_sums(X).astype(np.float64) - X.astype(np.float64)
+    assert np.max(np.abs(res)) <= 0.5
+    assert abs(res.mean()) <= 1e-12
 
 
 def test_sr_nan_keeps_code_inf_and_huge_saturate():
@@ -411,7 +461,7 @@ def test_sr_small_updates_keep_their_mean():
     m, n = 1000, 1000
     out = _sr(np.zeros((m, n), np.int8), np.ones(-(-m * n // 256), np.float32),
               np.full((m, n), 1e-3, np.float32), seed=5)
-    assert abs(out.mean() - 1e-3) < 5 * np.sqrt(1e-3 / (m * n)) + 2 ** -16
+    assert abs(out.mean() - 1e-3) < 5 * np.sqrt(1e-3 / (m * n)) + 2 ** -17
 
 
 # ---------------------------------------------------------------- re-scaling instead of saturating
@@ -434,7 +484,7 @@ def test_rescale_equals_saturating_inside_the_grid():
                                   (-90, -100 * 65536 - 12345.25), (0, 2.0 ** 31)])
 def test_rescale_exhaustive_over_the_draw_space(q0, X):
     # alpha = 1, s_g = 2^16: c' = 1, so every element of the 256 x 256 array has the
-    # same value T = q0 2^16 + ceil(X) (X clipped to 2^30) in units of 2^-16 code,
+    # same value T = q0 2^16 + rint(X) (X clipped to 2^30) in units of 2^-16 code,
     # outside the grid, and meets each 16-bit draw once.  Every group is re-scaled
     # to the same s', so the codes' sum over the draws is their exact mean: the
     # value q0 s + X 2^-16 s must come back as sum / 2^16 * s' up to float32
@@ -445,7 +495,7 @@ def test_rescale_exhaustive_over_the_draw_space(q0, X):
     U = np.full((256, 256), X, np.float32)
     cfg = O.Config(m=256, n=256, r=1, alpha=1.0)
     q, s2 = O.stochastic_round_rescale(W, sW, U, cfg, 1, u16=np.arange(65536, dtype=np.uint32).reshape(256, 256))
-    T = q0 * 65536 + math.ceil(max(-2.0 ** 30, min(2.0 ** 30, float(np.float32(X)))))
+    T = q0 * 65536 + round(max(-2.0 ** 30, min(2.0 ** 30, float(np.float32(X)))))
     assert abs(T) > 127 * 65536
     assert np.all(s2 == s2[0]) and s2[0] > sW[0]
     assert abs(float(s2[0]) - 65536.0 * abs(T) / (127 * 65536)) <= 3e-7 * float(s2[0])
