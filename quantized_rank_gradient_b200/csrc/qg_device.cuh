@@ -201,6 +201,44 @@ QG_DEV void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[32]) {
 
 QG_DEV void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// The same wait with the destination registers of the loads it waits for tied
+// to it, so that the compiler schedules no use of them before the wait.  With
+// a load of the next chunk in flight while this one is computed, the tie is
+// what keeps each chunk's arithmetic behind its own wait.
+QG_DEV void tmem_ld_wait(uint32_t (&v)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]),
+                 "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]),
+                 "+r"(v[14]), "+r"(v[15])
+               :
+               : "memory");
+}
+
+QG_DEV void tmem_ld_wait(uint32_t (&v)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]),
+                 "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]),
+                 "+r"(v[14]), "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]),
+                 "+r"(v[20]), "+r"(v[21]), "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]),
+                 "+r"(v[26]), "+r"(v[27]), "+r"(v[28]), "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
+               :
+               : "memory");
+}
+
+// p, produced afresh by an empty asm statement each time it is evaluated.  A
+// lane-varying predicate (a row past the matrix's edge, a row that takes
+// another arithmetic path) that guards work inside a loop which also issues
+// warp-collective .sync.aligned tcgen05 instructions is read through this in
+// every iteration: the compiler then cannot see it as loop-invariant and
+// cannot unswitch the loop into one copy per predicate value, which would
+// leave the lanes of one warp at two different copies of an instruction that
+// all of them must execute together.
+QG_DEV bool lane_pred(bool p) {
+  uint32_t v = p ? 1u : 0u;
+  asm volatile("" : "+r"(v));
+  return v != 0u;
+}
+
 // ------------------------------------------------------------------ CTA pairs (clusters of 2)
 
 QG_DEV uint32_t cluster_ctarank() {

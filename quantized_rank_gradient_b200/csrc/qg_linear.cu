@@ -120,12 +120,15 @@ struct StoreBF16Epi {
     const int c0 = ep.group * nchunk;
     const int c1 = min(c0 + nchunk, (ncols + 31) >> 5);
     uint16_t* drow = a.D + static_cast<int64_t>(grow) * a.ldd + j0;
+    __syncwarp();
 #pragma unroll 1
     for (int c = c0; c < c1; ++c) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(taddr + c * 32, v);
-      tmem_ld_wait();
-      if (!ok) continue;
+      tmem_ld_wait(v);
+      // ok varies across the lanes at the matrix's last row; re-read per chunk
+      // so that the loop is not unswitched around the warp-collective load
+      if (!lane_pred(ok)) continue;
       uint32_t packed[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {

@@ -265,19 +265,27 @@ struct AdamEpi {
     }
     float amax_m = 0.f, amax_vv = 0.f, mmin = __int_as_float(0x7f800000), vmin = __int_as_float(0x7f800000);
 
+    // The loop control of both passes is warp-uniform (s0, s1 depend on the
+    // tile only); the lane-varying row predicate guards the arithmetic alone and
+    // is re-read per sub-chunk (lane_pred).
+    auto p1 = [&](const uint32_t (&v)[16], int s, const uint4& qm, const uint4& qv) {
+      if (!lane_pred(row_ok)) return;
+      const int valid = ncols - s * 16;
+      if (valid >= 16)
+        pass1_sub<true>(a, v, qm, qv, sm, sv, valid, amax_m, amax_vv, mmin, vmin);
+      else
+        pass1_sub<false>(a, v, qm, qv, sm, sv, valid, amax_m, amax_vv, mmin, vmin);
+    };
+    // Each sub-chunk's moment codes are read from shared memory while its
+    // accumulators are on their way from tensor memory.
+    __syncwarp();
 #pragma unroll 1
     for (int s = s0; s < s1; ++s) {
       uint32_t v[16];
       tmem_ld_32x32b_x16(taddr + s * 16, v);
-      tmem_ld_wait();
-      if (row_ok) {
-        const uint4 qm = side_granule(side, row, s), qv = side_granule(side + 32768, row, s);
-        const int valid = ncols - s * 16;
-        if (valid >= 16)
-          pass1_sub<true>(a, v, qm, qv, sm, sv, valid, amax_m, amax_vv, mmin, vmin);
-        else
-          pass1_sub<false>(a, v, qm, qv, sm, sv, valid, amax_m, amax_vv, mmin, vmin);
-      }
+      const uint4 qm = side_granule(side, row, s), qv = side_granule(side + 32768, row, s);
+      tmem_ld_wait(v);
+      p1(v, s, qm, qv);
     }
 
     // a non-finite gradient reaches the maxima (they propagate NaN and Inf)
@@ -310,18 +318,23 @@ struct AdamEpi {
     const float inv_m = live_m ? __fdiv_rn(127.0f, amax_m) : 0.f;
     const float inv_v = live_v ? __fdiv_rn(127.0f, amax_v) : 0.f;
 
+    // both predicates vary across the lanes of a warp (exact depends on the
+    // row's maxima), so both are re-read per sub-chunk
+    auto p2 = [&](const uint32_t (&v)[16], int s, const uint4& qm, const uint4& qv) {
+      if (!lane_pred(row_ok)) return;
+      if (lane_pred(exact))
+        pass2_sub<true>(a, v, qm, qv, sm, sv, inv_m, inv_v, nrow + s * 16, mrow + s * 16, vrow + s * 16);
+      else
+        pass2_sub<false>(a, v, qm, qv, sm, sv, inv_m, inv_v, nrow + s * 16, mrow + s * 16, vrow + s * 16);
+    };
+    __syncwarp();
 #pragma unroll 1
     for (int s = s0; s < s1; ++s) {
       uint32_t v[16];
       tmem_ld_32x32b_x16(taddr + s * 16, v);
-      tmem_ld_wait();
-      if (row_ok) {
-        const uint4 qm = side_granule(side, row, s), qv = side_granule(side + 32768, row, s);
-        if (exact)
-          pass2_sub<true>(a, v, qm, qv, sm, sv, inv_m, inv_v, nrow + s * 16, mrow + s * 16, vrow + s * 16);
-        else
-          pass2_sub<false>(a, v, qm, qv, sm, sv, inv_m, inv_v, nrow + s * 16, mrow + s * 16, vrow + s * 16);
-      }
+      const uint4 qm = side_granule(side, row, s), qv = side_granule(side + 32768, row, s);
+      tmem_ld_wait(v);
+      p2(v, s, qm, qv);
     }
     if (row_ok && ep.group == 0) {
       a.sM[static_cast<int64_t>(arow) * a.nblk + nb] = s_m;
@@ -384,16 +397,17 @@ struct StochRoundEpi {
 
   // One 32-column chunk: W codes in (wa, wb), U from TMEM, draws d; the new codes
   // in out[8].  With X = U c' (the update in units of 2^-16 code) and
-  // K = ceil(X), the new code is clamp(q + floor((K + draw) / 2^16), -127, 127),
-  // and a NaN X keeps q.
+  // K = rint(X) (nearest, ties to even), the new code is
+  // clamp(q + floor((K + draw) / 2^16), -127, 127), and a NaN X keeps q.
   //
-  // Fast form, valid while |X| < 2^22: fadd.rp(X, 1.5 * 2^23) has the bits
-  // 0x4B400000 + K; adding the draw less 0x4B400000 and q * 2^16 leaves
-  // K + draw + q * 2^16, whose bits [16, 32) are q + r with
-  // r = floor((K + draw) / 2^16) (|q + r| <= 191).  Two such sums give one pair
-  // of 16-bit lanes, clamped to [-127, 127] by one max and one min on both
-  // lanes; the low bytes of four lanes are the four new codes.  When |X|
-  // reaches 2^22, or X is NaN, the chunk is redone in the general form.
+  // Fast form, valid while |X| < 2^22: fadd.rn(X, 1.5 * 2^23) has the bits
+  // 0x4B400000 + K (the sum lies in [2^23, 2^24), where the float32 step is 1,
+  // and 1.5 * 2^23 is even, so ties go to the even K); adding the draw less
+  // 0x4B400000 and q * 2^16 leaves K + draw + q * 2^16, whose bits [16, 32) are
+  // q + r with r = floor((K + draw) / 2^16) (|q + r| <= 191).  Two such sums
+  // give one pair of 16-bit lanes, clamped to [-127, 127] by one max and one
+  // min on both lanes; the low bytes of four lanes are the four new codes.
+  // When |X| reaches 2^22, or X is NaN, the chunk is redone in the general form.
   //
   // kTrack: also the largest and smallest T = q 2^16 + K over the chunk (K = 0
   // where X is NaN), each element's value in units of 2^-16 code; in the fast
@@ -410,7 +424,7 @@ struct StochRoundEpi {
       const float cp = (kOneFactor || k < split) ? cp0 : cp1;
       const float X = __fmul_rn(__uint_as_float(U[k]), cp);
       mx = max_nan_abs(mx, X);
-      const uint32_t tb = __float_as_uint(__fadd_ru(X, kMagic));
+      const uint32_t tb = __float_as_uint(__fadd_rn(X, kMagic));
       const uint32_t dq = prmt(d[k >> 1], 0xB4C00000u, (k & 1) ? 0x7632u : 0x7610u);
       const uint32_t wsel = 0x44u | (static_cast<uint32_t>(k & 3) << 8) | (static_cast<uint32_t>((k & 3) | 8) << 12);
       const uint32_t q16 = prmt(word_of(k < 16 ? wa : wb, (k >> 2) & 3), 0u, wsel);
@@ -434,7 +448,7 @@ struct StochRoundEpi {
         const int q = static_cast<int8_t>((word_of(w, (k >> 2) & 3) >> (8 * (k & 3))) & 0xFFu);
         int v = q, K = 0;
         if (X == X) {
-          K = __float2int_ru(fminf(fmaxf(X, -1073741824.0f), 1073741824.0f));
+          K = __float2int_rn(fminf(fmaxf(X, -1073741824.0f), 1073741824.0f));
           const int draw = static_cast<int>((d[k >> 1] >> (16 * (k & 1))) & 0xFFFFu);
           v = min(max(q + ((K + draw) >> 16), -127), 127);
         }
@@ -468,13 +482,21 @@ struct StochRoundEpi {
     if (kOneGroup && row_ok) cp_row = update_factor(a.alpha, a.sW[(static_cast<int64_t>(irow) * N + j0) >> 8]);
     int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + j0;
     const PhiloxRoundKeys rk = philox_round_keys(a.key);
+    // The chunk's tensor-memory load is in flight while its Philox draws are
+    // formed (pure ALU work, computed for every lane: a row past the matrix's
+    // edge draws for nothing).  The loop control is warp-uniform; the
+    // lane-varying row predicate guards the rounding and the stores alone and
+    // is re-read per chunk (lane_pred).
+    __syncwarp();
 #pragma unroll 1
     for (int c = c0; c < c1; ++c) {
       uint32_t U[32];
       tmem_ld_32x32b_x32(taddr + c * 32, U);
-      tmem_ld_wait();
-      if (!row_ok) continue;
       const int jc = c * 32;
+      uint32_t d[16];
+      draws(a, rk, irow, j0 + jc, d);
+      tmem_ld_wait(U);
+      if (!lane_pred(row_ok)) continue;
       const int valid = min(32, ncols - jc);
       const int64_t e0 = static_cast<int64_t>(irow) * N + j0 + jc;
       float cp0 = cp_row, cp1 = cp_row;
@@ -486,8 +508,6 @@ struct StochRoundEpi {
         split = g1 != g0 ? static_cast<int>((g1 << 8) - e0) : 32;
       }
       const uint4 wa = side_granule(side, row, 2 * c), wb = side_granule(side, row, 2 * c + 1);
-      uint32_t d[16];
-      draws(a, rk, irow, j0 + jc, d);
       uint32_t out[8];
       sr_chunk<kOneGroup>(U, wa, wb, d, cp0, cp1, split, out);
       if (valid == 32) {
@@ -513,14 +533,14 @@ struct StochRoundEpi {
 // ------------------------------------------------------------------ a4 + a5, re-scaling variant
 
 // A weight group that the update would carry off the INT8 grid gets a larger
-// scale instead of saturating.  With X = U c' and K = ceil(X) as above, every
+// scale instead of saturating.  With X = U c' and K = rint(X) as above, every
 // element's value in units of 2^-16 code is the integer T = q 2^16 + K
 // (T = q 2^16 where X is NaN); per group, A = max |T|.
 //   A <= 127 2^16: the codes are those of the saturating form (no element can
 //                  reach the clamp) and the scale stays;
 //   otherwise:     rho = (127 2^16) / A and s' = s / rho (IEEE float32
 //                  divisions), and every code of the group becomes
-//                  clamp(floor((ceil(fl(T) rho) + draw) / 2^16), -127, 127)
+//                  clamp(floor((rint(fl(T) rho) + draw) / 2^16), -127, 127)
 //                  with the same draw, fl(T) the nearest float32.
 // The expected value of code' s' stays q s + alpha U (up to the 2^-16 draw
 // grid and float32 rounding).  Needs n % 256 == 0, so that a group is one row
@@ -540,10 +560,10 @@ struct StochRoundRescaleEpi : StochRoundEpi {
       const float X = __fmul_rn(__uint_as_float(U[k]), cp);
       const uint4& w = k < 16 ? wa : wb;
       const int q = static_cast<int8_t>((word_of(w, (k >> 2) & 3) >> (8 * (k & 3))) & 0xFFu);
-      const int K = X == X ? __float2int_ru(fminf(fmaxf(X, -1073741824.0f), 1073741824.0f)) : 0;
+      const int K = X == X ? __float2int_rn(fminf(fmaxf(X, -1073741824.0f), 1073741824.0f)) : 0;
       const float Z = __fmul_rn(__int2float_rn(q * 65536 + K), rho);
       const int draw = static_cast<int>((d[k >> 1] >> (16 * (k & 1))) & 0xFFFFu);
-      const int v = min(max((__float2int_ru(Z) + draw) >> 16, -127), 127);
+      const int v = min(max((__float2int_rn(Z) + draw) >> 16, -127), 127);
       const uint32_t sh = 8 * (k & 3);
       if ((k & 3) == 0) out[k >> 2] = 0u;
       out[k >> 2] |= (static_cast<uint32_t>(v) & 0xFFu) << sh;
@@ -568,12 +588,13 @@ struct StochRoundRescaleEpi : StochRoundEpi {
     int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + j0;
     const PhiloxRoundKeys rk = philox_round_keys(a.key);
     int tmax = INT_MIN, tmin = INT_MAX;
+    __syncwarp();
 #pragma unroll 1
     for (int c = c0; c < c0 + nchunk; ++c) {
       uint32_t U[32];
       tmem_ld_32x32b_x32(taddr + c * 32, U);
-      tmem_ld_wait();
-      if (!row_ok) continue;
+      tmem_ld_wait(U);
+      if (!lane_pred(row_ok)) continue;
       const uint4 wa = side_granule(side, row, 2 * c), wb = side_granule(side, row, 2 * c + 1);
       uint32_t d[16];
       draws(a, rk, irow, j0 + c * 32, d);
@@ -598,12 +619,13 @@ struct StochRoundRescaleEpi : StochRoundEpi {
     const bool grow = row_ok && s > 0.f && amax > static_cast<uint32_t>(kLimit);
     if (!__any_sync(0xFFFFFFFFu, grow)) return;
     const float rho = grow ? __fdiv_rn(static_cast<float>(kLimit), __uint2float_rn(amax)) : 1.f;
+    __syncwarp();
 #pragma unroll 1
     for (int c = c0; c < c0 + nchunk; ++c) {
       uint32_t U[32];
       tmem_ld_32x32b_x32(taddr + c * 32, U);
-      tmem_ld_wait();
-      if (!grow) continue;
+      tmem_ld_wait(U);
+      if (!lane_pred(grow)) continue;
       const uint4 wa = side_granule(side, row, 2 * c), wb = side_granule(side, row, 2 * c + 1);
       uint32_t d[16];
       draws(a, rk, irow, j0 + c * 32, d);
@@ -637,11 +659,12 @@ struct StoreF32Epi {
     const int nchunk = BN / 32 / ep.groups;
     const int c0 = ep.group * nchunk;
     const int c1 = min(c0 + nchunk, (ncols + 31) >> 5);
+    __syncwarp();
     for (int c = c0; c < c1; ++c) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(taddr + c * 32, v);
-      tmem_ld_wait();
-      if (!ok) continue;
+      tmem_ld_wait(v);
+      if (!lane_pred(ok)) continue;
       float* d = a.D + static_cast<int64_t>(grow) * a.ldd + j0 + c * 32;
       const int valid = ncols - c * 32;
       if (a.accumulate) {
