@@ -359,15 +359,14 @@ def sr_uniform16(m, n, seed, t, layer_id):
     (seed low 32 bits, seed high 32 bits)): one Philox call serves eight
     consecutive elements of a row, and every row starts a call.
     """
-    i = np.arange(m, dtype=np.uint64)[:, None]
-    j = np.arange(n, dtype=np.uint64)[None, :]
-    call = np.broadcast_to(j >> np.uint64(3), (m, n))
-    row = np.broadcast_to(i, (m, n))
-    w = philox4x32_10(call.ravel(), row.ravel(), t, layer_id, seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
-    sel = np.broadcast_to(((j >> np.uint64(1)) & np.uint64(3)).astype(np.int64), (m, n)).ravel()
-    words = np.stack(w, axis=0)[sel, np.arange(m * n)]
-    shift = np.broadcast_to(((j & np.uint64(1)) * np.uint64(16)).astype(np.uint32), (m, n)).ravel()
-    return ((words >> shift) & np.uint32(0xFFFF)).reshape(m, n)
+    calls = -(-n // 8)
+    row = np.repeat(np.arange(m, dtype=np.uint64), calls)          # call (i, c) for c = j / 8
+    call = np.tile(np.arange(calls, dtype=np.uint64), m)
+    w = philox4x32_10(call, row, t, layer_id, seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
+    words = np.stack(w, axis=1).reshape(m, calls, 4)                 # [i, c, k]: word k of call (i, c)
+    halves = np.stack([words & np.uint32(0xFFFF), words >> np.uint32(16)], axis=3)  # [i, c, k, h]
+    # element j = 8 c + 2 k + h: word k = (j / 2) mod 4, half h = j mod 2
+    return halves.reshape(m, calls * 8)[:, :n].astype(np.uint32)
 
 
 def stochastic_round_update(Wq, sW, U, cfg: Config, t: int, u16=None):

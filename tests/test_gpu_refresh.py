@@ -216,3 +216,117 @@ def test_refresh_moment_policy_matches_oracle(policy, side):
         np.testing.assert_allclose(gs, os_, rtol=1e-4, atol=0)
         assert np.abs(gq.astype(np.int32) - oq.astype(np.int32)).max() <= 1
     assert gl.status() == qg.QG_OK
+
+
+# ---------------------------------------------------------------- LLaMA-7B shapes, r = 1024 (k = 1040)
+
+def test_refresh_gap_input_r1024_matches_oracle_subspace():
+    # k = 1040: the Jacobi runs a 65-block tournament, the Cholesky takes many
+    # 32-wide panels and the Gram matrices are split over K.  The top 1024
+    # singular values lie in [0.2, 1] (relative neighbour gaps of 0.4 % and
+    # less), so single columns are not stable under float32 rounding but every
+    # leading subspace is: the top 128, 256, 512 and all 1024 directions must
+    # agree with the oracle's (principal cosines >= 0.999).
+    m = n = 4096
+    r = 1024
+    G, Gb = synth.gap_gradient(m, n, r, seed=77)
+    ost, oinfo, gl, info, Pg = _refresh_pair(m, n, r, G, Gb, seed=5, layer_id=9)
+    assert info.refreshed == 1 and info.n_refresh == 1
+    Po = oinfo["P"]
+    for j in (128, 256, 512, 1024):
+        cos = principal_cosines(Pg[:, :j], Po[:, :j])
+        assert cos.min() >= 0.999, (j, cos.min())
+    G64 = np.asarray(G, np.float64)
+    cos = principal_cosines(Pg, O.exact_topr(G64, r)[0])
+    assert cos.min() >= 0.999, cos.min()
+    np.testing.assert_allclose(Pg.T @ Pg, np.eye(r), atol=2e-3)
+    assert gl.status() == qg.QG_OK
+
+
+def test_refresh_noise_dominated_4096x11008_leading_directions():
+    # The gate-projection shape at r = 1024 with a signal whose leading
+    # singular values stand clear of the noise edge 1e-4 (sqrt(m) + sqrt(n)):
+    # the well-separated leading block must agree with the oracle's.
+    m, n, r = 4096, 11008, 1024
+    gen = synth.lowrank_gradient(m, n, rank=256, s0=0.1, decay=0.8, sigma=1e-4, seed=4096)
+    G, Gb = gen.draw(0)
+    ost, oinfo, gl, info, Pg = _refresh_pair(m, n, r, G, Gb, seed=6, layer_id=4)
+    edge = 1e-4 * (np.sqrt(m) + np.sqrt(n))
+    k_sig = leading_block(np.linalg.svd(G.astype(np.float64), compute_uv=False), edge)
+    assert k_sig >= 4
+    cos = principal_cosines(Pg[:, :k_sig], oinfo["P"][:, :k_sig])
+    assert cos.min() >= 0.999, (k_sig, cos.min())
+    np.testing.assert_allclose(Pg.T @ Pg, np.eye(r), atol=2e-3)
+    assert gl.status() == qg.QG_OK
+
+
+# ---------------------------------------------------------------- the schedule on drifting gradients
+
+def _schedule_parity(m, n, r, delta0, steps, draw):
+    """Runs qg_refresh (force only at t = 0) + qg_step and the oracle's refresh +
+    step on the same gradients, the oracle taking the GPU's INT4 projection
+    after every refresh (teacher forcing).  Returns the refreshes as
+    (t, gpu CosSim, oracle CosSim, delta after)."""
+    oc = O.Config(m=m, n=n, r=r, delta0=delta0, gamma=0.4, seed=21, layer_id=5)
+    Wq, sW = synth.weight_codes(m, n, 21), synth.weight_scales(m, n, seed=21)
+    ost = O.LayerState.create(oc, Wq, sW)
+    gl = GpuLayer(oc, Wq, sW)
+    log = []
+    for t in range(steps):
+        dG, ldg, G = draw(t)
+        oi = O.refresh(ost, G, force=(t == 0))
+        info, _ = gl.refresh(dG, ldg, force=1 if t == 0 else 0)
+        assert bool(info.refreshed) == (oi is not None), t
+        if oi is not None:
+            assert (info.delta, info.t_next, info.n_refresh) == (ost.delta, ost.t_next, ost.n_refresh), t
+            assert bool(info.has_cossim) == (oi["cossim"] is not None)
+            if oi["cossim"] is not None:
+                assert abs(info.cossim - oi["cossim"]) <= 1e-3, (t, info.cossim, oi["cossim"])
+            log.append((t, info.cossim if info.has_cossim else None, oi["cossim"], info.delta))
+            ost.Pq, ost.sP = (x.copy() for x in gl.projection())      # teacher forcing
+        gl.step(dG, ldg)
+        O.step(ost, G)
+    assert gl.sched().t == steps and gl.status() == qg.QG_OK
+    return log
+
+
+def test_schedule_parity_on_a_drifting_gradient():
+    # The refresh-stress drift law at a reduced shape: a rank-128 signal whose
+    # left singular vectors turn in fixed planes by 0.075 rad per step until
+    # step 100 and then stay.  With an interval of 20 steps the subspace turns
+    # 1.5 rad between refreshes (CosSim = |cos 1.5| = 0.07, no doubling); once
+    # it has settled CosSim is 1 and the interval doubles at every check.
+    m, n, r = 512, 1376, 128
+    gen = synth.DeviceDriftingGradient(m, n, rank=r, s0=1.0, decay=0.99, sigma=1e-4, rate=0.075, freeze=100,
+                                       seed=8, device=torch.device("cuda"))
+
+    def draw(t):
+        g = gen.draw(t)
+        return g, gen.ld, g[:, :n].float().cpu().numpy()
+
+    log = _schedule_parity(m, n, r, 20, 200, draw)
+    assert [t for t, *_ in log] == [0, 20, 40, 60, 80, 100, 120, 160]
+    assert [d for *_, d in log] == [20, 20, 20, 20, 20, 20, 40, 80]
+    turning = [c for t, c, _, _ in log if 0 < t <= 100]
+    assert max(turning) < 0.2 and min(c for t, c, _, _ in log if t > 100) > 0.9
+
+
+def test_schedule_parity_on_linear_layer_gradients():
+    # The weight-gradient model of the second refresh workload, G = D^T X over
+    # 1024 tokens (D and X drawn on the device, G formed here in float64 and
+    # rounded to bf16): the output-gradient subspace turns 1.5 rad between
+    # refreshes until step 100 and then settles.
+    m, n, r = 512, 1376, 64
+    gen = synth.DeviceLinearLayerBatch(m, n, 1024, r, 0.99, 1e-3, 0.075, 100, seed=12, device=torch.device("cuda"))
+
+    def draw(t):
+        X, D = gen.draw(t)
+        Xf = X[:, :n].double().cpu().numpy()
+        Df = D[:, :m].double().cpu().numpy()
+        G, Gb = synth.to_bf16(Df.T @ Xf)
+        dG, ldg = upload_gradient(Gb)
+        return dG, ldg, G
+
+    log = _schedule_parity(m, n, r, 20, 200, draw)
+    assert [t for t, *_ in log] == [0, 20, 40, 60, 80, 100, 120, 160]
+    assert [d for *_, d in log] == [20, 20, 20, 20, 20, 20, 40, 80]

@@ -400,3 +400,79 @@ def test_step_batch_mixed_rescale_equals_single_steps():
     for a, b in zip(singles, batched):
         np.testing.assert_array_equal(a.weights(), b.weights())
         np.testing.assert_array_equal(a.sW.cpu().numpy(), b.sW.cpu().numpy())
+
+
+# ---------------------------------------------------------------- LLaMA-7B shapes, r = 1024
+
+def _orth_layer(m, n, r, seed, layer_id, side=0):
+    # The signal of the 7B workload (rank 256, s_i = 1e-2 0.97^i, noise 1e-4) and a
+    # seeded orthonormal projection (a full SVD of a 4096 x 11008 gradient would
+    # take the oracle a minute and adds nothing to the step's parity).
+    oc = O.Config(m=m, n=n, r=r, seed=seed, layer_id=layer_id, proj_side=side)
+    Wq = synth.weight_codes(m, n, seed)
+    sW = synth.weight_scales(m, n, seed=seed)
+    gen = synth.lowrank_gradient(m, n, rank=min(256, m, n), s0=1e-2, decay=0.97, sigma=1e-4, seed=seed)
+    ost = O.LayerState.create(oc, Wq, sW)
+    O.set_projection(ost, synth.orthonormal(n if side else m, r, seed))
+    gl = GpuLayer(oc, Wq, sW)
+    gl.set_projection(ost.Pq, ost.sP)
+    return ost, gl, gen
+
+
+@pytest.mark.parametrize("m,n", [(4096, 4096), (4096, 11008), (11008, 4096)])
+def test_step_parity_llama7b_shapes_r1024(m, n):
+    # The shapes and rank the throughput is quoted on.  A 4096 x 11008 step has
+    # 43 x 4 pair tiles in a2+a3 and 16 x 43 in a4+a5 on 74 CTA pairs, so every
+    # pair runs several tiles: both TMEM accumulators, the accumulator phase
+    # flip, the side-tile ring past its depth and both exchange slots are used;
+    # the 11008 x 4096 case runs a2+a3 with K = 11008 (172 k-blocks through the
+    # ring).
+    r = 1024
+    ost, gl, gen = _orth_layer(m, n, r, seed=m + 3 * n, layer_id=6)
+    for t in range(2):
+        G, Gb = gen.draw(t)
+        dG, ldg = upload_gradient(Gb)
+        gl.step(dG, ldg)
+        inter = O.step(ost, G)
+        if t == 0:
+            assert float((gl.scratch_N() != O.bf16_bits(inter["N"])).mean()) <= 1e-3
+        compare_state(ost, gl, f"{m} x {n}, step {t + 1}")
+    assert gl.status() == qg.QG_OK
+
+
+def _run_batch(layers, grads):
+    cfgs = [gl.cfg for gl in layers]
+    arr = (qg.POINTER(qg.qg_config) * len(cfgs))(*[qg.ctypes.pointer(c) for c in cfgs])
+    wsb = qg.qg_step_batch_workspace_bytes(arr, len(cfgs))
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    hs = (c_void_p * len(layers))(*[gl.h.value for gl in layers])
+    gs = (c_void_p * len(layers))(*[g.data_ptr() for g, _ in grads])
+    lds = (qg.c_int64 * len(layers))(*[ld for _, ld in grads])
+    qg.check(qg.qg_step_batch(hs, gs, lds, len(layers), ws.data_ptr(), wsb, stream()))
+    torch.cuda.synchronize()
+
+
+def test_step_batch_multi_tile_matches_oracle():
+    # One qg_step_batch launch pair over seven matrices: a2+a3 has 436 pair
+    # tiles and a4+a5 2174 on 74 CTA pairs, so every pair walks at least five
+    # tiles of several problems (persistent loop, both accumulators and phases,
+    # side ring and exchange slots on their second and later rounds), one
+    # problem has K = 11008, and two are ragged.  Every matrix is compared with
+    # the oracle, two steps in a row.
+    specs = [(4096, 4096, 1024), (4096, 4096, 1024), (4096, 4096, 1024), (11008, 4096, 1024),
+             (4096, 11008, 1024), (640, 1365, 96), (1376, 512, 128)]
+    osts, gls, gens = [], [], []
+    for i, (m, n, r) in enumerate(specs):
+        ost, gl, gen = _orth_layer(m, n, r, seed=100 + i, layer_id=i)
+        osts.append(ost)
+        gls.append(gl)
+        gens.append(gen)
+    for t in range(2):
+        draws = [gen.draw(t) for gen in gens]
+        grads = [upload_gradient(Gb) for _, Gb in draws]
+        _run_batch(gls, grads)
+        for i, (ost, gl, (G, _)) in enumerate(zip(osts, gls, draws)):
+            O.step(ost, G)
+            compare_state(ost, gl, f"matrix {i} {specs[i]}, step {t + 1}")
+    for gl in gls:
+        assert gl.status() == qg.QG_OK
