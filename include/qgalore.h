@@ -134,7 +134,13 @@ size_t qg_state_bytes(const qg_config* cfg);
 size_t qg_step_workspace_bytes(const qg_config* cfg);
 size_t qg_refresh_workspace_bytes(const qg_config* cfg);
 
-/* Create a layer handle over caller-owned device memory.
+/* Create a layer handle over caller-owned device memory: the per-matrix state
+ * of the AIMech Q-GaLore page, mechanism "INT4 projection and INT8 stochastic
+ * rounding" (paper section 3.2) -- INT8 master weights with their scales, the
+ * INT4 projection P_t and the previous one, and the INT8 low-rank moments
+ * (M_t^Q, V_t^Q) -- plus the layer's refresh schedule of the mechanism
+ * "layer-adaptive subspace cosine schedule" (paper section 3.1, Eq. (5)):
+ * t = 0, interval delta0, first refresh due at t = 0.
  *   d_state : >= qg_state_bytes(cfg) bytes, 256-byte aligned; zero-initialised
  *             here (moments and scales start at zero) on `stream`.
  *   d_W     : m x ldw INT8 weight codes, 16-byte aligned, ldw >= n, ldw % 16 == 0;
@@ -158,14 +164,19 @@ qg_status qg_layer_sched_set(qg_layer* layer, const qg_sched* sched);
 qg_status qg_layer_set_projection(qg_layer* layer, const uint8_t* d_Pq, const float* d_sP,
                                   int32_t keep_prev, void* stream);
 
-/* One optimizer step a1..a5 (paper section 3.2) on one matrix.
+/* One optimizer step a1..a5 (AIMech Q-GaLore page, mechanism "INT4 projection
+ * and INT8 stochastic rounding", paper section 3.2) on one matrix.
  *   d_G : m x ldg bf16 gradient, 16-byte aligned, ldg >= n, ldg % 8 == 0.
  *   d_ws: >= qg_step_workspace_bytes(cfg) bytes, 256-byte aligned.
  * Never refreshes; QG_ESTATE if no projection is installed. */
 qg_status qg_step(qg_layer* layer, const void* d_G, int64_t ldg, void* d_ws, size_t ws_bytes,
                   void* stream);
 
-/* The same step for `count` matrices in few launches: batches of up to 8
+/* The step of the AIMech Q-GaLore page, mechanism "INT4 projection and INT8
+ * stochastic rounding" (paper section 3.2), applied to `count` independent
+ * matrices (every layer of a model carries its own W, P and moments and steps
+ * on its own gradient): the same arithmetic as qg_step for each, in few
+ * launches: batches of up to 8
  * matrices, three launches per batch (dequantize the batch's projections, then
  * one persistent tcgen05 grid per GEMM stage).  With more than one batch, the
  * batches alternate between `stream` and a second stream that the library
@@ -192,16 +203,20 @@ size_t qg_step_batch_workspace_bytes(const qg_config* const* cfgs, int32_t count
  *   QG_NOALLOC_SCRATCH_BYTES (32 MiB), held by every GPU that loads the library
  *   until the process exits; every LLaMA-7B-shaped matrix at r = 1024 fits.
  *   Larger matrices are refused with QG_ESHAPE before anything is launched.
- *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.  All calls share the array and it keeps the
+ *   The first call in each CUDA context looks up the array's device address
+ *   (cudaGetSymbolAddress) with the device current; make that first call
+ *   before any stream capture.  The address is cached with the context, so a
+ *   device reset (which builds a new context and loads the array anew) makes
+ *   the next call look it up again.  All calls share the array and it keeps the
  *   previous call's contents (the step overwrites everything it reads), so
  *   calls whose GPU work overlaps, from other streams or threads, race.
  * Arguments, state handling and errors are otherwise those of qg_step. */
 #define QG_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 qg_status qg_step_noalloc(qg_layer* layer, const void* d_G, int64_t ldg, void* stream);
 
-/* Layer-adaptive subspace refresh (paper section 3.1, Eq. (5)).  Runs when
+/* Layer-adaptive subspace refresh (AIMech Q-GaLore page, mechanism
+ * "layer-adaptive subspace cosine schedule", paper section 3.1, Eq. (5); the
+ * SVD that finds the subspace: the paper-index record's abstract).  Runs when
  * force != 0 or the layer is due (t == t_next); otherwise returns QG_OK with
  * info->refreshed = 0 and touches nothing.  When it runs: randomized top-r SVD
  * of G -> new INT4 P; if a projection existed, CosSim(P_new, P_prev) on the
@@ -217,15 +232,24 @@ qg_status qg_step_noalloc(qg_layer* layer, const void* d_G, int64_t ldg, void* s
 qg_status qg_refresh(qg_layer* layer, const void* d_G, int64_t ldg, int32_t force, void* d_ws,
                      size_t ws_bytes, qg_refresh_info* info, void* stream);
 
-/* CosSim(Pa, Pb) = (1/r) sum_i sigma_i(Pa^T Pb) for float32 m x r matrices with
- * row stride ld (elements), result written to d_out[0] on the device.
+/* CosSim(Pa, Pb) = (1/r) sum_i sigma_i(Pa^T Pb), the subspace similarity of the
+ * AIMech Q-GaLore page, mechanism "layer-adaptive subspace cosine schedule"
+ * (paper section 3.1, Eq. (5)), for float32 m x r matrices with row stride ld
+ * (elements), result written to d_out[0] on the device.  The sum of the
+ * singular values is taken as the nuclear norm of Pa^T Pb through its polar
+ * factor (Newton-Schulz iteration), not by an SVD.
  * d_ws >= qg_cossim_workspace_bytes(m, r). */
 size_t qg_cossim_workspace_bytes(int32_t m, int32_t r);
 qg_status qg_cossim(const float* d_Pa, const float* d_Pb, int32_t m, int32_t r, int64_t ld,
                     float* d_out, void* d_ws, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, reads and clears the layer's device status word:
- * QG_OK, QG_ETIMEOUT or QG_ENONFINITE. */
+ * QG_OK, QG_ETIMEOUT or QG_ENONFINITE.  The pages define no error reporting;
+ * the word records the two device-side failures of the step of the AIMech
+ * Q-GaLore page, mechanism "INT4 projection and INT8 stochastic rounding"
+ * (paper section 3.2): a bounded wait that ran out, and a non-finite projected
+ * gradient R = P^T G (whose Adam update, and so the step's outputs, are then
+ * unspecified). */
 qg_status qg_layer_status(qg_layer* layer, void* stream);
 
 /* Host-only rule of the paper's layer-adaptive schedule: after a refresh at

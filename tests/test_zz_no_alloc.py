@@ -23,11 +23,11 @@ from gpu_layer import GpuLayer, stream, upload_gradient
 pytestmark = pytest.mark.gpu
 
 
-def _twin_layers(m, n, r, seed):
-    oc = O.Config(m=m, n=n, r=r, seed=seed, layer_id=7)
+def _twin_layers(m, n, r, seed, side=0):
+    oc = O.Config(m=m, n=n, r=r, seed=seed, layer_id=7, proj_side=side)
     Wq = synth.weight_codes(m, n, seed)
     sW = synth.weight_scales(m, n, seed=seed)
-    P = synth.orthonormal(m, r, seed)
+    P = synth.orthonormal(n if side else m, r, seed)
     codes, sP = O.quant_int4_groups(P.astype(np.float32))
     Pq = O.pack_int4(codes)
     a, b = GpuLayer(oc, Wq, sW), GpuLayer(oc, Wq, sW)
@@ -36,9 +36,13 @@ def _twin_layers(m, n, r, seed):
     return a, b
 
 
-@pytest.mark.parametrize("m,n,r", [(512, 1376, 128), (640, 1365, 96), (4096, 11008, 1024)])
-def test_noalloc_step_matches_workspace_step_twice(cuda_ok, m, n, r):
-    a, b = _twin_layers(m, n, r, seed=m + n)
+# Left-side layouts (P m x r, N r x n) and right-side ones (P n x r, N m x r),
+# among them the largest LLaMA-7B matrices at r = 1024 on both sides: the
+# 11008 x 4096 down projection is the one a right-side caller projects.
+@pytest.mark.parametrize("m,n,r,side", [(512, 1376, 128, 0), (640, 1365, 96, 0), (4096, 11008, 1024, 0),
+                                        (700, 300, 64, 1), (11008, 4096, 1024, 1)])
+def test_noalloc_step_matches_workspace_step_twice(cuda_ok, m, n, r, side):
+    a, b = _twin_layers(m, n, r, seed=m + n, side=side)
     gen = synth.lowrank_gradient(m, n, rank=min(64, m, n), seed=m + n)
     for t in range(2):
         _, Gb = gen.draw(t)
