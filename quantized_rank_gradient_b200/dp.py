@@ -6,7 +6,8 @@ matrix can be owned by one rank:
 
 1. every rank holds the full model's gradients of its own slice of the batch;
 2. the gradients are reduce-scattered by ownership: the owner of a matrix
-   receives the mean over the ranks;
+   receives the mean over the ranks, summed in float32 and rounded once to
+   bf16;
 3. each rank runs the optimizer step (qg_step_batch) on the matrices it owns;
 4. the updated INT8 weights are all-gathered, so that every rank holds the
    whole model for the next forward pass.  Each matrix's group scales sit
@@ -107,17 +108,34 @@ def scale_view(flat, plan, i, shape):
 
 def reduce_scatter_gradients(flat, plan, rank, group=None):
     """Mean over the ranks of every gradient, delivered to its owner: afterwards
-    this rank's shard of `flat` holds the means of the gradients it owns (the
-    other shards are left unspecified)."""
+    this rank's shard of the bf16 buffer `flat` holds the means of the
+    gradients it owns (the other shards are left unspecified).
+
+    Numerics: the local bf16 gradients are widened to float32, summed over the
+    ranks in float32 (in the collective's own order), divided by the rank count
+    in float32, and rounded once to bf16 (nearest, ties to even) on the owner:
+    G = bf16(fl32(fl32(sum_k G_k) / world)).  A bf16 sum on the wire would round
+    at every hop of a ring or tree, so its result would depend on the algorithm
+    and the rank count; in float32 the only order-dependent rounding is the
+    sum's, at most (world - 1) 2^-24 sum_k |G_k| per element, and for two ranks
+    the sum is exact whenever the two exponents are within 15 of each other.
+    The float32 copy doubles the bytes on the wire and, for the time of the
+    call, the gradient memory (26 GB for the LLaMA-7B stack)."""
     n = plan.grad_shard
     mine = flat[rank * n: (rank + 1) * n]
     if plan.world == 1:
         return mine
+    if flat.dtype != torch.bfloat16:
+        raise TypeError("the gradient buffer holds bf16, the dtype qg_step takes")
+    wide = flat.to(torch.float32)
     if dist.get_backend(group) == "nccl":
-        dist.reduce_scatter_tensor(mine, flat, op=dist.ReduceOp.AVG, group=group)
+        total = torch.empty(n, dtype=torch.float32, device=flat.device)
+        dist.reduce_scatter_tensor(total, wide, op=dist.ReduceOp.SUM, group=group)
     else:
-        dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
-        mine.div_(plan.world)
+        dist.all_reduce(wide, op=dist.ReduceOp.SUM, group=group)
+        total = wide[rank * n: (rank + 1) * n]
+    total.div_(plan.world)
+    mine.copy_(total)  # float32 -> bf16, round to nearest even
     return mine
 
 

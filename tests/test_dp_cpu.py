@@ -1,14 +1,21 @@
 """Layer-sharded data parallelism (quantized_rank_gradient_b200.dp) on CPU: two
-gloo ranks (127.0.0.1), with the oracle's optimizer step standing in for
-qg_step_batch on the owned matrices.
+and three gloo ranks (127.0.0.1), with the oracle's optimizer step standing in
+for qg_step_batch on the owned matrices.
 
-Every rank holds the gradients of its own slice of the batch for all matrices;
-after the reduce-scatter each owner steps its matrices on the mean gradient, and
-after the all-gather every rank must hold, bit for bit, the weights (codes and
-group scales) of one process that averaged the gradients and stepped every
-matrix itself.  The second case mixes projection sides and weight policies: a
-matrix whose groups are re-scaled (w_rescale = 1) changes its scales on the
-owner, and the all-gather must carry them.
+Every rank holds the bf16 gradients of its own slice of the batch for all
+matrices.  The reduce-scatter must deliver to each owner
+G = bf16(fl32(fl32(sum_k G_k) / world)): a float32 sum over the ranks, one
+float32 division and one rounding to bf16.  The local gradients differ in
+magnitude by up to 2^20 between ranks, so that some float32 sums are inexact and
+their order matters: with two ranks the float32 sum is the same in either order
+and the result is checked bit for bit; with three, every element must equal the
+rule taken in one of the three association orders, and lie within the rule's
+error bound of the exact mean.  Each owner then steps its matrices on the
+gradient it received, and after the all-gather every rank must hold, bit for
+bit, the weights (codes and group scales) of one process that stepped every
+matrix itself on those gradients.  The mixed case also varies projection sides
+and weight policies: a matrix whose groups are re-scaled (w_rescale = 1)
+changes its scales on the owner, and the all-gather must carry them.
 """
 import os
 import socket
@@ -45,11 +52,14 @@ def _initial_state(i, spec):
 
 
 def _local_gradient(rank, i, m, n):
-    # on the 2^-24 grid (|G| << 1/3): a sum over up to three ranks is exact in
-    # float32 in any order, so the mean is one correctly rounded division
+    """Rank `rank`'s bf16 gradient of matrix i (float32 values, uint16 bits).
+    The ranks' magnitudes differ (a factor 2^(10 rank) on alternate rows), so
+    the float32 sums over ranks are not all exact."""
     import synth
     G, _ = synth.lowrank_gradient(m, n, rank=16, seed=1000 * (rank + 1) + i).draw(1)
-    return (np.round(np.asarray(G, np.float64) * 2.0 ** 24) / 2.0 ** 24).astype(np.float32)
+    scale = np.ones((m, 1))
+    scale[1::2] = 2.0 ** (10 * rank)
+    return synth.to_bf16(np.asarray(G, np.float64) * scale)
 
 
 def _worker(rank, world, port, out, specs):
@@ -66,24 +76,27 @@ def _worker(rank, world, port, out, specs):
     try:
         shapes = [_spec(s)[:2] for s in specs]
         plan = dp.plan_shards(shapes, [R] * len(shapes), world)
-        flat_g = torch.zeros(world * plan.grad_shard, dtype=torch.float32)
+        flat_g = torch.zeros(world * plan.grad_shard, dtype=torch.bfloat16)
         flat_w = torch.zeros(world * plan.weight_shard, dtype=torch.uint8)
         states = [_initial_state(i, s) for i, s in enumerate(specs)]
         for i, (m, n) in enumerate(shapes):
-            dp.grad_view(flat_g, plan, i, (m, n))[:, :n] = torch.from_numpy(_local_gradient(rank, i, m, n))
+            bits = _local_gradient(rank, i, m, n)[1]
+            dp.grad_view(flat_g, plan, i, (m, n))[:, :n] = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
             dp.weight_view(flat_w, plan, i, (m, n))[:, :n] = torch.from_numpy(states[i].Wq.view(np.uint8))
             dp.scale_view(flat_w, plan, i, (m, n))[:] = torch.from_numpy(states[i].sW)
         dp.reduce_scatter_gradients(flat_g, plan, rank)
+        received = {}
         for i in plan.owned(rank):
             m, n = shapes[i]
-            G = dp.grad_view(flat_g, plan, i, (m, n))[:, :n].numpy().astype(np.float32)
+            G = dp.grad_view(flat_g, plan, i, (m, n))[:, :n].float().numpy()
+            received[i] = G.copy()
             O.step(states[i], G)
             dp.weight_view(flat_w, plan, i, (m, n))[:, :n] = torch.from_numpy(states[i].Wq.view(np.uint8))
             dp.scale_view(flat_w, plan, i, (m, n))[:] = torch.from_numpy(states[i].sW)
         dp.all_gather_weights(flat_w, plan, rank)
         W = [dp.weight_view(flat_w, plan, i, s)[:, : s[1]].numpy().view(np.int8).copy() for i, s in enumerate(shapes)]
         S = [dp.scale_view(flat_w, plan, i, s).numpy().copy() for i, s in enumerate(shapes)]
-        out.put((rank, plan.owner, plan.work, W, S))
+        out.put((rank, plan.owner, plan.work, W, S, received))
     finally:
         dist.destroy_process_group()
 
@@ -130,27 +143,39 @@ def test_gloo_ranks_match_one_process_bit_for_bit(world, specs):
         p.start()
     res = {}
     for _ in range(world):
-        rank, owner, work, W, S = out.get(timeout=180)
-        res[rank] = (owner, work, W, S)
+        rank, owner, work, W, S, got = out.get(timeout=180)
+        res[rank] = (owner, work, W, S, got)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
     assert all(res[k][0] == res[0][0] for k in range(world)) and set(res[0][0]) == set(range(world))
-    # one process: the mean gradient (an exact float32 sum, then one division)
-    # and every matrix stepped here
-    grown = 0
+    owner = res[0][0]
+    f32 = np.float32
+    grown, inexact = 0, 0
     for i, spec in enumerate(specs):
         m, n = _spec(spec)[:2]
+        g = [_local_gradient(k, i, m, n)[0].astype(np.float32) for k in range(world)]
+        G = res[owner[i]][4][i]
+        # the rule in every association order of the float32 sum
+        if world == 2:
+            orders = [(g[0] + g[1]).astype(f32)]
+        else:
+            orders = [((g[a] + g[b]).astype(f32) + g[c]).astype(f32) for a, b, c in ((0, 1, 2), (0, 2, 1), (1, 2, 0))]
+        cands = [O.bf16_round((s / f32(world)).astype(f32)) for s in orders]
+        assert np.all(np.any([G == c for c in cands], axis=0)), f"matrix {i}: a mean outside the rule"
+        exact = sum(x.astype(np.float64) for x in g)
+        inexact += int((orders[0].astype(np.float64) != exact).sum())
+        bound = (world - 1) * 2.0 ** -24 * sum(np.abs(x.astype(np.float64)) for x in g) / world
+        err = np.abs(G.astype(np.float64) - exact / world)
+        assert np.all(err <= 2.0 ** -8 * np.abs(exact / world) * (1 + 2.0 ** -23) + bound * (1 + 2.0 ** -8) + 1e-45)
+        # one process stepping every matrix on the gradient its owner received
         st = _initial_state(i, spec)
         s0 = st.sW.copy()
-        total = _local_gradient(0, i, m, n)
-        for k in range(1, world):
-            total = (total + _local_gradient(k, i, m, n)).astype(np.float32)
-        G = (total / np.float32(world)).astype(np.float32)
         O.step(st, G)
         grown += int((st.sW != s0).sum())
         for rank in range(world):
             np.testing.assert_array_equal(res[rank][2][i], st.Wq, err_msg=f"matrix {i} on rank {rank}")
             np.testing.assert_array_equal(res[rank][3][i], st.sW, err_msg=f"scales {i} on rank {rank}")
+    assert inexact > 0  # some float32 sums rounded: the rule, not an exact grid, is what is checked
     if specs is MIXED:
         assert grown > 0  # some owner changed its scales, and every rank received them
