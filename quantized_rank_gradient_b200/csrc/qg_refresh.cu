@@ -5,8 +5,9 @@
 // Top-r left singular vectors of G by randomized subspace iteration (Halko,
 // Martinsson, Tropp 2011): Omega (n x k, Rademacher from Philox), Y = G Omega,
 // Q = orth(Y); q times { Z = orth(G^T Q); Q = orth(G Z) }; B = Q^T G;
-// S = B B^T = V diag(lambda) V^T; P = Q V[:, top r].  The products with G run on
-// the tcgen05 core (bf16 operands, fp32 accumulation); orth() is shifted
+// S = B B^T = V diag(lambda) V^T; P = Q V[:, top r].  The products with G and
+// S = B B^T run on the tcgen05 core (bf16 operands, fp32 accumulation; float32
+// operands as bf16 hi + lo parts); orth() is shifted
 // Cholesky-QR (Fukaya et al. 2020) with fp32 SIMT Gram matrices and X L^-T
 // formed on the tensor cores from the explicit inverse: two passes for the
 // intermediate bases of the power iterations, three for the final Q;
@@ -37,9 +38,19 @@ constexpr float kJacobiTol = 1e-5f;
 
 size_t r256(size_t x) { return (x + 255) / 256 * 256; }
 
+// CosSim's buffers for an r x r problem: four float32 r x r matrices (C, the
+// iterate, the next iterate, the product), then, when the tensor cores take the
+// Newton-Schulz steps, four bf16 r x 3r operand stacks.
+bool ns_on_tensor_cores(int r) { return r % 32 == 0 && r >= 128; }
+size_t cossim_buffer_bytes(int r) {
+  const size_t rr = size_t(r) * r;
+  return r256(rr * 4 * 4) + (ns_on_tensor_cores(r) ? 4 * r256(rr * 3 * 2) : 0);
+}
+
 struct RefreshLayout {
-  int k, ldk, ldn4;
-  size_t P, omega, Y, Yb, Ylo, Z, Zb, Zlo, gram, gpart, linv, Li, Tt, Lih, Lil, Bm, At, Vt, lam, perm, Vsel, Pa, Pb, Ct, jx,
+  int k, ldk, ldn4, ldn8;
+  size_t P, omega, Y, Yb, Ylo, Z, Zb, Zlo, gram, gpart, linv, Li, Tt, Lih, Lil, Bm, Bh, Bl, At, Vt, lam, perm, Vsel, Pa, Pb,
+      Ct, jx,
       mom, misc, total;
 };
 
@@ -61,6 +72,7 @@ RefreshLayout refresh_layout(int m, int n, int r, int p) {
   L.k = std::min(std::min(r + p, m), n);
   L.ldk = (L.k + 7) / 8 * 8;
   L.ldn4 = (n + 3) / 4 * 4;
+  L.ldn8 = (n + 7) / 8 * 8;
   const size_t k = L.k, ldk = L.ldk;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -84,6 +96,8 @@ RefreshLayout refresh_layout(int m, int n, int r, int p) {
   L.Lih = take(k * ldk * 2);
   L.Lil = take(k * ldk * 2);
   L.Bm = take(k * L.ldn4 * 4);
+  L.Bh = take(k * L.ldn8 * 2);
+  L.Bl = take(k * L.ldn8 * 2);
   L.At = take(k * ldk * 4);
   L.Vt = take(k * ldk * 4);
   L.lam = take(k * 4);
@@ -91,7 +105,7 @@ RefreshLayout refresh_layout(int m, int n, int r, int p) {
   L.Vsel = take(k * size_t(r) * 4);
   L.Pa = take(size_t(m) * r * 4);
   L.Pb = take(size_t(m) * r * 4);
-  L.Ct = take(size_t(r) * r * 4 * 4);  // CosSim: C and three Newton-Schulz buffers
+  L.Ct = take(cossim_buffer_bytes(r));  // CosSim: C, the Newton-Schulz iterates and their bf16 operands
   L.jx = take(jacobi_scratch_bytes(L.k));
   // the rotated moments: r x n fp32 for the left projection; for the right one
   // (refresh called with m and n swapped) n x r, which is r x n here as well
@@ -336,6 +350,46 @@ __global__ void ns_shift_kernel(float* __restrict__ T, int r) {
   T[i] = __fmaf_rn(-0.5f, T[i], d);
 }
 
+// bf16 hi + lo parts of the r x r float32 matrix M (or of 1.5 I - 0.5 M when
+// kShift), written into the operand stacks of a product whose K is tripled:
+// with A' = [A_hi | A_hi | A_lo] and B' = [B_hi ; B_lo ; B_hi], A' B' is
+// A_hi B_hi + A_hi B_lo + A_lo B_hi, the float32 product up to the lo-lo term
+// and about 2^-17 relative rounding of each operand.
+//   ha (r x 3r): [hi | hi | lo]   the left operand, K-major
+//   hb (r x 3r): [hi | lo | hi]   the right operand given transposed (K-major)
+//   vb (3r x r): [hi ; lo ; hi]   the right operand as it stands (MN-major)
+// Each may be null.
+template <bool kShift>
+__global__ void ns_split_kernel(const float* __restrict__ M, int r, uint16_t* __restrict__ ha,
+                                uint16_t* __restrict__ hb, uint16_t* __restrict__ vb) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t rr = static_cast<int64_t>(r) * r;
+  if (idx >= rr) return;
+  const int64_t i = idx / r, j = idx % r;
+  float x = M[idx];
+  if (kShift) x = __fmaf_rn(-0.5f, x, i == j ? 1.5f : 0.f);
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(h)));
+  const uint16_t hu = __bfloat16_as_ushort(h), lu = __bfloat16_as_ushort(l);
+  if (ha) {
+    uint16_t* row = ha + i * 3 * r;
+    row[j] = hu;
+    row[r + j] = hu;
+    row[2 * r + j] = lu;
+  }
+  if (hb) {
+    uint16_t* row = hb + i * 3 * r;
+    row[j] = hu;
+    row[r + j] = lu;
+    row[2 * r + j] = hu;
+  }
+  if (vb) {
+    vb[idx] = hu;
+    vb[rr + idx] = lu;
+    vb[2 * rr + idx] = hu;
+  }
+}
+
 // out[0] = (1/r) sum_ij X_ij C_ij = (1/r) trace(X^T C); one block.
 __global__ void __launch_bounds__(1024) trace_product_kernel(const float* __restrict__ X, const float* __restrict__ C,
                                                              int r, float* out) {
@@ -520,29 +574,59 @@ cudaError_t jacobi(float* At, float* Vt, int64_t ld, int k, unsigned* bar, int* 
   return e;
 }
 
-// CosSim of Pa, Pb (fp32 m x r, stride ld) into d_out: C = Pb^T Pa (the
-// transpose of Pa^T Pb: the same singular values), then the nuclear norm by the
-// Newton-Schulz polar iteration above.  buf: 4 r x r floats; scal: one float.
+// CosSim of Pa, Pb (fp32 m x r, stride ld) into d_out.  The Newton-Schulz
+// iteration above runs on Y = X^T, where it reads
+//   T = Y Y^T,   Y <- (1.5 I - 0.5 T) Y,
+// two left-multiplications, from Y_0 = C' / ||C'||_F with C' = Pa^T Pb (= C^T:
+// the same singular values).  The nuclear norm is then (1/r) trace(Y C') summed
+// as sum_ij Y_ij C'_ij.  For r % 32 == 0 and r >= 128 the first
+// kNsIters - kNsPolish steps run on the tcgen05 core with bf16 hi + lo operands
+// (one launch per product, K = 3r); each step's rounding is then about 2^-17
+// of the iterate, which the iteration itself damps, and the last kNsPolish
+// steps run in float32 to bring the iterate to float32 orthogonality.
+// buf: cossim_buffer_bytes(r); scal: one float.
+constexpr int kNsPolish = 2;
+
 cudaError_t cossim_core(const float* Pa, const float* Pb, int m, int r, int64_t ld, float* buf, float* scal,
                         float* d_out, cudaStream_t s) {
   const int64_t rr = int64_t(r) * r;
   float* C = buf;
-  float* X = buf + rr;
-  float* Xn = buf + 2 * rr;
+  float* Y = buf + rr;
+  float* Yn = buf + 2 * rr;
   float* T = buf + 3 * rr;
-  cudaError_t e = sgemm(true, false, Pb, ld, Pa, ld, C, r, r, r, m, s);
+  cudaError_t e = sgemm(true, false, Pa, ld, Pb, ld, C, r, r, r, m, s);
   if (e != cudaSuccess) return e;
   const unsigned blocks = static_cast<unsigned>((rr + 255) / 256);
   inv_frobenius_kernel<<<1, 1024, 0, s>>>(C, rr, scal);
-  scale_kernel<<<blocks, 256, 0, s>>>(C, scal, X, rr);
+  scale_kernel<<<blocks, 256, 0, s>>>(C, scal, Y, rr);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  for (int it = 0; it < kNsIters; ++it) {
-    if ((e = sgemm(true, false, X, r, X, r, T, r, r, r, r, s)) != cudaSuccess) return e;
-    ns_shift_kernel<<<blocks, 256, 0, s>>>(T, r);
-    if ((e = sgemm(false, false, X, r, T, r, Xn, r, r, r, r, s)) != cudaSuccess) return e;
-    std::swap(X, Xn);
+  int it = 0;
+  if (ns_on_tensor_cores(r)) {
+    uint8_t* ops = reinterpret_cast<uint8_t*>(buf) + r256(size_t(rr) * 4 * 4);
+    const size_t stack = r256(size_t(rr) * 3 * 2);
+    uint16_t* Yha = reinterpret_cast<uint16_t*>(ops);
+    uint16_t* Yhb = reinterpret_cast<uint16_t*>(ops + stack);
+    uint16_t* Yvb = reinterpret_cast<uint16_t*>(ops + 2 * stack);
+    uint16_t* Tha = reinterpret_cast<uint16_t*>(ops + 3 * stack);
+    const int64_t l3 = 3 * int64_t(r);
+    for (; it < kNsIters - kNsPolish; ++it) {
+      ns_split_kernel<false><<<blocks, 256, 0, s>>>(Y, r, Yha, Yhb, Yvb);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      // T = Y Y^T
+      if ((e = launch_gemm_f32(Yha, l3, false, Yhb, l3, true, T, r, r, r, 3 * r, s)) != cudaSuccess) return e;
+      ns_split_kernel<true><<<blocks, 256, 0, s>>>(T, r, Tha, nullptr, nullptr);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      // Y <- (1.5 I - 0.5 T) Y
+      if ((e = launch_gemm_f32(Tha, l3, false, Yvb, r, false, Y, r, r, r, 3 * r, s)) != cudaSuccess) return e;
+    }
   }
-  trace_product_kernel<<<1, 1024, 0, s>>>(X, C, r, d_out);
+  for (; it < kNsIters; ++it) {
+    if ((e = sgemm(false, true, Y, r, Y, r, T, r, r, r, r, s)) != cudaSuccess) return e;
+    ns_shift_kernel<<<blocks, 256, 0, s>>>(T, r);
+    if ((e = sgemm(false, false, T, r, Y, r, Yn, r, r, r, r, s)) != cudaSuccess) return e;
+    std::swap(Y, Yn);
+  }
+  trace_product_kernel<<<1, 1024, 0, s>>>(Y, C, r, d_out);
   return cudaGetLastError();
 }
 
@@ -644,7 +728,7 @@ size_t refresh_scratch_bytes(int32_t m, int32_t n, int32_t r, int32_t oversample
   return refresh_layout(m, n, r, oversample).total;
 }
 
-size_t cossim_scratch_bytes(int32_t, int32_t r) { return r256(size_t(r) * r * 4 * 4) + 256; }
+size_t cossim_scratch_bytes(int32_t, int32_t r) { return cossim_buffer_bytes(r) + 256; }
 
 qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaStream_t s, float* cossim) {
   const RefreshLayout L = refresh_layout(a.m, a.n, a.r, a.oversample);
@@ -702,7 +786,20 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
   if (launch_gemm_f32(Yb, ldk, true, a.G, a.ldg, tr, Bm, L.ldn4, k, n, m, s) != cudaSuccess) return QG_ECUDA;
   if (launch_gemm_f32(Ylo, ldk, true, a.G, a.ldg, tr, Bm, L.ldn4, k, n, m, s, true) != cudaSuccess)
     return QG_ECUDA;
-  if (sgemm(false, true, Bm, L.ldn4, Bm, L.ldn4, At, ldk, k, k, n, s) != cudaSuccess) return QG_ECUDA;
+  // S = B B^T on the tensor cores: B split into bf16 hi + lo parts, three
+  // products accumulated in float32 (hi hi^T + hi lo^T + lo hi^T)
+  {
+    uint16_t* Bh = reinterpret_cast<uint16_t*>(ws + L.Bh);
+    uint16_t* Bl = reinterpret_cast<uint16_t*>(ws + L.Bl);
+    const int64_t cnt = int64_t(k) * L.ldn8;
+    split_bf16_kernel<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, s>>>(Bm, L.ldn4, k, n, Bh, Bl, L.ldn8);
+    if (cudaGetLastError() != cudaSuccess) return QG_ECUDA;
+    if (launch_gemm_f32(Bh, L.ldn8, false, Bh, L.ldn8, true, At, ldk, k, k, n, s) != cudaSuccess) return QG_ECUDA;
+    if (launch_gemm_f32(Bh, L.ldn8, false, Bl, L.ldn8, true, At, ldk, k, k, n, s, true) != cudaSuccess)
+      return QG_ECUDA;
+    if (launch_gemm_f32(Bl, L.ldn8, false, Bh, L.ldn8, true, At, ldk, k, k, n, s, true) != cudaSuccess)
+      return QG_ECUDA;
+  }
   {
     const int64_t cnt = int64_t(k) * ldk;
     identity_kernel<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, s>>>(Vt, ldk, k);
@@ -749,7 +846,7 @@ qg_status run_refresh(const RefreshArgs& a, uint8_t* ws, size_t ws_bytes, cudaSt
 qg_status run_cossim(const float* Pa, const float* Pb, int32_t m, int32_t r, int64_t ld, float* d_out, uint8_t* ws,
                      cudaStream_t stream) {
   float* buf = reinterpret_cast<float*>(ws);
-  float* scal = reinterpret_cast<float*>(ws + r256(size_t(r) * r * 4 * 4));
+  float* scal = reinterpret_cast<float*>(ws + cossim_buffer_bytes(r));
   return st_of(cossim_core(Pa, Pb, m, r, ld, buf, scal, d_out, stream));
 }
 

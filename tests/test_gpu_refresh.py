@@ -42,9 +42,11 @@ def gpu_cossim(Pa, Pb):
     return float(out.item())
 
 
-def test_cossim_closed_forms_and_oracle():
-    rng = np.random.default_rng(0)
-    m, r = 256, 32
+@pytest.mark.parametrize("m,r", [(256, 32), (512, 128), (2048, 1024)])
+def test_cossim_closed_forms(m, r):
+    # r = 32: the float32 Newton-Schulz steps only; r = 128 and 1024: the
+    # tensor-core steps (bf16 hi + lo operands) followed by float32 ones
+    rng = np.random.default_rng(r)
     P = np.linalg.qr(rng.standard_normal((m, r)))[0]
     Orot = np.linalg.qr(rng.standard_normal((r, r)))[0]
     assert abs(gpu_cossim(P, P) - 1) < 1e-4
@@ -58,7 +60,11 @@ def test_cossim_closed_forms_and_oracle():
     B[np.arange(r), np.arange(r)] = np.cos(theta)
     B[r + np.arange(r), np.arange(r)] = np.sin(theta)
     assert abs(gpu_cossim(A, B) - np.cos(theta).mean()) < 1e-4
-    for (mm, rr) in [(300, 64), (1376, 128), (4096, 1024)]:
+
+
+def test_cossim_matches_oracle():
+    rng = np.random.default_rng(0)
+    for (mm, rr) in [(300, 64), (1376, 128), (4096, 1024), (11008, 1024)]:
         X = np.linalg.qr(rng.standard_normal((mm, rr)))[0]
         Y = np.linalg.qr(X + 0.7 * rng.standard_normal((mm, rr)) / np.sqrt(mm))[0]
         assert abs(gpu_cossim(X, Y) - O.cossim(X.astype(np.float32), Y.astype(np.float32))) < 1e-4
