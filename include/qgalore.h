@@ -58,7 +58,8 @@ typedef enum {
  * used by the paper's setting where the pages give one (gamma = 0.4) and the
  * plain readings elsewhere. */
 typedef struct {
-  int32_t m, n, r;          /* W is m x n, P is m x r; 32 <= r <= min(m, n), r % 32 == 0 */
+  int32_t m, n, r;          /* W is m x n, P is m x r; 32 <= r <= min(m, n), r % 32 == 0;
+                               m, n < 2^30, m n < 2^40, max(m, n) r < 2^34 */
   int32_t w_group;          /* weight-scale group (consecutive elements), must be 256 */
   int32_t p_group;          /* INT4 projection group, must be 64 */
   int32_t mom_block;        /* moment block along a row, must be 256 */

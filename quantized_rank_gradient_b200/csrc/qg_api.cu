@@ -84,6 +84,8 @@ qg_status check_config(const qg_config* c) {
   if (c->r % 32 != 0 || c->r > c->m || c->r > c->n) return QG_ESHAPE;
   if (static_cast<int64_t>(c->m) * c->n >= (int64_t(1) << 40)) return QG_ESHAPE;
   if (c->m >= (1 << 30) || c->n >= (1 << 30)) return QG_ESHAPE;
+  // the projection's INT4 codes are indexed by 32-bit words (8 codes each)
+  if (static_cast<int64_t>(c->m > c->n ? c->m : c->n) * c->r >= (int64_t(1) << 34)) return QG_ESHAPE;
   if (c->w_group != 256 || c->p_group != 64 || c->mom_block != 256) return QG_ESHAPE;
   if (!(c->beta1 >= 0.f && c->beta1 < 1.f) || !(c->beta2 >= 0.f && c->beta2 < 1.f)) return QG_EINVAL;
   if (!(c->eps > 0.f) || !isfinite(c->eps) || !isfinite(c->lr) || !isfinite(c->alpha)) return QG_EINVAL;

@@ -285,7 +285,7 @@ template <class Epi>
 struct PairLayout {
   static constexpr int kGroups = Epi::kPairGroups;  // epilogue warpgroups per CTA
   static constexpr int kThreads = 64 + 128 * kGroups;
-  static_assert(kGroups == 2 || kGroups == 4, "the tile's 256 columns split into 2 or 4 slices");
+  static_assert(kGroups >= 2 && kGroups <= 4, "two to four epilogue warpgroups");
   static constexpr int kSideBytes = Epi::kSideBytes;
   static constexpr int kSideBufs = Epi::kSideBufs;
   static constexpr int kSideTotal = kSideBytes * kSideBufs;

@@ -31,9 +31,6 @@
 #ifndef QG_SR_REVERSE
 #define QG_SR_REVERSE 1
 #endif
-#ifndef QG_DEQUANT_CHUNKS
-#define QG_DEQUANT_CHUNKS 2
-#endif
 #include "../../include/qgalore.h"
 
 namespace qg {
@@ -368,8 +365,8 @@ struct StochRoundEpi {
   };
 
   // the pair kernel drains every tile with two epilogue warpgroups, 128 columns
-  // each (the rounding's registers fit the two-warpgroup budget; measured, four
-  // warpgroups with 16-column sub-chunks ran no faster under the power cap)
+  // each (measured on the 7B stack, three warpgroups, and four with 16-column
+  // sub-chunks, ran no faster)
   static constexpr int kPairGroups = 2;
 
   // The 16-bit draws of columns jc .. jc+31 of row irow (jc a multiple of 32):
@@ -475,9 +472,9 @@ struct StochRoundEpi {
     const bool row_ok = irow < M;
     const int j0 = nb * BN;
     const int ncols = min(BN, N - j0);
-    const int nchunk = BN / 32 / ep.groups;
-    const int c0 = ep.group * nchunk;
-    const int c1 = min(c0 + nchunk, (ncols + 31) >> 5);
+    // group g of G takes the 32-column chunks [8 g / G, 8 (g + 1) / G) of the tile
+    const int c0 = ep.group * (BN / 32) / ep.groups;
+    const int c1 = min((ep.group + 1) * (BN / 32) / ep.groups, (ncols + 31) >> 5);
     float cp_row = 0.f;
     if (kOneGroup && row_ok) cp_row = update_factor(a.alpha, a.sW[(static_cast<int64_t>(irow) * N + j0) >> 8]);
     int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + j0;
@@ -551,6 +548,7 @@ struct StochRoundEpi {
 // and overwritten.
 struct StochRoundRescaleEpi : StochRoundEpi {
   static constexpr bool kExchange = true;
+  static constexpr int kPairGroups = 2;  // 128 columns per warpgroup, the exchange pairs the two halves of a row
   static constexpr int kLimit = 127 * 65536;
 
   static QG_DEV void rescaled_chunk(const uint32_t (&U)[32], const uint4& wa, const uint4& wb,
@@ -694,70 +692,86 @@ static_assert(sizeof(GemmParams<StoreF32Epi>) <= 32764, "kernel parameter block"
 
 // ------------------------------------------------------------------ a1 and test kernels
 
-// Thirty-two INT4 codes (16 bytes, element 2i in the low nibble of byte i) ->
-// thirty-two bf16 of P~ = bf16_rn(code * scale).  Every projection has
-// m*r % 32 == 0 (r % 32 == 0), so a 32-element chunk stays inside one matrix and
-// one 64-element scale group.  One launch covers up to kMaxProblems projections.
-// HBM-bound: 16 bytes read and 64 bytes written per thread, coalesced across
-// the warp; nibbles become floats by exact integer/FP-add arithmetic (no
-// conversion-pipe instructions), and pairs are rounded to bf16 together.
+// Eight INT4 codes (one 32-bit word, element 2i in the low nibble of byte i) ->
+// eight bf16 of P~ = bf16_rn(code * scale), one 16-byte store.  One thread per
+// word, kDqUnits words per thread a block apart, so that every warp-wide load
+// covers 128 contiguous bytes and every store 512; the loads of a thread's
+// words are issued together.  Each block works on one projection (found once
+// per block from the prefix sums of the blocks per projection), with 32-bit
+// indices inside it.  Every projection has m*r % 32 == 0 (r % 32 == 0), so a
+// word stays inside one 64-element scale group (word i uses scale i / 8).  One
+// launch covers up to kMaxProblems projections.  Nibbles become floats by
+// exact integer/FP-add arithmetic (no conversion-pipe instructions), and pairs
+// are rounded to bf16 together.  kVec: every code array 4-byte and every output
+// 16-byte aligned.
+constexpr int kDqThreads = 256;
+constexpr int kDqUnits = 4;
+constexpr int kDqBlockUnits = kDqThreads * kDqUnits;
+
 struct DequantBatch {
   const uint8_t* Pq[kMaxProblems];
   const float* sP[kMaxProblems];
   uint16_t* out[kMaxProblems];
-  int64_t chunk_begin[kMaxProblems + 1];  // prefix sums of (m*r / 32)
+  int32_t units[kMaxProblems];              // m*r / 8 per projection
+  int32_t block_begin[kMaxProblems + 1];    // prefix sums of the blocks per projection
   int32_t n;
 };
 
-constexpr int kDequantChunks = QG_DEQUANT_CHUNKS;  // 32-element chunks per thread, their loads issued together
+QG_DEV uint4 dequant_word(uint32_t w, float s) {
+  // nibble x ^ 8 is code + 8 in [1, 15]; 0x4B400000 | (code + 8) is the float
+  // 1.5 * 2^23 + code + 8, exact
+  const uint32_t f = w ^ 0x88888888u;
+  uint32_t out[4];
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    const float lo = __fsub_rn(__uint_as_float(0x4B400000u | ((f >> (8 * h)) & 0xFu)), 12582920.0f);
+    const float hi = __fsub_rn(__uint_as_float(0x4B400000u | ((f >> (8 * h + 4)) & 0xFu)), 12582920.0f);
+    const __nv_bfloat162 pr = __floats2bfloat162_rn(__fmul_rn(lo, s), __fmul_rn(hi, s));
+    out[h] = *reinterpret_cast<const uint32_t*>(&pr);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
 
-template <bool kVec16>
-__global__ void __launch_bounds__(256) dequant_projection_kernel(const __grid_constant__ DequantBatch b) {
-  const int64_t total = b.chunk_begin[b.n];
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  uint32_t w[kDequantChunks][4];
-  float s[kDequantChunks];
-  uint16_t* dst[kDequantChunks];
+template <bool kVec>
+__global__ void __launch_bounds__(kDqThreads) dequant_projection_kernel(const __grid_constant__ DequantBatch b) {
+  int p = 0;
+  while (p + 1 < b.n && static_cast<int>(blockIdx.x) >= b.block_begin[p + 1]) ++p;
+  const int units = b.units[p];
+  const int first = (static_cast<int>(blockIdx.x) - b.block_begin[p]) * kDqBlockUnits + static_cast<int>(threadIdx.x);
+  const uint8_t* src = b.Pq[p];
+  const float* sp = b.sP[p];
+  uint16_t* dst = b.out[p];
+  uint32_t w[kDqUnits];
+  float s[kDqUnits];
 #pragma unroll
-  for (int c = 0; c < kDequantChunks; ++c) {
-    const int64_t i = first + c * stride;
-    dst[c] = nullptr;
-    if (i >= total) continue;
-    int p = 0;
-    while (p + 1 < b.n && i >= b.chunk_begin[p + 1]) ++p;
-    const int64_t e0 = (i - b.chunk_begin[p]) * 32;
-    const uint8_t* src = b.Pq[p] + (e0 >> 1);
-    if (kVec16) {
-      const uint4 v = *reinterpret_cast<const uint4*>(src);
-      w[c][0] = v.x, w[c][1] = v.y, w[c][2] = v.z, w[c][3] = v.w;
+  for (int u = 0; u < kDqUnits; ++u) {
+    const int i = first + u * kDqThreads;
+    if (i >= units) continue;
+    if (kVec) {
+      w[u] = reinterpret_cast<const uint32_t*>(src)[i];
     } else {
-#pragma unroll
-      for (int k = 0; k < 4; ++k) w[c][k] = reinterpret_cast<const uint32_t*>(src)[k];
+      const uint8_t* q = src + 4 * static_cast<int64_t>(i);
+      w[u] = static_cast<uint32_t>(q[0]) | (static_cast<uint32_t>(q[1]) << 8) | (static_cast<uint32_t>(q[2]) << 16) |
+             (static_cast<uint32_t>(q[3]) << 24);
     }
-    s[c] = b.sP[p][e0 >> 6];
-    dst[c] = b.out[p] + e0;
+    s[u] = sp[i >> 3];
   }
 #pragma unroll
-  for (int c = 0; c < kDequantChunks; ++c) {
-    if (!dst[c]) continue;
-    uint32_t out[16];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      // nibble x ^ 8 is code + 8 in [1, 15]; 0x4B400000 | (code + 8) is the float
-      // 1.5 * 2^23 + code + 8, exact
-      const uint32_t f = w[c][k] ^ 0x88888888u;
+  for (int u = 0; u < kDqUnits; ++u) {
+    const int i = first + u * kDqThreads;
+    if (i >= units) continue;
+    const uint4 v = dequant_word(w[u], s[u]);
+    if (kVec) {
+      reinterpret_cast<uint4*>(dst)[i] = v;
+    } else {
+      uint16_t* d = dst + 8 * static_cast<int64_t>(i);
+      const uint32_t o[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        const float lo = __fsub_rn(__uint_as_float(0x4B400000u | ((f >> (8 * h)) & 0xFu)), 12582920.0f);
-        const float hi = __fsub_rn(__uint_as_float(0x4B400000u | ((f >> (8 * h + 4)) & 0xFu)), 12582920.0f);
-        const __nv_bfloat162 pr = __floats2bfloat162_rn(__fmul_rn(lo, s[c]), __fmul_rn(hi, s[c]));
-        out[4 * k + h] = *reinterpret_cast<const uint32_t*>(&pr);
+        d[2 * h] = static_cast<uint16_t>(o[h] & 0xFFFFu);
+        d[2 * h + 1] = static_cast<uint16_t>(o[h] >> 16);
       }
     }
-    uint4* d = reinterpret_cast<uint4*>(dst[c]);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) d[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
   }
 }
 
@@ -878,32 +892,38 @@ static void add_problem(GemmParams<Epi>& p, int M, int N, int K) {
   p.nprob += 1;
 }
 
-static cudaError_t launch_dequant_batch(const DequantBatch& b, cudaStream_t stream) {
-  const int64_t chunks = b.chunk_begin[b.n];
-  if (chunks == 0) return cudaSuccess;
-  const int threads = 256;
-  const int64_t blocks = (chunks + int64_t(threads) * kDequantChunks - 1) / (int64_t(threads) * kDequantChunks);
-  const double total = chunks * 32.0;
+// Fills the per-projection unit counts' block prefix sums and launches.
+static cudaError_t launch_dequant_batch(DequantBatch& b, cudaStream_t stream) {
+  b.block_begin[0] = 0;
+  double total = 0.0;
+  for (int i = 0; i < b.n; ++i) {
+    b.block_begin[i + 1] = b.block_begin[i] + (b.units[i] + kDqBlockUnits - 1) / kDqBlockUnits;
+    total += b.units[i] * 8.0;
+  }
+  const int blocks = b.block_begin[b.n];
+  if (blocks == 0) return cudaSuccess;
   const double bytes = total / 2.0 + total / 64.0 * 4.0 + total * 2.0;
-  bool vec16 = true;
-  for (int i = 0; i < b.n; ++i) vec16 = vec16 && (reinterpret_cast<uintptr_t>(b.Pq[i]) % 16 == 0);
+  bool vec = true;
+  for (int i = 0; i < b.n; ++i)
+    vec = vec && (reinterpret_cast<uintptr_t>(b.Pq[i]) % 4 == 0) && (reinterpret_cast<uintptr_t>(b.out[i]) % 16 == 0);
   const int tok = profile_begin(stream, QG_KERNEL_DEQUANT, 0.0, bytes);
-  if (vec16)
-    dequant_projection_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(b);
+  if (vec)
+    dequant_projection_kernel<true><<<static_cast<unsigned>(blocks), kDqThreads, 0, stream>>>(b);
   else
-    dequant_projection_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(b);
+    dequant_projection_kernel<false><<<static_cast<unsigned>(blocks), kDqThreads, 0, stream>>>(b);
   profile_end(stream, tok);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequant_projection(const uint8_t* Pq, const float* sP, int64_t total, uint16_t* out,
                                       cudaStream_t stream) {
+  if (total / 8 > INT32_MAX) return cudaErrorInvalidValue;
   DequantBatch b;
   memset(&b, 0, sizeof(b));
   b.Pq[0] = Pq;
   b.sP[0] = sP;
   b.out[0] = out;
-  b.chunk_begin[1] = total / 32;
+  b.units[0] = static_cast<int32_t>(total / 8);
   b.n = 1;
   return launch_dequant_batch(b, stream);
 }
@@ -925,7 +945,7 @@ static cudaError_t launch_dequant_for(const StepProblem* probs, int cnt, cudaStr
     db.Pq[i] = s.Pq;
     db.sP[i] = s.sP;
     db.out[i] = s.Pbf;
-    db.chunk_begin[i + 1] = db.chunk_begin[i] + static_cast<int64_t>(s.side ? s.n : s.m) * s.r / 32;
+    db.units[i] = static_cast<int32_t>(static_cast<int64_t>(s.side ? s.n : s.m) * s.r / 8);
   }
   db.n = cnt;
   return launch_dequant_batch(db, stream);
