@@ -279,32 +279,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // the loads complete on side_full.
 // ---------------------------------------------------------------------------
 
-constexpr int kHalfStageBytes = 128 * BK * 2;  // 16 KiB: 128 rows of A or 128 columns of B
-
-template <class Epi>
+// Epilogues of the pair kernel declare kPairBKMN, the K depth of a ring stage
+// when both operands are MN-major (K is then the outer dimension of every TMA
+// box, so any multiple of 16 works; a K-major operand's 128-byte swizzled rows
+// hold exactly 64 bf16 of K, so with one the depth is 64), and kPairMaxStages,
+// a cap on the ring's depth.  Smaller stages let more of them, and more bytes,
+// stay in flight beside the side buffers.
+template <class Epi, int kBK>
 struct PairLayout {
   static constexpr int kGroups = Epi::kPairGroups;  // epilogue warpgroups per CTA
   static constexpr int kThreads = 64 + 128 * kGroups;
   static_assert(kGroups >= 2 && kGroups <= 4, "two to four epilogue warpgroups");
+  static_assert(kBK % 16 == 0 && kBK >= 16 && kBK <= 64, "K depth of a stage");
+  static constexpr int kHalfStageBytes = 128 * kBK * 2;  // 128 rows of A or 128 columns of B
+  static constexpr int kChunkBytes = 64 * kBK * 2;       // one 64-wide M/N chunk of an MN-major stage
   static constexpr int kSideBytes = Epi::kSideBytes;
   static constexpr int kSideBufs = Epi::kSideBufs;
   static constexpr int kSideTotal = kSideBytes * kSideBufs;
   // shared memory a CTA may hold (227 KiB) less the static part: barriers and
   // flags, plus the row-maxima exchange when the epilogue uses it
   static constexpr int kBudget = 232448 - 512 - (Epi::kExchange ? int(sizeof(float2)) * 2 * kGroups * BM : 0) - 1024;
-  // as many ring stages as fit beside the side buffers, at most 6
-  static constexpr int kStages = (kBudget - kSideTotal) / (2 * kHalfStageBytes) > 6
-                                     ? 6
-                                     : (kBudget - kSideTotal) / (2 * kHalfStageBytes);
+  // as many ring stages as fit beside the side buffers, at most kPairMaxStages
+  static constexpr int kFit = (kBudget - kSideTotal) / (2 * kHalfStageBytes);
+  static constexpr int kStages = kFit > Epi::kPairMaxStages ? Epi::kPairMaxStages : kFit;
   static constexpr size_t kSmemBytes = size_t(kStages) * 2 * kHalfStageBytes + kSideTotal + 1024;
   static_assert(kStages >= 3, "side buffers leave too few ring stages");
+  static_assert(kStages <= 32, "stage bit masks are 32 bits wide");
   static_assert(kSideBytes % 1024 == 0, "side buffers keep 1024-byte alignment");
 };
 
+// The layout a pair-kernel instantiation uses.
 template <class Epi, bool kAMN, bool kBMN>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<Epi>::kThreads, 1)
+struct PairCfg {
+  static constexpr int kBK = (kAMN && kBMN) ? Epi::kPairBKMN : 64;
+  using L = PairLayout<Epi, kBK>;
+};
+
+template <class Epi, bool kAMN, bool kBMN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<Epi, kAMN, kBMN>::L::kThreads, 1)
     gemm_tc_pair_kernel(const __grid_constant__ GemmParams<Epi> p) {
-  using L = PairLayout<Epi>;
+  using L = typename PairCfg<Epi, kAMN, kBMN>::L;
+  constexpr int kBKp = PairCfg<Epi, kAMN, kBMN>::kBK;
+  constexpr int kHalfStageBytes = L::kHalfStageBytes;
+  constexpr int kChunk = L::kChunkBytes;
   constexpr int kGroups = L::kGroups;
   constexpr int kEpiWarps = 4 * kGroups;
   constexpr int kStagesP = L::kStages;
@@ -398,7 +415,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<Epi>::kTh
         int pi, mb2, nb;
         locate(tile, pi, mb2, nb);
         const GemmProblem<Epi>& pr = p.prob[pi];
-        const int nkb = (pr.K + BK - 1) / BK;
+        const int nkb = (pr.K + kBKp - 1) / kBKp;
         const int row0 = mb2 * 256 + static_cast<int>(rank) * 128;
         const int col0 = nb * BN + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -411,16 +428,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<Epi>::kTh
           uint8_t* a_dst = sA + stage * kHalfStageBytes;
           uint8_t* b_dst = sB + stage * kHalfStageBytes;
           if (kAMN) {
-            tma_load_2d_pair(a_dst, &pr.tmA, fb, row0, kb * BK);
-            tma_load_2d_pair(a_dst + 8192, &pr.tmA, fb, row0 + 64, kb * BK);
+            tma_load_2d_pair(a_dst, &pr.tmA, fb, row0, kb * kBKp);
+            tma_load_2d_pair(a_dst + kChunk, &pr.tmA, fb, row0 + 64, kb * kBKp);
           } else {
-            tma_load_2d_pair(a_dst, &pr.tmA, fb, kb * BK, row0);
+            tma_load_2d_pair(a_dst, &pr.tmA, fb, kb * kBKp, row0);
           }
           if (kBMN) {
-            tma_load_2d_pair(b_dst, &pr.tmB, fb, col0, kb * BK);
-            tma_load_2d_pair(b_dst + 8192, &pr.tmB, fb, col0 + 64, kb * BK);
+            tma_load_2d_pair(b_dst, &pr.tmB, fb, col0, kb * kBKp);
+            tma_load_2d_pair(b_dst + kChunk, &pr.tmB, fb, col0 + 64, kb * kBKp);
           } else {
-            tma_load_2d_pair(b_dst, &pr.tmB, fb, kb * BK, col0);
+            tma_load_2d_pair(b_dst, &pr.tmB, fb, kb * kBKp, col0);
           }
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -444,8 +461,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<Epi>::kTh
       // descriptors of any stage and step are one 64-bit add away.  This keeps
       // the issuing thread's instruction stream short while the epilogue warps
       // share its scheduler.
-      const uint64_t a_desc0 = kAMN ? sdesc_sw128(smem_u32(sA), 8192, 1024) : sdesc_sw128(smem_u32(sA), 16, 1024);
-      const uint64_t b_desc0 = kBMN ? sdesc_sw128(smem_u32(sB), 8192, 1024) : sdesc_sw128(smem_u32(sB), 16, 1024);
+      const uint64_t a_desc0 = kAMN ? sdesc_sw128(smem_u32(sA), kChunk, 1024) : sdesc_sw128(smem_u32(sA), 16, 1024);
+      const uint64_t b_desc0 = kBMN ? sdesc_sw128(smem_u32(sB), kChunk, 1024) : sdesc_sw128(smem_u32(sB), 16, 1024);
       constexpr uint64_t kStageStep = kHalfStageBytes >> 4;
       constexpr uint64_t kAStep = kAMN ? (2048 >> 4) : (32 >> 4);  // one K step of 16
       constexpr uint64_t kBStep = kBMN ? (2048 >> 4) : (32 >> 4);
@@ -455,7 +472,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<Epi>::kTh
         int pi, mb2, nb;
         locate(tile, pi, mb2, nb);
         const int K = p.prob[pi].K;
-        const int nkb = (K + BK - 1) / BK;
+        const int nkb = (K + kBKp - 1) / kBKp;
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, &abort_flag, status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
@@ -467,11 +484,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<Epi>::kTh
           tc_fence_after();
           const uint64_t ad = a_desc0 + stage * kStageStep;
           const uint64_t bd = b_desc0 + stage * kStageStep;
-          const int kleft = K - kb * BK;
-          if (kleft >= BK) {
+          const int kleft = K - kb * kBKp;
+          if (kleft >= kBKp) {
             umma_bf16_pair(d_tmem, ad, bd, idesc, kb != 0 ? 1u : 0u);
 #pragma unroll
-            for (int kk = 1; kk < BK / 16; ++kk) umma_bf16_pair(d_tmem, ad + kk * kAStep, bd + kk * kBStep, idesc, 1u);
+            for (int kk = 1; kk < kBKp / 16; ++kk) umma_bf16_pair(d_tmem, ad + kk * kAStep, bd + kk * kBStep, idesc, 1u);
           } else {
             const int ksteps = (kleft + 15) / 16;
             for (int kk = 0; kk < ksteps; ++kk)

@@ -105,6 +105,8 @@ struct StoreBF16Epi {
   static constexpr int kSideBufs = 1;
   static constexpr bool kExchange = false;
   static constexpr int kPairGroups = 2;
+  static constexpr int kPairBKMN = 64;
+  static constexpr int kPairMaxStages = 6;
   static QG_DEV void issue_side(const CUtensorMap*, int, int, uint8_t*, uint64_t*) {}
   struct Args {
     uint16_t* D;
@@ -180,7 +182,8 @@ cudaError_t launch_bf16(const void* A, int64_t lda, const void* B, int64_t ldb, 
   p.total_tiles = pr.tiles_m * pr.tiles_n;
 
   auto kern = gemm_tc_pair_kernel<StoreBF16Epi, kAMN, kBMN>;
-  constexpr size_t kSmem = PairLayout<StoreBF16Epi>::kSmemBytes;
+  using L = typename PairCfg<StoreBF16Epi, kAMN, kBMN>::L;
+  constexpr size_t kSmem = L::kSmemBytes;
   static std::once_flag once;  // per instantiation
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [&] {
@@ -191,7 +194,7 @@ cudaError_t launch_bf16(const void* A, int64_t lda, const void* B, int64_t ldb, 
   const int clusters = std::min(pair_tiles, std::max(1, sm_count() / 2));
   const double flops = 2.0 * M * N * K, bytes = 2.0 * M * K + 2.0 * K * N + 2.0 * M * N;
   const int tok = profile_begin(stream, QG_KERNEL_LINEAR_GEMM, flops, bytes);
-  kern<<<2 * clusters, PairLayout<StoreBF16Epi>::kThreads, kSmem, stream>>>(p);
+  kern<<<2 * clusters, L::kThreads, kSmem, stream>>>(p);
   profile_end(stream, tok);
   return cudaGetLastError();
 }

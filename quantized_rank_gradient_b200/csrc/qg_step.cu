@@ -154,6 +154,12 @@ struct AdamEpi {
 
   // the pair kernel drains every tile with four epilogue warpgroups, 64 columns each
   static constexpr int kPairGroups = 4;
+  // Ring stages of K = 64 (32 KiB per CTA): four fit beside the 64 KiB side
+  // tiles.  Measured on the 7B stack: three stages made the launch 12 % slower;
+  // nine stages of K = 32 (more bytes in flight, but two MMAs per stage) 25 %
+  // slower.
+  static constexpr int kPairBKMN = 64;
+  static constexpr int kPairMaxStages = 6;
 
   // Pass 1 on one 16-column sub-chunk (moment codes in qm, qv): the new moments
   // and the running block maxima of |m| and of v (max over the block of sqrt(v)
@@ -368,6 +374,10 @@ struct StochRoundEpi {
   // each (measured on the 7B stack, three warpgroups, and four with 16-column
   // sub-chunks, ran no faster)
   static constexpr int kPairGroups = 2;
+  // A is K-major (stages of K = 64); four stages measured 2-7 % faster than
+  // five on the 7B stack
+  static constexpr int kPairBKMN = 64;
+  static constexpr int kPairMaxStages = 4;
 
   // The 16-bit draws of columns jc .. jc+31 of row irow (jc a multiple of 32):
   // column j's draw is half (j mod 2) of word ((j / 2) mod 4) of
@@ -861,7 +871,8 @@ template <class Epi, bool kAMN, bool kBMN = true>
 static cudaError_t launch_gemm_pair(const GemmParams<Epi>& p, cudaStream_t stream, int kind, double flops,
                                     double bytes) {
   auto kern = gemm_tc_pair_kernel<Epi, kAMN, kBMN>;
-  constexpr size_t kSmem = PairLayout<Epi>::kSmemBytes;
+  using L = typename PairCfg<Epi, kAMN, kBMN>::L;
+  constexpr size_t kSmem = L::kSmemBytes;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -874,7 +885,7 @@ static cudaError_t launch_gemm_pair(const GemmParams<Epi>& p, cudaStream_t strea
   if (pair_tiles == 0) return cudaSuccess;
   const int clusters = std::min(pair_tiles, std::max(1, sm_count() / 2));
   const int tok = profile_begin(stream, kind, flops, bytes);
-  kern<<<2 * clusters, PairLayout<Epi>::kThreads, kSmem, stream>>>(p);
+  kern<<<2 * clusters, L::kThreads, kSmem, stream>>>(p);
   profile_end(stream, tok);
   return cudaGetLastError();
 }
@@ -1019,10 +1030,12 @@ static cudaError_t launch_gemms_side(const StepProblem* probs, const int* idx, i
       if (!encode_map_i8_side(&pr.tmS[0], s.Mq, s.r, s.m, s.ld_mom)) return cudaErrorInvalidValue;
       if (!encode_map_i8_side(&pr.tmS[1], s.Vq, s.r, s.m, s.ld_mom)) return cudaErrorInvalidValue;
     } else {
-      // A = P~^T (M = r, K = m), MN-major over P~ (m x r): box {64 (r), 64 (m)}
-      if (!encode_map_bf16(&pr.tmA, s.Pbf, s.r, s.m, s.r, 64, 64)) return cudaErrorInvalidValue;
-      // B = G (K = m, N = n), MN-major: box {64 (n), 64 (m)}
-      if (!encode_map_bf16(&pr.tmB, s.G, s.n, s.m, s.ldg, 64, 64)) return cudaErrorInvalidValue;
+      // both operands MN-major: boxes of kPairBKMN rows of K
+      constexpr uint32_t kBKb = AdamEpi::kPairBKMN;
+      // A = P~^T (M = r, K = m), MN-major over P~ (m x r): box {64 (r), kBK (m)}
+      if (!encode_map_bf16(&pr.tmA, s.Pbf, s.r, s.m, s.r, 64, kBKb)) return cudaErrorInvalidValue;
+      // B = G (K = m, N = n), MN-major: box {64 (n), kBK (m)}
+      if (!encode_map_bf16(&pr.tmB, s.G, s.n, s.m, s.ldg, 64, kBKb)) return cudaErrorInvalidValue;
       // side operands: M^Q and V^Q (r x n int8, leading dimension ld_mom)
       if (!encode_map_i8_side(&pr.tmS[0], s.Mq, s.n, s.r, s.ld_mom)) return cudaErrorInvalidValue;
       if (!encode_map_i8_side(&pr.tmS[1], s.Vq, s.n, s.r, s.ld_mom)) return cudaErrorInvalidValue;
