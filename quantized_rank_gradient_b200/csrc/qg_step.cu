@@ -415,16 +415,10 @@ struct StochRoundEpi {
   // give one pair of 16-bit lanes, clamped to [-127, 127] by one max and one
   // min on both lanes; the low bytes of four lanes are the four new codes.
   // When |X| reaches 2^22, or X is NaN, the chunk is redone in the general form.
-  //
-  // kTrack: also the largest and smallest T = q 2^16 + K over the chunk (K = 0
-  // where X is NaN), each element's value in units of 2^-16 code; in the fast
-  // form T is the magic sum's low bits plus q 2^16.
-  template <bool kOneFactor, bool kTrack = false>
+  template <bool kOneFactor>
   static QG_DEV void sr_chunk(const uint32_t (&U)[32], const uint4& wa, const uint4& wb, const uint32_t (&d)[16],
-                              float cp0, float cp1, int split, uint32_t (&out)[8], int* tmax = nullptr,
-                              int* tmin = nullptr) {
+                              float cp0, float cp1, int split, uint32_t (&out)[8]) {
     float mx = 0.f;
-    int cmax = INT_MIN, cmin = INT_MAX;
     uint32_t sum[2], lanes[2];
 #pragma unroll
     for (int k = 0; k < 32; ++k) {
@@ -436,17 +430,10 @@ struct StochRoundEpi {
       const uint32_t wsel = 0x44u | (static_cast<uint32_t>(k & 3) << 8) | (static_cast<uint32_t>((k & 3) | 8) << 12);
       const uint32_t q16 = prmt(word_of(k < 16 ? wa : wb, (k >> 2) & 3), 0u, wsel);
       sum[k & 1] = tb + dq + q16;
-      if (kTrack) {
-        const int T = static_cast<int>(tb + q16 - kMagicBits);
-        cmax = max(cmax, T);
-        cmin = min(cmin, T);
-      }
       if (k & 1) lanes[(k >> 1) & 1] = clamp127_s16x2(prmt(sum[0], sum[1], 0x7632u));
       if ((k & 3) == 3) out[k >> 2] = prmt(lanes[0], lanes[1], 0x6420u);
     }
     if (!(mx < 4194304.0f)) {
-      cmax = INT_MIN;
-      cmin = INT_MAX;
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
         const float cp = (kOneFactor || k < split) ? cp0 : cp1;
@@ -459,17 +446,9 @@ struct StochRoundEpi {
           const int draw = static_cast<int>((d[k >> 1] >> (16 * (k & 1))) & 0xFFFFu);
           v = min(max(q + ((K + draw) >> 16), -127), 127);
         }
-        if (kTrack) {
-          cmax = max(cmax, q * 65536 + K);
-          cmin = min(cmin, q * 65536 + K);
-        }
         const uint32_t sh = 8 * (k & 3);
         out[k >> 2] = (out[k >> 2] & ~(0xFFu << sh)) | ((static_cast<uint32_t>(v) & 0xFFu) << sh);
       }
-    }
-    if (kTrack) {
-      *tmax = max(*tmax, cmax);
-      *tmin = min(*tmin, cmin);
     }
   }
 
@@ -551,11 +530,9 @@ struct StochRoundEpi {
 //                  with the same draw, fl(T) the nearest float32.
 // The expected value of code' s' stays q s + alpha U (up to the 2^-16 draw
 // grid and float32 rounding).  Needs n % 256 == 0, so that a group is one row
-// of a 256-column tile.  The rounding pass runs as in the saturating form and
-// also takes the row slice's exact max |T|; the two warpgroups combine their
-// maxima through the exchange slots, and only a row whose group grows is
-// rounded again on the new grid (its accumulator and W codes are still staged)
-// and overwritten.
+// of a 256-column tile.  A first pass takes the row slice's exact max |T|, the
+// two warpgroups combine their maxima through the exchange slots, and a
+// second pass rounds every element once, on the grid its group ends up with.
 struct StochRoundRescaleEpi : StochRoundEpi {
   static constexpr bool kExchange = true;
   static constexpr int kPairGroups = 2;  // 128 columns per warpgroup, the exchange pairs the two halves of a row
@@ -583,6 +560,44 @@ struct StochRoundRescaleEpi : StochRoundEpi {
     *reinterpret_cast<uint4*>(dst + 16) = make_uint4(out[4], out[5], out[6], out[7]);
   }
 
+  // max |T| over one 32-column chunk, T = q 2^16 + K with K = rint(X) (0 where
+  // X is NaN), the values in units of 2^-16 code; no draws.  Fast form while
+  // |X| < 2^22: the bits of fadd.rn(X, 1.5 2^23) less 0x4B400000 are K; a chunk
+  // with a larger or NaN X is redone with the conversion (X clipped to 2^30, as
+  // the rounding does).  |T| < 2^31.
+  static QG_DEV uint32_t chunk_tmax(const uint32_t (&U)[32], const uint4& wa, const uint4& wb, float cp) {
+    float mx = 0.f;
+    uint32_t amax = 0u;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const float X = __fmul_rn(__uint_as_float(U[k]), cp);
+      mx = max_nan_abs(mx, X);
+      const uint32_t tb = __float_as_uint(__fadd_rn(X, kMagic));
+      const uint32_t wsel = 0x44u | (static_cast<uint32_t>(k & 3) << 8) | (static_cast<uint32_t>((k & 3) | 8) << 12);
+      const uint32_t q16 = prmt(word_of(k < 16 ? wa : wb, (k >> 2) & 3), 0u, wsel);
+      const int T = static_cast<int>(tb + q16 - kMagicBits);
+      amax = max(amax, static_cast<uint32_t>(abs(T)));
+    }
+    if (!(mx < 4194304.0f)) {
+      amax = 0u;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const float X = __fmul_rn(__uint_as_float(U[k]), cp);
+        const uint4& w = k < 16 ? wa : wb;
+        const int q = static_cast<int8_t>((word_of(w, (k >> 2) & 3) >> (8 * (k & 3))) & 0xFFu);
+        const int K = X == X ? __float2int_rn(fminf(fmaxf(X, -1073741824.0f), 1073741824.0f)) : 0;
+        amax = max(amax, static_cast<uint32_t>(abs(q * 65536 + K)));
+      }
+    }
+    return amax;
+  }
+
+  // Two passes over the row slice.  Pass 1 takes the exact max |T| (no draws,
+  // no stores); the two warpgroups combine their maxima through the exchange
+  // slots; pass 2 rounds every element once, on the grown grid where the group
+  // grows and on the saturating form's otherwise.  Loop control is
+  // warp-uniform; the lane-varying predicates (row inside the matrix, group
+  // grows) are re-read per chunk (lane_pred) and guard no tensor-memory load.
   static QG_DEV void apply(const Args& a, int M, int N, int mb, int nb, int row, uint32_t taddr,
                            const EpiPair& ep, const uint8_t* side) {
     const int irow = mb * BM + row;
@@ -594,24 +609,17 @@ struct StochRoundRescaleEpi : StochRoundEpi {
     const float s = row_ok ? a.sW[g] : 0.f;
     const float cp = update_factor(a.alpha, s);
     int8_t* wrow = a.W + static_cast<int64_t>(irow) * a.ldw + j0;
-    const PhiloxRoundKeys rk = philox_round_keys(a.key);
-    int tmax = INT_MIN, tmin = INT_MAX;
+    uint32_t amax = 0u;
     __syncwarp();
 #pragma unroll 1
     for (int c = c0; c < c0 + nchunk; ++c) {
       uint32_t U[32];
       tmem_ld_32x32b_x32(taddr + c * 32, U);
+      const uint4 wa = side_granule(side, row, 2 * c), wb = side_granule(side, row, 2 * c + 1);
       tmem_ld_wait(U);
       if (!lane_pred(row_ok)) continue;
-      const uint4 wa = side_granule(side, row, 2 * c), wb = side_granule(side, row, 2 * c + 1);
-      uint32_t d[16];
-      draws(a, rk, irow, j0 + c * 32, d);
-      uint32_t out[8];
-      sr_chunk<true, true>(U, wa, wb, d, cp, cp, 32, out, &tmax, &tmin);
-      store_chunk(wrow + c * 32, out);
+      amax = max(amax, chunk_tmax(U, wa, wb, cp));
     }
-    // |T| < 2^31: |q 2^16| <= 127 2^16 and |K| <= 2^30
-    uint32_t amax = row_ok ? static_cast<uint32_t>(max(tmax, -tmin)) : 0u;
 
     // the group's maximum over both column slices (the other group's warps own
     // the same rows); the slots carry the integer's bits
@@ -625,20 +633,23 @@ struct StochRoundRescaleEpi : StochRoundEpi {
         if (o != ep.group) amax = max(amax, __float_as_uint(ep.xchg[o * BM + lane].x));
     }
     const bool grow = row_ok && s > 0.f && amax > static_cast<uint32_t>(kLimit);
-    if (!__any_sync(0xFFFFFFFFu, grow)) return;
     const float rho = grow ? __fdiv_rn(static_cast<float>(kLimit), __uint2float_rn(amax)) : 1.f;
+    const PhiloxRoundKeys rk = philox_round_keys(a.key);
     __syncwarp();
 #pragma unroll 1
     for (int c = c0; c < c0 + nchunk; ++c) {
       uint32_t U[32];
       tmem_ld_32x32b_x32(taddr + c * 32, U);
-      tmem_ld_wait(U);
-      if (!lane_pred(grow)) continue;
-      const uint4 wa = side_granule(side, row, 2 * c), wb = side_granule(side, row, 2 * c + 1);
       uint32_t d[16];
       draws(a, rk, irow, j0 + c * 32, d);
+      tmem_ld_wait(U);
+      if (!lane_pred(row_ok)) continue;
+      const uint4 wa = side_granule(side, row, 2 * c), wb = side_granule(side, row, 2 * c + 1);
       uint32_t out[8];
-      rescaled_chunk(U, wa, wb, d, cp, rho, out);
+      if (lane_pred(grow))
+        rescaled_chunk(U, wa, wb, d, cp, rho, out);
+      else
+        sr_chunk<true>(U, wa, wb, d, cp, cp, 32, out);
       store_chunk(wrow + c * 32, out);
     }
     if (grow && ep.group == 0) a.sW[g] = __fdiv_rn(s, rho);
