@@ -290,7 +290,7 @@ class Stack:
                 group.append(dict(cfg=c, h=h, W=W, sW=sW, G=G, ldg=G.shape[1], state=state, m=m, n=n, side=side))
                 lid += 1
             self.layers.append(group)
-        # the step: one batched call for all matrices (batches of 8 on two lanes
+        # the step: one batched call for all matrices (batches of 8 on three lanes
         # inside the library), or with QG_BENCH_PER_LAYER=1 one call per decoder
         # layer.  The per-layer calls (the 7 matrices of a layer in one batch, one
         # stream, kernels one after another) also serve the kernel-timing pass.
@@ -422,7 +422,7 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     ms = reduce_max(ms, world)
 
-    # ---- kernel durations: in the timed region the two lanes' kernels overlap,
+    # ---- kernel durations: in the timed region the lanes' kernels overlap,
     # so a launch's events would also span the other lane's work.  The same
     # kernels on the same data are timed again one after another: one call per
     # decoder layer on one stream (a step counts once more for every matrix's t).

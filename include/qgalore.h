@@ -180,15 +180,15 @@ qg_status qg_step(qg_layer* layer, const void* d_G, int64_t ldg, void* d_ws, siz
  * launches: batches of up to 8
  * matrices, three launches per batch (dequantize the batch's projections, then
  * one persistent tcgen05 grid per GEMM stage).  With more than one batch, the
- * batches alternate between `stream` and a second stream that the library
- * creates on the current device at its first such call and keeps until the
- * process exits; they fork from `stream` and join back to it through events,
- * so the call is ordered on `stream` (and may be captured into a CUDA graph
- * once that stream exists) and the two lanes' kernels overlap.  Calls from
+ * batches take turns among three lanes: `stream` and two streams that the
+ * library creates on the current device at its first such call and keeps until
+ * the process exits; they fork from `stream` and join back to it through
+ * events, so the call is ordered on `stream` (and may be captured into a CUDA
+ * graph once those streams exist) and the lanes' kernels overlap.  Calls from
  * several host threads are serialised while they enqueue.
  * d_ws (256-byte aligned) must hold qg_step_batch_workspace_bytes of the same
- * configurations in the same order: one slot per lane (one, or two when there
- * are several batches), each the largest batch's sum of
+ * configurations in the same order: one slot per lane in use (as many as there
+ * are batches, at most three), each the largest batch's sum of
  * qg_step_workspace_bytes, reused by the lane's batches.  A smaller d_ws gives
  * QG_ESTATE before anything is launched. */
 qg_status qg_step_batch(qg_layer* const* layers, const void* const* d_G, const int64_t* ldg,
