@@ -22,7 +22,7 @@ Variants of the stack workload, by environment (the workload name says which ran
     QG_BENCH_PER_LAYER=1       one qg_step_batch call per decoder layer, one stream
 A run still going after QG_BENCH_WATCHDOG_S seconds (default 1800) ends itself.
 Other workloads: --workload llama1b-stack | llama60m-stack | refresh-stress |
-linear-grad-stress | linear-7b.
+linear-grad-stress | linear-7b | linear-7b-decode.
 """
 from __future__ import annotations
 
@@ -58,14 +58,17 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=None, help="decoder layers (default: the stack's own count)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=sorted(STACKS) + ["refresh-stress", "linear-grad-stress", "linear-7b"],
+    ap.add_argument("--tokens", type=int, default=16, help="linear-7b-decode: tokens of the headline line (1..16)")
+    ap.add_argument("--workload", choices=sorted(STACKS) + ["refresh-stress", "linear-grad-stress", "linear-7b",
+                                                            "linear-7b-decode"],
                     default="llama7b-stack",
                     help="a decoder stack (llama7b-stack is the default and the headline); refresh-stress: "
                          "one 4096 x 11008 layer, r = 1024, a drifting gradient subspace, subspace refreshes on "
                          "the layer-adaptive schedule (--steps defaults to 2000); linear-grad-stress: the same "
                          "layer and schedule with G = D^T X of a linear layer over 8192 tokens whose output-"
                          "gradient subspace turns for 600 steps and then settles; linear-7b: the INT8-weight "
-                         "forward and backward products of the LLaMA-7B stack's 224 linear layers at 8192 tokens")
+                         "forward and backward products of the LLaMA-7B stack's 224 linear layers at 8192 tokens; "
+                         "linear-7b-decode: Y = X W~^T of the same 224 INT8 weights for a few tokens, W read once")
     return ap.parse_args()
 
 
@@ -710,6 +713,154 @@ def run_linear(args, rank, world, local_rank):
     return 0
 
 
+DECODE_TOKENS = (1, 4, 8, 16)
+
+
+def run_linear_decode(args, rank, world, local_rank):
+    """The forward product Y = X W~^T of the LLaMA-7B stack's INT8 weights for a
+    few tokens (--tokens, default 16; the line also sweeps T = 1, 4, 8, 16).
+
+    The weights are laid out as decoders run them for inference: per layer the
+    q, k and v weights stacked in one 12288 x 4096 buffer and gate and up in one
+    22016 x 4096 buffer (the matrices of a stack read the same input), o and down
+    alone, each buffer's group scales the concatenation of its matrices' (the
+    groups never straddle two matrices, n % 256 == 0).  The optimizer still sees
+    each matrix as a row slice of its buffer.  One step runs
+    qg_linear_forward_int8 once per buffer (4 per layer, 128 launches), each
+    INT8 weight read once and dequantized in registers.  Beside it, on the same
+    buffers: the two-step path (qg_linear_dequant_weight into a bf16 scratch,
+    then the tcgen05 qg_linear_forward), and the fused kernel once per matrix
+    (224 launches).  The weights (6.5 GB) are larger than L2, so every step reads
+    them from HBM.  Every rank runs its own stack (weak scaling)."""
+    import torch
+    import torch.distributed as dist
+
+    import quantized_rank_gradient_b200 as qg
+    import synth
+    qg.lib()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    spec = STACKS["llama7b-stack"]
+    layers = args.layers or spec["layers"]
+    if not 1 <= args.tokens <= 16:
+        raise SystemExit("--tokens must be in 1..16")
+    stream = c_void_p(torch.cuda.current_stream().cuda_stream)
+    h, f = spec["hidden"], spec["inter"]
+    # per layer: (rows of each stacked matrix, n)
+    layout = [((h, h, h), h), ((h,), h), ((f, f), h), ((h,), f)]
+    bufs, mats = [], []
+    for layer in range(layers):
+        for bi, (rows, n) in enumerate(layout):
+            m = sum(rows)
+            ldw = -(-n // 16) * 16
+            seed = matrix_seed(rank, layer * len(layout) + bi)
+            W = synth.device_weight_codes(m, n, ldw, seed, device)
+            sW = synth.device_weight_scales(m, n, seed, device)
+            bufs.append((m, n, W, ldw, sW))
+            r0 = 0
+            for r in rows:  # the matrices as row slices of the buffer
+                mats.append((r, n, W[r0:], ldw, sW[(r0 * n) // 256:]))
+                r0 += r
+    gen = torch.Generator(device=device)
+    gen.manual_seed(5_000_011 * (rank + 1))
+    bf = torch.bfloat16
+    shapes = sorted({(m, n) for (m, n, *_r) in bufs} | {(m, n) for (m, n, *_r) in mats})
+    io = {(m, n): dict(X=torch.randn(16, n, generator=gen, device=device).to(bf),
+                       Y=torch.empty(16, m, dtype=bf, device=device),
+                       Wt=torch.empty(m, -(-n // 8) * 8, dtype=bf, device=device))
+          for (m, n) in shapes}
+
+    def fused(T, items=bufs):
+        for (m, n, W, ldw, sW) in items:
+            b = io[(m, n)]
+            qg.check(qg.qg_linear_forward_int8(b["X"].data_ptr(), n, W.data_ptr(), ldw, sW.data_ptr(), T, m, n,
+                                               b["Y"].data_ptr(), m, stream), "qg_linear_forward_int8")
+
+    def per_matrix(T):
+        fused(T, mats)
+
+    def two_step(T):
+        for (m, n, W, ldw, sW) in bufs:
+            b = io[(m, n)]
+            ldt = b["Wt"].shape[1]
+            qg.check(qg.qg_linear_dequant_weight(W.data_ptr(), ldw, sW.data_ptr(), m, n, b["Wt"].data_ptr(), ldt,
+                                                 stream), "qg_linear_dequant_weight")
+            qg.check(qg.qg_linear_forward(b["X"].data_ptr(), n, b["Wt"].data_ptr(), ldt, T, m, n, b["Y"].data_ptr(),
+                                          m, stream), "qg_linear_forward")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def timed(fn, T, steps, warmup, profile=False):
+        for _ in range(warmup):
+            fn(T)
+        barrier()
+        torch.cuda.synchronize()
+        if profile:
+            qg.check(qg.qg_profile_enable(1))
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(steps):
+            fn(T)
+        t1.record()
+        torch.cuda.synchronize()
+        kt = None
+        if profile:
+            kt = (qg.qg_kernel_times * qg.QG_KERNEL_KINDS)()
+            qg.check(qg.qg_profile_collect(kt, qg.QG_KERNEL_KINDS))
+            qg.check(qg.qg_profile_enable(0))
+        barrier()
+        return reduce_max(t0.elapsed_time(t1) / steps, world), kt
+
+    weights = sum(m * n for (m, n, *_r) in bufs)
+    T = args.tokens
+    clocks = ClockSampler(bus_id_of(device))
+    clocks.start()
+    time.sleep(0.3)
+    ms, _ = timed(fused, T, args.steps, args.warmup)
+    clk = clocks.stop()
+    # per-launch device times (events around each launch) from a separate pass,
+    # so that the headline time carries no profiling events
+    _, kt = timed(fused, T, max(3, args.steps // 4), 1, profile=True)
+    sweep = {}
+    for Ts in DECODE_TOKENS:
+        n_steps = max(3, args.steps // 4)
+        f_ms, _ = timed(fused, Ts, n_steps, args.warmup)
+        p_ms, _ = timed(per_matrix, Ts, n_steps, args.warmup)
+        t_ms, _ = timed(two_step, Ts, n_steps, args.warmup)
+        sweep[str(Ts)] = {"fused_ms": f_ms, "fused_per_matrix_ms": p_ms, "two_step_ms": t_ms,
+                          "speedup_vs_two_step": t_ms / f_ms, "fused_tbs": weights / (f_ms / 1000.0) / 1e12}
+    if rank != 0:
+        return 0
+    peaks = load_peaks()
+    k = kt[qg.QG_KERNEL_LINEAR_FUSED]
+    achieved = (k.bytes / k.launches) / (k.device_ms / k.launches / 1000.0) / 1e9
+    line = {
+        "metric": "INT8-weight forward for a few tokens (Y = X W~^T, W read once): INT8 weights/s",
+        "value": weights / (ms / 1000.0) * world, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "INT8 weights, bf16 activations, f32 accumulate, bf16 out",
+        "data": "synthetic (seeded bf16 activations; seeded INT8 weights and scales)",
+        "config": {"workload": f"linear-llama7b-stack-decode-{T}tok" + ("" if layers == spec["layers"]
+                                                                       else f"-{layers}l"),
+                   "buffers": len(bufs), "matrices": len(mats), "tokens": T, "weights_per_gpu": weights,
+                   "layout": "per layer: qkv 12288x4096, o 4096x4096, gate_up 22016x4096, down 4096x11008",
+                   "l2": "inputs larger than L2 (6.5 GB of INT8 weights per step)",
+                   "parallelism": f"independent stacks x{world}"},
+        "roofline": {"bound": "hbm", "kernel": "linear_forward_int8", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": None, "peak_kind": "HBM copy (%s)" % peaks["source"]},
+        "kernels": {"linear_forward_int8": {"launches_per_step": len(bufs),
+                                            "device_ms_per_launch": k.device_ms / k.launches, "gbs": achieved}},
+        "tokens_sweep": sweep,
+        "gpu_launches": len(bufs) * args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_e2e(stack, args, stream, world, device, barrier):
     import torch
     import torch.distributed as dist
@@ -823,6 +974,8 @@ def main():
             return run_refresh_stress(args, rank, world, local_rank)
         if args.workload == "linear-7b":
             return run_linear(args, rank, world, local_rank)
+        if args.workload == "linear-7b-decode":
+            return run_linear_decode(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:

@@ -55,7 +55,7 @@ class qg_kernel_times(Structure):
 
 
 (QG_KERNEL_DEQUANT, QG_KERNEL_PROJECT_ADAM, QG_KERNEL_BACKPROJECT_SR, QG_KERNEL_OTHER, QG_KERNEL_LINEAR_DEQUANT,
- QG_KERNEL_LINEAR_GEMM, QG_KERNEL_KINDS) = range(7)
+ QG_KERNEL_LINEAR_GEMM, QG_KERNEL_LINEAR_FUSED, QG_KERNEL_KINDS) = range(8)
 
 _SIGNATURES = {
     "qg_status_str": (c_char_p, [c_int32]),
@@ -96,6 +96,8 @@ _SIGNATURES = {
                                            c_void_p]),
     "qg_linear_forward": (c_int32, [c_void_p, c_int64, c_void_p, c_int64, c_int32, c_int32, c_int32, c_void_p,
                                     c_int64, c_void_p]),
+    "qg_linear_forward_int8": (c_int32, [c_void_p, c_int64, c_void_p, c_int64, c_void_p, c_int32, c_int32, c_int32,
+                                         c_void_p, c_int64, c_void_p]),
     "qg_linear_backward_data": (c_int32, [c_void_p, c_int64, c_void_p, c_int64, c_int32, c_int32, c_int32,
                                           c_void_p, c_int64, c_void_p]),
     "qg_linear_backward_weight": (c_int32, [c_void_p, c_int64, c_void_p, c_int64, c_int32, c_int32, c_int32,

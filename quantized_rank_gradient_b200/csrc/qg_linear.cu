@@ -16,6 +16,8 @@
 // repeat the conversion once per 128-row tile of activations on the same
 // schedulers that issue the MMAs, while the separate pass costs three bytes of
 // HBM traffic per weight.
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 #include <cstring>
 #include <mutex>
@@ -94,6 +96,457 @@ __global__ void __launch_bounds__(256) dequant_weight_kernel(const int8_t* __res
       if (c < total) dequant_chunk(q[u], c / chunks, static_cast<int>(c % chunks) * 16, n, sW, Wt, ldt);
     }
   }
+}
+
+// ---------------------------------------------------------------- Y = X W~^T for a few tokens, W read once
+
+// For T <= 16 tokens the forward product is bound by reading the weight: the
+// separate dequantization moves three bytes per weight and the GEMM two more,
+// where this kernel reads the INT8 codes once and forms W~ = bf16(fp32(q) * s)
+// in registers, rounded exactly as dequant_weight_kernel rounds it.
+//
+// Work split.  A CTA owns kF8Rows rows of W and one slice of its columns; the
+// S slices of one row block form a thread-block cluster (split K), sized so
+// that the clusters fit the GPU at once.  The partial sums are added across
+// the cluster through distributed shared memory in the order of the CTA ranks,
+// so every output is the same sum whichever CTA adds it, rounded once to bf16.
+//
+// Data movement.  One producer thread streams the slice through a ring of
+// kF8Stages shared-memory stages by TMA, 128 columns a stage: the W tile (64
+// rows x 128 bytes) and the X tile (8 or 16 token rows x 128 columns, two
+// boxes of 64 columns), all with the 128-byte swizzle.  Rows past m or T and
+// columns past n arrive as zeros, and the bytes in flight cost no registers.
+//
+// Arithmetic.  Four consumer warps own 16 rows each.  The product runs on the
+// tensor cores with mma.sync m16n8k16 (bf16 in, f32 accumulate), whose A
+// operand comes from registers: the dequantized weight goes from the
+// conversion straight into the fragment.  Any bijection of a stage's columns
+// onto k-positions gives the same sum.  In step s (of two) the lane with
+// thread-in-group t takes the 16 columns of chunk w = 2t + (s ^ (t >> 1)) (16
+// columns, 16 bytes of W); in MMA j its k-pairs (2t, 2t+1) and (2t+8, 2t+9)
+// are columns 4j + {0, 1} and 4j + {2, 3} of those 16, and the B fragment of
+// token g is the eight bytes of X there.  With this order the eight lanes of a
+// quarter warp read eight distinct 16-byte bank groups of the swizzled W tile
+// (distinct w >> 1, two rows) and of the X tile (distinct w & 3, two tokens).
+// The work is bound by HBM at 2T <= 32 flops per weight byte; the tensor cores
+// keep the multiply-adds off the schedulers, which the conversion occupies
+// (about 2.75 instructions a weight).
+constexpr int kF8Warps = 4;                        // consumer warps, 16 rows each
+constexpr int kF8Rows = 16 * kF8Warps;             // rows of W per CTA
+constexpr int kF8Threads = 32 * (kF8Warps + 1);    // + the producer warp
+constexpr int kF8Tile = 128;                       // columns per ring stage
+constexpr int kF8WBytes = kF8Rows * kF8Tile;       // W tile: 8 KB
+constexpr int kF8Stages = 4;
+constexpr int kF8MaxCluster = 8;                   // portable cluster size
+
+// X tile of a stage: kNT * 8 token rows x 128 columns of bf16, two 64-column boxes
+template <int kNT>
+__host__ __device__ constexpr int f8_xbox_bytes() {
+  return kNT * 8 * 128;
+}
+
+template <int kNT>
+__host__ __device__ constexpr int f8_stage_bytes() {
+  return kF8WBytes + 2 * f8_xbox_bytes<kNT>();  // a multiple of 1024 (the swizzle atom)
+}
+
+template <int kNT>
+__host__ __device__ constexpr int f8_smem_bytes() {
+  return 1024 + kF8Stages * f8_stage_bytes<kNT>();  // + alignment slack for the ring
+}
+
+// CTAs per SM (shared memory: four rings of 40 or 48 KB; registers)
+constexpr int kF8CtasPerSm = 4;
+
+QG_DEV float ld_shared_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+QG_DEV uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+
+QG_DEV void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                           uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+QG_DEV uint64_t pack_f32x2(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+
+// Four weights (the bytes of a word of codes, lowest first) as two bf16 pairs,
+// each bf16(fp32(q) * s) with its own scale (sc01: weights 0, 1; sc23: 2, 3).
+// The codes biased by 128 (q ^ 0x80 as unsigned bytes u) are placed two at a
+// time in the low mantissa bits of two fp16 halves of 1024 (0x6400 | u = the
+// fp16 1024 + u, exact); one mixed-precision addition per weight widens a half
+// to float32 and subtracts 1152, giving q exactly; the products with the
+// scales are packed f32x2 multiplies (round to nearest), then each pair is
+// rounded to bf16 (nearest even), the lower column in the low half.
+QG_DEV void w_tilde4(uint32_t word, uint64_t sc01, uint64_t sc23, uint32_t& p01, uint32_t& p23) {
+  const uint32_t biased = word ^ 0x80808080u;
+  const uint32_t h01 = __byte_perm(biased, 0x64646464u, 0x5140u);
+  const uint32_t h23 = __byte_perm(biased, 0x64646464u, 0x7362u);
+  uint64_t v01, v23;
+  asm("{\n\t.reg .b16 a, b, c, d;\n\t.reg .f32 fa, fb, fc, fd;\n\t"
+      "mov.b32 {a, b}, %2;\n\tmov.b32 {c, d}, %3;\n\t"
+      "add.rn.f32.f16 fa, a, 0fC4900000;\n\tadd.rn.f32.f16 fb, b, 0fC4900000;\n\t"
+      "add.rn.f32.f16 fc, c, 0fC4900000;\n\tadd.rn.f32.f16 fd, d, 0fC4900000;\n\t"
+      "mov.b64 %0, {fa, fb};\n\tmov.b64 %1, {fc, fd};\n\t}"
+      : "=l"(v01), "=l"(v23)
+      : "r"(h01), "r"(h23));
+  asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(v01) : "l"(sc01));
+  asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(v23) : "l"(sc23));
+  uint32_t a, b, c, d;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(v01));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(c), "=r"(d) : "l"(v23));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p01) : "r"(b), "r"(a));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p23) : "r"(d), "r"(c));
+}
+
+// W~ of sixteen consecutive weights as eight bf16 pairs: weights k < split
+// take scale s0, the others s1 (kOneGroup: all take s1).
+template <bool kOneGroup>
+QG_DEV void w_tilde16(const uint4& q, float s0, float s1, int split, uint32_t (&out)[8]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  const uint64_t one = pack_f32x2(__float_as_uint(s1), __float_as_uint(s1));
+#pragma unroll
+  for (int k = 0; k < 16; k += 4) {
+    uint64_t sc01 = one, sc23 = one;
+    if (!kOneGroup) {
+      sc01 = pack_f32x2(__float_as_uint(k < split ? s0 : s1), __float_as_uint(k + 1 < split ? s0 : s1));
+      sc23 = pack_f32x2(__float_as_uint(k + 2 < split ? s0 : s1), __float_as_uint(k + 3 < split ? s0 : s1));
+    }
+    w_tilde4(w[k >> 2], sc01, sc23, out[k >> 1], out[(k >> 1) + 1]);
+  }
+}
+
+// The scales of sixteen consecutive weights of row i (columns j0..j0+15) when
+// n is not a multiple of 256: weights k < split take s0, the others s1
+// (split <= 0: one group).  Columns at or past n take the group of the row's
+// last weight (their codes arrive as zeros), so every index stays inside s_W.
+struct Scales16 {
+  float s0, s1;
+  int split;
+};
+
+QG_DEV Scales16 scales16(int64_t i, int j0, int32_t n, const float* __restrict__ sW) {
+  const int64_t e0 = i * n + j0;
+  const int64_t g0 = (i * n + min(j0, n - 1)) >> 8, g1 = (i * n + min(j0 + 15, n - 1)) >> 8;
+  Scales16 r;
+  r.s1 = __ldg(sW + g1);
+  r.s0 = g1 != g0 ? __ldg(sW + g0) : r.s1;
+  r.split = static_cast<int>((g1 << 8) - e0);
+  return r;
+}
+
+// The four MMAs of a step on two accumulator sets (MMAs 0, 1 and 2, 3), so
+// that the chain of dependent MMAs is half as long.  x0, x1: this lane's two
+// 8-column chunks of X in the step, for tokens g (+ 8 nt).
+template <int kNT>
+QG_DEV void f8_mma(const uint32_t (&wa)[8], const uint32_t (&wb)[8], const uint4 (&x0)[kNT], const uint4 (&x1)[kNT],
+                   float (&acc)[2][kNT][4]) {
+#pragma unroll
+  for (int nt = 0; nt < kNT; ++nt) {
+    mma_bf16_16816(acc[0][nt], wa[0], wb[0], wa[1], wb[1], x0[nt].x, x0[nt].y);
+    mma_bf16_16816(acc[0][nt], wa[2], wb[2], wa[3], wb[3], x0[nt].z, x0[nt].w);
+    mma_bf16_16816(acc[1][nt], wa[4], wb[4], wa[5], wb[5], x1[nt].x, x1[nt].y);
+    mma_bf16_16816(acc[1][nt], wa[6], wb[6], wa[7], wb[7], x1[nt].z, x1[nt].w);
+  }
+}
+
+// Grid: one CTA per (row block, column slice), blockIdx.x = block * S + slice,
+// launched in clusters of S along x; slice is a multiple of kF8Tile (of 256
+// when kGroupRows: n % 256 == 0, so that a stage of a row lies in one scale
+// group).
+template <int kNT, bool kGroupRows>
+__global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) linear_forward_int8_kernel(
+    const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const float* __restrict__ sW,
+    int32_t T, int32_t m, int32_t n, int32_t slice, uint16_t* __restrict__ Y, int64_t ldy) {
+  constexpr int kStage = f8_stage_bytes<kNT>();
+  constexpr int kXBox = f8_xbox_bytes<kNT>();
+  extern __shared__ uint8_t f8_smem[];
+  __shared__ float red[kNT * 8][kF8Rows];  // this CTA's partial sums, [token][row]
+  __shared__ uint64_t full[kF8Stages], empty[kF8Stages];
+  __shared__ int abort_flag;
+  uint8_t* ring = f8_smem + ((1024 - (smem_u32(f8_smem) & 1023)) & 1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = static_cast<int>(cluster_nctarank());
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int block = blockIdx.x / S;
+  const int kbeg = rank * slice, kend = min(n, kbeg + slice);
+  const int nstage = (kend - kbeg + kF8Tile - 1) / kF8Tile;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kF8Stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kF8Warps);
+    }
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kF8Warps) {
+    // producer: one thread streams the slice's stages (W tile, two X boxes) through the ring
+    if (lane == 0) {
+      tma_prefetch_map(&tmW);
+      tma_prefetch_map(&tmX);
+      int issued = 0;
+      for (int k = 0; k < nstage; ++k) {
+        const int slot = k % kF8Stages;
+        if (k >= kF8Stages && !mbar_wait(&empty[slot], ((k / kF8Stages) - 1) & 1, &abort_flag, nullptr)) break;
+        uint8_t* st = ring + slot * kStage;
+        const int col = kbeg + k * kF8Tile;
+        mbar_arrive_expect_tx(&full[slot], kStage);
+        tma_load_2d(st, &tmW, &full[slot], col, block * kF8Rows);
+        tma_load_2d(st + kF8WBytes, &tmX, &full[slot], col, 0);
+        tma_load_2d(st + kF8WBytes + kXBox, &tmX, &full[slot], col + 64, 0);
+        issued = k + 1;
+      }
+      // every load issued has landed before the CTA can leave (bounded)
+      for (int k = max(0, issued - kF8Stages); k < issued; ++k)
+        mbar_wait_drain(&full[k % kF8Stages], (k / kF8Stages) & 1);
+    }
+    __syncwarp();
+  } else {
+    const int g = lane >> 2, t = lane & 3;
+    const int r0 = warp * 16 + g;  // fragment rows r0 and r0 + 8 of the CTA's block
+    const int64_t ra = static_cast<int64_t>(block) * kF8Rows + r0, rb = ra + 8;
+    const int64_t ia = ra < m ? ra : 0, ib = rb < m ? rb : 0;  // rows past m: zero codes, row 0's scales
+    const float* srow_a = sW + (kGroupRows ? ia * (n >> 8) : 0);
+    const float* srow_b = sW + (kGroupRows ? ib * (n >> 8) : 0);
+    // per step s: the lane's chunk w (16 columns), its swizzled W offset in rows
+    // r0 and r0 + 8 (same row & 7), and its two 8-column X chunks (token g)
+    int woff[2], xoff0[2], xoff1[2], wcol[2];
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int w = 2 * t + (s ^ (t >> 1));
+      wcol[s] = 16 * w;
+      woff[s] = r0 * kF8Tile + ((w ^ (r0 & 7)) << 4);
+      const int xb = kF8WBytes + (w >> 2) * kXBox + g * 128, c = 2 * (w & 3);
+      xoff0[s] = xb + ((c ^ (g & 7)) << 4);
+      xoff1[s] = xb + (((c + 1) ^ (g & 7)) << 4);
+    }
+    float acc[2][kNT][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) acc[h][nt][0] = acc[h][nt][1] = acc[h][nt][2] = acc[h][nt][3] = 0.f;
+    // kGroupRows: the scales of the current and the next pair of stages (one group per row each)
+    float sa = 0.f, sb = 0.f, na = 0.f, nb = 0.f;
+    if (kGroupRows) {
+      na = __ldg(srow_a + (kbeg >> 8));
+      nb = __ldg(srow_b + (kbeg >> 8));
+    }
+    // after a timed-out wait (abort) the loop does no more work
+    bool ok = true;
+    for (int k = 0; k < nstage && ok; ++k) {
+      const int col = kbeg + k * kF8Tile;
+      if (kGroupRows && (k & 1) == 0) {
+        sa = na;
+        sb = nb;
+        if (k + 2 < nstage) {
+          na = __ldg(srow_a + ((col + 256) >> 8));
+          nb = __ldg(srow_b + ((col + 256) >> 8));
+        }
+      }
+      const int slot = k % kF8Stages;
+      // a warp vote, so that the lanes of a warp agree even when a wait times out
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[slot], (k / kF8Stages) & 1, &abort_flag, nullptr));
+      if (!ok) break;
+      const uint8_t* st = ring + slot * kStage;
+      uint4 qa[2], qb[2], x0[2][kNT], x1[2][kNT];
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        qa[s] = *reinterpret_cast<const uint4*>(st + woff[s]);
+        qb[s] = *reinterpret_cast<const uint4*>(st + woff[s] + 8 * kF8Tile);
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+          x0[s][nt] = *reinterpret_cast<const uint4*>(st + xoff0[s] + nt * 8 * 128);
+          x1[s][nt] = *reinterpret_cast<const uint4*>(st + xoff1[s] + nt * 8 * 128);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);  // the stage is in registers
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        uint32_t wa[8], wb[8];
+        if constexpr (kGroupRows) {
+          w_tilde16<true>(qa[s], 0.f, sa, 0, wa);
+          w_tilde16<true>(qb[s], 0.f, sb, 0, wb);
+        } else {
+          const int j0 = col + wcol[s];
+          const Scales16 za = scales16(ia, j0, n, sW), zb = scales16(ib, j0, n, sW);
+          // a warp vote: every lane takes the same path to the MMAs
+          if (__all_sync(0xFFFFFFFFu, za.split <= 0 && zb.split <= 0)) {
+            w_tilde16<true>(qa[s], 0.f, za.s1, 0, wa);
+            w_tilde16<true>(qb[s], 0.f, zb.s1, 0, wb);
+          } else {
+            w_tilde16<false>(qa[s], za.s0, za.s1, za.split, wa);
+            w_tilde16<false>(qb[s], zb.s0, zb.s1, zb.split, wb);
+          }
+        }
+        f8_mma<kNT>(wa, wb, x0[s], x1[s], acc);
+      }
+    }
+    // partial sums: lane (g, t) holds rows r0 and r0 + 8, tokens 2t, 2t + 1 of each 8
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) {
+      const int tok = nt * 8 + 2 * t;
+      red[tok][r0] = __fadd_rn(acc[0][nt][0], acc[1][nt][0]);
+      red[tok + 1][r0] = __fadd_rn(acc[0][nt][1], acc[1][nt][1]);
+      red[tok][r0 + 8] = __fadd_rn(acc[0][nt][2], acc[1][nt][2]);
+      red[tok + 1][r0 + 8] = __fadd_rn(acc[0][nt][3], acc[1][nt][3]);
+    }
+  }
+  cluster_sync();  // every CTA's partial sums are written
+  constexpr int kOut = kNT * 8 * kF8Rows;
+  const int o0 = rank * kOut / S, o1 = (rank + 1) * kOut / S;
+  for (int o = o0 + static_cast<int>(threadIdx.x); o < o1; o += kF8Threads) {
+    const int tok = o / kF8Rows, row = o % kF8Rows;
+    const int64_t i = static_cast<int64_t>(block) * kF8Rows + row;
+    if (tok < T && i < m) {
+      const float* mine = &red[0][0] + o;
+      float part[kF8MaxCluster];
+#pragma unroll
+      for (int q = 0; q < kF8MaxCluster; ++q) part[q] = q < S ? ld_shared_cluster_f32(mapa_shared(mine, q)) : 0.f;
+      float v = part[0];
+#pragma unroll
+      for (int q = 1; q < kF8MaxCluster; ++q)
+        if (q < S) v = __fadd_rn(v, part[q]);
+      Y[static_cast<int64_t>(tok) * ldy + i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    }
+  }
+  cluster_sync();  // no CTA leaves while another reads its partial sums
+}
+
+// Column slices per row block: as many as keep all clusters resident at once
+// (the occupancy query, for each cluster size from the largest down), at most
+// a portable cluster, each a multiple of kF8Tile columns (of 256 when
+// n % 256 == 0).
+struct F8Split {
+  int S, slice, blocks;
+};
+
+F8Split forward_int8_split(int32_t m, int32_t n, const int (&clusters_fit)[kF8MaxCluster + 1]) {
+  F8Split f;
+  f.blocks = (m + kF8Rows - 1) / kF8Rows;
+  const int unit = n % 256 == 0 ? 256 : kF8Tile;
+  int S = std::max(1, std::min(kF8MaxCluster, (n + unit - 1) / unit));
+  while (S > 1 && f.blocks > clusters_fit[S]) --S;
+  f.slice = ((n + S - 1) / S + unit - 1) / unit * unit;
+  f.S = (n + f.slice - 1) / f.slice;  // no empty slice
+  return f;
+}
+
+// A row-major 2-D tensor (rows x cols elements of esize bytes, row stride ld
+// elements) as TMA boxes of box_rows x box_cols, 128-byte swizzle; rows and
+// columns past the edge read as zeros.
+PFN_cuTensorMapEncodeTiled_v12000 f8_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool encode_rows(CUtensorMap* map, CUtensorMapDataType dtype, int esize, const void* base, int64_t ld, int64_t rows,
+                 int64_t cols, int box_rows, int box_cols) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = f8_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * esize)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Per instantiation: the dynamic shared memory attribute, and how many
+// clusters of each size fit on the device at once.
+template <int kNT, bool kGroupRows>
+struct F8Kernel {
+  cudaError_t err = cudaSuccess;
+  int fit[kF8MaxCluster + 1] = {};
+  F8Kernel() {
+    const auto kern = linear_forward_int8_kernel<kNT, kGroupRows>;
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, f8_smem_bytes<kNT>());
+    for (int S = 1; S <= kF8MaxCluster && err == cudaSuccess; ++S) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(S));
+      cfg.blockDim = dim3(kF8Threads);
+      cfg.dynamicSmemBytes = static_cast<size_t>(f8_smem_bytes<kNT>());
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      err = cudaOccupancyMaxActiveClusters(&fit[S], kern, &cfg);
+    }
+  }
+};
+
+template <int kNT, bool kGroupRows>
+cudaError_t launch_forward_int8_as(const CUtensorMap& tmW, const uint16_t* X, int64_t ldx, const float* sW, int T,
+                                   int m, int n, uint16_t* Y, int64_t ldy, cudaStream_t s) {
+  static F8Kernel<kNT, kGroupRows> kinfo;  // per process: one device
+  if (kinfo.err != cudaSuccess) return kinfo.err;
+  const F8Split f = forward_int8_split(m, n, kinfo.fit);
+  if (static_cast<int64_t>(f.blocks) * f.S > INT32_MAX) return cudaErrorInvalidValue;
+  CUtensorMap tmX;
+  if (!encode_rows(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, ldx, T, n, kNT * 8, 64)) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(f.blocks * f.S));
+  cfg.blockDim = dim3(kF8Threads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(f8_smem_bytes<kNT>());
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(f.S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, linear_forward_int8_kernel<kNT, kGroupRows>, tmW, tmX, sW, T, m, n, f.slice, Y,
+                            ldy);
+}
+
+cudaError_t launch_forward_int8(const uint16_t* X, int64_t ldx, const int8_t* W, int64_t ldw, const float* sW, int T,
+                                int m, int n, uint16_t* Y, int64_t ldy, cudaStream_t s) {
+  CUtensorMap tmW;
+  if (!encode_rows(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, W, ldw, m, n, kF8Rows, kF8Tile))
+    return cudaErrorInvalidValue;
+  const double bytes = static_cast<double>(m) * n + 4.0 * ((static_cast<double>(m) * n + 255) / 256) +
+                       2.0 * T * n + 2.0 * T * m;
+  const int tok = profile_begin(s, QG_KERNEL_LINEAR_FUSED, 2.0 * T * m * n, bytes);
+  const bool rows = n % 256 == 0;
+  cudaError_t e;
+  if (T <= 8)
+    e = rows ? launch_forward_int8_as<1, true>(tmW, X, ldx, sW, T, m, n, Y, ldy, s)
+             : launch_forward_int8_as<1, false>(tmW, X, ldx, sW, T, m, n, Y, ldy, s);
+  else
+    e = rows ? launch_forward_int8_as<2, true>(tmW, X, ldx, sW, T, m, n, Y, ldy, s)
+             : launch_forward_int8_as<2, false>(tmW, X, ldx, sW, T, m, n, Y, ldy, s);
+  profile_end(s, tok);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- bf16 store epilogue
@@ -246,6 +699,21 @@ qg_status qg_linear_forward(const void* d_X, int64_t ldx, const void* d_Wt, int6
   // Y (T x m) = X (T x n, K-major) W~^T (W~ m x n is B given N x K: K-major)
   return status_of(launch_bf16<false, false>(d_X, ldx, d_Wt, ldwt, static_cast<uint16_t*>(d_Y), ldy, T, m, n,
                                              static_cast<cudaStream_t>(stream)));
+}
+
+qg_status qg_linear_forward_int8(const void* d_X, int64_t ldx, const int8_t* d_W, int64_t ldw, const float* d_sW,
+                                 int32_t T, int32_t m, int32_t n, void* d_Y, int64_t ldy, void* stream) {
+  if (T < 0 || T > 16 || m <= 0 || n <= 0) return QG_ESHAPE;
+  if (!d_W || !d_sW) return QG_EINVAL;
+  if (ldw < n || ldw % 16 != 0) return QG_ESHAPE;
+  if (!aligned16(d_W)) return QG_EALIGN;
+  qg_status st;
+  if ((st = check_bf16(d_X, ldx, T, n)) != QG_OK || (st = check_bf16(d_Y, ldy, T, m)) != QG_OK) return st;
+  if (T == 0) return QG_OK;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint16_t* X = static_cast<const uint16_t*>(d_X);
+  uint16_t* Y = static_cast<uint16_t*>(d_Y);
+  return status_of(launch_forward_int8(X, ldx, d_W, ldw, d_sW, T, m, n, Y, ldy, s));
 }
 
 qg_status qg_linear_backward_data(const void* d_dY, int64_t lddy, const void* d_Wt, int64_t ldwt, int32_t T,

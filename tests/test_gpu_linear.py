@@ -213,3 +213,123 @@ def test_full_size_sampled(m, n):
             S = float(np.abs(a64) @ np.abs(b64))
             g = float(O.bf16_from_bits(np.array([got], np.uint16))[0])
             assert abs(g - exact) <= 2.0 ** -8 * abs(exact) + a.size * 2.0 ** -21 * S, (t, i, j, g, exact)
+
+
+# ---------------------------------------------------------------- Y = X W~^T for a few tokens, INT8 W read once
+
+def _weights_junk_pad(m, n, seed, ldw):
+    """INT8 codes with random bytes in the row padding (columns n..ldw), which
+    the fused forward must not let into Y."""
+    Wq, sW, _, _, dsW = _weights(m, n, seed, ldw=ldw)
+    Wpad = np.random.default_rng(seed + 1).integers(-128, 128, size=(m, ldw)).astype(np.int8)
+    Wpad[:, :n] = Wq
+    return Wq, sW, torch.from_numpy(Wpad).cuda(), dsW
+
+
+def _forward_int8(dXa, ldx, dW, ldw, dsW, T, m, n, ld_extra=8):
+    Y, ldy = _empty_bf16(T, m, ld=-(-m // 8) * 8 + ld_extra)
+    qg.check(qg.qg_linear_forward_int8(dXa.data_ptr(), ldx, dW.data_ptr(), ldw, dsW.data_ptr(), T, m, n,
+                                       Y.data_ptr(), ldy, stream()))
+    return Y
+
+
+# (m, n, ldw): ragged rows and columns, scale groups straddling 16-column
+# chunks (n % 256 != 0), one column slice per CTA (m large: several phases of
+# staged X) and eight (m small)
+FUSED_SHAPES = [(37, 64, 64), (300, 700, 720), (640, 1365, 1376), (129, 4096, 4096), (20000, 2600, 2608)]
+
+
+@pytest.mark.parametrize("T", [1, 3, 8, 9, 16])
+@pytest.mark.parametrize("m,n,ldw", FUSED_SHAPES)
+def test_forward_int8_parity(T, m, n, ldw):
+    Wq, sW, dW, dsW = _weights_junk_pad(m, n, seed=7 * T + m, ldw=ldw)
+    Xb = _acts(T, n, seed=T + n)
+    dXa, ldx = _bf16_dev(Xb, ld=-(-n // 8) * 8 + 8)
+    Y = _forward_int8(dXa, ldx, dW, ldw, dsW, T, m, n)
+    Wt = O.dequant_weight_bf16(Wq, sW)
+    X = O.bf16_from_bits(Xb)
+    _within_bar(_read_bf16(Y, T, m), X, Wt.T, O.linear_forward(X, Wt))
+    # nothing written past T rows or m columns
+    Yh = Y.cpu().numpy().view(np.uint16)
+    assert (Yh[:T, m:] == 0x7FC0).all() and (Yh[T:] == 0x7FC0).all()
+
+
+@pytest.mark.parametrize("m,n", [(4096, 11008), (11008, 4096)])
+@pytest.mark.parametrize("T", [1, 16])
+def test_forward_int8_full_size(T, m, n):
+    # the 7B stack's MLP shapes at decode sizes, every output against the oracle
+    Wq, sW, dW, ldw, dsW = _weights(m, n, seed=m + T)
+    Xb = _acts(T, n, seed=T)
+    dXa, ldx = _bf16_dev(Xb)
+    Y = _forward_int8(dXa, ldx, dW, ldw, dsW, T, m, n, ld_extra=0)
+    Wt = O.dequant_weight_bf16(Wq, sW)
+    X = O.bf16_from_bits(Xb)
+    _within_bar(_read_bf16(Y, T, m), X, Wt.T, O.linear_forward(X, Wt))
+
+
+def test_forward_int8_bit_exact_on_small_integers():
+    # codes in {-1, 0, 1} (one in 32 nonzero), power-of-two scales and X in
+    # {-1, 0, 1}: every partial sum, the sum over the cluster's slices and the
+    # result are integers times 2^-3 of magnitude < 256 * 2^-3, exact in
+    # float32 and in bf16, so the split-K reduction and the operand layouts are
+    # checked bit for bit
+    rng = np.random.default_rng(33)
+    T, m, n = 16, 300, 4000
+    Wq = (rng.integers(-1, 2, size=(m, n)) * (rng.integers(0, 32, size=(m, n)) == 0)).astype(np.int8)
+    sW = np.full(-(-(m * n) // 256), 0.125, np.float32)
+    X = rng.integers(-1, 2, size=(T, n)).astype(np.float32)
+    exact = X.astype(np.int64) @ Wq.astype(np.int64).T
+    assert np.abs(exact).max() < 256
+    ldw = -(-n // 16) * 16
+    Wpad = np.zeros((m, ldw), np.int8)
+    Wpad[:, :n] = Wq
+    dW, dsW = torch.from_numpy(Wpad).cuda(), torch.from_numpy(sW).cuda()
+    dXa, ldx = _bf16_dev(O.bf16_bits(X))
+    Y = _forward_int8(dXa, ldx, dW, ldw, dsW, T, m, n)
+    np.testing.assert_array_equal(_read_bf16(Y, T, m), (exact * 0.125).astype(np.float32))
+
+
+def test_forward_int8_deterministic_and_agrees_with_two_step_path():
+    # the same bits on every call (the slices' partial sums are added in a
+    # fixed order); the dequantize-then-GEMM path meets the same bar on the
+    # same inputs
+    T, m, n = 8, 4096, 4096
+    Wq, sW, dW, ldw, dsW = _weights(m, n, seed=5)
+    Xb = _acts(T, n, seed=6)
+    dXa, ldx = _bf16_dev(Xb)
+    Y1 = _forward_int8(dXa, ldx, dW, ldw, dsW, T, m, n)
+    Y2 = _forward_int8(dXa, ldx, dW, ldw, dsW, T, m, n)
+    assert torch.equal(Y1, Y2)
+    Wt_dev, ldt = _dequant_dev(dW, ldw, dsW, m, n)
+    Y3, ldy = _empty_bf16(T, m)
+    qg.check(qg.qg_linear_forward(dXa.data_ptr(), ldx, Wt_dev.data_ptr(), ldt, T, m, n, Y3.data_ptr(), ldy, stream()))
+    X, Wt = O.bf16_from_bits(Xb), O.dequant_weight_bf16(Wq, sW)
+    exact = O.linear_forward(X, Wt)
+    for Y in (Y1, Y3):
+        _within_bar(_read_bf16(Y, T, m), X, Wt.T, exact)
+
+
+def test_forward_int8_edges():
+    m, n = 64, 128
+    Wq, sW, dW, ldw, dsW = _weights(m, n, seed=1)
+    X, ldx = _bf16_dev(np.zeros((17, n), np.uint16))
+    Y, ldy = _empty_bf16(17, m)
+    s = stream()
+    # T = 0: nothing written
+    qg.check(qg.qg_linear_forward_int8(X.data_ptr(), ldx, dW.data_ptr(), ldw, dsW.data_ptr(), 0, m, n, Y.data_ptr(),
+                                       ldy, s))
+    torch.cuda.synchronize()
+    assert (Y.cpu().numpy().view(np.uint16) == 0x7FC0).all()
+    # more than 16 tokens, a weight stride that is not a multiple of 16, a
+    # misaligned X: refused before any launch
+    assert qg.qg_linear_forward_int8(X.data_ptr(), ldx, dW.data_ptr(), ldw, dsW.data_ptr(), 17, m, n,
+                                     Y.data_ptr(), ldy, s) == qg.QG_ESHAPE
+    assert qg.qg_linear_forward_int8(X.data_ptr(), ldx, dW.data_ptr(), 136, dsW.data_ptr(), 4, m, n,
+                                     Y.data_ptr(), ldy, s) == qg.QG_ESHAPE
+    assert qg.qg_linear_forward_int8(X.data_ptr() + 2, ldx, dW.data_ptr(), ldw, dsW.data_ptr(), 4, m, n,
+                                     Y.data_ptr(), ldy, s) == qg.QG_EALIGN
+    # zero activations give zero outputs
+    qg.check(qg.qg_linear_forward_int8(X.data_ptr(), ldx, dW.data_ptr(), ldw, dsW.data_ptr(), 16, m, n,
+                                       Y.data_ptr(), ldy, s))
+    torch.cuda.synchronize()
+    assert (_read_bf16(Y, 16, m) == 0).all()
