@@ -130,7 +130,9 @@ __global__ void __launch_bounds__(256) dequant_weight_kernel(const int8_t* __res
 // (distinct w >> 1, two rows) and of the X tile (distinct w & 3, two tokens).
 // The work is bound by HBM at 2T <= 32 flops per weight byte; the tensor cores
 // keep the multiply-adds off the schedulers, which the conversion occupies
-// (about 2.75 instructions a weight).
+// (about 2.75 instructions a weight).  The kernel is launched with
+// programmatic stream serialization, so that its launch and set-up overlap the
+// end of the kernel before it in the stream.
 constexpr int kF8Warps = 4;                        // consumer warps, 16 rows each
 constexpr int kF8Rows = 16 * kF8Warps;             // rows of W per CTA
 constexpr int kF8Threads = 32 * (kF8Warps + 1);    // + the producer warp
@@ -187,24 +189,18 @@ QG_DEV uint64_t pack_f32x2(uint32_t lo, uint32_t hi) {
 
 // Four weights (the bytes of a word of codes, lowest first) as two bf16 pairs,
 // each bf16(fp32(q) * s) with its own scale (sc01: weights 0, 1; sc23: 2, 3).
-// The codes biased by 128 (q ^ 0x80 as unsigned bytes u) are placed two at a
-// time in the low mantissa bits of two fp16 halves of 1024 (0x6400 | u = the
-// fp16 1024 + u, exact); one mixed-precision addition per weight widens a half
-// to float32 and subtracts 1152, giving q exactly; the products with the
-// scales are packed f32x2 multiplies (round to nearest), then each pair is
-// rounded to bf16 (nearest even), the lower column in the low half.
+// The codes biased by 128 (q ^ 0x80 as unsigned bytes u) are placed in the low
+// mantissa bits of 2^23 (the float 2^23 + u, exact); less 2^23 + 128 they are q
+// exactly; the products with the scales round to nearest in float32; each pair
+// is then rounded to bf16 (nearest even), the lower column in the low half.
+// Packed f32x2 arithmetic, two weights per instruction.
 QG_DEV void w_tilde4(uint32_t word, uint64_t sc01, uint64_t sc23, uint32_t& p01, uint32_t& p23) {
   const uint32_t biased = word ^ 0x80808080u;
-  const uint32_t h01 = __byte_perm(biased, 0x64646464u, 0x5140u);
-  const uint32_t h23 = __byte_perm(biased, 0x64646464u, 0x7362u);
-  uint64_t v01, v23;
-  asm("{\n\t.reg .b16 a, b, c, d;\n\t.reg .f32 fa, fb, fc, fd;\n\t"
-      "mov.b32 {a, b}, %2;\n\tmov.b32 {c, d}, %3;\n\t"
-      "add.rn.f32.f16 fa, a, 0fC4900000;\n\tadd.rn.f32.f16 fb, b, 0fC4900000;\n\t"
-      "add.rn.f32.f16 fc, c, 0fC4900000;\n\tadd.rn.f32.f16 fd, d, 0fC4900000;\n\t"
-      "mov.b64 %0, {fa, fb};\n\tmov.b64 %1, {fc, fd};\n\t}"
-      : "=l"(v01), "=l"(v23)
-      : "r"(h01), "r"(h23));
+  uint64_t v01 = pack_f32x2(__byte_perm(biased, 0x4B000000u, 0x7540u), __byte_perm(biased, 0x4B000000u, 0x7541u));
+  uint64_t v23 = pack_f32x2(__byte_perm(biased, 0x4B000000u, 0x7542u), __byte_perm(biased, 0x4B000000u, 0x7543u));
+  const uint64_t offset = pack_f32x2(0x4B000080u, 0x4B000080u);  // 2^23 + 128
+  asm("sub.rn.f32x2 %0, %0, %1;" : "+l"(v01) : "l"(offset));
+  asm("sub.rn.f32x2 %0, %0, %1;" : "+l"(v23) : "l"(offset));
   asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(v01) : "l"(sc01));
   asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(v23) : "l"(sc23));
   uint32_t a, b, c, d;
@@ -295,6 +291,10 @@ __global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) linear_forward_int8_
     fence_barrier_init();
   }
   __syncthreads();
+  // launched with programmatic stream serialization: the set-up above may overlap
+  // the end of the preceding kernel, whose writes (X, W, the scales) are visible
+  // after this wait; every global access of this kernel comes after it
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == kF8Warps) {
     // producer: one thread streams the slice's stages (W tile, two X boxes) through the ring
@@ -409,6 +409,8 @@ __global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) linear_forward_int8_
       red[tok + 1][r0 + 8] = __fadd_rn(acc[0][nt][3], acc[1][nt][3]);
     }
   }
+  // the next kernel in the stream may launch now (its own wait orders it after this one)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   cluster_sync();  // every CTA's partial sums are written
   constexpr int kOut = kNT * 8 * kF8Rows;
   const int o0 = rank * kOut / S, o1 = (rank + 1) * kOut / S;
@@ -518,13 +520,15 @@ cudaError_t launch_forward_int8_as(const CUtensorMap& tmW, const uint16_t* X, in
   cfg.blockDim = dim3(kF8Threads);
   cfg.dynamicSmemBytes = static_cast<size_t>(f8_smem_bytes<kNT>());
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(f.S);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, linear_forward_int8_kernel<kNT, kGroupRows>, tmW, tmX, sW, T, m, n, f.slice, Y,
                             ldy);
 }
