@@ -112,18 +112,20 @@ __global__ void __launch_bounds__(256) dequant_weight_kernel(const int8_t* __res
 // so every output is the same sum whichever CTA adds it, rounded once to bf16.
 //
 // Data movement.  One producer thread streams the slice through a ring of
-// kF8Stages shared-memory stages by TMA, 128 columns a stage: the W tile (64
-// rows x 128 bytes) and the X tile (8 or 16 token rows x 128 columns, two
-// boxes of 64 columns), all with the 128-byte swizzle.  Rows past m or T and
-// columns past n arrive as zeros, and the bytes in flight cost no registers.
+// f8_stages shared-memory stages by TMA, 256 columns a stage; per 128 columns
+// the W box (64 rows x 128 bytes) and the X boxes (8 or 16 token rows x 64
+// columns, two), all with the 128-byte swizzle.  Rows past m or T and columns
+// past n arrive as zeros, and the bytes in flight cost no registers.  Wider
+// stages halve the consumers' per-stage work (waits, arrivals, addresses,
+// scales) per weight.
 //
 // Arithmetic.  Four consumer warps own 16 rows each.  The product runs on the
 // tensor cores with mma.sync m16n8k16 (bf16 in, f32 accumulate), whose A
 // operand comes from registers: the dequantized weight goes from the
 // conversion straight into the fragment.  Any bijection of a stage's columns
-// onto k-positions gives the same sum.  In step s (of two) the lane with
-// thread-in-group t takes the 16 columns of chunk w = 2t + (s ^ (t >> 1)) (16
-// columns, 16 bytes of W); in MMA j its k-pairs (2t, 2t+1) and (2t+8, 2t+9)
+// onto k-positions gives the same sum.  In step s (two per 128 columns) the
+// lane with thread-in-group t takes the 16 columns of chunk w = 2t + (s ^ (t >>
+// 1)) (16 columns, 16 bytes of W); in MMA j its k-pairs (2t, 2t+1) and (2t+8, 2t+9)
 // are columns 4j + {0, 1} and 4j + {2, 3} of those 16, and the B fragment of
 // token g is the eight bytes of X there.  With this order the eight lanes of a
 // quarter warp read eight distinct 16-byte bank groups of the swizzled W tile
@@ -136,9 +138,18 @@ __global__ void __launch_bounds__(256) dequant_weight_kernel(const int8_t* __res
 constexpr int kF8Warps = 4;                        // consumer warps, 16 rows each
 constexpr int kF8Rows = 16 * kF8Warps;             // rows of W per CTA
 constexpr int kF8Threads = 32 * (kF8Warps + 1);    // + the producer warp
-constexpr int kF8Tile = 128;                       // columns per ring stage
-constexpr int kF8WBytes = kF8Rows * kF8Tile;       // W tile: 8 KB
-constexpr int kF8Stages = 4;
+constexpr int kF8Tile = 128;                       // columns per TMA box of W (128 bytes)
+constexpr int kF8Halves = 2;                       // W boxes per ring stage
+constexpr int kF8StageCols = kF8Tile * kF8Halves;  // columns per ring stage
+constexpr int kF8WBytes = kF8Rows * kF8Tile;       // W box: 8 KB
+// ring depth: three stages of 256 columns (60 KB with the X boxes of up to 8
+// tokens, three CTAs a SM; 72 KB with those of 16, two CTAs a SM).  Two
+// stages for 16 tokens (four CTAs a SM) ran each matrix shape alone slightly
+// faster, but the mixed sequence of a decoder stack 9 % slower.
+template <int kNT>
+__host__ __device__ constexpr int f8_stages() {
+  return 3;
+}
 constexpr int kF8MaxCluster = 8;                   // portable cluster size
 
 // X tile of a stage: kNT * 8 token rows x 128 columns of bf16, two 64-column boxes
@@ -147,18 +158,25 @@ __host__ __device__ constexpr int f8_xbox_bytes() {
   return kNT * 8 * 128;
 }
 
+// a stage: per 128 columns, the W box and the two X boxes; a multiple of 1024
+// bytes (the swizzle atom), as is every box in it
+template <int kNT>
+__host__ __device__ constexpr int f8_half_bytes() {
+  return kF8WBytes + 2 * f8_xbox_bytes<kNT>();
+}
+
 template <int kNT>
 __host__ __device__ constexpr int f8_stage_bytes() {
-  return kF8WBytes + 2 * f8_xbox_bytes<kNT>();  // a multiple of 1024 (the swizzle atom)
+  return kF8Halves * f8_half_bytes<kNT>();
 }
 
 template <int kNT>
 __host__ __device__ constexpr int f8_smem_bytes() {
-  return 1024 + kF8Stages * f8_stage_bytes<kNT>();  // + alignment slack for the ring
+  return 1024 + f8_stages<kNT>() * f8_stage_bytes<kNT>();  // + alignment slack for the ring
 }
 
-// CTAs per SM (shared memory: four rings of 40 or 48 KB; registers)
-constexpr int kF8CtasPerSm = 4;
+// CTAs per SM for the register budget (at most 136 registers a thread)
+constexpr int kF8CtasPerSm = 3;
 
 QG_DEV float ld_shared_cluster_f32(uint32_t addr) {
   float v;
@@ -262,15 +280,16 @@ QG_DEV void f8_mma(const uint32_t (&wa)[8], const uint32_t (&wb)[8], const uint4
 }
 
 // Grid: one CTA per (row block, column slice), blockIdx.x = block * S + slice,
-// launched in clusters of S along x; slice is a multiple of kF8Tile (of 256
-// when kGroupRows: n % 256 == 0, so that a stage of a row lies in one scale
-// group).
+// launched in clusters of S along x; slice is a multiple of kF8StageCols (and
+// of 256 when kGroupRows: n % 256 == 0, so that a group of 256 columns of a row
+// lies in one scale group).
 template <int kNT, bool kGroupRows>
 __global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) linear_forward_int8_kernel(
     const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const float* __restrict__ sW,
     int32_t T, int32_t m, int32_t n, int32_t slice, uint16_t* __restrict__ Y, int64_t ldy) {
   constexpr int kStage = f8_stage_bytes<kNT>();
   constexpr int kXBox = f8_xbox_bytes<kNT>();
+  constexpr int kF8Stages = f8_stages<kNT>();
   extern __shared__ uint8_t f8_smem[];
   __shared__ float red[kNT * 8][kF8Rows];  // this CTA's partial sums, [token][row]
   __shared__ uint64_t full[kF8Stages], empty[kF8Stages];
@@ -281,7 +300,7 @@ __global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) linear_forward_int8_
   const int rank = static_cast<int>(cluster_ctarank());
   const int block = blockIdx.x / S;
   const int kbeg = rank * slice, kend = min(n, kbeg + slice);
-  const int nstage = (kend - kbeg + kF8Tile - 1) / kF8Tile;
+  const int nstage = (kend - kbeg + kF8StageCols - 1) / kF8StageCols;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kF8Stages; ++i) {
       mbar_init(&full[i], 1);
@@ -306,11 +325,15 @@ __global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) linear_forward_int8_
         const int slot = k % kF8Stages;
         if (k >= kF8Stages && !mbar_wait(&empty[slot], ((k / kF8Stages) - 1) & 1, &abort_flag, nullptr)) break;
         uint8_t* st = ring + slot * kStage;
-        const int col = kbeg + k * kF8Tile;
         mbar_arrive_expect_tx(&full[slot], kStage);
-        tma_load_2d(st, &tmW, &full[slot], col, block * kF8Rows);
-        tma_load_2d(st + kF8WBytes, &tmX, &full[slot], col, 0);
-        tma_load_2d(st + kF8WBytes + kXBox, &tmX, &full[slot], col + 64, 0);
+#pragma unroll
+        for (int h = 0; h < kF8Halves; ++h) {
+          uint8_t* sh = st + h * f8_half_bytes<kNT>();
+          const int col = kbeg + k * kF8StageCols + h * kF8Tile;
+          tma_load_2d(sh, &tmW, &full[slot], col, block * kF8Rows);
+          tma_load_2d(sh + kF8WBytes, &tmX, &full[slot], col, 0);
+          tma_load_2d(sh + kF8WBytes + kXBox, &tmX, &full[slot], col + 64, 0);
+        }
         issued = k + 1;
       }
       // every load issued has landed before the CTA can leave (bounded)
@@ -342,7 +365,8 @@ __global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) linear_forward_int8_
     for (int h = 0; h < 2; ++h)
 #pragma unroll
       for (int nt = 0; nt < kNT; ++nt) acc[h][nt][0] = acc[h][nt][1] = acc[h][nt][2] = acc[h][nt][3] = 0.f;
-    // kGroupRows: the scales of the current and the next pair of stages (one group per row each)
+    // kGroupRows: the scales of the current and the next group of 256 columns (one per row)
+    constexpr int kStagesPerGroup = 256 / kF8StageCols;
     float sa = 0.f, sb = 0.f, na = 0.f, nb = 0.f;
     if (kGroupRows) {
       na = __ldg(srow_a + (kbeg >> 8));
@@ -351,13 +375,13 @@ __global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) linear_forward_int8_
     // after a timed-out wait (abort) the loop does no more work
     bool ok = true;
     for (int k = 0; k < nstage && ok; ++k) {
-      const int col = kbeg + k * kF8Tile;
-      if (kGroupRows && (k & 1) == 0) {
+      const int col0 = kbeg + k * kF8StageCols;
+      if (kGroupRows && k % kStagesPerGroup == 0) {
         sa = na;
         sb = nb;
-        if (k + 2 < nstage) {
-          na = __ldg(srow_a + ((col + 256) >> 8));
-          nb = __ldg(srow_b + ((col + 256) >> 8));
+        if (k + kStagesPerGroup < nstage) {
+          na = __ldg(srow_a + ((col0 + 256) >> 8));
+          nb = __ldg(srow_b + ((col0 + 256) >> 8));
         }
       }
       const int slot = k % kF8Stages;
@@ -365,38 +389,45 @@ __global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) linear_forward_int8_
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[slot], (k / kF8Stages) & 1, &abort_flag, nullptr));
       if (!ok) break;
       const uint8_t* st = ring + slot * kStage;
-      uint4 qa[2], qb[2], x0[2][kNT], x1[2][kNT];
 #pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        qa[s] = *reinterpret_cast<const uint4*>(st + woff[s]);
-        qb[s] = *reinterpret_cast<const uint4*>(st + woff[s] + 8 * kF8Tile);
+      for (int h = 0; h < kF8Halves; ++h) {
+        const uint8_t* sh = st + h * f8_half_bytes<kNT>();
+        const int col = col0 + h * kF8Tile;
+        uint4 qa[2], qb[2], x0[2][kNT], x1[2][kNT];
 #pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) {
-          x0[s][nt] = *reinterpret_cast<const uint4*>(st + xoff0[s] + nt * 8 * 128);
-          x1[s][nt] = *reinterpret_cast<const uint4*>(st + xoff1[s] + nt * 8 * 128);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);  // the stage is in registers
+        for (int s = 0; s < 2; ++s) {
+          qa[s] = *reinterpret_cast<const uint4*>(sh + woff[s]);
+          qb[s] = *reinterpret_cast<const uint4*>(sh + woff[s] + 8 * kF8Tile);
 #pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        uint32_t wa[8], wb[8];
-        if constexpr (kGroupRows) {
-          w_tilde16<true>(qa[s], 0.f, sa, 0, wa);
-          w_tilde16<true>(qb[s], 0.f, sb, 0, wb);
-        } else {
-          const int j0 = col + wcol[s];
-          const Scales16 za = scales16(ia, j0, n, sW), zb = scales16(ib, j0, n, sW);
-          // a warp vote: every lane takes the same path to the MMAs
-          if (__all_sync(0xFFFFFFFFu, za.split <= 0 && zb.split <= 0)) {
-            w_tilde16<true>(qa[s], 0.f, za.s1, 0, wa);
-            w_tilde16<true>(qb[s], 0.f, zb.s1, 0, wb);
-          } else {
-            w_tilde16<false>(qa[s], za.s0, za.s1, za.split, wa);
-            w_tilde16<false>(qb[s], zb.s0, zb.s1, zb.split, wb);
+          for (int nt = 0; nt < kNT; ++nt) {
+            x0[s][nt] = *reinterpret_cast<const uint4*>(sh + xoff0[s] + nt * 8 * 128);
+            x1[s][nt] = *reinterpret_cast<const uint4*>(sh + xoff1[s] + nt * 8 * 128);
           }
         }
-        f8_mma<kNT>(wa, wb, x0[s], x1[s], acc);
+        if (h == kF8Halves - 1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[slot]);  // the stage is in registers
+        }
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          uint32_t wa[8], wb[8];
+          if constexpr (kGroupRows) {
+            w_tilde16<true>(qa[s], 0.f, sa, 0, wa);
+            w_tilde16<true>(qb[s], 0.f, sb, 0, wb);
+          } else {
+            const int j0 = col + wcol[s];
+            const Scales16 za = scales16(ia, j0, n, sW), zb = scales16(ib, j0, n, sW);
+            // a warp vote: every lane takes the same path to the MMAs
+            if (__all_sync(0xFFFFFFFFu, za.split <= 0 && zb.split <= 0)) {
+              w_tilde16<true>(qa[s], 0.f, za.s1, 0, wa);
+              w_tilde16<true>(qb[s], 0.f, zb.s1, 0, wb);
+            } else {
+              w_tilde16<false>(qa[s], za.s0, za.s1, za.split, wa);
+              w_tilde16<false>(qb[s], zb.s0, zb.s1, zb.split, wb);
+            }
+          }
+          f8_mma<kNT>(wa, wb, x0[s], x1[s], acc);
+        }
       }
     }
     // partial sums: lane (g, t) holds rows r0 and r0 + 8, tokens 2t, 2t + 1 of each 8
@@ -434,8 +465,8 @@ __global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) linear_forward_int8_
 
 // Column slices per row block: as many as keep all clusters resident at once
 // (the occupancy query, for each cluster size from the largest down), at most
-// a portable cluster, each a multiple of kF8Tile columns (of 256 when
-// n % 256 == 0).
+// a portable cluster, each a multiple of kF8StageCols columns (and of 256
+// when n % 256 == 0).
 struct F8Split {
   int S, slice, blocks;
 };
@@ -443,7 +474,7 @@ struct F8Split {
 F8Split forward_int8_split(int32_t m, int32_t n, const int (&clusters_fit)[kF8MaxCluster + 1]) {
   F8Split f;
   f.blocks = (m + kF8Rows - 1) / kF8Rows;
-  const int unit = n % 256 == 0 ? 256 : kF8Tile;
+  const int unit = std::max(n % 256 == 0 ? 256 : kF8Tile, kF8StageCols);
   int S = std::max(1, std::min(kF8MaxCluster, (n + unit - 1) / unit));
   while (S > 1 && f.blocks > clusters_fit[S]) --S;
   f.slice = ((n + S - 1) / S + unit - 1) / unit * unit;
