@@ -88,26 +88,29 @@ def stack_shapes(layers, hidden=4096, inter=11008):
 
 KERNEL_SOURCES = ["qg_step.cu", "qg_gemm.cuh", "qg_device.cuh", "qg_philox.cuh", "qg_exact.cuh"]
 PROFILE = os.path.join(ROOT, "profiles", "step_kernels_llama7b_layer_ncu.md")
+FUSED_SOURCES = ["qg_linear.cu", "qg_device.cuh"]
+FUSED_PROFILE = os.path.join(ROOT, "profiles", "linear_forward_int8_llama7b_decode_ncu.md")
 
 
-def kernel_digest():
+def kernel_digest(sources=KERNEL_SOURCES):
     import hashlib
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in sources:
         with open(os.path.join(ROOT, "quantized_rank_gradient_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel, alg_bytes_per_launch):
+def profiled_traffic(kernel, alg_bytes_per_launch, profile=PROFILE, sources=KERNEL_SOURCES):
     """DRAM bytes per launch of `kernel`: the ratio of measured DRAM traffic to
     algorithmic bytes in the committed ncu capture, times this run's
-    algorithmic bytes per launch.  The ratio is taken from one launch of
-    the same kernel, the 7-matrix batch of one decoder layer. Traffic grows in
-    proportion to the matrices in a launch. None when the kernel sources
-    changed since that capture."""
+    algorithmic bytes per launch.  For the step kernels the ratio is taken
+    from one launch of the same kernel, the 7-matrix batch of one decoder
+    layer; for the fused INT8 forward, from the four launches of one decoder
+    layer.  Traffic grows in proportion to the bytes a launch reads.  None when
+    the kernel sources changed since that capture."""
     try:
-        text = open(PROFILE).read()
+        text = open(profile).read()
     except OSError:
         return None
     digest = ratio = None
@@ -116,7 +119,7 @@ def profiled_traffic(kernel, alg_bytes_per_launch):
             digest = line.split(":", 1)[1].strip()
         if line.startswith("traffic_over_algorithmic:"):
             ratio = dict(kv.split("=") for kv in line.split(":", 1)[1].split())
-    if digest != kernel_digest() or not ratio or kernel not in ratio:
+    if digest != kernel_digest(sources) or not ratio or kernel not in ratio:
         return None
     return float(ratio[kernel]) * alg_bytes_per_launch
 
@@ -850,7 +853,11 @@ def run_linear_decode(args, rank, world, local_rank):
                    "parallelism": f"independent stacks x{world}"},
         "roofline": {"bound": "hbm", "kernel": "linear_forward_int8", "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": None, "peak_kind": "HBM copy (%s)" % peaks["source"]},
+                     "traffic": profiled_traffic("linear_forward_int8", k.bytes / k.launches, FUSED_PROFILE,
+                                                 FUSED_SOURCES),
+                     "traffic_unit": "DRAM bytes per launch (ncu traffic/algorithmic ratio x this launch)",
+                     "algorithmic_bytes_per_launch": k.bytes / k.launches,
+                     "peak_kind": "HBM copy (%s)" % peaks["source"]},
         "kernels": {"linear_forward_int8": {"launches_per_step": len(bufs),
                                             "device_ms_per_launch": k.device_ms / k.launches, "gbs": achieved}},
         "tokens_sweep": sweep,
