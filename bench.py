@@ -218,6 +218,25 @@ def cpu_baseline(cols=2048):
             "host_cpus": os.cpu_count()}
 
 
+def cpu_baseline_forward(T, m=4096, n=4096, reps=3, seed=1):
+    """The oracle's forward for a few tokens, W~ = bf16(q s) then Y = X W~^T in
+    float64, on one 4096 x 4096 matrix, `reps` times (INT8 weights per second)."""
+    import numpy as np
+
+    import oracle as O
+    import synth
+    Wq = synth.weight_codes(m, n, seed)
+    sW = synth.weight_scales(m, n, seed=seed)
+    X = O.bf16_round(np.random.default_rng(seed).standard_normal((T, n)).astype(np.float32))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        O.linear_forward(X, O.dequant_weight_bf16(Wq, sW))
+    t = time.perf_counter() - t0
+    return {"value": reps * m * n / t, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{reps} oracle forwards (dequantize, then a float64 product) of one {m}x{n} INT8 matrix "
+                      f"at T = {T} ({t:.1f} s)", "host_cpus": os.cpu_count()}
+
+
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
@@ -864,6 +883,8 @@ def run_linear_decode(args, rank, world, local_rank):
         "gpu_launches": len(bufs) * args.steps,
         "clocks": clk,
     }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline_forward(T)
     print(json.dumps(line), flush=True)
     return 0
 
