@@ -58,7 +58,7 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=None, help="decoder layers (default: the stack's own count)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--tokens", type=int, default=16, help="linear-7b-decode: tokens of the headline line (1..16)")
+    ap.add_argument("--tokens", type=int, default=16, help="linear-7b-decode: tokens of the headline line (1..64)")
     ap.add_argument("--workload", choices=sorted(STACKS) + ["refresh-stress", "linear-grad-stress", "linear-7b",
                                                             "linear-7b-decode"],
                     default="llama7b-stack",
@@ -735,12 +735,12 @@ def run_linear(args, rank, world, local_rank):
     return 0
 
 
-DECODE_TOKENS = (1, 4, 8, 16)
+DECODE_TOKENS = (1, 4, 8, 16, 32, 64)
 
 
 def run_linear_decode(args, rank, world, local_rank):
     """The forward product Y = X W~^T of the LLaMA-7B stack's INT8 weights for a
-    few tokens (--tokens, default 16; the line also sweeps T = 1, 4, 8, 16).
+    few tokens (--tokens, default 16; the line also sweeps T = 1 to 64).
 
     The weights are laid out as decoders run them for inference: per layer the
     q, k and v weights stacked in one 12288 x 4096 buffer and gate and up in one
@@ -764,8 +764,8 @@ def run_linear_decode(args, rank, world, local_rank):
     torch.cuda.set_device(device)
     spec = STACKS["llama7b-stack"]
     layers = args.layers or spec["layers"]
-    if not 1 <= args.tokens <= 16:
-        raise SystemExit("--tokens must be in 1..16")
+    if not 1 <= args.tokens <= 64:
+        raise SystemExit("--tokens must be in 1..64")
     stream = c_void_p(torch.cuda.current_stream().cuda_stream)
     h, f = spec["hidden"], spec["inter"]
     # per layer: (rows of each stacked matrix, n)
@@ -787,8 +787,8 @@ def run_linear_decode(args, rank, world, local_rank):
     gen.manual_seed(5_000_011 * (rank + 1))
     bf = torch.bfloat16
     shapes = sorted({(m, n) for (m, n, *_r) in bufs} | {(m, n) for (m, n, *_r) in mats})
-    io = {(m, n): dict(X=torch.randn(16, n, generator=gen, device=device).to(bf),
-                       Y=torch.empty(16, m, dtype=bf, device=device),
+    io = {(m, n): dict(X=torch.randn(64, n, generator=gen, device=device).to(bf),
+                       Y=torch.empty(64, m, dtype=bf, device=device),
                        Wt=torch.empty(m, -(-n // 8) * 8, dtype=bf, device=device))
           for (m, n) in shapes}
 

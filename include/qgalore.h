@@ -371,14 +371,18 @@ qg_status qg_linear_forward(const void* d_X, int64_t ldx, const void* d_Wt, int6
 /* The forward product for a few tokens straight from the INT8 weight:
  * Y = X W~^T with W~ = bf16(fp32(q_ij) * s_W[(i n + j) / 256]) formed in
  * registers, never stored (the same limitation passage of the AIMech Q-GaLore
- * page: the dequantization fused into the product).  For 1 <= T <= 16 tokens
+ * page: the dequantization fused into the product).  For 1 <= T <= 64 tokens
  * the product is bound by reading the weight: this reads its INT8 codes once,
  * where qg_linear_dequant_weight and qg_linear_forward move five bytes per
  * weight.  X: T x n bf16 (ldx, 16-byte aligned); W: m x ldw INT8 and its group
  * scales as qg_layer_init takes them; Y: T x m bf16 (ldy).  float32
  * accumulation in another order than qg_linear_forward's, each output rounded
- * once to bf16.  T > 16 gives QG_ESHAPE (use the dequantization and the
- * tcgen05 product there); T = 0 is a no-op.  Other errors as above. */
+ * once to bf16; two calls give the same bits.  The kernel is launched with
+ * programmatic stream serialization: its set-up may overlap the end of the
+ * preceding kernel in the stream, and every read of X, W and the scales comes
+ * after that kernel has finished.  T > 64 gives QG_ESHAPE (use the
+ * dequantization and the tcgen05 product there); T = 0 is a no-op.  Other
+ * errors as above. */
 qg_status qg_linear_forward_int8(const void* d_X, int64_t ldx, const int8_t* d_W, int64_t ldw, const float* d_sW,
                                  int32_t T, int32_t m, int32_t n, void* d_Y, int64_t ldy, void* stream);
 qg_status qg_linear_backward_data(const void* d_dY, int64_t lddy, const void* d_Wt, int64_t ldwt, int32_t T,

@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(256) dequant_weight_kernel(const int8_t* __res
 
 // ---------------------------------------------------------------- Y = X W~^T for a few tokens, W read once
 
-// For T <= 16 tokens the forward product is bound by reading the weight: the
+// For T <= 64 tokens the forward product is bound by reading the weight: the
 // separate dequantization moves three bytes per weight and the GEMM two more,
 // where this kernel reads the INT8 codes once and forms W~ = bf16(fp32(q) * s)
 // in registers, rounded exactly as dequant_weight_kernel rounds it.
@@ -113,8 +113,8 @@ __global__ void __launch_bounds__(256) dequant_weight_kernel(const int8_t* __res
 //
 // Data movement.  One producer thread streams the slice through a ring of
 // f8_stages shared-memory stages by TMA, 256 columns a stage; per 128 columns
-// the W box (64 rows x 128 bytes) and the X boxes (8 or 16 token rows x 64
-// columns, two), all with the 128-byte swizzle.  Rows past m or T and columns
+// the W box (64 rows x 128 bytes) and the X boxes (8, 16, 32 or 64 token rows
+// x 64 columns, two), all with the 128-byte swizzle.  Rows past m or T and columns
 // past n arrive as zeros, and the bytes in flight cost no registers.  Wider
 // stages halve the consumers' per-stage work (waits, arrivals, addresses,
 // scales) per weight.
@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(256) dequant_weight_kernel(const int8_t* __res
 // token g is the eight bytes of X there.  With this order the eight lanes of a
 // quarter warp read eight distinct 16-byte bank groups of the swizzled W tile
 // (distinct w >> 1, two rows) and of the X tile (distinct w & 3, two tokens).
-// The work is bound by HBM at 2T <= 32 flops per weight byte; the tensor cores
+// At 2T <= 128 flops per weight byte the work is bound by HBM; the tensor cores
 // keep the multiply-adds off the schedulers, which the conversion occupies
 // (about 2.75 instructions a weight).  The kernel is launched with
 // programmatic stream serialization, so that its launch and set-up overlap the
@@ -142,13 +142,14 @@ constexpr int kF8Tile = 128;                       // columns per TMA box of W (
 constexpr int kF8Halves = 2;                       // W boxes per ring stage
 constexpr int kF8StageCols = kF8Tile * kF8Halves;  // columns per ring stage
 constexpr int kF8WBytes = kF8Rows * kF8Tile;       // W box: 8 KB
-// ring depth: three stages of 256 columns (60 KB with the X boxes of up to 8
-// tokens, three CTAs a SM; 72 KB with those of 16, two CTAs a SM).  Two
-// stages for 16 tokens (four CTAs a SM) ran each matrix shape alone slightly
-// faster, but the mixed sequence of a decoder stack 9 % slower.
+// ring depth in stages of 256 columns: three up to 32 tokens (60, 72 and 96 KB
+// with the X boxes of 8, 16 and 32 tokens: three, two and two CTAs a SM), two
+// for 64 tokens (96 KB).  Two stages for 16 tokens (four CTAs a SM) ran each
+// matrix shape alone slightly faster, but the mixed sequence of a decoder
+// stack 9 % slower.
 template <int kNT>
 __host__ __device__ constexpr int f8_stages() {
-  return 3;
+  return kNT >= 8 ? 2 : 3;
 }
 constexpr int kF8MaxCluster = 8;                   // portable cluster size
 
@@ -175,8 +176,12 @@ __host__ __device__ constexpr int f8_smem_bytes() {
   return 1024 + f8_stages<kNT>() * f8_stage_bytes<kNT>();  // + alignment slack for the ring
 }
 
-// CTAs per SM for the register budget (at most 136 registers a thread)
-constexpr int kF8CtasPerSm = 3;
+// CTAs per SM for the register budget: at most 136 registers a thread up to 16
+// tokens, 204 beyond (the accumulators grow with the tokens)
+template <int kNT>
+__host__ __device__ constexpr int f8_ctas_per_sm() {
+  return kNT <= 2 ? 3 : 2;
+}
 
 QG_DEV float ld_shared_cluster_f32(uint32_t addr) {
   float v;
@@ -284,7 +289,7 @@ QG_DEV void f8_mma(const uint32_t (&wa)[8], const uint32_t (&wb)[8], const uint4
 // of 256 when kGroupRows: n % 256 == 0, so that a group of 256 columns of a row
 // lies in one scale group).
 template <int kNT, bool kGroupRows>
-__global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) linear_forward_int8_kernel(
+__global__ void __launch_bounds__(kF8Threads, f8_ctas_per_sm<kNT>()) linear_forward_int8_kernel(
     const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const float* __restrict__ sW,
     int32_t T, int32_t m, int32_t n, int32_t slice, uint16_t* __restrict__ Y, int64_t ldy) {
   constexpr int kStage = f8_stage_bytes<kNT>();
@@ -393,18 +398,24 @@ __global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) linear_forward_int8_
       for (int h = 0; h < kF8Halves; ++h) {
         const uint8_t* sh = st + h * f8_half_bytes<kNT>();
         const int col = col0 + h * kF8Tile;
-        uint4 qa[2], qb[2], x0[2][kNT], x1[2][kNT];
+        // W (and, up to 16 tokens, X) of this half in registers; with more tokens X is
+        // read per step, and the stage is released after its last half
+        constexpr bool kPrefetchX = kNT <= 2;
+        constexpr int kXN = kPrefetchX ? kNT : 1;
+        uint4 qa[2], qb[2], x0[2][kXN], x1[2][kXN];
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
           qa[s] = *reinterpret_cast<const uint4*>(sh + woff[s]);
           qb[s] = *reinterpret_cast<const uint4*>(sh + woff[s] + 8 * kF8Tile);
+          if constexpr (kPrefetchX) {
 #pragma unroll
-          for (int nt = 0; nt < kNT; ++nt) {
-            x0[s][nt] = *reinterpret_cast<const uint4*>(sh + xoff0[s] + nt * 8 * 128);
-            x1[s][nt] = *reinterpret_cast<const uint4*>(sh + xoff1[s] + nt * 8 * 128);
+            for (int nt = 0; nt < kNT; ++nt) {
+              x0[s][nt] = *reinterpret_cast<const uint4*>(sh + xoff0[s] + nt * 8 * 128);
+              x1[s][nt] = *reinterpret_cast<const uint4*>(sh + xoff1[s] + nt * 8 * 128);
+            }
           }
         }
-        if (h == kF8Halves - 1) {
+        if (kPrefetchX && h == kF8Halves - 1) {
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[slot]);  // the stage is in registers
         }
@@ -426,7 +437,23 @@ __global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) linear_forward_int8_
               w_tilde16<false>(qb[s], zb.s0, zb.s1, zb.split, wb);
             }
           }
-          f8_mma<kNT>(wa, wb, x0[s], x1[s], acc);
+          if constexpr (kPrefetchX) {
+            f8_mma<kNT>(wa, wb, x0[s], x1[s], acc);
+          } else {
+#pragma unroll
+            for (int nt = 0; nt < kNT; ++nt) {
+              const uint4 y0 = *reinterpret_cast<const uint4*>(sh + xoff0[s] + nt * 8 * 128);
+              const uint4 y1 = *reinterpret_cast<const uint4*>(sh + xoff1[s] + nt * 8 * 128);
+              mma_bf16_16816(acc[0][nt], wa[0], wb[0], wa[1], wb[1], y0.x, y0.y);
+              mma_bf16_16816(acc[0][nt], wa[2], wb[2], wa[3], wb[3], y0.z, y0.w);
+              mma_bf16_16816(acc[1][nt], wa[4], wb[4], wa[5], wb[5], y1.x, y1.y);
+              mma_bf16_16816(acc[1][nt], wa[6], wb[6], wa[7], wb[7], y1.z, y1.w);
+            }
+          }
+        }
+        if (!kPrefetchX && h == kF8Halves - 1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[slot]);  // every read of the stage is done
         }
       }
     }
@@ -577,9 +604,15 @@ cudaError_t launch_forward_int8(const uint16_t* X, int64_t ldx, const int8_t* W,
   if (T <= 8)
     e = rows ? launch_forward_int8_as<1, true>(tmW, X, ldx, sW, T, m, n, Y, ldy, s)
              : launch_forward_int8_as<1, false>(tmW, X, ldx, sW, T, m, n, Y, ldy, s);
-  else
+  else if (T <= 16)
     e = rows ? launch_forward_int8_as<2, true>(tmW, X, ldx, sW, T, m, n, Y, ldy, s)
              : launch_forward_int8_as<2, false>(tmW, X, ldx, sW, T, m, n, Y, ldy, s);
+  else if (T <= 32)
+    e = rows ? launch_forward_int8_as<4, true>(tmW, X, ldx, sW, T, m, n, Y, ldy, s)
+             : launch_forward_int8_as<4, false>(tmW, X, ldx, sW, T, m, n, Y, ldy, s);
+  else
+    e = rows ? launch_forward_int8_as<8, true>(tmW, X, ldx, sW, T, m, n, Y, ldy, s)
+             : launch_forward_int8_as<8, false>(tmW, X, ldx, sW, T, m, n, Y, ldy, s);
   profile_end(s, tok);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -738,7 +771,7 @@ qg_status qg_linear_forward(const void* d_X, int64_t ldx, const void* d_Wt, int6
 
 qg_status qg_linear_forward_int8(const void* d_X, int64_t ldx, const int8_t* d_W, int64_t ldw, const float* d_sW,
                                  int32_t T, int32_t m, int32_t n, void* d_Y, int64_t ldy, void* stream) {
-  if (T < 0 || T > 16 || m <= 0 || n <= 0) return QG_ESHAPE;
+  if (T < 0 || T > 64 || m <= 0 || n <= 0) return QG_ESHAPE;
   if (!d_W || !d_sW) return QG_EINVAL;
   if (ldw < n || ldw % 16 != 0) return QG_ESHAPE;
   if (!aligned16(d_W)) return QG_EALIGN;

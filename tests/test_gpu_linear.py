@@ -239,7 +239,7 @@ def _forward_int8(dXa, ldx, dW, ldw, dsW, T, m, n, ld_extra=8):
 FUSED_SHAPES = [(37, 64, 64), (300, 700, 720), (640, 1365, 1376), (129, 4096, 4096), (20000, 2600, 2608)]
 
 
-@pytest.mark.parametrize("T", [1, 3, 8, 9, 16])
+@pytest.mark.parametrize("T", [1, 3, 8, 9, 16, 17, 32, 33, 64])
 @pytest.mark.parametrize("m,n,ldw", FUSED_SHAPES)
 def test_forward_int8_parity(T, m, n, ldw):
     Wq, sW, dW, dsW = _weights_junk_pad(m, n, seed=7 * T + m, ldw=ldw)
@@ -255,7 +255,7 @@ def test_forward_int8_parity(T, m, n, ldw):
 
 
 @pytest.mark.parametrize("m,n", [(4096, 11008), (11008, 4096)])
-@pytest.mark.parametrize("T", [1, 16])
+@pytest.mark.parametrize("T", [1, 16, 64])
 def test_forward_int8_full_size(T, m, n):
     # the 7B stack's MLP shapes at decode sizes, every output against the oracle
     Wq, sW, dW, ldw, dsW = _weights(m, n, seed=m + T)
@@ -267,14 +267,15 @@ def test_forward_int8_full_size(T, m, n):
     _within_bar(_read_bf16(Y, T, m), X, Wt.T, O.linear_forward(X, Wt))
 
 
-def test_forward_int8_bit_exact_on_small_integers():
+@pytest.mark.parametrize("T", [16, 64])
+def test_forward_int8_bit_exact_on_small_integers(T):
     # codes in {-1, 0, 1} (one in 32 nonzero), power-of-two scales and X in
     # {-1, 0, 1}: every partial sum, the sum over the cluster's slices and the
     # result are integers times 2^-3 of magnitude < 256 * 2^-3, exact in
     # float32 and in bf16, so the split-K reduction and the operand layouts are
     # checked bit for bit
-    rng = np.random.default_rng(33)
-    T, m, n = 16, 300, 4000
+    rng = np.random.default_rng(33 + T)
+    m, n = 300, 4000
     Wq = (rng.integers(-1, 2, size=(m, n)) * (rng.integers(0, 32, size=(m, n)) == 0)).astype(np.int8)
     sW = np.full(-(-(m * n) // 256), 0.125, np.float32)
     X = rng.integers(-1, 2, size=(T, n)).astype(np.float32)
@@ -312,24 +313,24 @@ def test_forward_int8_deterministic_and_agrees_with_two_step_path():
 def test_forward_int8_edges():
     m, n = 64, 128
     Wq, sW, dW, ldw, dsW = _weights(m, n, seed=1)
-    X, ldx = _bf16_dev(np.zeros((17, n), np.uint16))
-    Y, ldy = _empty_bf16(17, m)
+    X, ldx = _bf16_dev(np.zeros((65, n), np.uint16))
+    Y, ldy = _empty_bf16(65, m)
     s = stream()
     # T = 0: nothing written
     qg.check(qg.qg_linear_forward_int8(X.data_ptr(), ldx, dW.data_ptr(), ldw, dsW.data_ptr(), 0, m, n, Y.data_ptr(),
                                        ldy, s))
     torch.cuda.synchronize()
     assert (Y.cpu().numpy().view(np.uint16) == 0x7FC0).all()
-    # more than 16 tokens, a weight stride that is not a multiple of 16, a
+    # more than 64 tokens, a weight stride that is not a multiple of 16, a
     # misaligned X: refused before any launch
-    assert qg.qg_linear_forward_int8(X.data_ptr(), ldx, dW.data_ptr(), ldw, dsW.data_ptr(), 17, m, n,
+    assert qg.qg_linear_forward_int8(X.data_ptr(), ldx, dW.data_ptr(), ldw, dsW.data_ptr(), 65, m, n,
                                      Y.data_ptr(), ldy, s) == qg.QG_ESHAPE
     assert qg.qg_linear_forward_int8(X.data_ptr(), ldx, dW.data_ptr(), 136, dsW.data_ptr(), 4, m, n,
                                      Y.data_ptr(), ldy, s) == qg.QG_ESHAPE
     assert qg.qg_linear_forward_int8(X.data_ptr() + 2, ldx, dW.data_ptr(), ldw, dsW.data_ptr(), 4, m, n,
                                      Y.data_ptr(), ldy, s) == qg.QG_EALIGN
     # zero activations give zero outputs
-    qg.check(qg.qg_linear_forward_int8(X.data_ptr(), ldx, dW.data_ptr(), ldw, dsW.data_ptr(), 16, m, n,
+    qg.check(qg.qg_linear_forward_int8(X.data_ptr(), ldx, dW.data_ptr(), ldw, dsW.data_ptr(), 64, m, n,
                                        Y.data_ptr(), ldy, s))
     torch.cuda.synchronize()
-    assert (_read_bf16(Y, 16, m) == 0).all()
+    assert (_read_bf16(Y, 64, m) == 0).all()
