@@ -183,6 +183,9 @@ __host__ __device__ constexpr int f8_ctas_per_sm() {
   return kNT <= 2 ? 3 : 2;
 }
 
+// barrier among the consumer warps only
+QG_DEV void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kF8Warps) : "memory"); }
+
 QG_DEV float ld_shared_cluster_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
@@ -296,10 +299,13 @@ __global__ void __launch_bounds__(kF8Threads, f8_ctas_per_sm<kNT>()) linear_forw
   constexpr int kXBox = f8_xbox_bytes<kNT>();
   constexpr int kF8Stages = f8_stages<kNT>();
   extern __shared__ uint8_t f8_smem[];
-  __shared__ float red[kNT * 8][kF8Rows];  // this CTA's partial sums, [token][row]
   __shared__ uint64_t full[kF8Stages], empty[kF8Stages];
   __shared__ int abort_flag;
   uint8_t* ring = f8_smem + ((1024 - (smem_u32(f8_smem) & 1023)) & 1023);
+  // this CTA's partial sums, [token][row], in the ring once every stage is read
+  // (the same offset in every CTA of the cluster)
+  float (*red)[kF8Rows] = reinterpret_cast<float (*)[kF8Rows]>(ring);
+  static_assert(kNT * 8 * kF8Rows * 4 <= kF8Stages * kStage, "partial sums fit in the ring");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = static_cast<int>(cluster_nctarank());
   const int rank = static_cast<int>(cluster_ctarank());
@@ -457,7 +463,10 @@ __global__ void __launch_bounds__(kF8Threads, f8_ctas_per_sm<kNT>()) linear_forw
         }
       }
     }
-    // partial sums: lane (g, t) holds rows r0 and r0 + 8, tokens 2t, 2t + 1 of each 8
+    // partial sums: lane (g, t) holds rows r0 and r0 + 8, tokens 2t, 2t + 1 of each 8;
+    // they overwrite the ring once every consumer warp has read its last stage (all
+    // the producer's loads have landed by then: each was waited for)
+    consumers_sync();
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) {
       const int tok = nt * 8 + 2 * t;

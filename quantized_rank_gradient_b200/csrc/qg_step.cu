@@ -739,16 +739,28 @@ struct DequantBatch {
 };
 
 QG_DEV uint4 dequant_word(uint32_t w, float s) {
-  // nibble x ^ 8 is code + 8 in [1, 15]; 0x4B400000 | (code + 8) is the float
-  // 1.5 * 2^23 + code + 8, exact
+  // nibble x ^ 8 is code + 8 in [0, 15]; the even and the odd nibbles are
+  // spread one to a byte, and each byte placed below the bits of 1.5 * 2^23
+  // (0x4B4000vv) is the float 1.5 * 2^23 + code + 8, exact; less that offset it
+  // is the code, times the group's scale (round to nearest), two weights per
+  // packed f32x2 instruction, then rounded to bf16 in pairs
   const uint32_t f = w ^ 0x88888888u;
+  const uint32_t ev = f & 0x0F0F0F0Fu, od = (f >> 4) & 0x0F0F0F0Fu;  // elements 2h and 2h + 1 in byte h
+  uint64_t sc;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(sc) : "f"(s));
+  uint64_t off;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(off) : "r"(0x4B400008u));  // 1.5 * 2^23 + 8
   uint32_t out[4];
 #pragma unroll
   for (int h = 0; h < 4; ++h) {
-    const float lo = __fsub_rn(__uint_as_float(0x4B400000u | ((f >> (8 * h)) & 0xFu)), 12582920.0f);
-    const float hi = __fsub_rn(__uint_as_float(0x4B400000u | ((f >> (8 * h + 4)) & 0xFu)), 12582920.0f);
-    const __nv_bfloat162 pr = __floats2bfloat162_rn(__fmul_rn(lo, s), __fmul_rn(hi, s));
-    out[h] = *reinterpret_cast<const uint32_t*>(&pr);
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "r"(__byte_perm(ev, 0x4B400000u, 0x7640u | h)),
+        "r"(__byte_perm(od, 0x4B400000u, 0x7640u | h)));
+    asm("sub.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(off));
+    asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(sc));
+    uint32_t lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out[h]) : "r"(hi), "r"(lo));  // element 2h in the low half
   }
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
