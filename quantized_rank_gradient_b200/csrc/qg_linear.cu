@@ -143,10 +143,10 @@ constexpr int kF8Halves = 2;                       // W boxes per ring stage
 constexpr int kF8StageCols = kF8Tile * kF8Halves;  // columns per ring stage
 constexpr int kF8WBytes = kF8Rows * kF8Tile;       // W box: 8 KB
 // ring depth in stages of 256 columns: three up to 32 tokens (60, 72 and 96 KB
-// with the X boxes of 8, 16 and 32 tokens: three, two and two CTAs a SM), two
-// for 64 tokens (96 KB).  Two stages for 16 tokens (four CTAs a SM) ran each
-// matrix shape alone slightly faster, but the mixed sequence of a decoder
-// stack 9 % slower.
+// with the X boxes of 8, 16 and 32 tokens: three, three and two CTAs a SM), two
+// for 64 tokens (96 KB, two CTAs a SM).  Two stages for 16 tokens (four CTAs a
+// SM) ran each matrix shape alone slightly faster, but the mixed sequence of a
+// decoder stack 9 % slower.
 template <int kNT>
 __host__ __device__ constexpr int f8_stages() {
   return kNT >= 8 ? 2 : 3;
