@@ -93,6 +93,29 @@ def test_entry_points_reject_bad_arguments_without_launching():
     assert qg.qg_philox4x32_10(0, 0, 0, 0, 10, 0, 0, 0, None) == qg.QG_EINVAL
 
 
+def test_fused_forward_rejects_bad_arguments_without_launching():
+    f = qg.qg_linear_forward_int8
+    X, W, sW, Y = 0x10000, 0x20000, 0x30000, 0x40000
+    # (X, ldx, W, ldw, sW, T, m, n, Y, ldy): T in 0..64, m and n positive
+    assert f(X, 128, W, 128, sW, 65, 64, 128, Y, 64, None) == qg.QG_ESHAPE
+    assert f(X, 128, W, 128, sW, -1, 64, 128, Y, 64, None) == qg.QG_ESHAPE
+    assert f(X, 128, W, 128, sW, 4, 0, 128, Y, 64, None) == qg.QG_ESHAPE
+    assert f(X, 128, W, 128, sW, 4, 64, 0, Y, 64, None) == qg.QG_ESHAPE
+    # W and its scales are required; its stride is a multiple of 16 bytes, at least n
+    assert f(X, 128, 0, 128, sW, 4, 64, 128, Y, 64, None) == qg.QG_EINVAL
+    assert f(X, 128, W, 128, 0, 4, 64, 128, Y, 64, None) == qg.QG_EINVAL
+    assert f(X, 128, W, 136, sW, 4, 64, 128, Y, 64, None) == qg.QG_ESHAPE
+    assert f(X, 128, W, 112, sW, 4, 64, 128, Y, 64, None) == qg.QG_ESHAPE
+    assert f(X, 128, W + 8, 128, sW, 4, 64, 128, Y, 64, None) == qg.QG_EALIGN
+    # bf16 X and Y: strides a multiple of 8 elements and at least a row, 16-byte aligned
+    assert f(X, 124, W, 128, sW, 4, 64, 128, Y, 64, None) == qg.QG_ESHAPE
+    assert f(X, 128, W, 128, sW, 4, 64, 128, Y, 60, None) == qg.QG_ESHAPE
+    assert f(X + 2, 128, W, 128, sW, 4, 64, 128, Y, 64, None) == qg.QG_EALIGN
+    assert f(0, 128, W, 128, sW, 4, 64, 128, Y, 64, None) == qg.QG_EINVAL
+    # no tokens: nothing to do, nothing launched
+    assert f(X, 128, W, 128, sW, 0, 64, 128, Y, 64, None) == qg.QG_OK
+
+
 def _lib_sched(t, delta, cs, gamma):
     d = c_int32()
     tn = c_int64()
