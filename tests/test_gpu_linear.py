@@ -234,8 +234,8 @@ def _forward_int8(dXa, ldx, dW, ldw, dsW, T, m, n, ld_extra=8):
 
 
 # (m, n, ldw): ragged rows and columns, scale groups straddling 16-column
-# chunks (n % 256 != 0), one column slice per CTA (m large: several phases of
-# staged X) and eight (m small)
+# chunks (n % 256 != 0), one column slice per row block (m large: each CTA
+# streams many stages through its ring) and eight (m small: a cluster of 8)
 FUSED_SHAPES = [(37, 64, 64), (300, 700, 720), (640, 1365, 1376), (129, 4096, 4096), (20000, 2600, 2608)]
 
 
